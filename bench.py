@@ -1,0 +1,463 @@
+#!/usr/bin/env python
+"""Throughput of the chunkwise Gated DeltaNet forward + backward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config I]
+
+One step = gdn_chunk_fwd + gdn_chunk_bwd (every kernel of the forward and the backward)
+over one batch of the workload, inputs resident in HBM.  The default workload is the
+Qwen3-Next-shaped layer: B=1, T=32768, H=16 q/k heads, HV=32 value heads, K=V=128, bf16
+q/k/v/o/dO, fp32 gates/beta/states, random initial state and final-state gradient.
+Synthetic seeded inputs (no dataset).  Every step streams ~1 GB of inputs, outputs and
+intermediates, far more than the 126 MB L2, so no explicit L2 flush is needed.
+
+Reports M tokens/s (tokens = B*T per GPU, summed over GPUs; weak scaling: every rank runs
+its own batch, no collective in the data path), the end-to-end number through the public
+API with host buffers, the dominant kernel's roofline, and the fp64 CPU oracle timed on a
+bounded sample on the host cores.  ``--impl reference`` times that oracle alone.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_deltanet_chunkwise_chunk_b200 import synth  # noqa: E402
+
+C = 64
+METRIC = "GDN chunk fwd+bwd M tokens/s at T=32k,H=16,HV=32,D=128 bf16; % of roofline"
+DATASHEET = dict(tensor_tflops=2250.0, hbm_gbs=8000.0)
+FALLBACK = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
+# fp32 FFMA peak: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+# ----------------------------------------------------------------- algorithmic work
+def kernel_flops_per_token_head(K: int, V: int) -> dict:
+    """FLOPs each kernel must do per token per value head (its products; 64-row tiles)."""
+    return {
+        "ffma_wy": 2 * C * K + C * C / 3 + 2 * C * (K + V),
+        "ffma_scan_fwd": 4 * K * V,
+        "ffma_out": 2 * C * K + 2 * C * V + 2 * K * V,
+        "ffma_dvlocal": 2 * C * K + 2 * C * V,
+        "ffma_scan_bwd": 6 * K * V,
+        "ffma_dqkwg": 6 * C * K + 2 * C * V + 6 * K * V,
+        "ffma_wy_bwd": 10 * C * K + 4 * C * V + 4 * C * C,
+    }
+
+
+def step_flops_per_token_head(K: int, V: int) -> tuple[float, float]:
+    """Algorithmic FLOPs of the method per token per value head (fwd, bwd)."""
+    fwd = 2 * C * (3 * K + 2 * V) + 6 * K * V + C * C / 3
+    bwd = 2 * C * (9 * K + 5 * V) + 16 * K * V + 4 * C * C + C * C / 3
+    return fwd, bwd
+
+
+def step_bytes(case, e: int) -> tuple[float, float]:
+    """Minimum HBM bytes of one forward and one backward (inputs read once, outputs written
+    once; intermediates not counted)."""
+    B, T, H, HV, K, V = case.B, case.T, case.H, case.HV, case.K, case.V
+    ntok = B * T
+    Nst = case.N
+    states = 4 * K * V * HV * Nst
+    fwd = ntok * (2 * H * K * e + HV * V * e + 8 * HV + HV * V * e) + (states if case.h0 is not None else 0) + states
+    bwd_in = ntok * (2 * H * K * e + 2 * HV * V * e + 8 * HV)
+    bwd_out = ntok * (2 * H * K * e + HV * V * e + 8 * HV)
+    bwd = bwd_in + bwd_out + states * (1 + (case.h0 is not None) + (case.dht is not None))
+    return fwd, bwd
+
+
+def peaks() -> dict:
+    p = dict(FALLBACK)
+    src = "fallback"
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        p.update({k: m[k] for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained") if k in m})
+        src = "measured"
+    except (OSError, ValueError):
+        pass
+    p["source"] = src
+    return p
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                 power=float(parts[3]) if parts[3] not in ("[N/A]", "N/A") else 0.0,
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        load = [r for r in rows if r["power"] > 300] or rows
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["smax"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ----------------------------------------------------------------- oracle baseline
+def oracle_sample(case, budget_s: float = 12.0) -> dict:
+    """fp64 oracle (fwd + bwd) on the first Ts tokens of every batch row and every head of
+    the workload, Ts doubled from 64 until one run costs about a third of the budget."""
+    from oracle import oracle
+
+    def run(Ts):
+        sub = dict(q=case.q[:, :Ts], k=case.k[:, :Ts], v=case.v[:, :Ts], a=case.a[:, :Ts],
+                   A_log=case.A_log, dt_bias=case.dt_bias, beta=case.beta[:, :Ts])
+        t0 = time.perf_counter()
+        oracle.fwd(**sub, h0=case.h0)
+        oracle.bwd(**sub, dO=case.dO[:, :Ts], h0=case.h0, dht=case.dht)
+        return time.perf_counter() - t0
+
+    if case.cu_seqlens is not None:
+        raise ValueError("the oracle sample uses dense batches")
+    Ts = 64
+    dt = run(Ts)
+    while dt < budget_s / 3 and Ts * 2 <= case.T:
+        Ts *= 2
+        dt = run(Ts)
+    units = case.B * case.HV
+    cores = min(os.cpu_count() or 1, units)
+    tok = case.B * Ts
+    return {"value": tok / dt / 1e6, "unit": "M tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 token-by-token oracle fwd+bwd, all {case.HV} value heads x {case.B} "
+                      f"batch rows, first {Ts} of {case.T} tokens ({tok} tokens, {dt:.1f} s)",
+            "seconds": dt}
+
+
+# ----------------------------------------------------------------- our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() and args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+
+    if args.impl == "reference":
+        return reference_arm(args, rank, world, dist)
+
+    import gated_deltanet_chunkwise_chunk_b200 as gdn
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    case = synth.config_case(args.config, seed=1000 + args.config + 7919 * rank)
+    e = 2 if case.dtype == "bf16" else 4
+    t = lambda x: None if x is None else x.to(dev).contiguous()
+    inp = dict(q=t(case.q), k=t(case.k), v=t(case.v), g_raw=t(case.a), A_log=t(case.A_log),
+               dt_bias=t(case.dt_bias), beta=t(case.beta), cu_seqlens=t(case.cu_seqlens),
+               initial_state=t(case.h0))
+    dO, dht = t(case.dO), t(case.dht)
+    dims = gdn.make_dims(inp["q"], inp["v"], inp["cu_seqlens"])
+    varlen = case.cu_seqlens is not None
+    ws = torch.empty(max(gdn.workspace_bytes(dims, varlen, False), gdn.workspace_bytes(dims, varlen, True)),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty_like(inp["v"])
+    ht = torch.empty((case.N, case.HV, case.K, case.V), dtype=torch.float32, device=dev)
+    outs = dict(dq=torch.empty_like(inp["q"]), dk=torch.empty_like(inp["k"]), dv=torch.empty_like(inp["v"]),
+                dg=torch.empty_like(inp["g_raw"]), dbeta=torch.empty_like(inp["beta"]),
+                dh0=torch.empty_like(ht), dg_raw=torch.empty_like(inp["g_raw"]),
+                dA_log=torch.empty_like(inp["A_log"]), ddt_bias=torch.empty_like(inp["A_log"]))
+
+    def fwd():
+        gdn.gdn_chunk_fwd(**inp, workspace=ws, out=o, final_state=ht)
+
+    def step():
+        fwd()
+        gdn.gdn_chunk_bwd(**inp, d_o=dO, dht=dht, workspace=ws, outs=outs)
+
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n):
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        return a.elapsed_time(b) / n
+
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+    sampler = ClockSampler(vis[local].strip() if len(vis) > local and vis[local].strip() else local)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    n0 = gdn.launch_count()
+    ms = timed(step, args.steps)
+    launches = gdn.launch_count() - n0
+    clocks = sampler.stop()
+    ms_fwd = timed(fwd, max(1, args.steps))
+    if dist:
+        tt = torch.tensor([ms, ms_fwd], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, ms_fwd = float(tt[0]), float(tt[1])
+
+    # per-kernel device time (separate pass: events around every launch on its stream)
+    gdn.profile(True)
+    for _ in range(2):
+        step()
+    prof = gdn.profile_read()
+    gdn.profile(False)
+
+    # end to end through the public API with host buffers
+    e2e = e2e_measure(gdn, case, dev, ws, args.e2e_steps, dist)
+
+    tokens = case.tokens
+    value = world * tokens / (ms / 1e3) / 1e6
+    pk = peaks()
+    fflop, bflop = step_flops_per_token_head(case.K, case.V)
+    th = tokens * case.HV
+    fbytes, bbytes = step_bytes(case, e)
+    flops = th * (fflop + bflop)
+    nbytes = fbytes + bbytes
+    t_roof_ds = max(flops / (DATASHEET["tensor_tflops"] * 1e12), nbytes / (DATASHEET["hbm_gbs"] * 1e9))
+    t_roof_m = max(flops / (pk["bf16_tflops_sustained"] * 1e12), nbytes / (pk["hbm_gbs"] * 1e9))
+    roof = kernel_roofline(prof, case, pk)
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "M tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": case.dtype, "data": "synthetic (seeded N(0,1)/sigmoid/log-uniform inputs; no dataset)",
+        "config": {"workload": case.name, "B": case.B, "T": case.T, "H": case.H, "HV": case.HV,
+                   "K": case.K, "V": case.V, "chunk": C, "global_batch": case.B * world,
+                   "seq_len": case.T, "parallelism": f"dp{world} (independent batches)",
+                   "l2": "no flush: each step streams ~1 GB (inputs alone > 126 MB L2)"},
+        "fwd_mtok_s": round(world * tokens / (ms_fwd / 1e3) / 1e6, 3),
+        "ms_fwd": round(ms_fwd, 4),
+        "step_roofline": {"flops": flops, "bytes": nbytes,
+                          "frac_datasheet": round(t_roof_ds / (ms / 1e3), 4),
+                          "frac_measured": round(t_roof_m / (ms / 1e3), 4),
+                          "roofline_mtok_s_datasheet": round(tokens / t_roof_ds / 1e6, 2),
+                          "note": "max(FLOP/bf16 peak, bytes/HBM) over the whole fwd+bwd step"},
+        "roofline": roof,
+        "kernels": {k: {"launches": v[0], "ms_per_step": round(v[1] / 2, 4)} for k, v in prof.items()},
+        "gpu_launches": int(launches),
+        "e2e": e2e,
+        "clocks": clocks,
+        "peaks_source": pk["source"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        try:
+            line["cpu_baseline"] = oracle_sample(case)
+            line["cpu_baseline"].pop("seconds", None)
+        except Exception as ex:  # noqa: BLE001
+            line["cpu_baseline"] = {"error": str(ex)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def kernel_roofline(prof: dict, case, pk: dict) -> dict | None:
+    """Roofline of the kernel with the largest share of device time."""
+    if not prof:
+        return None
+    name, (launches, total_ms) = max(prof.items(), key=lambda kv: kv[1][1])
+    per_launch_s = total_ms / launches / 1e3
+    fl = kernel_flops_per_token_head(case.K, case.V).get(name)
+    th = case.tokens * case.HV
+    out = {"kernel": name, "launch_ms": round(per_launch_s * 1e3, 4),
+           "share": round(total_ms / sum(v[1] for v in prof.values()), 4)}
+    traffic = _traffic(name, case)
+    if fl is not None and name.startswith("ffma_"):
+        achieved = fl * th / per_launch_s / 1e12
+        peak = FP32_ALU_TFLOPS
+        out.update({"bound": "alu", "achieved": round(achieved, 3), "peak": round(peak, 1),
+                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                    "peak_source": "fp32 FFMA: 148 SM x 128 lanes x 2 FLOP x 1.965 GHz"})
+    elif fl is not None:
+        achieved = fl * th / per_launch_s / 1e12
+        peak = pk["bf16_tflops"]
+        out.update({"bound": "tensor", "achieved": round(achieved, 3), "peak": peak,
+                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                    "peak_source": f"bf16 burst, {pk['source']}"})
+    return out
+
+
+def _traffic(name: str, case):
+    """DRAM bytes per launch from the committed ncu summary, when it covers this kernel."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        rec = d.get(name)
+        if rec and rec.get("workload") == case.name:
+            return rec["bytes_per_launch"]
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+def e2e_measure(gdn, case, dev, ws, nsteps: int, dist) -> dict:
+    """Same step through the public API, with the inputs copied from pinned host memory and
+    every output copied back to pinned host memory inside the timed region."""
+    pin = lambda x: None if x is None else x.contiguous().pin_memory()
+    host_in = dict(q=pin(case.q), k=pin(case.k), v=pin(case.v), g_raw=pin(case.a), A_log=pin(case.A_log),
+                   dt_bias=pin(case.dt_bias), beta=pin(case.beta), cu_seqlens=pin(case.cu_seqlens),
+                   initial_state=pin(case.h0), d_o=pin(case.dO), dht=pin(case.dht))
+    dev_in = {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in host_in.items()}
+    o = torch.empty_like(dev_in["v"])
+    ht = torch.empty((case.N, case.HV, case.K, case.V), dtype=torch.float32, device=dev)
+    outs = dict(dq=torch.empty_like(dev_in["q"]), dk=torch.empty_like(dev_in["k"]),
+                dv=torch.empty_like(dev_in["v"]), dg=torch.empty_like(dev_in["g_raw"]),
+                dbeta=torch.empty_like(dev_in["beta"]), dh0=torch.empty_like(ht))
+    host_out = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in
+                dict(o=o, ht=ht, **outs).items()}
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values() if v is not None)
+    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+    stream = torch.cuda.current_stream()
+
+    def one():
+        for k, v in host_in.items():
+            if v is not None:
+                dev_in[k].copy_(v, non_blocking=True)
+        fw = {k: dev_in[k] for k in ("q", "k", "v", "g_raw", "A_log", "dt_bias", "beta",
+                                     "cu_seqlens", "initial_state")}
+        gdn.gdn_chunk_fwd(**fw, workspace=ws, out=o, final_state=ht)
+        gdn.gdn_chunk_bwd(**fw, d_o=dev_in["d_o"], dht=dev_in["dht"], workspace=ws, outs=outs,
+                          want_param_grads=False)
+        for k, v in dict(o=o, ht=ht, **outs).items():
+            host_out[k].copy_(v, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(nsteps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / nsteps
+    world = 1
+    if dist:
+        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt[0])
+        world = dist.get_world_size()
+    return {"value": round(world * case.tokens / (ms / 1e3) / 1e6, 3), "unit": "M tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(ms, 3)}
+
+
+# ----------------------------------------------------------------- reference arm (oracle)
+def reference_arm(args, rank, world, dist):
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return
+    case = synth.config_case(args.config, seed=1000 + args.config)
+    from oracle import oracle
+    oracle.build()
+    samples = []
+    budget = max(2.0, 90.0 / max(1, args.steps + args.warmup))
+    info = None
+    for i in range(args.warmup + args.steps):
+        info = oracle_sample(case, budget_s=budget)
+        if i >= args.warmup:
+            samples.append(info["value"])
+    value = statistics.mean(samples)
+    tokens_per_step = case.tokens
+    ms = tokens_per_step / (value * 1e6) * 1e3
+    cpu = {k: info[k] for k in ("unit", "cores", "kind", "sample")}
+    cpu["value"] = round(value, 6)
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "M tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": case.name, "B": case.B, "T": case.T, "H": case.H, "HV": case.HV,
+                       "K": case.K, "V": case.V, "chunk": C},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(value, 6), "unit": "M tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "note": "the reference arm is the fp64 token-by-token oracle on the host cores, "
+                    "each step a bounded sample of the workload (tokens/s of that sample)"}
+    print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,245 @@
+"""Thin ctypes binding of libgdn_b200.so (include/gdn.h).
+
+Argument marshalling only: it checks torch tensors (device, dtype, contiguity, shape),
+allocates outputs and the workspace with torch, and passes raw pointers plus the current
+CUDA stream to the C entry points of the same names.  Every step of the computation runs
+in the library's CUDA kernels.  There is no fallback: if the shared library is missing,
+importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(6)
+GDN_DTYPE_FP32, GDN_DTYPE_BF16 = 0, 1
+
+# Every symbol include/gdn.h declares (checked by the tests).
+EXPORTED = ("gdn_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_max_chunks",
+            "gdn_build_chunk_indices", "gdn_chunk_table_device", "gdn_device_status",
+            "gdn_status_string", "gdn_version", "gdn_launch_count", "gdn_profile",
+            "gdn_profile_read")
+
+
+class gdn_dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("T", ctypes.c_int64), ("H", ctypes.c_int64),
+                ("HV", ctypes.c_int64), ("K", ctypes.c_int64), ("V", ctypes.c_int64),
+                ("N", ctypes.c_int64), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class GDNError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m gated_deltanet_chunkwise_chunk_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    D = ctypes.POINTER(gdn_dims)
+    lib.gdn_workspace_bytes.argtypes = [D, I32, I32]
+    lib.gdn_workspace_bytes.restype = SZ
+    lib.gdn_chunk_fwd.argtypes = [D] + [P] * 12 + [SZ, P]
+    lib.gdn_chunk_fwd.restype = I32
+    lib.gdn_chunk_bwd.argtypes = [D] + [P] * 21 + [SZ, P]
+    lib.gdn_chunk_bwd.restype = I32
+    lib.gdn_max_chunks.argtypes = [D, I32]
+    lib.gdn_max_chunks.restype = I64
+    lib.gdn_build_chunk_indices.argtypes = [D, P, P, I64]
+    lib.gdn_build_chunk_indices.restype = I64
+    lib.gdn_chunk_table_device.argtypes = [D, P, P, I64, P, P]
+    lib.gdn_chunk_table_device.restype = I32
+    lib.gdn_device_status.argtypes = [P, P]
+    lib.gdn_device_status.restype = I32
+    lib.gdn_status_string.argtypes = [I32]
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_version.argtypes = []
+    lib.gdn_version.restype = ctypes.c_char_p
+    lib.gdn_launch_count.argtypes = []
+    lib.gdn_launch_count.restype = I64
+    lib.gdn_profile.argtypes = [I32]
+    lib.gdn_profile.restype = I32
+    lib.gdn_profile_read.argtypes = [ctypes.c_char_p, SZ]
+    lib.gdn_profile_read.restype = I64
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.gdn_status_string(int(status)).decode()
+
+
+def version() -> str:
+    return lib.gdn_version().decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def make_dims(q, v, cu_seqlens=None, scale=0.0) -> gdn_dims:
+    B, T, H, K = q.shape
+    HV, V = v.shape[2], v.shape[3]
+    N = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
+    dt = GDN_DTYPE_BF16 if q.dtype == torch.bfloat16 else GDN_DTYPE_FP32
+    return gdn_dims(B, T, H, HV, K, V, N, dt, float(scale or 0.0))
+
+
+def workspace_bytes(dims: gdn_dims, varlen: bool, backward: bool) -> int:
+    return int(lib.gdn_workspace_bytes(ctypes.byref(dims), int(varlen), int(backward)))
+
+
+def max_chunks(dims: gdn_dims, varlen: bool) -> int:
+    return int(lib.gdn_max_chunks(ctypes.byref(dims), int(varlen)))
+
+
+def _workspace(dims, varlen, backward, workspace, device):
+    n = workspace_bytes(dims, varlen, backward)
+    if n == 0:
+        raise GDNError("gdn_workspace_bytes", GDN_ERR_INVALID_ARG)
+    if workspace is not None and workspace.numel() >= n:
+        return workspace
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _check(name, t, dtype, shape, device):
+    if t is None:
+        return
+    if t.device != device or t.dtype != dtype or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected contiguous {dtype} {tuple(shape)} on {device}, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device} (contiguous={t.is_contiguous()})")
+
+
+def _check_inputs(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens, initial_state):
+    dev = q.device
+    B, T, H, K = q.shape
+    HV, V = v.shape[2], v.shape[3]
+    Nst = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
+    _check("q", q, q.dtype, (B, T, H, K), dev)
+    _check("k", k, q.dtype, (B, T, H, K), dev)
+    _check("v", v, q.dtype, (B, T, HV, V), dev)
+    _check("g_raw", g_raw, torch.float32, (B, T, HV), dev)
+    _check("beta", beta, torch.float32, (B, T, HV), dev)
+    _check("A_log", A_log, torch.float32, (HV,), dev)
+    _check("dt_bias", dt_bias, torch.float32, (HV,), dev)
+    _check("cu_seqlens", cu_seqlens, torch.int64, (Nst + 1,), dev)
+    _check("initial_state", initial_state, torch.float32, (Nst, HV, K, V), dev)
+    return Nst
+
+
+def gdn_chunk_fwd(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None, initial_state=None,
+                  scale=0.0, output_final_state=True, workspace=None, out=None, final_state=None):
+    """Forward: returns (o, final_state or None).  See include/gdn.h for layouts."""
+    Nst = _check_inputs(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens, initial_state)
+    dims = make_dims(q, v, cu_seqlens, scale)
+    ws = _workspace(dims, cu_seqlens is not None, False, workspace, q.device)
+    o = out if out is not None else torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    ht = None
+    if output_final_state:
+        ht = final_state if final_state is not None else torch.empty(
+            (Nst, v.shape[2], q.shape[3], v.shape[3]), dtype=torch.float32, device=q.device)
+    rc = lib.gdn_chunk_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g_raw), _ptr(A_log),
+                           _ptr(dt_bias), _ptr(beta), _ptr(cu_seqlens), _ptr(initial_state), _ptr(o),
+                           _ptr(ht), _ptr(ws), ws.numel(), _stream())
+    if rc != GDN_OK:
+        raise GDNError("gdn_chunk_fwd", rc)
+    return o, ht
+
+
+def gdn_chunk_bwd(q, k, v, g_raw, A_log, dt_bias, beta, d_o, cu_seqlens=None, initial_state=None,
+                  dht=None, scale=0.0, want_dh0=True, want_param_grads=True, workspace=None,
+                  outs=None):
+    """Backward of sum(d_o*o) + sum(dht*final_state).  Returns a dict with dq, dk, dv, dg,
+    dbeta and (when asked) dh0, dg_raw, dA_log, ddt_bias."""
+    Nst = _check_inputs(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens, initial_state)
+    B, T, H, K = q.shape
+    HV, V = v.shape[2], v.shape[3]
+    _check("d_o", d_o, q.dtype, (B, T, HV, V), q.device)
+    _check("dht", dht, torch.float32, (Nst, HV, K, V), q.device)
+    dims = make_dims(q, v, cu_seqlens, scale)
+    ws = _workspace(dims, cu_seqlens is not None, True, workspace, q.device)
+    dev = q.device
+    if outs is None:
+        outs = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                    dg=torch.empty((B, T, HV), dtype=torch.float32, device=dev),
+                    dbeta=torch.empty((B, T, HV), dtype=torch.float32, device=dev))
+        if want_dh0:
+            outs["dh0"] = torch.empty((Nst, HV, K, V), dtype=torch.float32, device=dev)
+        if want_param_grads:
+            outs["dg_raw"] = torch.empty((B, T, HV), dtype=torch.float32, device=dev)
+            outs["dA_log"] = torch.empty((HV,), dtype=torch.float32, device=dev)
+            outs["ddt_bias"] = torch.empty((HV,), dtype=torch.float32, device=dev)
+    g = outs.get
+    rc = lib.gdn_chunk_bwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g_raw), _ptr(A_log),
+                           _ptr(dt_bias), _ptr(beta), _ptr(cu_seqlens), _ptr(initial_state),
+                           _ptr(d_o), _ptr(dht), _ptr(g("dq")), _ptr(g("dk")), _ptr(g("dv")),
+                           _ptr(g("dg")), _ptr(g("dbeta")), _ptr(g("dh0")), _ptr(g("dg_raw")),
+                           _ptr(g("dA_log")), _ptr(g("ddt_bias")), _ptr(ws), ws.numel(), _stream())
+    if rc != GDN_OK:
+        raise GDNError("gdn_chunk_bwd", rc)
+    return outs
+
+
+def gdn_build_chunk_indices(dims: gdn_dims, cu_host=None):
+    """Host chunk table as a [count, 4] int32 tensor (see include/gdn.h)."""
+    import numpy as np
+    cu = None if cu_host is None else np.ascontiguousarray(np.asarray(cu_host, dtype=np.int64))
+    cp = None if cu is None else cu.ctypes.data_as(ctypes.c_void_p)
+    n = lib.gdn_build_chunk_indices(ctypes.byref(dims), cp, None, 0)
+    if n < 0:
+        raise GDNError("gdn_build_chunk_indices", -n)
+    out = np.zeros((max(n, 1), 4), dtype=np.int32)
+    lib.gdn_build_chunk_indices(ctypes.byref(dims), cp, out.ctypes.data_as(ctypes.c_void_p), n)
+    return out[:n]
+
+
+def gdn_chunk_table_device(dims: gdn_dims, cu_seqlens=None, cap=None, device="cuda"):
+    """Device-built chunk table ([cap, 4] int32 on the device) and its count (int)."""
+    if cap is None:
+        cap = max_chunks(dims, cu_seqlens is not None)
+    table = torch.empty((cap, 4), dtype=torch.int32, device=device)
+    count = torch.empty((4,), dtype=torch.int32, device=device)
+    rc = lib.gdn_chunk_table_device(ctypes.byref(dims), _ptr(cu_seqlens), _ptr(table), int(cap),
+                                    _ptr(count), _stream())
+    if rc != GDN_OK:
+        raise GDNError("gdn_chunk_table_device", rc)
+    return table, int(count[0].item())
+
+
+def gdn_device_status(workspace) -> int:
+    return int(lib.gdn_device_status(_ptr(workspace), _stream()))
+
+
+def launch_count() -> int:
+    """Kernel launches issued by the library since it was loaded."""
+    return int(lib.gdn_launch_count())
+
+
+def profile(enable: bool) -> None:
+    """Bracket every launch with CUDA events on its stream (measurement passes only)."""
+    lib.gdn_profile(int(bool(enable)))
+
+
+def profile_read() -> dict:
+    """Per-kernel {name: (launches, total_ms)} since the last read (synchronises)."""
+    import json
+    n = lib.gdn_profile_read(None, 0)
+    if n < 0:
+        raise GDNError("gdn_profile_read", -n)
+    buf = ctypes.create_string_buffer(int(n) + 1)
+    lib.gdn_profile_read(buf, len(buf))
+    return {k: tuple(v) for k, v in json.loads(buf.value.decode() or "{}").items()}

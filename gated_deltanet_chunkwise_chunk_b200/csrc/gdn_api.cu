@@ -1,0 +1,321 @@
+// C-ABI entry points: argument validation, workspace carve-up and the launch sequences.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "gdn.h"
+#include "gdn_common.cuh"
+#include "gdn_launch.h"
+#include "gdn_tc.h"
+
+namespace gdn {
+namespace {
+
+constexpr size_t kAlign = 256;
+
+inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t max_chunks(const gdn_dims& d, bool varlen) {
+  if (varlen) return (d.T + 63 * d.N) / CH;
+  return d.B * ((d.T + CH - 1) / CH);
+}
+
+// Validates dims; 0 on success.
+int check_dims(const gdn_dims* d, bool varlen) {
+  if (!d) return GDN_ERR_INVALID_ARG;
+  if (d->B <= 0 || d->T < 0 || d->H <= 0 || d->HV <= 0 || d->K <= 0 || d->V <= 0)
+    return GDN_ERR_INVALID_ARG;
+  if (d->HV % d->H) return GDN_ERR_INVALID_ARG;
+  if (varlen && (d->B != 1 || d->N <= 0)) return GDN_ERR_INVALID_ARG;
+  if ((d->K != 64 && d->K != 128) || (d->V != 64 && d->V != 128)) return GDN_ERR_UNSUPPORTED;
+  if (d->dtype != GDN_DTYPE_FP32 && d->dtype != GDN_DTYPE_BF16) return GDN_ERR_UNSUPPORTED;
+  if (d->B * d->T >= (int64_t)1 << 31 || d->HV > 65535) return GDN_ERR_INVALID_ARG;
+  if (max_chunks(*d, varlen) >= (int64_t)1 << 30) return GDN_ERR_INVALID_ARG;
+  if (!(d->scale >= 0.f) || std::isinf(d->scale)) return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
+// Byte offsets of the workspace regions (FFMA path layout; the tcgen05 path appends its
+// own regions after the common ones).
+struct Plan {
+  size_t status, seq_tab, chunk_tab, G, beta_p;
+  size_t W, Ut, Tm, h, U, dU, dh, dW, dqp, dkp, dG, tmp;
+  size_t tc;     // start of the tcgen05 path's region
+  size_t total;
+};
+
+Plan make_plan(const gdn_dims& d, bool varlen, int pass) {
+  Plan pl{};
+  const size_t NC = (size_t)max_chunks(d, varlen);
+  const size_t Nst = varlen ? (size_t)d.N : (size_t)d.B;
+  const size_t HV = d.HV, K = d.K, V = d.V, f = sizeof(float);
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o += up(bytes);
+    return at;
+  };
+  pl.status = take(64);
+  pl.seq_tab = take(Nst * sizeof(int4));
+  pl.chunk_tab = take(NC * sizeof(int4));
+  pl.G = take(HV * NC * CH * f);
+  pl.beta_p = take(HV * NC * CH * f);
+  const bool ffma = d.dtype == GDN_DTYPE_FP32 || !tc_supported(d);
+  if (ffma) {
+    pl.W = take(NC * HV * CH * K * f);
+    pl.Ut = take(NC * HV * CH * V * f);
+    pl.h = take(NC * HV * V * K * f);
+    pl.U = take(NC * HV * CH * V * f);
+    if (pass == 1) {
+      pl.Tm = take(NC * HV * CH * CH * f);
+      pl.dU = take(NC * HV * CH * V * f);
+      pl.dh = take(NC * HV * V * K * f);
+      pl.dW = take(NC * HV * CH * K * f);
+      pl.dqp = take(NC * HV * CH * K * f);
+      pl.dkp = take(NC * HV * CH * K * f);
+      pl.dG = take(HV * NC * CH * f);
+      pl.tmp = take(NC * HV * CH * 128 * f);
+    }
+  } else {
+    pl.tc = take(tc_workspace_bytes(d, NC, pass));
+  }
+  pl.total = o;
+  return pl;
+}
+
+Work carve(const Plan& pl, void* ws) {
+  char* b = static_cast<char*>(ws);
+  Work w{};
+  w.status = reinterpret_cast<int*>(b + pl.status);
+  w.seq_tab = reinterpret_cast<int4*>(b + pl.seq_tab);
+  w.chunk_tab = reinterpret_cast<int4*>(b + pl.chunk_tab);
+  w.G = reinterpret_cast<float*>(b + pl.G);
+  w.beta_p = reinterpret_cast<float*>(b + pl.beta_p);
+  auto fp = [&](size_t off) { return off ? reinterpret_cast<float*>(b + off) : nullptr; };
+  w.W = fp(pl.W);
+  w.Ut = fp(pl.Ut);
+  w.Tm = fp(pl.Tm);
+  w.h = fp(pl.h);
+  w.U = fp(pl.U);
+  w.dU = fp(pl.dU);
+  w.dh = fp(pl.dh);
+  w.dW = fp(pl.dW);
+  w.dqp = fp(pl.dqp);
+  w.dkp = fp(pl.dkp);
+  w.dG = fp(pl.dG);
+  w.tmp = fp(pl.tmp);
+  return w;
+}
+
+Problem make_problem(const gdn_dims& d, bool varlen) {
+  Problem p{};
+  p.B = (int)d.B;
+  p.T = (int)d.T;
+  p.H = (int)d.H;
+  p.HV = (int)d.HV;
+  p.K = (int)d.K;
+  p.V = (int)d.V;
+  p.Nst = varlen ? (int)d.N : (int)d.B;
+  p.G = (int)(d.HV / d.H);
+  p.varlen = varlen ? 1 : 0;
+  p.NCmax = (int)max_chunks(d, varlen);
+  p.scale = d.scale > 0.f ? d.scale : 1.f / std::sqrt((float)d.K);
+  return p;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+// Steps shared by the forward and the backward: chunk table, gate + in-chunk cumsum.
+cudaError_t prologue(const Problem& p, const Args& a, const Work& w, cudaStream_t s) {
+  cudaError_t e = launch_chunk_table(p, a.cu, w, s);
+  if (e != cudaSuccess) return e;
+  return launch_gate_cumsum(p, a, w, s);
+}
+
+}  // namespace
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+size_t gdn_workspace_bytes(const gdn_dims* d, int varlen, int pass) {
+  if (check_dims(d, varlen != 0) != GDN_OK || (pass != 0 && pass != 1)) return 0;
+  return make_plan(*d, varlen != 0, pass).total;
+}
+
+int64_t gdn_max_chunks(const gdn_dims* d, int varlen) {
+  if (check_dims(d, varlen != 0) != GDN_OK) return -GDN_ERR_INVALID_ARG;
+  return max_chunks(*d, varlen != 0);
+}
+
+int gdn_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                  const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,
+                  const int64_t* cu_seqlens, const float* initial_state, void* o, float* final_state,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  const bool varlen = cu_seqlens != nullptr;
+  int rc = check_dims(d, varlen);
+  if (rc) return rc;
+  // per-token tensors may be null when there are no tokens (B*T == 0)
+  const bool empty = d->B * d->T == 0;
+  const void* tok[] = {q, k, v, g_raw, beta, o};
+  for (const void* x : tok)
+    if ((!x && !empty) || !aligned16(x)) return GDN_ERR_INVALID_ARG;
+  if (!A_log || !dt_bias || !aligned16(A_log) || !aligned16(dt_bias)) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(cu_seqlens) || !aligned16(initial_state) || !aligned16(final_state))
+    return GDN_ERR_INVALID_ARG;
+  const Plan pl = make_plan(*d, varlen, 0);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) || workspace_bytes < pl.total)
+    return GDN_ERR_WORKSPACE;
+  const Problem p = make_problem(*d, varlen);
+  Args a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.g_raw = g_raw;
+  a.A_log = A_log;
+  a.dt_bias = dt_bias;
+  a.beta = beta;
+  a.cu = cu_seqlens;
+  a.h0 = initial_state;
+  a.o = o;
+  a.ht = final_state;
+  const Work w = carve(pl, workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = prologue(p, a, w, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  const bool bf16 = d->dtype == GDN_DTYPE_BF16;
+  if (bf16 && tc_supported(*d))
+    e = tc_forward(p, a, w, static_cast<char*>(workspace) + pl.tc, s);
+  else
+    e = ffma_forward(p, a, w, bf16, false, s);
+  return cuda_status(e);
+}
+
+int gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                  const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,
+                  const int64_t* cu_seqlens, const float* initial_state, const void* d_o,
+                  const float* dht, void* dq, void* dk, void* dv, float* dg, float* dbeta,
+                  float* dh0, float* dg_raw, float* dA_log, float* ddt_bias, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  const bool varlen = cu_seqlens != nullptr;
+  int rc = check_dims(d, varlen);
+  if (rc) return rc;
+  const bool empty = d->B * d->T == 0;
+  const void* tok[] = {q, k, v, g_raw, beta, d_o, dq, dk, dv, dg, dbeta};
+  for (const void* x : tok)
+    if ((!x && !empty) || !aligned16(x)) return GDN_ERR_INVALID_ARG;
+  if (!A_log || !dt_bias || !aligned16(A_log) || !aligned16(dt_bias)) return GDN_ERR_INVALID_ARG;
+  const void* opt[] = {cu_seqlens, initial_state, dht, dh0, dg_raw, dA_log, ddt_bias};
+  for (const void* x : opt)
+    if (!aligned16(x)) return GDN_ERR_INVALID_ARG;
+  const Plan pl = make_plan(*d, varlen, 1);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) || workspace_bytes < pl.total)
+    return GDN_ERR_WORKSPACE;
+  const Problem p = make_problem(*d, varlen);
+  Args a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.g_raw = g_raw;
+  a.A_log = A_log;
+  a.dt_bias = dt_bias;
+  a.beta = beta;
+  a.cu = cu_seqlens;
+  a.h0 = initial_state;
+  a.dO = d_o;
+  a.dht = dht;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dg = dg;
+  a.dbeta = dbeta;
+  a.dh0 = dh0;
+  a.dg_raw = dg_raw;
+  a.dA_log = dA_log;
+  a.ddt_bias = ddt_bias;
+  const Work w = carve(pl, workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = prologue(p, a, w, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  const bool bf16 = d->dtype == GDN_DTYPE_BF16;
+  if (bf16 && tc_supported(*d)) {
+    e = tc_backward(p, a, w, static_cast<char*>(workspace) + pl.tc, s);
+    if (e != cudaSuccess) return cuda_status(e);
+  } else {
+    e = ffma_forward(p, a, w, bf16, true, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = ffma_backward(p, a, w, bf16, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = launch_bwd_tokens(p, a, w, bf16, s);
+  }
+  return cuda_status(e);
+}
+
+int64_t gdn_build_chunk_indices(const gdn_dims* d, const int64_t* cu_host, int32_t* out_host,
+                                int64_t cap) {
+  const bool varlen = cu_host != nullptr;
+  if (check_dims(d, varlen) != GDN_OK) return -GDN_ERR_INVALID_ARG;
+  if (cap > 0 && !out_host) return -GDN_ERR_INVALID_ARG;
+  const int64_t Nst = varlen ? d->N : d->B;
+  if (varlen) {
+    if (cu_host[0] != 0 || cu_host[Nst] != d->T) return -GDN_ERR_INVALID_ARG;
+    for (int64_t n = 0; n < Nst; ++n)
+      if (cu_host[n + 1] < cu_host[n]) return -GDN_ERR_INVALID_ARG;
+  }
+  int64_t count = 0;
+  for (int64_t n = 0; n < Nst; ++n) {
+    const int64_t bos = varlen ? cu_host[n] : n * d->T;
+    const int64_t len = varlen ? cu_host[n + 1] - cu_host[n] : d->T;
+    for (int64_t c = 0; c * CH < len; ++c, ++count) {
+      if (count < cap) {
+        out_host[4 * count + 0] = (int32_t)n;
+        out_host[4 * count + 1] = (int32_t)c;
+        out_host[4 * count + 2] = (int32_t)(len - c * CH < CH ? len - c * CH : CH);
+        out_host[4 * count + 3] = (int32_t)(bos + c * CH);
+      }
+    }
+  }
+  return count;
+}
+
+int gdn_chunk_table_device(const gdn_dims* d, const int64_t* cu_seqlens, int32_t* table,
+                           int64_t cap, int32_t* count_dev, void* stream) {
+  const bool varlen = cu_seqlens != nullptr;
+  int rc = check_dims(d, varlen);
+  if (rc) return rc;
+  if (!table || !count_dev || cap <= 0 || cap >= ((int64_t)1 << 30) || !aligned16(table))
+    return GDN_ERR_INVALID_ARG;
+  Problem p = make_problem(*d, varlen);
+  p.NCmax = (int)cap;
+  return cuda_status(launch_chunk_table_only(p, cu_seqlens, reinterpret_cast<int4*>(table),
+                                             count_dev, static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_device_status(const void* workspace, void* stream) {
+  if (!workspace) return GDN_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int st = 0;
+  cudaError_t e = cudaMemcpyAsync(&st, workspace, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return GDN_ERR_CUDA;
+  return st;
+}
+
+const char* gdn_status_string(int status) {
+  switch (status) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+    case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+    case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+    default: return "GDN_ERR_UNKNOWN";
+  }
+}
+
+const char* gdn_version(void) { return "gdn-b200 0.1 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,103 @@
+// Shared device-side definitions of the chunkwise Gated DeltaNet library (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+constexpr int CH = 64;  // tokens per chunk
+
+// Launch-wide problem description (passed by value to every kernel).
+struct Problem {
+  int B, T, H, HV, K, V;
+  int Nst;      // number of independent state sequences (N when varlen, else B)
+  int G;        // value heads per k-head (HV / H)
+  int varlen;   // 1 when cu_seqlens is used
+  int NCmax;    // grid bound on the number of chunks
+  float scale;
+};
+
+// Workspace carve-up (device pointers into the caller's workspace).  Intermediates are
+// indexed per chunk gc in [0, NCmax) and value head hv.
+struct Work {
+  int* status;        // [0] device status word, [1] chunk count
+  int4* seq_tab;      // [Nst]   {first chunk, number of chunks, flat bos, length}
+  int4* chunk_tab;    // [NCmax] {sequence, chunk in sequence, tokens L, flat token of row 0}
+  float* G;           // [HV][NCmax][64]   in-chunk inclusive cumsum of g, padded with G[L-1]
+  float* beta_p;      // [HV][NCmax][64]   beta, zero past the chunk's last token
+  // fp32 intermediates of the FFMA path
+  float* W;           // [NCmax][HV][64][K]
+  float* Ut;          // [NCmax][HV][64][V]
+  float* Tm;          // [NCmax][HV][64][64]   (I + A)^-1
+  float* h;           // [NCmax][HV][V][K]     state entering the chunk (S orientation)
+  float* U;           // [NCmax][HV][64][V]    v_new = U~ - W S^T
+  float* dU;          // [NCmax][HV][64][V]    dU_loc, then the full dU
+  float* dh;          // [NCmax][HV][V][K]     dL/dS leaving the chunk
+  float* dW;          // [NCmax][HV][64][K]
+  float* dqp;         // [NCmax][HV][64][K]    per-value-head dq share
+  float* dkp;         // [NCmax][HV][64][K]    per-value-head dk share
+  float* dG;          // [HV][NCmax][64]       dL/dG (before the reverse cumsum)
+  float* tmp;         // [NCmax][HV][64][128]  per-unit scratch
+};
+
+// Pointers of one call (inputs and outputs as given by the caller).
+struct Args {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g_raw;
+  const float* A_log;
+  const float* dt_bias;
+  const float* beta;
+  const int64_t* cu;
+  const float* h0;
+  void* o;
+  float* ht;
+  const void* dO;
+  const float* dht;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* dg;
+  float* dbeta;
+  float* dh0;
+  float* dg_raw;
+  float* dA_log;
+  float* ddt_bias;
+};
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// The gate of one token: g = -exp(A_log) * softplus(x), softplus(x) = x for x > 20.
+__device__ __forceinline__ float gate_value(float a, float A_log, float dt_bias) {
+  const float x = a + dt_bias;
+  const float sp = x > 20.f ? x : log1pf(expf(x));
+  return -expf(A_log) * sp;
+}
+
+// d softplus / dx with the same branch.
+__device__ __forceinline__ float gate_dsoftplus(float x) {
+  return x > 20.f ? 1.f : 1.f / (1.f + expf(-x));
+}
+
+__device__ __forceinline__ bool call_failed(const Work& w) {
+  return *((volatile int*)w.status) != 0;
+}
+
+}  // namespace gdn

@@ -1,0 +1,38 @@
+// Host-side launcher declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "gdn_common.cuh"
+
+namespace gdn {
+
+// Counts a launch and, while profiling is on, brackets it with CUDA events on `s`.
+class ProfScope {
+ public:
+  ProfScope(const char* name, cudaStream_t s);
+  ~ProfScope();
+  ProfScope(const ProfScope&) = delete;
+  ProfScope& operator=(const ProfScope&) = delete;
+
+ private:
+  const char* name_;
+  cudaStream_t s_;
+  cudaEvent_t a_{}, b_{};
+  bool active_ = false;
+};
+
+cudaError_t launch_chunk_table(const Problem& p, const int64_t* cu, const Work& w, cudaStream_t s);
+cudaError_t launch_chunk_table_only(const Problem& p, const int64_t* cu, int4* table, int* count,
+                                    cudaStream_t s);
+cudaError_t launch_gate_cumsum(const Problem& p, const Args& a, const Work& w, cudaStream_t s);
+cudaError_t launch_bwd_tokens(const Problem& p, const Args& a, const Work& w, bool bf16,
+                              cudaStream_t s);
+
+// fp32 CUDA-core path (FFMA tiles): used for fp32 tensors.
+cudaError_t ffma_forward(const Problem& p, const Args& a, const Work& w, bool bf16, bool bwd_prep,
+                         cudaStream_t s);
+cudaError_t ffma_backward(const Problem& p, const Args& a, const Work& w, bool bf16,
+                          cudaStream_t s);
+
+}  // namespace gdn

@@ -1,0 +1,143 @@
+/*
+ * gdn.h — C ABI of the B200 (sm_100a) chunkwise Gated DeltaNet library.
+ *
+ * The operation (per sequence and value head; gated delta rule as used by Qwen3-Next-style
+ * linear-attention layers and by flash-linear-attention's chunk kernels named on the
+ * "flash-linear-attention 中的 G_T_CONTIG" page: chunk_fwd_kernel_o, chunk_bwd_kernel_dv_local,
+ * chunk_bwd_kernel_dqkwg, chunk_bwd_kernel_dg, wy_fast / prepare_wy_repr_bwd, chunk_delta_h):
+ *
+ *   gate   x_t = g_raw_t + dt_bias[hv];  g_t = -exp(A_log[hv]) * (x_t > 20 ? x_t : log(1 + e^{x_t}))
+ *          (formula and stable softplus: MindSpeed-Ops issue 9, "KDA gate", section "数学公式")
+ *   state  S_t = e^{g_t} S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T      (S: V x K)
+ *   output o_t = scale * S_t q_t
+ *
+ * computed in 64-token chunks (the GDN "cv fusion" block size of 64, Ascend GDN blog,
+ * section "昇腾亲和的Tiling优化") by an exact reassociation of that recurrence.
+ *
+ * Layouts (row-major, contiguous, every base 16-byte aligned):
+ *   q, k              [B, T, H,  K]    dtype (bf16 or fp32)
+ *   v, o, do, dv      [B, T, HV, V]    dtype
+ *   dq, dk            [B, T, H,  K]    dtype
+ *   g_raw, beta       [B, T, HV]       fp32   (raw gate input a_t and the write strength)
+ *   dg, dbeta, dg_raw [B, T, HV]       fp32   (dg = dL/dg_t; dg_raw = dL/d g_raw_t)
+ *   A_log, dt_bias    [HV]             fp32
+ *   dA_log, ddt_bias  [HV]             fp32
+ *   initial_state, final_state, dht, dh0   [Nst, HV, K, V] fp32, h[k][v] = S[v][k],
+ *                     Nst = N (varlen) or B.
+ * Value head hv reads the q/k of k-head hv / (HV / H) (HV must be a multiple of H).
+ * Varlen: cu_seqlens (DEVICE pointer, int64, N+1 entries, cu[0] = 0, non-decreasing,
+ * cu[N] = T) packs N sequences into batch row 0 (B must be 1); chunks never cross a
+ * sequence boundary and each sequence has its own state ("G_T_CONTIG" page, section
+ * "Varlen 场景的三条检查清单": local lengths, offsets relative to bos, int64 cu_seqlens).
+ *
+ * Per-token buffers may be NULL when B*T == 0 (then only states are read or written).
+ *
+ * Ownership: the caller owns every buffer, including the workspace (size from
+ * gdn_workspace_bytes).  Entry points allocate nothing, launch asynchronously on `stream`
+ * (a cudaStream_t passed as void*, NULL = legacy default stream) and return after the
+ * launches are queued.  No exception crosses this boundary.
+ *
+ * Errors: each entry point returns a gdn_status.  Host-detectable problems (null or
+ * misaligned pointers, bad sizes, unsupported K/V/dtype, small workspace) return before any
+ * launch.  Problems only the device can see (cu_seqlens values that are not a valid
+ * partition of [0,T), a bounded wait that ran out) set a status word inside the workspace;
+ * every later kernel of the call then skips its work, and gdn_device_status() returns the
+ * word (it synchronises the stream).
+ */
+#ifndef GDN_B200_H
+#define GDN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gdn_status {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad cu_seqlens */
+  GDN_ERR_UNSUPPORTED = 2,   /* K or V not in {64,128}, unknown dtype */
+  GDN_ERR_WORKSPACE = 3,     /* workspace null/misaligned or smaller than gdn_workspace_bytes */
+  GDN_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
+  GDN_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up (reported by gdn_device_status) */
+} gdn_status;
+
+typedef enum gdn_dtype { GDN_DTYPE_FP32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype;
+
+typedef struct gdn_dims {
+  int64_t B, T, H, HV, K, V;
+  int64_t N;       /* number of packed sequences when cu_seqlens != NULL; ignored otherwise */
+  int32_t dtype;   /* gdn_dtype of q,k,v,o,do,dq,dk,dv; gates, beta and states are fp32 */
+  float scale;     /* output scale; 0 selects 1/sqrt(K) */
+} gdn_dims;
+
+/* Bytes of workspace needed by gdn_chunk_fwd (pass = 0) or gdn_chunk_bwd (pass = 1) for
+ * these dimensions, or 0 if the dimensions are invalid.  With cu_seqlens the bound uses
+ * at most (T + 63 N) / 64 chunks.  `varlen` is 1 when cu_seqlens will be passed. */
+size_t gdn_workspace_bytes(const gdn_dims* d, int varlen, int pass);
+
+/* Forward: o and (optionally) final_state.  initial_state NULL = zero state;
+ * final_state NULL = not written.  Output rows of o are all written. */
+int gdn_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                  const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,
+                  const int64_t* cu_seqlens, const float* initial_state,
+                  void* o, float* final_state,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of L = sum(do * o) + sum(dht * final_state), recomputing the forward
+ * intermediates from the inputs (no saved context).  dht NULL = zero.  Required outputs:
+ * dq, dk, dv, dg, dbeta.  Optional (NULL = skipped): dh0, dg_raw, dA_log, ddt_bias. */
+int gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                  const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,
+                  const int64_t* cu_seqlens, const float* initial_state,
+                  const void* d_o, const float* dht,
+                  void* dq, void* dk, void* dv, float* dg, float* dbeta, float* dh0,
+                  float* dg_raw, float* dA_log, float* ddt_bias,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Upper bound on the number of 64-token chunks (the grid size used for chunk kernels). */
+int64_t gdn_max_chunks(const gdn_dims* d, int varlen);
+
+/* Host-side chunk table: for each chunk in order (sequence-major), 4 int32 values
+ * {sequence n, chunk index c within the sequence, tokens L in the chunk (1..64),
+ *  flat token index of its first token in [B*T]}.  cu_host is a HOST copy of cu_seqlens
+ * (NULL = dense batch).  Writes min(count, cap) entries; returns the chunk count, or a
+ * negative gdn_status on invalid input. */
+int64_t gdn_build_chunk_indices(const gdn_dims* d, const int64_t* cu_host, int32_t* out_host,
+                                int64_t cap);
+
+/* The same table built by the device kernel the forward/backward use (cu_seqlens is a
+ * device pointer, table a device buffer of cap*4 int32 written in the same format; entries
+ * past the count are {-1,-1,0,0}); count_dev (device int32) receives the chunk count, or -1
+ * when cu_seqlens is not a valid partition of [0, T). */
+int gdn_chunk_table_device(const gdn_dims* d, const int64_t* cu_seqlens, int32_t* table,
+                           int64_t cap, int32_t* count_dev, void* stream);
+
+/* Synchronise `stream` and return the device status word of the last call that used
+ * `workspace` (GDN_OK, GDN_ERR_INVALID_ARG for bad cu_seqlens, GDN_ERR_TIMEOUT). */
+int gdn_device_status(const void* workspace, void* stream);
+
+/* Number of kernel launches this library has issued since it was loaded (all threads). */
+int64_t gdn_launch_count(void);
+
+/* Per-kernel device timing: while enabled, every launch is bracketed by CUDA events
+ * recorded on its own stream (adds a little host overhead; for measurement passes only). */
+int gdn_profile(int enable);
+
+/* Synchronises the recorded events, writes {"kernel": [launches, total_ms], ...} as a
+ * NUL-terminated JSON object into buf (truncated to cap-1 bytes), clears the records and
+ * returns the full text length (negative gdn_status on a CUDA error). */
+int64_t gdn_profile_read(char* buf, size_t cap);
+
+/* Human-readable name of a status code (static string). */
+const char* gdn_status_string(int status);
+
+/* Version and build tag (static string), e.g. "gdn-b200 0.1 sm_100a". */
+const char* gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_B200_H */

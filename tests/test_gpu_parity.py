@@ -1,0 +1,157 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle, element by element,
+on the same seeded inputs (the five workloads, block-edge lengths, ragged varlen tails,
+long-memory decay) plus the device chunk table, the device status word, determinism and
+degenerate cases."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from gated_deltanet_chunkwise_chunk_b200 import synth
+
+from .gpu_common import compare, head_select, run_gpu, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _edge_lengths(limit):
+    vals = [int(x) for l in open(os.path.join(GOLDEN, "edge_lengths.txt"))
+            if not l.startswith("#") for x in l.split()]
+    return [v for v in vals if v <= limit]
+
+
+def _assert_parity(case, gpu=None, ref=None, select=None):
+    gpu = run_gpu(case) if gpu is None else gpu
+    ref = run_oracle(case) if ref is None else ref
+    fails, report = compare(gpu, ref, case.dtype, select=select)
+    assert not fails, f"{case.name}: {fails}\n{report}"
+    return report
+
+
+def test_config0_fp32_full():
+    _assert_parity(synth.config_case(0))
+
+
+def test_config1_bf16_full():
+    _assert_parity(synth.config_case(1))
+
+
+@pytest.mark.parametrize("cfg,kheads", [(2, [0, 15]), (3, [5]), (4, [3])])
+def test_full_size_sampled_heads(cfg, kheads):
+    """Full-size run in the bench's launch configuration; the oracle recomputes a sample of
+    k-heads (with their value heads), which are independent problems."""
+    case = synth.config_case(cfg)
+    gpu = run_gpu(case)
+    sub = synth.subset_heads(case, kheads)
+    ref = run_oracle(sub)
+    _assert_parity(sub, gpu=gpu, ref=ref, select=head_select(case, kheads))
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("T", _edge_lengths(300) + [257])
+def test_block_edge_lengths(dtype, T):
+    case = synth.make_case(B=2, T=T, H=1, HV=2, K=128, V=128, dtype=dtype, seed=50 + T, h0=True,
+                           dht=True, name=f"edge{T}")
+    _assert_parity(case)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("KV", [(64, 64), (64, 128), (128, 64)])
+def test_head_dims(dtype, KV):
+    K, V = KV
+    case = synth.make_case(B=1, T=200, H=2, HV=4, K=K, V=V, dtype=dtype, seed=7, h0=True, dht=True,
+                           name=f"K{K}V{V}")
+    _assert_parity(case)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_varlen_ragged(dtype):
+    lens = [1, 63, 64, 65, 127, 128, 129, 300, 0, 17]
+    case = synth.make_case(H=2, HV=4, K=128, V=128, dtype=dtype, seed=11, lengths=lens, h0=True,
+                           dht=True, name="varlen_ragged")
+    _assert_parity(case)
+
+
+def test_long_memory_decay_bf16():
+    """Weak decay (g ~ -1e-3 per token): the state carries information across all chunks."""
+    case = synth.make_case(B=1, T=1024, H=2, HV=4, K=128, V=128, dtype="bf16", seed=12,
+                           long_memory=True, h0=True, dht=True, name="long_memory")
+    _assert_parity(case)
+
+
+def test_long_memory_decay_fp32():
+    case = synth.make_case(B=1, T=1024, H=2, HV=4, K=64, V=64, dtype="fp32", seed=13,
+                           long_memory=True, h0=True, dht=True, name="long_memory32")
+    _assert_parity(case)
+
+
+def test_softplus_passthrough_branch():
+    case = synth.make_case(B=1, T=256, H=2, HV=2, K=64, V=64, dtype="fp32", seed=14, big_a=True,
+                           h0=True, dht=True, name="big_a")
+    a = case.a.numpy()
+    assert (a > 20.5).any() and (a < -20.5).any()
+    _assert_parity(case)
+
+
+def test_empty_input_passes_state_through():
+    case = synth.make_case(B=2, T=0, H=1, HV=2, K=64, V=64, dtype="bf16", seed=15, h0=True,
+                           dht=True, name="T0")
+    gpu = run_gpu(case)
+    np.testing.assert_array_equal(gpu["ht"], case.h0.double().numpy())
+    np.testing.assert_array_equal(gpu["dh0"], case.dht.double().numpy())
+    assert gpu["o"].size == 0 and np.all(gpu["dA_log"] == 0)
+
+
+def test_varlen_with_empty_sequences():
+    case = synth.make_case(H=1, HV=2, K=64, V=64, dtype="fp32", seed=16, lengths=[0, 70, 0, 5],
+                           h0=True, dht=True, name="varlen_empty")
+    rep = _assert_parity(case)
+    gpu = run_gpu(case)
+    np.testing.assert_array_equal(gpu["ht"][0], case.h0[0].double().numpy())
+
+
+def test_device_chunk_table_bit_exact():
+    import gated_deltanet_chunkwise_chunk_b200 as gdn
+    for lens in ([5, 1, 70, 64, 17], [4095, 257, 1000], [0, 64, 0], [1]):
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+        d = gdn.gdn_dims(1, int(cu[-1]), 1, 1, 64, 64, len(lens), 1, 0.0)
+        cap = gdn.max_chunks(d, True)
+        table, count = gdn.gdn_chunk_table_device(d, torch.from_numpy(cu).cuda(), cap)
+        host = gdn.gdn_build_chunk_indices(d, cu)
+        assert count == len(host)
+        t = table.cpu().numpy()
+        assert np.array_equal(t[:count], host)
+        assert (t[count:] == np.array([-1, -1, 0, 0])).all()
+    for B, T in ((2, 200), (1, 32768)):
+        d = gdn.gdn_dims(B, T, 1, 1, 64, 64, B, 1, 0.0)
+        table, count = gdn.gdn_chunk_table_device(d, None)
+        assert np.array_equal(table.cpu().numpy()[:count], gdn.gdn_build_chunk_indices(d, None))
+
+
+def test_invalid_cu_seqlens_sets_device_status():
+    import gated_deltanet_chunkwise_chunk_b200 as gdn
+    case = synth.make_case(H=1, HV=1, K=64, V=64, dtype="bf16", seed=17, lengths=[10, 20])
+    d = {k: (v.cuda() if v is not None else None) for k, v in dict(
+        q=case.q, k=case.k, v=case.v, g_raw=case.a, A_log=case.A_log, dt_bias=case.dt_bias,
+        beta=case.beta).items()}
+    bad = torch.tensor([0, 25, 20], dtype=torch.int64, device="cuda")  # decreasing
+    dims = gdn.make_dims(d["q"], d["v"], bad)
+    ws = torch.zeros(gdn.workspace_bytes(dims, True, False), dtype=torch.uint8, device="cuda")
+    o = torch.full_like(d["v"], 7.0)
+    gdn.gdn_chunk_fwd(**d, cu_seqlens=bad, output_final_state=False, workspace=ws, out=o)
+    assert gdn.gdn_device_status(ws) == 1
+    assert torch.all(o == 7.0)  # no kernel wrote past the failed check
+    good = case.cu_seqlens.cuda()
+    gdn.gdn_chunk_fwd(**d, cu_seqlens=good, output_final_state=False, workspace=ws, out=o)
+    assert gdn.gdn_device_status(ws) == 0
+
+
+def test_run_to_run_bitwise_reproducible():
+    case = synth.make_case(B=1, T=700, H=2, HV=4, K=128, V=128, dtype="bf16", seed=18, h0=True,
+                           dht=True)
+    a, b = run_gpu(case), run_gpu(case)
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
