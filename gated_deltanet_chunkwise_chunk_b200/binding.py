@@ -237,9 +237,10 @@ def profile(enable: bool) -> None:
 def profile_read() -> dict:
     """Per-kernel {name: (launches, total_ms)} since the last read (synchronises)."""
     import json
-    n = lib.gdn_profile_read(None, 0)
+    buf = ctypes.create_string_buffer(1 << 16)
+    n = lib.gdn_profile_read(buf, len(buf))
     if n < 0:
         raise GDNError("gdn_profile_read", -n)
-    buf = ctypes.create_string_buffer(int(n) + 1)
-    lib.gdn_profile_read(buf, len(buf))
+    if n >= len(buf):
+        raise RuntimeError("profile record does not fit the buffer")
     return {k: tuple(v) for k, v in json.loads(buf.value.decode() or "{}").items()}
