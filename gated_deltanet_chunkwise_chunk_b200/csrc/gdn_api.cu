@@ -62,7 +62,8 @@ Plan make_plan(const gdn_dims& d, bool varlen, int pass) {
   pl.chunk_tab = take(NC * sizeof(int4));
   pl.G = take(HV * NC * CH * f);
   pl.beta_p = take(HV * NC * CH * f);
-  const bool ffma = d.dtype == GDN_DTYPE_FP32 || !tc_supported(d);
+  const bool ffma = pass == 0 ? !(d.dtype == GDN_DTYPE_BF16 && tc_supported(d))
+                              : !(d.dtype == GDN_DTYPE_BF16 && tc_bwd_supported(d));
   if (ffma) {
     pl.W = take(NC * HV * CH * K * f);
     pl.Ut = take(NC * HV * CH * V * f);
@@ -241,7 +242,7 @@ int gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v
   cudaError_t e = prologue(p, a, w, s);
   if (e != cudaSuccess) return cuda_status(e);
   const bool bf16 = d->dtype == GDN_DTYPE_BF16;
-  if (bf16 && tc_supported(*d)) {
+  if (bf16 && tc_bwd_supported(*d)) {
     e = tc_backward(p, a, w, static_cast<char*>(workspace) + pl.tc, s);
     if (e != cudaSuccess) return cuda_status(e);
   } else {

@@ -1,13 +1,687 @@
-// tcgen05 path (bf16).  Not yet enabled: every bf16 call takes the FFMA path.
+// tcgen05 path for bf16 tensors with K = V = 128: chunk products on the 5th-generation tensor
+// cores (operands in 128-byte-swizzled shared memory, fed by TMA; fp32 accumulators in TMEM).
+//
+// Per chunk (64 tokens) and value head, with S the state entering the chunk (V x K):
+//   A  = strict_lower(diag(beta) (K K^T * Gam)),  T = (I + A)^-1          (CUDA cores, fp32)
+//   W^T = K^T diag(beta e^G) T^T,   U~^T = V^T diag(beta) T^T              (tensor cores)
+//   U^T = U~^T - S W^T;   S' = e^{G_C} S + (U^T diag(e^{G_C-G})) K         (sequential scan)
+//   O   = scale (diag(e^G) Q S^T + (Q K^T * Gam) U)                        (chunk_fwd_o)
+// Intermediates between kernels are bf16 tiles in HBM, laid out so that one TMA box loads
+// each as a tensor-core operand:  W^T, U~^T, U^T: [unit][128][64];  S (h): [unit][128][128].
+#include <cstdio>
+#include <mutex>
+
+#include "gdn_launch.h"
 #include "gdn_tc.h"
+#include "tc_prims.cuh"
 
 namespace gdn {
 
-bool tc_supported(const gdn_dims&) { return false; }
-size_t tc_workspace_bytes(const gdn_dims&, size_t, int) { return 0; }
-cudaError_t tc_forward(const Problem&, const Args&, const Work&, void*, cudaStream_t) {
-  return cudaErrorNotSupported;
+using bf16 = __nv_bfloat16;
+using namespace tc;
+
+namespace {
+
+constexpr int D = 128;                 // head dimension (K = V = 128 on this path)
+constexpr int TILE64 = 64 * 128;       // bytes of a [64 rows x 64 bf16] block
+constexpr int TILE128 = 128 * 128;     // bytes of a [128 rows x 64 bf16] block
+
+// ------------------------------------------------------------------ tensor maps (host)
+typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                             const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                             CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                             CUtensorMapFloatOOBfill);
+
+EncodeFn encoder() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  return fn;
 }
+
+// bf16 tensor viewed as [outer][rows][cols] (cols contiguous) with box {64, box_rows, 1}
+// (128-byte swizzle, out-of-bounds rows read as zero).
+bool map3(CUtensorMap* m, const void* base, uint64_t cols, uint64_t mid, uint64_t outer,
+          uint64_t mid_stride_elems, uint64_t outer_stride_elems, uint32_t box_mid, uint32_t box_outer) {
+  EncodeFn enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cols, mid, outer};
+  cuuint64_t strides[2] = {mid_stride_elems * 2, outer_stride_elems * 2};
+  cuuint32_t box[3] = {64, box_mid, box_outer};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// token tensor [ntok][heads][128] -> 3D map (col, head, token), box = 64 cols x 1 head x 64 tokens
+bool map_tokens(CUtensorMap* m, const void* base, int ntok, int heads) {
+  return map3(m, base, D, heads, ntok, D, (uint64_t)heads * D, 1, 64);
+}
+// 2D row-major [rows][cols] bf16, box = 64 cols x box_rows rows (as a 3D map with outer = 1)
+bool map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  return map3(m, base, cols, rows, 1, cols, rows * cols, box_rows, 1);
+}
+
+struct TcMaps {
+  CUtensorMap q, k, v, dO;     // token tensors
+  CUtensorMap WT, UtT, UT;     // [unit*128][64]
+  CUtensorMap h;               // [unit*128][128]
+};
+
+struct TcWork {
+  bf16* WT;     // [NC*HV][128][64]
+  bf16* UtT;    // [NC*HV][128][64]
+  bf16* UT;     // [NC*HV][128][64]
+  bf16* h;      // [NC*HV][128][128]
+  bf16* Tm;     // [NC*HV][64][64]   (backward only)
+};
+
+size_t align_up(size_t x) { return (x + 1023) / 1024 * 1024; }
+
+TcWork carve_tc(void* base, size_t NC, size_t HV, int pass) {
+  char* b = static_cast<char*>(base);
+  TcWork t{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    char* p = b + o;
+    o += align_up(bytes);
+    return p;
+  };
+  const size_t units = NC * HV;
+  t.WT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
+  t.UtT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
+  t.UT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
+  t.h = reinterpret_cast<bf16*>(take(units * D * D * 2));
+  if (pass == 1) t.Tm = reinterpret_cast<bf16*>(take(units * 64 * 64 * 2));
+  return t;
+}
+
+size_t tc_bytes(size_t NC, size_t HV, int pass) {
+  const size_t units = NC * HV;
+  size_t o = 3 * align_up(units * D * 64 * 2) + align_up(units * D * D * 2);
+  if (pass == 1) o += align_up(units * 64 * 64 * 2);
+  return o;
+}
+
+// ------------------------------------------------------------------ device helpers
+__device__ __forceinline__ unsigned char* align1k(unsigned char* p) {
+  return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Zero rows [L, 64) of a [64 x 128] bf16 token tile (two 8 KB column blocks).
+__device__ __forceinline__ void zero_tail_rows(unsigned char* tile, int L, int tid, int nthr) {
+  const int n = (64 - L) * 16;  // 16-byte chunks per row (2 blocks x 8)
+  for (int i = tid; i < n; i += nthr) {
+    const int r = L + i / 16, j = i % 16;
+    *reinterpret_cast<uint4*>(tile + sw128_chunk(r, j, TILE64)) = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Reads 8 bf16 (one 16-byte swizzled chunk) as floats.
+__device__ __forceinline__ void ld_chunk_f(const unsigned char* tile, int r, int j, int block_bytes,
+                                           float* f) {
+  const uint4 v = *reinterpret_cast<const uint4*>(tile + sw128_chunk(r, j, block_bytes));
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 x = __bfloat1622float2(h[i]);
+    f[2 * i] = x.x;
+    f[2 * i + 1] = x.y;
+  }
+}
+__device__ __forceinline__ void st_chunk_f(unsigned char* tile, int r, int j, int block_bytes,
+                                           const float* f) {
+  uint4 v;
+  v.x = pack_bf16(f[0], f[1]);
+  v.y = pack_bf16(f[2], f[3]);
+  v.z = pack_bf16(f[4], f[5]);
+  v.w = pack_bf16(f[6], f[7]);
+  *reinterpret_cast<uint4*>(tile + sw128_chunk(r, j, block_bytes)) = v;
+}
+
+__device__ __forceinline__ bool failed(const Work& w) { return *((volatile int*)w.status) != 0; }
+
+// ======================================================================================
+// WY representation.  One CTA (128 threads) per (chunk, value head).
+//   KK^T (M=64) -> A, T = (I+A)^-1 (fp32, one column per thread) ->
+//   W^T = K^T (T diag(beta e^G))^T,  U~^T = V^T (T diag(beta))^T   (M=128, N=64, K=64)
+// ======================================================================================
+__global__ void __launch_bounds__(128) k_tc_wy(Problem p, Work w, TcWork t,
+                                               const __grid_constant__ CUtensorMap mk,
+                                               const __grid_constant__ CUtensorMap mv, int store_T) {
+  if (failed(w)) return;
+  const int gc = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
+  const int4 e = w.chunk_tab[gc];
+  if (e.x < 0) return;
+  const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  extern __shared__ unsigned char smraw[];
+  unsigned char* sm = align1k(smraw);
+  unsigned char* sK = sm;                    // [64][128] bf16, 2 blocks
+  unsigned char* sV = sK + 2 * TILE64;       // [64][128]
+  unsigned char* sTX = sV + 2 * TILE64;      // [64][64]  T diag(beta e^G)
+  unsigned char* sTY = sTX + TILE64;         // [64][64]  T diag(beta)
+  float* sA = reinterpret_cast<float*>(sTY + TILE64);  // [64][65]
+  float* sT = sA + 64 * 65;                            // [64][65]
+  float* sG = sT + 64 * 65;
+  float* sb = sG + 64;
+  __shared__ uint64_t bar[2];
+  __shared__ uint32_t tslot;
+  int* err = w.status;
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tslot, 256);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_expect_tx(&bar[0], 4 * TILE64);
+    tma_load_3d(sK, &mk, 0, hk, tok0, &bar[0]);
+    tma_load_3d(sK + TILE64, &mk, 64, hk, tok0, &bar[0]);
+    tma_load_3d(sV, &mv, 0, hv, tok0, &bar[0]);
+    tma_load_3d(sV + TILE64, &mv, 64, hv, tok0, &bar[0]);
+  }
+  if (tid < 64) {
+    const size_t o = ((size_t)hv * p.NCmax + gc) * 64 + tid;
+    sG[tid] = w.G[o];
+    sb[tid] = w.beta_p[o];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tslot;
+  bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
+  if (L < 64) {
+    zero_tail_rows(sK, L, tid, 128);
+    zero_tail_rows(sV, L, tid, 128);
+  }
+  fence_proxy_async();
+  __syncthreads();
+  // KK^T: M=64, N=64, K=128 (both K-major) -> TMEM cols [0,64)
+  if (ok && tid == 0) {
+    const uint32_t k = smem_u32(sK);
+    for (int s = 0; s < 8; ++s)
+      mma_bf16(taddr(tb, 0, 0), desc_kmajor(k, s, TILE64), desc_kmajor(k, s, TILE64),
+               idesc_bf16(64, 64, false, false), s > 0);
+    mma_commit(&bar[1]);
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
+  tc_fence_after();
+  if (ok) {
+    // M=64 accumulator: row 16*warp + lane (lanes 0..15) of the warp's sub-partition
+    float v[16];
+    const int r = warp * 16 + lane;
+    for (int c = 0; c < 64; c += 16) {
+      tmem_ld16(taddr(tb, warp * 32, c), v);
+      tmem_wait_ld();
+      if (lane < 16)
+        for (int i = 0; i < 16; ++i) {
+          const int cc = c + i;
+          sA[r * 65 + cc] = cc < r ? sb[r] * v[i] * expf(sG[r] - sG[cc]) : 0.f;
+        }
+    }
+  }
+  __syncthreads();
+  // T = (I + A)^-1 by forward substitution, one column per thread
+  if (tid < 64) {
+    const int n = tid;
+    for (int rr = 0; rr < 64; ++rr) {
+      float s = rr == n ? 1.f : 0.f;
+      if (rr > n)
+        for (int j = n; j < rr; ++j) s -= sA[rr * 65 + j] * sT[j * 65 + n];
+      sT[rr * 65 + n] = s;
+    }
+  }
+  __syncthreads();
+  // bf16 operand tiles TX[i][j] = T[i][j] beta_j e^{G_j}, TY[i][j] = T[i][j] beta_j
+  for (int idx = tid; idx < 64 * 8; idx += 128) {
+    const int i = idx / 8, jc = idx % 8;
+    float fx[8], fy[8];
+    for (int q = 0; q < 8; ++q) {
+      const int j = jc * 8 + q;
+      const float tv = sT[i * 65 + j];
+      fy[q] = tv * sb[j];
+      fx[q] = fy[q] * expf(sG[j]);
+    }
+    st_chunk_f(sTX, i, jc, TILE64, fx);
+    st_chunk_f(sTY, i, jc, TILE64, fy);
+    if (store_T) {
+      float ft[8];
+      for (int q = 0; q < 8; ++q) ft[q] = sT[i * 65 + jc * 8 + q];
+      uint4 pk;
+      pk.x = pack_bf16(ft[0], ft[1]);
+      pk.y = pack_bf16(ft[2], ft[3]);
+      pk.z = pack_bf16(ft[4], ft[5]);
+      pk.w = pack_bf16(ft[6], ft[7]);
+      *reinterpret_cast<uint4*>(t.Tm + (((size_t)gc * p.HV + hv) * 64 + i) * 64 + jc * 8) = pk;
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // W^T = K^T TX^T, U~^T = V^T TY^T: M=128 (A MN-major), N=64, K=64 (B K-major)
+  if (ok && tid == 0) {
+    const uint32_t k = smem_u32(sK), vv = smem_u32(sV), tx = smem_u32(sTX), ty = smem_u32(sTY);
+    for (int s = 0; s < 4; ++s) {
+      mma_bf16(taddr(tb, 0, 64), desc_mnmajor(k, s, TILE64), desc_kmajor(tx, s, TILE64),
+               idesc_bf16(128, 64, true, false), s > 0);
+      mma_bf16(taddr(tb, 0, 128), desc_mnmajor(vv, s, TILE64), desc_kmajor(ty, s, TILE64),
+               idesc_bf16(128, 64, true, false), s > 0);
+    }
+    mma_commit(&bar[1]);
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
+  tc_fence_after();
+  if (ok) {
+    // row = feature index (k for W^T, v for U~^T), 64 token columns -> global rows of 128 B
+    const int r = warp * 32 + lane;
+    const size_t unit = (size_t)gc * p.HV + hv;
+    bf16* wrow = t.WT + (unit * D + r) * 64;
+    bf16* urow = t.UtT + (unit * D + r) * 64;
+    float v[16];
+    for (int c = 0; c < 64; c += 16) {
+      tmem_ld16(taddr(tb, warp * 32, 64 + c), v);
+      tmem_wait_ld();
+      uint4 a, b;
+      a.x = pack_bf16(v[0], v[1]); a.y = pack_bf16(v[2], v[3]);
+      a.z = pack_bf16(v[4], v[5]); a.w = pack_bf16(v[6], v[7]);
+      b.x = pack_bf16(v[8], v[9]); b.y = pack_bf16(v[10], v[11]);
+      b.z = pack_bf16(v[12], v[13]); b.w = pack_bf16(v[14], v[15]);
+      *reinterpret_cast<uint4*>(wrow + c) = a;
+      *reinterpret_cast<uint4*>(wrow + c + 8) = b;
+      tmem_ld16(taddr(tb, warp * 32, 128 + c), v);
+      tmem_wait_ld();
+      a.x = pack_bf16(v[0], v[1]); a.y = pack_bf16(v[2], v[3]);
+      a.z = pack_bf16(v[4], v[5]); a.w = pack_bf16(v[6], v[7]);
+      b.x = pack_bf16(v[8], v[9]); b.y = pack_bf16(v[10], v[11]);
+      b.z = pack_bf16(v[12], v[13]); b.w = pack_bf16(v[14], v[15]);
+      *reinterpret_cast<uint4*>(urow + c) = a;
+      *reinterpret_cast<uint4*>(urow + c + 8) = b;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 256);
+}
+
+// ======================================================================================
+// Sequential state scan.  One CTA (256 threads) per (sequence, value head).  Thread
+// (v = 32*(warp%4) + lane, half = warp/4) keeps S[v][64*half .. 64*half+63] in fp32
+// registers.  Per chunk:
+//   MMA1: D1 = S_bf16 W^T          (M=128 v, N=64 i, K=128 k)
+//   U^T = U~^T - D1; Ud^T = U^T diag(e^{G_C-G})  (bf16 tiles in smem)
+//   MMA2: D2 = Ud^T K              (M=128 v, N=128 k, K=64 i)
+//   S = e^{G_C} S + D2
+// S (bf16, the state entering each chunk) and U^T are written out by TMA stores; the
+// chunk's W^T, U~^T and K tiles are prefetched one chunk ahead (double buffer).
+// ======================================================================================
+struct ScanSmem {
+  static constexpr int S = 0;                       // [128][128] bf16: 2 x 16 KB
+  static constexpr int BUF = 2 * TILE128;           // 2 x {W^T 16K, U~^T 16K, K 16K}
+  static constexpr int BUF_BYTES = 3 * TILE128;
+  static constexpr int UD = BUF + 2 * BUF_BYTES;    // [128][64] Ud^T
+  static constexpr int UO = UD + TILE128;           // [128][64] U^T staging
+  static constexpr int G = UO + TILE128;            // 2 x 64 floats
+  static constexpr int DEC = G + 2 * 256;           // 64 floats e^{G_C - G_i}
+  static constexpr int TOTAL = DEC + 256;
+};
+
+__global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, TcWork t,
+                                                     const __grid_constant__ CUtensorMap mk,
+                                                     const __grid_constant__ CUtensorMap mWT,
+                                                     const __grid_constant__ CUtensorMap mUtT,
+                                                     const __grid_constant__ CUtensorMap mUT,
+                                                     const __grid_constant__ CUtensorMap mh,
+                                                     int write_final) {
+  if (failed(w)) return;
+  const int n = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
+  const int4 sq = w.seq_tab[n];
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int v = 32 * (warp & 3) + lane, half = warp >> 2;
+  extern __shared__ unsigned char smraw[];
+  unsigned char* sm = align1k(smraw);
+  unsigned char* sS = sm + ScanSmem::S;
+  unsigned char* sUd = sm + ScanSmem::UD;
+  unsigned char* sUo = sm + ScanSmem::UO;
+  float* sGb = reinterpret_cast<float*>(sm + ScanSmem::G);
+  float* sDec = reinterpret_cast<float*>(sm + ScanSmem::DEC);
+  __shared__ uint64_t barT[2], barM;
+  __shared__ uint32_t tslot;
+  int* err = w.status;
+  if (tid == 0) {
+    mbar_init(&barT[0], 1);
+    mbar_init(&barT[1], 1);
+    mbar_init(&barM, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tslot, 256);
+    tmem_relinquish();
+  }
+  // initial state (fp32) -> registers; bf16 copy -> sS
+  float S[64];
+  const size_t st = ((size_t)n * p.HV + hv) * D * D;  // [K][V] fp32 states
+  for (int i = 0; i < 64; ++i) {
+    const int kk = half * 64 + i;
+    S[i] = a.h0 ? a.h0[st + (size_t)kk * D + v] : 0.f;
+  }
+  for (int j = 0; j < 8; ++j) st_chunk_f(sS, v, half * 8 + j, TILE128, &S[8 * j]);
+  auto issue = [&](int c) {
+    const int gc = sq.x + c, buf = c & 1;
+    const int4 e = w.chunk_tab[gc];
+    unsigned char* b = sm + ScanSmem::BUF + buf * ScanSmem::BUF_BYTES;
+    const int row = (gc * p.HV + hv) * D;
+    mbar_expect_tx(&barT[buf], 3 * TILE128);
+    tma_load_3d(b, &mWT, 0, row, 0, &barT[buf]);
+    tma_load_3d(b + TILE128, &mUtT, 0, row, 0, &barT[buf]);
+    tma_load_3d(b + 2 * TILE128, &mk, 0, hk, e.w, &barT[buf]);
+    tma_load_3d(b + 2 * TILE128 + TILE64, &mk, 64, hk, e.w, &barT[buf]);
+  };
+  if (tid == 0 && sq.y > 0) issue(0);
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tslot;
+  const uint32_t tD1 = taddr(tb, 0, 0), tD2 = taddr(tb, 0, 64);
+  uint32_t phT[2] = {0, 0}, phM = 0;
+  bool ok = true;
+  for (int c = 0; c < sq.y && ok; ++c) {
+    const int gc = sq.x + c, buf = c & 1;
+    unsigned char* b = sm + ScanSmem::BUF + buf * ScanSmem::BUF_BYTES;
+    const uint32_t unit_row = (uint32_t)(gc * p.HV + hv) * D;
+    float* sG = sGb + buf * 64;
+    if (tid == 0 && c + 1 < sq.y) issue(c + 1);
+    if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
+    ok = __syncthreads_and(mbar_wait(&barT[buf], phT[buf], err));
+    phT[buf] ^= 1;
+    if (tid < 64) sDec[tid] = expf(sG[63] - sG[tid]);
+    // S entering this chunk -> h (TMA store), MMA1
+    if (ok && tid == 0) {
+      tma_store_3d(&mh, sS, 0, unit_row, 0);
+      tma_store_3d(&mh, sS + TILE128, 64, unit_row, 0);
+      tma_store_commit();
+      const uint32_t s_ = smem_u32(sS), wt = smem_u32(b);
+      for (int s = 0; s < 8; ++s)
+        mma_bf16(tD1, desc_kmajor(s_, s, TILE128), desc_mnmajor(wt, s, TILE128),
+                 idesc_bf16(128, 64, false, true), s > 0);
+      mma_commit(&barM);
+    }
+    ok = __syncthreads_and(ok && mbar_wait(&barM, phM, err));
+    phM ^= 1;
+    tc_fence_after();
+    if (!ok) break;
+    // U^T = U~^T - D1 for columns [32*half, 32*half+32); Ud^T = U^T * e^{G_C - G}
+    {
+      float d[32];
+      tmem_ld16(taddr(tb, 32 * (warp & 3), 32 * half), d);
+      tmem_ld16(taddr(tb, 32 * (warp & 3), 32 * half + 16), d + 16);
+      tmem_wait_ld();
+      const unsigned char* ut = b + TILE128;
+      if (tid == 0) tma_store_wait_read0();  // previous U^T staging store has read sUo
+      __syncthreads();
+      for (int j = 0; j < 4; ++j) {
+        float u[8], ud[8];
+        ld_chunk_f(ut, v, half * 4 + j, TILE128, u);
+        for (int q = 0; q < 8; ++q) {
+          u[q] -= d[8 * j + q];
+          ud[q] = u[q] * sDec[32 * half + 8 * j + q];
+        }
+        st_chunk_f(sUo, v, half * 4 + j, TILE128, u);
+        st_chunk_f(sUd, v, half * 4 + j, TILE128, ud);
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      tma_store_3d(&mUT, sUo, 0, unit_row, 0);
+      tma_store_commit();
+      const uint32_t ud = smem_u32(sUd), kt = smem_u32(b + 2 * TILE128);
+      for (int s = 0; s < 4; ++s)
+        mma_bf16(tD2, desc_kmajor(ud, s, TILE128), desc_mnmajor(kt, s, TILE64),
+                 idesc_bf16(128, 128, false, true), s > 0);
+      mma_commit(&barM);
+    }
+    ok = __syncthreads_and(mbar_wait(&barM, phM, err));
+    phM ^= 1;
+    tc_fence_after();
+    if (!ok) break;
+    {
+      const float eg = expf(sG[63]);
+      for (int cc = 0; cc < 64; cc += 16) {
+        float d[16];
+        tmem_ld16(taddr(tb, 32 * (warp & 3), 64 + 64 * half + cc), d);
+        tmem_wait_ld();
+        for (int i = 0; i < 16; ++i) S[cc + i] = eg * S[cc + i] + d[i];
+      }
+    }
+    if (tid == 0) tma_store_wait_read0();  // the h store has finished reading sS
+    __syncthreads();
+    for (int j = 0; j < 8; ++j) st_chunk_f(sS, v, half * 8 + j, TILE128, &S[8 * j]);
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  if (tid == 0) tma_store_wait0();
+  if (ok && write_final && a.ht)
+    for (int i = 0; i < 64; ++i) a.ht[st + (size_t)(half * 64 + i) * D + v] = S[i];
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tslot, 256);
+}
+
+// ======================================================================================
+// chunk_fwd_o.  One CTA (256 threads) per (chunk, value head):
+//   X = Q S^T (M=64, N=128), QK = Q K^T (M=64, N=64) -> P = QK * Gam (bf16 tile)
+//   Y = P U (M=64, N=128, B = U^T K-major);  O = scale (e^{G_i} X + Y)
+// ======================================================================================
+__global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWork t,
+                                                const __grid_constant__ CUtensorMap mq,
+                                                const __grid_constant__ CUtensorMap mk,
+                                                const __grid_constant__ CUtensorMap mUT,
+                                                const __grid_constant__ CUtensorMap mh) {
+  if (failed(w)) return;
+  const int gc = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
+  const int4 e = w.chunk_tab[gc];
+  if (e.x < 0) return;
+  const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  extern __shared__ unsigned char smraw[];
+  unsigned char* sm = align1k(smraw);
+  unsigned char* sQ = sm;                    // [64][128]
+  unsigned char* sK = sQ + 2 * TILE64;       // [64][128]
+  unsigned char* sH = sK + 2 * TILE64;       // [128][128]
+  unsigned char* sU = sH + 2 * TILE128;      // [128][64]  U^T
+  unsigned char* sP = sU + TILE128;          // [64][64]
+  float* sG = reinterpret_cast<float*>(sP + TILE64);
+  __shared__ uint64_t bar[2];
+  __shared__ uint32_t tslot;
+  int* err = w.status;
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tslot, 256);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    const int row = (gc * p.HV + hv) * D;
+    mbar_expect_tx(&bar[0], 4 * TILE64 + 3 * TILE128);
+    tma_load_3d(sQ, &mq, 0, hk, tok0, &bar[0]);
+    tma_load_3d(sQ + TILE64, &mq, 64, hk, tok0, &bar[0]);
+    tma_load_3d(sK, &mk, 0, hk, tok0, &bar[0]);
+    tma_load_3d(sK + TILE64, &mk, 64, hk, tok0, &bar[0]);
+    tma_load_3d(sH, &mh, 0, row, 0, &bar[0]);
+    tma_load_3d(sH + TILE128, &mh, 64, row, 0, &bar[0]);
+    tma_load_3d(sU, &mUT, 0, row, 0, &bar[0]);
+  }
+  if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tslot;
+  bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
+  if (ok && tid == 0) {
+    const uint32_t q = smem_u32(sQ), k = smem_u32(sK), h = smem_u32(sH);
+    for (int s = 0; s < 8; ++s) {
+      mma_bf16(taddr(tb, 0, 0), desc_kmajor(q, s, TILE64), desc_kmajor(h, s, TILE128),
+               idesc_bf16(64, 128, false, false), s > 0);
+      mma_bf16(taddr(tb, 0, 128), desc_kmajor(q, s, TILE64), desc_kmajor(k, s, TILE64),
+               idesc_bf16(64, 64, false, false), s > 0);
+    }
+    mma_commit(&bar[1]);
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
+  tc_fence_after();
+  // P = QK * Gam (lower incl. diagonal): row i = 16*(warp%4) + lane (lanes < 16), columns
+  // [32*half, 32*half + 32)
+  const int i = 16 * (warp & 3) + lane, half = warp >> 2;
+  if (ok) {
+    float d[32];
+    tmem_ld16(taddr(tb, 32 * (warp & 3), 128 + 32 * half), d);
+    tmem_ld16(taddr(tb, 32 * (warp & 3), 128 + 32 * half + 16), d + 16);
+    tmem_wait_ld();
+    if (lane < 16) {
+      const float gi = sG[i];
+      for (int j = 0; j < 4; ++j) {
+        float f[8];
+        for (int q = 0; q < 8; ++q) {
+          const int jj = 32 * half + 8 * j + q;
+          f[q] = jj <= i ? d[8 * j + q] * expf(gi - sG[jj]) : 0.f;
+        }
+        st_chunk_f(sP, i, half * 4 + j, TILE64, f);
+      }
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (ok && tid == 0) {
+    const uint32_t pp = smem_u32(sP), u = smem_u32(sU);
+    for (int s = 0; s < 4; ++s)
+      mma_bf16(taddr(tb, 0, 128), desc_kmajor(pp, s, TILE64), desc_kmajor(u, s, TILE128),
+               idesc_bf16(64, 128, false, false), s > 0);
+    mma_commit(&bar[1]);
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
+  tc_fence_after();
+  if (ok) {
+    const float eg = expf(sG[i]) * p.scale;
+    bf16* orow = static_cast<bf16*>(a.o) + ((size_t)(tok0 + i) * p.HV + hv) * D + 64 * half;
+    for (int cc = 0; cc < 64; cc += 16) {
+      float x[16], y[16];
+      tmem_ld16(taddr(tb, 32 * (warp & 3), 64 * half + cc), x);
+      tmem_ld16(taddr(tb, 32 * (warp & 3), 128 + 64 * half + cc), y);
+      tmem_wait_ld();
+      if (lane < 16 && i < L) {
+        uint4 o0, o1;
+        float f[16];
+        for (int q = 0; q < 16; ++q) f[q] = eg * x[q] + p.scale * y[q];
+        o0.x = pack_bf16(f[0], f[1]); o0.y = pack_bf16(f[2], f[3]);
+        o0.z = pack_bf16(f[4], f[5]); o0.w = pack_bf16(f[6], f[7]);
+        o1.x = pack_bf16(f[8], f[9]); o1.y = pack_bf16(f[10], f[11]);
+        o1.z = pack_bf16(f[12], f[13]); o1.w = pack_bf16(f[14], f[15]);
+        *reinterpret_cast<uint4*>(orow + cc) = o0;
+        *reinterpret_cast<uint4*>(orow + cc + 8) = o1;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 256);
+}
+
+// ------------------------------------------------------------------ host side
+struct Launch {
+  TcMaps m;
+  TcWork t;
+  bool ok = true;
+};
+
+Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
+  Launch L;
+  const int ntok = p.B * p.T;
+  L.t = carve_tc(tc_ws, (size_t)p.NCmax, (size_t)p.HV, pass);
+  const uint64_t urows = (uint64_t)p.NCmax * p.HV * D;
+  L.ok &= map_tokens(&L.m.q, a.q, ntok, p.H);
+  L.ok &= map_tokens(&L.m.k, a.k, ntok, p.H);
+  L.ok &= map_tokens(&L.m.v, a.v, ntok, p.HV);
+  if (a.dO) L.ok &= map_tokens(&L.m.dO, a.dO, ntok, p.HV);
+  L.ok &= map_rows(&L.m.WT, L.t.WT, urows, 64, 128);
+  L.ok &= map_rows(&L.m.UtT, L.t.UtT, urows, 64, 128);
+  L.ok &= map_rows(&L.m.UT, L.t.UT, urows, 64, 128);
+  L.ok &= map_rows(&L.m.h, L.t.h, urows, 128, 128);
+  return L;
+}
+
+template <typename K, typename... Args_>
+cudaError_t go(const char* name, K kern, dim3 grid, int threads, size_t smem, cudaStream_t s,
+               Args_... args) {
+  if (grid.x == 0 || grid.y == 0) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  ProfScope ps(name, s);
+  kern<<<grid, threads, smem, s>>>(args...);
+  return cudaGetLastError();
+}
+
+cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const Launch& L,
+                         bool bwd_prep, cudaStream_t s) {
+  if (!L.ok) return cudaErrorInvalidValue;
+  cudaError_t e;
+  const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV);
+  const size_t wy_smem = 1024 + 6 * TILE64 + 2 * 64 * 65 * 4 + 2 * 64 * 4;
+  if ((e = go("tc_wy", k_tc_wy, gu, 128, wy_smem, s, p, w, L.t, L.m.k, L.m.v, bwd_prep ? 1 : 0)))
+    return e;
+  Args a2 = a;
+  if ((e = go("tc_scan_fwd", k_tc_scan_fwd, gs, 256, (size_t)1024 + ScanSmem::TOTAL, s, p, a2, w,
+              L.t, L.m.k, L.m.WT, L.m.UtT, L.m.UT, L.m.h, bwd_prep ? 0 : 1)))
+    return e;
+  if (!bwd_prep) {
+    const size_t out_smem = 1024 + 5 * TILE64 + 3 * TILE128 + 256;
+    if ((e = go("tc_out", k_tc_out, gu, 256, out_smem, s, p, a, w, L.t, L.m.q, L.m.k, L.m.UT, L.m.h)))
+      return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+bool tc_supported(const gdn_dims& d) {
+  static const bool disabled = getenv("GDN_DISABLE_TC") != nullptr;
+  return !disabled && d.dtype == GDN_DTYPE_BF16 && d.K == 128 && d.V == 128 && d.B * d.T > 0 &&
+         encoder() != nullptr;
+}
+
+bool tc_bwd_supported(const gdn_dims&) { return false; }
+
+size_t tc_workspace_bytes(const gdn_dims& d, size_t NC, int pass) {
+  return tc_bytes(NC, (size_t)d.HV, pass);
+}
+
+cudaError_t tc_forward(const Problem& p, const Args& a, const Work& w, void* tc_ws, cudaStream_t s) {
+  Launch L = setup(p, a, tc_ws, 0);
+  return forward_impl(p, a, w, L, false, s);
+}
+
 cudaError_t tc_backward(const Problem&, const Args&, const Work&, void*, cudaStream_t) {
   return cudaErrorNotSupported;
 }

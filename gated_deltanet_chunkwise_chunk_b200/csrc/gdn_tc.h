@@ -10,6 +10,8 @@ namespace gdn {
 
 // True when the tcgen05 kernels cover these dimensions (bf16, K = V = 128).
 bool tc_supported(const gdn_dims& d);
+// True when the tcgen05 backward kernels cover them as well.
+bool tc_bwd_supported(const gdn_dims& d);
 // Bytes of the tcgen05 path's own workspace region for NC chunks.
 size_t tc_workspace_bytes(const gdn_dims& d, size_t NC, int pass);
 cudaError_t tc_forward(const Problem& p, const Args& a, const Work& w, void* tc_ws, cudaStream_t s);
