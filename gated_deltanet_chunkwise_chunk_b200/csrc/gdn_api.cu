@@ -80,6 +80,11 @@ Plan make_plan(const gdn_dims& d, bool varlen, int pass) {
       pl.tmp = take(NC * HV * CH * 128 * f);
     }
   } else {
+    if (pass == 1) {  // fp32 per-value-head dq/dk shares and dG, read by the final assembly
+      pl.dqp = take(NC * HV * CH * K * f);
+      pl.dkp = take(NC * HV * CH * K * f);
+      pl.dG = take(HV * NC * CH * f);
+    }
     pl.tc = take(tc_workspace_bytes(d, NC, pass));
   }
   pl.total = o;

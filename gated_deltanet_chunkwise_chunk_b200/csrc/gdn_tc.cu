@@ -9,144 +9,14 @@
 // Intermediates between kernels are bf16 tiles in HBM, laid out so that one TMA box loads
 // each as a tensor-core operand:  W^T, U~^T, U^T: [unit][128][64];  S (h): [unit][128][128].
 #include <cstdio>
-#include <mutex>
 
-#include "gdn_launch.h"
-#include "gdn_tc.h"
-#include "tc_prims.cuh"
+#include "gdn_tc_common.cuh"
 
 namespace gdn {
 
-using bf16 = __nv_bfloat16;
-using namespace tc;
+using namespace tcx;
 
 namespace {
-
-constexpr int D = 128;                 // head dimension (K = V = 128 on this path)
-constexpr int TILE64 = 64 * 128;       // bytes of a [64 rows x 64 bf16] block
-constexpr int TILE128 = 128 * 128;     // bytes of a [128 rows x 64 bf16] block
-
-// ------------------------------------------------------------------ tensor maps (host)
-typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                             const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
-                             CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                             CUtensorMapFloatOOBfill);
-
-EncodeFn encoder() {
-  static EncodeFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn>(p);
-  });
-  return fn;
-}
-
-// bf16 tensor viewed as [outer][rows][cols] (cols contiguous) with box {64, box_rows, 1}
-// (128-byte swizzle, out-of-bounds rows read as zero).
-bool map3(CUtensorMap* m, const void* base, uint64_t cols, uint64_t mid, uint64_t outer,
-          uint64_t mid_stride_elems, uint64_t outer_stride_elems, uint32_t box_mid, uint32_t box_outer) {
-  EncodeFn enc = encoder();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {cols, mid, outer};
-  cuuint64_t strides[2] = {mid_stride_elems * 2, outer_stride_elems * 2};
-  cuuint32_t box[3] = {64, box_mid, box_outer};
-  cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// token tensor [ntok][heads][128] -> 3D map (col, head, token), box = 64 cols x 1 head x 64 tokens
-bool map_tokens(CUtensorMap* m, const void* base, int ntok, int heads) {
-  return map3(m, base, D, heads, ntok, D, (uint64_t)heads * D, 1, 64);
-}
-// 2D row-major [rows][cols] bf16, box = 64 cols x box_rows rows (as a 3D map with outer = 1)
-bool map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  return map3(m, base, cols, rows, 1, cols, rows * cols, box_rows, 1);
-}
-
-struct TcMaps {
-  CUtensorMap q, k, v, dO;     // token tensors
-  CUtensorMap WT, UtT, UT;     // [unit*128][64]
-  CUtensorMap h;               // [unit*128][128]
-};
-
-struct TcWork {
-  bf16* WT;     // [NC*HV][128][64]
-  bf16* UtT;    // [NC*HV][128][64]
-  bf16* UT;     // [NC*HV][128][64]
-  bf16* h;      // [NC*HV][128][128]
-  bf16* Tm;     // [NC*HV][64][64]   (backward only)
-};
-
-size_t align_up(size_t x) { return (x + 1023) / 1024 * 1024; }
-
-TcWork carve_tc(void* base, size_t NC, size_t HV, int pass) {
-  char* b = static_cast<char*>(base);
-  TcWork t{};
-  size_t o = 0;
-  auto take = [&](size_t bytes) {
-    char* p = b + o;
-    o += align_up(bytes);
-    return p;
-  };
-  const size_t units = NC * HV;
-  t.WT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
-  t.UtT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
-  t.UT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
-  t.h = reinterpret_cast<bf16*>(take(units * D * D * 2));
-  if (pass == 1) t.Tm = reinterpret_cast<bf16*>(take(units * 64 * 64 * 2));
-  return t;
-}
-
-size_t tc_bytes(size_t NC, size_t HV, int pass) {
-  const size_t units = NC * HV;
-  size_t o = 3 * align_up(units * D * 64 * 2) + align_up(units * D * D * 2);
-  if (pass == 1) o += align_up(units * 64 * 64 * 2);
-  return o;
-}
-
-// ------------------------------------------------------------------ device helpers
-__device__ __forceinline__ unsigned char* align1k(unsigned char* p) {
-  return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-// Zero rows [L, 64) of a [64 x 128] bf16 token tile (two 8 KB column blocks).
-__device__ __forceinline__ void zero_tail_rows(unsigned char* tile, int L, int tid, int nthr) {
-  const int n = (64 - L) * 16;  // 16-byte chunks per row (2 blocks x 8)
-  for (int i = tid; i < n; i += nthr) {
-    const int r = L + i / 16, j = i % 16;
-    *reinterpret_cast<uint4*>(tile + sw128_chunk(r, j, TILE64)) = make_uint4(0, 0, 0, 0);
-  }
-}
-
-// Reads 8 bf16 (one 16-byte swizzled chunk) as floats.
-__device__ __forceinline__ void ld_chunk_f(const unsigned char* tile, int r, int j, int block_bytes,
-                                           float* f) {
-  const uint4 v = *reinterpret_cast<const uint4*>(tile + sw128_chunk(r, j, block_bytes));
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 x = __bfloat1622float2(h[i]);
-    f[2 * i] = x.x;
-    f[2 * i + 1] = x.y;
-  }
-}
-__device__ __forceinline__ void st_chunk_f(unsigned char* tile, int r, int j, int block_bytes,
-                                           const float* f) {
-  uint4 v;
-  v.x = pack_bf16(f[0], f[1]);
-  v.y = pack_bf16(f[2], f[3]);
-  v.z = pack_bf16(f[4], f[5]);
-  v.w = pack_bf16(f[6], f[7]);
-  *reinterpret_cast<uint4*>(tile + sw128_chunk(r, j, block_bytes)) = v;
-}
-
-__device__ __forceinline__ bool failed(const Work& w) { return *((volatile int*)w.status) != 0; }
 
 // ======================================================================================
 // WY representation.  One CTA (128 threads) per (chunk, value head).
@@ -629,18 +499,15 @@ Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
   L.ok &= map_rows(&L.m.UtT, L.t.UtT, urows, 64, 128);
   L.ok &= map_rows(&L.m.UT, L.t.UT, urows, 64, 128);
   L.ok &= map_rows(&L.m.h, L.t.h, urows, 128, 128);
+  if (pass == 1) {
+    const uint64_t trows = (uint64_t)p.NCmax * p.HV * 64;
+    L.ok &= map_rows(&L.m.dUlT, L.t.dUlT, urows, 64, 128);
+    L.ok &= map_rows(&L.m.dUT, L.t.dUT, urows, 64, 128);
+    L.ok &= map_rows(&L.m.dh, L.t.dh, urows, 128, 128);
+    L.ok &= map_rows(&L.m.dW, L.t.dW, trows, 128, 64);
+    L.ok &= map_rows(&L.m.Tm, L.t.Tm, trows, 64, 64);
+  }
   return L;
-}
-
-template <typename K, typename... Args_>
-cudaError_t go(const char* name, K kern, dim3 grid, int threads, size_t smem, cudaStream_t s,
-               Args_... args) {
-  if (grid.x == 0 || grid.y == 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  ProfScope ps(name, s);
-  kern<<<grid, threads, smem, s>>>(args...);
-  return cudaGetLastError();
 }
 
 cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const Launch& L,
@@ -649,15 +516,15 @@ cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const L
   cudaError_t e;
   const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV);
   const size_t wy_smem = 1024 + 6 * TILE64 + 2 * 64 * 65 * 4 + 2 * 64 * 4;
-  if ((e = go("tc_wy", k_tc_wy, gu, 128, wy_smem, s, p, w, L.t, L.m.k, L.m.v, bwd_prep ? 1 : 0)))
+  if ((e = tgo("tc_wy", k_tc_wy, gu, 128, wy_smem, s, p, w, L.t, L.m.k, L.m.v, bwd_prep ? 1 : 0)))
     return e;
   Args a2 = a;
-  if ((e = go("tc_scan_fwd", k_tc_scan_fwd, gs, 256, (size_t)1024 + ScanSmem::TOTAL, s, p, a2, w,
+  if ((e = tgo("tc_scan_fwd", k_tc_scan_fwd, gs, 256, (size_t)1024 + ScanSmem::TOTAL, s, p, a2, w,
               L.t, L.m.k, L.m.WT, L.m.UtT, L.m.UT, L.m.h, bwd_prep ? 0 : 1)))
     return e;
   if (!bwd_prep) {
     const size_t out_smem = 1024 + 5 * TILE64 + 3 * TILE128 + 256;
-    if ((e = go("tc_out", k_tc_out, gu, 256, out_smem, s, p, a, w, L.t, L.m.q, L.m.k, L.m.UT, L.m.h)))
+    if ((e = tgo("tc_out", k_tc_out, gu, 256, out_smem, s, p, a, w, L.t, L.m.q, L.m.k, L.m.UT, L.m.h)))
       return e;
   }
   return cudaSuccess;
@@ -671,7 +538,10 @@ bool tc_supported(const gdn_dims& d) {
          encoder() != nullptr;
 }
 
-bool tc_bwd_supported(const gdn_dims&) { return false; }
+bool tc_bwd_supported(const gdn_dims& d) {
+  static const bool disabled = getenv("GDN_DISABLE_TC_BWD") != nullptr;
+  return !disabled && tc_supported(d);
+}
 
 size_t tc_workspace_bytes(const gdn_dims& d, size_t NC, int pass) {
   return tc_bytes(NC, (size_t)d.HV, pass);
@@ -682,8 +552,12 @@ cudaError_t tc_forward(const Problem& p, const Args& a, const Work& w, void* tc_
   return forward_impl(p, a, w, L, false, s);
 }
 
-cudaError_t tc_backward(const Problem&, const Args&, const Work&, void*, cudaStream_t) {
-  return cudaErrorNotSupported;
+cudaError_t tc_backward(const Problem& p, const Args& a, const Work& w, void* tc_ws, cudaStream_t s) {
+  Launch L = setup(p, a, tc_ws, 1);
+  cudaError_t e = forward_impl(p, a, w, L, true, s);
+  if (e != cudaSuccess) return e;
+  if ((e = tc_backward_kernels(p, a, w, L.t, L.m, s)) != cudaSuccess) return e;
+  return launch_bwd_tokens(p, a, w, true, s);
 }
 
 }  // namespace gdn

@@ -1,0 +1,871 @@
+// tcgen05 backward kernels (bf16, K = V = 128).  Per chunk (64 tokens) and value head, with
+// S the state entering the chunk, dS' = dL/dS leaving it, P = (Q K^T) * Gam (lower incl.
+// diagonal), D_j = e^{G_C - G_j}:
+//   dv_local  dU_loc = scale P^T dO
+//   scan      dU = dU_loc + diag(D) K dS'^T;  dS = e^{G_C} dS' + scale (diag(e^G) dO)^T Q - dU^T W
+//   dqkwg     dP = scale dO U^T (masked);  dQ = scale diag(e^G) dO S + (dP*Gam) K;
+//             dK = (dP*Gam)^T Q + diag(D) U dS';  dW = -dU S;  dG terms
+//   wy_bwd    dT = dU Y^T + dW X^T;  dX = T^T dW;  dY = T^T dU;  dA = -(T^T dT T^T) strict lower;
+//             dv = beta dY;  dbeta;  dk += diag(beta e^G) dX + dAs K + dAs^T K;  dG terms
+// (X = diag(beta e^G) K, Y = diag(beta) V, dAs = dA * Gam * beta_i).  Column sums go through
+// shared memory in a fixed order, so results are bitwise reproducible.
+#include "gdn_tc_common.cuh"
+
+namespace gdn {
+namespace tcx {
+
+namespace {
+
+__device__ __forceinline__ float warp_sum(float x) {
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+// ======================================================================================
+// dv_local: dU_loc^T = scale dO^T P  (M=128 v, N=64 j, K=64 i), after QK^T (M=64).
+// ======================================================================================
+__global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
+                                                    const __grid_constant__ CUtensorMap mq,
+                                                    const __grid_constant__ CUtensorMap mk,
+                                                    const __grid_constant__ CUtensorMap mdO) {
+  if (failed(w)) return;
+  const int gc = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
+  const int4 e = w.chunk_tab[gc];
+  if (e.x < 0) return;
+  const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  extern __shared__ unsigned char smraw[];
+  unsigned char* sm = align1k(smraw);
+  unsigned char* sQ = sm;
+  unsigned char* sK = sQ + 2 * TILE64;
+  unsigned char* sO = sK + 2 * TILE64;
+  unsigned char* sP = sO + 2 * TILE64;
+  float* sG = reinterpret_cast<float*>(sP + TILE64);
+  __shared__ uint64_t bar[2];
+  __shared__ uint32_t tslot;
+  int* err = w.status;
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tslot, 128);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_expect_tx(&bar[0], 6 * TILE64);
+    tma_load_3d(sQ, &mq, 0, hk, tok0, &bar[0]);
+    tma_load_3d(sQ + TILE64, &mq, 64, hk, tok0, &bar[0]);
+    tma_load_3d(sK, &mk, 0, hk, tok0, &bar[0]);
+    tma_load_3d(sK + TILE64, &mk, 64, hk, tok0, &bar[0]);
+    tma_load_3d(sO, &mdO, 0, hv, tok0, &bar[0]);
+    tma_load_3d(sO + TILE64, &mdO, 64, hv, tok0, &bar[0]);
+  }
+  if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tslot;
+  bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
+  if (ok && tid == 0) {
+    const uint32_t q = smem_u32(sQ), k = smem_u32(sK);
+    for (int s = 0; s < 8; ++s)
+      mma_bf16(taddr(tb, 0, 0), desc_kmajor(q, s, TILE64), desc_kmajor(k, s, TILE64),
+               idesc_bf16(64, 64, false, false), s > 0);
+    mma_commit(&bar[1]);
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
+  tc_fence_after();
+  if (ok) {
+    const int i = 16 * warp + lane;
+    for (int c = 0; c < 64; c += 16) {
+      float d[16];
+      tmem_ld16(taddr(tb, 32 * warp, c), d);
+      tmem_wait_ld();
+      if (lane < 16) {
+        const float gi = sG[i];
+        float f[16];
+        for (int q = 0; q < 16; ++q) {
+          const int j = c + q;
+          f[q] = (j <= i && i < L) ? d[q] * expf(gi - sG[j]) : 0.f;
+        }
+        st_chunk_f(sP, i, c / 8, TILE64, f);
+        st_chunk_f(sP, i, c / 8 + 1, TILE64, f + 8);
+      }
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (ok && tid == 0) {
+    const uint32_t o = smem_u32(sO), pp = smem_u32(sP);
+    for (int s = 0; s < 4; ++s)
+      mma_bf16(taddr(tb, 0, 64), desc_mnmajor(o, s, TILE64), desc_mnmajor(pp, s, TILE64),
+               idesc_bf16(128, 64, true, true), s > 0);
+    mma_commit(&bar[1]);
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
+  tc_fence_after();
+  if (ok) {
+    const int v = 32 * warp + lane;
+    bf16* row = t.dUlT + (((size_t)gc * p.HV + hv) * D + v) * 64;
+    for (int c = 0; c < 64; c += 16) {
+      float d[16];
+      tmem_ld16(taddr(tb, 32 * warp, 64 + c), d);
+      tmem_wait_ld();
+      uint4 a0, a1;
+      for (int q = 0; q < 16; ++q) d[q] *= p.scale;
+      a0.x = pack_bf16(d[0], d[1]); a0.y = pack_bf16(d[2], d[3]);
+      a0.z = pack_bf16(d[4], d[5]); a0.w = pack_bf16(d[6], d[7]);
+      a1.x = pack_bf16(d[8], d[9]); a1.y = pack_bf16(d[10], d[11]);
+      a1.z = pack_bf16(d[12], d[13]); a1.w = pack_bf16(d[14], d[15]);
+      *reinterpret_cast<uint4*>(row + c) = a0;
+      *reinterpret_cast<uint4*>(row + c + 8) = a1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 128);
+}
+
+// ======================================================================================
+// Reverse state scan.  One CTA (256 threads) per (sequence, value head); thread
+// (v = 32*(warp%4)+lane, half = warp/4) keeps dS[v][64*half..+63] in fp32 registers.
+// ======================================================================================
+struct BwdScanSmem {
+  static constexpr int S = 0;                          // dS bf16 [128][128]
+  static constexpr int BUF = 2 * TILE128;
+  static constexpr int OFF_K = 0, OFF_Q = 2 * TILE64, OFF_O = 4 * TILE64, OFF_W = 6 * TILE64,
+                       OFF_UL = 6 * TILE64 + TILE128;
+  static constexpr int BUF_BYTES = 6 * TILE64 + 2 * TILE128;
+  static constexpr int AT = BUF + 2 * BUF_BYTES;       // -dU^T [128][64]
+  static constexpr int UO = AT + TILE128;              // +dU^T staging
+  static constexpr int G = UO + TILE128;               // 2 x 64 floats
+  static constexpr int DEC = G + 512;                  // e^{G_C - G_j}
+  static constexpr int EG = DEC + 256;                 // scale e^{G_i}
+  static constexpr int TOTAL = EG + 256;
+};
+
+__global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, TcWork t,
+                                                     const __grid_constant__ CUtensorMap mq,
+                                                     const __grid_constant__ CUtensorMap mk,
+                                                     const __grid_constant__ CUtensorMap mdO,
+                                                     const __grid_constant__ CUtensorMap mWT,
+                                                     const __grid_constant__ CUtensorMap mdUlT,
+                                                     const __grid_constant__ CUtensorMap mdUT,
+                                                     const __grid_constant__ CUtensorMap mdh) {
+  if (failed(w)) return;
+  const int n = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
+  const int4 sq = w.seq_tab[n];
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int v = 32 * (warp & 3) + lane, half = warp >> 2;
+  extern __shared__ unsigned char smraw[];
+  unsigned char* sm = align1k(smraw);
+  unsigned char* sS = sm + BwdScanSmem::S;
+  unsigned char* sAT = sm + BwdScanSmem::AT;
+  unsigned char* sUO = sm + BwdScanSmem::UO;
+  float* sGb = reinterpret_cast<float*>(sm + BwdScanSmem::G);
+  float* sDec = reinterpret_cast<float*>(sm + BwdScanSmem::DEC);
+  float* sEG = reinterpret_cast<float*>(sm + BwdScanSmem::EG);
+  __shared__ uint64_t barT[2], barM;
+  __shared__ uint32_t tslot;
+  int* err = w.status;
+  if (tid == 0) {
+    mbar_init(&barT[0], 1);
+    mbar_init(&barT[1], 1);
+    mbar_init(&barM, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tslot, 256);
+    tmem_relinquish();
+  }
+  float S[64];
+  const size_t st = ((size_t)n * p.HV + hv) * D * D;
+  for (int i = 0; i < 64; ++i) S[i] = a.dht ? a.dht[st + (size_t)(half * 64 + i) * D + v] : 0.f;
+  for (int j = 0; j < 8; ++j) st_chunk_f(sS, v, half * 8 + j, TILE128, &S[8 * j]);
+  auto issue = [&](int c, int buf) {
+    const int gc = sq.x + c;
+    const int4 e = w.chunk_tab[gc];
+    unsigned char* b = sm + BwdScanSmem::BUF + buf * BwdScanSmem::BUF_BYTES;
+    const int row = (gc * p.HV + hv) * D;
+    mbar_expect_tx(&barT[buf], BwdScanSmem::BUF_BYTES);
+    tma_load_3d(b + BwdScanSmem::OFF_K, &mk, 0, hk, e.w, &barT[buf]);
+    tma_load_3d(b + BwdScanSmem::OFF_K + TILE64, &mk, 64, hk, e.w, &barT[buf]);
+    tma_load_3d(b + BwdScanSmem::OFF_Q, &mq, 0, hk, e.w, &barT[buf]);
+    tma_load_3d(b + BwdScanSmem::OFF_Q + TILE64, &mq, 64, hk, e.w, &barT[buf]);
+    tma_load_3d(b + BwdScanSmem::OFF_O, &mdO, 0, hv, e.w, &barT[buf]);
+    tma_load_3d(b + BwdScanSmem::OFF_O + TILE64, &mdO, 64, hv, e.w, &barT[buf]);
+    tma_load_3d(b + BwdScanSmem::OFF_W, &mWT, 0, row, 0, &barT[buf]);
+    tma_load_3d(b + BwdScanSmem::OFF_UL, &mdUlT, 0, row, 0, &barT[buf]);
+  };
+  if (tid == 0 && sq.y > 0) issue(sq.y - 1, 0);
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tslot;
+  const uint32_t tE = taddr(tb, 0, 0), tF = taddr(tb, 0, 64);
+  uint32_t phT[2] = {0, 0}, phM = 0;
+  bool ok = true;
+  for (int idx = 0; idx < sq.y && ok; ++idx) {
+    const int c = sq.y - 1 - idx, gc = sq.x + c, buf = idx & 1;
+    unsigned char* b = sm + BwdScanSmem::BUF + buf * BwdScanSmem::BUF_BYTES;
+    const int L = w.chunk_tab[gc].z;
+    const uint32_t unit_row = (uint32_t)(gc * p.HV + hv) * D;
+    float* sG = sGb + buf * 64;
+    if (tid == 0 && idx + 1 < sq.y) issue(c - 1, buf ^ 1);
+    if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
+    ok = __syncthreads_and(mbar_wait(&barT[buf], phT[buf], err));
+    phT[buf] ^= 1;
+    if (!ok) break;
+    if (tid < 64) {
+      sDec[tid] = expf(sG[63] - sG[tid]);
+      sEG[tid] = tid < L ? p.scale * expf(sG[tid]) : 0.f;
+    }
+    __syncthreads();
+    // dO rows scaled by scale e^{G_i} (zero past the chunk end); K rows past the end zeroed
+    unsigned char* tO = b + BwdScanSmem::OFF_O;
+    for (int i = tid; i < 64 * 16; i += 256) {
+      const int r = i / 16, j = i % 16;
+      float f[8];
+      ld_chunk_f(tO, r, j, TILE64, f);
+      for (int q = 0; q < 8; ++q) f[q] *= sEG[r];
+      st_chunk_f(tO, r, j, TILE64, f);
+    }
+    if (L < 64) zero_tail_rows(b + BwdScanSmem::OFF_K, L, tid, 256);
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+      tma_store_3d(&mdh, sS, 0, unit_row, 0);
+      tma_store_3d(&mdh, sS + TILE128, 64, unit_row, 0);
+      tma_store_commit();
+      const uint32_t o = smem_u32(tO), q = smem_u32(b + BwdScanSmem::OFF_Q);
+      const uint32_t s_ = smem_u32(sS), k = smem_u32(b + BwdScanSmem::OFF_K);
+      for (int s = 0; s < 4; ++s)
+        mma_bf16(tF, desc_mnmajor(o, s, TILE64), desc_mnmajor(q, s, TILE64),
+                 idesc_bf16(128, 128, true, true), s > 0);
+      for (int s = 0; s < 8; ++s)
+        mma_bf16(tE, desc_kmajor(s_, s, TILE128), desc_kmajor(k, s, TILE64),
+                 idesc_bf16(128, 64, false, false), s > 0);
+      mma_commit(&barM);
+    }
+    ok = __syncthreads_and(mbar_wait(&barM, phM, err));
+    phM ^= 1;
+    tc_fence_after();
+    if (!ok) break;
+    {
+      float d[32];
+      tmem_ld16(taddr(tb, 32 * (warp & 3), 32 * half), d);
+      tmem_ld16(taddr(tb, 32 * (warp & 3), 32 * half + 16), d + 16);
+      tmem_wait_ld();
+      if (tid == 0) tma_store_wait_read0();
+      __syncthreads();
+      const unsigned char* ul = b + BwdScanSmem::OFF_UL;
+      for (int j = 0; j < 4; ++j) {
+        float u[8], nu[8];
+        ld_chunk_f(ul, v, half * 4 + j, TILE128, u);
+        for (int q = 0; q < 8; ++q) {
+          u[q] += sDec[32 * half + 8 * j + q] * d[8 * j + q];
+          nu[q] = -u[q];
+        }
+        st_chunk_f(sUO, v, half * 4 + j, TILE128, u);
+        st_chunk_f(sAT, v, half * 4 + j, TILE128, nu);
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      tma_store_3d(&mdUT, sUO, 0, unit_row, 0);
+      tma_store_commit();
+      const uint32_t at = smem_u32(sAT), wt = smem_u32(b + BwdScanSmem::OFF_W);
+      for (int s = 0; s < 4; ++s)
+        mma_bf16(tF, desc_kmajor(at, s, TILE128), desc_kmajor(wt, s, TILE128),
+                 idesc_bf16(128, 128, false, false), 1);
+      mma_commit(&barM);
+    }
+    ok = __syncthreads_and(mbar_wait(&barM, phM, err));
+    phM ^= 1;
+    tc_fence_after();
+    if (!ok) break;
+    {
+      const float eg = expf(sG[63]);
+      for (int cc = 0; cc < 64; cc += 16) {
+        float d[16];
+        tmem_ld16(taddr(tb, 32 * (warp & 3), 64 + 64 * half + cc), d);
+        tmem_wait_ld();
+        for (int i = 0; i < 16; ++i) S[cc + i] = eg * S[cc + i] + d[i];
+      }
+    }
+    if (tid == 0) tma_store_wait_read0();
+    __syncthreads();
+    for (int j = 0; j < 8; ++j) st_chunk_f(sS, v, half * 8 + j, TILE128, &S[8 * j]);
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  if (tid == 0) tma_store_wait0();
+  if (ok && a.dh0)
+    for (int i = 0; i < 64; ++i) a.dh0[st + (size_t)(half * 64 + i) * D + v] = S[i];
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tslot, 256);
+}
+
+// ======================================================================================
+// dqkwg.  One CTA (256 threads) per (chunk, value head).  TMEM columns:
+//   [0,64) Q K^T   [64,128) dO U^T   [128,256) dO S -> dQ   [256,384) U dS' -> dK   [384,512) dU S
+// M=64 accumulators: row i in lanes 0..15 of sub-partition i/16; the two warps sharing a
+// sub-partition split the columns.
+// ======================================================================================
+struct DqkSmem {
+  static constexpr int Q = 0, K = 2 * TILE64, O = 4 * TILE64, UT = 6 * TILE64,
+                       DUT = 6 * TILE64 + TILE128, H = 6 * TILE64 + 2 * TILE128,
+                       DH = 6 * TILE64 + 4 * TILE128, PG = 6 * TILE64 + 6 * TILE128,
+                       M = PG + TILE64;                      // fp32 [64][65] dP*P
+  static constexpr int G = M + 64 * 65 * 4;
+  static constexpr int ROW = G + 256;                        // [3][2][64] per-row partials
+  static constexpr int RED = ROW + 3 * 2 * 64 * 4;           // [8]
+  static constexpr int TOTAL = RED + 64;
+  static constexpr int LOAD_BYTES = 6 * TILE64 + 6 * TILE128;
+};
+
+__global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
+                                                  const __grid_constant__ CUtensorMap mq,
+                                                  const __grid_constant__ CUtensorMap mk,
+                                                  const __grid_constant__ CUtensorMap mdO,
+                                                  const __grid_constant__ CUtensorMap mUT,
+                                                  const __grid_constant__ CUtensorMap mdUT,
+                                                  const __grid_constant__ CUtensorMap mh,
+                                                  const __grid_constant__ CUtensorMap mdh) {
+  if (failed(w)) return;
+  const int gc = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
+  const int4 e = w.chunk_tab[gc];
+  if (e.x < 0) return;
+  const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int i = 16 * (warp & 3) + lane, half = warp >> 2, sub = 32 * (warp & 3);
+  extern __shared__ unsigned char smraw[];
+  unsigned char* sm = align1k(smraw);
+  unsigned char* sQ = sm + DqkSmem::Q;
+  unsigned char* sK = sm + DqkSmem::K;
+  unsigned char* sO = sm + DqkSmem::O;
+  unsigned char* sUT = sm + DqkSmem::UT;
+  unsigned char* sdUT = sm + DqkSmem::DUT;
+  unsigned char* sH = sm + DqkSmem::H;
+  unsigned char* sdH = sm + DqkSmem::DH;
+  unsigned char* sPG = sm + DqkSmem::PG;
+  float* sM = reinterpret_cast<float*>(sm + DqkSmem::M);
+  float* sG = reinterpret_cast<float*>(sm + DqkSmem::G);
+  float* sRow = reinterpret_cast<float*>(sm + DqkSmem::ROW);  // [kind][half][64]
+  float* sRed = reinterpret_cast<float*>(sm + DqkSmem::RED);
+  __shared__ uint64_t bar[2];
+  __shared__ uint32_t tslot;
+  int* err = w.status;
+  const size_t unit = (size_t)gc * p.HV + hv;
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tslot, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    const int row = (int)unit * D;
+    mbar_expect_tx(&bar[0], DqkSmem::LOAD_BYTES);
+    tma_load_3d(sQ, &mq, 0, hk, tok0, &bar[0]);
+    tma_load_3d(sQ + TILE64, &mq, 64, hk, tok0, &bar[0]);
+    tma_load_3d(sK, &mk, 0, hk, tok0, &bar[0]);
+    tma_load_3d(sK + TILE64, &mk, 64, hk, tok0, &bar[0]);
+    tma_load_3d(sO, &mdO, 0, hv, tok0, &bar[0]);
+    tma_load_3d(sO + TILE64, &mdO, 64, hv, tok0, &bar[0]);
+    tma_load_3d(sUT, &mUT, 0, row, 0, &bar[0]);
+    tma_load_3d(sdUT, &mdUT, 0, row, 0, &bar[0]);
+    tma_load_3d(sH, &mh, 0, row, 0, &bar[0]);
+    tma_load_3d(sH + TILE128, &mh, 64, row, 0, &bar[0]);
+    tma_load_3d(sdH, &mdh, 0, row, 0, &bar[0]);
+    tma_load_3d(sdH + TILE128, &mdh, 64, row, 0, &bar[0]);
+  }
+  if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tslot;
+  bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
+  if (L < 64) {
+    zero_tail_rows(sQ, L, tid, 256);
+    zero_tail_rows(sK, L, tid, 256);
+    zero_tail_rows(sO, L, tid, 256);
+  }
+  fence_proxy_async();
+  __syncthreads();
+  if (ok && tid == 0) {
+    const uint32_t q = smem_u32(sQ), k = smem_u32(sK), o = smem_u32(sO), ut = smem_u32(sUT),
+                   dut = smem_u32(sdUT), h = smem_u32(sH), dh = smem_u32(sdH);
+    for (int s = 0; s < 8; ++s) {
+      const uint32_t acc = s > 0;
+      mma_bf16(taddr(tb, 0, 0), desc_kmajor(q, s, TILE64), desc_kmajor(k, s, TILE64),
+               idesc_bf16(64, 64, false, false), acc);
+      mma_bf16(taddr(tb, 0, 64), desc_kmajor(o, s, TILE64), desc_mnmajor(ut, s, TILE128),
+               idesc_bf16(64, 64, false, true), acc);
+      mma_bf16(taddr(tb, 0, 128), desc_kmajor(o, s, TILE64), desc_mnmajor(h, s, TILE128),
+               idesc_bf16(64, 128, false, true), acc);
+      mma_bf16(taddr(tb, 0, 256), desc_mnmajor(ut, s, TILE128), desc_mnmajor(dh, s, TILE128),
+               idesc_bf16(64, 128, true, true), acc);
+      mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dut, s, TILE128), desc_mnmajor(h, s, TILE128),
+               idesc_bf16(64, 128, true, true), acc);
+    }
+    mma_commit(&bar[1]);
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
+  tc_fence_after();
+  const float Gi = sG[i & 63], GC = sG[63];
+  if (ok) {
+    // P, dP for columns [32*half, 32*half+32)
+    float qk[32], dp[32];
+    tmem_ld16(taddr(tb, sub, 32 * half), qk);
+    tmem_ld16(taddr(tb, sub, 32 * half + 16), qk + 16);
+    tmem_ld16(taddr(tb, sub, 64 + 32 * half), dp);
+    tmem_ld16(taddr(tb, sub, 64 + 32 * half + 16), dp + 16);
+    tmem_wait_ld();
+    if (lane < 16) {
+      float rs = 0.f, pg[8];
+      for (int jj = 0; jj < 32; ++jj) {
+        const int j = 32 * half + jj;
+        float dpp = 0.f, g = 0.f;
+        if (j <= i) {
+          const float gam = expf(Gi - sG[j]);
+          const float dpv = p.scale * dp[jj];
+          dpp = dpv * qk[jj] * gam;
+          g = dpv * gam;
+        }
+        sM[i * 65 + j] = dpp;
+        rs += dpp;
+        pg[jj & 7] = g;
+        if ((jj & 7) == 7) st_chunk_f(sPG, i, (32 * half + jj) / 8, TILE64, pg);
+      }
+      sRow[(0 * 2 + half) * 64 + i] = rs;
+    }
+    // dQ part 1: scale e^{G_i} dO S  -> back into TMEM; dG2 = sum_k (.) Q[i,k]
+    float x2 = 0.f;
+    const float egi = p.scale * expf(Gi);
+    for (int cc = 0; cc < 64; cc += 16) {
+      float x[16], qv[16];
+      tmem_ld16(taddr(tb, sub, 128 + 64 * half + cc), x);
+      tmem_wait_ld();
+      ld_chunk_f(sQ, i & 63, (64 * half + cc) / 8, TILE64, qv);
+      ld_chunk_f(sQ, i & 63, (64 * half + cc) / 8 + 1, TILE64, qv + 8);
+      for (int q = 0; q < 16; ++q) {
+        x[q] *= egi;
+        x2 += x[q] * qv[q];
+      }
+      tmem_st16(taddr(tb, sub, 128 + 64 * half + cc), x);
+    }
+    // dK part 1: D_i U dS' -> back into TMEM; r_i = sum_k (.) K[i,k]
+    float r = 0.f;
+    const float Di = expf(GC - Gi);
+    for (int cc = 0; cc < 64; cc += 16) {
+      float y[16], kv[16];
+      tmem_ld16(taddr(tb, sub, 256 + 64 * half + cc), y);
+      tmem_wait_ld();
+      ld_chunk_f(sK, i & 63, (64 * half + cc) / 8, TILE64, kv);
+      ld_chunk_f(sK, i & 63, (64 * half + cc) / 8 + 1, TILE64, kv + 8);
+      for (int q = 0; q < 16; ++q) {
+        y[q] *= Di;
+        r += y[q] * kv[q];
+      }
+      tmem_st16(taddr(tb, sub, 256 + 64 * half + cc), y);
+    }
+    // dW = -dU S
+    bf16* dwrow = t.dW + (unit * 64 + (i & 63)) * D + 64 * half;
+    for (int cc = 0; cc < 64; cc += 16) {
+      float z[16];
+      tmem_ld16(taddr(tb, sub, 384 + 64 * half + cc), z);
+      tmem_wait_ld();
+      if (lane < 16) {
+        uint4 a0, a1;
+        a0.x = pack_bf16(-z[0], -z[1]); a0.y = pack_bf16(-z[2], -z[3]);
+        a0.z = pack_bf16(-z[4], -z[5]); a0.w = pack_bf16(-z[6], -z[7]);
+        a1.x = pack_bf16(-z[8], -z[9]); a1.y = pack_bf16(-z[10], -z[11]);
+        a1.z = pack_bf16(-z[12], -z[13]); a1.w = pack_bf16(-z[14], -z[15]);
+        *reinterpret_cast<uint4*>(dwrow + cc) = a0;
+        *reinterpret_cast<uint4*>(dwrow + cc + 8) = a1;
+      }
+    }
+    if (lane < 16) {
+      sRow[(1 * 2 + half) * 64 + i] = x2;
+      sRow[(2 * 2 + half) * 64 + i] = r;
+    }
+    tmem_wait_st();
+  }
+  // <dS', S> over the two bf16 state tiles
+  float dot = 0.f;
+  for (int c = tid; c < 128 * 16; c += 256) {
+    const int rr = c / 16, j = c % 16;
+    float a8[8], b8[8];
+    ld_chunk_f(sH, rr, j, TILE128, a8);
+    ld_chunk_f(sdH, rr, j, TILE128, b8);
+    for (int q = 0; q < 8; ++q) dot += a8[q] * b8[q];
+  }
+  dot = warp_sum(dot);
+  if (lane == 0) sRed[warp] = dot;
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (ok && tid == 0) {
+    const uint32_t pg = smem_u32(sPG), k = smem_u32(sK), q = smem_u32(sQ);
+    for (int s = 0; s < 4; ++s) {
+      mma_bf16(taddr(tb, 0, 128), desc_kmajor(pg, s, TILE64), desc_mnmajor(k, s, TILE64),
+               idesc_bf16(64, 128, false, true), 1);
+      mma_bf16(taddr(tb, 0, 256), desc_mnmajor(pg, s, TILE64), desc_mnmajor(q, s, TILE64),
+               idesc_bf16(64, 128, true, true), 1);
+    }
+    mma_commit(&bar[1]);
+  }
+  // dG for this chunk (rows j = tid < 64), deterministic column sums
+  if (tid < 64) {
+    const int j = tid;
+    float cs = 0.f;
+    for (int ii = 0; ii < 64; ++ii) cs += sM[ii * 65 + j];
+    float g = sRow[0 * 64 + j] + sRow[1 * 64 + j] - cs + sRow[2 * 64 + j] + sRow[3 * 64 + j] -
+              (sRow[4 * 64 + j] + sRow[5 * 64 + j]);
+    if (j == 63) {
+      float d8 = 0.f, rsum = 0.f;
+      for (int q = 0; q < 8; ++q) d8 += sRed[q];
+      for (int q = 0; q < 64; ++q) rsum += sRow[4 * 64 + q] + sRow[5 * 64 + q];
+      g += expf(GC) * d8 + rsum;
+    }
+    w.dG[((size_t)hv * p.NCmax + gc) * 64 + j] = g;
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
+  tc_fence_after();
+  if (ok) {
+    float* dq = w.dqp + (unit * 64 + (i & 63)) * D + 64 * half;
+    float* dk = w.dkp + (unit * 64 + (i & 63)) * D + 64 * half;
+    for (int cc = 0; cc < 64; cc += 16) {
+      float x[16], y[16];
+      tmem_ld16(taddr(tb, sub, 128 + 64 * half + cc), x);
+      tmem_ld16(taddr(tb, sub, 256 + 64 * half + cc), y);
+      tmem_wait_ld();
+      if (lane < 16)
+        for (int q = 0; q < 16; q += 4) {
+          *reinterpret_cast<float4*>(dq + cc + q) = make_float4(x[q], x[q + 1], x[q + 2], x[q + 3]);
+          *reinterpret_cast<float4*>(dk + cc + q) = make_float4(y[q], y[q + 1], y[q + 2], y[q + 3]);
+        }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 512);
+}
+
+// ======================================================================================
+// WY backward.  One CTA (256 threads) per (chunk, value head).  TMEM columns:
+//   [0,64) dU V^T, then T^T dT   [64,128) dW K^T, then Z T^T   [128,192) K K^T
+//   [256,384) T^T dW -> dk       [384,512) T^T dU
+// ======================================================================================
+struct WyBwdSmem {
+  static constexpr int K = 0, V = 2 * TILE64, T = 4 * TILE64, DW = 5 * TILE64, DUT = 7 * TILE64,
+                       DT = 7 * TILE64 + TILE128, Z = DT + TILE64, AS = Z + TILE64, F = AS + TILE64;
+  static constexpr int KKG = F, AA = KKG + 64 * 65 * 4;        // fp32 [64][65] each
+  static constexpr int G = AA + 64 * 65 * 4, B = G + 256, ROW = B + 256;  // ROW [4][2][64]
+  static constexpr int TOTAL = ROW + 4 * 2 * 64 * 4;
+  static constexpr int LOAD_BYTES = 7 * TILE64 + TILE128;
+};
+
+__global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, TcWork t,
+                                                   const __grid_constant__ CUtensorMap mk,
+                                                   const __grid_constant__ CUtensorMap mv,
+                                                   const __grid_constant__ CUtensorMap mTm,
+                                                   const __grid_constant__ CUtensorMap mdW,
+                                                   const __grid_constant__ CUtensorMap mdUT) {
+  if (failed(w)) return;
+  const int gc = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
+  const int4 e = w.chunk_tab[gc];
+  if (e.x < 0) return;
+  const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int i = 16 * (warp & 3) + lane, half = warp >> 2, sub = 32 * (warp & 3);
+  const int ii = i & 63;
+  extern __shared__ unsigned char smraw[];
+  unsigned char* sm = align1k(smraw);
+  unsigned char* sK = sm + WyBwdSmem::K;
+  unsigned char* sV = sm + WyBwdSmem::V;
+  unsigned char* sT = sm + WyBwdSmem::T;
+  unsigned char* sdW = sm + WyBwdSmem::DW;
+  unsigned char* sdUT = sm + WyBwdSmem::DUT;
+  unsigned char* sdT = sm + WyBwdSmem::DT;
+  unsigned char* sZ = sm + WyBwdSmem::Z;
+  unsigned char* sAs = sm + WyBwdSmem::AS;
+  float* sKKG = reinterpret_cast<float*>(sm + WyBwdSmem::KKG);
+  float* sAA = reinterpret_cast<float*>(sm + WyBwdSmem::AA);
+  float* sG = reinterpret_cast<float*>(sm + WyBwdSmem::G);
+  float* sb = reinterpret_cast<float*>(sm + WyBwdSmem::B);
+  float* sRow = reinterpret_cast<float*>(sm + WyBwdSmem::ROW);  // [kind][half][64]
+  __shared__ uint64_t bar[2];
+  __shared__ uint32_t tslot;
+  int* err = w.status;
+  const size_t unit = (size_t)gc * p.HV + hv;
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tslot, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_expect_tx(&bar[0], WyBwdSmem::LOAD_BYTES);
+    tma_load_3d(sK, &mk, 0, hk, tok0, &bar[0]);
+    tma_load_3d(sK + TILE64, &mk, 64, hk, tok0, &bar[0]);
+    tma_load_3d(sV, &mv, 0, hv, tok0, &bar[0]);
+    tma_load_3d(sV + TILE64, &mv, 64, hv, tok0, &bar[0]);
+    tma_load_3d(sT, &mTm, 0, (int)unit * 64, 0, &bar[0]);
+    tma_load_3d(sdW, &mdW, 0, (int)unit * 64, 0, &bar[0]);
+    tma_load_3d(sdW + TILE64, &mdW, 64, (int)unit * 64, 0, &bar[0]);
+    tma_load_3d(sdUT, &mdUT, 0, (int)unit * D, 0, &bar[0]);
+  }
+  if (tid < 64) {
+    const size_t o = ((size_t)hv * p.NCmax + gc) * 64 + tid;
+    sG[tid] = w.G[o];
+    sb[tid] = w.beta_p[o];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tslot;
+  bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
+  if (L < 64) {
+    zero_tail_rows(sK, L, tid, 256);
+    zero_tail_rows(sV, L, tid, 256);
+  }
+  fence_proxy_async();
+  __syncthreads();
+  const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aT = smem_u32(sT), aW = smem_u32(sdW),
+                 aU = smem_u32(sdUT);
+  if (ok && tid == 0) {
+    for (int s = 0; s < 8; ++s) {
+      const uint32_t acc = s > 0;
+      mma_bf16(taddr(tb, 0, 0), desc_mnmajor(aU, s, TILE128), desc_kmajor(aV, s, TILE64),
+               idesc_bf16(64, 64, true, false), acc);
+      mma_bf16(taddr(tb, 0, 64), desc_kmajor(aW, s, TILE64), desc_kmajor(aK, s, TILE64),
+               idesc_bf16(64, 64, false, false), acc);
+      mma_bf16(taddr(tb, 0, 128), desc_kmajor(aK, s, TILE64), desc_kmajor(aK, s, TILE64),
+               idesc_bf16(64, 64, false, false), acc);
+    }
+    for (int s = 0; s < 4; ++s) {
+      const uint32_t acc = s > 0;
+      mma_bf16(taddr(tb, 0, 256), desc_mnmajor(aT, s, TILE64), desc_mnmajor(aW, s, TILE64),
+               idesc_bf16(64, 128, true, true), acc);
+      mma_bf16(taddr(tb, 0, 384), desc_mnmajor(aT, s, TILE64), desc_kmajor(aU, s, TILE128),
+               idesc_bf16(64, 128, true, false), acc);
+    }
+    mma_commit(&bar[1]);
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
+  tc_fence_after();
+  const float Gi = sG[ii], bi = sb[ii], egi = expf(Gi);
+  if (ok) {
+    float r1[32], r2[32], kk[32];
+    tmem_ld16(taddr(tb, sub, 32 * half), r1);
+    tmem_ld16(taddr(tb, sub, 32 * half + 16), r1 + 16);
+    tmem_ld16(taddr(tb, sub, 64 + 32 * half), r2);
+    tmem_ld16(taddr(tb, sub, 64 + 32 * half + 16), r2 + 16);
+    tmem_ld16(taddr(tb, sub, 128 + 32 * half), kk);
+    tmem_ld16(taddr(tb, sub, 128 + 32 * half + 16), kk + 16);
+    tmem_wait_ld();
+    if (lane < 16) {
+      float f[8];
+      for (int jj = 0; jj < 32; ++jj) {
+        const int j = 32 * half + jj;
+        f[jj & 7] = sb[j] * (r1[jj] + expf(sG[j]) * r2[jj]);
+        if ((jj & 7) == 7) st_chunk_f(sdT, ii, j / 8, TILE64, f);
+        sKKG[ii * 65 + j] = j < ii ? expf(Gi - sG[j]) * kk[jj] : 0.f;
+      }
+    }
+    // dX: dbeta/dG parts, then beta_i e^{G_i} dX back into TMEM
+    float px = 0.f;
+    for (int cc = 0; cc < 64; cc += 16) {
+      float x[16], kv[16];
+      tmem_ld16(taddr(tb, sub, 256 + 64 * half + cc), x);
+      tmem_wait_ld();
+      ld_chunk_f(sK, ii, (64 * half + cc) / 8, TILE64, kv);
+      ld_chunk_f(sK, ii, (64 * half + cc) / 8 + 1, TILE64, kv + 8);
+      for (int q = 0; q < 16; ++q) {
+        px += x[q] * kv[q];
+        x[q] *= bi * egi;
+      }
+      tmem_st16(taddr(tb, sub, 256 + 64 * half + cc), x);
+    }
+    // dY: dv = beta dY, dbeta part
+    float py = 0.f;
+    bf16* dvrow = static_cast<bf16*>(a.dv) + ((size_t)(tok0 + ii) * p.HV + hv) * D + 64 * half;
+    for (int cc = 0; cc < 64; cc += 16) {
+      float y[16], vv[16];
+      tmem_ld16(taddr(tb, sub, 384 + 64 * half + cc), y);
+      tmem_wait_ld();
+      ld_chunk_f(sV, ii, (64 * half + cc) / 8, TILE64, vv);
+      ld_chunk_f(sV, ii, (64 * half + cc) / 8 + 1, TILE64, vv + 8);
+      for (int q = 0; q < 16; ++q) py += y[q] * vv[q];
+      if (lane < 16 && ii < L) {
+        uint4 a0, a1;
+        a0.x = pack_bf16(bi * y[0], bi * y[1]); a0.y = pack_bf16(bi * y[2], bi * y[3]);
+        a0.z = pack_bf16(bi * y[4], bi * y[5]); a0.w = pack_bf16(bi * y[6], bi * y[7]);
+        a1.x = pack_bf16(bi * y[8], bi * y[9]); a1.y = pack_bf16(bi * y[10], bi * y[11]);
+        a1.z = pack_bf16(bi * y[12], bi * y[13]); a1.w = pack_bf16(bi * y[14], bi * y[15]);
+        *reinterpret_cast<uint4*>(dvrow + cc) = a0;
+        *reinterpret_cast<uint4*>(dvrow + cc + 8) = a1;
+      }
+    }
+    if (lane < 16) {
+      sRow[(0 * 2 + half) * 64 + ii] = px;
+      sRow[(1 * 2 + half) * 64 + ii] = py;
+    }
+    tmem_wait_st();
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // Z = T^T dT
+  if (ok && tid == 0) {
+    const uint32_t dt = smem_u32(sdT);
+    for (int s = 0; s < 4; ++s)
+      mma_bf16(taddr(tb, 0, 0), desc_mnmajor(aT, s, TILE64), desc_mnmajor(dt, s, TILE64),
+               idesc_bf16(64, 64, true, true), s > 0);
+    mma_commit(&bar[1]);
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
+  tc_fence_after();
+  if (ok) {
+    float z[32];
+    tmem_ld16(taddr(tb, sub, 32 * half), z);
+    tmem_ld16(taddr(tb, sub, 32 * half + 16), z + 16);
+    tmem_wait_ld();
+    if (lane < 16)
+      for (int j = 0; j < 4; ++j) st_chunk_f(sZ, ii, 4 * half + j, TILE64, z + 8 * j);
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // dA' = Z T^T
+  if (ok && tid == 0) {
+    const uint32_t zz = smem_u32(sZ);
+    for (int s = 0; s < 4; ++s)
+      mma_bf16(taddr(tb, 0, 64), desc_kmajor(zz, s, TILE64), desc_kmajor(aT, s, TILE64),
+               idesc_bf16(64, 64, false, false), s > 0);
+    mma_commit(&bar[1]);
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
+  tc_fence_after();
+  if (ok) {
+    float da[32];
+    tmem_ld16(taddr(tb, sub, 64 + 32 * half), da);
+    tmem_ld16(taddr(tb, sub, 64 + 32 * half + 16), da + 16);
+    tmem_wait_ld();
+    if (lane < 16) {
+      float pa = 0.f, paa = 0.f, f[8];
+      for (int jj = 0; jj < 32; ++jj) {
+        const int j = 32 * half + jj;
+        float dAs = 0.f, aa = 0.f;
+        if (j < ii) {
+          const float dA = -da[jj];
+          const float kkg = sKKG[ii * 65 + j];
+          pa += dA * kkg;
+          aa = dA * bi * kkg;
+          dAs = dA * expf(Gi - sG[j]) * bi;
+        }
+        sAA[ii * 65 + j] = aa;
+        paa += aa;
+        f[jj & 7] = dAs;
+        if ((jj & 7) == 7) st_chunk_f(sAs, ii, j / 8, TILE64, f);
+      }
+      sRow[(2 * 2 + half) * 64 + ii] = pa;
+      sRow[(3 * 2 + half) * 64 + ii] = paa;
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // dk += dAs K + dAs^T K onto beta e^G dX
+  if (ok && tid == 0) {
+    const uint32_t as = smem_u32(sAs);
+    for (int s = 0; s < 4; ++s) {
+      mma_bf16(taddr(tb, 0, 256), desc_kmajor(as, s, TILE64), desc_mnmajor(aK, s, TILE64),
+               idesc_bf16(64, 128, false, true), 1);
+      mma_bf16(taddr(tb, 0, 256), desc_mnmajor(as, s, TILE64), desc_mnmajor(aK, s, TILE64),
+               idesc_bf16(64, 128, true, true), 1);
+    }
+    mma_commit(&bar[1]);
+  }
+  if (tid < 64) {
+    const int j = tid;
+    float cs = 0.f;
+    for (int r = 0; r < 64; ++r) cs += sAA[r * 65 + j];
+    const float eg = expf(sG[j]), bj = sb[j];
+    const float px = sRow[0 * 64 + j] + sRow[1 * 64 + j];
+    const float py = sRow[2 * 64 + j] + sRow[3 * 64 + j];
+    const float pa = sRow[4 * 64 + j] + sRow[5 * 64 + j];
+    const float paa = sRow[6 * 64 + j] + sRow[7 * 64 + j];
+    if (j < L) a.dbeta[(size_t)(tok0 + j) * p.HV + hv] = eg * px + py + pa;
+    w.dG[((size_t)hv * p.NCmax + gc) * 64 + j] += bj * eg * px + paa - cs;
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
+  tc_fence_after();
+  if (ok) {
+    float* dk = w.dkp + (unit * 64 + ii) * D + 64 * half;
+    for (int cc = 0; cc < 64; cc += 16) {
+      float x[16];
+      tmem_ld16(taddr(tb, sub, 256 + 64 * half + cc), x);
+      tmem_wait_ld();
+      if (lane < 16)
+        for (int q = 0; q < 16; q += 4) {
+          float4 o = *reinterpret_cast<float4*>(dk + cc + q);
+          o.x += x[q];
+          o.y += x[q + 1];
+          o.z += x[q + 2];
+          o.w += x[q + 3];
+          *reinterpret_cast<float4*>(dk + cc + q) = o;
+        }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 512);
+}
+
+}  // namespace
+
+cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, const TcWork& t,
+                                const TcMaps& m, cudaStream_t s) {
+  cudaError_t e;
+  const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV);
+  if ((e = tgo("tc_dvlocal", k_tc_dvlocal, gu, 128, 1024 + 7 * TILE64 + 256, s, p, w, t, m.q, m.k,
+               m.dO)))
+    return e;
+  if ((e = tgo("tc_scan_bwd", k_tc_scan_bwd, gs, 256, 1024 + BwdScanSmem::TOTAL, s, p, a, w, t, m.q,
+               m.k, m.dO, m.WT, m.dUlT, m.dUT, m.dh)))
+    return e;
+  if ((e = tgo("tc_dqkwg", k_tc_dqkwg, gu, 256, 1024 + DqkSmem::TOTAL, s, p, w, t, m.q, m.k, m.dO,
+               m.UT, m.dUT, m.h, m.dh)))
+    return e;
+  if ((e = tgo("tc_wy_bwd", k_tc_wy_bwd, gu, 256, 1024 + WyBwdSmem::TOTAL, s, p, a, w, t, m.k, m.v,
+               m.Tm, m.dW, m.dUT)))
+    return e;
+  return cudaSuccess;
+}
+
+}  // namespace tcx
+}  // namespace gdn
