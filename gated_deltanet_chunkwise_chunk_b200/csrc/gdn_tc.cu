@@ -35,9 +35,11 @@ __global__ void __launch_bounds__(128) k_tc_wy(Problem p, Work w, TcWork t,
   unsigned char* sm = align1k(smraw);
   unsigned char* sK = sm;                    // [64][128] bf16, 2 blocks
   unsigned char* sV = sK + 2 * TILE64;       // [64][128]
-  unsigned char* sTX = sV + 2 * TILE64;      // [64][64]  T diag(beta e^G)
-  unsigned char* sTY = sTX + TILE64;         // [64][64]  T diag(beta)
-  float* sA = reinterpret_cast<float*>(sTY + TILE64);  // [64][65]
+  unsigned char* sTX = sV + 2 * TILE64;      // [64][64]  T diag(beta e^G), hi part
+  unsigned char* sTY = sTX + TILE64;         // [64][64]  T diag(beta), hi part
+  unsigned char* sTXl = sTY + TILE64;        // lo parts
+  unsigned char* sTYl = sTXl + TILE64;
+  float* sA = reinterpret_cast<float*>(sTYl + TILE64);  // [64][65]
   float* sT = sA + 64 * 65;                            // [64][65]
   float* sG = sT + 64 * 65;
   float* sb = sG + 64;
@@ -123,17 +125,26 @@ __global__ void __launch_bounds__(128) k_tc_wy(Problem p, Work w, TcWork t,
       fy[q] = tv * sb[j];
       fx[q] = fy[q] * expf(sG[j]);
     }
-    st_chunk_f(sTX, i, jc, TILE64, fx);
-    st_chunk_f(sTY, i, jc, TILE64, fy);
-    if (store_T) {
-      float ft[8];
-      for (int q = 0; q < 8; ++q) ft[q] = sT[i * 65 + jc * 8 + q];
+    st_chunk_split(sTX, sTXl, i, jc, TILE64, fx);
+    st_chunk_split(sTY, sTYl, i, jc, TILE64, fy);
+    if (store_T) {  // T as a compensated pair: rows [0,64) hi, [64,128) lo of the unit
+      float ft[8], fl[8];
+      for (int q = 0; q < 8; ++q) {
+        ft[q] = sT[i * 65 + jc * 8 + q];
+        fl[q] = ft[q] - __bfloat162float(__float2bfloat16_rn(ft[q]));
+      }
+      bf16* base = t.Tm + ((size_t)gc * p.HV + hv) * 128 * 64;
       uint4 pk;
       pk.x = pack_bf16(ft[0], ft[1]);
       pk.y = pack_bf16(ft[2], ft[3]);
       pk.z = pack_bf16(ft[4], ft[5]);
       pk.w = pack_bf16(ft[6], ft[7]);
-      *reinterpret_cast<uint4*>(t.Tm + (((size_t)gc * p.HV + hv) * 64 + i) * 64 + jc * 8) = pk;
+      *reinterpret_cast<uint4*>(base + i * 64 + jc * 8) = pk;
+      pk.x = pack_bf16(fl[0], fl[1]);
+      pk.y = pack_bf16(fl[2], fl[3]);
+      pk.z = pack_bf16(fl[4], fl[5]);
+      pk.w = pack_bf16(fl[6], fl[7]);
+      *reinterpret_cast<uint4*>(base + (64 + i) * 64 + jc * 8) = pk;
     }
   }
   fence_proxy_async();
@@ -142,12 +153,19 @@ __global__ void __launch_bounds__(128) k_tc_wy(Problem p, Work w, TcWork t,
   tc_fence_after();
   // W^T = K^T TX^T, U~^T = V^T TY^T: M=128 (A MN-major), N=64, K=64 (B K-major)
   if (ok && tid == 0) {
-    const uint32_t k = smem_u32(sK), vv = smem_u32(sV), tx = smem_u32(sTX), ty = smem_u32(sTY);
+    const uint32_t k = smem_u32(sK), vv = smem_u32(sV), tx = smem_u32(sTX), ty = smem_u32(sTY),
+                   txl = smem_u32(sTXl), tyl = smem_u32(sTYl);
     for (int s = 0; s < 4; ++s) {
       mma_bf16(taddr(tb, 0, 64), desc_mnmajor(k, s, TILE64), desc_kmajor(tx, s, TILE64),
                idesc_bf16(128, 64, true, false), s > 0);
       mma_bf16(taddr(tb, 0, 128), desc_mnmajor(vv, s, TILE64), desc_kmajor(ty, s, TILE64),
                idesc_bf16(128, 64, true, false), s > 0);
+    }
+    for (int s = 0; s < 4; ++s) {
+      mma_bf16(taddr(tb, 0, 64), desc_mnmajor(k, s, TILE64), desc_kmajor(txl, s, TILE64),
+               idesc_bf16(128, 64, true, false), 1);
+      mma_bf16(taddr(tb, 0, 128), desc_mnmajor(vv, s, TILE64), desc_kmajor(tyl, s, TILE64),
+               idesc_bf16(128, 64, true, false), 1);
     }
     mma_commit(&bar[1]);
   }
@@ -376,8 +394,9 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
   unsigned char* sK = sQ + 2 * TILE64;       // [64][128]
   unsigned char* sH = sK + 2 * TILE64;       // [128][128]
   unsigned char* sU = sH + 2 * TILE128;      // [128][64]  U^T
-  unsigned char* sP = sU + TILE128;          // [64][64]
-  float* sG = reinterpret_cast<float*>(sP + TILE64);
+  unsigned char* sP = sU + TILE128;          // [64][64] hi part
+  unsigned char* sPl = sP + TILE64;          // lo part
+  float* sG = reinterpret_cast<float*>(sPl + TILE64);
   __shared__ uint64_t bar[2];
   __shared__ uint32_t tslot;
   int* err = w.status;
@@ -436,7 +455,7 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
           const int jj = 32 * half + 8 * j + q;
           f[q] = jj <= i ? d[8 * j + q] * expf(gi - sG[jj]) : 0.f;
         }
-        st_chunk_f(sP, i, half * 4 + j, TILE64, f);
+        st_chunk_split(sP, sPl, i, half * 4 + j, TILE64, f);
       }
     }
   }
@@ -445,10 +464,13 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
   __syncthreads();
   tc_fence_after();
   if (ok && tid == 0) {
-    const uint32_t pp = smem_u32(sP), u = smem_u32(sU);
+    const uint32_t pp = smem_u32(sP), pl = smem_u32(sPl), u = smem_u32(sU);
     for (int s = 0; s < 4; ++s)
       mma_bf16(taddr(tb, 0, 128), desc_kmajor(pp, s, TILE64), desc_kmajor(u, s, TILE128),
                idesc_bf16(64, 128, false, false), s > 0);
+    for (int s = 0; s < 4; ++s)
+      mma_bf16(taddr(tb, 0, 128), desc_kmajor(pl, s, TILE64), desc_kmajor(u, s, TILE128),
+               idesc_bf16(64, 128, false, false), 1);
     mma_commit(&bar[1]);
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
@@ -505,7 +527,7 @@ Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
     L.ok &= map_rows(&L.m.dUT, L.t.dUT, urows, 64, 128);
     L.ok &= map_rows(&L.m.dh, L.t.dh, urows, 128, 128);
     L.ok &= map_rows(&L.m.dW, L.t.dW, trows, 128, 64);
-    L.ok &= map_rows(&L.m.Tm, L.t.Tm, trows, 64, 64);
+    L.ok &= map_rows(&L.m.Tm, L.t.Tm, 2 * trows, 64, 64);
   }
   return L;
 }
@@ -515,7 +537,7 @@ cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const L
   if (!L.ok) return cudaErrorInvalidValue;
   cudaError_t e;
   const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV);
-  const size_t wy_smem = 1024 + 6 * TILE64 + 2 * 64 * 65 * 4 + 2 * 64 * 4;
+  const size_t wy_smem = 1024 + 8 * TILE64 + 2 * 64 * 65 * 4 + 2 * 64 * 4;
   if ((e = tgo("tc_wy", k_tc_wy, gu, 128, wy_smem, s, p, w, L.t, L.m.k, L.m.v, bwd_prep ? 1 : 0)))
     return e;
   Args a2 = a;
@@ -523,7 +545,7 @@ cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const L
               L.t, L.m.k, L.m.WT, L.m.UtT, L.m.UT, L.m.h, bwd_prep ? 0 : 1)))
     return e;
   if (!bwd_prep) {
-    const size_t out_smem = 1024 + 5 * TILE64 + 3 * TILE128 + 256;
+    const size_t out_smem = 1024 + 6 * TILE64 + 3 * TILE128 + 256;
     if ((e = tgo("tc_out", k_tc_out, gu, 256, out_smem, s, p, a, w, L.t, L.m.q, L.m.k, L.m.UT, L.m.h)))
       return e;
   }

@@ -38,8 +38,9 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
   unsigned char* sQ = sm;
   unsigned char* sK = sQ + 2 * TILE64;
   unsigned char* sO = sK + 2 * TILE64;
-  unsigned char* sP = sO + 2 * TILE64;
-  float* sG = reinterpret_cast<float*>(sP + TILE64);
+  unsigned char* sP = sO + 2 * TILE64;      // P hi
+  unsigned char* sPl = sP + TILE64;         // P lo
+  float* sG = reinterpret_cast<float*>(sPl + TILE64);
   __shared__ uint64_t bar[2];
   __shared__ uint32_t tslot;
   int* err = w.status;
@@ -90,8 +91,8 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
           const int j = c + q;
           f[q] = (j <= i && i < L) ? d[q] * expf(gi - sG[j]) : 0.f;
         }
-        st_chunk_f(sP, i, c / 8, TILE64, f);
-        st_chunk_f(sP, i, c / 8 + 1, TILE64, f + 8);
+        st_chunk_split(sP, sPl, i, c / 8, TILE64, f);
+        st_chunk_split(sP, sPl, i, c / 8 + 1, TILE64, f + 8);
       }
     }
   }
@@ -100,10 +101,13 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
   __syncthreads();
   tc_fence_after();
   if (ok && tid == 0) {
-    const uint32_t o = smem_u32(sO), pp = smem_u32(sP);
+    const uint32_t o = smem_u32(sO), pp = smem_u32(sP), pl = smem_u32(sPl);
     for (int s = 0; s < 4; ++s)
       mma_bf16(taddr(tb, 0, 64), desc_mnmajor(o, s, TILE64), desc_mnmajor(pp, s, TILE64),
                idesc_bf16(128, 64, true, true), s > 0);
+    for (int s = 0; s < 4; ++s)
+      mma_bf16(taddr(tb, 0, 64), desc_mnmajor(o, s, TILE64), desc_mnmajor(pl, s, TILE64),
+               idesc_bf16(128, 64, true, true), 1);
     mma_commit(&bar[1]);
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
@@ -328,7 +332,7 @@ struct DqkSmem {
   static constexpr int Q = 0, K = 2 * TILE64, O = 4 * TILE64, UT = 6 * TILE64,
                        DUT = 6 * TILE64 + TILE128, H = 6 * TILE64 + 2 * TILE128,
                        DH = 6 * TILE64 + 4 * TILE128, PG = 6 * TILE64 + 6 * TILE128,
-                       M = PG + TILE64;                      // fp32 [64][65] dP*P
+                       PGL = PG + TILE64, M = PGL + TILE64;  // fp32 [64][65] dP*P
   static constexpr int G = M + 64 * 65 * 4;
   static constexpr int ROW = G + 256;                        // [3][2][64] per-row partials
   static constexpr int RED = ROW + 3 * 2 * 64 * 4;           // [8]
@@ -360,6 +364,7 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
   unsigned char* sH = sm + DqkSmem::H;
   unsigned char* sdH = sm + DqkSmem::DH;
   unsigned char* sPG = sm + DqkSmem::PG;
+  unsigned char* sPGl = sm + DqkSmem::PGL;
   float* sM = reinterpret_cast<float*>(sm + DqkSmem::M);
   float* sG = reinterpret_cast<float*>(sm + DqkSmem::G);
   float* sRow = reinterpret_cast<float*>(sm + DqkSmem::ROW);  // [kind][half][64]
@@ -450,7 +455,7 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
         sM[i * 65 + j] = dpp;
         rs += dpp;
         pg[jj & 7] = g;
-        if ((jj & 7) == 7) st_chunk_f(sPG, i, (32 * half + jj) / 8, TILE64, pg);
+        if ((jj & 7) == 7) st_chunk_split(sPG, sPGl, i, (32 * half + jj) / 8, TILE64, pg);
       }
       sRow[(0 * 2 + half) * 64 + i] = rs;
     }
@@ -522,12 +527,15 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
   __syncthreads();
   tc_fence_after();
   if (ok && tid == 0) {
-    const uint32_t pg = smem_u32(sPG), k = smem_u32(sK), q = smem_u32(sQ);
-    for (int s = 0; s < 4; ++s) {
-      mma_bf16(taddr(tb, 0, 128), desc_kmajor(pg, s, TILE64), desc_mnmajor(k, s, TILE64),
-               idesc_bf16(64, 128, false, true), 1);
-      mma_bf16(taddr(tb, 0, 256), desc_mnmajor(pg, s, TILE64), desc_mnmajor(q, s, TILE64),
-               idesc_bf16(64, 128, true, true), 1);
+    const uint32_t k = smem_u32(sK), q = smem_u32(sQ);
+    for (int part = 0; part < 2; ++part) {
+      const uint32_t pg = smem_u32(part ? sPGl : sPG);
+      for (int s = 0; s < 4; ++s) {
+        mma_bf16(taddr(tb, 0, 128), desc_kmajor(pg, s, TILE64), desc_mnmajor(k, s, TILE64),
+                 idesc_bf16(64, 128, false, true), 1);
+        mma_bf16(taddr(tb, 0, 256), desc_mnmajor(pg, s, TILE64), desc_mnmajor(q, s, TILE64),
+                 idesc_bf16(64, 128, true, true), 1);
+      }
     }
     mma_commit(&bar[1]);
   }
@@ -574,12 +582,14 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
 //   [256,384) T^T dW -> dk       [384,512) T^T dU
 // ======================================================================================
 struct WyBwdSmem {
-  static constexpr int K = 0, V = 2 * TILE64, T = 4 * TILE64, DW = 5 * TILE64, DUT = 7 * TILE64,
-                       DT = 7 * TILE64 + TILE128, Z = DT + TILE64, AS = Z + TILE64, F = AS + TILE64;
+  static constexpr int K = 0, V = 2 * TILE64, T = 4 * TILE64, TL = 5 * TILE64, DW = 6 * TILE64,
+                       DUT = 8 * TILE64, DT = 8 * TILE64 + TILE128, DTL = DT + TILE64,
+                       Z = DTL + TILE64, ZL = Z + TILE64, AS = ZL + TILE64, ASL = AS + TILE64,
+                       F = ASL + TILE64;
   static constexpr int KKG = F, AA = KKG + 64 * 65 * 4;        // fp32 [64][65] each
   static constexpr int G = AA + 64 * 65 * 4, B = G + 256, ROW = B + 256;  // ROW [4][2][64]
   static constexpr int TOTAL = ROW + 4 * 2 * 64 * 4;
-  static constexpr int LOAD_BYTES = 7 * TILE64 + TILE128;
+  static constexpr int LOAD_BYTES = 8 * TILE64 + TILE128;
 };
 
 __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, TcWork t,
@@ -600,11 +610,15 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   unsigned char* sK = sm + WyBwdSmem::K;
   unsigned char* sV = sm + WyBwdSmem::V;
   unsigned char* sT = sm + WyBwdSmem::T;
+  unsigned char* sTl = sm + WyBwdSmem::TL;
   unsigned char* sdW = sm + WyBwdSmem::DW;
   unsigned char* sdUT = sm + WyBwdSmem::DUT;
   unsigned char* sdT = sm + WyBwdSmem::DT;
+  unsigned char* sdTl = sm + WyBwdSmem::DTL;
   unsigned char* sZ = sm + WyBwdSmem::Z;
+  unsigned char* sZl = sm + WyBwdSmem::ZL;
   unsigned char* sAs = sm + WyBwdSmem::AS;
+  unsigned char* sAsl = sm + WyBwdSmem::ASL;
   float* sKKG = reinterpret_cast<float*>(sm + WyBwdSmem::KKG);
   float* sAA = reinterpret_cast<float*>(sm + WyBwdSmem::AA);
   float* sG = reinterpret_cast<float*>(sm + WyBwdSmem::G);
@@ -630,7 +644,8 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     tma_load_3d(sK + TILE64, &mk, 64, hk, tok0, &bar[0]);
     tma_load_3d(sV, &mv, 0, hv, tok0, &bar[0]);
     tma_load_3d(sV + TILE64, &mv, 64, hv, tok0, &bar[0]);
-    tma_load_3d(sT, &mTm, 0, (int)unit * 64, 0, &bar[0]);
+    tma_load_3d(sT, &mTm, 0, (int)unit * 128, 0, &bar[0]);
+    tma_load_3d(sTl, &mTm, 0, (int)unit * 128 + 64, 0, &bar[0]);
     tma_load_3d(sdW, &mdW, 0, (int)unit * 64, 0, &bar[0]);
     tma_load_3d(sdW + TILE64, &mdW, 64, (int)unit * 64, 0, &bar[0]);
     tma_load_3d(sdUT, &mdUT, 0, (int)unit * D, 0, &bar[0]);
@@ -651,8 +666,8 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   }
   fence_proxy_async();
   __syncthreads();
-  const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aT = smem_u32(sT), aW = smem_u32(sdW),
-                 aU = smem_u32(sdUT);
+  const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aT = smem_u32(sT), aTl = smem_u32(sTl),
+                 aW = smem_u32(sdW), aU = smem_u32(sdUT);
   if (ok && tid == 0) {
     for (int s = 0; s < 8; ++s) {
       const uint32_t acc = s > 0;
@@ -663,12 +678,15 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
       mma_bf16(taddr(tb, 0, 128), desc_kmajor(aK, s, TILE64), desc_kmajor(aK, s, TILE64),
                idesc_bf16(64, 64, false, false), acc);
     }
-    for (int s = 0; s < 4; ++s) {
-      const uint32_t acc = s > 0;
-      mma_bf16(taddr(tb, 0, 256), desc_mnmajor(aT, s, TILE64), desc_mnmajor(aW, s, TILE64),
-               idesc_bf16(64, 128, true, true), acc);
-      mma_bf16(taddr(tb, 0, 384), desc_mnmajor(aT, s, TILE64), desc_kmajor(aU, s, TILE128),
-               idesc_bf16(64, 128, true, false), acc);
+    for (int part = 0; part < 2; ++part) {
+      const uint32_t tt = part ? aTl : aT;
+      for (int s = 0; s < 4; ++s) {
+        const uint32_t acc = part > 0 || s > 0;
+        mma_bf16(taddr(tb, 0, 256), desc_mnmajor(tt, s, TILE64), desc_mnmajor(aW, s, TILE64),
+                 idesc_bf16(64, 128, true, true), acc);
+        mma_bf16(taddr(tb, 0, 384), desc_mnmajor(tt, s, TILE64), desc_kmajor(aU, s, TILE128),
+                 idesc_bf16(64, 128, true, false), acc);
+      }
     }
     mma_commit(&bar[1]);
   }
@@ -689,7 +707,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
       for (int jj = 0; jj < 32; ++jj) {
         const int j = 32 * half + jj;
         f[jj & 7] = sb[j] * (r1[jj] + expf(sG[j]) * r2[jj]);
-        if ((jj & 7) == 7) st_chunk_f(sdT, ii, j / 8, TILE64, f);
+        if ((jj & 7) == 7) st_chunk_split(sdT, sdTl, ii, j / 8, TILE64, f);
         sKKG[ii * 65 + j] = j < ii ? expf(Gi - sG[j]) * kk[jj] : 0.f;
       }
     }
@@ -739,10 +757,13 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   tc_fence_after();
   // Z = T^T dT
   if (ok && tid == 0) {
-    const uint32_t dt = smem_u32(sdT);
-    for (int s = 0; s < 4; ++s)
-      mma_bf16(taddr(tb, 0, 0), desc_mnmajor(aT, s, TILE64), desc_mnmajor(dt, s, TILE64),
-               idesc_bf16(64, 64, true, true), s > 0);
+    // (T_hi + T_lo)^T (dT_hi + dT_lo), dropping lo*lo
+    const uint32_t dt = smem_u32(sdT), dtl = smem_u32(sdTl);
+    const uint32_t pa[3] = {aT, aT, aTl}, pb[3] = {dt, dtl, dt};
+    for (int part = 0; part < 3; ++part)
+      for (int s = 0; s < 4; ++s)
+        mma_bf16(taddr(tb, 0, 0), desc_mnmajor(pa[part], s, TILE64), desc_mnmajor(pb[part], s, TILE64),
+                 idesc_bf16(64, 64, true, true), part > 0 || s > 0);
     mma_commit(&bar[1]);
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
@@ -753,7 +774,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     tmem_ld16(taddr(tb, sub, 32 * half + 16), z + 16);
     tmem_wait_ld();
     if (lane < 16)
-      for (int j = 0; j < 4; ++j) st_chunk_f(sZ, ii, 4 * half + j, TILE64, z + 8 * j);
+      for (int j = 0; j < 4; ++j) st_chunk_split(sZ, sZl, ii, 4 * half + j, TILE64, z + 8 * j);
   }
   fence_proxy_async();
   tc_fence_before();
@@ -761,10 +782,12 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   tc_fence_after();
   // dA' = Z T^T
   if (ok && tid == 0) {
-    const uint32_t zz = smem_u32(sZ);
-    for (int s = 0; s < 4; ++s)
-      mma_bf16(taddr(tb, 0, 64), desc_kmajor(zz, s, TILE64), desc_kmajor(aT, s, TILE64),
-               idesc_bf16(64, 64, false, false), s > 0);
+    const uint32_t zz = smem_u32(sZ), zl = smem_u32(sZl);
+    const uint32_t pa[3] = {zz, zz, zl}, pb[3] = {aT, aTl, aT};
+    for (int part = 0; part < 3; ++part)
+      for (int s = 0; s < 4; ++s)
+        mma_bf16(taddr(tb, 0, 64), desc_kmajor(pa[part], s, TILE64), desc_kmajor(pb[part], s, TILE64),
+                 idesc_bf16(64, 64, false, false), part > 0 || s > 0);
     mma_commit(&bar[1]);
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
@@ -789,7 +812,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
         sAA[ii * 65 + j] = aa;
         paa += aa;
         f[jj & 7] = dAs;
-        if ((jj & 7) == 7) st_chunk_f(sAs, ii, j / 8, TILE64, f);
+        if ((jj & 7) == 7) st_chunk_split(sAs, sAsl, ii, j / 8, TILE64, f);
       }
       sRow[(2 * 2 + half) * 64 + ii] = pa;
       sRow[(3 * 2 + half) * 64 + ii] = paa;
@@ -801,12 +824,14 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   tc_fence_after();
   // dk += dAs K + dAs^T K onto beta e^G dX
   if (ok && tid == 0) {
-    const uint32_t as = smem_u32(sAs);
-    for (int s = 0; s < 4; ++s) {
-      mma_bf16(taddr(tb, 0, 256), desc_kmajor(as, s, TILE64), desc_mnmajor(aK, s, TILE64),
-               idesc_bf16(64, 128, false, true), 1);
-      mma_bf16(taddr(tb, 0, 256), desc_mnmajor(as, s, TILE64), desc_mnmajor(aK, s, TILE64),
-               idesc_bf16(64, 128, true, true), 1);
+    for (int part = 0; part < 2; ++part) {
+      const uint32_t as = smem_u32(part ? sAsl : sAs);
+      for (int s = 0; s < 4; ++s) {
+        mma_bf16(taddr(tb, 0, 256), desc_kmajor(as, s, TILE64), desc_mnmajor(aK, s, TILE64),
+                 idesc_bf16(64, 128, false, true), 1);
+        mma_bf16(taddr(tb, 0, 256), desc_mnmajor(as, s, TILE64), desc_mnmajor(aK, s, TILE64),
+                 idesc_bf16(64, 128, true, true), 1);
+      }
     }
     mma_commit(&bar[1]);
   }
@@ -852,7 +877,7 @@ cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, 
                                 const TcMaps& m, cudaStream_t s) {
   cudaError_t e;
   const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV);
-  if ((e = tgo("tc_dvlocal", k_tc_dvlocal, gu, 128, 1024 + 7 * TILE64 + 256, s, p, w, t, m.q, m.k,
+  if ((e = tgo("tc_dvlocal", k_tc_dvlocal, gu, 128, 1024 + 8 * TILE64 + 256, s, p, w, t, m.q, m.k,
                m.dO)))
     return e;
   if ((e = tgo("tc_scan_bwd", k_tc_scan_bwd, gs, 256, 1024 + BwdScanSmem::TOTAL, s, p, a, w, t, m.q,

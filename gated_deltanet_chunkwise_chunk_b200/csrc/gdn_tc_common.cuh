@@ -76,7 +76,7 @@ struct TcWork {
   bf16* UtT;    // [NC*HV][128][64]
   bf16* UT;     // [NC*HV][128][64]
   bf16* h;      // [NC*HV][128][128]
-  bf16* Tm;     // [NC*HV][64][64]   (backward only) (I + A)^-1
+  bf16* Tm;     // [NC*HV][2][64][64] (backward only) (I + A)^-1 as hi, lo bf16 parts
   bf16* dUlT;   // [NC*HV][128][64]  dv_local^T = scale (P^T dO)^T
   bf16* dh;     // [NC*HV][128][128] dL/dS leaving the chunk (S orientation [v][k])
   bf16* dUT;    // [NC*HV][128][64]  dU^T (full)
@@ -100,7 +100,7 @@ inline TcWork carve_tc(void* base, size_t NC, size_t HV, int pass) {
   t.UT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
   t.h = reinterpret_cast<bf16*>(take(units * D * D * 2));
   if (pass == 1) {
-    t.Tm = reinterpret_cast<bf16*>(take(units * 64 * 64 * 2));
+    t.Tm = reinterpret_cast<bf16*>(take(units * 2 * 64 * 64 * 2));
     t.dUlT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
     t.dh = reinterpret_cast<bf16*>(take(units * D * D * 2));
     t.dUT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
@@ -113,7 +113,7 @@ inline size_t tc_bytes(size_t NC, size_t HV, int pass) {
   const size_t units = NC * HV;
   size_t o = 3 * align_up(units * D * 64 * 2) + align_up(units * D * D * 2);
   if (pass == 1)
-    o += align_up(units * 64 * 64 * 2) + 2 * align_up(units * D * 64 * 2) +
+    o += align_up(units * 2 * 64 * 64 * 2) + 2 * align_up(units * D * 64 * 2) +
          align_up(units * D * D * 2) + align_up(units * 64 * D * 2);
   return o;
 }
@@ -152,6 +152,20 @@ __device__ __forceinline__ void st_chunk_f(unsigned char* tile, int r, int j, in
   v.z = pack_bf16(f[4], f[5]);
   v.w = pack_bf16(f[6], f[7]);
   *reinterpret_cast<uint4*>(tile + sw128_chunk(r, j, block_bytes)) = v;
+}
+
+// Stores 8 floats as a compensated bf16 pair: hi = bf16(f), lo = bf16(f - hi), so that
+// A = A_hi + A_lo carries ~16 mantissa bits through two tensor-core products.
+__device__ __forceinline__ void st_chunk_split(unsigned char* hi, unsigned char* lo, int r, int j,
+                                               int block_bytes, const float* f) {
+  float h[8], l[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    h[q] = __bfloat162float(__float2bfloat16_rn(f[q]));
+    l[q] = f[q] - h[q];
+  }
+  st_chunk_f(hi, r, j, block_bytes, h);
+  st_chunk_f(lo, r, j, block_bytes, l);
 }
 
 __device__ __forceinline__ bool failed(const Work& w) { return *((volatile int*)w.status) != 0; }
