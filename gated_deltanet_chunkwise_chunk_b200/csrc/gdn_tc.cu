@@ -525,6 +525,7 @@ Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
     const uint64_t trows = (uint64_t)p.NCmax * p.HV * 64;
     L.ok &= map_rows(&L.m.dUlT, L.t.dUlT, urows, 64, 128);
     L.ok &= map_rows(&L.m.dUT, L.t.dUT, urows, 64, 128);
+    L.ok &= map_rows(&L.m.dUTl, L.t.dUTl, urows, 64, 128);
     L.ok &= map_rows(&L.m.dh, L.t.dh, urows, 128, 128);
     L.ok &= map_rows(&L.m.dW, L.t.dW, trows, 128, 64);
     L.ok &= map_rows(&L.m.Tm, L.t.Tm, 2 * trows, 64, 64);

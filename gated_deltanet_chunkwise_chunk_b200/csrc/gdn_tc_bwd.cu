@@ -136,19 +136,24 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
 
 // ======================================================================================
 // Reverse state scan.  One CTA (256 threads) per (sequence, value head); thread
-// (v = 32*(warp%4)+lane, half = warp/4) keeps dS[v][64*half..+63] in fp32 registers.
+// (v = 32*(warp%4)+lane, half = warp/4) keeps dS[v][64*half..+63] in fp32 registers.  The
+// tensor-core operands that carry the chain (dS and -dU^T) are compensated bf16 pairs
+// (hi + lo), and dU^T is written out as such a pair.  Tiles are single-buffered: each
+// group is reloaded for the next chunk as soon as its last reader is done.
+//   MMA2a (off the chain): F  = (scale diag(e^G) dO)^T Q        (M=128 v, N=128 k, K=64 i)
+//   MMA1:                   E  = dS K^T                         (M=128 v, N=64 j,  K=128 k)
+//   dU^T = dU_loc^T + E diag(e^{G_C-G})
+//   MMA2b:                  F -= dU^T W                         (M=128 v, N=128 k, K=64 j)
+//   dS = e^{G_C} dS + F
 // ======================================================================================
 struct BwdScanSmem {
-  static constexpr int S = 0;                          // dS bf16 [128][128]
-  static constexpr int BUF = 2 * TILE128;
-  static constexpr int OFF_K = 0, OFF_Q = 2 * TILE64, OFF_O = 4 * TILE64, OFF_W = 6 * TILE64,
-                       OFF_UL = 6 * TILE64 + TILE128;
-  static constexpr int BUF_BYTES = 6 * TILE64 + 2 * TILE128;
-  static constexpr int AT = BUF + 2 * BUF_BYTES;       // -dU^T [128][64]
-  static constexpr int UO = AT + TILE128;              // +dU^T staging
-  static constexpr int G = UO + TILE128;               // 2 x 64 floats
-  static constexpr int DEC = G + 512;                  // e^{G_C - G_j}
-  static constexpr int EG = DEC + 256;                 // scale e^{G_i}
+  static constexpr int SH = 0, SL = 2 * TILE128;                 // dS hi / lo [128][128]
+  static constexpr int K = 4 * TILE128, Q = K + 2 * TILE64, O = Q + 2 * TILE64;
+  static constexpr int W = O + 2 * TILE64, UL = W + TILE128;     // W^T, dU_loc^T [128][64]
+  static constexpr int ATH = UL + TILE128, ATL = ATH + TILE128;  // -dU^T hi / lo
+  static constexpr int G = ATL + TILE128;                        // 64 floats
+  static constexpr int DEC = G + 256;                            // e^{G_C - G_j}
+  static constexpr int EG = DEC + 256;                           // scale e^{G_i} (0 past L)
   static constexpr int TOTAL = EG + 256;
 };
 
@@ -158,7 +163,6 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
                                                      const __grid_constant__ CUtensorMap mdO,
                                                      const __grid_constant__ CUtensorMap mWT,
                                                      const __grid_constant__ CUtensorMap mdUlT,
-                                                     const __grid_constant__ CUtensorMap mdUT,
                                                      const __grid_constant__ CUtensorMap mdh) {
   if (failed(w)) return;
   const int n = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
@@ -167,18 +171,25 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
   const int v = 32 * (warp & 3) + lane, half = warp >> 2;
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
-  unsigned char* sS = sm + BwdScanSmem::S;
-  unsigned char* sAT = sm + BwdScanSmem::AT;
-  unsigned char* sUO = sm + BwdScanSmem::UO;
-  float* sGb = reinterpret_cast<float*>(sm + BwdScanSmem::G);
+  unsigned char* sSH = sm + BwdScanSmem::SH;
+  unsigned char* sSL = sm + BwdScanSmem::SL;
+  unsigned char* sK = sm + BwdScanSmem::K;
+  unsigned char* sQ = sm + BwdScanSmem::Q;
+  unsigned char* sO = sm + BwdScanSmem::O;
+  unsigned char* sW = sm + BwdScanSmem::W;
+  unsigned char* sUL = sm + BwdScanSmem::UL;
+  unsigned char* sATH = sm + BwdScanSmem::ATH;
+  unsigned char* sATL = sm + BwdScanSmem::ATL;
+  float* sG = reinterpret_cast<float*>(sm + BwdScanSmem::G);
   float* sDec = reinterpret_cast<float*>(sm + BwdScanSmem::DEC);
   float* sEG = reinterpret_cast<float*>(sm + BwdScanSmem::EG);
-  __shared__ uint64_t barT[2], barM;
+  __shared__ uint64_t barA, barW, barU, barM;
   __shared__ uint32_t tslot;
   int* err = w.status;
   if (tid == 0) {
-    mbar_init(&barT[0], 1);
-    mbar_init(&barT[1], 1);
+    mbar_init(&barA, 1);
+    mbar_init(&barW, 1);
+    mbar_init(&barU, 1);
     mbar_init(&barM, 1);
     mbar_fence_init();
   }
@@ -190,94 +201,109 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
   float S[64];
   const size_t st = ((size_t)n * p.HV + hv) * D * D;
   for (int i = 0; i < 64; ++i) S[i] = a.dht ? a.dht[st + (size_t)(half * 64 + i) * D + v] : 0.f;
-  for (int j = 0; j < 8; ++j) st_chunk_f(sS, v, half * 8 + j, TILE128, &S[8 * j]);
-  auto issue = [&](int c, int buf) {
-    const int gc = sq.x + c;
-    const int4 e = w.chunk_tab[gc];
-    unsigned char* b = sm + BwdScanSmem::BUF + buf * BwdScanSmem::BUF_BYTES;
-    const int row = (gc * p.HV + hv) * D;
-    mbar_expect_tx(&barT[buf], BwdScanSmem::BUF_BYTES);
-    tma_load_3d(b + BwdScanSmem::OFF_K, &mk, 0, hk, e.w, &barT[buf]);
-    tma_load_3d(b + BwdScanSmem::OFF_K + TILE64, &mk, 64, hk, e.w, &barT[buf]);
-    tma_load_3d(b + BwdScanSmem::OFF_Q, &mq, 0, hk, e.w, &barT[buf]);
-    tma_load_3d(b + BwdScanSmem::OFF_Q + TILE64, &mq, 64, hk, e.w, &barT[buf]);
-    tma_load_3d(b + BwdScanSmem::OFF_O, &mdO, 0, hv, e.w, &barT[buf]);
-    tma_load_3d(b + BwdScanSmem::OFF_O + TILE64, &mdO, 64, hv, e.w, &barT[buf]);
-    tma_load_3d(b + BwdScanSmem::OFF_W, &mWT, 0, row, 0, &barT[buf]);
-    tma_load_3d(b + BwdScanSmem::OFF_UL, &mdUlT, 0, row, 0, &barT[buf]);
+  for (int j = 0; j < 8; ++j) st_chunk_split(sSH, sSL, v, half * 8 + j, TILE128, &S[8 * j]);
+  auto row_of = [&](int c) { return ((sq.x + c) * p.HV + hv) * D; };
+  auto issue_A = [&](int c) {  // K, Q, dO of chunk c
+    const int tok = w.chunk_tab[sq.x + c].w;
+    mbar_expect_tx(&barA, 6 * TILE64);
+    tma_load_3d(sK, &mk, 0, hk, tok, &barA);
+    tma_load_3d(sK + TILE64, &mk, 64, hk, tok, &barA);
+    tma_load_3d(sQ, &mq, 0, hk, tok, &barA);
+    tma_load_3d(sQ + TILE64, &mq, 64, hk, tok, &barA);
+    tma_load_3d(sO, &mdO, 0, hv, tok, &barA);
+    tma_load_3d(sO + TILE64, &mdO, 64, hv, tok, &barA);
   };
-  if (tid == 0 && sq.y > 0) issue(sq.y - 1, 0);
+  auto issue_W = [&](int c) {
+    mbar_expect_tx(&barW, TILE128);
+    tma_load_3d(sW, &mWT, 0, row_of(c), 0, &barW);
+  };
+  auto issue_U = [&](int c) {
+    mbar_expect_tx(&barU, TILE128);
+    tma_load_3d(sUL, &mdUlT, 0, row_of(c), 0, &barU);
+  };
+  if (tid == 0 && sq.y > 0) {
+    issue_A(sq.y - 1);
+    issue_W(sq.y - 1);
+    issue_U(sq.y - 1);
+  }
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
   const uint32_t tE = taddr(tb, 0, 0), tF = taddr(tb, 0, 64);
-  uint32_t phT[2] = {0, 0}, phM = 0;
+  uint32_t ph = 0, phM = 0;  // barA/barW/barU complete once per chunk; barM twice
   bool ok = true;
   for (int idx = 0; idx < sq.y && ok; ++idx) {
-    const int c = sq.y - 1 - idx, gc = sq.x + c, buf = idx & 1;
-    unsigned char* b = sm + BwdScanSmem::BUF + buf * BwdScanSmem::BUF_BYTES;
+    const int c = sq.y - 1 - idx, gc = sq.x + c;
+    const bool more = idx + 1 < sq.y;
     const int L = w.chunk_tab[gc].z;
-    const uint32_t unit_row = (uint32_t)(gc * p.HV + hv) * D;
-    float* sG = sGb + buf * 64;
-    if (tid == 0 && idx + 1 < sq.y) issue(c - 1, buf ^ 1);
+    const uint32_t unit_row = (uint32_t)row_of(c);
     if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
-    ok = __syncthreads_and(mbar_wait(&barT[buf], phT[buf], err));
-    phT[buf] ^= 1;
+    ok = __syncthreads_and(mbar_wait(&barA, ph, err));
     if (!ok) break;
     if (tid < 64) {
       sDec[tid] = expf(sG[63] - sG[tid]);
       sEG[tid] = tid < L ? p.scale * expf(sG[tid]) : 0.f;
     }
     __syncthreads();
-    // dO rows scaled by scale e^{G_i} (zero past the chunk end); K rows past the end zeroed
-    unsigned char* tO = b + BwdScanSmem::OFF_O;
-    for (int i = tid; i < 64 * 16; i += 256) {
+    for (int i = tid; i < 64 * 16; i += 256) {  // dO rows scaled by scale e^{G_i}, 0 past L
       const int r = i / 16, j = i % 16;
       float f[8];
-      ld_chunk_f(tO, r, j, TILE64, f);
+      ld_chunk_f(sO, r, j, TILE64, f);
       for (int q = 0; q < 8; ++q) f[q] *= sEG[r];
-      st_chunk_f(tO, r, j, TILE64, f);
+      st_chunk_f(sO, r, j, TILE64, f);
     }
-    if (L < 64) zero_tail_rows(b + BwdScanSmem::OFF_K, L, tid, 256);
+    if (L < 64) zero_tail_rows(sK, L, tid, 256);
     fence_proxy_async();
     __syncthreads();
     if (tid == 0) {
-      tma_store_3d(&mdh, sS, 0, unit_row, 0);
-      tma_store_3d(&mdh, sS + TILE128, 64, unit_row, 0);
+      tma_store_3d(&mdh, sSH, 0, unit_row, 0);
+      tma_store_3d(&mdh, sSH + TILE128, 64, unit_row, 0);
       tma_store_commit();
-      const uint32_t o = smem_u32(tO), q = smem_u32(b + BwdScanSmem::OFF_Q);
-      const uint32_t s_ = smem_u32(sS), k = smem_u32(b + BwdScanSmem::OFF_K);
+      const uint32_t o = smem_u32(sO), q = smem_u32(sQ), k = smem_u32(sK);
       for (int s = 0; s < 4; ++s)
         mma_bf16(tF, desc_mnmajor(o, s, TILE64), desc_mnmajor(q, s, TILE64),
                  idesc_bf16(128, 128, true, true), s > 0);
-      for (int s = 0; s < 8; ++s)
-        mma_bf16(tE, desc_kmajor(s_, s, TILE128), desc_kmajor(k, s, TILE64),
-                 idesc_bf16(128, 64, false, false), s > 0);
+      for (int part = 0; part < 2; ++part) {
+        const uint32_t sa = smem_u32(part ? sSL : sSH);
+        for (int s = 0; s < 8; ++s)
+          mma_bf16(tE, desc_kmajor(sa, s, TILE128), desc_kmajor(k, s, TILE64),
+                   idesc_bf16(128, 64, false, false), part > 0 || s > 0);
+      }
       mma_commit(&barM);
     }
     ok = __syncthreads_and(mbar_wait(&barM, phM, err));
     phM ^= 1;
     tc_fence_after();
     if (!ok) break;
+    if (tid == 0 && more) issue_A(c - 1);  // K, Q, dO consumed by the MMAs above
+    ok = __syncthreads_and(mbar_wait(&barU, ph, err));
+    if (!ok) break;
     {
       float d[32];
       tmem_ld16(taddr(tb, 32 * (warp & 3), 32 * half), d);
       tmem_ld16(taddr(tb, 32 * (warp & 3), 32 * half + 16), d + 16);
       tmem_wait_ld();
-      if (tid == 0) tma_store_wait_read0();
-      __syncthreads();
-      const unsigned char* ul = b + BwdScanSmem::OFF_UL;
+      bf16* hi_row = t.dUT + ((size_t)unit_row + v) * 64 + 32 * half;
+      bf16* lo_row = t.dUTl + ((size_t)unit_row + v) * 64 + 32 * half;
       for (int j = 0; j < 4; ++j) {
-        float u[8], nu[8];
-        ld_chunk_f(ul, v, half * 4 + j, TILE128, u);
+        float u[8], nu[8], hl[8], ll[8];
+        ld_chunk_f(sUL, v, half * 4 + j, TILE128, u);
         for (int q = 0; q < 8; ++q) {
           u[q] += sDec[32 * half + 8 * j + q] * d[8 * j + q];
           nu[q] = -u[q];
+          hl[q] = __bfloat162float(__float2bfloat16_rn(u[q]));
+          ll[q] = u[q] - hl[q];
         }
-        st_chunk_f(sUO, v, half * 4 + j, TILE128, u);
-        st_chunk_f(sAT, v, half * 4 + j, TILE128, nu);
+        st_chunk_split(sATH, sATL, v, half * 4 + j, TILE128, nu);
+        uint4 ph4, pl4;
+        ph4.x = pack_bf16(hl[0], hl[1]); ph4.y = pack_bf16(hl[2], hl[3]);
+        ph4.z = pack_bf16(hl[4], hl[5]); ph4.w = pack_bf16(hl[6], hl[7]);
+        pl4.x = pack_bf16(ll[0], ll[1]); pl4.y = pack_bf16(ll[2], ll[3]);
+        pl4.z = pack_bf16(ll[4], ll[5]); pl4.w = pack_bf16(ll[6], ll[7]);
+        *reinterpret_cast<uint4*>(hi_row + 8 * j) = ph4;
+        *reinterpret_cast<uint4*>(lo_row + 8 * j) = pl4;
       }
     }
     fence_proxy_async();
@@ -285,18 +311,25 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     __syncthreads();
     tc_fence_after();
     if (tid == 0) {
-      tma_store_3d(&mdUT, sUO, 0, unit_row, 0);
-      tma_store_commit();
-      const uint32_t at = smem_u32(sAT), wt = smem_u32(b + BwdScanSmem::OFF_W);
-      for (int s = 0; s < 4; ++s)
-        mma_bf16(tF, desc_kmajor(at, s, TILE128), desc_kmajor(wt, s, TILE128),
-                 idesc_bf16(128, 128, false, false), 1);
-      mma_commit(&barM);
+      if (more) issue_U(c - 1);  // dU_loc^T consumed
+      bool wok = mbar_wait(&barW, ph, err);
+      if (wok) {
+        const uint32_t wt = smem_u32(sW);
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t at = smem_u32(part ? sATL : sATH);
+          for (int s = 0; s < 4; ++s)
+            mma_bf16(tF, desc_kmajor(at, s, TILE128), desc_kmajor(wt, s, TILE128),
+                     idesc_bf16(128, 128, false, false), 1);
+        }
+        mma_commit(&barM);
+      }
     }
     ok = __syncthreads_and(mbar_wait(&barM, phM, err));
     phM ^= 1;
+    ph ^= 1;
     tc_fence_after();
     if (!ok) break;
+    if (tid == 0 && more) issue_W(c - 1);  // W^T consumed
     {
       const float eg = expf(sG[63]);
       for (int cc = 0; cc < 64; cc += 16) {
@@ -306,9 +339,9 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
         for (int i = 0; i < 16; ++i) S[cc + i] = eg * S[cc + i] + d[i];
       }
     }
-    if (tid == 0) tma_store_wait_read0();
+    if (tid == 0) tma_store_wait_read0();  // the dh store has finished reading dS hi
     __syncthreads();
-    for (int j = 0; j < 8; ++j) st_chunk_f(sS, v, half * 8 + j, TILE128, &S[8 * j]);
+    for (int j = 0; j < 8; ++j) st_chunk_split(sSH, sSL, v, half * 8 + j, TILE128, &S[8 * j]);
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
@@ -332,12 +365,13 @@ struct DqkSmem {
   static constexpr int Q = 0, K = 2 * TILE64, O = 4 * TILE64, UT = 6 * TILE64,
                        DUT = 6 * TILE64 + TILE128, H = 6 * TILE64 + 2 * TILE128,
                        DH = 6 * TILE64 + 4 * TILE128, PG = 6 * TILE64 + 6 * TILE128,
-                       PGL = PG + TILE64, M = PGL + TILE64;  // fp32 [64][65] dP*P
+                       PGL = PG + TILE64, DUTL = PGL + TILE64,
+                       M = DUTL + TILE128;                   // fp32 [64][65] dP*P
   static constexpr int G = M + 64 * 65 * 4;
   static constexpr int ROW = G + 256;                        // [3][2][64] per-row partials
   static constexpr int RED = ROW + 3 * 2 * 64 * 4;           // [8]
   static constexpr int TOTAL = RED + 64;
-  static constexpr int LOAD_BYTES = 6 * TILE64 + 6 * TILE128;
+  static constexpr int LOAD_BYTES = 6 * TILE64 + 7 * TILE128;
 };
 
 __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
@@ -346,6 +380,7 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
                                                   const __grid_constant__ CUtensorMap mdO,
                                                   const __grid_constant__ CUtensorMap mUT,
                                                   const __grid_constant__ CUtensorMap mdUT,
+                                                  const __grid_constant__ CUtensorMap mdUTl,
                                                   const __grid_constant__ CUtensorMap mh,
                                                   const __grid_constant__ CUtensorMap mdh) {
   if (failed(w)) return;
@@ -365,6 +400,7 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
   unsigned char* sdH = sm + DqkSmem::DH;
   unsigned char* sPG = sm + DqkSmem::PG;
   unsigned char* sPGl = sm + DqkSmem::PGL;
+  unsigned char* sdUTl = sm + DqkSmem::DUTL;
   float* sM = reinterpret_cast<float*>(sm + DqkSmem::M);
   float* sG = reinterpret_cast<float*>(sm + DqkSmem::G);
   float* sRow = reinterpret_cast<float*>(sm + DqkSmem::ROW);  // [kind][half][64]
@@ -394,6 +430,7 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
     tma_load_3d(sO + TILE64, &mdO, 64, hv, tok0, &bar[0]);
     tma_load_3d(sUT, &mUT, 0, row, 0, &bar[0]);
     tma_load_3d(sdUT, &mdUT, 0, row, 0, &bar[0]);
+    tma_load_3d(sdUTl, &mdUTl, 0, row, 0, &bar[0]);
     tma_load_3d(sH, &mh, 0, row, 0, &bar[0]);
     tma_load_3d(sH + TILE128, &mh, 64, row, 0, &bar[0]);
     tma_load_3d(sdH, &mdh, 0, row, 0, &bar[0]);
@@ -428,6 +465,10 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
       mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dut, s, TILE128), desc_mnmajor(h, s, TILE128),
                idesc_bf16(64, 128, true, true), acc);
     }
+    const uint32_t dutl = smem_u32(sdUTl);
+    for (int s = 0; s < 8; ++s)
+      mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dutl, s, TILE128), desc_mnmajor(h, s, TILE128),
+               idesc_bf16(64, 128, true, true), 1);
     mma_commit(&bar[1]);
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
@@ -585,11 +626,11 @@ struct WyBwdSmem {
   static constexpr int K = 0, V = 2 * TILE64, T = 4 * TILE64, TL = 5 * TILE64, DW = 6 * TILE64,
                        DUT = 8 * TILE64, DT = 8 * TILE64 + TILE128, DTL = DT + TILE64,
                        Z = DTL + TILE64, ZL = Z + TILE64, AS = ZL + TILE64, ASL = AS + TILE64,
-                       F = ASL + TILE64;
+                       DUTL = ASL + TILE64, F = DUTL + TILE128;
   static constexpr int KKG = F, AA = KKG + 64 * 65 * 4;        // fp32 [64][65] each
   static constexpr int G = AA + 64 * 65 * 4, B = G + 256, ROW = B + 256;  // ROW [4][2][64]
   static constexpr int TOTAL = ROW + 4 * 2 * 64 * 4;
-  static constexpr int LOAD_BYTES = 8 * TILE64 + TILE128;
+  static constexpr int LOAD_BYTES = 8 * TILE64 + 2 * TILE128;
 };
 
 __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, TcWork t,
@@ -597,7 +638,8 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
                                                    const __grid_constant__ CUtensorMap mv,
                                                    const __grid_constant__ CUtensorMap mTm,
                                                    const __grid_constant__ CUtensorMap mdW,
-                                                   const __grid_constant__ CUtensorMap mdUT) {
+                                                   const __grid_constant__ CUtensorMap mdUT,
+                                                   const __grid_constant__ CUtensorMap mdUTl) {
   if (failed(w)) return;
   const int gc = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
   const int4 e = w.chunk_tab[gc];
@@ -619,6 +661,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   unsigned char* sZl = sm + WyBwdSmem::ZL;
   unsigned char* sAs = sm + WyBwdSmem::AS;
   unsigned char* sAsl = sm + WyBwdSmem::ASL;
+  unsigned char* sdUTl = sm + WyBwdSmem::DUTL;
   float* sKKG = reinterpret_cast<float*>(sm + WyBwdSmem::KKG);
   float* sAA = reinterpret_cast<float*>(sm + WyBwdSmem::AA);
   float* sG = reinterpret_cast<float*>(sm + WyBwdSmem::G);
@@ -649,6 +692,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     tma_load_3d(sdW, &mdW, 0, (int)unit * 64, 0, &bar[0]);
     tma_load_3d(sdW + TILE64, &mdW, 64, (int)unit * 64, 0, &bar[0]);
     tma_load_3d(sdUT, &mdUT, 0, (int)unit * D, 0, &bar[0]);
+    tma_load_3d(sdUTl, &mdUTl, 0, (int)unit * D, 0, &bar[0]);
   }
   if (tid < 64) {
     const size_t o = ((size_t)hv * p.NCmax + gc) * 64 + tid;
@@ -667,12 +711,14 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   fence_proxy_async();
   __syncthreads();
   const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aT = smem_u32(sT), aTl = smem_u32(sTl),
-                 aW = smem_u32(sdW), aU = smem_u32(sdUT);
+                 aW = smem_u32(sdW), aU = smem_u32(sdUT), aUl = smem_u32(sdUTl);
   if (ok && tid == 0) {
     for (int s = 0; s < 8; ++s) {
       const uint32_t acc = s > 0;
       mma_bf16(taddr(tb, 0, 0), desc_mnmajor(aU, s, TILE128), desc_kmajor(aV, s, TILE64),
                idesc_bf16(64, 64, true, false), acc);
+      mma_bf16(taddr(tb, 0, 0), desc_mnmajor(aUl, s, TILE128), desc_kmajor(aV, s, TILE64),
+               idesc_bf16(64, 64, true, false), 1);
       mma_bf16(taddr(tb, 0, 64), desc_kmajor(aW, s, TILE64), desc_kmajor(aK, s, TILE64),
                idesc_bf16(64, 64, false, false), acc);
       mma_bf16(taddr(tb, 0, 128), desc_kmajor(aK, s, TILE64), desc_kmajor(aK, s, TILE64),
@@ -686,6 +732,9 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
                  idesc_bf16(64, 128, true, true), acc);
         mma_bf16(taddr(tb, 0, 384), desc_mnmajor(tt, s, TILE64), desc_kmajor(aU, s, TILE128),
                  idesc_bf16(64, 128, true, false), acc);
+        if (part == 0)
+          mma_bf16(taddr(tb, 0, 384), desc_mnmajor(tt, s, TILE64), desc_kmajor(aUl, s, TILE128),
+                   idesc_bf16(64, 128, true, false), 1);
       }
     }
     mma_commit(&bar[1]);
@@ -881,13 +930,13 @@ cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, 
                m.dO)))
     return e;
   if ((e = tgo("tc_scan_bwd", k_tc_scan_bwd, gs, 256, 1024 + BwdScanSmem::TOTAL, s, p, a, w, t, m.q,
-               m.k, m.dO, m.WT, m.dUlT, m.dUT, m.dh)))
+               m.k, m.dO, m.WT, m.dUlT, m.dh)))
     return e;
   if ((e = tgo("tc_dqkwg", k_tc_dqkwg, gu, 256, 1024 + DqkSmem::TOTAL, s, p, w, t, m.q, m.k, m.dO,
-               m.UT, m.dUT, m.h, m.dh)))
+               m.UT, m.dUT, m.dUTl, m.h, m.dh)))
     return e;
   if ((e = tgo("tc_wy_bwd", k_tc_wy_bwd, gu, 256, 1024 + WyBwdSmem::TOTAL, s, p, a, w, t, m.k, m.v,
-               m.Tm, m.dW, m.dUT)))
+               m.Tm, m.dW, m.dUT, m.dUTl)))
     return e;
   return cudaSuccess;
 }

@@ -65,7 +65,7 @@ struct TcMaps {
   CUtensorMap q, k, v, dO;            // token tensors
   CUtensorMap WT, UtT, UT;            // [unit*128][64]
   CUtensorMap h;                      // [unit*128][128]
-  CUtensorMap dUlT, dUT;              // [unit*128][64]      (backward)
+  CUtensorMap dUlT, dUT, dUTl;        // [unit*128][64]      (backward)
   CUtensorMap dh;                     // [unit*128][128]     (backward)
   CUtensorMap dW;                     // [unit*64][128]      (backward)
   CUtensorMap Tm;                     // [unit*64][64]       (backward)
@@ -79,7 +79,8 @@ struct TcWork {
   bf16* Tm;     // [NC*HV][2][64][64] (backward only) (I + A)^-1 as hi, lo bf16 parts
   bf16* dUlT;   // [NC*HV][128][64]  dv_local^T = scale (P^T dO)^T
   bf16* dh;     // [NC*HV][128][128] dL/dS leaving the chunk (S orientation [v][k])
-  bf16* dUT;    // [NC*HV][128][64]  dU^T (full)
+  bf16* dUT;    // [NC*HV][128][64]  dU^T (full), hi part
+  bf16* dUTl;   // [NC*HV][128][64]  dU^T lo part (dU^T - hi)
   bf16* dW;     // [NC*HV][64][128]  dL/dW
 };
 
@@ -104,6 +105,7 @@ inline TcWork carve_tc(void* base, size_t NC, size_t HV, int pass) {
     t.dUlT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
     t.dh = reinterpret_cast<bf16*>(take(units * D * D * 2));
     t.dUT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
+    t.dUTl = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
     t.dW = reinterpret_cast<bf16*>(take(units * 64 * D * 2));
   }
   return t;
@@ -113,7 +115,7 @@ inline size_t tc_bytes(size_t NC, size_t HV, int pass) {
   const size_t units = NC * HV;
   size_t o = 3 * align_up(units * D * 64 * 2) + align_up(units * D * D * 2);
   if (pass == 1)
-    o += align_up(units * 2 * 64 * 64 * 2) + 2 * align_up(units * D * 64 * 2) +
+    o += align_up(units * 2 * 64 * 64 * 2) + 3 * align_up(units * D * 64 * 2) +
          align_up(units * D * D * 2) + align_up(units * 64 * D * 2);
   return o;
 }
