@@ -149,6 +149,26 @@ def test_invalid_cu_seqlens_sets_device_status():
     assert gdn.gdn_device_status(ws) == 0
 
 
+def test_param_grad_reductions_match_gpu_dg():
+    """dA_log and ddt_bias are the kernel's reductions of its own dg: they must equal the
+    fp64 sums sum_t dg_t g_t and sum_t dg_raw_t of the GPU's dg / dg_raw (g from the gate
+    formula), up to fp32 summation rounding relative to sum_t |terms|."""
+    for case in (synth.make_case(B=2, T=700, H=2, HV=4, K=128, V=128, dtype="bf16", seed=21,
+                                 h0=True, dht=True, big_a=True),
+                 synth.make_case(H=2, HV=4, K=128, V=128, dtype="bf16", seed=22,
+                                 lengths=[300, 1, 517, 64], dht=True)):
+        gpu = run_gpu(case)
+        x = case.a.double().numpy() + case.dt_bias.double().numpy()
+        sp = np.where(x > 20, x, np.log1p(np.exp(np.minimum(x, 50.0))))
+        g = -np.exp(case.A_log.double().numpy()) * sp
+        terms = gpu["dg"] * g
+        err = np.abs(gpu["dA_log"] - terms.sum(axis=(0, 1)))
+        assert (err <= 1e-5 * np.abs(terms).sum(axis=(0, 1)) + 1e-6).all(), err
+        terms2 = gpu["dg_raw"]
+        err2 = np.abs(gpu["ddt_bias"] - terms2.sum(axis=(0, 1)))
+        assert (err2 <= 1e-5 * np.abs(terms2).sum(axis=(0, 1)) + 1e-6).all(), err2
+
+
 def test_run_to_run_bitwise_reproducible():
     case = synth.make_case(B=1, T=700, H=2, HV=4, K=128, V=128, dtype="bf16", seed=18, h0=True,
                            dht=True)
