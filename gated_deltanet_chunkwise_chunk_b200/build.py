@@ -1,6 +1,8 @@
 """Builds the in-tree CUDA library libgdn_b200.so for sm_100a with nvcc.
 
-    python -m gated_deltanet_chunkwise_chunk_b200.build [--force]
+    python gated_deltanet_chunkwise_chunk_b200/build.py [--force] [--ptxas]
+
+(run it by path: importing the package loads the library this script builds).
 
 Each .cu under csrc/ is compiled to an object (in parallel), then linked into one shared
 library next to this file (cudart linked statically, so the library loads without
