@@ -23,7 +23,7 @@ GDN_DTYPE_FP32, GDN_DTYPE_BF16 = 0, 1
 EXPORTED = ("gdn_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_max_chunks",
             "gdn_build_chunk_indices", "gdn_chunk_table_device", "gdn_device_status",
             "gdn_status_string", "gdn_version", "gdn_launch_count", "gdn_profile",
-            "gdn_profile_read")
+            "gdn_profile_read", "gdn_chunk_fwd_noalloc", "gdn_noalloc_scratch_bytes")
 
 
 class gdn_dims(ctypes.Structure):
@@ -41,7 +41,7 @@ class GDNError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m gated_deltanet_chunkwise_chunk_b200.build`")
+                          "`python gated_deltanet_chunkwise_chunk_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
     D = ctypes.POINTER(gdn_dims)
@@ -63,6 +63,10 @@ def _load() -> ctypes.CDLL:
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_version.argtypes = []
     lib.gdn_version.restype = ctypes.c_char_p
+    lib.gdn_chunk_fwd_noalloc.argtypes = [D] + [P] * 12
+    lib.gdn_chunk_fwd_noalloc.restype = I32
+    lib.gdn_noalloc_scratch_bytes.argtypes = []
+    lib.gdn_noalloc_scratch_bytes.restype = SZ
     lib.gdn_launch_count.argtypes = []
     lib.gdn_launch_count.restype = I64
     lib.gdn_profile.argtypes = [I32]
@@ -158,6 +162,28 @@ def gdn_chunk_fwd(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None, initial
     if rc != GDN_OK:
         raise GDNError("gdn_chunk_fwd", rc)
     return o, ht
+
+
+def gdn_chunk_fwd_noalloc(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None,
+                          initial_state=None, scale=0.0, out=None, final_state=None):
+    """Forward through the library's allocation-free entry point: the scratch is the
+    library's own fixed device array (gdn_noalloc_scratch_bytes()), so the C call allocates
+    nothing.  The caller provides (or here: torch allocates) o and final_state only."""
+    Nst = _check_inputs(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens, initial_state)
+    dims = make_dims(q, v, cu_seqlens, scale)
+    o = out if out is not None else torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    ht = final_state if final_state is not None else torch.empty(
+        (Nst, v.shape[2], q.shape[3], v.shape[3]), dtype=torch.float32, device=q.device)
+    rc = lib.gdn_chunk_fwd_noalloc(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g_raw),
+                                   _ptr(A_log), _ptr(dt_bias), _ptr(beta), _ptr(cu_seqlens),
+                                   _ptr(initial_state), _ptr(o), _ptr(ht), _stream())
+    if rc != GDN_OK:
+        raise GDNError("gdn_chunk_fwd_noalloc", rc)
+    return o, ht
+
+
+def noalloc_scratch_bytes() -> int:
+    return int(lib.gdn_noalloc_scratch_bytes())
 
 
 def gdn_chunk_bwd(q, k, v, g_raw, A_log, dt_bias, beta, d_o, cu_seqlens=None, initial_state=None,

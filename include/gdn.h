@@ -96,6 +96,27 @@ int gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v
                   float* dg_raw, float* dA_log, float* ddt_bias,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* Forward for callers that cannot allocate device memory (no cudaMalloc, no workspace of
+ * their own: e.g. code inside someone else's stream capture, or a plugin whose host owns
+ * all device memory).  The paper has no counterpart; this is a packaging variant of
+ * gdn_chunk_fwd.  Same arguments and results as gdn_chunk_fwd without the workspace: the
+ * scratch is a file-scope device array of GDN_NOALLOC_SCRATCH_BYTES (32 MiB) that every
+ * GPU which loads the library holds until the process exits.  Calls whose
+ * gdn_workspace_bytes(d, varlen, 0) exceeds that size return GDN_ERR_WORKSPACE before any
+ * launch.  The entry point allocates nothing (no cudaMalloc/cudaFree, no library
+ * allocator).  Its first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's contents, so calls
+ * that overlap on the GPU (different streams, or host threads) race: serialise them. */
+#define GDN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+int gdn_chunk_fwd_noalloc(const gdn_dims* d, const void* q, const void* k, const void* v,
+                          const float* g_raw, const float* A_log, const float* dt_bias,
+                          const float* beta, const int64_t* cu_seqlens,
+                          const float* initial_state, void* o, float* final_state, void* stream);
+
+/* Size in bytes of the array gdn_chunk_fwd_noalloc uses (GDN_NOALLOC_SCRATCH_BYTES). */
+size_t gdn_noalloc_scratch_bytes(void);
+
 /* Upper bound on the number of 64-token chunks (the grid size used for chunk kernels). */
 int64_t gdn_max_chunks(const gdn_dims* d, int varlen);
 
