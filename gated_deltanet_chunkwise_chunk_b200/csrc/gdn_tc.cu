@@ -41,7 +41,8 @@ __global__ void __launch_bounds__(128) k_tc_wy(Problem p, Work w, TcWork t,
   unsigned char* sTYl = sTXl + TILE64;
   float* sA = reinterpret_cast<float*>(sTYl + TILE64);  // [64][65]
   float* sT = sA + 64 * 65;                            // [64][65]
-  float* sG = sT + 64 * 65;
+  float* sX = sT + 64 * 65;                            // [64][65] solve scratch
+  float* sG = sX + 64 * 65;
   float* sb = sG + 64;
   __shared__ uint64_t bar[2];
   __shared__ uint32_t tslot;
@@ -104,17 +105,8 @@ __global__ void __launch_bounds__(128) k_tc_wy(Problem p, Work w, TcWork t,
     }
   }
   __syncthreads();
-  // T = (I + A)^-1 by forward substitution, one column per thread
-  if (tid < 64) {
-    const int n = tid;
-    for (int rr = 0; rr < 64; ++rr) {
-      float s = rr == n ? 1.f : 0.f;
-      if (rr > n)
-        for (int j = n; j < rr; ++j) s -= sA[rr * 65 + j] * sT[j * 65 + n];
-      sT[rr * 65 + n] = s;
-    }
-  }
-  __syncthreads();
+  // T = (I + A)^-1 by 16x16 blocks
+  unit_lower_inverse64(sA, sT, sX, tid);
   // bf16 operand tiles TX[i][j] = T[i][j] beta_j e^{G_j}, TY[i][j] = T[i][j] beta_j
   for (int idx = tid; idx < 64 * 8; idx += 128) {
     const int i = idx / 8, jc = idx % 8;
@@ -268,16 +260,17 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
   for (int j = 0; j < 8; ++j) st_chunk_f(sS, v, half * 8 + j, TILE128, &S[8 * j]);
   auto issue = [&](int c) {
     const int gc = sq.x + c, buf = c & 1;
-    const int4 e = w.chunk_tab[gc];
+    const int tok = sq.z + 64 * c;  // chunks of a sequence are consecutive, 64 tokens apart
     unsigned char* b = sm + ScanSmem::BUF + buf * ScanSmem::BUF_BYTES;
     const int row = (gc * p.HV + hv) * D;
     mbar_expect_tx(&barT[buf], 3 * TILE128);
     tma_load_3d(b, &mWT, 0, row, 0, &barT[buf]);
     tma_load_3d(b + TILE128, &mUtT, 0, row, 0, &barT[buf]);
-    tma_load_3d(b + 2 * TILE128, &mk, 0, hk, e.w, &barT[buf]);
-    tma_load_3d(b + 2 * TILE128 + TILE64, &mk, 64, hk, e.w, &barT[buf]);
+    tma_load_3d(b + 2 * TILE128, &mk, 0, hk, tok, &barT[buf]);
+    tma_load_3d(b + 2 * TILE128 + TILE64, &mk, 64, hk, tok, &barT[buf]);
   };
   if (tid == 0 && sq.y > 0) issue(0);
+  if (tid < 64 && sq.y > 0) sGb[tid] = w.G[((size_t)hv * p.NCmax + sq.x) * 64 + tid];
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
@@ -292,7 +285,8 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
     const uint32_t unit_row = (uint32_t)(gc * p.HV + hv) * D;
     float* sG = sGb + buf * 64;
     if (tid == 0 && c + 1 < sq.y) issue(c + 1);
-    if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
+    float gnext = 0.f;  // G of the next chunk, stored to shared memory at the end of this step
+    if (tid < 64 && c + 1 < sq.y) gnext = w.G[((size_t)hv * p.NCmax + gc + 1) * 64 + tid];
     ok = __syncthreads_and(mbar_wait(&barT[buf], phT[buf], err));
     phT[buf] ^= 1;
     if (tid < 64) sDec[tid] = expf(sG[63] - sG[tid]);
@@ -360,6 +354,7 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
     if (tid == 0) tma_store_wait_read0();  // the h store has finished reading sS
     __syncthreads();
     for (int j = 0; j < 8; ++j) st_chunk_f(sS, v, half * 8 + j, TILE128, &S[8 * j]);
+    if (tid < 64 && c + 1 < sq.y) sGb[(buf ^ 1) * 64 + tid] = gnext;
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
@@ -538,7 +533,7 @@ cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const L
   if (!L.ok) return cudaErrorInvalidValue;
   cudaError_t e;
   const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV);
-  const size_t wy_smem = 1024 + 8 * TILE64 + 2 * 64 * 65 * 4 + 2 * 64 * 4;
+  const size_t wy_smem = 1024 + 8 * TILE64 + 3 * 64 * 65 * 4 + 2 * 64 * 4;
   if ((e = tgo("tc_wy", k_tc_wy, gu, 128, wy_smem, s, p, w, L.t, L.m.k, L.m.v, bwd_prep ? 1 : 0)))
     return e;
   Args a2 = a;

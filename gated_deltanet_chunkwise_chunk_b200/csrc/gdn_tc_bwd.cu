@@ -151,8 +151,8 @@ struct BwdScanSmem {
   static constexpr int K = 4 * TILE128, Q = K + 2 * TILE64, O = Q + 2 * TILE64;
   static constexpr int W = O + 2 * TILE64, UL = W + TILE128;     // W^T, dU_loc^T [128][64]
   static constexpr int ATH = UL + TILE128, ATL = ATH + TILE128;  // -dU^T hi / lo
-  static constexpr int G = ATL + TILE128;                        // 64 floats
-  static constexpr int DEC = G + 256;                            // e^{G_C - G_j}
+  static constexpr int G = ATL + TILE128;                        // 2 x 64 floats
+  static constexpr int DEC = G + 512;                            // e^{G_C - G_j}
   static constexpr int EG = DEC + 256;                           // scale e^{G_i} (0 past L)
   static constexpr int TOTAL = EG + 256;
 };
@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
   unsigned char* sUL = sm + BwdScanSmem::UL;
   unsigned char* sATH = sm + BwdScanSmem::ATH;
   unsigned char* sATL = sm + BwdScanSmem::ATL;
-  float* sG = reinterpret_cast<float*>(sm + BwdScanSmem::G);
+  float* sGb = reinterpret_cast<float*>(sm + BwdScanSmem::G);
   float* sDec = reinterpret_cast<float*>(sm + BwdScanSmem::DEC);
   float* sEG = reinterpret_cast<float*>(sm + BwdScanSmem::EG);
   __shared__ uint64_t barA, barW, barU, barM;
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
   for (int j = 0; j < 8; ++j) st_chunk_split(sSH, sSL, v, half * 8 + j, TILE128, &S[8 * j]);
   auto row_of = [&](int c) { return ((sq.x + c) * p.HV + hv) * D; };
   auto issue_A = [&](int c) {  // K, Q, dO of chunk c
-    const int tok = w.chunk_tab[sq.x + c].w;
+    const int tok = sq.z + 64 * c;
     mbar_expect_tx(&barA, 6 * TILE64);
     tma_load_3d(sK, &mk, 0, hk, tok, &barA);
     tma_load_3d(sK + TILE64, &mk, 64, hk, tok, &barA);
@@ -226,6 +226,7 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     issue_W(sq.y - 1);
     issue_U(sq.y - 1);
   }
+  if (tid < 64 && sq.y > 0) sGb[tid] = w.G[((size_t)hv * p.NCmax + sq.x + sq.y - 1) * 64 + tid];
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
@@ -237,9 +238,11 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
   for (int idx = 0; idx < sq.y && ok; ++idx) {
     const int c = sq.y - 1 - idx, gc = sq.x + c;
     const bool more = idx + 1 < sq.y;
-    const int L = w.chunk_tab[gc].z;
+    const int L = min(64, sq.w - 64 * c);
     const uint32_t unit_row = (uint32_t)row_of(c);
-    if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
+    float* sG = sGb + (idx & 1) * 64;
+    float gnext = 0.f;  // G of the next chunk (c - 1), stored at the end of this step
+    if (tid < 64 && more) gnext = w.G[((size_t)hv * p.NCmax + gc - 1) * 64 + tid];
     ok = __syncthreads_and(mbar_wait(&barA, ph, err));
     if (!ok) break;
     if (tid < 64) {
@@ -342,6 +345,7 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     if (tid == 0) tma_store_wait_read0();  // the dh store has finished reading dS hi
     __syncthreads();
     for (int j = 0; j < 8; ++j) st_chunk_split(sSH, sSL, v, half * 8 + j, TILE128, &S[8 * j]);
+    if (tid < 64 && more) sGb[((idx + 1) & 1) * 64 + tid] = gnext;
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
