@@ -4,7 +4,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config I]
 
 One step = gdn_chunk_fwd + gdn_chunk_bwd (every kernel of the forward and the backward)
-over one batch of the workload, inputs resident in HBM.  The default workload is the
+over one batch of the workload, inputs resident in HBM; the backward reads the chunk
+intermediates that the same step's forward saved in the shared workspace
+(GDN_FLAG_BWD_REUSE_FWD), as a training step keeps forward activations for its backward.  The default workload is the
 Qwen3-Next-shaped layer: B=1, T=32768, H=16 q/k heads, HV=32 value heads, K=V=128, bf16
 q/k/v/o/dO, fp32 gates/beta/states, random initial state and final-state gradient.
 Synthetic seeded inputs (no dataset).  Every step streams ~1 GB of inputs, outputs and
@@ -45,15 +47,16 @@ FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # ----------------------------------------------------------------- algorithmic work
 def kernel_flops_per_token_head(K: int, V: int) -> dict:
     """FLOPs each kernel must do per token per value head (its products; 64-row tiles)."""
-    return {
-        "ffma_wy": 2 * C * K + C * C / 3 + 2 * C * (K + V),
-        "ffma_scan_fwd": 4 * K * V,
-        "ffma_out": 2 * C * K + 2 * C * V + 2 * K * V,
-        "ffma_dvlocal": 2 * C * K + 2 * C * V,
-        "ffma_scan_bwd": 6 * K * V,
-        "ffma_dqkwg": 6 * C * K + 2 * C * V + 6 * K * V,
-        "ffma_wy_bwd": 10 * C * K + 4 * C * V + 4 * C * C,
+    per = {
+        "wy": 2 * C * K + C * C / 3 + 2 * C * (K + V),
+        "scan_fwd": 4 * K * V,
+        "out": 2 * C * K + 2 * C * V + 2 * K * V,
+        "dvlocal": 2 * C * K + 2 * C * V,
+        "scan_bwd": 6 * K * V,
+        "dqkwg": 6 * C * K + 2 * C * V + 6 * K * V,
+        "wy_bwd": 10 * C * K + 4 * C * V + 4 * C * C,
     }
+    return {f"{path}_{k}": v for k, v in per.items() for path in ("ffma", "tc")}
 
 
 def step_flops_per_token_head(K: int, V: int) -> tuple[float, float]:
@@ -223,7 +226,7 @@ def main():
     dims = gdn.make_dims(inp["q"], inp["v"], inp["cu_seqlens"])
     varlen = case.cu_seqlens is not None
     ws = torch.empty(max(gdn.workspace_bytes(dims, varlen, False), gdn.workspace_bytes(dims, varlen, True)),
-                     dtype=torch.uint8, device=dev)
+                     dtype=torch.uint8, device=dev)  # shared by the forward and the backward
     o = torch.empty_like(inp["v"])
     ht = torch.empty((case.N, case.HV, case.K, case.V), dtype=torch.float32, device=dev)
     outs = dict(dq=torch.empty_like(inp["q"]), dk=torch.empty_like(inp["k"]), dv=torch.empty_like(inp["v"]),
@@ -235,8 +238,9 @@ def main():
         gdn.gdn_chunk_fwd(**inp, workspace=ws, out=o, final_state=ht)
 
     def step():
+        # the backward reads the chunk intermediates this step's forward left in `ws`
         fwd()
-        gdn.gdn_chunk_bwd(**inp, d_o=dO, dht=dht, workspace=ws, outs=outs)
+        gdn.gdn_chunk_bwd(**inp, d_o=dO, dht=dht, workspace=ws, outs=outs, reuse_forward=True)
 
     stream = torch.cuda.current_stream()
 
@@ -396,7 +400,7 @@ def e2e_measure(gdn, case, dev, ws, nsteps: int, dist) -> dict:
                                      "cu_seqlens", "initial_state")}
         gdn.gdn_chunk_fwd(**fw, workspace=ws, out=o, final_state=ht)
         gdn.gdn_chunk_bwd(**fw, d_o=dev_in["d_o"], dht=dev_in["dht"], workspace=ws, outs=outs,
-                          want_param_grads=False)
+                          want_param_grads=False, reuse_forward=True)
         for k, v in dict(o=o, ht=ht, **outs).items():
             host_out[k].copy_(v, non_blocking=True)
 

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(6)
 GDN_DTYPE_FP32, GDN_DTYPE_BF16 = 0, 1
+GDN_FLAG_BWD_REUSE_FWD = 1
 
 # Every symbol include/gdn.h declares (checked by the tests).
 EXPORTED = ("gdn_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_max_chunks",
@@ -29,7 +30,8 @@ EXPORTED = ("gdn_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_max_ch
 class gdn_dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("T", ctypes.c_int64), ("H", ctypes.c_int64),
                 ("HV", ctypes.c_int64), ("K", ctypes.c_int64), ("V", ctypes.c_int64),
-                ("N", ctypes.c_int64), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+                ("N", ctypes.c_int64), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("flags", ctypes.c_int32)]
 
 
 class GDNError(RuntimeError):
@@ -188,16 +190,24 @@ def noalloc_scratch_bytes() -> int:
 
 def gdn_chunk_bwd(q, k, v, g_raw, A_log, dt_bias, beta, d_o, cu_seqlens=None, initial_state=None,
                   dht=None, scale=0.0, want_dh0=True, want_param_grads=True, workspace=None,
-                  outs=None):
+                  outs=None, reuse_forward=False):
     """Backward of sum(d_o*o) + sum(dht*final_state).  Returns a dict with dq, dk, dv, dg,
-    dbeta and (when asked) dh0, dg_raw, dA_log, ddt_bias."""
+    dbeta and (when asked) dh0, dg_raw, dA_log, ddt_bias.  reuse_forward=True passes
+    GDN_FLAG_BWD_REUSE_FWD: `workspace` must be the one the matching gdn_chunk_fwd call used
+    (sized for the backward) with inputs unchanged since."""
     Nst = _check_inputs(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens, initial_state)
     B, T, H, K = q.shape
     HV, V = v.shape[2], v.shape[3]
     _check("d_o", d_o, q.dtype, (B, T, HV, V), q.device)
     _check("dht", dht, torch.float32, (Nst, HV, K, V), q.device)
     dims = make_dims(q, v, cu_seqlens, scale)
+    if reuse_forward:
+        if workspace is None:
+            raise ValueError("reuse_forward needs the forward's workspace")
+        dims.flags = GDN_FLAG_BWD_REUSE_FWD
     ws = _workspace(dims, cu_seqlens is not None, True, workspace, q.device)
+    if reuse_forward and ws is not workspace:
+        raise ValueError("the forward's workspace is smaller than the backward needs")
     dev = q.device
     if outs is None:
         outs = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),

@@ -80,12 +80,14 @@ Plan make_plan(const gdn_dims& d, bool varlen, int pass) {
       pl.tmp = take(NC * HV * CH * 128 * f);
     }
   } else {
+    // the tcgen05 region starts at the same offset for both passes, so a backward can read
+    // what the forward left in the same workspace
+    pl.tc = take(tc_workspace_bytes(d, NC, pass));
     if (pass == 1) {  // fp32 per-value-head dq/dk shares and dG, read by the final assembly
       pl.dqp = take(NC * HV * CH * K * f);
       pl.dkp = take(NC * HV * CH * K * f);
       pl.dG = take(HV * NC * CH * f);
     }
-    pl.tc = take(tc_workspace_bytes(d, NC, pass));
   }
   pl.total = o;
   return pl;
@@ -248,7 +250,8 @@ int gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v
   if (e != cudaSuccess) return cuda_status(e);
   const bool bf16 = d->dtype == GDN_DTYPE_BF16;
   if (bf16 && tc_bwd_supported(*d)) {
-    e = tc_backward(p, a, w, static_cast<char*>(workspace) + pl.tc, s);
+    e = tc_backward(p, a, w, static_cast<char*>(workspace) + pl.tc,
+                    (d->flags & GDN_FLAG_BWD_REUSE_FWD) != 0, s);
     if (e != cudaSuccess) return cuda_status(e);
   } else {
     e = ffma_forward(p, a, w, bf16, true, s);

@@ -534,7 +534,7 @@ cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const L
   cudaError_t e;
   const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV);
   const size_t wy_smem = 1024 + 8 * TILE64 + 3 * 64 * 65 * 4 + 2 * 64 * 4;
-  if ((e = tgo("tc_wy", k_tc_wy, gu, 128, wy_smem, s, p, w, L.t, L.m.k, L.m.v, bwd_prep ? 1 : 0)))
+  if ((e = tgo("tc_wy", k_tc_wy, gu, 128, wy_smem, s, p, w, L.t, L.m.k, L.m.v, 1)))
     return e;
   Args a2 = a;
   if ((e = tgo("tc_scan_fwd", k_tc_scan_fwd, gs, 256, (size_t)1024 + ScanSmem::TOTAL, s, p, a2, w,
@@ -570,10 +570,12 @@ cudaError_t tc_forward(const Problem& p, const Args& a, const Work& w, void* tc_
   return forward_impl(p, a, w, L, false, s);
 }
 
-cudaError_t tc_backward(const Problem& p, const Args& a, const Work& w, void* tc_ws, cudaStream_t s) {
+cudaError_t tc_backward(const Problem& p, const Args& a, const Work& w, void* tc_ws, bool reuse_fwd,
+                        cudaStream_t s) {
   Launch L = setup(p, a, tc_ws, 1);
-  cudaError_t e = forward_impl(p, a, w, L, true, s);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (!reuse_fwd && (e = forward_impl(p, a, w, L, true, s)) != cudaSuccess) return e;
+  if (!L.ok) return cudaErrorInvalidValue;
   if ((e = tc_backward_kernels(p, a, w, L.t, L.m, s)) != cudaSuccess) return e;
   return launch_bwd_tokens(p, a, w, true, s);
 }

@@ -15,7 +15,8 @@ bool tc_bwd_supported(const gdn_dims& d);
 // Bytes of the tcgen05 path's own workspace region for NC chunks.
 size_t tc_workspace_bytes(const gdn_dims& d, size_t NC, int pass);
 cudaError_t tc_forward(const Problem& p, const Args& a, const Work& w, void* tc_ws, cudaStream_t s);
+// reuse_fwd: the tcgen05 region still holds the forward's intermediates for these inputs.
 cudaError_t tc_backward(const Problem& p, const Args& a, const Work& w, void* tc_ws,
-                        cudaStream_t s);
+                        bool reuse_fwd, cudaStream_t s);
 
 }  // namespace gdn

@@ -100,8 +100,8 @@ inline TcWork carve_tc(void* base, size_t NC, size_t HV, int pass) {
   t.UtT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
   t.UT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
   t.h = reinterpret_cast<bf16*>(take(units * D * D * 2));
+  t.Tm = reinterpret_cast<bf16*>(take(units * 2 * 64 * 64 * 2));  // written by every forward
   if (pass == 1) {
-    t.Tm = reinterpret_cast<bf16*>(take(units * 2 * 64 * 64 * 2));
     t.dUlT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
     t.dh = reinterpret_cast<bf16*>(take(units * D * D * 2));
     t.dUT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
@@ -114,8 +114,9 @@ inline TcWork carve_tc(void* base, size_t NC, size_t HV, int pass) {
 inline size_t tc_bytes(size_t NC, size_t HV, int pass) {
   const size_t units = NC * HV;
   size_t o = 3 * align_up(units * D * 64 * 2) + align_up(units * D * D * 2);
+  o += align_up(units * 2 * 64 * 64 * 2);
   if (pass == 1)
-    o += align_up(units * 2 * 64 * 64 * 2) + 3 * align_up(units * D * 64 * 2) +
+    o += 3 * align_up(units * D * 64 * 2) +
          align_up(units * D * D * 2) + align_up(units * 64 * D * 2);
   return o;
 }

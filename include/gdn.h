@@ -70,7 +70,19 @@ typedef struct gdn_dims {
   int64_t N;       /* number of packed sequences when cu_seqlens != NULL; ignored otherwise */
   int32_t dtype;   /* gdn_dtype of q,k,v,o,do,dq,dk,dv; gates, beta and states are fp32 */
   float scale;     /* output scale; 0 selects 1/sqrt(K) */
+  int32_t flags;   /* bitwise OR of gdn_flags (0 = none) */
 } gdn_dims;
+
+typedef enum gdn_flags {
+  /* gdn_chunk_bwd only: `workspace` still holds what gdn_chunk_fwd wrote for the same
+   * dimensions and the same input contents (the caller ran the forward with this workspace
+   * and changed neither since), so the backward uses the forward's saved chunk
+   * intermediates (W, U~, T, v_new, per-chunk states) instead of recomputing them.  The
+   * workspace must be sized for the backward (gdn_workspace_bytes(.., 1) >= the forward's)
+   * and passed to both calls.  Honoured by the bf16 K = V = 128 path; other paths always
+   * recompute, with identical results. */
+  GDN_FLAG_BWD_REUSE_FWD = 1
+} gdn_flags;
 
 /* Bytes of workspace needed by gdn_chunk_fwd (pass = 0) or gdn_chunk_bwd (pass = 1) for
  * these dimensions, or 0 if the dimensions are invalid.  With cu_seqlens the bound uses
@@ -85,8 +97,9 @@ int gdn_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const void* v
                   void* o, float* final_state,
                   void* workspace, size_t workspace_bytes, void* stream);
 
-/* Backward of L = sum(do * o) + sum(dht * final_state), recomputing the forward
- * intermediates from the inputs (no saved context).  dht NULL = zero.  Required outputs:
+/* Backward of L = sum(do * o) + sum(dht * final_state).  By default it recomputes the
+ * forward's chunk intermediates from the inputs (stateless); with GDN_FLAG_BWD_REUSE_FWD
+ * in d->flags it takes them from the workspace the forward filled.  dht NULL = zero.  Required outputs:
  * dq, dk, dv, dg, dbeta.  Optional (NULL = skipped): dh0, dg_raw, dA_log, ddt_bias. */
 int gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v,
                   const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,

@@ -169,6 +169,29 @@ def test_param_grad_reductions_match_gpu_dg():
         assert (err2 <= 1e-5 * np.abs(terms2).sum(axis=(0, 1)) + 1e-6).all(), err2
 
 
+@pytest.mark.parametrize("lengths", [None, [300, 1, 517, 64, 129]])
+def test_backward_reusing_forward_workspace(lengths):
+    """GDN_FLAG_BWD_REUSE_FWD: the backward that reads the forward's saved intermediates from
+    the shared workspace equals the recomputing backward bit for bit, and the oracle."""
+    import gated_deltanet_chunkwise_chunk_b200 as gdn
+    case = synth.make_case(B=1 if lengths else 2, T=700, H=2, HV=4, K=128, V=128, dtype="bf16",
+                           seed=23, lengths=lengths, h0=True, dht=True, name="reuse_fwd")
+    d = lambda x: None if x is None else x.cuda()
+    args = dict(q=d(case.q), k=d(case.k), v=d(case.v), g_raw=d(case.a), A_log=d(case.A_log),
+                dt_bias=d(case.dt_bias), beta=d(case.beta), cu_seqlens=d(case.cu_seqlens),
+                initial_state=d(case.h0))
+    dims = gdn.make_dims(args["q"], args["v"], args["cu_seqlens"])
+    ws = torch.empty(gdn.workspace_bytes(dims, lengths is not None, True), dtype=torch.uint8, device="cuda")
+    o, ht = gdn.gdn_chunk_fwd(**args, workspace=ws)
+    g1 = gdn.gdn_chunk_bwd(**args, d_o=d(case.dO), dht=d(case.dht), workspace=ws, reuse_forward=True)
+    g2 = gdn.gdn_chunk_bwd(**args, d_o=d(case.dO), dht=d(case.dht))
+    torch.cuda.synchronize()
+    for key in g1:
+        assert torch.equal(g1[key], g2[key]), key
+    gpu = {k: v.double().cpu().numpy() for k, v in dict(o=o, ht=ht, **g1).items()}
+    _assert_parity(case, gpu=gpu)
+
+
 def test_run_to_run_bitwise_reproducible():
     case = synth.make_case(B=1, T=700, H=2, HV=4, K=128, V=128, dtype="bf16", seed=18, h0=True,
                            dht=True)
