@@ -19,11 +19,23 @@ using namespace tcx;
 namespace {
 
 // ======================================================================================
-// WY representation.  One CTA (128 threads) per (chunk, value head).
-//   KK^T (M=64) -> A, T = (I+A)^-1 (fp32, one column per thread) ->
+// WY representation.  One CTA (256 threads) per (chunk, value head).
+//   KK^T (M=64) -> A, T = (I+A)^-1 (fp32, 16x16 blocks) ->
 //   W^T = K^T (T diag(beta e^G))^T,  U~^T = V^T (T diag(beta))^T   (M=128, N=64, K=64)
+// The fp32 A and the solve's scratch share shared memory with the bf16 T tiles written
+// after the solve, so two CTAs fit on an SM.
 // ======================================================================================
-__global__ void __launch_bounds__(128) k_tc_wy(Problem p, Work w, TcWork t,
+struct WySmem {
+  static constexpr int K = 0, V = 2 * TILE64;
+  static constexpr int R1 = 4 * TILE64;                  // {A, X} during the solve, then TX/TY
+  static constexpr int TX = R1, TY = R1 + TILE64, TXL = R1 + 2 * TILE64, TYL = R1 + 3 * TILE64;
+  static constexpr int A = R1, X = R1 + 64 * 65 * 4;
+  static constexpr int T = R1 + 34 * 1024;              // fp32 [64][65]
+  static constexpr int G = T + 64 * 65 * 4, B = G + 256, EG = B + 256;
+  static constexpr int TOTAL = EG + 256;
+};
+
+__global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
                                                const __grid_constant__ CUtensorMap mk,
                                                const __grid_constant__ CUtensorMap mv, int store_T) {
   if (failed(w)) return;
@@ -31,19 +43,21 @@ __global__ void __launch_bounds__(128) k_tc_wy(Problem p, Work w, TcWork t,
   const int4 e = w.chunk_tab[gc];
   if (e.x < 0) return;
   const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int sub = 32 * (warp & 3), half = warp >> 2;
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
-  unsigned char* sK = sm;                    // [64][128] bf16, 2 blocks
-  unsigned char* sV = sK + 2 * TILE64;       // [64][128]
-  unsigned char* sTX = sV + 2 * TILE64;      // [64][64]  T diag(beta e^G), hi part
-  unsigned char* sTY = sTX + TILE64;         // [64][64]  T diag(beta), hi part
-  unsigned char* sTXl = sTY + TILE64;        // lo parts
-  unsigned char* sTYl = sTXl + TILE64;
-  float* sA = reinterpret_cast<float*>(sTYl + TILE64);  // [64][65]
-  float* sT = sA + 64 * 65;                            // [64][65]
-  float* sX = sT + 64 * 65;                            // [64][65] solve scratch
-  float* sG = sX + 64 * 65;
-  float* sb = sG + 64;
+  unsigned char* sK = sm + WySmem::K;
+  unsigned char* sV = sm + WySmem::V;
+  unsigned char* sTX = sm + WySmem::TX;
+  unsigned char* sTY = sm + WySmem::TY;
+  unsigned char* sTXl = sm + WySmem::TXL;
+  unsigned char* sTYl = sm + WySmem::TYL;
+  float* sA = reinterpret_cast<float*>(sm + WySmem::A);
+  float* sX = reinterpret_cast<float*>(sm + WySmem::X);
+  float* sT = reinterpret_cast<float*>(sm + WySmem::T);
+  float* sG = reinterpret_cast<float*>(sm + WySmem::G);
+  float* sb = reinterpret_cast<float*>(sm + WySmem::B);
+  float* sEG = reinterpret_cast<float*>(sm + WySmem::EG);   // beta_j e^{G_j}
   __shared__ uint64_t bar[2];
   __shared__ uint32_t tslot;
   int* err = w.status;
@@ -66,8 +80,10 @@ __global__ void __launch_bounds__(128) k_tc_wy(Problem p, Work w, TcWork t,
   }
   if (tid < 64) {
     const size_t o = ((size_t)hv * p.NCmax + gc) * 64 + tid;
-    sG[tid] = w.G[o];
-    sb[tid] = w.beta_p[o];
+    const float g = w.G[o], bb = w.beta_p[o];
+    sG[tid] = g;
+    sb[tid] = bb;
+    sEG[tid] = bb * expf(g);
   }
   tc_fence_before();
   __syncthreads();
@@ -75,8 +91,8 @@ __global__ void __launch_bounds__(128) k_tc_wy(Problem p, Work w, TcWork t,
   const uint32_t tb = tslot;
   bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
   if (L < 64) {
-    zero_tail_rows(sK, L, tid, 128);
-    zero_tail_rows(sV, L, tid, 128);
+    zero_tail_rows(sK, L, tid, 256);
+    zero_tail_rows(sV, L, tid, 256);
   }
   fence_proxy_async();
   __syncthreads();
@@ -91,52 +107,48 @@ __global__ void __launch_bounds__(128) k_tc_wy(Problem p, Work w, TcWork t,
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
   tc_fence_after();
   if (ok) {
-    // M=64 accumulator: row 16*warp + lane (lanes 0..15) of the warp's sub-partition
-    float v[16];
-    const int r = warp * 16 + lane;
-    for (int c = 0; c < 64; c += 16) {
-      tmem_ld16(taddr(tb, warp * 32, c), v);
-      tmem_wait_ld();
-      if (lane < 16)
-        for (int i = 0; i < 16; ++i) {
-          const int cc = c + i;
-          sA[r * 65 + cc] = cc < r ? sb[r] * v[i] * expf(sG[r] - sG[cc]) : 0.f;
-        }
+    // M=64 accumulator: row 16*(warp%4) + lane (lanes 0..15); columns [32*half, +32)
+    float v[32];
+    tmem_ld16(taddr(tb, sub, 32 * half), v);
+    tmem_ld16(taddr(tb, sub, 32 * half + 16), v + 16);
+    tmem_wait_ld();
+    if (lane < 16) {
+      const int r = 16 * (warp & 3) + lane;
+      const float br = sb[r], gr = sG[r];
+      for (int i = 0; i < 32; ++i) {
+        const int cc = 32 * half + i;
+        sA[r * 65 + cc] = cc < r ? br * v[i] * expf(gr - sG[cc]) : 0.f;
+      }
     }
   }
   __syncthreads();
-  // T = (I + A)^-1 by 16x16 blocks
-  unit_lower_inverse64(sA, sT, sX, tid);
-  // bf16 operand tiles TX[i][j] = T[i][j] beta_j e^{G_j}, TY[i][j] = T[i][j] beta_j
-  for (int idx = tid; idx < 64 * 8; idx += 128) {
+  unit_lower_inverse64(sA, sT, sX, tid, 256);   // T = (I + A)^-1 (ends with a barrier)
+  // bf16 operand tiles TX[i][j] = T[i][j] beta_j e^{G_j}, TY[i][j] = T[i][j] beta_j (hi + lo)
+  bf16* tbase = t.Tm + ((size_t)gc * p.HV + hv) * 128 * 64;
+  for (int idx = tid; idx < 64 * 8; idx += 256) {
     const int i = idx / 8, jc = idx % 8;
-    float fx[8], fy[8];
+    float fx[8], fy[8], ft[8], fl[8];
     for (int q = 0; q < 8; ++q) {
       const int j = jc * 8 + q;
-      const float tv = sT[i * 65 + j];
-      fy[q] = tv * sb[j];
-      fx[q] = fy[q] * expf(sG[j]);
+      ft[q] = sT[i * 65 + j];
+      fy[q] = ft[q] * sb[j];
+      fx[q] = ft[q] * sEG[j];
+      fl[q] = ft[q] - __bfloat162float(__float2bfloat16_rn(ft[q]));
     }
     st_chunk_split(sTX, sTXl, i, jc, TILE64, fx);
     st_chunk_split(sTY, sTYl, i, jc, TILE64, fy);
     if (store_T) {  // T as a compensated pair: rows [0,64) hi, [64,128) lo of the unit
-      float ft[8], fl[8];
-      for (int q = 0; q < 8; ++q) {
-        ft[q] = sT[i * 65 + jc * 8 + q];
-        fl[q] = ft[q] - __bfloat162float(__float2bfloat16_rn(ft[q]));
-      }
-      bf16* base = t.Tm + ((size_t)gc * p.HV + hv) * 128 * 64;
       uint4 pk;
       pk.x = pack_bf16(ft[0], ft[1]);
       pk.y = pack_bf16(ft[2], ft[3]);
       pk.z = pack_bf16(ft[4], ft[5]);
       pk.w = pack_bf16(ft[6], ft[7]);
-      *reinterpret_cast<uint4*>(base + i * 64 + jc * 8) = pk;
+      *reinterpret_cast<uint4*>(tbase + i * 64 + jc * 8) = pk;
       pk.x = pack_bf16(fl[0], fl[1]);
       pk.y = pack_bf16(fl[2], fl[3]);
       pk.z = pack_bf16(fl[4], fl[5]);
       pk.w = pack_bf16(fl[6], fl[7]);
-      *reinterpret_cast<uint4*>(base + (64 + i) * 64 + jc * 8) = pk;
+      *reinterpret_cast<uint4*>(tbase + (64 + i) * 64 + jc * 8) = pk;
     }
   }
   fence_proxy_async();
@@ -164,30 +176,25 @@ __global__ void __launch_bounds__(128) k_tc_wy(Problem p, Work w, TcWork t,
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
   tc_fence_after();
   if (ok) {
-    // row = feature index (k for W^T, v for U~^T), 64 token columns -> global rows of 128 B
-    const int r = warp * 32 + lane;
+    // row = feature index (k for W^T, v for U~^T); this thread's 32 token columns
+    const int r = sub + lane;
     const size_t unit = (size_t)gc * p.HV + hv;
-    bf16* wrow = t.WT + (unit * D + r) * 64;
-    bf16* urow = t.UtT + (unit * D + r) * 64;
-    float v[16];
-    for (int c = 0; c < 64; c += 16) {
-      tmem_ld16(taddr(tb, warp * 32, 64 + c), v);
-      tmem_wait_ld();
+    bf16* wrow = t.WT + (unit * D + r) * 64 + 32 * half;
+    bf16* urow = t.UtT + (unit * D + r) * 64 + 32 * half;
+    float x[32], y[32];
+    tmem_ld16(taddr(tb, sub, 64 + 32 * half), x);
+    tmem_ld16(taddr(tb, sub, 64 + 32 * half + 16), x + 16);
+    tmem_ld16(taddr(tb, sub, 128 + 32 * half), y);
+    tmem_ld16(taddr(tb, sub, 128 + 32 * half + 16), y + 16);
+    tmem_wait_ld();
+    for (int c = 0; c < 32; c += 8) {
       uint4 a, b;
-      a.x = pack_bf16(v[0], v[1]); a.y = pack_bf16(v[2], v[3]);
-      a.z = pack_bf16(v[4], v[5]); a.w = pack_bf16(v[6], v[7]);
-      b.x = pack_bf16(v[8], v[9]); b.y = pack_bf16(v[10], v[11]);
-      b.z = pack_bf16(v[12], v[13]); b.w = pack_bf16(v[14], v[15]);
+      a.x = pack_bf16(x[c], x[c + 1]); a.y = pack_bf16(x[c + 2], x[c + 3]);
+      a.z = pack_bf16(x[c + 4], x[c + 5]); a.w = pack_bf16(x[c + 6], x[c + 7]);
+      b.x = pack_bf16(y[c], y[c + 1]); b.y = pack_bf16(y[c + 2], y[c + 3]);
+      b.z = pack_bf16(y[c + 4], y[c + 5]); b.w = pack_bf16(y[c + 6], y[c + 7]);
       *reinterpret_cast<uint4*>(wrow + c) = a;
-      *reinterpret_cast<uint4*>(wrow + c + 8) = b;
-      tmem_ld16(taddr(tb, warp * 32, 128 + c), v);
-      tmem_wait_ld();
-      a.x = pack_bf16(v[0], v[1]); a.y = pack_bf16(v[2], v[3]);
-      a.z = pack_bf16(v[4], v[5]); a.w = pack_bf16(v[6], v[7]);
-      b.x = pack_bf16(v[8], v[9]); b.y = pack_bf16(v[10], v[11]);
-      b.z = pack_bf16(v[12], v[13]); b.w = pack_bf16(v[14], v[15]);
-      *reinterpret_cast<uint4*>(urow + c) = a;
-      *reinterpret_cast<uint4*>(urow + c + 8) = b;
+      *reinterpret_cast<uint4*>(urow + c) = b;
     }
   }
   tc_fence_before();
@@ -533,8 +540,7 @@ cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const L
   if (!L.ok) return cudaErrorInvalidValue;
   cudaError_t e;
   const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV);
-  const size_t wy_smem = 1024 + 8 * TILE64 + 3 * 64 * 65 * 4 + 2 * 64 * 4;
-  if ((e = tgo("tc_wy", k_tc_wy, gu, 128, wy_smem, s, p, w, L.t, L.m.k, L.m.v, 1)))
+  if ((e = tgo("tc_wy", k_tc_wy, gu, 256, (size_t)1024 + WySmem::TOTAL, s, p, w, L.t, L.m.k, L.m.v, 1)))
     return e;
   Args a2 = a;
   if ((e = tgo("tc_scan_fwd", k_tc_scan_fwd, gs, 256, (size_t)1024 + ScanSmem::TOTAL, s, p, a2, w,

@@ -172,16 +172,17 @@ __device__ __forceinline__ void st_chunk_split(unsigned char* hi, unsigned char*
 }
 
 // T = (I + A)^-1 for a strictly lower-triangular 64x64 fp32 A (row stride 65) by 16x16
-// blocks, with 128 threads: the four diagonal blocks by forward substitution (one warp per
-// block, one column per lane), then the block sub-diagonals d = 1, 2, 3 as
+// blocks, with nthr >= 128 threads: the four diagonal blocks by forward substitution (warps
+// 0..3, one column per lane), then the block sub-diagonals d = 1, 2, 3 as
 // T[b+d][b] = -T[b+d][b+d] * sum_{k=b}^{b+d-1} A[b+d][k] T[k][b].   sX: [64][65] scratch.
-__device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT, float* sX, int tid) {
+__device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT, float* sX, int tid,
+                                                     int nthr = 128) {
   const int w = tid >> 5, lane = tid & 31;
-  for (int i = tid; i < 64 * 64; i += 128) {  // zero the strictly upper blocks
+  for (int i = tid; i < 64 * 64; i += nthr) {  // zero the strictly upper blocks
     const int r = i >> 6, c = i & 63;
     if ((c >> 4) > (r >> 4)) sT[r * 65 + c] = 0.f;
   }
-  if (lane < 16) {
+  if (w < 4 && lane < 16) {
     const int b0 = 16 * w, c = lane;
     float col[16];
 #pragma unroll
@@ -197,7 +198,7 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT,
   __syncthreads();
   for (int d = 1; d < 4; ++d) {
     const int nblk = 4 - d;
-    for (int e = tid; e < nblk * 256; e += 128) {
+    for (int e = tid; e < nblk * 256; e += nthr) {
       const int b = e >> 8, r = (e >> 4) & 15, c = e & 15;
       const int R = 16 * (b + d) + r, Cc = 16 * b + c;
       float s = 0.f;
@@ -205,7 +206,7 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT,
       sX[R * 65 + Cc] = s;
     }
     __syncthreads();
-    for (int e = tid; e < nblk * 256; e += 128) {
+    for (int e = tid; e < nblk * 256; e += nthr) {
       const int b = e >> 8, r = (e >> 4) & 15, c = e & 15;
       const int R = 16 * (b + d) + r, Cc = 16 * b + c, D0 = 16 * (b + d);
       float s = 0.f;
