@@ -362,8 +362,8 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
 // ======================================================================================
 // dqkwg.  One CTA (256 threads) per (chunk, value head).  TMEM columns:
 //   [0,64) Q K^T   [64,128) dO U^T   [128,256) dO S -> dQ   [256,384) U dS' -> dK   [384,512) dU S
-// M=64 accumulators: row i in lanes 0..15 of sub-partition i/16; the two warps sharing a
-// sub-partition split the columns.
+// M=64 accumulators are read with 16-lane loads: warp w covers rows 16(w%4) .. +15, thread t
+// rows r0 = 16(w%4) + t/4 and r0 + 8, and the two warps of a sub-partition split columns.
 // ======================================================================================
 struct DqkSmem {
   static constexpr int Q = 0, K = 2 * TILE64, O = 4 * TILE64, UT = 6 * TILE64,
@@ -386,19 +386,21 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
                                                   const __grid_constant__ CUtensorMap mdUT,
                                                   const __grid_constant__ CUtensorMap mdUTl,
                                                   const __grid_constant__ CUtensorMap mh,
-                                                  const __grid_constant__ CUtensorMap mdh) {
+                                                  const __grid_constant__ CUtensorMap mdh,
+                                                  const __grid_constant__ CUtensorMap mdW) {
   if (failed(w)) return;
   const int gc = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
   const int4 e = w.chunk_tab[gc];
   if (e.x < 0) return;
   const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int i = 16 * (warp & 3) + lane, half = warp >> 2, sub = 32 * (warp & 3);
+  const int half = warp >> 2, sub = 32 * (warp & 3);
+  const int r0 = 16 * (warp & 3) + lane / 4, r1 = r0 + 8, cq = 2 * (lane & 3);
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
   unsigned char* sQ = sm + DqkSmem::Q;
   unsigned char* sK = sm + DqkSmem::K;
   unsigned char* sO = sm + DqkSmem::O;
-  unsigned char* sUT = sm + DqkSmem::UT;
+  unsigned char* sUT = sm + DqkSmem::UT;     // later: dW staging [64][128]
   unsigned char* sdUT = sm + DqkSmem::DUT;
   unsigned char* sH = sm + DqkSmem::H;
   unsigned char* sdH = sm + DqkSmem::DH;
@@ -455,7 +457,7 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
   __syncthreads();
   if (ok && tid == 0) {
     const uint32_t q = smem_u32(sQ), k = smem_u32(sK), o = smem_u32(sO), ut = smem_u32(sUT),
-                   dut = smem_u32(sdUT), h = smem_u32(sH), dh = smem_u32(sdH);
+                   dut = smem_u32(sdUT), dutl = smem_u32(sdUTl), h = smem_u32(sH), dh = smem_u32(sdH);
     for (int s = 0; s < 8; ++s) {
       const uint32_t acc = s > 0;
       mma_bf16(taddr(tb, 0, 0), desc_kmajor(q, s, TILE64), desc_kmajor(k, s, TILE64),
@@ -469,7 +471,6 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
       mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dut, s, TILE128), desc_mnmajor(h, s, TILE128),
                idesc_bf16(64, 128, true, true), acc);
     }
-    const uint32_t dutl = smem_u32(sdUTl);
     for (int s = 0; s < 8; ++s)
       mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dutl, s, TILE128), desc_mnmajor(h, s, TILE128),
                idesc_bf16(64, 128, true, true), 1);
@@ -477,82 +478,80 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
   tc_fence_after();
-  const float Gi = sG[i & 63], GC = sG[63];
+  const float G0 = sG[r0], G1 = sG[r1], GC = sG[63];
   if (ok) {
-    // P, dP for columns [32*half, 32*half+32)
-    float qk[32], dp[32];
-    tmem_ld16(taddr(tb, sub, 32 * half), qk);
-    tmem_ld16(taddr(tb, sub, 32 * half + 16), qk + 16);
-    tmem_ld16(taddr(tb, sub, 64 + 32 * half), dp);
-    tmem_ld16(taddr(tb, sub, 64 + 32 * half + 16), dp + 16);
+    // P = QK * Gam, dP = scale dO U^T (lower incl. diagonal), columns [32*half, +32)
+    float qk[16], dp[16];
+    tmem_ld16dp_x4(taddr(tb, sub, 32 * half), qk);
+    tmem_ld16dp_x4(taddr(tb, sub, 64 + 32 * half), dp);
     tmem_wait_ld();
-    if (lane < 16) {
-      float rs = 0.f, pg[8];
-      for (int jj = 0; jj < 32; ++jj) {
-        const int j = 32 * half + jj;
-        float dpp = 0.f, g = 0.f;
-        if (j <= i) {
-          const float gam = expf(Gi - sG[j]);
-          const float dpv = p.scale * dp[jj];
-          dpp = dpv * qk[jj] * gam;
-          g = dpv * gam;
+    float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = 32 * half + 8 * j + cq;
+      float g[4], m[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int row = q < 2 ? r0 : r1, col = c + (q & 1);
+        const float Gi = q < 2 ? G0 : G1;
+        float dpp = 0.f, gg = 0.f;
+        if (col <= row) {
+          const float gam = __expf(Gi - sG[col]);
+          const float dpv = p.scale * dp[4 * j + q];
+          dpp = dpv * qk[4 * j + q] * gam;
+          gg = dpv * gam;
         }
-        sM[i * 65 + j] = dpp;
-        rs += dpp;
-        pg[jj & 7] = g;
-        if ((jj & 7) == 7) st_chunk_split(sPG, sPGl, i, (32 * half + jj) / 8, TILE64, pg);
+        g[q] = gg;
+        m[q] = dpp;
       }
-      sRow[(0 * 2 + half) * 64 + i] = rs;
+      sM[r0 * 65 + c] = m[0];
+      sM[r0 * 65 + c + 1] = m[1];
+      sM[r1 * 65 + c] = m[2];
+      sM[r1 * 65 + c + 1] = m[3];
+      rs0 += m[0] + m[1];
+      rs1 += m[2] + m[3];
+      st_pair_split(sPG, sPGl, r0, c, TILE64, g[0], g[1]);
+      st_pair_split(sPG, sPGl, r1, c, TILE64, g[2], g[3]);
     }
-    // dQ part 1: scale e^{G_i} dO S  -> back into TMEM; dG2 = sum_k (.) Q[i,k]
-    float x2 = 0.f;
-    const float egi = p.scale * expf(Gi);
-    for (int cc = 0; cc < 64; cc += 16) {
-      float x[16], qv[16];
-      tmem_ld16(taddr(tb, sub, 128 + 64 * half + cc), x);
-      tmem_wait_ld();
-      ld_chunk_f(sQ, i & 63, (64 * half + cc) / 8, TILE64, qv);
-      ld_chunk_f(sQ, i & 63, (64 * half + cc) / 8 + 1, TILE64, qv + 8);
-      for (int q = 0; q < 16; ++q) {
-        x[q] *= egi;
-        x2 += x[q] * qv[q];
-      }
-      tmem_st16(taddr(tb, sub, 128 + 64 * half + cc), x);
+    rs0 = quad_sum(rs0);
+    rs1 = quad_sum(rs1);
+    // dQ part 1: scale e^{G_i} dO S back into TMEM; dG2 = sum_k (.) Q[i,k]
+    float x[32], y[32], z[32];
+    tmem_ld16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
+    tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), y);
+    tmem_ld16dp_x8(taddr(tb, sub, 384 + 64 * half), z);
+    tmem_wait_ld();
+    const float e0 = p.scale * __expf(G0), e1 = p.scale * __expf(G1);
+    const float D0 = __expf(GC - G0), D1 = __expf(GC - G1);
+    float x0 = 0.f, x1 = 0.f, y0 = 0.f, y1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = 64 * half + 8 * j + cq;
+      const float2 q0 = ld_pair(sQ, r0, c, TILE64), q1 = ld_pair(sQ, r1, c, TILE64);
+      const float2 k0 = ld_pair(sK, r0, c, TILE64), k1 = ld_pair(sK, r1, c, TILE64);
+      x[4 * j] *= e0; x[4 * j + 1] *= e0; x[4 * j + 2] *= e1; x[4 * j + 3] *= e1;
+      x0 += x[4 * j] * q0.x + x[4 * j + 1] * q0.y;
+      x1 += x[4 * j + 2] * q1.x + x[4 * j + 3] * q1.y;
+      y[4 * j] *= D0; y[4 * j + 1] *= D0; y[4 * j + 2] *= D1; y[4 * j + 3] *= D1;
+      y0 += y[4 * j] * k0.x + y[4 * j + 1] * k0.y;
+      y1 += y[4 * j + 2] * k1.x + y[4 * j + 3] * k1.y;
+      // dW = -dU S, staged as a bf16 [64][128] tile in the (now free) U^T buffer
+      st_pair(sUT, r0, c, TILE64, -z[4 * j], -z[4 * j + 1]);
+      st_pair(sUT, r1, c, TILE64, -z[4 * j + 2], -z[4 * j + 3]);
     }
-    // dK part 1: D_i U dS' -> back into TMEM; r_i = sum_k (.) K[i,k]
-    float r = 0.f;
-    const float Di = expf(GC - Gi);
-    for (int cc = 0; cc < 64; cc += 16) {
-      float y[16], kv[16];
-      tmem_ld16(taddr(tb, sub, 256 + 64 * half + cc), y);
-      tmem_wait_ld();
-      ld_chunk_f(sK, i & 63, (64 * half + cc) / 8, TILE64, kv);
-      ld_chunk_f(sK, i & 63, (64 * half + cc) / 8 + 1, TILE64, kv + 8);
-      for (int q = 0; q < 16; ++q) {
-        y[q] *= Di;
-        r += y[q] * kv[q];
-      }
-      tmem_st16(taddr(tb, sub, 256 + 64 * half + cc), y);
-    }
-    // dW = -dU S
-    bf16* dwrow = t.dW + (unit * 64 + (i & 63)) * D + 64 * half;
-    for (int cc = 0; cc < 64; cc += 16) {
-      float z[16];
-      tmem_ld16(taddr(tb, sub, 384 + 64 * half + cc), z);
-      tmem_wait_ld();
-      if (lane < 16) {
-        uint4 a0, a1;
-        a0.x = pack_bf16(-z[0], -z[1]); a0.y = pack_bf16(-z[2], -z[3]);
-        a0.z = pack_bf16(-z[4], -z[5]); a0.w = pack_bf16(-z[6], -z[7]);
-        a1.x = pack_bf16(-z[8], -z[9]); a1.y = pack_bf16(-z[10], -z[11]);
-        a1.z = pack_bf16(-z[12], -z[13]); a1.w = pack_bf16(-z[14], -z[15]);
-        *reinterpret_cast<uint4*>(dwrow + cc) = a0;
-        *reinterpret_cast<uint4*>(dwrow + cc + 8) = a1;
-      }
-    }
-    if (lane < 16) {
-      sRow[(1 * 2 + half) * 64 + i] = x2;
-      sRow[(2 * 2 + half) * 64 + i] = r;
+    tmem_st16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
+    tmem_st16dp_x8(taddr(tb, sub, 256 + 64 * half), y);
+    x0 = quad_sum(x0);
+    x1 = quad_sum(x1);
+    y0 = quad_sum(y0);
+    y1 = quad_sum(y1);
+    if ((lane & 3) == 0) {
+      sRow[(0 * 2 + half) * 64 + r0] = rs0;
+      sRow[(0 * 2 + half) * 64 + r1] = rs1;
+      sRow[(1 * 2 + half) * 64 + r0] = x0;
+      sRow[(1 * 2 + half) * 64 + r1] = x1;
+      sRow[(2 * 2 + half) * 64 + r0] = y0;  // D_i sum_k Y K (y already carries D_i)
+      sRow[(2 * 2 + half) * 64 + r1] = y1;
     }
     tmem_wait_st();
   }
@@ -572,6 +571,9 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
   __syncthreads();
   tc_fence_after();
   if (ok && tid == 0) {
+    tma_store_3d(&mdW, sUT, 0, (int)unit * 64, 0);
+    tma_store_3d(&mdW, sUT + TILE64, 64, (int)unit * 64, 0);
+    tma_store_commit();
     const uint32_t k = smem_u32(sK), q = smem_u32(sQ);
     for (int part = 0; part < 2; ++part) {
       const uint32_t pg = smem_u32(part ? sPGl : sPG);
@@ -595,27 +597,28 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
       float d8 = 0.f, rsum = 0.f;
       for (int q = 0; q < 8; ++q) d8 += sRed[q];
       for (int q = 0; q < 64; ++q) rsum += sRow[4 * 64 + q] + sRow[5 * 64 + q];
-      g += expf(GC) * d8 + rsum;
+      g += __expf(GC) * d8 + rsum;
     }
     w.dG[((size_t)hv * p.NCmax + gc) * 64 + j] = g;
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
   tc_fence_after();
   if (ok) {
-    float* dq = w.dqp + (unit * 64 + (i & 63)) * D + 64 * half;
-    float* dk = w.dkp + (unit * 64 + (i & 63)) * D + 64 * half;
-    for (int cc = 0; cc < 64; cc += 16) {
-      float x[16], y[16];
-      tmem_ld16(taddr(tb, sub, 128 + 64 * half + cc), x);
-      tmem_ld16(taddr(tb, sub, 256 + 64 * half + cc), y);
-      tmem_wait_ld();
-      if (lane < 16)
-        for (int q = 0; q < 16; q += 4) {
-          *reinterpret_cast<float4*>(dq + cc + q) = make_float4(x[q], x[q + 1], x[q + 2], x[q + 3]);
-          *reinterpret_cast<float4*>(dk + cc + q) = make_float4(y[q], y[q + 1], y[q + 2], y[q + 3]);
-        }
+    float x[32], y[32];
+    tmem_ld16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
+    tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), y);
+    tmem_wait_ld();
+    float* dq0 = w.dqp + (unit * 64 + r0) * D + 64 * half + cq;
+    float* dk0 = w.dkp + (unit * 64 + r0) * D + 64 * half + cq;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      *reinterpret_cast<float2*>(dq0 + 8 * j) = make_float2(x[4 * j], x[4 * j + 1]);
+      *reinterpret_cast<float2*>(dq0 + 8 * D + 8 * j) = make_float2(x[4 * j + 2], x[4 * j + 3]);
+      *reinterpret_cast<float2*>(dk0 + 8 * j) = make_float2(y[4 * j], y[4 * j + 1]);
+      *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j) = make_float2(y[4 * j + 2], y[4 * j + 3]);
     }
   }
+  if (tid == 0) tma_store_wait0();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tb, 512);
@@ -625,6 +628,7 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
 // WY backward.  One CTA (256 threads) per (chunk, value head).  TMEM columns:
 //   [0,64) dU V^T, then T^T dT   [64,128) dW K^T, then Z T^T   [128,192) K K^T
 //   [256,384) T^T dW -> dk       [384,512) T^T dU
+// 16-lane TMEM loads as in dqkwg: thread rows r0 = 16(w%4) + t/4 and r0 + 8.
 // ======================================================================================
 struct WyBwdSmem {
   static constexpr int K = 0, V = 2 * TILE64, T = 4 * TILE64, TL = 5 * TILE64, DW = 6 * TILE64,
@@ -632,8 +636,8 @@ struct WyBwdSmem {
                        Z = DTL + TILE64, ZL = Z + TILE64, AS = ZL + TILE64, ASL = AS + TILE64,
                        DUTL = ASL + TILE64, F = DUTL + TILE128;
   static constexpr int KKG = F, AA = KKG + 64 * 65 * 4;        // fp32 [64][65] each
-  static constexpr int G = AA + 64 * 65 * 4, B = G + 256, ROW = B + 256;  // ROW [4][2][64]
-  static constexpr int TOTAL = ROW + 4 * 2 * 64 * 4;
+  static constexpr int G = AA + 64 * 65 * 4, B = G + 256, EG = B + 256, ROW = EG + 256;
+  static constexpr int TOTAL = ROW + 4 * 2 * 64 * 4;            // ROW [4][2][64]
   static constexpr int LOAD_BYTES = 8 * TILE64 + 2 * TILE128;
 };
 
@@ -649,8 +653,8 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   const int4 e = w.chunk_tab[gc];
   if (e.x < 0) return;
   const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int i = 16 * (warp & 3) + lane, half = warp >> 2, sub = 32 * (warp & 3);
-  const int ii = i & 63;
+  const int half = warp >> 2, sub = 32 * (warp & 3);
+  const int r0 = 16 * (warp & 3) + lane / 4, r1 = r0 + 8, cq = 2 * (lane & 3);
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
   unsigned char* sK = sm + WyBwdSmem::K;
@@ -670,6 +674,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   float* sAA = reinterpret_cast<float*>(sm + WyBwdSmem::AA);
   float* sG = reinterpret_cast<float*>(sm + WyBwdSmem::G);
   float* sb = reinterpret_cast<float*>(sm + WyBwdSmem::B);
+  float* sEG = reinterpret_cast<float*>(sm + WyBwdSmem::EG);   // e^{G_j}
   float* sRow = reinterpret_cast<float*>(sm + WyBwdSmem::ROW);  // [kind][half][64]
   __shared__ uint64_t bar[2];
   __shared__ uint32_t tslot;
@@ -700,8 +705,10 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   }
   if (tid < 64) {
     const size_t o = ((size_t)hv * p.NCmax + gc) * 64 + tid;
-    sG[tid] = w.G[o];
+    const float g = w.G[o];
+    sG[tid] = g;
     sb[tid] = w.beta_p[o];
+    sEG[tid] = __expf(g);
   }
   tc_fence_before();
   __syncthreads();
@@ -745,62 +752,60 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
   tc_fence_after();
-  const float Gi = sG[ii], bi = sb[ii], egi = expf(Gi);
+  const float G0 = sG[r0], G1 = sG[r1], b0 = sb[r0], b1 = sb[r1];
   if (ok) {
-    float r1[32], r2[32], kk[32];
-    tmem_ld16(taddr(tb, sub, 32 * half), r1);
-    tmem_ld16(taddr(tb, sub, 32 * half + 16), r1 + 16);
-    tmem_ld16(taddr(tb, sub, 64 + 32 * half), r2);
-    tmem_ld16(taddr(tb, sub, 64 + 32 * half + 16), r2 + 16);
-    tmem_ld16(taddr(tb, sub, 128 + 32 * half), kk);
-    tmem_ld16(taddr(tb, sub, 128 + 32 * half + 16), kk + 16);
+    float r1v[16], r2v[16], kk[16];
+    tmem_ld16dp_x4(taddr(tb, sub, 32 * half), r1v);
+    tmem_ld16dp_x4(taddr(tb, sub, 64 + 32 * half), r2v);
+    tmem_ld16dp_x4(taddr(tb, sub, 128 + 32 * half), kk);
     tmem_wait_ld();
-    if (lane < 16) {
-      float f[8];
-      for (int jj = 0; jj < 32; ++jj) {
-        const int j = 32 * half + jj;
-        f[jj & 7] = sb[j] * (r1[jj] + expf(sG[j]) * r2[jj]);
-        if ((jj & 7) == 7) st_chunk_split(sdT, sdTl, ii, j / 8, TILE64, f);
-        sKKG[ii * 65 + j] = j < ii ? expf(Gi - sG[j]) * kk[jj] : 0.f;
-      }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = 32 * half + 8 * j + cq;
+      const float bc0 = sb[c], bc1 = sb[c + 1], ec0 = sEG[c], ec1 = sEG[c + 1];
+      st_pair_split(sdT, sdTl, r0, c, TILE64, bc0 * (r1v[4 * j] + ec0 * r2v[4 * j]),
+                    bc1 * (r1v[4 * j + 1] + ec1 * r2v[4 * j + 1]));
+      st_pair_split(sdT, sdTl, r1, c, TILE64, bc0 * (r1v[4 * j + 2] + ec0 * r2v[4 * j + 2]),
+                    bc1 * (r1v[4 * j + 3] + ec1 * r2v[4 * j + 3]));
+      sKKG[r0 * 65 + c] = c < r0 ? __expf(G0 - sG[c]) * kk[4 * j] : 0.f;
+      sKKG[r0 * 65 + c + 1] = c + 1 < r0 ? __expf(G0 - sG[c + 1]) * kk[4 * j + 1] : 0.f;
+      sKKG[r1 * 65 + c] = c < r1 ? __expf(G1 - sG[c]) * kk[4 * j + 2] : 0.f;
+      sKKG[r1 * 65 + c + 1] = c + 1 < r1 ? __expf(G1 - sG[c + 1]) * kk[4 * j + 3] : 0.f;
     }
-    // dX: dbeta/dG parts, then beta_i e^{G_i} dX back into TMEM
-    float px = 0.f;
-    for (int cc = 0; cc < 64; cc += 16) {
-      float x[16], kv[16];
-      tmem_ld16(taddr(tb, sub, 256 + 64 * half + cc), x);
-      tmem_wait_ld();
-      ld_chunk_f(sK, ii, (64 * half + cc) / 8, TILE64, kv);
-      ld_chunk_f(sK, ii, (64 * half + cc) / 8 + 1, TILE64, kv + 8);
-      for (int q = 0; q < 16; ++q) {
-        px += x[q] * kv[q];
-        x[q] *= bi * egi;
-      }
-      tmem_st16(taddr(tb, sub, 256 + 64 * half + cc), x);
+    // dX: dbeta/dG parts, then beta_i e^{G_i} dX back into TMEM; dY: dv = beta dY, dbeta part
+    float x[32], y[32];
+    tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
+    tmem_ld16dp_x8(taddr(tb, sub, 384 + 64 * half), y);
+    tmem_wait_ld();
+    const float s0 = b0 * sEG[r0], s1 = b1 * sEG[r1];
+    float px0 = 0.f, px1 = 0.f, py0 = 0.f, py1 = 0.f;
+    bf16* dv0 = static_cast<bf16*>(a.dv) + ((size_t)(tok0 + r0) * p.HV + hv) * D + 64 * half + cq;
+    bf16* dv1 = dv0 + (size_t)8 * p.HV * D;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = 64 * half + 8 * j + cq;
+      const float2 k0 = ld_pair(sK, r0, c, TILE64), k1 = ld_pair(sK, r1, c, TILE64);
+      const float2 v0 = ld_pair(sV, r0, c, TILE64), v1 = ld_pair(sV, r1, c, TILE64);
+      px0 += x[4 * j] * k0.x + x[4 * j + 1] * k0.y;
+      px1 += x[4 * j + 2] * k1.x + x[4 * j + 3] * k1.y;
+      x[4 * j] *= s0; x[4 * j + 1] *= s0; x[4 * j + 2] *= s1; x[4 * j + 3] *= s1;
+      py0 += y[4 * j] * v0.x + y[4 * j + 1] * v0.y;
+      py1 += y[4 * j + 2] * v1.x + y[4 * j + 3] * v1.y;
+      if (r0 < L)
+        *reinterpret_cast<uint32_t*>(dv0 + 8 * j) = pack_bf16(b0 * y[4 * j], b0 * y[4 * j + 1]);
+      if (r1 < L)
+        *reinterpret_cast<uint32_t*>(dv1 + 8 * j) = pack_bf16(b1 * y[4 * j + 2], b1 * y[4 * j + 3]);
     }
-    // dY: dv = beta dY, dbeta part
-    float py = 0.f;
-    bf16* dvrow = static_cast<bf16*>(a.dv) + ((size_t)(tok0 + ii) * p.HV + hv) * D + 64 * half;
-    for (int cc = 0; cc < 64; cc += 16) {
-      float y[16], vv[16];
-      tmem_ld16(taddr(tb, sub, 384 + 64 * half + cc), y);
-      tmem_wait_ld();
-      ld_chunk_f(sV, ii, (64 * half + cc) / 8, TILE64, vv);
-      ld_chunk_f(sV, ii, (64 * half + cc) / 8 + 1, TILE64, vv + 8);
-      for (int q = 0; q < 16; ++q) py += y[q] * vv[q];
-      if (lane < 16 && ii < L) {
-        uint4 a0, a1;
-        a0.x = pack_bf16(bi * y[0], bi * y[1]); a0.y = pack_bf16(bi * y[2], bi * y[3]);
-        a0.z = pack_bf16(bi * y[4], bi * y[5]); a0.w = pack_bf16(bi * y[6], bi * y[7]);
-        a1.x = pack_bf16(bi * y[8], bi * y[9]); a1.y = pack_bf16(bi * y[10], bi * y[11]);
-        a1.z = pack_bf16(bi * y[12], bi * y[13]); a1.w = pack_bf16(bi * y[14], bi * y[15]);
-        *reinterpret_cast<uint4*>(dvrow + cc) = a0;
-        *reinterpret_cast<uint4*>(dvrow + cc + 8) = a1;
-      }
-    }
-    if (lane < 16) {
-      sRow[(0 * 2 + half) * 64 + ii] = px;
-      sRow[(1 * 2 + half) * 64 + ii] = py;
+    tmem_st16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
+    px0 = quad_sum(px0);
+    px1 = quad_sum(px1);
+    py0 = quad_sum(py0);
+    py1 = quad_sum(py1);
+    if ((lane & 3) == 0) {
+      sRow[(0 * 2 + half) * 64 + r0] = px0;
+      sRow[(0 * 2 + half) * 64 + r1] = px1;
+      sRow[(1 * 2 + half) * 64 + r0] = py0;
+      sRow[(1 * 2 + half) * 64 + r1] = py1;
     }
     tmem_wait_st();
   }
@@ -808,9 +813,8 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // Z = T^T dT
+  // Z = T^T dT, dropping lo*lo
   if (ok && tid == 0) {
-    // (T_hi + T_lo)^T (dT_hi + dT_lo), dropping lo*lo
     const uint32_t dt = smem_u32(sdT), dtl = smem_u32(sdTl);
     const uint32_t pa[3] = {aT, aT, aTl}, pb[3] = {dt, dtl, dt};
     for (int part = 0; part < 3; ++part)
@@ -822,12 +826,15 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
   tc_fence_after();
   if (ok) {
-    float z[32];
-    tmem_ld16(taddr(tb, sub, 32 * half), z);
-    tmem_ld16(taddr(tb, sub, 32 * half + 16), z + 16);
+    float z[16];
+    tmem_ld16dp_x4(taddr(tb, sub, 32 * half), z);
     tmem_wait_ld();
-    if (lane < 16)
-      for (int j = 0; j < 4; ++j) st_chunk_split(sZ, sZl, ii, 4 * half + j, TILE64, z + 8 * j);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = 32 * half + 8 * j + cq;
+      st_pair_split(sZ, sZl, r0, c, TILE64, z[4 * j], z[4 * j + 1]);
+      st_pair_split(sZ, sZl, r1, c, TILE64, z[4 * j + 2], z[4 * j + 3]);
+    }
   }
   fence_proxy_async();
   tc_fence_before();
@@ -846,29 +853,42 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
   tc_fence_after();
   if (ok) {
-    float da[32];
-    tmem_ld16(taddr(tb, sub, 64 + 32 * half), da);
-    tmem_ld16(taddr(tb, sub, 64 + 32 * half + 16), da + 16);
+    float da[16];
+    tmem_ld16dp_x4(taddr(tb, sub, 64 + 32 * half), da);
     tmem_wait_ld();
-    if (lane < 16) {
-      float pa = 0.f, paa = 0.f, f[8];
-      for (int jj = 0; jj < 32; ++jj) {
-        const int j = 32 * half + jj;
+    float pa0 = 0.f, pa1 = 0.f, paa0 = 0.f, paa1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = 32 * half + 8 * j + cq;
+      float as[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int row = q < 2 ? r0 : r1, col = c + (q & 1);
+        const float Gi = q < 2 ? G0 : G1, bi = q < 2 ? b0 : b1;
         float dAs = 0.f, aa = 0.f;
-        if (j < ii) {
-          const float dA = -da[jj];
-          const float kkg = sKKG[ii * 65 + j];
-          pa += dA * kkg;
+        if (col < row) {
+          const float dA = -da[4 * j + q];
+          const float kkg = sKKG[row * 65 + col];
+          if (q < 2) pa0 += dA * kkg; else pa1 += dA * kkg;
           aa = dA * bi * kkg;
-          dAs = dA * expf(Gi - sG[j]) * bi;
+          dAs = dA * __expf(Gi - sG[col]) * bi;
         }
-        sAA[ii * 65 + j] = aa;
-        paa += aa;
-        f[jj & 7] = dAs;
-        if ((jj & 7) == 7) st_chunk_split(sAs, sAsl, ii, j / 8, TILE64, f);
+        sAA[row * 65 + col] = aa;
+        if (q < 2) paa0 += aa; else paa1 += aa;
+        as[q] = dAs;
       }
-      sRow[(2 * 2 + half) * 64 + ii] = pa;
-      sRow[(3 * 2 + half) * 64 + ii] = paa;
+      st_pair_split(sAs, sAsl, r0, c, TILE64, as[0], as[1]);
+      st_pair_split(sAs, sAsl, r1, c, TILE64, as[2], as[3]);
+    }
+    pa0 = quad_sum(pa0);
+    pa1 = quad_sum(pa1);
+    paa0 = quad_sum(paa0);
+    paa1 = quad_sum(paa1);
+    if ((lane & 3) == 0) {
+      sRow[(2 * 2 + half) * 64 + r0] = pa0;
+      sRow[(2 * 2 + half) * 64 + r1] = pa1;
+      sRow[(3 * 2 + half) * 64 + r0] = paa0;
+      sRow[(3 * 2 + half) * 64 + r1] = paa1;
     }
   }
   fence_proxy_async();
@@ -892,7 +912,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     const int j = tid;
     float cs = 0.f;
     for (int r = 0; r < 64; ++r) cs += sAA[r * 65 + j];
-    const float eg = expf(sG[j]), bj = sb[j];
+    const float eg = sEG[j], bj = sb[j];
     const float px = sRow[0 * 64 + j] + sRow[1 * 64 + j];
     const float py = sRow[2 * 64 + j] + sRow[3 * 64 + j];
     const float pa = sRow[4 * 64 + j] + sRow[5 * 64 + j];
@@ -903,20 +923,18 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
   tc_fence_after();
   if (ok) {
-    float* dk = w.dkp + (unit * 64 + ii) * D + 64 * half;
-    for (int cc = 0; cc < 64; cc += 16) {
-      float x[16];
-      tmem_ld16(taddr(tb, sub, 256 + 64 * half + cc), x);
-      tmem_wait_ld();
-      if (lane < 16)
-        for (int q = 0; q < 16; q += 4) {
-          float4 o = *reinterpret_cast<float4*>(dk + cc + q);
-          o.x += x[q];
-          o.y += x[q + 1];
-          o.z += x[q + 2];
-          o.w += x[q + 3];
-          *reinterpret_cast<float4*>(dk + cc + q) = o;
-        }
+    float x[32];
+    tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
+    tmem_wait_ld();
+    float* dk0 = w.dkp + (unit * 64 + r0) * D + 64 * half + cq;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float2 o0 = *reinterpret_cast<float2*>(dk0 + 8 * j);
+      float2 o1 = *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j);
+      o0.x += x[4 * j]; o0.y += x[4 * j + 1];
+      o1.x += x[4 * j + 2]; o1.y += x[4 * j + 3];
+      *reinterpret_cast<float2*>(dk0 + 8 * j) = o0;
+      *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j) = o1;
     }
   }
   tc_fence_before();
@@ -937,7 +955,7 @@ cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, 
                m.k, m.dO, m.WT, m.dUlT, m.dh)))
     return e;
   if ((e = tgo("tc_dqkwg", k_tc_dqkwg, gu, 256, 1024 + DqkSmem::TOTAL, s, p, w, t, m.q, m.k, m.dO,
-               m.UT, m.dUT, m.dUTl, m.h, m.dh)))
+               m.UT, m.dUT, m.dUTl, m.h, m.dh, m.dW)))
     return e;
   if ((e = tgo("tc_wy_bwd", k_tc_wy_bwd, gu, 256, 1024 + WyBwdSmem::TOTAL, s, p, a, w, t, m.k, m.v,
                m.Tm, m.dW, m.dUT, m.dUTl)))

@@ -218,6 +218,29 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT,
   }
 }
 
+// Two adjacent bf16 columns (c even) of row r as one 32-bit store, hi and lo parts.
+__device__ __forceinline__ void st_pair_split(unsigned char* hi, unsigned char* lo, int r, int c,
+                                              int block_bytes, float a, float b) {
+  const float ha = __bfloat162float(__float2bfloat16_rn(a));
+  const float hb = __bfloat162float(__float2bfloat16_rn(b));
+  *reinterpret_cast<uint32_t*>(hi + sw128(r, c, block_bytes)) = pack_bf16(ha, hb);
+  *reinterpret_cast<uint32_t*>(lo + sw128(r, c, block_bytes)) = pack_bf16(a - ha, b - hb);
+}
+__device__ __forceinline__ void st_pair(unsigned char* tile, int r, int c, int block_bytes, float a,
+                                        float b) {
+  *reinterpret_cast<uint32_t*>(tile + sw128(r, c, block_bytes)) = pack_bf16(a, b);
+}
+__device__ __forceinline__ float2 ld_pair(const unsigned char* tile, int r, int c, int block_bytes) {
+  const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(tile + sw128(r, c, block_bytes));
+  return __bfloat1622float2(h);
+}
+// Sum over the 4 lanes (t, t^1, t^2, t^3) that hold the same 16dp row.
+__device__ __forceinline__ float quad_sum(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  x += __shfl_xor_sync(0xffffffffu, x, 2);
+  return x;
+}
+
 __device__ __forceinline__ bool failed(const Work& w) { return *((volatile int*)w.status) != 0; }
 
 
