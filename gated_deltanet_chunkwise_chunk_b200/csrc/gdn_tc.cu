@@ -214,12 +214,12 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
 // chunk's W^T, U~^T and K tiles are prefetched one chunk ahead (double buffer).
 // ======================================================================================
 struct ScanSmem {
-  static constexpr int S = 0;                       // [128][128] bf16: 2 x 16 KB
-  static constexpr int BUF = 2 * TILE128;           // 2 x {W^T 16K, U~^T 16K, K 16K}
+  static constexpr int S = 0;                       // 2 x [128][128] bf16 (alternating chunks)
+  static constexpr int BUF = 4 * TILE128;           // 2 x {W^T 16K, U~^T 16K, K 16K}
   static constexpr int BUF_BYTES = 3 * TILE128;
   static constexpr int UD = BUF + 2 * BUF_BYTES;    // [128][64] Ud^T
-  static constexpr int UO = UD + TILE128;           // [128][64] U^T staging
-  static constexpr int G = UO + TILE128;            // 2 x 64 floats
+  static constexpr int UO = UD + TILE128;           // 2 x [128][64] U^T staging
+  static constexpr int G = UO + 2 * TILE128;        // 2 x 64 floats
   static constexpr int DEC = G + 2 * 256;           // 64 floats e^{G_C - G_i}
   static constexpr int TOTAL = DEC + 256;
 };
@@ -238,9 +238,7 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
   const int v = 32 * (warp & 3) + lane, half = warp >> 2;
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
-  unsigned char* sS = sm + ScanSmem::S;
   unsigned char* sUd = sm + ScanSmem::UD;
-  unsigned char* sUo = sm + ScanSmem::UO;
   float* sGb = reinterpret_cast<float*>(sm + ScanSmem::G);
   float* sDec = reinterpret_cast<float*>(sm + ScanSmem::DEC);
   __shared__ uint64_t barT[2], barM;
@@ -257,14 +255,14 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
     tmem_alloc(&tslot, 256);
     tmem_relinquish();
   }
-  // initial state (fp32) -> registers; bf16 copy -> sS
+  // initial state (fp32) -> registers; bf16 copy -> state buffer 0
   float S[64];
   const size_t st = ((size_t)n * p.HV + hv) * D * D;  // [K][V] fp32 states
   for (int i = 0; i < 64; ++i) {
     const int kk = half * 64 + i;
     S[i] = a.h0 ? a.h0[st + (size_t)kk * D + v] : 0.f;
   }
-  for (int j = 0; j < 8; ++j) st_chunk_f(sS, v, half * 8 + j, TILE128, &S[8 * j]);
+  for (int j = 0; j < 8; ++j) st_chunk_f(sm + ScanSmem::S, v, half * 8 + j, TILE128, &S[8 * j]);
   auto issue = [&](int c) {
     const int gc = sq.x + c, buf = c & 1;
     const int tok = sq.z + 64 * c;  // chunks of a sequence are consecutive, 64 tokens apart
@@ -281,6 +279,8 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
+  if (tid < 64 && sq.y > 0) sDec[tid] = expf(sGb[63] - sGb[tid]);
+  __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
   const uint32_t tD1 = taddr(tb, 0, 0), tD2 = taddr(tb, 0, 64);
@@ -289,6 +289,9 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
   for (int c = 0; c < sq.y && ok; ++c) {
     const int gc = sq.x + c, buf = c & 1;
     unsigned char* b = sm + ScanSmem::BUF + buf * ScanSmem::BUF_BYTES;
+    unsigned char* sS = sm + ScanSmem::S + buf * 2 * TILE128;       // S entering chunk c
+    unsigned char* sSn = sm + ScanSmem::S + (buf ^ 1) * 2 * TILE128;
+    unsigned char* sUo = sm + ScanSmem::UO + buf * TILE128;
     const uint32_t unit_row = (uint32_t)(gc * p.HV + hv) * D;
     float* sG = sGb + buf * 64;
     if (tid == 0 && c + 1 < sq.y) issue(c + 1);
@@ -296,9 +299,11 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
     if (tid < 64 && c + 1 < sq.y) gnext = w.G[((size_t)hv * p.NCmax + gc + 1) * 64 + tid];
     ok = __syncthreads_and(mbar_wait(&barT[buf], phT[buf], err));
     phT[buf] ^= 1;
-    if (tid < 64) sDec[tid] = expf(sG[63] - sG[tid]);
+    if (!ok) break;
     // S entering this chunk -> h (TMA store), MMA1
-    if (ok && tid == 0) {
+    if (tid == 0) {
+      // the stores of two chunks ago (same S and U^T buffers) must have finished reading
+      tma_store_wait_read0();
       tma_store_3d(&mh, sS, 0, unit_row, 0);
       tma_store_3d(&mh, sS + TILE128, 64, unit_row, 0);
       tma_store_commit();
@@ -308,7 +313,7 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
                  idesc_bf16(128, 64, false, true), s > 0);
       mma_commit(&barM);
     }
-    ok = __syncthreads_and(ok && mbar_wait(&barM, phM, err));
+    ok = __syncthreads_and(mbar_wait(&barM, phM, err));
     phM ^= 1;
     tc_fence_after();
     if (!ok) break;
@@ -319,8 +324,6 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
       tmem_ld16(taddr(tb, 32 * (warp & 3), 32 * half + 16), d + 16);
       tmem_wait_ld();
       const unsigned char* ut = b + TILE128;
-      if (tid == 0) tma_store_wait_read0();  // previous U^T staging store has read sUo
-      __syncthreads();
       for (int j = 0; j < 4; ++j) {
         float u[8], ud[8];
         ld_chunk_f(ut, v, half * 4 + j, TILE128, u);
@@ -351,19 +354,19 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
     if (!ok) break;
     {
       const float eg = expf(sG[63]);
-      for (int cc = 0; cc < 64; cc += 16) {
-        float d[16];
-        tmem_ld16(taddr(tb, 32 * (warp & 3), 64 + 64 * half + cc), d);
-        tmem_wait_ld();
-        for (int i = 0; i < 16; ++i) S[cc + i] = eg * S[cc + i] + d[i];
-      }
+      float d[64];
+      tmem_ld64(taddr(tb, 32 * (warp & 3), 64 + 64 * half), d);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 64; ++i) S[i] = eg * S[i] + d[i];
     }
-    if (tid == 0) tma_store_wait_read0();  // the h store has finished reading sS
-    __syncthreads();
-    for (int j = 0; j < 8; ++j) st_chunk_f(sS, v, half * 8 + j, TILE128, &S[8 * j]);
+    // the next chunk's state goes to the other buffer (its last h store was two chunks ago)
+    for (int j = 0; j < 8; ++j) st_chunk_f(sSn, v, half * 8 + j, TILE128, &S[8 * j]);
     if (tid < 64 && c + 1 < sq.y) sGb[(buf ^ 1) * 64 + tid] = gnext;
     fence_proxy_async();
     tc_fence_before();
+    __syncthreads();
+    if (tid < 64 && c + 1 < sq.y) sDec[tid] = expf(sGb[(buf ^ 1) * 64 + 63] - sGb[(buf ^ 1) * 64 + tid]);
     __syncthreads();
     tc_fence_after();
   }

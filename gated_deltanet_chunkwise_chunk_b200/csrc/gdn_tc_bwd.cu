@@ -151,8 +151,8 @@ struct BwdScanSmem {
   static constexpr int K = 4 * TILE128, Q = K + 2 * TILE64, O = Q + 2 * TILE64;
   static constexpr int W = O + 2 * TILE64, UL = W + TILE128;     // W^T, dU_loc^T [128][64]
   static constexpr int ATH = UL + TILE128, ATL = ATH + TILE128;  // -dU^T hi / lo
-  static constexpr int G = ATL + TILE128;                        // 2 x 64 floats
-  static constexpr int DEC = G + 512;                            // e^{G_C - G_j}
+  static constexpr int G = ATL + TILE128;                        // 64 floats
+  static constexpr int DEC = G + 256;                            // e^{G_C - G_j}
   static constexpr int EG = DEC + 256;                           // scale e^{G_i} (0 past L)
   static constexpr int TOTAL = EG + 256;
 };
@@ -180,14 +180,15 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
   unsigned char* sUL = sm + BwdScanSmem::UL;
   unsigned char* sATH = sm + BwdScanSmem::ATH;
   unsigned char* sATL = sm + BwdScanSmem::ATL;
-  float* sGb = reinterpret_cast<float*>(sm + BwdScanSmem::G);
+  float* sG = reinterpret_cast<float*>(sm + BwdScanSmem::G);
   float* sDec = reinterpret_cast<float*>(sm + BwdScanSmem::DEC);
   float* sEG = reinterpret_cast<float*>(sm + BwdScanSmem::EG);
-  __shared__ uint64_t barA, barW, barU, barM;
+  __shared__ uint64_t barK, barQO, barW, barU, barM;
   __shared__ uint32_t tslot;
   int* err = w.status;
   if (tid == 0) {
-    mbar_init(&barA, 1);
+    mbar_init(&barK, 1);
+    mbar_init(&barQO, 1);
     mbar_init(&barW, 1);
     mbar_init(&barU, 1);
     mbar_init(&barM, 1);
@@ -203,15 +204,18 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
   for (int i = 0; i < 64; ++i) S[i] = a.dht ? a.dht[st + (size_t)(half * 64 + i) * D + v] : 0.f;
   for (int j = 0; j < 8; ++j) st_chunk_split(sSH, sSL, v, half * 8 + j, TILE128, &S[8 * j]);
   auto row_of = [&](int c) { return ((sq.x + c) * p.HV + hv) * D; };
-  auto issue_A = [&](int c) {  // K, Q, dO of chunk c
-    const int tok = sq.z + 64 * c;
-    mbar_expect_tx(&barA, 6 * TILE64);
-    tma_load_3d(sK, &mk, 0, hk, tok, &barA);
-    tma_load_3d(sK + TILE64, &mk, 64, hk, tok, &barA);
-    tma_load_3d(sQ, &mq, 0, hk, tok, &barA);
-    tma_load_3d(sQ + TILE64, &mq, 64, hk, tok, &barA);
-    tma_load_3d(sO, &mdO, 0, hv, tok, &barA);
-    tma_load_3d(sO + TILE64, &mdO, 64, hv, tok, &barA);
+  auto tok_of = [&](int c) { return sq.z + 64 * c; };
+  auto issue_K = [&](int c) {
+    mbar_expect_tx(&barK, 2 * TILE64);
+    tma_load_3d(sK, &mk, 0, hk, tok_of(c), &barK);
+    tma_load_3d(sK + TILE64, &mk, 64, hk, tok_of(c), &barK);
+  };
+  auto issue_QO = [&](int c) {
+    mbar_expect_tx(&barQO, 4 * TILE64);
+    tma_load_3d(sQ, &mq, 0, hk, tok_of(c), &barQO);
+    tma_load_3d(sQ + TILE64, &mq, 64, hk, tok_of(c), &barQO);
+    tma_load_3d(sO, &mdO, 0, hv, tok_of(c), &barQO);
+    tma_load_3d(sO + TILE64, &mdO, 64, hv, tok_of(c), &barQO);
   };
   auto issue_W = [&](int c) {
     mbar_expect_tx(&barW, TILE128);
@@ -222,52 +226,47 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     tma_load_3d(sUL, &mdUlT, 0, row_of(c), 0, &barU);
   };
   if (tid == 0 && sq.y > 0) {
-    issue_A(sq.y - 1);
+    issue_K(sq.y - 1);
+    issue_QO(sq.y - 1);
     issue_W(sq.y - 1);
     issue_U(sq.y - 1);
   }
-  if (tid < 64 && sq.y > 0) sGb[tid] = w.G[((size_t)hv * p.NCmax + sq.x + sq.y - 1) * 64 + tid];
+  if (tid < 64 && sq.y > 0) {
+    const int c = sq.y - 1, L = min(64, sq.w - 64 * c);
+    const float g = w.G[((size_t)hv * p.NCmax + sq.x + c) * 64 + tid];
+    sG[tid] = g;
+    sEG[tid] = tid < L ? p.scale * expf(g) : 0.f;
+  }
   fence_proxy_async();
   tc_fence_before();
+  __syncthreads();
+  if (tid < 64 && sq.y > 0) sDec[tid] = expf(sG[63] - sG[tid]);
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
   const uint32_t tE = taddr(tb, 0, 0), tF = taddr(tb, 0, 64);
-  uint32_t ph = 0, phM = 0;  // barA/barW/barU complete once per chunk; barM twice
+  uint32_t ph = 0, phM = 0;  // the tile barriers complete once per chunk, barM twice
   bool ok = true;
   for (int idx = 0; idx < sq.y && ok; ++idx) {
     const int c = sq.y - 1 - idx, gc = sq.x + c;
     const bool more = idx + 1 < sq.y;
     const int L = min(64, sq.w - 64 * c);
     const uint32_t unit_row = (uint32_t)row_of(c);
-    float* sG = sGb + (idx & 1) * 64;
     float gnext = 0.f;  // G of the next chunk (c - 1), stored at the end of this step
     if (tid < 64 && more) gnext = w.G[((size_t)hv * p.NCmax + gc - 1) * 64 + tid];
-    ok = __syncthreads_and(mbar_wait(&barA, ph, err));
+    ok = __syncthreads_and(mbar_wait(&barK, ph, err));
     if (!ok) break;
-    if (tid < 64) {
-      sDec[tid] = expf(sG[63] - sG[tid]);
-      sEG[tid] = tid < L ? p.scale * expf(sG[tid]) : 0.f;
+    if (L < 64) {
+      zero_tail_rows(sK, L, tid, 256);
+      fence_proxy_async();
+      __syncthreads();
     }
-    __syncthreads();
-    for (int i = tid; i < 64 * 16; i += 256) {  // dO rows scaled by scale e^{G_i}, 0 past L
-      const int r = i / 16, j = i % 16;
-      float f[8];
-      ld_chunk_f(sO, r, j, TILE64, f);
-      for (int q = 0; q < 8; ++q) f[q] *= sEG[r];
-      st_chunk_f(sO, r, j, TILE64, f);
-    }
-    if (L < 64) zero_tail_rows(sK, L, tid, 256);
-    fence_proxy_async();
-    __syncthreads();
+    // MMA1 (the chain): E = dS K^T with the compensated dS pair
     if (tid == 0) {
       tma_store_3d(&mdh, sSH, 0, unit_row, 0);
       tma_store_3d(&mdh, sSH + TILE128, 64, unit_row, 0);
       tma_store_commit();
-      const uint32_t o = smem_u32(sO), q = smem_u32(sQ), k = smem_u32(sK);
-      for (int s = 0; s < 4; ++s)
-        mma_bf16(tF, desc_mnmajor(o, s, TILE64), desc_mnmajor(q, s, TILE64),
-                 idesc_bf16(128, 128, true, true), s > 0);
+      const uint32_t k = smem_u32(sK);
       for (int part = 0; part < 2; ++part) {
         const uint32_t sa = smem_u32(part ? sSL : sSH);
         for (int s = 0; s < 8; ++s)
@@ -276,11 +275,21 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
       }
       mma_commit(&barM);
     }
-    ok = __syncthreads_and(mbar_wait(&barM, phM, err));
+    // off the chain while MMA1 runs: dO rows scaled by scale e^{G_i} (zero past L)
+    ok = mbar_wait(&barQO, ph, err);
+    for (int i = tid; i < 64 * 16; i += 256) {
+      const int r = i / 16, j = i % 16;
+      float f[8];
+      ld_chunk_f(sO, r, j, TILE64, f);
+      for (int q = 0; q < 8; ++q) f[q] *= sEG[r];
+      st_chunk_f(sO, r, j, TILE64, f);
+    }
+    fence_proxy_async();
+    ok = __syncthreads_and(ok && mbar_wait(&barM, phM, err));
     phM ^= 1;
     tc_fence_after();
     if (!ok) break;
-    if (tid == 0 && more) issue_A(c - 1);  // K, Q, dO consumed by the MMAs above
+    if (tid == 0 && more) issue_K(c - 1);  // K consumed by MMA1
     ok = __syncthreads_and(mbar_wait(&barU, ph, err));
     if (!ok) break;
     {
@@ -315,10 +324,13 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     tc_fence_after();
     if (tid == 0) {
       if (more) issue_U(c - 1);  // dU_loc^T consumed
-      bool wok = mbar_wait(&barW, ph, err);
+      const bool wok = mbar_wait(&barW, ph, err);
       if (wok) {
-        const uint32_t wt = smem_u32(sW);
-        for (int part = 0; part < 2; ++part) {
+        const uint32_t o = smem_u32(sO), q = smem_u32(sQ), wt = smem_u32(sW);
+        for (int s = 0; s < 4; ++s)  // F = (scale diag(e^G) dO)^T Q
+          mma_bf16(tF, desc_mnmajor(o, s, TILE64), desc_mnmajor(q, s, TILE64),
+                   idesc_bf16(128, 128, true, true), s > 0);
+        for (int part = 0; part < 2; ++part) {  // F -= dU^T W
           const uint32_t at = smem_u32(part ? sATL : sATH);
           for (int s = 0; s < 4; ++s)
             mma_bf16(tF, desc_kmajor(at, s, TILE128), desc_kmajor(wt, s, TILE128),
@@ -332,22 +344,30 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     ph ^= 1;
     tc_fence_after();
     if (!ok) break;
-    if (tid == 0 && more) issue_W(c - 1);  // W^T consumed
+    if (tid == 0 && more) {  // W^T, Q, dO consumed
+      issue_W(c - 1);
+      issue_QO(c - 1);
+    }
     {
       const float eg = expf(sG[63]);
-      for (int cc = 0; cc < 64; cc += 16) {
-        float d[16];
-        tmem_ld16(taddr(tb, 32 * (warp & 3), 64 + 64 * half + cc), d);
-        tmem_wait_ld();
-        for (int i = 0; i < 16; ++i) S[cc + i] = eg * S[cc + i] + d[i];
-      }
+      float d[64];
+      tmem_ld64(taddr(tb, 32 * (warp & 3), 64 + 64 * half), d);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 64; ++i) S[i] = eg * S[i] + d[i];
     }
     if (tid == 0) tma_store_wait_read0();  // the dh store has finished reading dS hi
     __syncthreads();
     for (int j = 0; j < 8; ++j) st_chunk_split(sSH, sSL, v, half * 8 + j, TILE128, &S[8 * j]);
-    if (tid < 64 && more) sGb[((idx + 1) & 1) * 64 + tid] = gnext;
+    if (tid < 64 && more) {
+      const int Ln = min(64, sq.w - 64 * (c - 1));
+      sG[tid] = gnext;
+      sEG[tid] = tid < Ln ? p.scale * expf(gnext) : 0.f;
+    }
     fence_proxy_async();
     tc_fence_before();
+    __syncthreads();
+    if (tid < 64 && more) sDec[tid] = expf(sG[63] - sG[tid]);
     __syncthreads();
     tc_fence_after();
   }
