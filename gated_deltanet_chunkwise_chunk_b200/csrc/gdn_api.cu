@@ -40,7 +40,7 @@ int check_dims(const gdn_dims* d, bool varlen) {
 // Byte offsets of the workspace regions (FFMA path layout; the tcgen05 path appends its
 // own regions after the common ones).
 struct Plan {
-  size_t status, seq_tab, chunk_tab, G, beta_p;
+  size_t status, seq_tab, chunk_tab, G, beta_p, Dec, EG;
   size_t W, Ut, Tm, h, U, dU, dh, dW, dqp, dkp, dG, tmp;
   size_t tc;     // start of the tcgen05 path's region
   size_t total;
@@ -62,6 +62,8 @@ Plan make_plan(const gdn_dims& d, bool varlen, int pass) {
   pl.chunk_tab = take(NC * sizeof(int4));
   pl.G = take(HV * NC * CH * f);
   pl.beta_p = take(HV * NC * CH * f);
+  pl.Dec = take(HV * NC * CH * f);
+  pl.EG = take(HV * NC * CH * f);
   const bool ffma = pass == 0 ? !(d.dtype == GDN_DTYPE_BF16 && tc_supported(d))
                               : !(d.dtype == GDN_DTYPE_BF16 && tc_bwd_supported(d));
   if (ffma) {
@@ -101,6 +103,8 @@ Work carve(const Plan& pl, void* ws) {
   w.chunk_tab = reinterpret_cast<int4*>(b + pl.chunk_tab);
   w.G = reinterpret_cast<float*>(b + pl.G);
   w.beta_p = reinterpret_cast<float*>(b + pl.beta_p);
+  w.Dec = reinterpret_cast<float*>(b + pl.Dec);
+  w.EG = reinterpret_cast<float*>(b + pl.EG);
   auto fp = [&](size_t off) { return off ? reinterpret_cast<float*>(b + off) : nullptr; };
   w.W = fp(pl.W);
   w.Ut = fp(pl.Ut);

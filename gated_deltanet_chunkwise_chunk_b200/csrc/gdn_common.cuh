@@ -29,6 +29,8 @@ struct Work {
   int4* chunk_tab;    // [NCmax] {sequence, chunk in sequence, tokens L, flat token of row 0}
   float* G;           // [HV][NCmax][64]   in-chunk inclusive cumsum of g, padded with G[L-1]
   float* beta_p;      // [HV][NCmax][64]   beta, zero past the chunk's last token
+  float* Dec;         // [HV][NCmax][64]   e^{G_63 - G_i}  (decay from token i to the chunk end)
+  float* EG;          // [HV][NCmax][64]   e^{G_i}
   // fp32 intermediates of the FFMA path
   float* W;           // [NCmax][HV][64][K]
   float* Ut;          // [NCmax][HV][64][V]

@@ -114,6 +114,12 @@ __global__ void __launch_bounds__(256) k_gate_cumsum(Problem p, Args a, Work w) 
     float2* Bp = reinterpret_cast<float2*>(w.beta_p + ((size_t)hv * p.NCmax + gc) * CH);
     Gp[lane] = make_float2(incl0, incl1);
     Bp[lane] = make_float2(s_b[(2 * lane) * HV + hv], s_b[(2 * lane + 1) * HV + hv]);
+    // decay vectors of the chunk: e^{G_63 - G_i} (G_63 = the last lane's inclusive sum) and e^{G_i}
+    const float gl = __shfl_sync(0xffffffffu, incl1, 31);
+    float2* Dp = reinterpret_cast<float2*>(w.Dec + ((size_t)hv * p.NCmax + gc) * CH);
+    float2* Ep = reinterpret_cast<float2*>(w.EG + ((size_t)hv * p.NCmax + gc) * CH);
+    Dp[lane] = make_float2(expf(gl - incl0), expf(gl - incl1));
+    Ep[lane] = make_float2(expf(incl0), expf(incl1));
   }
 }
 

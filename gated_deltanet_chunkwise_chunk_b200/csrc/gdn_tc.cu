@@ -219,11 +219,14 @@ struct ScanSmem {
   static constexpr int BUF_BYTES = 3 * TILE128;
   static constexpr int UD = BUF + 2 * BUF_BYTES;    // [128][64] Ud^T
   static constexpr int UO = UD + TILE128;           // 2 x [128][64] U^T staging
-  static constexpr int G = UO + 2 * TILE128;        // 2 x 64 floats
-  static constexpr int DEC = G + 2 * 256;           // 64 floats e^{G_C - G_i}
-  static constexpr int TOTAL = DEC + 256;
+  static constexpr int DEC = UO + 2 * TILE128;      // 2 x 64 floats e^{G_C - G_i}
+  static constexpr int EGC = DEC + 2 * 256;         // 2 floats e^{G_C}
+  static constexpr int TOTAL = EGC + 64;
 };
 
+// Roles inside the scan CTAs: thread 0 issues the tensor-core MMAs, thread 32 the TMA stores
+// (and waits on them; bulk-copy groups are per thread), thread 64 the TMA loads.  Every
+// thread waits on the mbarriers itself; a chunk step has two CTA-wide barriers.
 __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, TcWork t,
                                                      const __grid_constant__ CUtensorMap mk,
                                                      const __grid_constant__ CUtensorMap mWT,
@@ -239,15 +242,16 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
   unsigned char* sUd = sm + ScanSmem::UD;
-  float* sGb = reinterpret_cast<float*>(sm + ScanSmem::G);
-  float* sDec = reinterpret_cast<float*>(sm + ScanSmem::DEC);
-  __shared__ uint64_t barT[2], barM;
+  float* sDecb = reinterpret_cast<float*>(sm + ScanSmem::DEC);
+  float* sEGC = reinterpret_cast<float*>(sm + ScanSmem::EGC);
+  __shared__ uint64_t barT[2], barM1, barM2;
   __shared__ uint32_t tslot;
   int* err = w.status;
   if (tid == 0) {
     mbar_init(&barT[0], 1);
     mbar_init(&barT[1], 1);
-    mbar_init(&barM, 1);
+    mbar_init(&barM1, 1);
+    mbar_init(&barM2, 1);
     mbar_fence_init();
   }
   __syncthreads();
@@ -274,49 +278,53 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
     tma_load_3d(b + 2 * TILE128, &mk, 0, hk, tok, &barT[buf]);
     tma_load_3d(b + 2 * TILE128 + TILE64, &mk, 64, hk, tok, &barT[buf]);
   };
-  if (tid == 0 && sq.y > 0) issue(0);
-  if (tid < 64 && sq.y > 0) sGb[tid] = w.G[((size_t)hv * p.NCmax + sq.x) * 64 + tid];
+  const size_t vec0 = ((size_t)hv * p.NCmax + sq.x) * 64;  // chunk vectors of this sequence
+  if (tid == 64 && sq.y > 0) issue(0);
+  if (tid < 64 && sq.y > 0) sDecb[tid] = w.Dec[vec0 + tid];
+  if (tid == 0 && sq.y > 0) sEGC[0] = w.EG[vec0 + 63];
   fence_proxy_async();
   tc_fence_before();
-  __syncthreads();
-  if (tid < 64 && sq.y > 0) sDec[tid] = expf(sGb[63] - sGb[tid]);
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
   const uint32_t tD1 = taddr(tb, 0, 0), tD2 = taddr(tb, 0, 64);
   uint32_t phT[2] = {0, 0}, phM = 0;
   bool ok = true;
-  for (int c = 0; c < sq.y && ok; ++c) {
+  for (int c = 0; c < sq.y; ++c) {
     const int gc = sq.x + c, buf = c & 1;
+    const bool more = c + 1 < sq.y;
     unsigned char* b = sm + ScanSmem::BUF + buf * ScanSmem::BUF_BYTES;
     unsigned char* sS = sm + ScanSmem::S + buf * 2 * TILE128;       // S entering chunk c
     unsigned char* sSn = sm + ScanSmem::S + (buf ^ 1) * 2 * TILE128;
     unsigned char* sUo = sm + ScanSmem::UO + buf * TILE128;
+    const float* sDec = sDecb + buf * 64;
     const uint32_t unit_row = (uint32_t)(gc * p.HV + hv) * D;
-    float* sG = sGb + buf * 64;
-    if (tid == 0 && c + 1 < sq.y) issue(c + 1);
-    float gnext = 0.f;  // G of the next chunk, stored to shared memory at the end of this step
-    if (tid < 64 && c + 1 < sq.y) gnext = w.G[((size_t)hv * p.NCmax + gc + 1) * 64 + tid];
-    ok = __syncthreads_and(mbar_wait(&barT[buf], phT[buf], err));
-    phT[buf] ^= 1;
-    if (!ok) break;
-    // S entering this chunk -> h (TMA store), MMA1
-    if (tid == 0) {
-      // the stores of two chunks ago (same S and U^T buffers) must have finished reading
-      tma_store_wait_read0();
+    bool okt = true;
+    if (tid == 0) {  // MMA1: D1 = S W^T
+      okt = mbar_wait(&barT[buf], phT[buf], err);
+      if (okt) {
+        const uint32_t s_ = smem_u32(sS), wt = smem_u32(b);
+        for (int s = 0; s < 8; ++s)
+          mma_bf16(tD1, desc_kmajor(s_, s, TILE128), desc_mnmajor(wt, s, TILE128),
+                   idesc_bf16(128, 64, false, true), s > 0);
+        mma_commit(&barM1);
+      }
+    } else if (tid == 32) {  // S entering this chunk -> h
       tma_store_3d(&mh, sS, 0, unit_row, 0);
       tma_store_3d(&mh, sS + TILE128, 64, unit_row, 0);
       tma_store_commit();
-      const uint32_t s_ = smem_u32(sS), wt = smem_u32(b);
-      for (int s = 0; s < 8; ++s)
-        mma_bf16(tD1, desc_kmajor(s_, s, TILE128), desc_mnmajor(wt, s, TILE128),
-                 idesc_bf16(128, 64, false, true), s > 0);
-      mma_commit(&barM);
+    } else if (tid == 64 && more) {
+      issue(c + 1);
     }
-    ok = __syncthreads_and(mbar_wait(&barM, phM, err));
-    phM ^= 1;
+    float dn = 0.f, en = 0.f;  // next chunk's decay vectors, stored at the end of this step
+    if (tid < 64 && more) {
+      dn = w.Dec[vec0 + (size_t)(c + 1) * 64 + tid];
+      if (tid == 0) en = w.EG[vec0 + (size_t)(c + 1) * 64 + 63];
+    }
+    okt = okt && mbar_wait(&barT[buf], phT[buf], err);
+    phT[buf] ^= 1;
+    okt = okt && mbar_wait(&barM1, phM, err);
     tc_fence_after();
-    if (!ok) break;
     // U^T = U~^T - D1 for columns [32*half, 32*half+32); Ud^T = U^T * e^{G_C - G}
     {
       float d[32];
@@ -335,42 +343,49 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
         st_chunk_f(sUd, v, half * 4 + j, TILE128, ud);
       }
     }
+    // the stores of chunk c-1 (h and U^T) must be done reading before the barrier below
+    // releases writes into their buffers (this step's next-state tile, the next U^T staging)
+    if (tid == 32) tma_store_wait_read<1>();
     fence_proxy_async();
     tc_fence_before();
-    __syncthreads();
+    ok = __syncthreads_and(ok && okt);
     tc_fence_after();
-    if (tid == 0) {
-      tma_store_3d(&mUT, sUo, 0, unit_row, 0);
-      tma_store_commit();
+    if (!ok) break;
+    if (tid == 0) {  // MMA2: D2 = Ud^T K
       const uint32_t ud = smem_u32(sUd), kt = smem_u32(b + 2 * TILE128);
       for (int s = 0; s < 4; ++s)
         mma_bf16(tD2, desc_kmajor(ud, s, TILE128), desc_mnmajor(kt, s, TILE64),
                  idesc_bf16(128, 128, false, true), s > 0);
-      mma_commit(&barM);
+      mma_commit(&barM2);
+    } else if (tid == 32) {
+      tma_store_3d(&mUT, sUo, 0, unit_row, 0);
+      tma_store_commit();
     }
-    ok = __syncthreads_and(mbar_wait(&barM, phM, err));
+    okt = mbar_wait(&barM2, phM, err);
     phM ^= 1;
     tc_fence_after();
-    if (!ok) break;
     {
-      const float eg = expf(sG[63]);
+      const float eg = sEGC[buf];
       float d[64];
       tmem_ld64(taddr(tb, 32 * (warp & 3), 64 + 64 * half), d);
       tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < 64; ++i) S[i] = eg * S[i] + d[i];
     }
-    // the next chunk's state goes to the other buffer (its last h store was two chunks ago)
+    // the next chunk's state goes to the other buffer (its last reader, the h store of chunk
+    // c-1, finished before the mid-step barrier)
     for (int j = 0; j < 8; ++j) st_chunk_f(sSn, v, half * 8 + j, TILE128, &S[8 * j]);
-    if (tid < 64 && c + 1 < sq.y) sGb[(buf ^ 1) * 64 + tid] = gnext;
+    if (tid < 64 && more) {
+      sDecb[(buf ^ 1) * 64 + tid] = dn;
+      if (tid == 0) sEGC[buf ^ 1] = en;
+    }
     fence_proxy_async();
     tc_fence_before();
-    __syncthreads();
-    if (tid < 64 && c + 1 < sq.y) sDec[tid] = expf(sGb[(buf ^ 1) * 64 + 63] - sGb[(buf ^ 1) * 64 + tid]);
-    __syncthreads();
+    ok = __syncthreads_and(ok && okt);
     tc_fence_after();
+    if (!ok) break;
   }
-  if (tid == 0) tma_store_wait0();
+  if (tid == 32) tma_store_wait0();
   if (ok && write_final && a.ht)
     for (int i = 0; i < 64; ++i) a.ht[st + (size_t)(half * 64 + i) * D + v] = S[i];
   tc_fence_before();

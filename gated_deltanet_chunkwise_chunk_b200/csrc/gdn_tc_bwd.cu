@@ -151,12 +151,14 @@ struct BwdScanSmem {
   static constexpr int K = 4 * TILE128, Q = K + 2 * TILE64, O = Q + 2 * TILE64;
   static constexpr int W = O + 2 * TILE64, UL = W + TILE128;     // W^T, dU_loc^T [128][64]
   static constexpr int ATH = UL + TILE128, ATL = ATH + TILE128;  // -dU^T hi / lo
-  static constexpr int G = ATL + TILE128;                        // 64 floats
-  static constexpr int DEC = G + 256;                            // e^{G_C - G_j}
-  static constexpr int EG = DEC + 256;                           // scale e^{G_i} (0 past L)
-  static constexpr int TOTAL = EG + 256;
+  static constexpr int DEC = ATL + TILE128;                      // 2 x 64: e^{G_C - G_j}
+  static constexpr int EG = DEC + 512;                           // 2 x 64: scale e^{G_i} (0 past L)
+  static constexpr int EGC = EG + 512;                           // 2 floats e^{G_C}
+  static constexpr int TOTAL = EGC + 64;
 };
 
+// Roles as in the forward scan: thread 0 MMAs, thread 32 TMA stores, thread 64 TMA loads;
+// two CTA-wide barriers per chunk step.
 __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, TcWork t,
                                                      const __grid_constant__ CUtensorMap mq,
                                                      const __grid_constant__ CUtensorMap mk,
@@ -180,10 +182,10 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
   unsigned char* sUL = sm + BwdScanSmem::UL;
   unsigned char* sATH = sm + BwdScanSmem::ATH;
   unsigned char* sATL = sm + BwdScanSmem::ATL;
-  float* sG = reinterpret_cast<float*>(sm + BwdScanSmem::G);
-  float* sDec = reinterpret_cast<float*>(sm + BwdScanSmem::DEC);
-  float* sEG = reinterpret_cast<float*>(sm + BwdScanSmem::EG);
-  __shared__ uint64_t barK, barQO, barW, barU, barM;
+  float* sDecb = reinterpret_cast<float*>(sm + BwdScanSmem::DEC);
+  float* sEGb = reinterpret_cast<float*>(sm + BwdScanSmem::EG);
+  float* sEGC = reinterpret_cast<float*>(sm + BwdScanSmem::EGC);
+  __shared__ uint64_t barK, barQO, barW, barU, barM1, barM2;
   __shared__ uint32_t tslot;
   int* err = w.status;
   if (tid == 0) {
@@ -191,7 +193,8 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     mbar_init(&barQO, 1);
     mbar_init(&barW, 1);
     mbar_init(&barU, 1);
-    mbar_init(&barM, 1);
+    mbar_init(&barM1, 1);
+    mbar_init(&barM2, 1);
     mbar_fence_init();
   }
   __syncthreads();
@@ -225,58 +228,70 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     mbar_expect_tx(&barU, TILE128);
     tma_load_3d(sUL, &mdUlT, 0, row_of(c), 0, &barU);
   };
-  if (tid == 0 && sq.y > 0) {
+  const size_t vec0 = ((size_t)hv * p.NCmax + sq.x) * 64;  // chunk vectors of this sequence
+  auto len_of = [&](int c) { return min(64, sq.w - 64 * c); };
+  if (tid == 64 && sq.y > 0) {
     issue_K(sq.y - 1);
     issue_QO(sq.y - 1);
     issue_W(sq.y - 1);
     issue_U(sq.y - 1);
   }
   if (tid < 64 && sq.y > 0) {
-    const int c = sq.y - 1, L = min(64, sq.w - 64 * c);
-    const float g = w.G[((size_t)hv * p.NCmax + sq.x + c) * 64 + tid];
-    sG[tid] = g;
-    sEG[tid] = tid < L ? p.scale * expf(g) : 0.f;
+    const int c = sq.y - 1;
+    const size_t o = vec0 + (size_t)c * 64 + tid;
+    sDecb[tid] = w.Dec[o];
+    sEGb[tid] = tid < len_of(c) ? p.scale * w.EG[o] : 0.f;
+    if (tid == 63) sEGC[0] = w.EG[o];
   }
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
-  if (tid < 64 && sq.y > 0) sDec[tid] = expf(sG[63] - sG[tid]);
-  __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
   const uint32_t tE = taddr(tb, 0, 0), tF = taddr(tb, 0, 64);
-  uint32_t ph = 0, phM = 0;  // the tile barriers complete once per chunk, barM twice
+  uint32_t ph = 0, phM = 0;  // the tile barriers complete once per chunk, barM1/barM2 once each
   bool ok = true;
-  for (int idx = 0; idx < sq.y && ok; ++idx) {
-    const int c = sq.y - 1 - idx, gc = sq.x + c;
+  for (int idx = 0; idx < sq.y; ++idx) {
+    const int c = sq.y - 1 - idx, buf = idx & 1;
     const bool more = idx + 1 < sq.y;
-    const int L = min(64, sq.w - 64 * c);
+    const int L = len_of(c);
     const uint32_t unit_row = (uint32_t)row_of(c);
-    float gnext = 0.f;  // G of the next chunk (c - 1), stored at the end of this step
-    if (tid < 64 && more) gnext = w.G[((size_t)hv * p.NCmax + gc - 1) * 64 + tid];
-    ok = __syncthreads_and(mbar_wait(&barK, ph, err));
-    if (!ok) break;
-    if (L < 64) {
+    const float* sDec = sDecb + buf * 64;
+    const float* sEG = sEGb + buf * 64;
+    bool okt = true;
+    if (L < 64) {  // ragged chunk: K rows past its end are zeroed before the chain MMA
+      okt = mbar_wait(&barK, ph, err);
       zero_tail_rows(sK, L, tid, 256);
       fence_proxy_async();
       __syncthreads();
     }
-    // MMA1 (the chain): E = dS K^T with the compensated dS pair
-    if (tid == 0) {
+    if (tid == 0) {  // MMA1 (the chain): E = dS K^T with the compensated dS pair
+      okt = okt && mbar_wait(&barK, ph, err);
+      if (okt) {
+        const uint32_t k = smem_u32(sK);
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t sa = smem_u32(part ? sSL : sSH);
+          for (int s = 0; s < 8; ++s)
+            mma_bf16(tE, desc_kmajor(sa, s, TILE128), desc_kmajor(k, s, TILE64),
+                     idesc_bf16(128, 64, false, false), part > 0 || s > 0);
+        }
+        mma_commit(&barM1);
+      }
+    } else if (tid == 32) {  // dS leaving this chunk -> dh
       tma_store_3d(&mdh, sSH, 0, unit_row, 0);
       tma_store_3d(&mdh, sSH + TILE128, 64, unit_row, 0);
       tma_store_commit();
-      const uint32_t k = smem_u32(sK);
-      for (int part = 0; part < 2; ++part) {
-        const uint32_t sa = smem_u32(part ? sSL : sSH);
-        for (int s = 0; s < 8; ++s)
-          mma_bf16(tE, desc_kmajor(sa, s, TILE128), desc_kmajor(k, s, TILE64),
-                   idesc_bf16(128, 64, false, false), part > 0 || s > 0);
-      }
-      mma_commit(&barM);
+    }
+    float dn = 0.f, en = 0.f, egc = 0.f;  // next chunk's vectors, stored at the end of the step
+    if (tid < 64 && more) {
+      const size_t o = vec0 + (size_t)(c - 1) * 64 + tid;
+      dn = w.Dec[o];
+      const float eg = w.EG[o];
+      en = tid < len_of(c - 1) ? p.scale * eg : 0.f;
+      egc = eg;
     }
     // off the chain while MMA1 runs: dO rows scaled by scale e^{G_i} (zero past L)
-    ok = mbar_wait(&barQO, ph, err);
+    okt = okt && mbar_wait(&barQO, ph, err);
     for (int i = tid; i < 64 * 16; i += 256) {
       const int r = i / 16, j = i % 16;
       float f[8];
@@ -285,13 +300,10 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
       st_chunk_f(sO, r, j, TILE64, f);
     }
     fence_proxy_async();
-    ok = __syncthreads_and(ok && mbar_wait(&barM, phM, err));
-    phM ^= 1;
+    okt = okt && mbar_wait(&barM1, phM, err);
     tc_fence_after();
-    if (!ok) break;
-    if (tid == 0 && more) issue_K(c - 1);  // K consumed by MMA1
-    ok = __syncthreads_and(mbar_wait(&barU, ph, err));
-    if (!ok) break;
+    if (tid == 64 && more) issue_K(c - 1);  // K consumed by MMA1
+    okt = okt && mbar_wait(&barU, ph, err);
     {
       float d[32];
       tmem_ld16(taddr(tb, 32 * (warp & 3), 32 * half), d);
@@ -318,14 +330,17 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
         *reinterpret_cast<uint4*>(lo_row + 8 * j) = pl4;
       }
     }
+    // the dh store of this chunk must be done reading dS before the barrier releases the
+    // dS update below
+    if (tid == 32) tma_store_wait_read0();
     fence_proxy_async();
     tc_fence_before();
-    __syncthreads();
+    ok = __syncthreads_and(ok && okt);
     tc_fence_after();
+    if (!ok) break;
     if (tid == 0) {
-      if (more) issue_U(c - 1);  // dU_loc^T consumed
-      const bool wok = mbar_wait(&barW, ph, err);
-      if (wok) {
+      okt = mbar_wait(&barW, ph, err);
+      if (okt) {
         const uint32_t o = smem_u32(sO), q = smem_u32(sQ), wt = smem_u32(sW);
         for (int s = 0; s < 4; ++s)  // F = (scale diag(e^G) dO)^T Q
           mma_bf16(tF, desc_mnmajor(o, s, TILE64), desc_mnmajor(q, s, TILE64),
@@ -336,42 +351,40 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
             mma_bf16(tF, desc_kmajor(at, s, TILE128), desc_kmajor(wt, s, TILE128),
                      idesc_bf16(128, 128, false, false), 1);
         }
-        mma_commit(&barM);
+        mma_commit(&barM2);
       }
+    } else if (tid == 64 && more) {
+      issue_U(c - 1);  // dU_loc^T consumed
     }
-    ok = __syncthreads_and(mbar_wait(&barM, phM, err));
+    okt = okt && mbar_wait(&barM2, phM, err);
     phM ^= 1;
     ph ^= 1;
     tc_fence_after();
-    if (!ok) break;
-    if (tid == 0 && more) {  // W^T, Q, dO consumed
+    if (tid == 64 && more) {  // W^T, Q, dO consumed
       issue_W(c - 1);
       issue_QO(c - 1);
     }
     {
-      const float eg = expf(sG[63]);
+      const float eg = sEGC[buf];
       float d[64];
       tmem_ld64(taddr(tb, 32 * (warp & 3), 64 + 64 * half), d);
       tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < 64; ++i) S[i] = eg * S[i] + d[i];
     }
-    if (tid == 0) tma_store_wait_read0();  // the dh store has finished reading dS hi
-    __syncthreads();
     for (int j = 0; j < 8; ++j) st_chunk_split(sSH, sSL, v, half * 8 + j, TILE128, &S[8 * j]);
     if (tid < 64 && more) {
-      const int Ln = min(64, sq.w - 64 * (c - 1));
-      sG[tid] = gnext;
-      sEG[tid] = tid < Ln ? p.scale * expf(gnext) : 0.f;
+      sDecb[(buf ^ 1) * 64 + tid] = dn;
+      sEGb[(buf ^ 1) * 64 + tid] = en;
+      if (tid == 63) sEGC[buf ^ 1] = egc;
     }
     fence_proxy_async();
     tc_fence_before();
-    __syncthreads();
-    if (tid < 64 && more) sDec[tid] = expf(sG[63] - sG[tid]);
-    __syncthreads();
+    ok = __syncthreads_and(ok && okt);
     tc_fence_after();
+    if (!ok) break;
   }
-  if (tid == 0) tma_store_wait0();
+  if (tid == 32) tma_store_wait0();
   if (ok && a.dh0)
     for (int i = 0; i < 64; ++i) a.dh0[st + (size_t)(half * 64 + i) * D + v] = S[i];
   tc_fence_before();
