@@ -203,42 +203,43 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
 }
 
 // ======================================================================================
-// Sequential state scan.  One CTA (256 threads) per (sequence, value head).  Thread
-// (v = 32*(warp%4) + lane, half = warp/4) keeps S[v][64*half .. 64*half+63] in fp32
-// registers.  Per chunk:
-//   MMA1: D1 = S_bf16 W^T          (M=128 v, N=64 i, K=128 k)
-//   U^T = U~^T - D1; Ud^T = U^T diag(e^{G_C-G})  (bf16 tiles in smem)
-//   MMA2: D2 = Ud^T K              (M=128 v, N=128 k, K=64 i)
-//   S = e^{G_C} S + D2
-// S (bf16, the state entering each chunk) and U^T are written out by TMA stores; the
-// chunk's W^T, U~^T and K tiles are prefetched one chunk ahead (double buffer).
+// Sequential state scan.  The rows of S (value index v) evolve independently: row v of
+//   U = U~ - W S^T   and   S' = e^{G_C} S + U^T diag(e^{G_C-G}) K
+// only involves row v of S and column v of U~.  So the scan is split over value slices:
+// CTA (sequence, value head, z) carries rows v0 = 32z .. v0+31 (4 CTAs per head), which
+// quarters the work on each chunk step of the sequential chain and fills 4x more SMs.
+// The products are taken transposed, so that the 32-row slice is the N side:
+//   MMA1: D1 = W S_z^T           (M=64 i, N=32 v, K=128 k)     W^T tile as MN-major A
+//   U = U~ - D1;  Ud = diag(e^{G_C-G}) U      (bf16 [32 v][64 i] tiles, K-major B)
+//   MMA2: D2 = K^T Ud            (M=128 k, N=32 v, K=64 i)     K tile as MN-major A
+//   S_z^T = e^{G_C} S_z^T + D2   (thread k keeps S[v0..v0+31][k] in fp32 registers)
+// 128 threads: thread 0 issues the MMAs, thread 32 the TMA stores (and waits on them; bulk
+// groups are per thread), thread 64 the TMA loads; two CTA-wide barriers per chunk step.
+// The slice of S entering each chunk and the slice of U^T are written out by TMA stores;
+// the chunk's W^T, U~^T slice and K tiles are prefetched one chunk ahead (double buffer).
 // ======================================================================================
 struct ScanSmem {
-  static constexpr int S = 0;                       // 2 x [128][128] bf16 (alternating chunks)
-  static constexpr int BUF = 4 * TILE128;           // 2 x {W^T 16K, U~^T 16K, K 16K}
-  static constexpr int BUF_BYTES = 3 * TILE128;
-  static constexpr int UD = BUF + 2 * BUF_BYTES;    // [128][64] Ud^T
-  static constexpr int UO = UD + TILE128;           // 2 x [128][64] U^T staging
-  static constexpr int DEC = UO + 2 * TILE128;      // 2 x 64 floats e^{G_C - G_i}
-  static constexpr int EGC = DEC + 2 * 256;         // 2 floats e^{G_C}
+  static constexpr int BUF = 0;                               // 2 x {W^T, K, U~^T slice}
+  static constexpr int BUF_BYTES = 2 * TILE128 + TILE_VS;
+  static constexpr int S = 2 * BUF_BYTES;                     // 2 x [32][128] bf16 state slice
+  static constexpr int UD = S + 4 * TILE_VS;                  // [32][64] Ud^T slice
+  static constexpr int UO = UD + TILE_VS;                     // 2 x [32][64] U^T staging
+  static constexpr int DEC = UO + 2 * TILE_VS;                // 2 x 64 floats e^{G_C - G_i}
+  static constexpr int EGC = DEC + 2 * 256;                   // 2 floats e^{G_C}
   static constexpr int TOTAL = EGC + 64;
 };
 
-// Roles inside the scan CTAs: thread 0 issues the tensor-core MMAs, thread 32 the TMA stores
-// (and waits on them; bulk-copy groups are per thread), thread 64 the TMA loads.  Every
-// thread waits on the mbarriers itself; a chunk step has two CTA-wide barriers.
-__global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, TcWork t,
+__global__ void __launch_bounds__(128) k_tc_scan_fwd(Problem p, Args a, Work w, TcWork t,
                                                      const __grid_constant__ CUtensorMap mk,
                                                      const __grid_constant__ CUtensorMap mWT,
-                                                     const __grid_constant__ CUtensorMap mUtT,
-                                                     const __grid_constant__ CUtensorMap mUT,
-                                                     const __grid_constant__ CUtensorMap mh,
+                                                     const __grid_constant__ CUtensorMap mUtT32,
+                                                     const __grid_constant__ CUtensorMap mUT32,
+                                                     const __grid_constant__ CUtensorMap mh32,
                                                      int write_final) {
   if (failed(w)) return;
-  const int n = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
+  const int n = blockIdx.x, hv = blockIdx.y, hk = hv / p.G, v0 = VS * blockIdx.z;
   const int4 sq = w.seq_tab[n];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int v = 32 * (warp & 3) + lane, half = warp >> 2;
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
   unsigned char* sUd = sm + ScanSmem::UD;
@@ -256,91 +257,107 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
   }
   __syncthreads();
   if (warp == 0) {
-    tmem_alloc(&tslot, 256);
+    tmem_alloc(&tslot, 64);
     tmem_relinquish();
   }
-  // initial state (fp32) -> registers; bf16 copy -> state buffer 0
-  float S[64];
-  const size_t st = ((size_t)n * p.HV + hv) * D * D;  // [K][V] fp32 states
-  for (int i = 0; i < 64; ++i) {
-    const int kk = half * 64 + i;
-    S[i] = a.h0 ? a.h0[st + (size_t)kk * D + v] : 0.f;
+  // thread k = tid holds S[v0 + i][k], i < 32 (initial state h0[k][v] = S[v][k], fp32)
+  float S[VS];
+  const size_t st = ((size_t)n * p.HV + hv) * D * D + (size_t)tid * D + v0;
+#pragma unroll
+  for (int i = 0; i < VS; i += 4) {
+    const float4 x = a.h0 ? *reinterpret_cast<const float4*>(a.h0 + st + i) : make_float4(0, 0, 0, 0);
+    S[i] = x.x; S[i + 1] = x.y; S[i + 2] = x.z; S[i + 3] = x.w;
   }
-  for (int j = 0; j < 8; ++j) st_chunk_f(sm + ScanSmem::S, v, half * 8 + j, TILE128, &S[8 * j]);
+  // element (v, k) of a [32][128] slice tile: the thread's column k, rows i < 32
+  const uint32_t scol = (uint32_t)((tid >> 6) * TILE_VS + ((tid & 7) << 1));
+  const int sj = (tid & 63) >> 3;
+#define S_OFF(i) (scol + (uint32_t)((i) * 128 + (((sj) ^ ((i) & 7)) << 4)))
+#pragma unroll
+  for (int i = 0; i < VS; ++i) st_bf16(sm + ScanSmem::S, S_OFF(i), S[i]);
   auto issue = [&](int c) {
     const int gc = sq.x + c, buf = c & 1;
     const int tok = sq.z + 64 * c;  // chunks of a sequence are consecutive, 64 tokens apart
     unsigned char* b = sm + ScanSmem::BUF + buf * ScanSmem::BUF_BYTES;
     const int row = (gc * p.HV + hv) * D;
-    mbar_expect_tx(&barT[buf], 3 * TILE128);
+    mbar_expect_tx(&barT[buf], 2 * TILE128 + TILE_VS);
     tma_load_3d(b, &mWT, 0, row, 0, &barT[buf]);
-    tma_load_3d(b + TILE128, &mUtT, 0, row, 0, &barT[buf]);
-    tma_load_3d(b + 2 * TILE128, &mk, 0, hk, tok, &barT[buf]);
-    tma_load_3d(b + 2 * TILE128 + TILE64, &mk, 64, hk, tok, &barT[buf]);
+    tma_load_3d(b + TILE128, &mk, 0, hk, tok, &barT[buf]);
+    tma_load_3d(b + TILE128 + TILE64, &mk, 64, hk, tok, &barT[buf]);
+    tma_load_3d(b + 2 * TILE128, &mUtT32, 0, row + v0, 0, &barT[buf]);
   };
   const size_t vec0 = ((size_t)hv * p.NCmax + sq.x) * 64;  // chunk vectors of this sequence
   if (tid == 64 && sq.y > 0) issue(0);
-  if (tid < 64 && sq.y > 0) sDecb[tid] = w.Dec[vec0 + tid];
-  if (tid == 0 && sq.y > 0) sEGC[0] = w.EG[vec0 + 63];
+  if (tid >= 64 && sq.y > 0) {
+    sDecb[tid - 64] = w.Dec[vec0 + tid - 64];
+    if (tid == 127) sEGC[0] = w.EG[vec0 + 63];
+  }
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
-  const uint32_t tD1 = taddr(tb, 0, 0), tD2 = taddr(tb, 0, 64);
+  const uint32_t tD1 = taddr(tb, 0, 0), tD2 = taddr(tb, 0, 32);
+  // U-phase element mapping (16-lane TMEM loads of the M=64 accumulator): rows
+  // i = 16 warp + lane/4 (+8), columns v = 8j + 2(lane%4) + {0,1}
+  const int ui = 16 * warp + (lane >> 2), uv = 2 * (lane & 3);
   uint32_t phT[2] = {0, 0}, phM = 0;
   bool ok = true;
   for (int c = 0; c < sq.y; ++c) {
     const int gc = sq.x + c, buf = c & 1;
     const bool more = c + 1 < sq.y;
     unsigned char* b = sm + ScanSmem::BUF + buf * ScanSmem::BUF_BYTES;
-    unsigned char* sS = sm + ScanSmem::S + buf * 2 * TILE128;       // S entering chunk c
-    unsigned char* sSn = sm + ScanSmem::S + (buf ^ 1) * 2 * TILE128;
-    unsigned char* sUo = sm + ScanSmem::UO + buf * TILE128;
+    unsigned char* sS = sm + ScanSmem::S + buf * 2 * TILE_VS;       // S slice entering chunk c
+    unsigned char* sSn = sm + ScanSmem::S + (buf ^ 1) * 2 * TILE_VS;
+    unsigned char* sUo = sm + ScanSmem::UO + buf * TILE_VS;
     const float* sDec = sDecb + buf * 64;
-    const uint32_t unit_row = (uint32_t)(gc * p.HV + hv) * D;
+    const int srow = (gc * p.HV + hv) * D + v0;
     bool okt = true;
-    if (tid == 0) {  // MMA1: D1 = S W^T
+    if (tid == 0) {  // MMA1: D1 = W S_z^T
       okt = mbar_wait(&barT[buf], phT[buf], err);
       if (okt) {
-        const uint32_t s_ = smem_u32(sS), wt = smem_u32(b);
+        const uint64_t da = desc_mnmajor(smem_u32(b), 0, TILE128);
+        const uint64_t db = desc_kmajor(smem_u32(sS), 0, TILE_VS);
+        constexpr uint32_t id = idesc_bf16(64, VS, true, false);
+#pragma unroll
         for (int s = 0; s < 8; ++s)
-          mma_bf16(tD1, desc_kmajor(s_, s, TILE128), desc_mnmajor(wt, s, TILE128),
-                   idesc_bf16(128, 64, false, true), s > 0);
+          mma_bf16(tD1, da + mnstep_off(s), db + kstep_off(s, TILE_VS), id, s > 0);
         mma_commit(&barM1);
       }
-    } else if (tid == 32) {  // S entering this chunk -> h
-      tma_store_3d(&mh, sS, 0, unit_row, 0);
-      tma_store_3d(&mh, sS + TILE128, 64, unit_row, 0);
+    } else if (tid == 32) {  // S slice entering this chunk -> h
+      tma_store_3d(&mh32, sS, 0, srow, 0);
+      tma_store_3d(&mh32, sS + TILE_VS, 64, srow, 0);
       tma_store_commit();
     } else if (tid == 64 && more) {
       issue(c + 1);
     }
     float dn = 0.f, en = 0.f;  // next chunk's decay vectors, stored at the end of this step
-    if (tid < 64 && more) {
-      dn = w.Dec[vec0 + (size_t)(c + 1) * 64 + tid];
-      if (tid == 0) en = w.EG[vec0 + (size_t)(c + 1) * 64 + 63];
+    if (tid >= 64 && more) {
+      dn = w.Dec[vec0 + (size_t)(c + 1) * 64 + tid - 64];
+      if (tid == 127) en = w.EG[vec0 + (size_t)(c + 1) * 64 + 63];
     }
     okt = okt && mbar_wait(&barT[buf], phT[buf], err);
     phT[buf] ^= 1;
     okt = okt && mbar_wait(&barM1, phM, err);
     tc_fence_after();
-    // U^T = U~^T - D1 for columns [32*half, 32*half+32); Ud^T = U^T * e^{G_C - G}
-    {
-      float d[32];
-      tmem_ld16(taddr(tb, 32 * (warp & 3), 32 * half), d);
-      tmem_ld16(taddr(tb, 32 * (warp & 3), 32 * half + 16), d + 16);
+    {  // U = U~ - D1 -> U^T staging; Ud = e^{G_C-G_i} U -> MMA2 operand
+      float d[16];
+      tmem_ld16dp_x4(taddr(tb, 32 * warp, 0), d);
       tmem_wait_ld();
-      const unsigned char* ut = b + TILE128;
-      for (int j = 0; j < 4; ++j) {
-        float u[8], ud[8];
-        ld_chunk_f(ut, v, half * 4 + j, TILE128, u);
-        for (int q = 0; q < 8; ++q) {
-          u[q] -= d[8 * j + q];
-          ud[q] = u[q] * sDec[32 * half + 8 * j + q];
-        }
-        st_chunk_f(sUo, v, half * 4 + j, TILE128, u);
-        st_chunk_f(sUd, v, half * 4 + j, TILE128, ud);
+      const unsigned char* ut = b + 2 * TILE128;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int i = ui + 8 * r;
+        const float dec = sDec[i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int vv = 8 * j + uv + e;
+            const uint32_t off = sw128(vv, i, TILE_VS);
+            const float u = ld_bf16(ut, off) - d[4 * j + 2 * r + e];
+            st_bf16(sUo, off, u);
+            st_bf16(sUd, off, u * dec);
+          }
       }
     }
     // the stores of chunk c-1 (h and U^T) must be done reading before the barrier below
@@ -351,14 +368,16 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
     ok = __syncthreads_and(ok && okt);
     tc_fence_after();
     if (!ok) break;
-    if (tid == 0) {  // MMA2: D2 = Ud^T K
-      const uint32_t ud = smem_u32(sUd), kt = smem_u32(b + 2 * TILE128);
+    if (tid == 0) {  // MMA2: D2 = K^T Ud
+      const uint64_t da = desc_mnmajor(smem_u32(b + TILE128), 0, TILE64);
+      const uint64_t db = desc_kmajor(smem_u32(sUd), 0, TILE_VS);
+      constexpr uint32_t id = idesc_bf16(128, VS, true, false);
+#pragma unroll
       for (int s = 0; s < 4; ++s)
-        mma_bf16(tD2, desc_kmajor(ud, s, TILE128), desc_mnmajor(kt, s, TILE64),
-                 idesc_bf16(128, 128, false, true), s > 0);
+        mma_bf16(tD2, da + mnstep_off(s), db + kstep_off(s, TILE_VS), id, s > 0);
       mma_commit(&barM2);
     } else if (tid == 32) {
-      tma_store_3d(&mUT, sUo, 0, unit_row, 0);
+      tma_store_3d(&mUT32, sUo, 0, srow, 0);
       tma_store_commit();
     }
     okt = mbar_wait(&barM2, phM, err);
@@ -366,18 +385,19 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
     tc_fence_after();
     {
       const float eg = sEGC[buf];
-      float d[64];
-      tmem_ld64(taddr(tb, 32 * (warp & 3), 64 + 64 * half), d);
+      float d[VS];
+      tmem_ld16(taddr(tb, 32 * warp, 32), d);
+      tmem_ld16(taddr(tb, 32 * warp, 48), d + 16);
       tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 64; ++i) S[i] = eg * S[i] + d[i];
+      for (int i = 0; i < VS; ++i) {
+        S[i] = eg * S[i] + d[i];
+        st_bf16(sSn, S_OFF(i), S[i]);  // its last reader, the h store of chunk c-1, is done
+      }
     }
-    // the next chunk's state goes to the other buffer (its last reader, the h store of chunk
-    // c-1, finished before the mid-step barrier)
-    for (int j = 0; j < 8; ++j) st_chunk_f(sSn, v, half * 8 + j, TILE128, &S[8 * j]);
-    if (tid < 64 && more) {
-      sDecb[(buf ^ 1) * 64 + tid] = dn;
-      if (tid == 0) sEGC[buf ^ 1] = en;
+    if (tid >= 64 && more) {
+      sDecb[(buf ^ 1) * 64 + tid - 64] = dn;
+      if (tid == 127) sEGC[buf ^ 1] = en;
     }
     fence_proxy_async();
     tc_fence_before();
@@ -385,12 +405,16 @@ __global__ void __launch_bounds__(256) k_tc_scan_fwd(Problem p, Args a, Work w, 
     tc_fence_after();
     if (!ok) break;
   }
+#undef S_OFF
   if (tid == 32) tma_store_wait0();
-  if (ok && write_final && a.ht)
-    for (int i = 0; i < 64; ++i) a.ht[st + (size_t)(half * 64 + i) * D + v] = S[i];
+  if (ok && write_final && a.ht) {
+#pragma unroll
+    for (int i = 0; i < VS; i += 4)
+      *reinterpret_cast<float4*>(a.ht + st + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
+  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tslot, 256);
+  if (warp == 0) tmem_dealloc(tslot, 64);
 }
 
 // ======================================================================================
@@ -541,6 +565,9 @@ Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
   L.ok &= map_rows(&L.m.UtT, L.t.UtT, urows, 64, 128);
   L.ok &= map_rows(&L.m.UT, L.t.UT, urows, 64, 128);
   L.ok &= map_rows(&L.m.h, L.t.h, urows, 128, 128);
+  L.ok &= map_rows(&L.m.UtT32, L.t.UtT, urows, 64, VS);
+  L.ok &= map_rows(&L.m.UT32, L.t.UT, urows, 64, VS);
+  L.ok &= map_rows(&L.m.h32, L.t.h, urows, 128, VS);
   if (pass == 1) {
     const uint64_t trows = (uint64_t)p.NCmax * p.HV * 64;
     L.ok &= map_rows(&L.m.dUlT, L.t.dUlT, urows, 64, 128);
@@ -549,6 +576,10 @@ Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
     L.ok &= map_rows(&L.m.dh, L.t.dh, urows, 128, 128);
     L.ok &= map_rows(&L.m.dW, L.t.dW, trows, 128, 64);
     L.ok &= map_rows(&L.m.Tm, L.t.Tm, 2 * trows, 64, 64);
+    L.ok &= map_rows(&L.m.dUlT32, L.t.dUlT, urows, 64, VS);
+    L.ok &= map_rows(&L.m.dUT32, L.t.dUT, urows, 64, VS);
+    L.ok &= map_rows(&L.m.dUTl32, L.t.dUTl, urows, 64, VS);
+    L.ok &= map_rows(&L.m.dh32, L.t.dh, urows, 128, VS);
   }
   return L;
 }
@@ -557,12 +588,12 @@ cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const L
                          bool bwd_prep, cudaStream_t s) {
   if (!L.ok) return cudaErrorInvalidValue;
   cudaError_t e;
-  const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV);
+  const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV, NVS);
   if ((e = tgo("tc_wy", k_tc_wy, gu, 256, (size_t)1024 + WySmem::TOTAL, s, p, w, L.t, L.m.k, L.m.v, 1)))
     return e;
   Args a2 = a;
-  if ((e = tgo("tc_scan_fwd", k_tc_scan_fwd, gs, 256, (size_t)1024 + ScanSmem::TOTAL, s, p, a2, w,
-              L.t, L.m.k, L.m.WT, L.m.UtT, L.m.UT, L.m.h, bwd_prep ? 0 : 1)))
+  if ((e = tgo("tc_scan_fwd", k_tc_scan_fwd, gs, 128, (size_t)1024 + ScanSmem::TOTAL, s, p, a2, w,
+              L.t, L.m.k, L.m.WT, L.m.UtT32, L.m.UT32, L.m.h32, bwd_prep ? 0 : 1)))
     return e;
   if (!bwd_prep) {
     const size_t out_smem = 1024 + 6 * TILE64 + 3 * TILE128 + 256;

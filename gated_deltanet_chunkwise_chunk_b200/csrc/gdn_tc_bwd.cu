@@ -135,53 +135,55 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
 }
 
 // ======================================================================================
-// Reverse state scan.  One CTA (256 threads) per (sequence, value head); thread
-// (v = 32*(warp%4)+lane, half = warp/4) keeps dS[v][64*half..+63] in fp32 registers.  The
-// tensor-core operands that carry the chain (dS and -dU^T) are compensated bf16 pairs
-// (hi + lo), and dU^T is written out as such a pair.  Tiles are single-buffered: each
+// Reverse state scan.  As in the forward, the rows v of dS evolve independently, so CTA
+// (sequence, value head, z) carries the slice dS[v0 .. v0+31][:] (v0 = 32z), with the
+// products taken transposed (the slice is the N side).  Thread k keeps dS[v0+i][k] (i < 32)
+// in fp32 registers.  The operands that carry the chain (dS and dU) are compensated bf16
+// pairs (hi + lo), and dU^T is written out as such a pair.  Tiles are single-buffered: each
 // group is reloaded for the next chunk as soon as its last reader is done.
-//   MMA2a (off the chain): F  = (scale diag(e^G) dO)^T Q        (M=128 v, N=128 k, K=64 i)
-//   MMA1:                   E  = dS K^T                         (M=128 v, N=64 j,  K=128 k)
-//   dU^T = dU_loc^T + E diag(e^{G_C-G})
-//   MMA2b:                  F -= dU^T W                         (M=128 v, N=128 k, K=64 j)
-//   dS = e^{G_C} dS + F
+//   MMA1:  E = K dS_z^T                                (M=64 j, N=32 v, K=128 k)
+//   dU = dU_loc + diag(e^{G_C-G}) E                    (bf16 hi/lo [32 v][64 j] tiles)
+//   MMA2:  F' = Q^T (-scale diag(e^G) dO_z) + W^T dU   (M=128 k, N=32 v, K=64 i)
+//   dS_z^T = e^{G_C} dS_z^T - F'
 // ======================================================================================
 struct BwdScanSmem {
-  static constexpr int SH = 0, SL = 2 * TILE128;                 // dS hi / lo [128][128]
-  static constexpr int K = 4 * TILE128, Q = K + 2 * TILE64, O = Q + 2 * TILE64;
-  static constexpr int W = O + 2 * TILE64, UL = W + TILE128;     // W^T, dU_loc^T [128][64]
-  static constexpr int ATH = UL + TILE128, ATL = ATH + TILE128;  // -dU^T hi / lo
-  static constexpr int DEC = ATL + TILE128;                      // 2 x 64: e^{G_C - G_j}
-  static constexpr int EG = DEC + 512;                           // 2 x 64: scale e^{G_i} (0 past L)
-  static constexpr int EGC = EG + 512;                           // 2 floats e^{G_C}
+  static constexpr int K = 0, Q = 2 * TILE64, O = 4 * TILE64;  // [64][128], [64][128], [64][64]
+  static constexpr int W = 5 * TILE64;                          // W^T [128][64]
+  static constexpr int UL = W + TILE128;                        // dU_loc^T slice [32][64]
+  static constexpr int SH = UL + TILE_VS, SL = SH + 2 * TILE_VS;  // dS slice hi / lo [32][128]
+  static constexpr int OS = SL + 2 * TILE_VS;                   // -scale e^G dO^T slice [32][64]
+  static constexpr int UH = OS + TILE_VS, ULO = UH + 2 * TILE_VS;  // 2 x dU^T hi / lo [32][64]
+  static constexpr int DEC = ULO + 2 * TILE_VS;                 // 2 x 64: e^{G_C - G_j}
+  static constexpr int EG = DEC + 512;                          // 2 x 64: scale e^{G_i} (0 past L)
+  static constexpr int EGC = EG + 512;                          // 2 floats e^{G_C}
   static constexpr int TOTAL = EGC + 64;
 };
 
 // Roles as in the forward scan: thread 0 MMAs, thread 32 TMA stores, thread 64 TMA loads;
 // two CTA-wide barriers per chunk step.
-__global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, TcWork t,
+__global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, TcWork t,
                                                      const __grid_constant__ CUtensorMap mq,
                                                      const __grid_constant__ CUtensorMap mk,
                                                      const __grid_constant__ CUtensorMap mdO,
                                                      const __grid_constant__ CUtensorMap mWT,
-                                                     const __grid_constant__ CUtensorMap mdUlT,
-                                                     const __grid_constant__ CUtensorMap mdh) {
+                                                     const __grid_constant__ CUtensorMap mdUlT32,
+                                                     const __grid_constant__ CUtensorMap mdUT32,
+                                                     const __grid_constant__ CUtensorMap mdUTl32,
+                                                     const __grid_constant__ CUtensorMap mdh32) {
   if (failed(w)) return;
-  const int n = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
+  const int n = blockIdx.x, hv = blockIdx.y, hk = hv / p.G, v0 = VS * blockIdx.z;
   const int4 sq = w.seq_tab[n];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int v = 32 * (warp & 3) + lane, half = warp >> 2;
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
-  unsigned char* sSH = sm + BwdScanSmem::SH;
-  unsigned char* sSL = sm + BwdScanSmem::SL;
   unsigned char* sK = sm + BwdScanSmem::K;
   unsigned char* sQ = sm + BwdScanSmem::Q;
   unsigned char* sO = sm + BwdScanSmem::O;
   unsigned char* sW = sm + BwdScanSmem::W;
   unsigned char* sUL = sm + BwdScanSmem::UL;
-  unsigned char* sATH = sm + BwdScanSmem::ATH;
-  unsigned char* sATL = sm + BwdScanSmem::ATL;
+  unsigned char* sSH = sm + BwdScanSmem::SH;
+  unsigned char* sSL = sm + BwdScanSmem::SL;
+  unsigned char* sOS = sm + BwdScanSmem::OS;
   float* sDecb = reinterpret_cast<float*>(sm + BwdScanSmem::DEC);
   float* sEGb = reinterpret_cast<float*>(sm + BwdScanSmem::EG);
   float* sEGC = reinterpret_cast<float*>(sm + BwdScanSmem::EGC);
@@ -199,34 +201,49 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
   }
   __syncthreads();
   if (warp == 0) {
-    tmem_alloc(&tslot, 256);
+    tmem_alloc(&tslot, 64);
     tmem_relinquish();
   }
-  float S[64];
-  const size_t st = ((size_t)n * p.HV + hv) * D * D;
-  for (int i = 0; i < 64; ++i) S[i] = a.dht ? a.dht[st + (size_t)(half * 64 + i) * D + v] : 0.f;
-  for (int j = 0; j < 8; ++j) st_chunk_split(sSH, sSL, v, half * 8 + j, TILE128, &S[8 * j]);
+  float S[VS];
+  const size_t st = ((size_t)n * p.HV + hv) * D * D + (size_t)tid * D + v0;
+#pragma unroll
+  for (int i = 0; i < VS; i += 4) {
+    const float4 x = a.dht ? *reinterpret_cast<const float4*>(a.dht + st + i) : make_float4(0, 0, 0, 0);
+    S[i] = x.x; S[i + 1] = x.y; S[i + 2] = x.z; S[i + 3] = x.w;
+  }
+  const uint32_t scol = (uint32_t)((tid >> 6) * TILE_VS + ((tid & 7) << 1));
+  const int sj = (tid & 63) >> 3;
+#define S_OFF(i) (scol + (uint32_t)((i) * 128 + (((sj) ^ ((i) & 7)) << 4)))
+  auto store_dS = [&]() {
+#pragma unroll
+    for (int i = 0; i < VS; ++i) {
+      const bf16 h = __float2bfloat16_rn(S[i]);
+      st_bf16_raw(sSH, S_OFF(i), h);
+      st_bf16_raw(sSL, S_OFF(i), __float2bfloat16_rn(S[i] - __bfloat162float(h)));
+    }
+  };
+  store_dS();
   auto row_of = [&](int c) { return ((sq.x + c) * p.HV + hv) * D; };
   auto tok_of = [&](int c) { return sq.z + 64 * c; };
+  const int ocol = v0 & ~63, vo = v0 & 63;  // dO column block holding the slice, offset in it
   auto issue_K = [&](int c) {
     mbar_expect_tx(&barK, 2 * TILE64);
     tma_load_3d(sK, &mk, 0, hk, tok_of(c), &barK);
     tma_load_3d(sK + TILE64, &mk, 64, hk, tok_of(c), &barK);
   };
   auto issue_QO = [&](int c) {
-    mbar_expect_tx(&barQO, 4 * TILE64);
+    mbar_expect_tx(&barQO, 3 * TILE64);
     tma_load_3d(sQ, &mq, 0, hk, tok_of(c), &barQO);
     tma_load_3d(sQ + TILE64, &mq, 64, hk, tok_of(c), &barQO);
-    tma_load_3d(sO, &mdO, 0, hv, tok_of(c), &barQO);
-    tma_load_3d(sO + TILE64, &mdO, 64, hv, tok_of(c), &barQO);
+    tma_load_3d(sO, &mdO, ocol, hv, tok_of(c), &barQO);
   };
   auto issue_W = [&](int c) {
     mbar_expect_tx(&barW, TILE128);
     tma_load_3d(sW, &mWT, 0, row_of(c), 0, &barW);
   };
   auto issue_U = [&](int c) {
-    mbar_expect_tx(&barU, TILE128);
-    tma_load_3d(sUL, &mdUlT, 0, row_of(c), 0, &barU);
+    mbar_expect_tx(&barU, TILE_VS);
+    tma_load_3d(sUL, &mdUlT32, 0, row_of(c) + v0, 0, &barU);
   };
   const size_t vec0 = ((size_t)hv * p.NCmax + sq.x) * 64;  // chunk vectors of this sequence
   auto len_of = [&](int c) { return min(64, sq.w - 64 * c); };
@@ -236,102 +253,106 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     issue_W(sq.y - 1);
     issue_U(sq.y - 1);
   }
-  if (tid < 64 && sq.y > 0) {
-    const int c = sq.y - 1;
-    const size_t o = vec0 + (size_t)c * 64 + tid;
-    sDecb[tid] = w.Dec[o];
-    sEGb[tid] = tid < len_of(c) ? p.scale * w.EG[o] : 0.f;
-    if (tid == 63) sEGC[0] = w.EG[o];
+  if (tid >= 64 && sq.y > 0) {
+    const int c = sq.y - 1, j = tid - 64;
+    const size_t o = vec0 + (size_t)c * 64 + j;
+    sDecb[j] = w.Dec[o];
+    const float eg = w.EG[o];
+    sEGb[j] = j < len_of(c) ? p.scale * eg : 0.f;
+    if (j == 63) sEGC[0] = eg;
   }
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
-  const uint32_t tE = taddr(tb, 0, 0), tF = taddr(tb, 0, 64);
+  const uint32_t tE = taddr(tb, 0, 0), tF = taddr(tb, 0, 32);
+  const int ui = 16 * warp + (lane >> 2), uv = 2 * (lane & 3);
   uint32_t ph = 0, phM = 0;  // the tile barriers complete once per chunk, barM1/barM2 once each
   bool ok = true;
   for (int idx = 0; idx < sq.y; ++idx) {
     const int c = sq.y - 1 - idx, buf = idx & 1;
     const bool more = idx + 1 < sq.y;
     const int L = len_of(c);
-    const uint32_t unit_row = (uint32_t)row_of(c);
+    const int srow = row_of(c) + v0;
     const float* sDec = sDecb + buf * 64;
     const float* sEG = sEGb + buf * 64;
+    unsigned char* sUH = sm + BwdScanSmem::UH + buf * TILE_VS;
+    unsigned char* sULo = sm + BwdScanSmem::ULO + buf * TILE_VS;
     bool okt = true;
     if (L < 64) {  // ragged chunk: K rows past its end are zeroed before the chain MMA
       okt = mbar_wait(&barK, ph, err);
-      zero_tail_rows(sK, L, tid, 256);
+      zero_tail_rows(sK, L, tid, 128);
       fence_proxy_async();
       __syncthreads();
     }
-    if (tid == 0) {  // MMA1 (the chain): E = dS K^T with the compensated dS pair
+    if (tid == 0) {  // MMA1 (the chain): E = K dS_z^T with the compensated dS pair
       okt = okt && mbar_wait(&barK, ph, err);
       if (okt) {
-        const uint32_t k = smem_u32(sK);
-        for (int part = 0; part < 2; ++part) {
-          const uint32_t sa = smem_u32(part ? sSL : sSH);
-          for (int s = 0; s < 8; ++s)
-            mma_bf16(tE, desc_kmajor(sa, s, TILE128), desc_kmajor(k, s, TILE64),
-                     idesc_bf16(128, 64, false, false), part > 0 || s > 0);
-        }
+        const uint64_t dk = desc_kmajor(smem_u32(sK), 0, TILE64);
+        const uint64_t dh = desc_kmajor(smem_u32(sSH), 0, TILE_VS);
+        const uint64_t dl = desc_kmajor(smem_u32(sSL), 0, TILE_VS);
+        constexpr uint32_t id = idesc_bf16(64, VS, false, false);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          mma_bf16(tE, dk + kstep_off(s, TILE64), dh + kstep_off(s, TILE_VS), id, s > 0);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          mma_bf16(tE, dk + kstep_off(s, TILE64), dl + kstep_off(s, TILE_VS), id, 1);
         mma_commit(&barM1);
       }
-    } else if (tid == 32) {  // dS leaving this chunk -> dh
-      tma_store_3d(&mdh, sSH, 0, unit_row, 0);
-      tma_store_3d(&mdh, sSH + TILE128, 64, unit_row, 0);
+    } else if (tid == 32) {  // dS slice leaving this chunk -> dh
+      tma_store_3d(&mdh32, sSH, 0, srow, 0);
+      tma_store_3d(&mdh32, sSH + TILE_VS, 64, srow, 0);
       tma_store_commit();
     }
     float dn = 0.f, en = 0.f, egc = 0.f;  // next chunk's vectors, stored at the end of the step
-    if (tid < 64 && more) {
-      const size_t o = vec0 + (size_t)(c - 1) * 64 + tid;
+    if (tid >= 64 && more) {
+      const int j = tid - 64;
+      const size_t o = vec0 + (size_t)(c - 1) * 64 + j;
       dn = w.Dec[o];
       const float eg = w.EG[o];
-      en = tid < len_of(c - 1) ? p.scale * eg : 0.f;
+      en = j < len_of(c - 1) ? p.scale * eg : 0.f;
       egc = eg;
     }
-    // off the chain while MMA1 runs: dO rows scaled by scale e^{G_i} (zero past L)
+    // off the chain while MMA1 runs: -scale e^{G_i} dO[i][v0+v] -> [32 v][64 i] (0 past L)
     okt = okt && mbar_wait(&barQO, ph, err);
-    for (int i = tid; i < 64 * 16; i += 256) {
-      const int r = i / 16, j = i % 16;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int task = tid + 128 * r, i = task & 63, cq = task >> 6;
       float f[8];
-      ld_chunk_f(sO, r, j, TILE64, f);
-      for (int q = 0; q < 8; ++q) f[q] *= sEG[r];
-      st_chunk_f(sO, r, j, TILE64, f);
+      ld_chunk_f(sO, i, (vo >> 3) + cq, TILE64, f);
+      const float sc = -sEG[i];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) st_bf16(sOS, sw128(8 * cq + e, i, TILE_VS), f[e] * sc);
     }
-    fence_proxy_async();
     okt = okt && mbar_wait(&barM1, phM, err);
     tc_fence_after();
     if (tid == 64 && more) issue_K(c - 1);  // K consumed by MMA1
     okt = okt && mbar_wait(&barU, ph, err);
     {
-      float d[32];
-      tmem_ld16(taddr(tb, 32 * (warp & 3), 32 * half), d);
-      tmem_ld16(taddr(tb, 32 * (warp & 3), 32 * half + 16), d + 16);
+      float d[16];
+      tmem_ld16dp_x4(taddr(tb, 32 * warp, 0), d);
       tmem_wait_ld();
-      bf16* hi_row = t.dUT + ((size_t)unit_row + v) * 64 + 32 * half;
-      bf16* lo_row = t.dUTl + ((size_t)unit_row + v) * 64 + 32 * half;
-      for (int j = 0; j < 4; ++j) {
-        float u[8], nu[8], hl[8], ll[8];
-        ld_chunk_f(sUL, v, half * 4 + j, TILE128, u);
-        for (int q = 0; q < 8; ++q) {
-          u[q] += sDec[32 * half + 8 * j + q] * d[8 * j + q];
-          nu[q] = -u[q];
-          hl[q] = __bfloat162float(__float2bfloat16_rn(u[q]));
-          ll[q] = u[q] - hl[q];
-        }
-        st_chunk_split(sATH, sATL, v, half * 4 + j, TILE128, nu);
-        uint4 ph4, pl4;
-        ph4.x = pack_bf16(hl[0], hl[1]); ph4.y = pack_bf16(hl[2], hl[3]);
-        ph4.z = pack_bf16(hl[4], hl[5]); ph4.w = pack_bf16(hl[6], hl[7]);
-        pl4.x = pack_bf16(ll[0], ll[1]); pl4.y = pack_bf16(ll[2], ll[3]);
-        pl4.z = pack_bf16(ll[4], ll[5]); pl4.w = pack_bf16(ll[6], ll[7]);
-        *reinterpret_cast<uint4*>(hi_row + 8 * j) = ph4;
-        *reinterpret_cast<uint4*>(lo_row + 8 * j) = pl4;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int i = ui + 8 * r;
+        const float dec = sDec[i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int vv = 8 * j + uv + e;
+            const uint32_t off = sw128(vv, i, TILE_VS);
+            const float u = ld_bf16(sUL, off) + dec * d[4 * j + 2 * r + e];
+            const bf16 h = __float2bfloat16_rn(u);
+            st_bf16_raw(sUH, off, h);
+            st_bf16_raw(sULo, off, __float2bfloat16_rn(u - __bfloat162float(h)));
+          }
       }
     }
     // the dh store of this chunk must be done reading dS before the barrier releases the
-    // dS update below
+    // dS update below, and the dU^T store of chunk c+1 before its staging is rewritten
     if (tid == 32) tma_store_wait_read0();
     fence_proxy_async();
     tc_fence_before();
@@ -341,18 +362,28 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     if (tid == 0) {
       okt = mbar_wait(&barW, ph, err);
       if (okt) {
-        const uint32_t o = smem_u32(sO), q = smem_u32(sQ), wt = smem_u32(sW);
-        for (int s = 0; s < 4; ++s)  // F = (scale diag(e^G) dO)^T Q
-          mma_bf16(tF, desc_mnmajor(o, s, TILE64), desc_mnmajor(q, s, TILE64),
-                   idesc_bf16(128, 128, true, true), s > 0);
-        for (int part = 0; part < 2; ++part) {  // F -= dU^T W
-          const uint32_t at = smem_u32(part ? sATL : sATH);
-          for (int s = 0; s < 4; ++s)
-            mma_bf16(tF, desc_kmajor(at, s, TILE128), desc_kmajor(wt, s, TILE128),
-                     idesc_bf16(128, 128, false, false), 1);
-        }
+        const uint64_t dQ_ = desc_mnmajor(smem_u32(sQ), 0, TILE64);
+        const uint64_t dOS = desc_kmajor(smem_u32(sOS), 0, TILE_VS);
+        const uint64_t dW_ = desc_kmajor(smem_u32(sW), 0, TILE128);
+        const uint64_t dH_ = desc_kmajor(smem_u32(sUH), 0, TILE_VS);
+        const uint64_t dL_ = desc_kmajor(smem_u32(sULo), 0, TILE_VS);
+        constexpr uint32_t idQ = idesc_bf16(128, VS, true, false);
+        constexpr uint32_t idW = idesc_bf16(128, VS, false, false);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)  // F' = Q^T (-scale diag(e^G) dO_z)
+          mma_bf16(tF, dQ_ + mnstep_off(s), dOS + kstep_off(s, TILE_VS), idQ, s > 0);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)  // F' += W^T dU  (hi and lo parts)
+          mma_bf16(tF, dW_ + kstep_off(s, TILE128), dH_ + kstep_off(s, TILE_VS), idW, 1);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+          mma_bf16(tF, dW_ + kstep_off(s, TILE128), dL_ + kstep_off(s, TILE_VS), idW, 1);
         mma_commit(&barM2);
       }
+    } else if (tid == 32) {  // dU^T of this chunk (hi, lo) -> global
+      tma_store_3d(&mdUT32, sUH, 0, srow, 0);
+      tma_store_3d(&mdUTl32, sULo, 0, srow, 0);
+      tma_store_commit();
     } else if (tid == 64 && more) {
       issue_U(c - 1);  // dU_loc^T consumed
     }
@@ -366,17 +397,19 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     }
     {
       const float eg = sEGC[buf];
-      float d[64];
-      tmem_ld64(taddr(tb, 32 * (warp & 3), 64 + 64 * half), d);
+      float d[VS];
+      tmem_ld16(taddr(tb, 32 * warp, 32), d);
+      tmem_ld16(taddr(tb, 32 * warp, 48), d + 16);
       tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 64; ++i) S[i] = eg * S[i] + d[i];
+      for (int i = 0; i < VS; ++i) S[i] = eg * S[i] - d[i];
     }
-    for (int j = 0; j < 8; ++j) st_chunk_split(sSH, sSL, v, half * 8 + j, TILE128, &S[8 * j]);
-    if (tid < 64 && more) {
-      sDecb[(buf ^ 1) * 64 + tid] = dn;
-      sEGb[(buf ^ 1) * 64 + tid] = en;
-      if (tid == 63) sEGC[buf ^ 1] = egc;
+    store_dS();
+    if (tid >= 64 && more) {
+      const int j = tid - 64;
+      sDecb[(buf ^ 1) * 64 + j] = dn;
+      sEGb[(buf ^ 1) * 64 + j] = en;
+      if (j == 63) sEGC[buf ^ 1] = egc;
     }
     fence_proxy_async();
     tc_fence_before();
@@ -384,12 +417,16 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     tc_fence_after();
     if (!ok) break;
   }
+#undef S_OFF
   if (tid == 32) tma_store_wait0();
-  if (ok && a.dh0)
-    for (int i = 0; i < 64; ++i) a.dh0[st + (size_t)(half * 64 + i) * D + v] = S[i];
+  if (ok && a.dh0) {
+#pragma unroll
+    for (int i = 0; i < VS; i += 4)
+      *reinterpret_cast<float4*>(a.dh0 + st + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
+  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tslot, 256);
+  if (warp == 0) tmem_dealloc(tslot, 64);
 }
 
 // ======================================================================================
@@ -980,12 +1017,12 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
 cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, const TcWork& t,
                                 const TcMaps& m, cudaStream_t s) {
   cudaError_t e;
-  const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV);
+  const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV, NVS);
   if ((e = tgo("tc_dvlocal", k_tc_dvlocal, gu, 128, 1024 + 8 * TILE64 + 256, s, p, w, t, m.q, m.k,
                m.dO)))
     return e;
-  if ((e = tgo("tc_scan_bwd", k_tc_scan_bwd, gs, 256, 1024 + BwdScanSmem::TOTAL, s, p, a, w, t, m.q,
-               m.k, m.dO, m.WT, m.dUlT, m.dh)))
+  if ((e = tgo("tc_scan_bwd", k_tc_scan_bwd, gs, 128, 1024 + BwdScanSmem::TOTAL, s, p, a, w, t, m.q,
+               m.k, m.dO, m.WT, m.dUlT32, m.dUT32, m.dUTl32, m.dh32)))
     return e;
   if ((e = tgo("tc_dqkwg", k_tc_dqkwg, gu, 256, 1024 + DqkSmem::TOTAL, s, p, w, t, m.q, m.k, m.dO,
                m.UT, m.dUT, m.dUTl, m.h, m.dh, m.dW)))

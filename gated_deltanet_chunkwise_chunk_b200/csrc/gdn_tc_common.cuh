@@ -17,6 +17,9 @@ using namespace tc;
 constexpr int D = 128;                 // head dimension (K = V = 128 on this path)
 constexpr int TILE64 = 64 * 128;       // bytes of a [64 rows x 64 bf16] block
 constexpr int TILE128 = 128 * 128;     // bytes of a [128 rows x 64 bf16] block
+constexpr int VS = 32;                 // value rows of the state carried by one scan CTA
+constexpr int NVS = D / VS;            // scan CTAs per (sequence, value head)
+constexpr int TILE_VS = VS * 128;      // bytes of a [32 rows x 64 bf16] block
 
 // ------------------------------------------------------------------ tensor maps (host)
 typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -69,6 +72,8 @@ struct TcMaps {
   CUtensorMap dh;                     // [unit*128][128]     (backward)
   CUtensorMap dW;                     // [unit*64][128]      (backward)
   CUtensorMap Tm;                     // [unit*64][64]       (backward)
+  // the same [unit*128][..] arrays with 32-row boxes (one value slice of the scans)
+  CUtensorMap UtT32, UT32, h32, dUlT32, dUT32, dUTl32, dh32;
 };
 
 struct TcWork {
@@ -133,6 +138,17 @@ __device__ __forceinline__ void zero_tail_rows(unsigned char* tile, int L, int t
     const int r = L + i / 16, j = i % 16;
     *reinterpret_cast<uint4*>(tile + sw128_chunk(r, j, TILE64)) = make_uint4(0, 0, 0, 0);
   }
+}
+
+// One bf16 element of a tile at byte offset off (from sw128).
+__device__ __forceinline__ void st_bf16(unsigned char* tile, uint32_t off, float x) {
+  *reinterpret_cast<bf16*>(tile + off) = __float2bfloat16_rn(x);
+}
+__device__ __forceinline__ void st_bf16_raw(unsigned char* tile, uint32_t off, bf16 x) {
+  *reinterpret_cast<bf16*>(tile + off) = x;
+}
+__device__ __forceinline__ float ld_bf16(const unsigned char* tile, uint32_t off) {
+  return __bfloat162float(*reinterpret_cast<const bf16*>(tile + off));
 }
 
 // Reads 8 bf16 (one 16-byte swizzled chunk) as floats.

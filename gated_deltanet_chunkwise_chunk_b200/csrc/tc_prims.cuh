@@ -151,6 +151,13 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int s, int block_
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int s, int block_bytes) {
   return sdesc(tile + (uint32_t)(s * 2048), (uint32_t)block_bytes, 1024);
 }
+// Descriptor step offsets (added to a descriptor; the start address field holds bytes / 16,
+// and addresses stay below 2^18 bytes, so the additions never carry out of the field).
+__host__ __device__ constexpr uint64_t kstep_off(int s, int block_bytes) {
+  return (uint64_t)(((s >> 2) * block_bytes + (s & 3) * 32) >> 4);
+}
+__host__ __device__ constexpr uint64_t mnstep_off(int s) { return (uint64_t)((s * 2048) >> 4); }
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
