@@ -300,6 +300,14 @@ __global__ void __launch_bounds__(128) k_tc_scan_fwd(Problem p, Args a, Work w, 
   // U-phase element mapping (16-lane TMEM loads of the M=64 accumulator): rows
   // i = 16 warp + lane/4 (+8), columns v = 8j + 2(lane%4) + {0,1}
   const int ui = 16 * warp + (lane >> 2), uv = 2 * (lane & 3);
+  // per-thread byte offsets of the U-phase elements in a [32][64] slice tile:
+  // element (v = 8j + uv + e, i = ui + 8r) sits at uoff[r][e] + 1024 j
+  uint32_t uoff[2][2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+      uoff[r][e] = (uint32_t)((uv + e) * 128 + (((2 * warp + r) ^ (uv + e)) << 4) + ((lane >> 2) << 1));
   uint32_t phT[2] = {0, 0}, phM = 0;
   bool ok = true;
   for (int c = 0; c < sq.y; ++c) {
@@ -308,7 +316,6 @@ __global__ void __launch_bounds__(128) k_tc_scan_fwd(Problem p, Args a, Work w, 
     unsigned char* b = sm + ScanSmem::BUF + buf * ScanSmem::BUF_BYTES;
     unsigned char* sS = sm + ScanSmem::S + buf * 2 * TILE_VS;       // S slice entering chunk c
     unsigned char* sSn = sm + ScanSmem::S + (buf ^ 1) * 2 * TILE_VS;
-    unsigned char* sUo = sm + ScanSmem::UO + buf * TILE_VS;
     const float* sDec = sDecb + buf * 64;
     const int srow = (gc * p.HV + hv) * D + v0;
     bool okt = true;
@@ -323,9 +330,10 @@ __global__ void __launch_bounds__(128) k_tc_scan_fwd(Problem p, Args a, Work w, 
           mma_bf16(tD1, da + mnstep_off(s), db + kstep_off(s, TILE_VS), id, s > 0);
         mma_commit(&barM1);
       }
-    } else if (tid == 32) {  // S slice entering this chunk -> h
+    } else if (tid == 32) {  // S slice entering this chunk -> h;  U^T slice of chunk c-1
       tma_store_3d(&mh32, sS, 0, srow, 0);
       tma_store_3d(&mh32, sS + TILE_VS, 64, srow, 0);
+      if (c > 0) tma_store_3d(&mUT32, sm + ScanSmem::UO + (buf ^ 1) * TILE_VS, 0, srow - p.HV * D, 0);
       tma_store_commit();
     } else if (tid == 64 && more) {
       issue(c + 1);
@@ -335,33 +343,39 @@ __global__ void __launch_bounds__(128) k_tc_scan_fwd(Problem p, Args a, Work w, 
       dn = w.Dec[vec0 + (size_t)(c + 1) * 64 + tid - 64];
       if (tid == 127) en = w.EG[vec0 + (size_t)(c + 1) * 64 + 63];
     }
+    // while MMA1 runs: this thread's U~ elements and decay factors
     okt = okt && mbar_wait(&barT[buf], phT[buf], err);
     phT[buf] ^= 1;
+    float u[16];
+    {
+      const unsigned char* ut = b + 2 * TILE128;
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) u[4 * j + 2 * r + e] = ld_bf16(ut, uoff[r][e] + 1024 * j);
+    }
+    const float dec0 = sDec[ui], dec1 = sDec[ui + 8];
     okt = okt && mbar_wait(&barM1, phM, err);
     tc_fence_after();
-    {  // U = U~ - D1 -> U^T staging; Ud = e^{G_C-G_i} U -> MMA2 operand
+    {  // U = U~ - D1 (kept for the U^T staging); Ud = e^{G_C-G_i} U -> MMA2 operand
       float d[16];
       tmem_ld16dp_x4(taddr(tb, 32 * warp, 0), d);
       tmem_wait_ld();
-      const unsigned char* ut = b + 2 * TILE128;
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int i = ui + 8 * r;
-        const float dec = sDec[i];
+      for (int r = 0; r < 2; ++r)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int vv = 8 * j + uv + e;
-            const uint32_t off = sw128(vv, i, TILE_VS);
-            const float u = ld_bf16(ut, off) - d[4 * j + 2 * r + e];
-            st_bf16(sUo, off, u);
-            st_bf16(sUd, off, u * dec);
+            const int q = 4 * j + 2 * r + e;
+            u[q] -= d[q];
+            st_bf16(sUd, uoff[r][e] + 1024 * j, u[q] * (r ? dec1 : dec0));
           }
-      }
     }
-    // the stores of chunk c-1 (h and U^T) must be done reading before the barrier below
-    // releases writes into their buffers (this step's next-state tile, the next U^T staging)
+    // the stores of chunk c-1 (h, and U^T of c-2) must be done reading before the barrier
+    // below releases writes into their buffers (the next-state tile, this U^T staging)
     if (tid == 32) tma_store_wait_read<1>();
     fence_proxy_async();
     tc_fence_before();
@@ -376,9 +390,15 @@ __global__ void __launch_bounds__(128) k_tc_scan_fwd(Problem p, Args a, Work w, 
       for (int s = 0; s < 4; ++s)
         mma_bf16(tD2, da + mnstep_off(s), db + kstep_off(s, TILE_VS), id, s > 0);
       mma_commit(&barM2);
-    } else if (tid == 32) {
-      tma_store_3d(&mUT32, sUo, 0, srow, 0);
-      tma_store_commit();
+    }
+    {  // while MMA2 runs: U^T staging (stored by TMA at the start of the next step)
+      unsigned char* sUo = sm + ScanSmem::UO + buf * TILE_VS;
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) st_bf16(sUo, uoff[r][e] + 1024 * j, u[4 * j + 2 * r + e]);
     }
     okt = mbar_wait(&barM2, phM, err);
     phM ^= 1;
@@ -406,7 +426,14 @@ __global__ void __launch_bounds__(128) k_tc_scan_fwd(Problem p, Args a, Work w, 
     if (!ok) break;
   }
 #undef S_OFF
-  if (tid == 32) tma_store_wait0();
+  if (tid == 32) {
+    if (ok && sq.y > 0) {  // U^T slice of the last chunk
+      const int c = sq.y - 1;
+      tma_store_3d(&mUT32, sm + ScanSmem::UO + (c & 1) * TILE_VS, 0, ((sq.x + c) * p.HV + hv) * D + v0, 0);
+      tma_store_commit();
+    }
+    tma_store_wait0();
+  }
   if (ok && write_final && a.ht) {
 #pragma unroll
     for (int i = 0; i < VS; i += 4)

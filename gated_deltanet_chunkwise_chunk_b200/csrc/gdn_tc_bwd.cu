@@ -268,6 +268,14 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
   const uint32_t tb = tslot;
   const uint32_t tE = taddr(tb, 0, 0), tF = taddr(tb, 0, 32);
   const int ui = 16 * warp + (lane >> 2), uv = 2 * (lane & 3);
+  // per-thread byte offsets of the U-phase elements in a [32][64] slice tile:
+  // element (v = 8j + uv + e, j' = ui + 8r) sits at uoff[r][e] + 1024 j
+  uint32_t uoff[2][2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+      uoff[r][e] = (uint32_t)((uv + e) * 128 + (((2 * warp + r) ^ (uv + e)) << 4) + ((lane >> 2) << 1));
   uint32_t ph = 0, phM = 0;  // the tile barriers complete once per chunk, barM1/barM2 once each
   bool ok = true;
   for (int idx = 0; idx < sq.y; ++idx) {
@@ -315,7 +323,8 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
       en = j < len_of(c - 1) ? p.scale * eg : 0.f;
       egc = eg;
     }
-    // off the chain while MMA1 runs: -scale e^{G_i} dO[i][v0+v] -> [32 v][64 i] (0 past L)
+    // off the chain while MMA1 runs: -scale e^{G_i} dO[i][v0+v] -> [32 v][64 i] (0 past L),
+    // then this thread's dU_loc elements and decay factors
     okt = okt && mbar_wait(&barQO, ph, err);
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
@@ -326,30 +335,48 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
 #pragma unroll
       for (int e = 0; e < 8; ++e) st_bf16(sOS, sw128(8 * cq + e, i, TILE_VS), f[e] * sc);
     }
+    okt = okt && mbar_wait(&barU, ph, err);
+    float u[16];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) u[4 * j + 2 * r + e] = ld_bf16(sUL, uoff[r][e] + 1024 * j);
+    const float dec0 = sDec[ui], dec1 = sDec[ui + 8];
+    // the scaled dO tile is complete: its product with Q^T (off the chain) queues behind MMA1
+    fence_proxy_async();
+    tc_fence_before();
+    okt = __syncthreads_and(okt);
+    tc_fence_after();
+    if (tid == 0 && okt) {
+      const uint64_t dQ_ = desc_mnmajor(smem_u32(sQ), 0, TILE64);
+      const uint64_t dOS = desc_kmajor(smem_u32(sOS), 0, TILE_VS);
+      constexpr uint32_t idQ = idesc_bf16(128, VS, true, false);
+#pragma unroll
+      for (int s = 0; s < 4; ++s)  // F' = Q^T (-scale diag(e^G) dO_z)
+        mma_bf16(tF, dQ_ + mnstep_off(s), dOS + kstep_off(s, TILE_VS), idQ, s > 0);
+    }
     okt = okt && mbar_wait(&barM1, phM, err);
     tc_fence_after();
     if (tid == 64 && more) issue_K(c - 1);  // K consumed by MMA1
-    okt = okt && mbar_wait(&barU, ph, err);
     {
       float d[16];
       tmem_ld16dp_x4(taddr(tb, 32 * warp, 0), d);
       tmem_wait_ld();
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int i = ui + 8 * r;
-        const float dec = sDec[i];
+      for (int r = 0; r < 2; ++r)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int vv = 8 * j + uv + e;
-            const uint32_t off = sw128(vv, i, TILE_VS);
-            const float u = ld_bf16(sUL, off) + dec * d[4 * j + 2 * r + e];
-            const bf16 h = __float2bfloat16_rn(u);
+            const int q = 4 * j + 2 * r + e;
+            const float x = u[q] + (r ? dec1 : dec0) * d[q];
+            const bf16 h = __float2bfloat16_rn(x);
+            const uint32_t off = uoff[r][e] + 1024 * j;
             st_bf16_raw(sUH, off, h);
-            st_bf16_raw(sULo, off, __float2bfloat16_rn(u - __bfloat162float(h)));
+            st_bf16_raw(sULo, off, __float2bfloat16_rn(x - __bfloat162float(h)));
           }
-      }
     }
     // the dh store of this chunk must be done reading dS before the barrier releases the
     // dS update below, and the dU^T store of chunk c+1 before its staging is rewritten
@@ -362,16 +389,10 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
     if (tid == 0) {
       okt = mbar_wait(&barW, ph, err);
       if (okt) {
-        const uint64_t dQ_ = desc_mnmajor(smem_u32(sQ), 0, TILE64);
-        const uint64_t dOS = desc_kmajor(smem_u32(sOS), 0, TILE_VS);
         const uint64_t dW_ = desc_kmajor(smem_u32(sW), 0, TILE128);
         const uint64_t dH_ = desc_kmajor(smem_u32(sUH), 0, TILE_VS);
         const uint64_t dL_ = desc_kmajor(smem_u32(sULo), 0, TILE_VS);
-        constexpr uint32_t idQ = idesc_bf16(128, VS, true, false);
         constexpr uint32_t idW = idesc_bf16(128, VS, false, false);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)  // F' = Q^T (-scale diag(e^G) dO_z)
-          mma_bf16(tF, dQ_ + mnstep_off(s), dOS + kstep_off(s, TILE_VS), idQ, s > 0);
 #pragma unroll
         for (int s = 0; s < 4; ++s)  // F' += W^T dU  (hi and lo parts)
           mma_bf16(tF, dW_ + kstep_off(s, TILE128), dH_ + kstep_off(s, TILE_VS), idW, 1);
