@@ -182,6 +182,42 @@ def oracle_sample(case, budget_s: float = 12.0) -> dict:
             "seconds": dt}
 
 
+# ----------------------------------------------------------------- ranks
+def init_dist(impl: str):
+    """One process per GPU, launched by torch.distributed.run (RANK / LOCAL_RANK /
+    WORLD_SIZE / MASTER_* from the environment).  Every rank runs its own batch; the only
+    collectives are the barriers around the timed region and the max over ranks of the
+    timings (NCCL for our arm, gloo for the host-only reference arm)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() and impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return rank, world, local, dist
+
+
+def max_over_ranks(values, dist, device) -> list[float]:
+    """Element-wise maximum over ranks (identity with one rank): a multi-GPU time is the
+    slowest rank's."""
+    if not dist:
+        return [float(x) for x in values]
+    tt = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return [float(x) for x in tt.tolist()]
+
+
+def aggregate_mtok_s(world: int, tokens_per_rank: int, ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank / (ms / 1e3) / 1e6
+
+
 # ----------------------------------------------------------------- our arm
 def main():
     ap = argparse.ArgumentParser()
@@ -192,22 +228,13 @@ def main():
     ap.add_argument("--config", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--ref-budget", type=float, default=90.0,
+                    help="seconds of oracle work over the whole --impl reference run")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        backend = "nccl" if torch.cuda.is_available() and args.impl == "ours" else "gloo"
-        if backend == "nccl":
-            torch.cuda.set_device(local)
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    rank, world, local, dist = init_dist(args.impl)
 
     if args.impl == "reference":
         return reference_arm(args, rank, world, dist)
@@ -270,10 +297,7 @@ def main():
     launches = gdn.launch_count() - n0
     clocks = sampler.stop()
     ms_fwd = timed(fwd, max(1, args.steps))
-    if dist:
-        tt = torch.tensor([ms, ms_fwd], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, ms_fwd = float(tt[0]), float(tt[1])
+    ms, ms_fwd = max_over_ranks([ms, ms_fwd], dist, dev)
 
     # per-kernel device time (separate pass: events around every launch on its stream)
     gdn.profile(True)
@@ -286,7 +310,7 @@ def main():
     e2e = e2e_measure(gdn, case, dev, ws, args.e2e_steps, dist)
 
     tokens = case.tokens
-    value = world * tokens / (ms / 1e3) / 1e6
+    value = aggregate_mtok_s(world, tokens, ms)
     pk = peaks()
     fflop, bflop = step_flops_per_token_head(case.K, case.V)
     th = tokens * case.HV
@@ -306,7 +330,7 @@ def main():
                    "K": case.K, "V": case.V, "chunk": C, "global_batch": case.B * world,
                    "seq_len": case.T, "parallelism": f"dp{world} (independent batches)",
                    "l2": "no flush: each step streams ~1 GB (inputs alone > 126 MB L2)"},
-        "fwd_mtok_s": round(world * tokens / (ms_fwd / 1e3) / 1e6, 3),
+        "fwd_mtok_s": round(aggregate_mtok_s(world, tokens, ms_fwd), 3),
         "ms_fwd": round(ms_fwd, 4),
         "step_roofline": {"flops": flops, "bytes": nbytes,
                           "frac_datasheet": round(t_roof_ds / (ms / 1e3), 4),
@@ -415,13 +439,9 @@ def e2e_measure(gdn, case, dev, ws, nsteps: int, dist) -> dict:
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / nsteps
-    world = 1
-    if dist:
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt[0])
-        world = dist.get_world_size()
-    return {"value": round(world * case.tokens / (ms / 1e3) / 1e6, 3), "unit": "M tokens/s",
+    (ms,) = max_over_ranks([ms], dist, dev)
+    world = dist.get_world_size() if dist else 1
+    return {"value": round(aggregate_mtok_s(world, case.tokens, ms), 3), "unit": "M tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(ms, 3)}
 
@@ -436,7 +456,7 @@ def reference_arm(args, rank, world, dist):
     from oracle import oracle
     oracle.build()
     samples = []
-    budget = max(2.0, 90.0 / max(1, args.steps + args.warmup))
+    budget = max(0.5, args.ref_budget / max(1, args.steps + args.warmup))
     info = None
     for i in range(args.warmup + args.steps):
         info = oracle_sample(case, budget_s=budget)
