@@ -37,7 +37,9 @@ struct WySmem {
 
 __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
                                                const __grid_constant__ CUtensorMap mk,
-                                               const __grid_constant__ CUtensorMap mv, int store_T) {
+                                               const __grid_constant__ CUtensorMap mv,
+                                               const __grid_constant__ CUtensorMap mWT,
+                                               const __grid_constant__ CUtensorMap mUtT, int store_T) {
   if (failed(w)) return;
   const int gc = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
   const int4 e = w.chunk_tab[gc];
@@ -107,22 +109,22 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
   tc_fence_after();
   if (ok) {
-    // M=64 accumulator: row 16*(warp%4) + lane (lanes 0..15); columns [32*half, +32)
-    float v[32];
-    tmem_ld16(taddr(tb, sub, 32 * half), v);
-    tmem_ld16(taddr(tb, sub, 32 * half + 16), v + 16);
+    // M=64 accumulator read with 16-lane loads: rows r0 = 16 (warp%4) + lane/4 and r0 + 8,
+    // columns 32 half + 8j + 2 (lane%4) + {0,1}
+    float v[16];
+    tmem_ld16dp_x4(taddr(tb, sub, 32 * half), v);
     tmem_wait_ld();
-    if (lane < 16) {
-      const int r = 16 * (warp & 3) + lane;
-      const float br = sb[r], gr = sG[r];
-      for (int i = 0; i < 32; ++i) {
-        const int cc = 32 * half + i;
-        sA[r * 65 + cc] = cc < r ? br * v[i] * expf(gr - sG[cc]) : 0.f;
+    const int r0 = 16 * (warp & 3) + (lane >> 2);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int r = r0 + 8 * (q >> 1), cc = 32 * half + 8 * j + 2 * (lane & 3) + (q & 1);
+        sA[r * 65 + cc] = cc < r ? sb[r] * v[4 * j + q] * __expf(sG[r] - sG[cc]) : 0.f;
       }
-    }
   }
   __syncthreads();
-  unit_lower_inverse64(sA, sT, sX, tid, 256);   // T = (I + A)^-1 (ends with a barrier)
+  unit_lower_inverse64(sA, sT, sX, tid);   // T = (I + A)^-1 (ends with a barrier)
   // bf16 operand tiles TX[i][j] = T[i][j] beta_j e^{G_j}, TY[i][j] = T[i][j] beta_j (hi + lo)
   bf16* tbase = t.Tm + ((size_t)gc * p.HV + hv) * 128 * 64;
   for (int idx = tid; idx < 64 * 8; idx += 256) {
@@ -176,26 +178,31 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
   tc_fence_after();
   if (ok) {
-    // row = feature index (k for W^T, v for U~^T); this thread's 32 token columns
+    // row = feature index (k for W^T, v for U~^T), this thread's 32 token columns; staged
+    // as [128][64] bf16 tiles in the (now free) TX/TY region and stored by TMA
     const int r = sub + lane;
-    const size_t unit = (size_t)gc * p.HV + hv;
-    bf16* wrow = t.WT + (unit * D + r) * 64 + 32 * half;
-    bf16* urow = t.UtT + (unit * D + r) * 64 + 32 * half;
+    unsigned char* sWst = sm + WySmem::R1;
+    unsigned char* sUst = sWst + TILE128;
     float x[32], y[32];
     tmem_ld16(taddr(tb, sub, 64 + 32 * half), x);
     tmem_ld16(taddr(tb, sub, 64 + 32 * half + 16), x + 16);
     tmem_ld16(taddr(tb, sub, 128 + 32 * half), y);
     tmem_ld16(taddr(tb, sub, 128 + 32 * half + 16), y + 16);
     tmem_wait_ld();
-    for (int c = 0; c < 32; c += 8) {
-      uint4 a, b;
-      a.x = pack_bf16(x[c], x[c + 1]); a.y = pack_bf16(x[c + 2], x[c + 3]);
-      a.z = pack_bf16(x[c + 4], x[c + 5]); a.w = pack_bf16(x[c + 6], x[c + 7]);
-      b.x = pack_bf16(y[c], y[c + 1]); b.y = pack_bf16(y[c + 2], y[c + 3]);
-      b.z = pack_bf16(y[c + 4], y[c + 5]); b.w = pack_bf16(y[c + 6], y[c + 7]);
-      *reinterpret_cast<uint4*>(wrow + c) = a;
-      *reinterpret_cast<uint4*>(urow + c) = b;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      st_chunk_f(sWst, r, 4 * half + j, TILE128, x + 8 * j);
+      st_chunk_f(sUst, r, 4 * half + j, TILE128, y + 8 * j);
     }
+    fence_proxy_async();
+  }
+  __syncthreads();
+  if (ok && tid == 0) {
+    const int row = (gc * p.HV + hv) * D;
+    tma_store_3d(&mWT, sm + WySmem::R1, 0, row, 0);
+    tma_store_3d(&mUtT, sm + WySmem::R1 + TILE128, 0, row, 0);
+    tma_store_commit();
+    tma_store_wait_read0();
   }
   tc_fence_before();
   __syncthreads();
@@ -616,7 +623,8 @@ cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const L
   if (!L.ok) return cudaErrorInvalidValue;
   cudaError_t e;
   const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV, NVS);
-  if ((e = tgo("tc_wy", k_tc_wy, gu, 256, (size_t)1024 + WySmem::TOTAL, s, p, w, L.t, L.m.k, L.m.v, 1)))
+  if ((e = tgo("tc_wy", k_tc_wy, gu, 256, (size_t)1024 + WySmem::TOTAL, s, p, w, L.t, L.m.k, L.m.v,
+               L.m.WT, L.m.UtT, 1)))
     return e;
   Args a2 = a;
   if ((e = tgo("tc_scan_fwd", k_tc_scan_fwd, gs, 128, (size_t)1024 + ScanSmem::TOTAL, s, p, a2, w,

@@ -187,51 +187,96 @@ __device__ __forceinline__ void st_chunk_split(unsigned char* hi, unsigned char*
   st_chunk_f(lo, r, j, block_bytes, l);
 }
 
-// T = (I + A)^-1 for a strictly lower-triangular 64x64 fp32 A (row stride 65) by 16x16
-// blocks, with nthr >= 128 threads: the four diagonal blocks by forward substitution (warps
-// 0..3, one column per lane), then the block sub-diagonals d = 1, 2, 3 as
-// T[b+d][b] = -T[b+d][b+d] * sum_{k=b}^{b+d-1} A[b+d][k] T[k][b].   sX: [64][65] scratch.
-__device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT, float* sX, int tid,
-                                                     int nthr = 128) {
+// T = (I + A)^-1 for a strictly lower-triangular 64x64 fp32 A (row stride 65), 256 threads.
+// The four diagonal 16x16 blocks by forward substitution (warps 0..3, one column per lane)
+// while warps 4..7 zero the strictly upper 16-blocks; then the blocks below the diagonal by
+// block back-substitution, using [[L00, 0], [A10, L11]]^-1 = [[T00, 0], [-T11 A10 T00, T11]]:
+//   16-blocks of each 32x32 half:  T10 = -T11 (A10 T00)        (both halves at once)
+//   32-blocks:                     T[32:,:32] = -T[32:,32:] (A[32:,:32] T[:32,:32])
+// Each thread owns several outputs of a product (fully unrolled dot products).  sX: [64][65].
+__device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT, float* sX, int tid) {
   const int w = tid >> 5, lane = tid & 31;
-  for (int i = tid; i < 64 * 64; i += nthr) {  // zero the strictly upper blocks
-    const int r = i >> 6, c = i & 63;
-    if ((c >> 4) > (r >> 4)) sT[r * 65 + c] = 0.f;
-  }
-  if (w < 4 && lane < 16) {
-    const int b0 = 16 * w, c = lane;
-    float col[16];
+  if (w < 4) {
+    if (lane < 16) {
+      const int b0 = 16 * w, c = lane;
+      float col[16];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      float s = (r == c) ? 1.f : 0.f;
+      for (int r = 0; r < 16; ++r) {
+        float s = (r == c) ? 1.f : 0.f;
 #pragma unroll
-      for (int j = 0; j < r; ++j) s -= sA[(b0 + r) * 65 + b0 + j] * col[j];
-      col[r] = (r >= c) ? s : 0.f;
+        for (int j = 0; j < r; ++j) s -= sA[(b0 + r) * 65 + b0 + j] * col[j];
+        col[r] = (r >= c) ? s : 0.f;
+      }
+#pragma unroll
+      for (int r = 0; r < 16; ++r) sT[(b0 + r) * 65 + b0 + c] = col[r];
     }
-#pragma unroll
-    for (int r = 0; r < 16; ++r) sT[(b0 + r) * 65 + b0 + c] = col[r];
+  } else {
+    for (int i = tid - 128; i < 6 * 256; i += 128) {  // blocks (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+      const int blk = i >> 8, r = (i >> 4) & 15, c = i & 15;
+      const int br = blk < 3 ? 0 : (blk < 5 ? 1 : 2), bc = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+      sT[(16 * br + r) * 65 + 16 * bc + c] = 0.f;
+    }
   }
   __syncthreads();
-  for (int d = 1; d < 4; ++d) {
-    const int nblk = 4 - d;
-    for (int e = tid; e < nblk * 256; e += nthr) {
-      const int b = e >> 8, r = (e >> 4) & 15, c = e & 15;
-      const int R = 16 * (b + d) + r, Cc = 16 * b + c;
-      float s = 0.f;
-      for (int j = 16 * b; j < 16 * (b + d); ++j) s += sA[R * 65 + j] * sT[j * 65 + Cc];
-      sX[R * 65 + Cc] = s;
-    }
-    __syncthreads();
-    for (int e = tid; e < nblk * 256; e += nthr) {
-      const int b = e >> 8, r = (e >> 4) & 15, c = e & 15;
-      const int R = 16 * (b + d) + r, Cc = 16 * b + c, D0 = 16 * (b + d);
-      float s = 0.f;
+  {  // X = A10 T00 in each half p: rows 16(2p+1)+r, columns 32p + c, 32p + c + 8
+    const int p = tid >> 7, q = tid & 127, r = q >> 3, c = q & 7;
+    const int R = 16 * (2 * p + 1) + r, C0 = 32 * p + c;
+    const float* a = sA + R * 65 + 32 * p;
+    const float* t = sT + (32 * p) * 65 + C0;
+    float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-      for (int m = 0; m < 16; ++m) s += sT[R * 65 + D0 + m] * sX[(D0 + m) * 65 + Cc];
-      sT[R * 65 + Cc] = -s;
+    for (int j = 0; j < 16; ++j) {
+      const float av = a[j];
+      x0 += av * t[j * 65];
+      x1 += av * t[j * 65 + 8];
     }
-    __syncthreads();
+    sX[R * 65 + C0] = x0;
+    sX[R * 65 + C0 + 8] = x1;
   }
+  __syncthreads();
+  {  // T10 = -T11 X
+    const int p = tid >> 7, q = tid & 127, r = q >> 3, c = q & 7;
+    const int D0 = 16 * (2 * p + 1), R = D0 + r, C0 = 32 * p + c;
+    const float* tt = sT + R * 65 + D0;
+    const float* x = sX + D0 * 65 + C0;
+    float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const float tv = tt[m];
+      y0 += tv * x[m * 65];
+      y1 += tv * x[m * 65 + 8];
+    }
+    sT[R * 65 + C0] = -y0;
+    sT[R * 65 + C0 + 8] = -y1;
+  }
+  __syncthreads();
+  const int r2 = tid >> 3, c2 = tid & 7, R2 = 32 + r2;  // rows 32 + r2, columns c2 + 8q (q < 4)
+  {  // X = A[32:,:32] T[:32,:32]
+    const float* a = sA + R2 * 65;
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float av = a[j];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) x[q] += av * sT[j * 65 + c2 + 8 * q];
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) sX[R2 * 65 + c2 + 8 * q] = x[q];
+  }
+  __syncthreads();
+  {  // T[32:,:32] = -T[32:,32:] X
+    const float* tt = sT + R2 * 65 + 32;
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+      const float tv = tt[m];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) y[q] += tv * sX[(32 + m) * 65 + c2 + 8 * q];
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) sT[R2 * 65 + c2 + 8 * q] = -y[q];
+  }
+  __syncthreads();
 }
 
 // Two adjacent bf16 columns (c even) of row r as one 32-bit store, hi and lo parts.
