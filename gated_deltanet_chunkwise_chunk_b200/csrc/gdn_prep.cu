@@ -125,10 +125,9 @@ __global__ void __launch_bounds__(256) k_gate_cumsum(Problem p, Args a, Work w) 
 
 // ---------------------------------------------------------------------------------------
 // Backward assembly per chunk: dg = reverse in-chunk cumsum of dG (the gradient of
-// G = cumsum g), optional d g_raw through the gate, and dq/dk as the sum of the value
-// heads' shares over each k-head's group.
+// G = cumsum g) and the optional d g_raw through the gate (one warp per value head); then
+// dq/dk as the sum of the value heads' shares over each k-head's group.
 // ---------------------------------------------------------------------------------------
-template <typename T>
 __global__ void __launch_bounds__(256) k_bwd_tokens(Problem p, Args a, Work w) {
   if (call_failed(w)) return;
   const int gc = blockIdx.x;
@@ -159,20 +158,34 @@ __global__ void __launch_bounds__(256) k_bwd_tokens(Problem p, Args a, Work w) {
       }
     }
   }
+}
+
+// dq, dk of k-head h for one chunk: sums of the per-value-head shares over the G value heads
+// of the group (fp32 [chunk][hv][64][K] -> [token][h][K]), four columns per thread and step.
+template <typename T>
+__global__ void __launch_bounds__(256) k_dqdk_group_sum(Problem p, Args a, Work w) {
+  if (call_failed(w)) return;
+  const int gc = blockIdx.x, h = blockIdx.y;
+  const int4 e = w.chunk_tab[gc];
+  if (e.x < 0) return;
+  const int L = e.z, tok0 = e.w, K = p.K;
   T* dq = static_cast<T*>(a.dq);
   T* dk = static_cast<T*>(a.dk);
-  const int K = p.K;
-  for (int i = threadIdx.x; i < L * p.H * K; i += blockDim.x) {
-    const int t = i / (p.H * K), r = i % (p.H * K), h = r / K, c = r % K;
-    float sq = 0.f, sk = 0.f;
+  const size_t base = ((size_t)gc * p.HV + (size_t)h * p.G) * CH * K;  // value head h*G, row 0
+  for (int i = 4 * threadIdx.x; i < L * K; i += 4 * blockDim.x) {
+    float4 sq = make_float4(0.f, 0.f, 0.f, 0.f), sk = sq;
     for (int j = 0; j < p.G; ++j) {
-      const size_t o = (((size_t)gc * p.HV + h * p.G + j) * CH + t) * K + c;
-      sq += w.dqp[o];
-      sk += w.dkp[o];
+      const size_t o = base + (size_t)j * CH * K + i;
+      const float4 x = *reinterpret_cast<const float4*>(w.dqp + o);
+      const float4 y = *reinterpret_cast<const float4*>(w.dkp + o);
+      sq.x += x.x; sq.y += x.y; sq.z += x.z; sq.w += x.w;
+      sk.x += y.x; sk.y += y.y; sk.z += y.z; sk.w += y.w;
     }
-    const size_t oo = ((size_t)(tok0 + t) * p.H + h) * K + c;
-    dq[oo] = from_f<T>(sq);
-    dk[oo] = from_f<T>(sk);
+    const int t = i / K, c = i % K;
+    T* q4 = dq + ((size_t)(tok0 + t) * p.H + h) * K + c;
+    T* k4 = dk + ((size_t)(tok0 + t) * p.H + h) * K + c;
+    q4[0] = from_f<T>(sq.x); q4[1] = from_f<T>(sq.y); q4[2] = from_f<T>(sq.z); q4[3] = from_f<T>(sq.w);
+    k4[0] = from_f<T>(sk.x); k4[1] = from_f<T>(sk.y); k4[2] = from_f<T>(sk.z); k4[3] = from_f<T>(sk.w);
   }
 }
 
@@ -246,13 +259,19 @@ cudaError_t launch_bwd_tokens(const Problem& p, const Args& a, const Work& w, bo
   }
   {
     ProfScope ps("bwd_tokens", s);
-    if (bf16)
-      k_bwd_tokens<__nv_bfloat16><<<p.NCmax, 256, 0, s>>>(p, a, w);
-    else
-      k_bwd_tokens<float><<<p.NCmax, 256, 0, s>>>(p, a, w);
+    k_bwd_tokens<<<p.NCmax, 256, 0, s>>>(p, a, w);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  {
+    ProfScope ps("dqdk_group_sum", s);
+    const dim3 g(p.NCmax, p.H);
+    if (bf16)
+      k_dqdk_group_sum<__nv_bfloat16><<<g, 256, 0, s>>>(p, a, w);
+    else
+      k_dqdk_group_sum<float><<<g, 256, 0, s>>>(p, a, w);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.dA_log || a.ddt_bias) {
     ProfScope ps("param_grads", s);
     k_param_grads<<<p.HV, 256, 0, s>>>(p, a, w);
