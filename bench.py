@@ -228,6 +228,8 @@ def main():
     ap.add_argument("--config", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--T", type=int, default=None,
+                    help="override the sequence length of a dense workload (smaller profiling cases)")
     ap.add_argument("--ref-budget", type=float, default=90.0,
                     help="seconds of oracle work over the whole --impl reference run")
     args = ap.parse_args()
@@ -243,7 +245,7 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    case = synth.config_case(args.config, seed=1000 + args.config + 7919 * rank)
+    case = synth.config_case(args.config, seed=1000 + args.config + 7919 * rank, T=args.T)
     e = 2 if case.dtype == "bf16" else 4
     t = lambda x: None if x is None else x.to(dev).contiguous()
     inp = dict(q=t(case.q), k=t(case.k), v=t(case.v), g_raw=t(case.a), A_log=t(case.A_log),

@@ -480,10 +480,7 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
                                                   const __grid_constant__ CUtensorMap mdh,
                                                   const __grid_constant__ CUtensorMap mdW) {
   if (failed(w)) return;
-  const int gc = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
-  const int4 e = w.chunk_tab[gc];
-  if (e.x < 0) return;
-  const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int half = warp >> 2, sub = 32 * (warp & 3);
   const int r0 = 16 * (warp & 3) + lane / 4, r1 = r0 + 8, cq = 2 * (lane & 3);
   extern __shared__ unsigned char smraw[];
@@ -502,13 +499,15 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
   float* sG = reinterpret_cast<float*>(sm + DqkSmem::G);
   float* sRow = reinterpret_cast<float*>(sm + DqkSmem::ROW);  // [kind][half][64]
   float* sRed = reinterpret_cast<float*>(sm + DqkSmem::RED);
-  __shared__ uint64_t bar[2];
+  // barA: Q, K, U^T of a unit;  barB: dO, dU^T (hi, lo), S, dS';  barM: MMA batches
+  __shared__ uint64_t barA, barB, barM;
   __shared__ uint32_t tslot;
   int* err = w.status;
-  const size_t unit = (size_t)gc * p.HV + hv;
+  const int nunits = p.NCmax * p.HV;
   if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+    mbar_init(&barA, 1);
+    mbar_init(&barB, 1);
+    mbar_init(&barM, 1);
     mbar_fence_init();
   }
   __syncthreads();
@@ -516,200 +515,252 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
     tmem_alloc(&tslot, 512);
     tmem_relinquish();
   }
-  if (tid == 0) {
-    const int row = (int)unit * D;
-    mbar_expect_tx(&bar[0], DqkSmem::LOAD_BYTES);
-    tma_load_3d(sQ, &mq, 0, hk, tok0, &bar[0]);
-    tma_load_3d(sQ + TILE64, &mq, 64, hk, tok0, &bar[0]);
-    tma_load_3d(sK, &mk, 0, hk, tok0, &bar[0]);
-    tma_load_3d(sK + TILE64, &mk, 64, hk, tok0, &bar[0]);
-    tma_load_3d(sO, &mdO, 0, hv, tok0, &bar[0]);
-    tma_load_3d(sO + TILE64, &mdO, 64, hv, tok0, &bar[0]);
-    tma_load_3d(sUT, &mUT, 0, row, 0, &bar[0]);
-    tma_load_3d(sdUT, &mdUT, 0, row, 0, &bar[0]);
-    tma_load_3d(sdUTl, &mdUTl, 0, row, 0, &bar[0]);
-    tma_load_3d(sH, &mh, 0, row, 0, &bar[0]);
-    tma_load_3d(sH + TILE128, &mh, 64, row, 0, &bar[0]);
-    tma_load_3d(sdH, &mdh, 0, row, 0, &bar[0]);
-    tma_load_3d(sdH + TILE128, &mdh, 64, row, 0, &bar[0]);
+  // units u = gc * HV + hv in order; chunk-table entries past the chunk count are invalid
+  auto valid = [&](int u) { return u < nunits && w.chunk_tab[u / p.HV].x >= 0; };
+  auto load_A = [&](int u) {
+    const int gc = u / p.HV, hk = (u % p.HV) / p.G, tok0 = w.chunk_tab[gc].w;
+    mbar_expect_tx(&barA, 4 * TILE64 + TILE128);
+    tma_load_3d(sQ, &mq, 0, hk, tok0, &barA);
+    tma_load_3d(sQ + TILE64, &mq, 64, hk, tok0, &barA);
+    tma_load_3d(sK, &mk, 0, hk, tok0, &barA);
+    tma_load_3d(sK + TILE64, &mk, 64, hk, tok0, &barA);
+    tma_load_3d(sUT, &mUT, 0, u * D, 0, &barA);
+  };
+  auto load_B = [&](int u) {
+    const int gc = u / p.HV, hv = u % p.HV, tok0 = w.chunk_tab[gc].w;
+    mbar_expect_tx(&barB, 2 * TILE64 + 6 * TILE128);
+    tma_load_3d(sO, &mdO, 0, hv, tok0, &barB);
+    tma_load_3d(sO + TILE64, &mdO, 64, hv, tok0, &barB);
+    tma_load_3d(sdUT, &mdUT, 0, u * D, 0, &barB);
+    tma_load_3d(sdUTl, &mdUTl, 0, u * D, 0, &barB);
+    tma_load_3d(sH, &mh, 0, u * D, 0, &barB);
+    tma_load_3d(sH + TILE128, &mh, 64, u * D, 0, &barB);
+    tma_load_3d(sdH, &mdh, 0, u * D, 0, &barB);
+    tma_load_3d(sdH + TILE128, &mdh, 64, u * D, 0, &barB);
+  };
+  int u = blockIdx.x;
+  // parity of a load group issued and not yet waited on, or -1 (thread 0 issues all loads)
+  int pendA = -1, pendB = -1;
+  if (tid == 0 && valid(u)) {
+    load_A(u);
+    load_B(u);
+    pendA = pendB = 0;
   }
-  if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
-  bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
-  if (L < 64) {
-    zero_tail_rows(sQ, L, tid, 256);
-    zero_tail_rows(sK, L, tid, 256);
-    zero_tail_rows(sO, L, tid, 256);
-  }
-  fence_proxy_async();
-  __syncthreads();
-  if (ok && tid == 0) {
-    const uint32_t q = smem_u32(sQ), k = smem_u32(sK), o = smem_u32(sO), ut = smem_u32(sUT),
-                   dut = smem_u32(sdUT), dutl = smem_u32(sdUTl), h = smem_u32(sH), dh = smem_u32(sdH);
-    for (int s = 0; s < 8; ++s) {
-      const uint32_t acc = s > 0;
-      mma_bf16(taddr(tb, 0, 0), desc_kmajor(q, s, TILE64), desc_kmajor(k, s, TILE64),
-               idesc_bf16(64, 64, false, false), acc);
-      mma_bf16(taddr(tb, 0, 64), desc_kmajor(o, s, TILE64), desc_mnmajor(ut, s, TILE128),
-               idesc_bf16(64, 64, false, true), acc);
-      mma_bf16(taddr(tb, 0, 128), desc_kmajor(o, s, TILE64), desc_mnmajor(h, s, TILE128),
-               idesc_bf16(64, 128, false, true), acc);
-      mma_bf16(taddr(tb, 0, 256), desc_mnmajor(ut, s, TILE128), desc_mnmajor(dh, s, TILE128),
-               idesc_bf16(64, 128, true, true), acc);
-      mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dut, s, TILE128), desc_mnmajor(h, s, TILE128),
-               idesc_bf16(64, 128, true, true), acc);
+  bool ok = true;
+  for (uint32_t it = 0; valid(u); ++it, u += gridDim.x) {
+    const int gc = u / p.HV, hv = u % p.HV;
+    const int4 e = w.chunk_tab[gc];
+    const int L = e.z;
+    const size_t unit = (size_t)u;
+    const int nu = u + gridDim.x;
+    const bool nvalid = valid(nu);
+    const uint32_t ph = it & 1;
+    if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
+    const bool got = mbar_wait(&barA, ph, err) && mbar_wait(&barB, ph, err);
+    if (tid == 0) pendA = pendB = got ? -1 : (int)ph;
+    ok = __syncthreads_and(ok && got);
+    if (!ok) break;
+    if (L < 64) {
+      zero_tail_rows(sQ, L, tid, 256);
+      zero_tail_rows(sK, L, tid, 256);
+      zero_tail_rows(sO, L, tid, 256);
     }
-    for (int s = 0; s < 8; ++s)
-      mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dutl, s, TILE128), desc_mnmajor(h, s, TILE128),
-               idesc_bf16(64, 128, true, true), 1);
-    mma_commit(&bar[1]);
-  }
-  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
-  tc_fence_after();
-  const float G0 = sG[r0], G1 = sG[r1], GC = sG[63];
-  if (ok) {
-    // P = QK * Gam, dP = scale dO U^T (lower incl. diagonal), columns [32*half, +32)
-    float qk[16], dp[16];
-    tmem_ld16dp_x4(taddr(tb, sub, 32 * half), qk);
-    tmem_ld16dp_x4(taddr(tb, sub, 64 + 32 * half), dp);
-    tmem_wait_ld();
-    float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = 32 * half + 8 * j + cq;
-      float g[4], m[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int row = q < 2 ? r0 : r1, col = c + (q & 1);
-        const float Gi = q < 2 ? G0 : G1;
-        float dpp = 0.f, gg = 0.f;
-        if (col <= row) {
-          const float gam = __expf(Gi - sG[col]);
-          const float dpv = p.scale * dp[4 * j + q];
-          dpp = dpv * qk[4 * j + q] * gam;
-          gg = dpv * gam;
-        }
-        g[q] = gg;
-        m[q] = dpp;
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+      const uint32_t q = smem_u32(sQ), k = smem_u32(sK), o = smem_u32(sO), ut = smem_u32(sUT),
+                     dut = smem_u32(sdUT), dutl = smem_u32(sdUTl), h = smem_u32(sH), dh = smem_u32(sdH);
+      for (int s = 0; s < 8; ++s) {
+        const uint32_t acc = s > 0;
+        mma_bf16(taddr(tb, 0, 0), desc_kmajor(q, s, TILE64), desc_kmajor(k, s, TILE64),
+                 idesc_bf16(64, 64, false, false), acc);
+        mma_bf16(taddr(tb, 0, 64), desc_kmajor(o, s, TILE64), desc_mnmajor(ut, s, TILE128),
+                 idesc_bf16(64, 64, false, true), acc);
+        mma_bf16(taddr(tb, 0, 128), desc_kmajor(o, s, TILE64), desc_mnmajor(h, s, TILE128),
+                 idesc_bf16(64, 128, false, true), acc);
+        mma_bf16(taddr(tb, 0, 256), desc_mnmajor(ut, s, TILE128), desc_mnmajor(dh, s, TILE128),
+                 idesc_bf16(64, 128, true, true), acc);
+        mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dut, s, TILE128), desc_mnmajor(h, s, TILE128),
+                 idesc_bf16(64, 128, true, true), acc);
       }
-      sM[r0 * 65 + c] = m[0];
-      sM[r0 * 65 + c + 1] = m[1];
-      sM[r1 * 65 + c] = m[2];
-      sM[r1 * 65 + c + 1] = m[3];
-      rs0 += m[0] + m[1];
-      rs1 += m[2] + m[3];
-      st_pair_split(sPG, sPGl, r0, c, TILE64, g[0], g[1]);
-      st_pair_split(sPG, sPGl, r1, c, TILE64, g[2], g[3]);
-    }
-    rs0 = quad_sum(rs0);
-    rs1 = quad_sum(rs1);
-    // dQ part 1: scale e^{G_i} dO S back into TMEM; dG2 = sum_k (.) Q[i,k]
-    float x[32], y[32], z[32];
-    tmem_ld16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
-    tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), y);
-    tmem_ld16dp_x8(taddr(tb, sub, 384 + 64 * half), z);
-    tmem_wait_ld();
-    const float e0 = p.scale * __expf(G0), e1 = p.scale * __expf(G1);
-    const float D0 = __expf(GC - G0), D1 = __expf(GC - G1);
-    float x0 = 0.f, x1 = 0.f, y0 = 0.f, y1 = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = 64 * half + 8 * j + cq;
-      const float2 q0 = ld_pair(sQ, r0, c, TILE64), q1 = ld_pair(sQ, r1, c, TILE64);
-      const float2 k0 = ld_pair(sK, r0, c, TILE64), k1 = ld_pair(sK, r1, c, TILE64);
-      x[4 * j] *= e0; x[4 * j + 1] *= e0; x[4 * j + 2] *= e1; x[4 * j + 3] *= e1;
-      x0 += x[4 * j] * q0.x + x[4 * j + 1] * q0.y;
-      x1 += x[4 * j + 2] * q1.x + x[4 * j + 3] * q1.y;
-      y[4 * j] *= D0; y[4 * j + 1] *= D0; y[4 * j + 2] *= D1; y[4 * j + 3] *= D1;
-      y0 += y[4 * j] * k0.x + y[4 * j + 1] * k0.y;
-      y1 += y[4 * j + 2] * k1.x + y[4 * j + 3] * k1.y;
-      // dW = -dU S, staged as a bf16 [64][128] tile in the (now free) U^T buffer
-      st_pair(sUT, r0, c, TILE64, -z[4 * j], -z[4 * j + 1]);
-      st_pair(sUT, r1, c, TILE64, -z[4 * j + 2], -z[4 * j + 3]);
-    }
-    tmem_st16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
-    tmem_st16dp_x8(taddr(tb, sub, 256 + 64 * half), y);
-    x0 = quad_sum(x0);
-    x1 = quad_sum(x1);
-    y0 = quad_sum(y0);
-    y1 = quad_sum(y1);
-    if ((lane & 3) == 0) {
-      sRow[(0 * 2 + half) * 64 + r0] = rs0;
-      sRow[(0 * 2 + half) * 64 + r1] = rs1;
-      sRow[(1 * 2 + half) * 64 + r0] = x0;
-      sRow[(1 * 2 + half) * 64 + r1] = x1;
-      sRow[(2 * 2 + half) * 64 + r0] = y0;  // D_i sum_k Y K (y already carries D_i)
-      sRow[(2 * 2 + half) * 64 + r1] = y1;
-    }
-    tmem_wait_st();
-  }
-  // <dS', S> over the two bf16 state tiles
-  float dot = 0.f;
-  for (int c = tid; c < 128 * 16; c += 256) {
-    const int rr = c / 16, j = c % 16;
-    float a8[8], b8[8];
-    ld_chunk_f(sH, rr, j, TILE128, a8);
-    ld_chunk_f(sdH, rr, j, TILE128, b8);
-    for (int q = 0; q < 8; ++q) dot += a8[q] * b8[q];
-  }
-  dot = warp_sum(dot);
-  if (lane == 0) sRed[warp] = dot;
-  fence_proxy_async();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (ok && tid == 0) {
-    tma_store_3d(&mdW, sUT, 0, (int)unit * 64, 0);
-    tma_store_3d(&mdW, sUT + TILE64, 64, (int)unit * 64, 0);
-    tma_store_commit();
-    const uint32_t k = smem_u32(sK), q = smem_u32(sQ);
-    for (int part = 0; part < 2; ++part) {
-      const uint32_t pg = smem_u32(part ? sPGl : sPG);
-      for (int s = 0; s < 4; ++s) {
-        mma_bf16(taddr(tb, 0, 128), desc_kmajor(pg, s, TILE64), desc_mnmajor(k, s, TILE64),
-                 idesc_bf16(64, 128, false, true), 1);
-        mma_bf16(taddr(tb, 0, 256), desc_mnmajor(pg, s, TILE64), desc_mnmajor(q, s, TILE64),
+      for (int s = 0; s < 8; ++s)
+        mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dutl, s, TILE128), desc_mnmajor(h, s, TILE128),
                  idesc_bf16(64, 128, true, true), 1);
+      mma_commit(&barM);
+    }
+    // <dS', S> over the two bf16 state tiles (while the MMAs run)
+    {
+      float dot = 0.f;
+      for (int c = tid; c < 128 * 16; c += 256) {
+        const int rr = c / 16, j = c % 16;
+        float a8[8], b8[8];
+        ld_chunk_f(sH, rr, j, TILE128, a8);
+        ld_chunk_f(sdH, rr, j, TILE128, b8);
+        for (int q = 0; q < 8; ++q) dot += a8[q] * b8[q];
+      }
+      dot = warp_sum(dot);
+      if (lane == 0) sRed[warp] = dot;
+    }
+    fence_proxy_async();
+    ok = __syncthreads_and(ok && mbar_wait(&barM, 0, err));
+    tc_fence_after();
+    if (!ok) break;
+    // dO, dU^T, S and dS' are no longer read: the next unit's copies stream in from here
+    if (tid == 0 && nvalid) {
+      load_B(nu);
+      pendB = (int)(ph ^ 1);
+    }
+    const float G0 = sG[r0], G1 = sG[r1], GC = sG[63];
+    {
+      // P = QK * Gam, dP = scale dO U^T (lower incl. diagonal), columns [32*half, +32)
+      float qk[16], dp[16];
+      tmem_ld16dp_x4(taddr(tb, sub, 32 * half), qk);
+      tmem_ld16dp_x4(taddr(tb, sub, 64 + 32 * half), dp);
+      tmem_wait_ld();
+      float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = 32 * half + 8 * j + cq;
+        float g[4], m[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int row = q < 2 ? r0 : r1, col = c + (q & 1);
+          const float Gi = q < 2 ? G0 : G1;
+          float dpp = 0.f, gg = 0.f;
+          if (col <= row) {
+            const float gam = __expf(Gi - sG[col]);
+            const float dpv = p.scale * dp[4 * j + q];
+            dpp = dpv * qk[4 * j + q] * gam;
+            gg = dpv * gam;
+          }
+          g[q] = gg;
+          m[q] = dpp;
+        }
+        sM[r0 * 65 + c] = m[0];
+        sM[r0 * 65 + c + 1] = m[1];
+        sM[r1 * 65 + c] = m[2];
+        sM[r1 * 65 + c + 1] = m[3];
+        rs0 += m[0] + m[1];
+        rs1 += m[2] + m[3];
+        st_pair_split(sPG, sPGl, r0, c, TILE64, g[0], g[1]);
+        st_pair_split(sPG, sPGl, r1, c, TILE64, g[2], g[3]);
+      }
+      rs0 = quad_sum(rs0);
+      rs1 = quad_sum(rs1);
+      // dQ part 1: scale e^{G_i} dO S back into TMEM; dG2 = sum_k (.) Q[i,k]
+      float x[32], y[32], z[32];
+      tmem_ld16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
+      tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), y);
+      tmem_ld16dp_x8(taddr(tb, sub, 384 + 64 * half), z);
+      tmem_wait_ld();
+      const float e0 = p.scale * __expf(G0), e1 = p.scale * __expf(G1);
+      const float D0 = __expf(GC - G0), D1 = __expf(GC - G1);
+      float x0 = 0.f, x1 = 0.f, y0 = 0.f, y1 = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = 64 * half + 8 * j + cq;
+        const float2 q0 = ld_pair(sQ, r0, c, TILE64), q1 = ld_pair(sQ, r1, c, TILE64);
+        const float2 k0 = ld_pair(sK, r0, c, TILE64), k1 = ld_pair(sK, r1, c, TILE64);
+        x[4 * j] *= e0; x[4 * j + 1] *= e0; x[4 * j + 2] *= e1; x[4 * j + 3] *= e1;
+        x0 += x[4 * j] * q0.x + x[4 * j + 1] * q0.y;
+        x1 += x[4 * j + 2] * q1.x + x[4 * j + 3] * q1.y;
+        y[4 * j] *= D0; y[4 * j + 1] *= D0; y[4 * j + 2] *= D1; y[4 * j + 3] *= D1;
+        y0 += y[4 * j] * k0.x + y[4 * j + 1] * k0.y;
+        y1 += y[4 * j + 2] * k1.x + y[4 * j + 3] * k1.y;
+        // dW = -dU S, staged as a bf16 [64][128] tile in the (now free) U^T buffer
+        st_pair(sUT, r0, c, TILE64, -z[4 * j], -z[4 * j + 1]);
+        st_pair(sUT, r1, c, TILE64, -z[4 * j + 2], -z[4 * j + 3]);
+      }
+      tmem_st16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
+      tmem_st16dp_x8(taddr(tb, sub, 256 + 64 * half), y);
+      x0 = quad_sum(x0);
+      x1 = quad_sum(x1);
+      y0 = quad_sum(y0);
+      y1 = quad_sum(y1);
+      if ((lane & 3) == 0) {
+        sRow[(0 * 2 + half) * 64 + r0] = rs0;
+        sRow[(0 * 2 + half) * 64 + r1] = rs1;
+        sRow[(1 * 2 + half) * 64 + r0] = x0;
+        sRow[(1 * 2 + half) * 64 + r1] = x1;
+        sRow[(2 * 2 + half) * 64 + r0] = y0;  // D_i sum_k Y K (y already carries D_i)
+        sRow[(2 * 2 + half) * 64 + r1] = y1;
+      }
+      tmem_wait_st();
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      tma_store_3d(&mdW, sUT, 0, (int)unit * 64, 0);
+      tma_store_3d(&mdW, sUT + TILE64, 64, (int)unit * 64, 0);
+      tma_store_commit();
+      const uint32_t k = smem_u32(sK), q = smem_u32(sQ);
+      for (int part = 0; part < 2; ++part) {
+        const uint32_t pg = smem_u32(part ? sPGl : sPG);
+        for (int s = 0; s < 4; ++s) {
+          mma_bf16(taddr(tb, 0, 128), desc_kmajor(pg, s, TILE64), desc_mnmajor(k, s, TILE64),
+                   idesc_bf16(64, 128, false, true), 1);
+          mma_bf16(taddr(tb, 0, 256), desc_mnmajor(pg, s, TILE64), desc_mnmajor(q, s, TILE64),
+                   idesc_bf16(64, 128, true, true), 1);
+        }
+      }
+      mma_commit(&barM);
+    }
+    // dG for this chunk (rows j = tid < 64), deterministic column sums
+    if (tid < 64) {
+      const int j = tid;
+      float cs = 0.f;
+      for (int ii = 0; ii < 64; ++ii) cs += sM[ii * 65 + j];
+      float g = sRow[0 * 64 + j] + sRow[1 * 64 + j] - cs + sRow[2 * 64 + j] + sRow[3 * 64 + j] -
+                (sRow[4 * 64 + j] + sRow[5 * 64 + j]);
+      if (j == 63) {
+        float d8 = 0.f, rsum = 0.f;
+        for (int q = 0; q < 8; ++q) d8 += sRed[q];
+        for (int q = 0; q < 64; ++q) rsum += sRow[4 * 64 + q] + sRow[5 * 64 + q];
+        g += __expf(GC) * d8 + rsum;
+      }
+      w.dG[((size_t)hv * p.NCmax + gc) * 64 + j] = g;
+    }
+    ok = __syncthreads_and(ok && mbar_wait(&barM, 1, err));
+    tc_fence_after();
+    if (!ok) break;
+    // Q, K no longer read; U^T (the dW staging) once the dW store has read it
+    if (tid == 0 && nvalid) {
+      tma_store_wait_read0();
+      load_A(nu);
+      pendA = (int)(ph ^ 1);
+    }
+    {
+      float x[32], y[32];
+      tmem_ld16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
+      tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), y);
+      tmem_wait_ld();
+      float* dq0 = w.dqp + (unit * 64 + r0) * D + 64 * half + cq;
+      float* dk0 = w.dkp + (unit * 64 + r0) * D + 64 * half + cq;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        *reinterpret_cast<float2*>(dq0 + 8 * j) = make_float2(x[4 * j], x[4 * j + 1]);
+        *reinterpret_cast<float2*>(dq0 + 8 * D + 8 * j) = make_float2(x[4 * j + 2], x[4 * j + 3]);
+        *reinterpret_cast<float2*>(dk0 + 8 * j) = make_float2(y[4 * j], y[4 * j + 1]);
+        *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j) = make_float2(y[4 * j + 2], y[4 * j + 3]);
       }
     }
-    mma_commit(&bar[1]);
+    // the next unit's first MMAs overwrite every TMEM column read above
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
   }
-  // dG for this chunk (rows j = tid < 64), deterministic column sums
-  if (tid < 64) {
-    const int j = tid;
-    float cs = 0.f;
-    for (int ii = 0; ii < 64; ++ii) cs += sM[ii * 65 + j];
-    float g = sRow[0 * 64 + j] + sRow[1 * 64 + j] - cs + sRow[2 * 64 + j] + sRow[3 * 64 + j] -
-              (sRow[4 * 64 + j] + sRow[5 * 64 + j]);
-    if (j == 63) {
-      float d8 = 0.f, rsum = 0.f;
-      for (int q = 0; q < 8; ++q) d8 += sRed[q];
-      for (int q = 0; q < 64; ++q) rsum += sRow[4 * 64 + q] + sRow[5 * 64 + q];
-      g += __expf(GC) * d8 + rsum;
-    }
-    w.dG[((size_t)hv * p.NCmax + gc) * 64 + j] = g;
+  if (tid == 0) {
+    // after an error: let copies still in flight land before the shared memory is released
+    if (pendA >= 0) mbar_wait(&barA, (uint32_t)pendA, err);
+    if (pendB >= 0) mbar_wait(&barB, (uint32_t)pendB, err);
+    tma_store_wait0();
   }
-  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
-  tc_fence_after();
-  if (ok) {
-    float x[32], y[32];
-    tmem_ld16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
-    tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), y);
-    tmem_wait_ld();
-    float* dq0 = w.dqp + (unit * 64 + r0) * D + 64 * half + cq;
-    float* dk0 = w.dkp + (unit * 64 + r0) * D + 64 * half + cq;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      *reinterpret_cast<float2*>(dq0 + 8 * j) = make_float2(x[4 * j], x[4 * j + 1]);
-      *reinterpret_cast<float2*>(dq0 + 8 * D + 8 * j) = make_float2(x[4 * j + 2], x[4 * j + 3]);
-      *reinterpret_cast<float2*>(dk0 + 8 * j) = make_float2(y[4 * j], y[4 * j + 1]);
-      *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j) = make_float2(y[4 * j + 2], y[4 * j + 3]);
-    }
-  }
-  if (tid == 0) tma_store_wait0();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tb, 512);
@@ -1045,7 +1096,8 @@ cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, 
   if ((e = tgo("tc_scan_bwd", k_tc_scan_bwd, gs, 128, 1024 + BwdScanSmem::TOTAL, s, p, a, w, t, m.q,
                m.k, m.dO, m.WT, m.dUlT32, m.dUT32, m.dUTl32, m.dh32)))
     return e;
-  if ((e = tgo("tc_dqkwg", k_tc_dqkwg, gu, 256, 1024 + DqkSmem::TOTAL, s, p, w, t, m.q, m.k, m.dO,
+  const dim3 gp((unsigned)std::min<long long>((long long)p.NCmax * p.HV, num_sms()));
+  if ((e = tgo("tc_dqkwg", k_tc_dqkwg, gp, 256, 1024 + DqkSmem::TOTAL, s, p, w, t, m.q, m.k, m.dO,
                m.UT, m.dUT, m.dUTl, m.h, m.dh, m.dW)))
     return e;
   if ((e = tgo("tc_wy_bwd", k_tc_wy_bwd, gu, 256, 1024 + WyBwdSmem::TOTAL, s, p, a, w, t, m.k, m.v,

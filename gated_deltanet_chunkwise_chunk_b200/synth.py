@@ -140,9 +140,15 @@ def make_case(B=1, T=64, H=1, HV=1, K=64, V=64, dtype="fp32", seed=0, lengths=No
                 cu_seqlens=cu, h0=h0_t, dht=dht_t, seed=seed, name=name)
 
 
-def config_case(idx: int, seed: int | None = None) -> Case:
-    """The seeded case of workload ``idx`` (seed defaults to 1000 + idx)."""
-    c = CONFIGS[idx]
+def config_case(idx: int, seed: int | None = None, T: int | None = None) -> Case:
+    """The seeded case of workload ``idx`` (seed defaults to 1000 + idx).  ``T`` overrides
+    the sequence length of a dense workload (a smaller case of the same shape)."""
+    c = dict(CONFIGS[idx])
+    if T is not None:
+        if c.get("nseq"):
+            raise ValueError("T applies to dense workloads only")
+        c["T"] = T
+        c["name"] = c["name"].replace(f"_T{CONFIGS[idx]['T']}_", f"_T{T}_")
     seed = 1000 + idx if seed is None else seed
     lengths = None
     if c.get("nseq"):
