@@ -791,10 +791,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
                                                    const __grid_constant__ CUtensorMap mdUT,
                                                    const __grid_constant__ CUtensorMap mdUTl) {
   if (failed(w)) return;
-  const int gc = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
-  const int4 e = w.chunk_tab[gc];
-  if (e.x < 0) return;
-  const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int half = warp >> 2, sub = 32 * (warp & 3);
   const int r0 = 16 * (warp & 3) + lane / 4, r1 = r0 + 8, cq = 2 * (lane & 3);
   extern __shared__ unsigned char smraw[];
@@ -818,13 +815,16 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   float* sb = reinterpret_cast<float*>(sm + WyBwdSmem::B);
   float* sEG = reinterpret_cast<float*>(sm + WyBwdSmem::EG);   // e^{G_j}
   float* sRow = reinterpret_cast<float*>(sm + WyBwdSmem::ROW);  // [kind][half][64]
-  __shared__ uint64_t bar[2];
+  // barA: K;  barB: dW, dU^T (hi, lo);  barC: V, T (hi, lo);  barM: MMA batches (4 per unit)
+  __shared__ uint64_t barA, barB, barC, barM;
   __shared__ uint32_t tslot;
   int* err = w.status;
-  const size_t unit = (size_t)gc * p.HV + hv;
+  const int nunits = p.NCmax * p.HV;
   if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+    mbar_init(&barA, 1);
+    mbar_init(&barB, 1);
+    mbar_init(&barC, 1);
+    mbar_init(&barM, 1);
     mbar_fence_init();
   }
   __syncthreads();
@@ -832,252 +832,307 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     tmem_alloc(&tslot, 512);
     tmem_relinquish();
   }
-  if (tid == 0) {
-    mbar_expect_tx(&bar[0], WyBwdSmem::LOAD_BYTES);
-    tma_load_3d(sK, &mk, 0, hk, tok0, &bar[0]);
-    tma_load_3d(sK + TILE64, &mk, 64, hk, tok0, &bar[0]);
-    tma_load_3d(sV, &mv, 0, hv, tok0, &bar[0]);
-    tma_load_3d(sV + TILE64, &mv, 64, hv, tok0, &bar[0]);
-    tma_load_3d(sT, &mTm, 0, (int)unit * 128, 0, &bar[0]);
-    tma_load_3d(sTl, &mTm, 0, (int)unit * 128 + 64, 0, &bar[0]);
-    tma_load_3d(sdW, &mdW, 0, (int)unit * 64, 0, &bar[0]);
-    tma_load_3d(sdW + TILE64, &mdW, 64, (int)unit * 64, 0, &bar[0]);
-    tma_load_3d(sdUT, &mdUT, 0, (int)unit * D, 0, &bar[0]);
-    tma_load_3d(sdUTl, &mdUTl, 0, (int)unit * D, 0, &bar[0]);
-  }
-  if (tid < 64) {
-    const size_t o = ((size_t)hv * p.NCmax + gc) * 64 + tid;
-    const float g = w.G[o];
-    sG[tid] = g;
-    sb[tid] = w.beta_p[o];
-    sEG[tid] = __expf(g);
+  auto valid = [&](int u) { return u < nunits && w.chunk_tab[u / p.HV].x >= 0; };
+  auto load_A = [&](int u) {
+    const int hk = (u % p.HV) / p.G, tok0 = w.chunk_tab[u / p.HV].w;
+    mbar_expect_tx(&barA, 2 * TILE64);
+    tma_load_3d(sK, &mk, 0, hk, tok0, &barA);
+    tma_load_3d(sK + TILE64, &mk, 64, hk, tok0, &barA);
+  };
+  auto load_B = [&](int u) {
+    mbar_expect_tx(&barB, 2 * TILE64 + 2 * TILE128);
+    tma_load_3d(sdW, &mdW, 0, u * 64, 0, &barB);
+    tma_load_3d(sdW + TILE64, &mdW, 64, u * 64, 0, &barB);
+    tma_load_3d(sdUT, &mdUT, 0, u * D, 0, &barB);
+    tma_load_3d(sdUTl, &mdUTl, 0, u * D, 0, &barB);
+  };
+  auto load_C = [&](int u) {
+    const int hv = u % p.HV, tok0 = w.chunk_tab[u / p.HV].w;
+    mbar_expect_tx(&barC, 4 * TILE64);
+    tma_load_3d(sV, &mv, 0, hv, tok0, &barC);
+    tma_load_3d(sV + TILE64, &mv, 64, hv, tok0, &barC);
+    tma_load_3d(sT, &mTm, 0, u * 128, 0, &barC);
+    tma_load_3d(sTl, &mTm, 0, u * 128 + 64, 0, &barC);
+  };
+  int u = blockIdx.x;
+  int pendA = -1, pendB = -1, pendC = -1;  // parity of a load group in flight (thread 0)
+  if (tid == 0 && valid(u)) {
+    load_A(u);
+    load_B(u);
+    load_C(u);
+    pendA = pendB = pendC = 0;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
-  bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
-  if (L < 64) {
-    zero_tail_rows(sK, L, tid, 256);
-    zero_tail_rows(sV, L, tid, 256);
-  }
-  fence_proxy_async();
-  __syncthreads();
-  const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aT = smem_u32(sT), aTl = smem_u32(sTl),
-                 aW = smem_u32(sdW), aU = smem_u32(sdUT), aUl = smem_u32(sdUTl);
-  if (ok && tid == 0) {
-    for (int s = 0; s < 8; ++s) {
-      const uint32_t acc = s > 0;
-      mma_bf16(taddr(tb, 0, 0), desc_mnmajor(aU, s, TILE128), desc_kmajor(aV, s, TILE64),
-               idesc_bf16(64, 64, true, false), acc);
-      mma_bf16(taddr(tb, 0, 0), desc_mnmajor(aUl, s, TILE128), desc_kmajor(aV, s, TILE64),
-               idesc_bf16(64, 64, true, false), 1);
-      mma_bf16(taddr(tb, 0, 64), desc_kmajor(aW, s, TILE64), desc_kmajor(aK, s, TILE64),
-               idesc_bf16(64, 64, false, false), acc);
-      mma_bf16(taddr(tb, 0, 128), desc_kmajor(aK, s, TILE64), desc_kmajor(aK, s, TILE64),
-               idesc_bf16(64, 64, false, false), acc);
+  bool ok = true;
+  for (uint32_t it = 0; valid(u); ++it, u += gridDim.x) {
+    const int gc = u / p.HV, hv = u % p.HV;
+    const int4 e = w.chunk_tab[gc];
+    const int L = e.z, tok0 = e.w;
+    const size_t unit = (size_t)u;
+    const int nu = u + gridDim.x;
+    const bool nvalid = valid(nu);
+    const uint32_t ph = it & 1;
+    if (tid < 64) {
+      const size_t o = ((size_t)hv * p.NCmax + gc) * 64 + tid;
+      const float g = w.G[o];
+      sG[tid] = g;
+      sb[tid] = w.beta_p[o];
+      sEG[tid] = __expf(g);
     }
-    for (int part = 0; part < 2; ++part) {
-      const uint32_t tt = part ? aTl : aT;
-      for (int s = 0; s < 4; ++s) {
-        const uint32_t acc = part > 0 || s > 0;
-        mma_bf16(taddr(tb, 0, 256), desc_mnmajor(tt, s, TILE64), desc_mnmajor(aW, s, TILE64),
-                 idesc_bf16(64, 128, true, true), acc);
-        mma_bf16(taddr(tb, 0, 384), desc_mnmajor(tt, s, TILE64), desc_kmajor(aU, s, TILE128),
-                 idesc_bf16(64, 128, true, false), acc);
-        if (part == 0)
-          mma_bf16(taddr(tb, 0, 384), desc_mnmajor(tt, s, TILE64), desc_kmajor(aUl, s, TILE128),
-                   idesc_bf16(64, 128, true, false), 1);
+    const bool got = mbar_wait(&barA, ph, err) && mbar_wait(&barB, ph, err) && mbar_wait(&barC, ph, err);
+    if (tid == 0) pendA = pendB = pendC = got ? -1 : (int)ph;
+    ok = __syncthreads_and(ok && got);
+    if (!ok) break;
+    if (L < 64) {
+      zero_tail_rows(sK, L, tid, 256);
+      zero_tail_rows(sV, L, tid, 256);
+    }
+    fence_proxy_async();
+    __syncthreads();
+    const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aT = smem_u32(sT), aTl = smem_u32(sTl),
+                   aW = smem_u32(sdW), aU = smem_u32(sdUT), aUl = smem_u32(sdUTl);
+    if (tid == 0) {
+      for (int s = 0; s < 8; ++s) {
+        const uint32_t acc = s > 0;
+        mma_bf16(taddr(tb, 0, 0), desc_mnmajor(aU, s, TILE128), desc_kmajor(aV, s, TILE64),
+                 idesc_bf16(64, 64, true, false), acc);
+        mma_bf16(taddr(tb, 0, 0), desc_mnmajor(aUl, s, TILE128), desc_kmajor(aV, s, TILE64),
+                 idesc_bf16(64, 64, true, false), 1);
+        mma_bf16(taddr(tb, 0, 64), desc_kmajor(aW, s, TILE64), desc_kmajor(aK, s, TILE64),
+                 idesc_bf16(64, 64, false, false), acc);
+        mma_bf16(taddr(tb, 0, 128), desc_kmajor(aK, s, TILE64), desc_kmajor(aK, s, TILE64),
+                 idesc_bf16(64, 64, false, false), acc);
       }
-    }
-    mma_commit(&bar[1]);
-  }
-  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
-  tc_fence_after();
-  const float G0 = sG[r0], G1 = sG[r1], b0 = sb[r0], b1 = sb[r1];
-  if (ok) {
-    float r1v[16], r2v[16], kk[16];
-    tmem_ld16dp_x4(taddr(tb, sub, 32 * half), r1v);
-    tmem_ld16dp_x4(taddr(tb, sub, 64 + 32 * half), r2v);
-    tmem_ld16dp_x4(taddr(tb, sub, 128 + 32 * half), kk);
-    tmem_wait_ld();
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = 32 * half + 8 * j + cq;
-      const float bc0 = sb[c], bc1 = sb[c + 1], ec0 = sEG[c], ec1 = sEG[c + 1];
-      st_pair_split(sdT, sdTl, r0, c, TILE64, bc0 * (r1v[4 * j] + ec0 * r2v[4 * j]),
-                    bc1 * (r1v[4 * j + 1] + ec1 * r2v[4 * j + 1]));
-      st_pair_split(sdT, sdTl, r1, c, TILE64, bc0 * (r1v[4 * j + 2] + ec0 * r2v[4 * j + 2]),
-                    bc1 * (r1v[4 * j + 3] + ec1 * r2v[4 * j + 3]));
-      sKKG[r0 * 65 + c] = c < r0 ? __expf(G0 - sG[c]) * kk[4 * j] : 0.f;
-      sKKG[r0 * 65 + c + 1] = c + 1 < r0 ? __expf(G0 - sG[c + 1]) * kk[4 * j + 1] : 0.f;
-      sKKG[r1 * 65 + c] = c < r1 ? __expf(G1 - sG[c]) * kk[4 * j + 2] : 0.f;
-      sKKG[r1 * 65 + c + 1] = c + 1 < r1 ? __expf(G1 - sG[c + 1]) * kk[4 * j + 3] : 0.f;
-    }
-    // dX: dbeta/dG parts, then beta_i e^{G_i} dX back into TMEM; dY: dv = beta dY, dbeta part
-    float x[32], y[32];
-    tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
-    tmem_ld16dp_x8(taddr(tb, sub, 384 + 64 * half), y);
-    tmem_wait_ld();
-    const float s0 = b0 * sEG[r0], s1 = b1 * sEG[r1];
-    float px0 = 0.f, px1 = 0.f, py0 = 0.f, py1 = 0.f;
-    bf16* dv0 = static_cast<bf16*>(a.dv) + ((size_t)(tok0 + r0) * p.HV + hv) * D + 64 * half + cq;
-    bf16* dv1 = dv0 + (size_t)8 * p.HV * D;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = 64 * half + 8 * j + cq;
-      const float2 k0 = ld_pair(sK, r0, c, TILE64), k1 = ld_pair(sK, r1, c, TILE64);
-      const float2 v0 = ld_pair(sV, r0, c, TILE64), v1 = ld_pair(sV, r1, c, TILE64);
-      px0 += x[4 * j] * k0.x + x[4 * j + 1] * k0.y;
-      px1 += x[4 * j + 2] * k1.x + x[4 * j + 3] * k1.y;
-      x[4 * j] *= s0; x[4 * j + 1] *= s0; x[4 * j + 2] *= s1; x[4 * j + 3] *= s1;
-      py0 += y[4 * j] * v0.x + y[4 * j + 1] * v0.y;
-      py1 += y[4 * j + 2] * v1.x + y[4 * j + 3] * v1.y;
-      if (r0 < L)
-        *reinterpret_cast<uint32_t*>(dv0 + 8 * j) = pack_bf16(b0 * y[4 * j], b0 * y[4 * j + 1]);
-      if (r1 < L)
-        *reinterpret_cast<uint32_t*>(dv1 + 8 * j) = pack_bf16(b1 * y[4 * j + 2], b1 * y[4 * j + 3]);
-    }
-    tmem_st16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
-    px0 = quad_sum(px0);
-    px1 = quad_sum(px1);
-    py0 = quad_sum(py0);
-    py1 = quad_sum(py1);
-    if ((lane & 3) == 0) {
-      sRow[(0 * 2 + half) * 64 + r0] = px0;
-      sRow[(0 * 2 + half) * 64 + r1] = px1;
-      sRow[(1 * 2 + half) * 64 + r0] = py0;
-      sRow[(1 * 2 + half) * 64 + r1] = py1;
-    }
-    tmem_wait_st();
-  }
-  fence_proxy_async();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  // Z = T^T dT, dropping lo*lo
-  if (ok && tid == 0) {
-    const uint32_t dt = smem_u32(sdT), dtl = smem_u32(sdTl);
-    const uint32_t pa[3] = {aT, aT, aTl}, pb[3] = {dt, dtl, dt};
-    for (int part = 0; part < 3; ++part)
-      for (int s = 0; s < 4; ++s)
-        mma_bf16(taddr(tb, 0, 0), desc_mnmajor(pa[part], s, TILE64), desc_mnmajor(pb[part], s, TILE64),
-                 idesc_bf16(64, 64, true, true), part > 0 || s > 0);
-    mma_commit(&bar[1]);
-  }
-  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
-  tc_fence_after();
-  if (ok) {
-    float z[16];
-    tmem_ld16dp_x4(taddr(tb, sub, 32 * half), z);
-    tmem_wait_ld();
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = 32 * half + 8 * j + cq;
-      st_pair_split(sZ, sZl, r0, c, TILE64, z[4 * j], z[4 * j + 1]);
-      st_pair_split(sZ, sZl, r1, c, TILE64, z[4 * j + 2], z[4 * j + 3]);
-    }
-  }
-  fence_proxy_async();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  // dA' = Z T^T
-  if (ok && tid == 0) {
-    const uint32_t zz = smem_u32(sZ), zl = smem_u32(sZl);
-    const uint32_t pa[3] = {zz, zz, zl}, pb[3] = {aT, aTl, aT};
-    for (int part = 0; part < 3; ++part)
-      for (int s = 0; s < 4; ++s)
-        mma_bf16(taddr(tb, 0, 64), desc_kmajor(pa[part], s, TILE64), desc_kmajor(pb[part], s, TILE64),
-                 idesc_bf16(64, 64, false, false), part > 0 || s > 0);
-    mma_commit(&bar[1]);
-  }
-  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
-  tc_fence_after();
-  if (ok) {
-    float da[16];
-    tmem_ld16dp_x4(taddr(tb, sub, 64 + 32 * half), da);
-    tmem_wait_ld();
-    float pa0 = 0.f, pa1 = 0.f, paa0 = 0.f, paa1 = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = 32 * half + 8 * j + cq;
-      float as[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int row = q < 2 ? r0 : r1, col = c + (q & 1);
-        const float Gi = q < 2 ? G0 : G1, bi = q < 2 ? b0 : b1;
-        float dAs = 0.f, aa = 0.f;
-        if (col < row) {
-          const float dA = -da[4 * j + q];
-          const float kkg = sKKG[row * 65 + col];
-          if (q < 2) pa0 += dA * kkg; else pa1 += dA * kkg;
-          aa = dA * bi * kkg;
-          dAs = dA * __expf(Gi - sG[col]) * bi;
+      for (int part = 0; part < 2; ++part) {
+        const uint32_t tt = part ? aTl : aT;
+        for (int s = 0; s < 4; ++s) {
+          const uint32_t acc = part > 0 || s > 0;
+          mma_bf16(taddr(tb, 0, 256), desc_mnmajor(tt, s, TILE64), desc_mnmajor(aW, s, TILE64),
+                   idesc_bf16(64, 128, true, true), acc);
+          mma_bf16(taddr(tb, 0, 384), desc_mnmajor(tt, s, TILE64), desc_kmajor(aU, s, TILE128),
+                   idesc_bf16(64, 128, true, false), acc);
+          if (part == 0)
+            mma_bf16(taddr(tb, 0, 384), desc_mnmajor(tt, s, TILE64), desc_kmajor(aUl, s, TILE128),
+                     idesc_bf16(64, 128, true, false), 1);
         }
-        sAA[row * 65 + col] = aa;
-        if (q < 2) paa0 += aa; else paa1 += aa;
-        as[q] = dAs;
       }
-      st_pair_split(sAs, sAsl, r0, c, TILE64, as[0], as[1]);
-      st_pair_split(sAs, sAsl, r1, c, TILE64, as[2], as[3]);
+      mma_commit(&barM);
     }
-    pa0 = quad_sum(pa0);
-    pa1 = quad_sum(pa1);
-    paa0 = quad_sum(paa0);
-    paa1 = quad_sum(paa1);
-    if ((lane & 3) == 0) {
-      sRow[(2 * 2 + half) * 64 + r0] = pa0;
-      sRow[(2 * 2 + half) * 64 + r1] = pa1;
-      sRow[(3 * 2 + half) * 64 + r0] = paa0;
-      sRow[(3 * 2 + half) * 64 + r1] = paa1;
+    ok = __syncthreads_and(ok && mbar_wait(&barM, 0, err));
+    tc_fence_after();
+    if (!ok) break;
+    if (tid == 0 && nvalid) {  // dW, dU^T are read by the first MMA batch only
+      load_B(nu);
+      pendB = (int)(ph ^ 1);
     }
-  }
-  fence_proxy_async();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  // dk += dAs K + dAs^T K onto beta e^G dX
-  if (ok && tid == 0) {
-    for (int part = 0; part < 2; ++part) {
-      const uint32_t as = smem_u32(part ? sAsl : sAs);
-      for (int s = 0; s < 4; ++s) {
-        mma_bf16(taddr(tb, 0, 256), desc_kmajor(as, s, TILE64), desc_mnmajor(aK, s, TILE64),
-                 idesc_bf16(64, 128, false, true), 1);
-        mma_bf16(taddr(tb, 0, 256), desc_mnmajor(as, s, TILE64), desc_mnmajor(aK, s, TILE64),
-                 idesc_bf16(64, 128, true, true), 1);
+    const float G0 = sG[r0], G1 = sG[r1], b0 = sb[r0], b1 = sb[r1];
+    {
+      float r1v[16], r2v[16], kk[16];
+      tmem_ld16dp_x4(taddr(tb, sub, 32 * half), r1v);
+      tmem_ld16dp_x4(taddr(tb, sub, 64 + 32 * half), r2v);
+      tmem_ld16dp_x4(taddr(tb, sub, 128 + 32 * half), kk);
+      tmem_wait_ld();
+  #pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = 32 * half + 8 * j + cq;
+        const float bc0 = sb[c], bc1 = sb[c + 1], ec0 = sEG[c], ec1 = sEG[c + 1];
+        st_pair_split(sdT, sdTl, r0, c, TILE64, bc0 * (r1v[4 * j] + ec0 * r2v[4 * j]),
+                      bc1 * (r1v[4 * j + 1] + ec1 * r2v[4 * j + 1]));
+        st_pair_split(sdT, sdTl, r1, c, TILE64, bc0 * (r1v[4 * j + 2] + ec0 * r2v[4 * j + 2]),
+                      bc1 * (r1v[4 * j + 3] + ec1 * r2v[4 * j + 3]));
+        sKKG[r0 * 65 + c] = c < r0 ? __expf(G0 - sG[c]) * kk[4 * j] : 0.f;
+        sKKG[r0 * 65 + c + 1] = c + 1 < r0 ? __expf(G0 - sG[c + 1]) * kk[4 * j + 1] : 0.f;
+        sKKG[r1 * 65 + c] = c < r1 ? __expf(G1 - sG[c]) * kk[4 * j + 2] : 0.f;
+        sKKG[r1 * 65 + c + 1] = c + 1 < r1 ? __expf(G1 - sG[c + 1]) * kk[4 * j + 3] : 0.f;
+      }
+      // dX: dbeta/dG parts, then beta_i e^{G_i} dX back into TMEM; dY: dv = beta dY, dbeta part
+      float x[32], y[32];
+      tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
+      tmem_ld16dp_x8(taddr(tb, sub, 384 + 64 * half), y);
+      tmem_wait_ld();
+      const float s0 = b0 * sEG[r0], s1 = b1 * sEG[r1];
+      float px0 = 0.f, px1 = 0.f, py0 = 0.f, py1 = 0.f;
+      bf16* dv0 = static_cast<bf16*>(a.dv) + ((size_t)(tok0 + r0) * p.HV + hv) * D + 64 * half + cq;
+      bf16* dv1 = dv0 + (size_t)8 * p.HV * D;
+  #pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = 64 * half + 8 * j + cq;
+        const float2 k0 = ld_pair(sK, r0, c, TILE64), k1 = ld_pair(sK, r1, c, TILE64);
+        const float2 v0 = ld_pair(sV, r0, c, TILE64), v1 = ld_pair(sV, r1, c, TILE64);
+        px0 += x[4 * j] * k0.x + x[4 * j + 1] * k0.y;
+        px1 += x[4 * j + 2] * k1.x + x[4 * j + 3] * k1.y;
+        x[4 * j] *= s0; x[4 * j + 1] *= s0; x[4 * j + 2] *= s1; x[4 * j + 3] *= s1;
+        py0 += y[4 * j] * v0.x + y[4 * j + 1] * v0.y;
+        py1 += y[4 * j + 2] * v1.x + y[4 * j + 3] * v1.y;
+        if (r0 < L)
+          *reinterpret_cast<uint32_t*>(dv0 + 8 * j) = pack_bf16(b0 * y[4 * j], b0 * y[4 * j + 1]);
+        if (r1 < L)
+          *reinterpret_cast<uint32_t*>(dv1 + 8 * j) = pack_bf16(b1 * y[4 * j + 2], b1 * y[4 * j + 3]);
+      }
+      tmem_st16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
+      px0 = quad_sum(px0);
+      px1 = quad_sum(px1);
+      py0 = quad_sum(py0);
+      py1 = quad_sum(py1);
+      if ((lane & 3) == 0) {
+        sRow[(0 * 2 + half) * 64 + r0] = px0;
+        sRow[(0 * 2 + half) * 64 + r1] = px1;
+        sRow[(1 * 2 + half) * 64 + r0] = py0;
+        sRow[(1 * 2 + half) * 64 + r1] = py1;
+      }
+      tmem_wait_st();
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // Z = T^T dT, dropping lo*lo
+    if (tid == 0) {
+      const uint32_t dt = smem_u32(sdT), dtl = smem_u32(sdTl);
+      const uint32_t pa[3] = {aT, aT, aTl}, pb[3] = {dt, dtl, dt};
+      for (int part = 0; part < 3; ++part)
+        for (int s = 0; s < 4; ++s)
+          mma_bf16(taddr(tb, 0, 0), desc_mnmajor(pa[part], s, TILE64), desc_mnmajor(pb[part], s, TILE64),
+                   idesc_bf16(64, 64, true, true), part > 0 || s > 0);
+      mma_commit(&barM);
+    }
+    ok = __syncthreads_and(ok && mbar_wait(&barM, 1, err));
+    tc_fence_after();
+    if (!ok) break;
+    {
+      float z[16];
+      tmem_ld16dp_x4(taddr(tb, sub, 32 * half), z);
+      tmem_wait_ld();
+  #pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = 32 * half + 8 * j + cq;
+        st_pair_split(sZ, sZl, r0, c, TILE64, z[4 * j], z[4 * j + 1]);
+        st_pair_split(sZ, sZl, r1, c, TILE64, z[4 * j + 2], z[4 * j + 3]);
       }
     }
-    mma_commit(&bar[1]);
-  }
-  if (tid < 64) {
-    const int j = tid;
-    float cs = 0.f;
-    for (int r = 0; r < 64; ++r) cs += sAA[r * 65 + j];
-    const float eg = sEG[j], bj = sb[j];
-    const float px = sRow[0 * 64 + j] + sRow[1 * 64 + j];
-    const float py = sRow[2 * 64 + j] + sRow[3 * 64 + j];
-    const float pa = sRow[4 * 64 + j] + sRow[5 * 64 + j];
-    const float paa = sRow[6 * 64 + j] + sRow[7 * 64 + j];
-    if (j < L) a.dbeta[(size_t)(tok0 + j) * p.HV + hv] = eg * px + py + pa;
-    w.dG[((size_t)hv * p.NCmax + gc) * 64 + j] += bj * eg * px + paa - cs;
-  }
-  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
-  tc_fence_after();
-  if (ok) {
-    float x[32];
-    tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
-    tmem_wait_ld();
-    float* dk0 = w.dkp + (unit * 64 + r0) * D + 64 * half + cq;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float2 o0 = *reinterpret_cast<float2*>(dk0 + 8 * j);
-      float2 o1 = *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j);
-      o0.x += x[4 * j]; o0.y += x[4 * j + 1];
-      o1.x += x[4 * j + 2]; o1.y += x[4 * j + 3];
-      *reinterpret_cast<float2*>(dk0 + 8 * j) = o0;
-      *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j) = o1;
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // dA' = Z T^T
+    if (tid == 0) {
+      const uint32_t zz = smem_u32(sZ), zl = smem_u32(sZl);
+      const uint32_t pa[3] = {zz, zz, zl}, pb[3] = {aT, aTl, aT};
+      for (int part = 0; part < 3; ++part)
+        for (int s = 0; s < 4; ++s)
+          mma_bf16(taddr(tb, 0, 64), desc_kmajor(pa[part], s, TILE64), desc_kmajor(pb[part], s, TILE64),
+                   idesc_bf16(64, 64, false, false), part > 0 || s > 0);
+      mma_commit(&barM);
     }
+    ok = __syncthreads_and(ok && mbar_wait(&barM, 0, err));
+    tc_fence_after();
+    if (!ok) break;
+    if (tid == 0 && nvalid) {  // V (last read in the first epilogue) and T (by the MMAs above)
+      load_C(nu);
+      pendC = (int)(ph ^ 1);
+    }
+    {
+      float da[16];
+      tmem_ld16dp_x4(taddr(tb, sub, 64 + 32 * half), da);
+      tmem_wait_ld();
+      float pa0 = 0.f, pa1 = 0.f, paa0 = 0.f, paa1 = 0.f;
+  #pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = 32 * half + 8 * j + cq;
+        float as[4];
+  #pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int row = q < 2 ? r0 : r1, col = c + (q & 1);
+          const float Gi = q < 2 ? G0 : G1, bi = q < 2 ? b0 : b1;
+          float dAs = 0.f, aa = 0.f;
+          if (col < row) {
+            const float dA = -da[4 * j + q];
+            const float kkg = sKKG[row * 65 + col];
+            if (q < 2) pa0 += dA * kkg; else pa1 += dA * kkg;
+            aa = dA * bi * kkg;
+            dAs = dA * __expf(Gi - sG[col]) * bi;
+          }
+          sAA[row * 65 + col] = aa;
+          if (q < 2) paa0 += aa; else paa1 += aa;
+          as[q] = dAs;
+        }
+        st_pair_split(sAs, sAsl, r0, c, TILE64, as[0], as[1]);
+        st_pair_split(sAs, sAsl, r1, c, TILE64, as[2], as[3]);
+      }
+      pa0 = quad_sum(pa0);
+      pa1 = quad_sum(pa1);
+      paa0 = quad_sum(paa0);
+      paa1 = quad_sum(paa1);
+      if ((lane & 3) == 0) {
+        sRow[(2 * 2 + half) * 64 + r0] = pa0;
+        sRow[(2 * 2 + half) * 64 + r1] = pa1;
+        sRow[(3 * 2 + half) * 64 + r0] = paa0;
+        sRow[(3 * 2 + half) * 64 + r1] = paa1;
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // dk += dAs K + dAs^T K onto beta e^G dX
+    if (tid == 0) {
+      for (int part = 0; part < 2; ++part) {
+        const uint32_t as = smem_u32(part ? sAsl : sAs);
+        for (int s = 0; s < 4; ++s) {
+          mma_bf16(taddr(tb, 0, 256), desc_kmajor(as, s, TILE64), desc_mnmajor(aK, s, TILE64),
+                   idesc_bf16(64, 128, false, true), 1);
+          mma_bf16(taddr(tb, 0, 256), desc_mnmajor(as, s, TILE64), desc_mnmajor(aK, s, TILE64),
+                   idesc_bf16(64, 128, true, true), 1);
+        }
+      }
+      mma_commit(&barM);
+    }
+    if (tid < 64) {
+      const int j = tid;
+      float cs = 0.f;
+      for (int r = 0; r < 64; ++r) cs += sAA[r * 65 + j];
+      const float eg = sEG[j], bj = sb[j];
+      const float px = sRow[0 * 64 + j] + sRow[1 * 64 + j];
+      const float py = sRow[2 * 64 + j] + sRow[3 * 64 + j];
+      const float pa = sRow[4 * 64 + j] + sRow[5 * 64 + j];
+      const float paa = sRow[6 * 64 + j] + sRow[7 * 64 + j];
+      if (j < L) a.dbeta[(size_t)(tok0 + j) * p.HV + hv] = eg * px + py + pa;
+      w.dG[((size_t)hv * p.NCmax + gc) * 64 + j] += bj * eg * px + paa - cs;
+    }
+    ok = __syncthreads_and(ok && mbar_wait(&barM, 1, err));
+    tc_fence_after();
+    if (!ok) break;
+    if (tid == 0 && nvalid) {  // K read by the MMAs above for the last time
+      load_A(nu);
+      pendA = (int)(ph ^ 1);
+    }
+    {
+      float x[32];
+      tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
+      tmem_wait_ld();
+      float* dk0 = w.dkp + (unit * 64 + r0) * D + 64 * half + cq;
+  #pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float2 o0 = *reinterpret_cast<float2*>(dk0 + 8 * j);
+        float2 o1 = *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j);
+        o0.x += x[4 * j]; o0.y += x[4 * j + 1];
+        o1.x += x[4 * j + 2]; o1.y += x[4 * j + 3];
+        *reinterpret_cast<float2*>(dk0 + 8 * j) = o0;
+        *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j) = o1;
+      }
+    }
+    // the next unit's first MMAs overwrite every TMEM column read above
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  if (tid == 0) {  // after an error: let copies still in flight land first
+    if (pendA >= 0) mbar_wait(&barA, (uint32_t)pendA, err);
+    if (pendB >= 0) mbar_wait(&barB, (uint32_t)pendB, err);
+    if (pendC >= 0) mbar_wait(&barC, (uint32_t)pendC, err);
   }
   tc_fence_before();
   __syncthreads();
@@ -1100,7 +1155,7 @@ cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, 
   if ((e = tgo("tc_dqkwg", k_tc_dqkwg, gp, 256, 1024 + DqkSmem::TOTAL, s, p, w, t, m.q, m.k, m.dO,
                m.UT, m.dUT, m.dUTl, m.h, m.dh, m.dW)))
     return e;
-  if ((e = tgo("tc_wy_bwd", k_tc_wy_bwd, gu, 256, 1024 + WyBwdSmem::TOTAL, s, p, a, w, t, m.k, m.v,
+  if ((e = tgo("tc_wy_bwd", k_tc_wy_bwd, gp, 256, 1024 + WyBwdSmem::TOTAL, s, p, a, w, t, m.k, m.v,
                m.Tm, m.dW, m.dUT, m.dUTl)))
     return e;
   return cudaSuccess;
