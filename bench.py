@@ -59,6 +59,33 @@ def kernel_flops_per_token_head(K: int, V: int) -> dict:
     return {f"{path}_{k}": v for k, v in per.items() for path in ("ffma", "tc")}
 
 
+def kernel_bytes_per_unit(K: int, V: int, G: int, e: int) -> dict:
+    """Algorithmic HBM bytes each tcgen05 kernel moves per (chunk, value head) unit: every
+    operand tile it must read and every tile it must write once (a k-head's q/k tile is
+    shared by its G value heads and counted once), following the chunk dataflow between
+    the kernels (bf16 tiles W^T, U~^T, U^T, S, dS, dU_loc^T, dU^T hi/lo, dW, T hi/lo;
+    fp32 dq/dk shares; fp32 per-chunk vectors of 64)."""
+    tq = C * K * e / G            # q or k tile, per value head
+    tv = C * V * e                # v, o, dO, dv tile
+    wt = K * C * e                # W^T, dW
+    ut = V * C * e                # U~^T, U^T, dU_loc^T, dU^T (one part)
+    st = V * K * e                # S or dS entering/leaving the chunk
+    tm = 2 * C * C * e            # T = (I + A)^-1 as a hi/lo pair
+    f32 = C * K * 4               # fp32 dq or dk share
+    vec = C * 4                   # one per-chunk fp32 vector
+    per = {
+        "wy": tq + tv + 2 * vec + wt + ut + tm,
+        "scan_fwd": wt + ut + tq + 2 * vec + st + ut,
+        "out": 2 * tq + st + ut + vec + tv,
+        "dvlocal": 2 * tq + tv + vec + ut,
+        "scan_bwd": 2 * tq + tv + wt + ut + 2 * vec + st + 2 * ut,
+        "dqkwg": 2 * tq + tv + 3 * ut + 2 * st + vec + wt + 2 * f32 + vec,
+        "wy_bwd": tq + tv + tm + wt + 2 * ut + f32 + 2 * vec + tv + f32 + 2 * vec,
+        "dqdk_group_sum": 2 * f32 + 2 * tq,
+    }
+    return {f"tc_{k}" if k != "dqdk_group_sum" else k: v for k, v in per.items()}
+
+
 def step_flops_per_token_head(K: int, V: int) -> tuple[float, float]:
     """Algorithmic FLOPs of the method per token per value head (fwd, bwd)."""
     fwd = 2 * C * (3 * K + 2 * V) + 6 * K * V + C * C / 3
@@ -360,15 +387,21 @@ def main():
 
 
 def kernel_roofline(prof: dict, case, pk: dict) -> dict | None:
-    """Roofline of the kernel with the largest share of device time."""
+    """Roofline of the kernel with the largest share of device time: its algorithmic FLOPs
+    and HBM bytes per launch (per-unit figures x units), the bound being whichever of
+    FLOPs / bf16 peak and bytes / HBM bandwidth takes longer."""
     if not prof:
         return None
     name, (launches, total_ms) = max(prof.items(), key=lambda kv: kv[1][1])
     per_launch_s = total_ms / launches / 1e3
     fl = kernel_flops_per_token_head(case.K, case.V).get(name)
     th = case.tokens * case.HV
+    e = 2 if case.dtype == "bf16" else 4
+    units = chunks_of(case) * case.HV
+    by = kernel_bytes_per_unit(case.K, case.V, case.HV // case.H, e).get(name)
     out = {"kernel": name, "launch_ms": round(per_launch_s * 1e3, 4),
-           "share": round(total_ms / sum(v[1] for v in prof.values()), 4)}
+           "share": round(total_ms / sum(v[1] for v in prof.values()), 4),
+           "units_per_launch": units}
     traffic = _traffic(name, case)
     if fl is not None and name.startswith("ffma_"):
         achieved = fl * th / per_launch_s / 1e12
@@ -376,13 +409,29 @@ def kernel_roofline(prof: dict, case, pk: dict) -> dict | None:
         out.update({"bound": "alu", "achieved": round(achieved, 3), "peak": round(peak, 1),
                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                     "peak_source": "fp32 FFMA: 148 SM x 128 lanes x 2 FLOP x 1.965 GHz"})
+        return out
+    t_tc = fl * th / (pk["bf16_tflops"] * 1e12) if fl is not None else 0.0
+    t_hbm = by * units / (pk["hbm_gbs"] * 1e9) if by is not None else 0.0
+    if by is not None and t_hbm >= t_tc:
+        achieved = by * units / per_launch_s / 1e9
+        out.update({"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
+                    "algorithmic_bytes": int(by * units), "bytes_per_unit": int(by),
+                    "peak_source": f"HBM copy, {pk['source']}"})
     elif fl is not None:
         achieved = fl * th / per_launch_s / 1e12
-        peak = pk["bf16_tflops"]
-        out.update({"bound": "tensor", "achieved": round(achieved, 3), "peak": peak,
-                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+        out.update({"bound": "tensor", "achieved": round(achieved, 3), "peak": pk["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": traffic,
                     "peak_source": f"bf16 burst, {pk['source']}"})
     return out
+
+
+def chunks_of(case) -> int:
+    """64-token chunks of the workload (sequences never share a chunk)."""
+    if case.cu_seqlens is not None:
+        cu = case.cu_seqlens.tolist()
+        return sum((cu[i + 1] - cu[i] + C - 1) // C for i in range(len(cu) - 1))
+    return case.B * ((case.T + C - 1) // C)
 
 
 def _traffic(name: str, case):
@@ -391,8 +440,8 @@ def _traffic(name: str, case):
     try:
         with open(path) as f:
             d = json.load(f)
-        rec = d.get(name)
-        if rec and rec.get("workload") == case.name:
+        rec = d.get("kernels", {}).get(name)
+        if rec and d.get("workload") == case.name:
             return rec["bytes_per_launch"]
     except (OSError, ValueError):
         pass
