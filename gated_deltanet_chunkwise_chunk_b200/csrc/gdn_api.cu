@@ -41,7 +41,7 @@ int check_dims(const gdn_dims* d, bool varlen) {
 // own regions after the common ones).
 struct Plan {
   size_t status, seq_tab, chunk_tab, G, beta_p, Dec, EG;
-  size_t W, Ut, Tm, h, U, dU, dh, dW, dqp, dkp, dG, tmp;
+  size_t W, Ut, Tm, h, U, dU, dh, dW, dqp, dkp, dG, dkp2, dG2, tmp;
   size_t tc;     // start of the tcgen05 path's region
   size_t total;
 };
@@ -85,10 +85,12 @@ Plan make_plan(const gdn_dims& d, bool varlen, int pass) {
     // the tcgen05 region starts at the same offset for both passes, so a backward can read
     // what the forward left in the same workspace
     pl.tc = take(tc_workspace_bytes(d, NC, pass));
-    if (pass == 1) {  // fp32 per-value-head dq/dk shares and dG, read by the final assembly
+    if (pass == 1) {  // fp32 per-value-head dq/dk shares and dG parts, read by the final assembly
       pl.dqp = take(NC * HV * CH * K * f);
       pl.dkp = take(NC * HV * CH * K * f);
       pl.dG = take(HV * NC * CH * f);
+      pl.dkp2 = take(NC * HV * CH * K * f);
+      pl.dG2 = take(HV * NC * CH * f);
     }
   }
   pl.total = o;
@@ -117,6 +119,8 @@ Work carve(const Plan& pl, void* ws) {
   w.dqp = fp(pl.dqp);
   w.dkp = fp(pl.dkp);
   w.dG = fp(pl.dG);
+  w.dkp2 = fp(pl.dkp2);
+  w.dG2 = fp(pl.dG2);
   w.tmp = fp(pl.tmp);
   return w;
 }

@@ -138,7 +138,12 @@ __global__ void __launch_bounds__(256) k_bwd_tokens(Problem p, Args a, Work w) {
   for (int hv = warp; hv < p.HV; hv += blockDim.x / 32) {
     const float* dGp = w.dG + ((size_t)hv * p.NCmax + gc) * CH;
     // suffix sums: lane owns positions 2*lane, 2*lane+1; scan from the top lane down
-    const float d0 = dGp[2 * lane], d1 = dGp[2 * lane + 1];
+    float d0 = dGp[2 * lane], d1 = dGp[2 * lane + 1];
+    if (w.dG2) {
+      const float* dG2p = w.dG2 + ((size_t)hv * p.NCmax + gc) * CH;
+      d0 += dG2p[2 * lane];
+      d1 += dG2p[2 * lane + 1];
+    }
     float s = d0 + d1;
     for (int off = 1; off < 32; off <<= 1) {
       const float x = __shfl_down_sync(0xffffffffu, s, off);
@@ -180,6 +185,10 @@ __global__ void __launch_bounds__(256) k_dqdk_group_sum(Problem p, Args a, Work 
       const float4 y = *reinterpret_cast<const float4*>(w.dkp + o);
       sq.x += x.x; sq.y += x.y; sq.z += x.z; sq.w += x.w;
       sk.x += y.x; sk.y += y.y; sk.z += y.z; sk.w += y.w;
+      if (w.dkp2) {
+        const float4 z = *reinterpret_cast<const float4*>(w.dkp2 + o);
+        sk.x += z.x; sk.y += z.y; sk.z += z.z; sk.w += z.w;
+      }
     }
     const int t = i / K, c = i % K;
     T* q4 = dq + ((size_t)(tok0 + t) * p.H + h) * K + c;

@@ -773,14 +773,14 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
 // 16-lane TMEM loads as in dqkwg: thread rows r0 = 16(w%4) + t/4 and r0 + 8.
 // ======================================================================================
 struct WyBwdSmem {
-  static constexpr int K = 0, V = 2 * TILE64, T = 4 * TILE64, TL = 5 * TILE64, DW = 6 * TILE64,
-                       DUT = 8 * TILE64, DT = 8 * TILE64 + TILE128, DTL = DT + TILE64,
+  static constexpr int K = 0;                                    // 2 x [64][128] (double buffer)
+  static constexpr int V = 4 * TILE64, T = 6 * TILE64, TL = 7 * TILE64, DW = 8 * TILE64,
+                       DUT = 10 * TILE64, DT = 10 * TILE64 + TILE128, DTL = DT + TILE64,
                        Z = DTL + TILE64, ZL = Z + TILE64, AS = ZL + TILE64, ASL = AS + TILE64,
                        DUTL = ASL + TILE64, F = DUTL + TILE128;
   static constexpr int KKG = F, AA = KKG + 64 * 65 * 4;        // fp32 [64][65] each
   static constexpr int G = AA + 64 * 65 * 4, B = G + 256, EG = B + 256, ROW = EG + 256;
   static constexpr int TOTAL = ROW + 4 * 2 * 64 * 4;            // ROW [4][2][64]
-  static constexpr int LOAD_BYTES = 8 * TILE64 + 2 * TILE128;
 };
 
 __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, TcWork t,
@@ -796,7 +796,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   const int r0 = 16 * (warp & 3) + lane / 4, r1 = r0 + 8, cq = 2 * (lane & 3);
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
-  unsigned char* sK = sm + WyBwdSmem::K;
+  unsigned char* sKb = sm + WyBwdSmem::K;   // 2 x [64][128]: K of this unit and of the next
   unsigned char* sV = sm + WyBwdSmem::V;
   unsigned char* sT = sm + WyBwdSmem::T;
   unsigned char* sTl = sm + WyBwdSmem::TL;
@@ -815,7 +815,8 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   float* sb = reinterpret_cast<float*>(sm + WyBwdSmem::B);
   float* sEG = reinterpret_cast<float*>(sm + WyBwdSmem::EG);   // e^{G_j}
   float* sRow = reinterpret_cast<float*>(sm + WyBwdSmem::ROW);  // [kind][half][64]
-  // barA: K;  barB: dW, dU^T (hi, lo);  barC: V, T (hi, lo);  barM: MMA batches (4 per unit)
+  // barA: K (double-buffered);  barB: dW, dU^T (hi, lo);  barC: V, T (hi, lo);
+  // barM: MMA batches (4 per unit)
   __shared__ uint64_t barA, barB, barC, barM;
   __shared__ uint32_t tslot;
   int* err = w.status;
@@ -833,11 +834,12 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     tmem_relinquish();
   }
   auto valid = [&](int u) { return u < nunits && w.chunk_tab[u / p.HV].x >= 0; };
-  auto load_A = [&](int u) {
+  auto load_A = [&](int u, int buf) {
     const int hk = (u % p.HV) / p.G, tok0 = w.chunk_tab[u / p.HV].w;
+    unsigned char* dst = sKb + buf * 2 * TILE64;
     mbar_expect_tx(&barA, 2 * TILE64);
-    tma_load_3d(sK, &mk, 0, hk, tok0, &barA);
-    tma_load_3d(sK + TILE64, &mk, 64, hk, tok0, &barA);
+    tma_load_3d(dst, &mk, 0, hk, tok0, &barA);
+    tma_load_3d(dst + TILE64, &mk, 64, hk, tok0, &barA);
   };
   auto load_B = [&](int u) {
     mbar_expect_tx(&barB, 2 * TILE64 + 2 * TILE128);
@@ -857,7 +859,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   int u = blockIdx.x;
   int pendA = -1, pendB = -1, pendC = -1;  // parity of a load group in flight (thread 0)
   if (tid == 0 && valid(u)) {
-    load_A(u);
+    load_A(u, 0);
     load_B(u);
     load_C(u);
     pendA = pendB = pendC = 0;
@@ -886,6 +888,11 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     if (tid == 0) pendA = pendB = pendC = got ? -1 : (int)ph;
     ok = __syncthreads_and(ok && got);
     if (!ok) break;
+    unsigned char* sK = sKb + (it & 1) * 2 * TILE64;
+    if (tid == 0 && nvalid) {  // the other K buffer was last read by the previous unit
+      load_A(nu, (int)(ph ^ 1));
+      pendA = (int)(ph ^ 1);
+    }
     if (L < 64) {
       zero_tail_rows(sK, L, tid, 256);
       zero_tail_rows(sV, L, tid, 256);
@@ -1090,38 +1097,34 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
       }
       mma_commit(&barM);
     }
-    if (tid < 64) {
-      const int j = tid;
+    {  // column j = tid/4 of the dAs*beta*KKG products, four threads per column
+      const int j = tid >> 2, part = tid & 3;
       float cs = 0.f;
-      for (int r = 0; r < 64; ++r) cs += sAA[r * 65 + j];
-      const float eg = sEG[j], bj = sb[j];
-      const float px = sRow[0 * 64 + j] + sRow[1 * 64 + j];
-      const float py = sRow[2 * 64 + j] + sRow[3 * 64 + j];
-      const float pa = sRow[4 * 64 + j] + sRow[5 * 64 + j];
-      const float paa = sRow[6 * 64 + j] + sRow[7 * 64 + j];
-      if (j < L) a.dbeta[(size_t)(tok0 + j) * p.HV + hv] = eg * px + py + pa;
-      w.dG[((size_t)hv * p.NCmax + gc) * 64 + j] += bj * eg * px + paa - cs;
+  #pragma unroll
+      for (int i = 0; i < 16; ++i) cs += sAA[(part + 4 * i) * 65 + j];
+      cs = quad_sum(cs);
+      if (part == 0) {
+        const float eg = sEG[j], bj = sb[j];
+        const float px = sRow[0 * 64 + j] + sRow[1 * 64 + j];
+        const float py = sRow[2 * 64 + j] + sRow[3 * 64 + j];
+        const float pa = sRow[4 * 64 + j] + sRow[5 * 64 + j];
+        const float paa = sRow[6 * 64 + j] + sRow[7 * 64 + j];
+        if (j < L) a.dbeta[(size_t)(tok0 + j) * p.HV + hv] = eg * px + py + pa;
+        w.dG2[((size_t)hv * p.NCmax + gc) * 64 + j] = bj * eg * px + paa - cs;
+      }
     }
     ok = __syncthreads_and(ok && mbar_wait(&barM, 1, err));
     tc_fence_after();
     if (!ok) break;
-    if (tid == 0 && nvalid) {  // K read by the MMAs above for the last time
-      load_A(nu);
-      pendA = (int)(ph ^ 1);
-    }
-    {
+    {  // this kernel's dk share (the assembly adds it to dqkwg's)
       float x[32];
       tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
       tmem_wait_ld();
-      float* dk0 = w.dkp + (unit * 64 + r0) * D + 64 * half + cq;
+      float* dk0 = w.dkp2 + (unit * 64 + r0) * D + 64 * half + cq;
   #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        float2 o0 = *reinterpret_cast<float2*>(dk0 + 8 * j);
-        float2 o1 = *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j);
-        o0.x += x[4 * j]; o0.y += x[4 * j + 1];
-        o1.x += x[4 * j + 2]; o1.y += x[4 * j + 3];
-        *reinterpret_cast<float2*>(dk0 + 8 * j) = o0;
-        *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j) = o1;
+        *reinterpret_cast<float2*>(dk0 + 8 * j) = make_float2(x[4 * j], x[4 * j + 1]);
+        *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j) = make_float2(x[4 * j + 2], x[4 * j + 3]);
       }
     }
     // the next unit's first MMAs overwrite every TMEM column read above
