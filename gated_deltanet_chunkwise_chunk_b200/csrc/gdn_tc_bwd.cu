@@ -161,7 +161,7 @@ struct BwdScanSmem {
 
 // Roles as in the forward scan: thread 0 MMAs, thread 32 TMA stores, thread 64 TMA loads;
 // two CTA-wide barriers per chunk step.
-__global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, TcWork t,
+__global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, TcWork t,
                                                      const __grid_constant__ CUtensorMap mq,
                                                      const __grid_constant__ CUtensorMap mk,
                                                      const __grid_constant__ CUtensorMap mdO,
@@ -174,6 +174,8 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
   const int n = blockIdx.x, hv = blockIdx.y, hk = hv / p.G, v0 = VS * blockIdx.z;
   const int4 sq = w.seq_tab[n];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int wq = warp & 3, wg = warp >> 2;   // TMEM lane quarter, column half of the slice
+  const int kk = tid & 127, vc = 16 * wg;    // this thread: column kk of dS, slice rows vc..vc+15
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
   unsigned char* sK = sm + BwdScanSmem::K;
@@ -204,19 +206,19 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
     tmem_alloc(&tslot, 64);
     tmem_relinquish();
   }
-  float S[VS];
-  const size_t st = ((size_t)n * p.HV + hv) * D * D + (size_t)tid * D + v0;
+  float S[16];
+  const size_t st = ((size_t)n * p.HV + hv) * D * D + (size_t)kk * D + v0 + vc;
 #pragma unroll
-  for (int i = 0; i < VS; i += 4) {
+  for (int i = 0; i < 16; i += 4) {
     const float4 x = a.dht ? *reinterpret_cast<const float4*>(a.dht + st + i) : make_float4(0, 0, 0, 0);
     S[i] = x.x; S[i + 1] = x.y; S[i + 2] = x.z; S[i + 3] = x.w;
   }
-  const uint32_t scol = (uint32_t)((tid >> 6) * TILE_VS + ((tid & 7) << 1));
-  const int sj = (tid & 63) >> 3;
+  const uint32_t scol = (uint32_t)((kk >> 6) * TILE_VS + ((kk & 7) << 1) + vc * 128);
+  const int sj = (kk & 63) >> 3;
 #define S_OFF(i) (scol + (uint32_t)((i) * 128 + (((sj) ^ ((i) & 7)) << 4)))
   auto store_dS = [&]() {
 #pragma unroll
-    for (int i = 0; i < VS; ++i) {
+    for (int i = 0; i < 16; ++i) {
       const bf16 h = __float2bfloat16_rn(S[i]);
       st_bf16_raw(sSH, S_OFF(i), h);
       st_bf16_raw(sSL, S_OFF(i), __float2bfloat16_rn(S[i] - __bfloat162float(h)));
@@ -253,8 +255,9 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
     issue_W(sq.y - 1);
     issue_U(sq.y - 1);
   }
-  if (tid >= 64 && sq.y > 0) {
-    const int c = sq.y - 1, j = tid - 64;
+  const bool vec_thread = tid >= 128 && tid < 192;  // loads the per-chunk vectors
+  if (vec_thread && sq.y > 0) {
+    const int c = sq.y - 1, j = tid - 128;
     const size_t o = vec0 + (size_t)c * 64 + j;
     sDecb[j] = w.Dec[o];
     const float eg = w.EG[o];
@@ -267,15 +270,16 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
   tc_fence_after();
   const uint32_t tb = tslot;
   const uint32_t tE = taddr(tb, 0, 0), tF = taddr(tb, 0, 32);
-  const int ui = 16 * warp + (lane >> 2), uv = 2 * (lane & 3);
-  // per-thread byte offsets of the U-phase elements in a [32][64] slice tile:
-  // element (v = 8j + uv + e, j' = ui + 8r) sits at uoff[r][e] + 1024 j
+  // U-phase elements (this warpgroup's 16 of the 32 columns): rows j' = 16 wq + lane/4 (+8 r),
+  // columns v = vc + 8j + 2(lane%4) + e (j < 2), at byte offset uoff[r][e] + 1024 (2 wg + j)
+  const int ui = 16 * wq + (lane >> 2), uv = 2 * (lane & 3);
   uint32_t uoff[2][2];
 #pragma unroll
   for (int r = 0; r < 2; ++r)
 #pragma unroll
     for (int e = 0; e < 2; ++e)
-      uoff[r][e] = (uint32_t)((uv + e) * 128 + (((2 * warp + r) ^ (uv + e)) << 4) + ((lane >> 2) << 1));
+      uoff[r][e] = (uint32_t)(2048 * wg + (uv + e) * 128 + (((2 * wq + r) ^ (uv + e)) << 4) +
+                              ((lane >> 2) << 1));
   uint32_t ph = 0, phM = 0;  // the tile barriers complete once per chunk, barM1/barM2 once each
   bool ok = true;
   for (int idx = 0; idx < sq.y; ++idx) {
@@ -290,7 +294,7 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
     bool okt = true;
     if (L < 64) {  // ragged chunk: K rows past its end are zeroed before the chain MMA
       okt = mbar_wait(&barK, ph, err);
-      zero_tail_rows(sK, L, tid, 128);
+      zero_tail_rows(sK, L, tid, 256);
       fence_proxy_async();
       __syncthreads();
     }
@@ -315,8 +319,8 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
       tma_store_commit();
     }
     float dn = 0.f, en = 0.f, egc = 0.f;  // next chunk's vectors, stored at the end of the step
-    if (tid >= 64 && more) {
-      const int j = tid - 64;
+    if (vec_thread && more) {
+      const int j = tid - 128;
       const size_t o = vec0 + (size_t)(c - 1) * 64 + j;
       dn = w.Dec[o];
       const float eg = w.EG[o];
@@ -326,9 +330,8 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
     // off the chain while MMA1 runs: -scale e^{G_i} dO[i][v0+v] -> [32 v][64 i] (0 past L),
     // then this thread's dU_loc elements and decay factors
     okt = okt && mbar_wait(&barQO, ph, err);
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int task = tid + 128 * r, i = task & 63, cq = task >> 6;
+    {
+      const int i = tid & 63, cq = tid >> 6;
       float f[8];
       ld_chunk_f(sO, i, (vo >> 3) + cq, TILE64, f);
       const float sc = -sEG[i];
@@ -336,11 +339,11 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
       for (int e = 0; e < 8; ++e) st_bf16(sOS, sw128(8 * cq + e, i, TILE_VS), f[e] * sc);
     }
     okt = okt && mbar_wait(&barU, ph, err);
-    float u[16];
+    float u[8];
 #pragma unroll
     for (int r = 0; r < 2; ++r)
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+      for (int j = 0; j < 2; ++j)
 #pragma unroll
         for (int e = 0; e < 2; ++e) u[4 * j + 2 * r + e] = ld_bf16(sUL, uoff[r][e] + 1024 * j);
     const float dec0 = sDec[ui], dec1 = sDec[ui + 8];
@@ -361,13 +364,13 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
     tc_fence_after();
     if (tid == 64 && more) issue_K(c - 1);  // K consumed by MMA1
     {
-      float d[16];
-      tmem_ld16dp_x4(taddr(tb, 32 * warp, 0), d);
+      float d[8];
+      tmem_ld16dp_x2(taddr(tb, 32 * wq, vc), d);
       tmem_wait_ld();
 #pragma unroll
       for (int r = 0; r < 2; ++r)
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int q = 4 * j + 2 * r + e;
@@ -418,16 +421,15 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
     }
     {
       const float eg = sEGC[buf];
-      float d[VS];
-      tmem_ld16(taddr(tb, 32 * warp, 32), d);
-      tmem_ld16(taddr(tb, 32 * warp, 48), d + 16);
+      float d[16];
+      tmem_ld16(taddr(tb, 32 * wq, 32 + vc), d);
       tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < VS; ++i) S[i] = eg * S[i] - d[i];
+      for (int i = 0; i < 16; ++i) S[i] = eg * S[i] - d[i];
     }
     store_dS();
-    if (tid >= 64 && more) {
-      const int j = tid - 64;
+    if (vec_thread && more) {
+      const int j = tid - 128;
       sDecb[(buf ^ 1) * 64 + j] = dn;
       sEGb[(buf ^ 1) * 64 + j] = en;
       if (j == 63) sEGC[buf ^ 1] = egc;
@@ -442,7 +444,7 @@ __global__ void __launch_bounds__(128) k_tc_scan_bwd(Problem p, Args a, Work w, 
   if (tid == 32) tma_store_wait0();
   if (ok && a.dh0) {
 #pragma unroll
-    for (int i = 0; i < VS; i += 4)
+    for (int i = 0; i < 16; i += 4)
       *reinterpret_cast<float4*>(a.dh0 + st + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
   }
   tc_fence_before();
@@ -1151,7 +1153,7 @@ cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, 
   if ((e = tgo("tc_dvlocal", k_tc_dvlocal, gu, 128, 1024 + 8 * TILE64 + 256, s, p, w, t, m.q, m.k,
                m.dO)))
     return e;
-  if ((e = tgo("tc_scan_bwd", k_tc_scan_bwd, gs, 128, 1024 + BwdScanSmem::TOTAL, s, p, a, w, t, m.q,
+  if ((e = tgo("tc_scan_bwd", k_tc_scan_bwd, gs, 256, 1024 + BwdScanSmem::TOTAL, s, p, a, w, t, m.q,
                m.k, m.dO, m.WT, m.dUlT32, m.dUT32, m.dUTl32, m.dh32)))
     return e;
   const dim3 gp((unsigned)std::min<long long>((long long)p.NCmax * p.HV, num_sms()));
