@@ -145,15 +145,22 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
 //   dU = dU_loc + diag(e^{G_C-G}) E                    (bf16 hi/lo [32 v][64 j] tiles)
 //   MMA2:  F' = Q^T (-scale diag(e^G) dO_z) + W^T dU   (M=128 k, N=32 v, K=64 i)
 //   dS_z^T = e^{G_C} dS_z^T - F'
+// A tensor-core instruction costs about the same at N=32 and N=64 here, so each hi/lo pair
+// is one N=64 operand (hi rows, then lo rows) and the two halves of the result are summed in
+// the epilogue: 8 + 4 + 4 instructions per chunk instead of 16 + 4 + 8.
 // ======================================================================================
 struct BwdScanSmem {
   static constexpr int K = 0, Q = 2 * TILE64, O = 4 * TILE64;  // [64][128], [64][128], [64][64]
   static constexpr int W = 5 * TILE64;                          // W^T [128][64]
   static constexpr int UL = W + TILE128;                        // dU_loc^T slice [32][64]
-  static constexpr int SH = UL + TILE_VS, SL = SH + 2 * TILE_VS;  // dS slice hi / lo [32][128]
-  static constexpr int OS = SL + 2 * TILE_VS;                   // -scale e^G dO^T slice [32][64]
-  static constexpr int UH = OS + TILE_VS, ULO = UH + 2 * TILE_VS;  // 2 x dU^T hi / lo [32][64]
-  static constexpr int DEC = ULO + 2 * TILE_VS;                 // 2 x 64: e^{G_C - G_j}
+  // dS slice as a compensated pair stacked along N: k-block j (64 k) at SHL + 8K j holds the
+  // hi rows [32][64] then the lo rows, so one N=64 operand carries both parts
+  static constexpr int SHL = UL + TILE_VS;
+  // -scale e^G dO^T slice [32][64] followed by 32 zero rows (an N=64 operand whose second
+  // half initialises the lo columns of the accumulator)
+  static constexpr int OSZ = SHL + 4 * TILE_VS;
+  static constexpr int UHL = OSZ + 2 * TILE_VS;                 // 2 x {dU^T hi, lo} [32][64] each
+  static constexpr int DEC = UHL + 4 * TILE_VS;                 // 2 x 64: e^{G_C - G_j}
   static constexpr int EG = DEC + 512;                          // 2 x 64: scale e^{G_i} (0 past L)
   static constexpr int EGC = EG + 512;                          // 2 floats e^{G_C}
   static constexpr int TOTAL = EGC + 64;
@@ -183,9 +190,8 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
   unsigned char* sO = sm + BwdScanSmem::O;
   unsigned char* sW = sm + BwdScanSmem::W;
   unsigned char* sUL = sm + BwdScanSmem::UL;
-  unsigned char* sSH = sm + BwdScanSmem::SH;
-  unsigned char* sSL = sm + BwdScanSmem::SL;
-  unsigned char* sOS = sm + BwdScanSmem::OS;
+  unsigned char* sSHL = sm + BwdScanSmem::SHL;
+  unsigned char* sOS = sm + BwdScanSmem::OSZ;
   float* sDecb = reinterpret_cast<float*>(sm + BwdScanSmem::DEC);
   float* sEGb = reinterpret_cast<float*>(sm + BwdScanSmem::EG);
   float* sEGC = reinterpret_cast<float*>(sm + BwdScanSmem::EGC);
@@ -203,7 +209,7 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
   }
   __syncthreads();
   if (warp == 0) {
-    tmem_alloc(&tslot, 64);
+    tmem_alloc(&tslot, 128);
     tmem_relinquish();
   }
   float S[16];
@@ -213,18 +219,20 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     const float4 x = a.dht ? *reinterpret_cast<const float4*>(a.dht + st + i) : make_float4(0, 0, 0, 0);
     S[i] = x.x; S[i + 1] = x.y; S[i + 2] = x.z; S[i + 3] = x.w;
   }
-  const uint32_t scol = (uint32_t)((kk >> 6) * TILE_VS + ((kk & 7) << 1) + vc * 128);
+  const uint32_t scol = (uint32_t)((kk >> 6) * 2 * TILE_VS + ((kk & 7) << 1) + vc * 128);
   const int sj = (kk & 63) >> 3;
 #define S_OFF(i) (scol + (uint32_t)((i) * 128 + (((sj) ^ ((i) & 7)) << 4)))
   auto store_dS = [&]() {
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const bf16 h = __float2bfloat16_rn(S[i]);
-      st_bf16_raw(sSH, S_OFF(i), h);
-      st_bf16_raw(sSL, S_OFF(i), __float2bfloat16_rn(S[i] - __bfloat162float(h)));
+      st_bf16_raw(sSHL, S_OFF(i), h);
+      st_bf16_raw(sSHL + TILE_VS, S_OFF(i), __float2bfloat16_rn(S[i] - __bfloat162float(h)));
     }
   };
   store_dS();
+  for (int i = tid; i < TILE_VS / 16; i += 256)  // the zero half of the scaled-dO operand
+    reinterpret_cast<uint4*>(sOS + TILE_VS)[i] = make_uint4(0, 0, 0, 0);
   auto row_of = [&](int c) { return ((sq.x + c) * p.HV + hv) * D; };
   auto tok_of = [&](int c) { return sq.z + 64 * c; };
   const int ocol = v0 & ~63, vo = v0 & 63;  // dO column block holding the slice, offset in it
@@ -269,7 +277,8 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
-  const uint32_t tE = taddr(tb, 0, 0), tF = taddr(tb, 0, 32);
+  // TMEM: E (M=64) hi/lo parts in columns [0,32) / [32,64); F' (M=128) in [64,96) / [96,128)
+  const uint32_t tE = taddr(tb, 0, 0), tF = taddr(tb, 0, 64);
   // U-phase elements (this warpgroup's 16 of the 32 columns): rows j' = 16 wq + lane/4 (+8 r),
   // columns v = vc + 8j + 2(lane%4) + e (j < 2), at byte offset uoff[r][e] + 1024 (2 wg + j)
   const int ui = 16 * wq + (lane >> 2), uv = 2 * (lane & 3);
@@ -289,8 +298,8 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     const int srow = row_of(c) + v0;
     const float* sDec = sDecb + buf * 64;
     const float* sEG = sEGb + buf * 64;
-    unsigned char* sUH = sm + BwdScanSmem::UH + buf * TILE_VS;
-    unsigned char* sULo = sm + BwdScanSmem::ULO + buf * TILE_VS;
+    unsigned char* sUH = sm + BwdScanSmem::UHL + buf * 2 * TILE_VS;   // hi rows, then lo rows
+    unsigned char* sULo = sUH + TILE_VS;
     bool okt = true;
     if (L < 64) {  // ragged chunk: K rows past its end are zeroed before the chain MMA
       okt = mbar_wait(&barK, ph, err);
@@ -302,20 +311,16 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
       okt = okt && mbar_wait(&barK, ph, err);
       if (okt) {
         const uint64_t dk = desc_kmajor(smem_u32(sK), 0, TILE64);
-        const uint64_t dh = desc_kmajor(smem_u32(sSH), 0, TILE_VS);
-        const uint64_t dl = desc_kmajor(smem_u32(sSL), 0, TILE_VS);
-        constexpr uint32_t id = idesc_bf16(64, VS, false, false);
+        const uint64_t dhl = desc_kmajor(smem_u32(sSHL), 0, 2 * TILE_VS);
+        constexpr uint32_t id = idesc_bf16(64, 2 * VS, false, false);
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-          mma_bf16(tE, dk + kstep_off(s, TILE64), dh + kstep_off(s, TILE_VS), id, s > 0);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-          mma_bf16(tE, dk + kstep_off(s, TILE64), dl + kstep_off(s, TILE_VS), id, 1);
+        for (int s = 0; s < 8; ++s)  // [E_hi | E_lo] = K [dS_hi; dS_lo]^T
+          mma_bf16(tE, dk + kstep_off(s, TILE64), dhl + kstep_off(s, 2 * TILE_VS), id, s > 0);
         mma_commit(&barM1);
       }
     } else if (tid == 32) {  // dS slice leaving this chunk -> dh
-      tma_store_3d(&mdh32, sSH, 0, srow, 0);
-      tma_store_3d(&mdh32, sSH + TILE_VS, 64, srow, 0);
+      tma_store_3d(&mdh32, sSHL, 0, srow, 0);
+      tma_store_3d(&mdh32, sSHL + 2 * TILE_VS, 64, srow, 0);
       tma_store_commit();
     }
     float dn = 0.f, en = 0.f, egc = 0.f;  // next chunk's vectors, stored at the end of the step
@@ -354,8 +359,8 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     tc_fence_after();
     if (tid == 0 && okt) {
       const uint64_t dQ_ = desc_mnmajor(smem_u32(sQ), 0, TILE64);
-      const uint64_t dOS = desc_kmajor(smem_u32(sOS), 0, TILE_VS);
-      constexpr uint32_t idQ = idesc_bf16(128, VS, true, false);
+      const uint64_t dOS = desc_kmajor(smem_u32(sOS), 0, 2 * TILE_VS);
+      constexpr uint32_t idQ = idesc_bf16(128, 2 * VS, true, false);  // lo columns start at 0
 #pragma unroll
       for (int s = 0; s < 4; ++s)  // F' = Q^T (-scale diag(e^G) dO_z)
         mma_bf16(tF, dQ_ + mnstep_off(s), dOS + kstep_off(s, TILE_VS), idQ, s > 0);
@@ -364,9 +369,12 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     tc_fence_after();
     if (tid == 64 && more) issue_K(c - 1);  // K consumed by MMA1
     {
-      float d[8];
+      float d[8], dl[8];
       tmem_ld16dp_x2(taddr(tb, 32 * wq, vc), d);
+      tmem_ld16dp_x2(taddr(tb, 32 * wq, VS + vc), dl);
       tmem_wait_ld();
+#pragma unroll
+      for (int q = 0; q < 8; ++q) d[q] += dl[q];
 #pragma unroll
       for (int r = 0; r < 2; ++r)
 #pragma unroll
@@ -393,15 +401,11 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
       okt = mbar_wait(&barW, ph, err);
       if (okt) {
         const uint64_t dW_ = desc_kmajor(smem_u32(sW), 0, TILE128);
-        const uint64_t dH_ = desc_kmajor(smem_u32(sUH), 0, TILE_VS);
-        const uint64_t dL_ = desc_kmajor(smem_u32(sULo), 0, TILE_VS);
-        constexpr uint32_t idW = idesc_bf16(128, VS, false, false);
+        const uint64_t dHL = desc_kmajor(smem_u32(sUH), 0, 2 * TILE_VS);
+        constexpr uint32_t idW = idesc_bf16(128, 2 * VS, false, false);
 #pragma unroll
-        for (int s = 0; s < 4; ++s)  // F' += W^T dU  (hi and lo parts)
-          mma_bf16(tF, dW_ + kstep_off(s, TILE128), dH_ + kstep_off(s, TILE_VS), idW, 1);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)
-          mma_bf16(tF, dW_ + kstep_off(s, TILE128), dL_ + kstep_off(s, TILE_VS), idW, 1);
+        for (int s = 0; s < 4; ++s)  // [F'_hi | F'_lo] += W^T [dU_hi | dU_lo]
+          mma_bf16(tF, dW_ + kstep_off(s, TILE128), dHL + kstep_off(s, 2 * TILE_VS), idW, 1);
         mma_commit(&barM2);
       }
     } else if (tid == 32) {  // dU^T of this chunk (hi, lo) -> global
@@ -421,11 +425,12 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
     }
     {
       const float eg = sEGC[buf];
-      float d[16];
-      tmem_ld16(taddr(tb, 32 * wq, 32 + vc), d);
+      float d[16], dl[16];
+      tmem_ld16(taddr(tb, 32 * wq, 64 + vc), d);
+      tmem_ld16(taddr(tb, 32 * wq, 64 + VS + vc), dl);
       tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 16; ++i) S[i] = eg * S[i] - d[i];
+      for (int i = 0; i < 16; ++i) S[i] = eg * S[i] - (d[i] + dl[i]);
     }
     store_dS();
     if (vec_thread && more) {
@@ -449,7 +454,7 @@ __global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, 
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tslot, 64);
+  if (warp == 0) tmem_dealloc(tslot, 128);
 }
 
 // ======================================================================================
