@@ -29,9 +29,9 @@ struct WySmem {
   static constexpr int K = 0, V = 2 * TILE64;
   static constexpr int R1 = 4 * TILE64;                  // {A, X} during the solve, then TX/TY
   static constexpr int TX = R1, TY = R1 + TILE64, TXL = R1 + 2 * TILE64, TYL = R1 + 3 * TILE64;
-  static constexpr int A = R1, X = R1 + 64 * 65 * 4;
-  static constexpr int T = R1 + 34 * 1024;              // fp32 [64][65]
-  static constexpr int G = T + 64 * 65 * 4, B = G + 256, EG = B + 256;
+  static constexpr int A = R1, X = R1 + 64 * LDA * 4;    // fp32 [64][LDA] each
+  static constexpr int T = R1 + 34 * 1024;              // fp32 [64][LDA]
+  static constexpr int G = T + 64 * LDA * 4, B = G + 256, EG = B + 256;
   static constexpr int TOTAL = EG + 256;
 };
 
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int r = r0 + 8 * (q >> 1), cc = 32 * half + 8 * j + 2 * (lane & 3) + (q & 1);
-        sA[r * 65 + cc] = cc < r ? sb[r] * v[4 * j + q] * __expf(sG[r] - sG[cc]) : 0.f;
+        sA[r * LDA + cc] = cc < r ? sb[r] * v[4 * j + q] * __expf(sG[r] - sG[cc]) : 0.f;
       }
   }
   __syncthreads();
@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
     float fx[8], fy[8], ft[8], fl[8];
     for (int q = 0; q < 8; ++q) {
       const int j = jc * 8 + q;
-      ft[q] = sT[i * 65 + j];
+      ft[q] = sT[i * LDA + j];
       fy[q] = ft[q] * sb[j];
       fx[q] = ft[q] * sEG[j];
       fl[q] = ft[q] - __bfloat162float(__float2bfloat16_rn(ft[q]));

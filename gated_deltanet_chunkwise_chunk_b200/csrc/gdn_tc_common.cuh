@@ -188,13 +188,18 @@ __device__ __forceinline__ void st_chunk_split(unsigned char* hi, unsigned char*
   st_chunk_f(lo, r, j, block_bytes, l);
 }
 
-// T = (I + A)^-1 for a strictly lower-triangular 64x64 fp32 A (row stride 65), 256 threads.
+// Row stride (floats) of the fp32 64x64 scratch matrices of the triangular inverse: rows are
+// 16-byte aligned for 128-bit loads, and 68 = 4 (mod 32) spreads consecutive rows over banks.
+constexpr int LDA = 68;
+
+// T = (I + A)^-1 for a strictly lower-triangular 64x64 fp32 A (row stride LDA), 256 threads.
 // The four diagonal 16x16 blocks by forward substitution (warps 0..3, one column per lane)
 // while warps 4..7 zero the strictly upper 16-blocks; then the blocks below the diagonal by
 // block back-substitution, using [[L00, 0], [A10, L11]]^-1 = [[T00, 0], [-T11 A10 T00, T11]]:
 //   16-blocks of each 32x32 half:  T10 = -T11 (A10 T00)        (both halves at once)
 //   32-blocks:                     T[32:,:32] = -T[32:,32:] (A[32:,:32] T[:32,:32])
-// Each thread owns several outputs of a product (fully unrolled dot products).  sX: [64][65].
+// Each thread owns 4 consecutive columns of one output row of a product; operands are read
+// as float4 (a row of A four k at a time, a row of T four columns at a time).  sX: [64][LDA].
 __device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT, float* sX, int tid) {
   const int w = tid >> 5, lane = tid & 31;
   if (w < 4) {
@@ -205,77 +210,83 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT,
       for (int r = 0; r < 16; ++r) {
         float s = (r == c) ? 1.f : 0.f;
 #pragma unroll
-        for (int j = 0; j < r; ++j) s -= sA[(b0 + r) * 65 + b0 + j] * col[j];
+        for (int j = 0; j < r; ++j) s -= sA[(b0 + r) * LDA + b0 + j] * col[j];
         col[r] = (r >= c) ? s : 0.f;
       }
 #pragma unroll
-      for (int r = 0; r < 16; ++r) sT[(b0 + r) * 65 + b0 + c] = col[r];
+      for (int r = 0; r < 16; ++r) sT[(b0 + r) * LDA + b0 + c] = col[r];
     }
   } else {
-    for (int i = tid - 128; i < 6 * 256; i += 128) {  // blocks (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
-      const int blk = i >> 8, r = (i >> 4) & 15, c = i & 15;
+    for (int i = tid - 128; i < 6 * 64; i += 128) {  // blocks (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+      const int blk = i >> 6, r = (i >> 2) & 15, c4 = i & 3;
       const int br = blk < 3 ? 0 : (blk < 5 ? 1 : 2), bc = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-      sT[(16 * br + r) * 65 + 16 * bc + c] = 0.f;
+      *reinterpret_cast<float4*>(sT + (16 * br + r) * LDA + 16 * bc + 4 * c4) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
   __syncthreads();
-  {  // X = A10 T00 in each half p: rows 16(2p+1)+r, columns 32p + c, 32p + c + 8
-    const int p = tid >> 7, q = tid & 127, r = q >> 3, c = q & 7;
-    const int R = 16 * (2 * p + 1) + r, C0 = 32 * p + c;
-    const float* a = sA + R * 65 + 32 * p;
-    const float* t = sT + (32 * p) * 65 + C0;
-    float x0 = 0.f, x1 = 0.f;
+  auto fma4 = [](float4& acc, float a, const float4& b) {
+    acc.x += a * b.x; acc.y += a * b.y; acc.z += a * b.z; acc.w += a * b.w;
+  };
+  // X = A10 T00 in each half p: row 16(2p+1)+r, columns 32p + 4c4 .. +3 (threads 0..127)
+  const int p1 = (tid >> 6) & 1, r1 = (tid >> 2) & 15, c41 = tid & 3;
+  const int R1 = 16 * (2 * p1 + 1) + r1, C1 = 32 * p1 + 4 * c41;
+  if (tid < 128) {
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float av = a[j];
-      x0 += av * t[j * 65];
-      x1 += av * t[j * 65 + 8];
+    for (int j4 = 0; j4 < 4; ++j4) {
+      const float4 a = *reinterpret_cast<const float4*>(sA + R1 * LDA + 32 * p1 + 4 * j4);
+      const float* t = sT + (32 * p1 + 4 * j4) * LDA + C1;
+      fma4(x, a.x, *reinterpret_cast<const float4*>(t));
+      fma4(x, a.y, *reinterpret_cast<const float4*>(t + LDA));
+      fma4(x, a.z, *reinterpret_cast<const float4*>(t + 2 * LDA));
+      fma4(x, a.w, *reinterpret_cast<const float4*>(t + 3 * LDA));
     }
-    sX[R * 65 + C0] = x0;
-    sX[R * 65 + C0 + 8] = x1;
+    *reinterpret_cast<float4*>(sX + R1 * LDA + C1) = x;
   }
   __syncthreads();
-  {  // T10 = -T11 X
-    const int p = tid >> 7, q = tid & 127, r = q >> 3, c = q & 7;
-    const int D0 = 16 * (2 * p + 1), R = D0 + r, C0 = 32 * p + c;
-    const float* tt = sT + R * 65 + D0;
-    const float* x = sX + D0 * 65 + C0;
-    float y0 = 0.f, y1 = 0.f;
+  if (tid < 128) {  // T10 = -T11 X
+    const int D0 = 16 * (2 * p1 + 1);
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const float tv = tt[m];
-      y0 += tv * x[m * 65];
-      y1 += tv * x[m * 65 + 8];
+    for (int m4 = 0; m4 < 4; ++m4) {
+      const float4 tt = *reinterpret_cast<const float4*>(sT + R1 * LDA + D0 + 4 * m4);
+      const float* x = sX + (D0 + 4 * m4) * LDA + C1;
+      fma4(y, tt.x, *reinterpret_cast<const float4*>(x));
+      fma4(y, tt.y, *reinterpret_cast<const float4*>(x + LDA));
+      fma4(y, tt.z, *reinterpret_cast<const float4*>(x + 2 * LDA));
+      fma4(y, tt.w, *reinterpret_cast<const float4*>(x + 3 * LDA));
     }
-    sT[R * 65 + C0] = -y0;
-    sT[R * 65 + C0 + 8] = -y1;
+    *reinterpret_cast<float4*>(sT + R1 * LDA + C1) = make_float4(-y.x, -y.y, -y.z, -y.w);
   }
   __syncthreads();
-  const int r2 = tid >> 3, c2 = tid & 7, R2 = 32 + r2;  // rows 32 + r2, columns c2 + 8q (q < 4)
+  // rows 32 + r2, columns 4c4 .. +3 (all 256 threads)
+  const int r2 = tid >> 3, C2 = 4 * (tid & 7), R2 = 32 + r2;
   {  // X = A[32:,:32] T[:32,:32]
-    const float* a = sA + R2 * 65;
-    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float av = a[j];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) x[q] += av * sT[j * 65 + c2 + 8 * q];
+    for (int j4 = 0; j4 < 8; ++j4) {
+      const float4 a = *reinterpret_cast<const float4*>(sA + R2 * LDA + 4 * j4);
+      const float* t = sT + (4 * j4) * LDA + C2;
+      fma4(x, a.x, *reinterpret_cast<const float4*>(t));
+      fma4(x, a.y, *reinterpret_cast<const float4*>(t + LDA));
+      fma4(x, a.z, *reinterpret_cast<const float4*>(t + 2 * LDA));
+      fma4(x, a.w, *reinterpret_cast<const float4*>(t + 3 * LDA));
     }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) sX[R2 * 65 + c2 + 8 * q] = x[q];
+    *reinterpret_cast<float4*>(sX + R2 * LDA + C2) = x;
   }
   __syncthreads();
   {  // T[32:,:32] = -T[32:,32:] X
-    const float* tt = sT + R2 * 65 + 32;
-    float y[4] = {0.f, 0.f, 0.f, 0.f};
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int m = 0; m < 32; ++m) {
-      const float tv = tt[m];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) y[q] += tv * sX[(32 + m) * 65 + c2 + 8 * q];
+    for (int m4 = 0; m4 < 8; ++m4) {
+      const float4 tt = *reinterpret_cast<const float4*>(sT + R2 * LDA + 32 + 4 * m4);
+      const float* x = sX + (32 + 4 * m4) * LDA + C2;
+      fma4(y, tt.x, *reinterpret_cast<const float4*>(x));
+      fma4(y, tt.y, *reinterpret_cast<const float4*>(x + LDA));
+      fma4(y, tt.z, *reinterpret_cast<const float4*>(x + 2 * LDA));
+      fma4(y, tt.w, *reinterpret_cast<const float4*>(x + 3 * LDA));
     }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) sT[R2 * 65 + c2 + 8 * q] = -y[q];
+    *reinterpret_cast<float4*>(sT + R2 * LDA + C2) = make_float4(-y.x, -y.y, -y.z, -y.w);
   }
   __syncthreads();
 }
