@@ -337,6 +337,7 @@ def main():
 
     # end to end through the public API with host buffers
     e2e = e2e_measure(gdn, case, dev, ws, args.e2e_steps, dist)
+    decode = decode_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"]) if args.config == 2 and args.T is None else None
 
     tokens = case.tokens
     value = aggregate_mtok_s(world, tokens, ms)
@@ -370,6 +371,7 @@ def main():
         "kernels": {k: {"launches": v[0], "ms_per_step": round(v[1] / 2, 4)} for k, v in prof.items()},
         "gpu_launches": int(launches),
         "e2e": e2e,
+        "decode": decode,
         "clocks": clocks,
         "peaks_source": pk["source"],
     }
@@ -495,6 +497,47 @@ def e2e_measure(gdn, case, dev, ws, nsteps: int, dist) -> dict:
     return {"value": round(aggregate_mtok_s(world, case.tokens, ms), 3), "unit": "M tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(ms, 3)}
+
+
+DECODE = dict(B=256, H=16, HV=32, K=128, V=128)
+
+
+def decode_measure(gdn, dev, pk_hbm: float, steps: int = 20) -> dict:
+    """One decode step (T = 1) of 256 sequences with the layer's heads, through
+    gdn_recurrent_fwd with the state updated in place: HBM-bound on the fp32 state, read and
+    written once per (sequence, value head).  A secondary measurement beside the training step."""
+    c = DECODE
+    case = synth.make_case(B=c["B"], T=1, H=c["H"], HV=c["HV"], K=c["K"], V=c["V"], dtype="bf16",
+                           seed=4242, h0=True, name="decode")
+    t = lambda x: None if x is None else x.to(dev).contiguous()
+    d = dict(q=t(case.q), k=t(case.k), v=t(case.v), g_raw=t(case.a), A_log=t(case.A_log),
+             dt_bias=t(case.dt_bias), beta=t(case.beta))
+    st = t(case.h0)
+    o = torch.empty_like(d["v"])
+    ws = torch.empty(gdn.recurrent_workspace_bytes(), dtype=torch.uint8, device=dev)
+
+    def step():
+        gdn.gdn_recurrent_fwd(**d, initial_state=st, final_state=st, out=o, workspace=ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    B, H, HV, K, V = c["B"], c["H"], c["HV"], c["K"], c["V"]
+    nbytes = B * HV * K * V * 4 * 2 + B * (2 * H * K + 2 * HV * V) * 2 + B * HV * 8 + HV * 8
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": f"decode_B{B}_H{H}_HV{HV}_D{K}_bf16", "tokens_per_step": B,
+            "ms_per_step": round(ms, 4), "mtok_s": round(B / (ms / 1e3) / 1e6, 3),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk_hbm, "unit": "GB/s",
+                         "frac": round(gbs / pk_hbm, 4), "bytes_per_step": int(nbytes),
+                         "note": "fp32 state read and written once per (sequence, value head)"}}
 
 
 # ----------------------------------------------------------------- reference arm (oracle)

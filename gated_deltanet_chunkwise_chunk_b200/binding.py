@@ -24,7 +24,8 @@ GDN_FLAG_BWD_REUSE_FWD = 1
 EXPORTED = ("gdn_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_max_chunks",
             "gdn_build_chunk_indices", "gdn_chunk_table_device", "gdn_device_status",
             "gdn_status_string", "gdn_version", "gdn_launch_count", "gdn_profile",
-            "gdn_profile_read", "gdn_chunk_fwd_noalloc", "gdn_noalloc_scratch_bytes")
+            "gdn_profile_read", "gdn_chunk_fwd_noalloc", "gdn_noalloc_scratch_bytes",
+            "gdn_recurrent_fwd", "gdn_recurrent_workspace_bytes")
 
 
 class gdn_dims(ctypes.Structure):
@@ -53,6 +54,10 @@ def _load() -> ctypes.CDLL:
     lib.gdn_chunk_fwd.restype = I32
     lib.gdn_chunk_bwd.argtypes = [D] + [P] * 21 + [SZ, P]
     lib.gdn_chunk_bwd.restype = I32
+    lib.gdn_recurrent_fwd.argtypes = [D] + [P] * 12 + [SZ, P]
+    lib.gdn_recurrent_fwd.restype = I32
+    lib.gdn_recurrent_workspace_bytes.argtypes = []
+    lib.gdn_recurrent_workspace_bytes.restype = SZ
     lib.gdn_max_chunks.argtypes = [D, I32]
     lib.gdn_max_chunks.restype = I64
     lib.gdn_build_chunk_indices.argtypes = [D, P, P, I64]
@@ -182,6 +187,34 @@ def gdn_chunk_fwd_noalloc(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None,
     if rc != GDN_OK:
         raise GDNError("gdn_chunk_fwd_noalloc", rc)
     return o, ht
+
+
+def gdn_recurrent_fwd(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None, initial_state=None,
+                      scale=0.0, out=None, final_state=None, workspace=None):
+    """Token-by-token forward (decode steps, short prefills): returns (o, final_state).  Same
+    arguments and layouts as gdn_chunk_fwd; final_state may be initial_state itself (the
+    state is updated in place).  `workspace` (optional) holds the device status word."""
+    Nst = _check_inputs(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens, initial_state)
+    dims = make_dims(q, v, cu_seqlens, scale)
+    need = int(lib.gdn_recurrent_workspace_bytes())
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    elif workspace.numel() < need:
+        raise ValueError(f"workspace holds {workspace.numel()} bytes, the call needs {need}")
+    o = out if out is not None else torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    ht = final_state if final_state is not None else torch.empty(
+        (Nst, v.shape[2], q.shape[3], v.shape[3]), dtype=torch.float32, device=q.device)
+    rc = lib.gdn_recurrent_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g_raw),
+                               _ptr(A_log), _ptr(dt_bias), _ptr(beta), _ptr(cu_seqlens),
+                               _ptr(initial_state), _ptr(o), _ptr(ht), _ptr(workspace),
+                               workspace.numel(), _stream())
+    if rc != GDN_OK:
+        raise GDNError("gdn_recurrent_fwd", rc)
+    return o, ht
+
+
+def recurrent_workspace_bytes() -> int:
+    return int(lib.gdn_recurrent_workspace_bytes())
 
 
 def noalloc_scratch_bytes() -> int:

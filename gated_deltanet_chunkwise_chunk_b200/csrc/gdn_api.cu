@@ -311,6 +311,44 @@ int gdn_chunk_table_device(const gdn_dims* d, const int64_t* cu_seqlens, int32_t
                                              count_dev, static_cast<cudaStream_t>(stream)));
 }
 
+size_t gdn_recurrent_workspace_bytes(void) { return GDN_RECURRENT_WORKSPACE_BYTES; }
+
+int gdn_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                      const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,
+                      const int64_t* cu_seqlens, const float* initial_state, void* o,
+                      float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
+  const bool varlen = cu_seqlens != nullptr;
+  int rc = check_dims(d, varlen);
+  if (rc) return rc;
+  const bool empty = d->B * d->T == 0;
+  const void* tok[] = {q, k, v, g_raw, beta, o};
+  for (const void* x : tok)
+    if ((!x && !empty) || !aligned16(x)) return GDN_ERR_INVALID_ARG;
+  if (!A_log || !dt_bias || !aligned16(A_log) || !aligned16(dt_bias)) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(cu_seqlens) || !aligned16(initial_state) || !aligned16(final_state))
+    return GDN_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) ||
+      workspace_bytes < GDN_RECURRENT_WORKSPACE_BYTES)
+    return GDN_ERR_WORKSPACE;
+  const Problem p = make_problem(*d, varlen);
+  Args a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.g_raw = g_raw;
+  a.A_log = A_log;
+  a.dt_bias = dt_bias;
+  a.beta = beta;
+  a.cu = cu_seqlens;
+  a.h0 = initial_state;
+  a.o = o;
+  a.ht = final_state;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 64, s);  // the device status word
+  if (e == cudaSuccess) e = recurrent_forward(p, a, static_cast<int*>(workspace), d->dtype == GDN_DTYPE_BF16, s);
+  return cuda_status(e);
+}
+
 int gdn_device_status(const void* workspace, void* stream) {
   if (!workspace) return GDN_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

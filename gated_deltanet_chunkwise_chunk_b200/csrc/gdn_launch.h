@@ -30,6 +30,8 @@ cudaError_t launch_bwd_tokens(const Problem& p, const Args& a, const Work& w, bo
                               cudaStream_t s);
 
 // fp32 CUDA-core path (FFMA tiles): used for fp32 tensors.
+// Token-by-token forward (decoding, short prefills); status: device status word.
+cudaError_t recurrent_forward(const Problem& p, const Args& a, int* status, bool bf16, cudaStream_t s);
 cudaError_t ffma_forward(const Problem& p, const Args& a, const Work& w, bool bf16, bool bwd_prep,
                          cudaStream_t s);
 cudaError_t ffma_backward(const Problem& p, const Args& a, const Work& w, bool bf16,

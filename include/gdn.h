@@ -130,6 +130,27 @@ int gdn_chunk_fwd_noalloc(const gdn_dims* d, const void* q, const void* k, const
 /* Size in bytes of the array gdn_chunk_fwd_noalloc uses (GDN_NOALLOC_SCRATCH_BYTES). */
 size_t gdn_noalloc_scratch_bytes(void);
 
+/* Token-by-token (recurrent) forward for decoding and short prefills: the same operation and
+ * the same arguments as gdn_chunk_fwd (o for every token, final_state after each sequence's
+ * last token), computed one token after another as the recurrence at the top of this file is
+ * written, with each (sequence, value head) state read once and written once.  This is the
+ * form the chunkwise algorithm reassociates (Ascend GDN blog and the G_T_CONTIG page treat
+ * the chunk kernels; the decode step is the same recurrence with T = 1 per sequence).  Cost
+ * is linear in T per sequence with no parallelism across a sequence's tokens: use it for
+ * T = 1 decode steps and prefills of a few tokens, gdn_chunk_fwd for long sequences.
+ * final_state may be the same buffer as initial_state (the state is updated in place).
+ * workspace: at least GDN_RECURRENT_WORKSPACE_BYTES, 256-byte aligned; it holds the device
+ * status word (gdn_device_status reports invalid cu_seqlens as GDN_ERR_INVALID_ARG). */
+#define GDN_RECURRENT_WORKSPACE_BYTES ((size_t)256)
+int gdn_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                      const float* g_raw, const float* A_log, const float* dt_bias,
+                      const float* beta, const int64_t* cu_seqlens, const float* initial_state,
+                      void* o, float* final_state, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/* GDN_RECURRENT_WORKSPACE_BYTES. */
+size_t gdn_recurrent_workspace_bytes(void);
+
 /* Upper bound on the number of 64-token chunks (the grid size used for chunk kernels). */
 int64_t gdn_max_chunks(const gdn_dims* d, int varlen);
 

@@ -78,6 +78,17 @@ def test_entry_points_reject_bad_arguments_before_launch():
     rc = lib.gdn_chunk_bwd(ctypes.byref(d), al, al, al, al, al, al, al, null, null, al, null,
                            al, al, al, null, al, null, null, null, null, al, 1 << 40, null)
     assert rc == binding.GDN_ERR_INVALID_ARG
+    # recurrent forward: null input, small workspace, unsupported V
+    rc = lib.gdn_recurrent_fwd(ctypes.byref(d), null, al, al, al, al, al, al, null, null, al, null,
+                               al, 1 << 20, null)
+    assert rc == binding.GDN_ERR_INVALID_ARG
+    rc = lib.gdn_recurrent_fwd(ctypes.byref(d), al, al, al, al, al, al, al, null, null, al, null,
+                               al, 64, null)
+    assert rc == binding.GDN_ERR_WORKSPACE
+    rc = lib.gdn_recurrent_fwd(ctypes.byref(_dims(V=96)), al, al, al, al, al, al, al, null, null,
+                               al, null, al, 1 << 20, null)
+    assert rc == binding.GDN_ERR_UNSUPPORTED
+    assert lib.gdn_recurrent_workspace_bytes() == 256
 
 
 def _enumerate(cu, B, T):
