@@ -6,9 +6,10 @@
 // (the decay applies before the erase, as in the chunkwise algebra).  HBM-bound at T = 1:
 // 2 x 4KV bytes of state per (sequence, value head) plus the token vectors.
 //
-// CTA (sequence, value head, z) holds rows v0 = 32z .. v0+31 of S; thread (v, kq) keeps
-// S[v0+v][kq*K/4 .. (kq+1)*K/4) in fp32 registers, the four kq threads of a row being adjacent
-// lanes (row sums by two shuffles).
+// CTA (sequence, value head, z) holds rows v0 = 32z .. v0+31 of S.  Thread (kg, vg) keeps
+// S[v0+4vg .. +3][kg*K/16 .. (kg+1)*K/16) in fp32 registers, so the state moves as 16-byte
+// rows of h[k][v]; the 16 k-groups of a column block sit in one warp (lane = kg + 16 (vg%2)),
+// so row sums are four shuffles.
 #include "gdn_common.cuh"
 #include "gdn_launch.h"
 
@@ -19,9 +20,9 @@ constexpr int RV = 32;  // state rows per CTA
 
 template <typename T, int K>
 __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* status) {
-  constexpr int KQ = K / 4;  // state columns per thread
+  constexpr int KQ = K / 16;  // state columns per thread
   const int n = blockIdx.x, hv = blockIdx.y, hk = hv / p.G, v0 = RV * blockIdx.z;
-  const int tid = threadIdx.x, vl = tid >> 2, kq = tid & 3;
+  const int tid = threadIdx.x, lane = tid & 31, kg = lane & 15, vg = 2 * (tid >> 5) + (lane >> 4);
   __shared__ float sk[K], sq[K], sv[RV], sdec, sbeta;
   int bos, eos;
   if (p.varlen) {
@@ -37,16 +38,25 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
     bos = n * p.T;
     eos = bos + p.T;
   }
-  // state: h[k][v] = S[v][k], fp32 [Nst][HV][K][V]
-  const size_t st = ((size_t)n * p.HV + hv) * K * p.V + v0 + vl;
-  float S[KQ];
+  // state: h[k][v] = S[v][k], fp32 [Nst][HV][K][V]; S4[i] = S[v0+4vg .. +3][kg*KQ + i]
+  const size_t st = ((size_t)n * p.HV + hv) * K * p.V + v0 + 4 * vg;
+  float4 S4[KQ];
 #pragma unroll
-  for (int i = 0; i < KQ; ++i) S[i] = a.h0 ? a.h0[st + (size_t)(kq * KQ + i) * p.V] : 0.f;
+  for (int i = 0; i < KQ; ++i)
+    S4[i] = a.h0 ? *reinterpret_cast<const float4*>(a.h0 + st + (size_t)(kg * KQ + i) * p.V)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
   const T* q = static_cast<const T*>(a.q);
   const T* k = static_cast<const T*>(a.k);
   const T* v = static_cast<const T*>(a.v);
   T* o = static_cast<T*>(a.o);
   const float nexp = -expf(a.A_log[hv]), dtb = a.dt_bias[hv];
+  auto rowsum = [](float x) {  // over the 16 k-groups of this lane half
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    x += __shfl_xor_sync(0xffffffffu, x, 4);
+    x += __shfl_xor_sync(0xffffffffu, x, 8);
+    return x;
+  };
   for (int t = bos; t < eos; ++t) {
     __syncthreads();  // the previous token's vectors are no longer read
     const size_t qk0 = ((size_t)t * p.H + hk) * K, v_0 = ((size_t)t * p.HV + hv) * p.V + v0;
@@ -63,28 +73,37 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
     }
     __syncthreads();
     const float dec = sdec, b = sbeta;
-    float e = 0.f;
+    float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < KQ; ++i) {
-      S[i] *= dec;
-      e += S[i] * sk[kq * KQ + i];
+      const float kv = sk[kg * KQ + i];
+      S4[i].x *= dec; S4[i].y *= dec; S4[i].z *= dec; S4[i].w *= dec;
+      e.x += S4[i].x * kv; e.y += S4[i].y * kv; e.z += S4[i].z * kv; e.w += S4[i].w * kv;
     }
-    e += __shfl_xor_sync(0xffffffffu, e, 1);
-    e += __shfl_xor_sync(0xffffffffu, e, 2);
-    const float dl = b * (sv[vl] - e);
-    float y = 0.f;
+    e.x = rowsum(e.x); e.y = rowsum(e.y); e.z = rowsum(e.z); e.w = rowsum(e.w);
+    const float* vv = sv + 4 * vg;
+    const float dx = b * (vv[0] - e.x), dy = b * (vv[1] - e.y), dz = b * (vv[2] - e.z),
+                dw = b * (vv[3] - e.w);
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < KQ; ++i) {
-      S[i] += dl * sk[kq * KQ + i];
-      y += S[i] * sq[kq * KQ + i];
+      const float kv = sk[kg * KQ + i], qv = sq[kg * KQ + i];
+      S4[i].x += dx * kv; S4[i].y += dy * kv; S4[i].z += dz * kv; S4[i].w += dw * kv;
+      y.x += S4[i].x * qv; y.y += S4[i].y * qv; y.z += S4[i].z * qv; y.w += S4[i].w * qv;
     }
-    y += __shfl_xor_sync(0xffffffffu, y, 1);
-    y += __shfl_xor_sync(0xffffffffu, y, 2);
-    if (kq == 0) o[v_0 + vl] = from_f<T>(p.scale * y);
+    y.x = rowsum(y.x); y.y = rowsum(y.y); y.z = rowsum(y.z); y.w = rowsum(y.w);
+    if (kg == 0) {
+      T* oo = o + v_0 + 4 * vg;
+      oo[0] = from_f<T>(p.scale * y.x);
+      oo[1] = from_f<T>(p.scale * y.y);
+      oo[2] = from_f<T>(p.scale * y.z);
+      oo[3] = from_f<T>(p.scale * y.w);
+    }
   }
   if (a.ht) {
 #pragma unroll
-    for (int i = 0; i < KQ; ++i) a.ht[st + (size_t)(kq * KQ + i) * p.V] = S[i];
+    for (int i = 0; i < KQ; ++i)
+      *reinterpret_cast<float4*>(a.ht + st + (size_t)(kg * KQ + i) * p.V) = S4[i];
   }
 }
 
