@@ -517,24 +517,25 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
   tc_fence_after();
-  // P = QK * Gam (lower incl. diagonal): row i = 16*(warp%4) + lane (lanes < 16), columns
-  // [32*half, 32*half + 32)
-  const int i = 16 * (warp & 3) + lane, half = warp >> 2;
-  if (ok) {
-    float d[32];
-    tmem_ld16(taddr(tb, 32 * (warp & 3), 128 + 32 * half), d);
-    tmem_ld16(taddr(tb, 32 * (warp & 3), 128 + 32 * half + 16), d + 16);
+  // M=64 accumulators read with 16-lane loads: rows r0 = 16 (warp%4) + lane/4 and r0 + 8,
+  // this warp half's columns 8j + 2(lane%4) + {0,1}
+  const int half = warp >> 2, r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
+  const float g0 = sG[r0], g1 = sG[r0 + 8];
+  if (ok) {  // P = QK * Gam (lower incl. diagonal), columns [32 half, +32), as a hi/lo pair
+    float d[16];
+    tmem_ld16dp_x4(taddr(tb, 32 * (warp & 3), 128 + 32 * half), d);
     tmem_wait_ld();
-    if (lane < 16) {
-      const float gi = sG[i];
-      for (int j = 0; j < 4; ++j) {
-        float f[8];
-        for (int q = 0; q < 8; ++q) {
-          const int jj = 32 * half + 8 * j + q;
-          f[q] = jj <= i ? d[8 * j + q] * expf(gi - sG[jj]) : 0.f;
-        }
-        st_chunk_split(sP, sPl, i, half * 4 + j, TILE64, f);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = 32 * half + 8 * j + cq;
+      float f[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = r0 + 8 * (q >> 1), col = c + (q & 1);
+        f[q] = col <= i ? d[4 * j + q] * __expf((q < 2 ? g0 : g1) - sG[col]) : 0.f;
       }
+      st_pair_split(sP, sPl, r0, c, TILE64, f[0], f[1]);
+      st_pair_split(sP, sPl, r0 + 8, c, TILE64, f[2], f[3]);
     }
   }
   fence_proxy_async();
@@ -553,25 +554,22 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
   tc_fence_after();
-  if (ok) {
-    const float eg = expf(sG[i]) * p.scale;
-    bf16* orow = static_cast<bf16*>(a.o) + ((size_t)(tok0 + i) * p.HV + hv) * D + 64 * half;
-    for (int cc = 0; cc < 64; cc += 16) {
-      float x[16], y[16];
-      tmem_ld16(taddr(tb, 32 * (warp & 3), 64 * half + cc), x);
-      tmem_ld16(taddr(tb, 32 * (warp & 3), 128 + 64 * half + cc), y);
-      tmem_wait_ld();
-      if (lane < 16 && i < L) {
-        uint4 o0, o1;
-        float f[16];
-        for (int q = 0; q < 16; ++q) f[q] = eg * x[q] + p.scale * y[q];
-        o0.x = pack_bf16(f[0], f[1]); o0.y = pack_bf16(f[2], f[3]);
-        o0.z = pack_bf16(f[4], f[5]); o0.w = pack_bf16(f[6], f[7]);
-        o1.x = pack_bf16(f[8], f[9]); o1.y = pack_bf16(f[10], f[11]);
-        o1.z = pack_bf16(f[12], f[13]); o1.w = pack_bf16(f[14], f[15]);
-        *reinterpret_cast<uint4*>(orow + cc) = o0;
-        *reinterpret_cast<uint4*>(orow + cc + 8) = o1;
-      }
+  if (ok) {  // O = scale (e^{G_i} X + Y), columns [64 half, +64)
+    float x[32], y[32];
+    tmem_ld16dp_x8(taddr(tb, 32 * (warp & 3), 64 * half), x);
+    tmem_ld16dp_x8(taddr(tb, 32 * (warp & 3), 128 + 64 * half), y);
+    tmem_wait_ld();
+    const float e0 = __expf(g0) * p.scale, e1 = __expf(g1) * p.scale;
+    bf16* o0 = static_cast<bf16*>(a.o) + ((size_t)(tok0 + r0) * p.HV + hv) * D + 64 * half + cq;
+    bf16* o1 = o0 + (size_t)8 * p.HV * D;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (r0 < L)
+        *reinterpret_cast<uint32_t*>(o0 + 8 * j) =
+            pack_bf16(e0 * x[4 * j] + p.scale * y[4 * j], e0 * x[4 * j + 1] + p.scale * y[4 * j + 1]);
+      if (r0 + 8 < L)
+        *reinterpret_cast<uint32_t*>(o1 + 8 * j) =
+            pack_bf16(e1 * x[4 * j + 2] + p.scale * y[4 * j + 2], e1 * x[4 * j + 3] + p.scale * y[4 * j + 3]);
     }
   }
   tc_fence_before();

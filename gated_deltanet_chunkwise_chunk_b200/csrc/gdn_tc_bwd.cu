@@ -79,21 +79,24 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
   tc_fence_after();
   if (ok) {
-    const int i = 16 * warp + lane;
-    for (int c = 0; c < 64; c += 16) {
-      float d[16];
-      tmem_ld16(taddr(tb, 32 * warp, c), d);
-      tmem_wait_ld();
-      if (lane < 16) {
-        const float gi = sG[i];
-        float f[16];
-        for (int q = 0; q < 16; ++q) {
-          const int j = c + q;
-          f[q] = (j <= i && i < L) ? d[q] * expf(gi - sG[j]) : 0.f;
-        }
-        st_chunk_split(sP, sPl, i, c / 8, TILE64, f);
-        st_chunk_split(sP, sPl, i, c / 8 + 1, TILE64, f + 8);
+    // M=64 accumulator with 16-lane loads: rows r0 = 16 warp + lane/4 and r0 + 8,
+    // columns 8j + 2(lane%4) + {0,1}
+    float d[32];
+    tmem_ld16dp_x8(taddr(tb, 32 * warp, 0), d);
+    tmem_wait_ld();
+    const int r0 = 16 * warp + (lane >> 2), cq = 2 * (lane & 3);
+    const float g0 = sG[r0], g1 = sG[r0 + 8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = 8 * j + cq;
+      float f[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = r0 + 8 * (q >> 1), col = c + (q & 1);
+        f[q] = (col <= i && i < L) ? d[4 * j + q] * __expf((q < 2 ? g0 : g1) - sG[col]) : 0.f;
       }
+      st_pair_split(sP, sPl, r0, c, TILE64, f[0], f[1]);
+      st_pair_split(sP, sPl, r0 + 8, c, TILE64, f[2], f[3]);
     }
   }
   fence_proxy_async();
