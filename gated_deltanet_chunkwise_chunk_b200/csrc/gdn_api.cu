@@ -41,7 +41,7 @@ int check_dims(const gdn_dims* d, bool varlen) {
 // own regions after the common ones).
 struct Plan {
   size_t status, seq_tab, chunk_tab, G, beta_p, Dec, EG;
-  size_t W, Ut, Tm, h, U, dU, dh, dW, dqp, dkp, dG, dkp2, dG2, tmp;
+  size_t W, Ut, Tm, h, U, dU, dh, dW, dqp, dkp, dG, dkp2, dG2, tmp, pgp;
   size_t tc;     // start of the tcgen05 path's region
   size_t total;
 };
@@ -93,6 +93,7 @@ Plan make_plan(const gdn_dims& d, bool varlen, int pass) {
       pl.dG2 = take(HV * NC * CH * f);
     }
   }
+  if (pass == 1) pl.pgp = take((size_t)PG_BLOCKS * HV * 2 * f);
   pl.total = o;
   return pl;
 }
@@ -122,6 +123,7 @@ Work carve(const Plan& pl, void* ws) {
   w.dkp2 = fp(pl.dkp2);
   w.dG2 = fp(pl.dG2);
   w.tmp = fp(pl.tmp);
+  w.pgp = fp(pl.pgp);
   return w;
 }
 
@@ -254,10 +256,13 @@ int gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v
   a.ddt_bias = ddt_bias;
   const Work w = carve(pl, workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = prologue(p, a, w, s);
-  if (e != cudaSuccess) return cuda_status(e);
   const bool bf16 = d->dtype == GDN_DTYPE_BF16;
-  if (bf16 && tc_bwd_supported(*d)) {
+  const bool tc = bf16 && tc_bwd_supported(*d);
+  // with the forward's workspace reused, its chunk tables, gates and status word are kept
+  const bool reuse = tc && (d->flags & GDN_FLAG_BWD_REUSE_FWD) != 0;
+  cudaError_t e = reuse ? cudaSuccess : prologue(p, a, w, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (tc) {
     e = tc_backward(p, a, w, static_cast<char*>(workspace) + pl.tc,
                     (d->flags & GDN_FLAG_BWD_REUSE_FWD) != 0, s);
     if (e != cudaSuccess) return cuda_status(e);

@@ -9,7 +9,8 @@
 
 namespace gdn {
 
-constexpr int CH = 64;  // tokens per chunk
+constexpr int CH = 64;         // tokens per chunk
+constexpr int PG_BLOCKS = 128;  // token blocks of the gate-parameter gradient reduction
 
 // Launch-wide problem description (passed by value to every kernel).
 struct Problem {
@@ -46,6 +47,7 @@ struct Work {
   float* dkp2;        // [NCmax][HV][64][K]    tcgen05 path: the WY backward's dk share (or null)
   float* dG2;         // [HV][NCmax][64]       tcgen05 path: the WY backward's dG part (or null)
   float* tmp;         // [NCmax][HV][64][128]  per-unit scratch
+  float* pgp;         // [PG_BLOCKS][HV][2]    partial sums of the gate-parameter gradients
 };
 
 // Pointers of one call (inputs and outputs as given by the caller).

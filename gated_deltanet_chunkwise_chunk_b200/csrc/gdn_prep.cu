@@ -200,6 +200,53 @@ __global__ void __launch_bounds__(256) k_dqdk_group_sum(Problem p, Args a, Work 
 
 // dA_log[hv] = sum_t dg_t g_t ;  ddt_bias[hv] = sum_t dL/dx_t.  One block per value head,
 // deterministic order.
+// dA_log = sum_t dg_t g_t and ddt_bias = sum_t dg_t (-e^{A_log}) softplus'(x_t) per value head,
+// in two deterministic passes: PG_BLOCKS token blocks each write per-head partial sums
+// (threads read [token][head] rows contiguously; 256 % HV == 0 keeps a thread on one head),
+// then one thread per head adds the partials in block order.
+__global__ void __launch_bounds__(256) k_param_grads_partial(Problem p, Args a, Work w) {
+  if (call_failed(w)) return;
+  const int HV = p.HV, tid = threadIdx.x, h = tid % HV, lanes = 256 / HV, l = tid / HV;
+  const int ntok = p.B * p.T;
+  const int per = (ntok + PG_BLOCKS - 1) / PG_BLOCKS;
+  const int t0 = blockIdx.x * per, t1 = min(ntok, t0 + per);
+  const float Al = a.A_log[h], db = a.dt_bias[h], nexp = -expf(Al);
+  float s1 = 0.f, s2 = 0.f;
+  for (int t = t0 + l; t < t1; t += lanes) {
+    const size_t off = (size_t)t * HV + h;
+    const float dgv = a.dg[off], x = a.g_raw[off] + db;
+    s1 += dgv * gate_value(a.g_raw[off], Al, db);
+    s2 += dgv * nexp * gate_dsoftplus(x);
+  }
+  __shared__ float r1[256], r2[256];
+  r1[tid] = s1;
+  r2[tid] = s2;
+  __syncthreads();
+  if (tid < HV) {
+    float u1 = 0.f, u2 = 0.f;
+    for (int j = 0; j < lanes; ++j) {
+      u1 += r1[j * HV + tid];
+      u2 += r2[j * HV + tid];
+    }
+    w.pgp[((size_t)blockIdx.x * HV + tid) * 2] = u1;
+    w.pgp[((size_t)blockIdx.x * HV + tid) * 2 + 1] = u2;
+  }
+}
+
+__global__ void k_param_grads_final(Problem p, Args a, Work w) {
+  if (call_failed(w)) return;
+  for (int h = blockIdx.x * blockDim.x + threadIdx.x; h < p.HV; h += gridDim.x * blockDim.x) {
+    float u1 = 0.f, u2 = 0.f;
+    for (int b = 0; b < PG_BLOCKS; ++b) {
+      u1 += w.pgp[((size_t)b * p.HV + h) * 2];
+      u2 += w.pgp[((size_t)b * p.HV + h) * 2 + 1];
+    }
+    if (a.dA_log) a.dA_log[h] = u1;
+    if (a.ddt_bias) a.ddt_bias[h] = u2;
+  }
+}
+
+// One CTA per value head (any HV): the reduction when 256 % HV != 0.
 __global__ void __launch_bounds__(256) k_param_grads(Problem p, Args a, Work w) {
   if (call_failed(w)) return;
   const int hv = blockIdx.x;
@@ -258,14 +305,28 @@ cudaError_t launch_gate_cumsum(const Problem& p, const Args& a, const Work& w, c
   return cudaGetLastError();
 }
 
+cudaError_t launch_param_grads(const Problem& p, const Args& a, const Work& w, cudaStream_t s) {
+  if (!(a.dA_log || a.ddt_bias)) return cudaSuccess;
+  if (256 % p.HV == 0 && w.pgp) {
+    {
+      ProfScope ps("param_grads", s);
+      k_param_grads_partial<<<PG_BLOCKS, 256, 0, s>>>(p, a, w);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ProfScope ps("param_grads_final", s);
+    k_param_grads_final<<<(p.HV + 255) / 256, 256, 0, s>>>(p, a, w);
+  } else {
+    ProfScope ps("param_grads", s);
+    k_param_grads<<<p.HV, 256, 0, s>>>(p, a, w);
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_bwd_tokens(const Problem& p, const Args& a, const Work& w, bool bf16,
                               cudaStream_t s) {
   if (p.NCmax == 0 && !(a.dA_log || a.ddt_bias)) return cudaSuccess;
-  if (p.NCmax == 0) {
-    ProfScope ps("param_grads", s);
-    k_param_grads<<<p.HV, 256, 0, s>>>(p, a, w);
-    return cudaGetLastError();
-  }
+  if (p.NCmax == 0) return launch_param_grads(p, a, w, s);
   {
     ProfScope ps("bwd_tokens", s);
     k_bwd_tokens<<<p.NCmax, 256, 0, s>>>(p, a, w);
@@ -281,11 +342,7 @@ cudaError_t launch_bwd_tokens(const Problem& p, const Args& a, const Work& w, bo
       k_dqdk_group_sum<float><<<g, 256, 0, s>>>(p, a, w);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (a.dA_log || a.ddt_bias) {
-    ProfScope ps("param_grads", s);
-    k_param_grads<<<p.HV, 256, 0, s>>>(p, a, w);
-    e = cudaGetLastError();
-  }
+  if (a.dA_log || a.ddt_bias) e = launch_param_grads(p, a, w, s);
   return e;
 }
 

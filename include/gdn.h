@@ -77,7 +77,8 @@ typedef enum gdn_flags {
   /* gdn_chunk_bwd only: `workspace` still holds what gdn_chunk_fwd wrote for the same
    * dimensions and the same input contents (the caller ran the forward with this workspace
    * and changed neither since), so the backward uses the forward's saved chunk
-   * intermediates (W, U~, T, v_new, per-chunk states) instead of recomputing them.  The
+   * intermediates (chunk table, in-chunk gate sums, W, U~, T, v_new, per-chunk states) and
+   * its device status word instead of recomputing them.  The
    * workspace must be sized for the backward (gdn_workspace_bytes(.., 1) >= the forward's)
    * and passed to both calls.  Honoured by the bf16 K = V = 128 path; other paths always
    * recompute, with identical results. */
