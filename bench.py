@@ -80,8 +80,8 @@ def kernel_bytes_per_unit(K: int, V: int, G: int, e: int) -> dict:
         "dvlocal": 2 * tq + tv + vec + ut,
         "scan_bwd": 2 * tq + tv + wt + ut + 2 * vec + st + 2 * ut,
         "dqkwg": 2 * tq + tv + 3 * ut + 2 * st + vec + wt + 2 * f32 + vec,
-        "wy_bwd": tq + tv + tm + wt + 2 * ut + 2 * vec + tv + f32 + 2 * vec,
-        "dqdk_group_sum": 3 * f32 + 2 * tq,
+        "wy_bwd": tq + tv + tm + wt + 2 * ut + 2 * vec + tv + 2 * f32 + 2 * vec,  # dk share added in L2
+        "dqdk_group_sum": 2 * f32 + 2 * tq,
     }
     return {f"tc_{k}" if k != "dqdk_group_sum" else k: v for k, v in per.items()}
 

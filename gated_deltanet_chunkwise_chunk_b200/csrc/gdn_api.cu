@@ -89,7 +89,6 @@ Plan make_plan(const gdn_dims& d, bool varlen, int pass) {
       pl.dqp = take(NC * HV * CH * K * f);
       pl.dkp = take(NC * HV * CH * K * f);
       pl.dG = take(HV * NC * CH * f);
-      pl.dkp2 = take(NC * HV * CH * K * f);
       pl.dG2 = take(HV * NC * CH * f);
     }
   }

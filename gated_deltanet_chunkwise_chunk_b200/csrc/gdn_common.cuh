@@ -44,7 +44,7 @@ struct Work {
   float* dqp;         // [NCmax][HV][64][K]    per-value-head dq share
   float* dkp;         // [NCmax][HV][64][K]    per-value-head dk share
   float* dG;          // [HV][NCmax][64]       dL/dG (before the reverse cumsum)
-  float* dkp2;        // [NCmax][HV][64][K]    tcgen05 path: the WY backward's dk share (or null)
+  float* dkp2;        // [NCmax][HV][64][K]    a second dk share summed by the assembly (or null)
   float* dG2;         // [HV][NCmax][64]       tcgen05 path: the WY backward's dG part (or null)
   float* tmp;         // [NCmax][HV][64][128]  per-unit scratch
   float* pgp;         // [PG_BLOCKS][HV][2]    partial sums of the gate-parameter gradients

@@ -1126,15 +1126,16 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     ok = __syncthreads_and(ok && mbar_wait(&barM, 1, err));
     tc_fence_after();
     if (!ok) break;
-    {  // this kernel's dk share (the assembly adds it to dqkwg's)
+    {  // this kernel's dk share, added onto dqkwg's in L2 (one reduction per element onto a
+       // value written by the previous kernel: the sum is the same on every run)
       float x[32];
       tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
       tmem_wait_ld();
-      float* dk0 = w.dkp2 + (unit * 64 + r0) * D + 64 * half + cq;
+      float* dk0 = w.dkp + (unit * 64 + r0) * D + 64 * half + cq;
   #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        *reinterpret_cast<float2*>(dk0 + 8 * j) = make_float2(x[4 * j], x[4 * j + 1]);
-        *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j) = make_float2(x[4 * j + 2], x[4 * j + 3]);
+        atomicAdd(reinterpret_cast<float2*>(dk0 + 8 * j), make_float2(x[4 * j], x[4 * j + 1]));
+        atomicAdd(reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j), make_float2(x[4 * j + 2], x[4 * j + 3]));
       }
     }
     // the next unit's first MMAs overwrite every TMEM column read above
