@@ -254,7 +254,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--T", type=int, default=None,
                     help="override the sequence length of a dense workload (smaller profiling cases)")
     ap.add_argument("--ref-budget", type=float, default=90.0,
@@ -451,52 +451,94 @@ def _traffic(name: str, case):
 
 
 def e2e_measure(gdn, case, dev, ws, nsteps: int, dist) -> dict:
-    """Same step through the public API, with the inputs copied from pinned host memory and
-    every output copied back to pinned host memory inside the timed region."""
+    """Same step through the public API, with every step's inputs copied from pinned host
+    memory and every output copied back to pinned host memory inside the timed region.
+    Steps are pipelined the way a training loop overlaps I/O: step i+1's host-to-device
+    copies, step i's kernels and step i-1's device-to-host copies run on three streams,
+    with double-buffered device tensors and events ordering each buffer's reuse."""
     pin = lambda x: None if x is None else x.contiguous().pin_memory()
     host_in = dict(q=pin(case.q), k=pin(case.k), v=pin(case.v), g_raw=pin(case.a), A_log=pin(case.A_log),
                    dt_bias=pin(case.dt_bias), beta=pin(case.beta), cu_seqlens=pin(case.cu_seqlens),
                    initial_state=pin(case.h0), d_o=pin(case.dO), dht=pin(case.dht))
-    dev_in = {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in host_in.items()}
-    o = torch.empty_like(dev_in["v"])
-    ht = torch.empty((case.N, case.HV, case.K, case.V), dtype=torch.float32, device=dev)
-    outs = dict(dq=torch.empty_like(dev_in["q"]), dk=torch.empty_like(dev_in["k"]),
-                dv=torch.empty_like(dev_in["v"]), dg=torch.empty_like(dev_in["g_raw"]),
-                dbeta=torch.empty_like(dev_in["beta"]), dh0=torch.empty_like(ht))
-    host_out = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in
-                dict(o=o, ht=ht, **outs).items()}
+    NB = 2
+    dev_in = [{k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in host_in.items()}
+              for _ in range(NB)]
+
+    def outs_like(di):
+        ht = torch.empty((case.N, case.HV, case.K, case.V), dtype=torch.float32, device=dev)
+        return dict(o=torch.empty_like(di["v"]), ht=ht, dq=torch.empty_like(di["q"]),
+                    dk=torch.empty_like(di["k"]), dv=torch.empty_like(di["v"]),
+                    dg=torch.empty_like(di["g_raw"]), dbeta=torch.empty_like(di["beta"]),
+                    dh0=torch.empty_like(ht))
+
+    dev_out = [outs_like(dev_in[b]) for b in range(NB)]
+    host_out = [{k: torch.empty_like(v, device="cpu").pin_memory() for k, v in dev_out[0].items()}
+                for _ in range(NB)]
     h2d = sum(v.numel() * v.element_size() for v in host_in.values() if v is not None)
-    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
-    stream = torch.cuda.current_stream()
+    d2h = sum(v.numel() * v.element_size() for v in host_out[0].values())
+    s_in, s_run, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    loaded = [ev() for _ in range(NB)]      # inputs of buffer b on the device
+    consumed = [ev() for _ in range(NB)]    # kernels done with buffer b's inputs and outputs written
+    drained = [ev() for _ in range(NB)]     # outputs of buffer b copied back
+    for b in range(NB):  # nothing to wait for before the first use of each buffer
+        for e_ in (consumed[b], drained[b]):
+            e_.record(s_out)
 
-    def one():
-        for k, v in host_in.items():
-            if v is not None:
-                dev_in[k].copy_(v, non_blocking=True)
-        fw = {k: dev_in[k] for k in ("q", "k", "v", "g_raw", "A_log", "dt_bias", "beta",
+    def upload(b):
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(consumed[b])
+            for k, v in host_in.items():
+                if v is not None:
+                    dev_in[b][k].copy_(v, non_blocking=True)
+            loaded[b].record(s_in)
+
+    def run(b):
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(loaded[b])
+            s_run.wait_event(drained[b])
+            di, do = dev_in[b], dev_out[b]
+            fw = {k: di[k] for k in ("q", "k", "v", "g_raw", "A_log", "dt_bias", "beta",
                                      "cu_seqlens", "initial_state")}
-        gdn.gdn_chunk_fwd(**fw, workspace=ws, out=o, final_state=ht)
-        gdn.gdn_chunk_bwd(**fw, d_o=dev_in["d_o"], dht=dev_in["dht"], workspace=ws, outs=outs,
-                          want_param_grads=False, reuse_forward=True)
-        for k, v in dict(o=o, ht=ht, **outs).items():
-            host_out[k].copy_(v, non_blocking=True)
+            gdn.gdn_chunk_fwd(**fw, workspace=ws, out=do["o"], final_state=do["ht"])
+            gdn.gdn_chunk_bwd(**fw, d_o=di["d_o"], dht=di["dht"], workspace=ws,
+                              outs={k: do[k] for k in ("dq", "dk", "dv", "dg", "dbeta", "dh0")},
+                              want_param_grads=False, reuse_forward=True)
+            consumed[b].record(s_run)
 
-    one()
+    def download(b):
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(consumed[b])
+            for k, v in dev_out[b].items():
+                host_out[b][k].copy_(v, non_blocking=True)
+            drained[b].record(s_out)
+
+    def pipeline(n, t0=None):
+        upload(0)
+        for i in range(n):
+            b = i % NB
+            if i + 1 < n:
+                upload((i + 1) % NB)
+            run(b)
+            download(b)
+
+    pipeline(2)  # warm-up
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(nsteps):
-        one()
-    b.record(stream)
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s_in)
+    pipeline(nsteps)
+    s_in.wait_stream(s_out)
+    z.record(s_in)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / nsteps
+    ms = a.elapsed_time(z) / nsteps
     (ms,) = max_over_ranks([ms], dist, dev)
     world = dist.get_world_size() if dist else 1
     return {"value": round(aggregate_mtok_s(world, case.tokens, ms), 3), "unit": "M tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "ms_per_step": round(ms, 3)}
+            "ms_per_step": round(ms, 3), "steps": nsteps,
+            "pipelined": "copies of step i+1 in, step i's kernels, step i-1 out on three streams"}
 
 
 DECODE = dict(B=256, H=16, HV=32, K=128, V=128)
