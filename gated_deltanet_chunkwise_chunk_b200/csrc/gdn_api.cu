@@ -33,6 +33,8 @@ int check_dims(const gdn_dims* d, bool varlen) {
   if (d->dtype != GDN_DTYPE_FP32 && d->dtype != GDN_DTYPE_BF16) return GDN_ERR_UNSUPPORTED;
   if (d->B * d->T >= (int64_t)1 << 31 || d->HV > 65535) return GDN_ERR_INVALID_ARG;
   if (max_chunks(*d, varlen) >= (int64_t)1 << 30) return GDN_ERR_INVALID_ARG;
+  // per-(chunk, value head) tiles are addressed by 32-bit TMA row coordinates (unit x 128)
+  if (max_chunks(*d, varlen) * d->HV * 128 >= (int64_t)1 << 31) return GDN_ERR_INVALID_ARG;
   if (!(d->scale >= 0.f) || std::isinf(d->scale)) return GDN_ERR_INVALID_ARG;
   return GDN_OK;
 }

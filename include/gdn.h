@@ -85,7 +85,10 @@ typedef enum gdn_flags {
   GDN_FLAG_BWD_REUSE_FWD = 1
 } gdn_flags;
 
-/* Bytes of workspace needed by gdn_chunk_fwd (pass = 0) or gdn_chunk_bwd (pass = 1) for
+/* Size limits (GDN_ERR_INVALID_ARG beyond them): B*T < 2^31 tokens, HV <= 65535, and
+ * chunks x HV x 128 < 2^31 (the per-chunk tiles are addressed by 32-bit tensor-map rows).
+ *
+ * Bytes of workspace needed by gdn_chunk_fwd (pass = 0) or gdn_chunk_bwd (pass = 1) for
  * these dimensions, or 0 if the dimensions are invalid.  With cu_seqlens the bound uses
  * at most (T + 63 N) / 64 chunks.  `varlen` is 1 when cu_seqlens will be passed. */
 size_t gdn_workspace_bytes(const gdn_dims* d, int varlen, int pass);

@@ -50,6 +50,15 @@ def test_workspace_bytes_rejects_bad_dims():
     assert gdn.workspace_bytes(_dims(dtype=7), False, False) == 0
 
 
+def test_size_limits():
+    """Tokens < 2^31 and chunks x HV x 128 < 2^31 (32-bit tensor-map rows); at the limits the
+    dimensions are rejected before any allocation or launch."""
+    assert gdn.workspace_bytes(_dims(T=1 << 20, H=16, HV=32), False, True) > 0
+    assert gdn.workspace_bytes(_dims(T=1 << 24, H=16, HV=32), False, True) > 0  # 2^18 chunks x 32 x 128 = 2^30
+    assert gdn.workspace_bytes(_dims(T=1 << 25, H=16, HV=32), False, True) == 0  # = 2^31
+    assert gdn.workspace_bytes(_dims(B=1 << 12, T=1 << 19, H=1, HV=1), False, False) == 0  # 2^31 tokens
+
+
 def test_entry_points_reject_bad_arguments_before_launch():
     d = _dims()
     lib = binding.lib

@@ -198,3 +198,12 @@ def test_run_to_run_bitwise_reproducible():
     a, b = run_gpu(case), run_gpu(case)
     for k in a:
         assert np.array_equal(a[k], b[k]), k
+
+
+def test_long_sequence_four_times_the_layer_length():
+    """T = 131072 (2048 chunks in one sequence, both scans 2048 steps long), one k-head with
+    two value heads, random initial state and final-state gradient: the longest chain the
+    suite runs, fwd and bwd against the oracle."""
+    case = synth.make_case(B=1, T=131072, H=1, HV=2, K=128, V=128, dtype="bf16", seed=77,
+                           h0=True, dht=True, name="long_T131072")
+    _assert_parity(case)
