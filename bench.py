@@ -337,7 +337,9 @@ def main():
 
     # end to end through the public API with host buffers
     e2e = e2e_measure(gdn, case, dev, ws, args.e2e_steps, dist)
-    decode = decode_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"]) if args.config == 2 and args.T is None else None
+    full = args.config == 2 and args.T is None
+    decode = decode_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"]) if full else None
+    kda = kda_gate_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"]) if full else None
 
     tokens = case.tokens
     value = aggregate_mtok_s(world, tokens, ms)
@@ -372,6 +374,7 @@ def main():
         "gpu_launches": int(launches),
         "e2e": e2e,
         "decode": decode,
+        "kda_gate": kda,
         "clocks": clocks,
         "peaks_source": pk["source"],
     }
@@ -580,6 +583,45 @@ def decode_measure(gdn, dev, pk_hbm: float, steps: int = 20) -> dict:
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk_hbm, "unit": "GB/s",
                          "frac": round(gbs / pk_hbm, 4), "bytes_per_step": int(nbytes),
                          "note": "fp32 state read and written once per (sequence, value head)"}}
+
+
+def kda_gate_measure(gdn, dev, pk_hbm: float, steps: int = 20) -> dict:
+    """The KDA gate at the layer's token count and heads (T = 32768, H = 16, D = 128, dt_bias
+    on): forward bf16 g -> fp32 yg, and backward (bf16 g, fp32 dyg -> bf16 dg and the two
+    parameter sums).  Both are element-wise and HBM-bound; each input (>= 134 MB) exceeds L2."""
+    T, H, D = 32768, 16, 128
+    gen = torch.Generator().manual_seed(77)
+    g = torch.randn(T, H, D, generator=gen).to(torch.bfloat16).to(dev)
+    A_log = torch.randn(H, generator=gen).to(dev)
+    dt_bias = torch.randn(H * D, generator=gen).to(dev)
+    dyg = torch.randn(T, H, D, generator=gen).to(dev)
+    yg = torch.empty(T, H, D, dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.kda_gate_workspace_bytes(T, H, D), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    ms_f = timed(lambda: gdn.kda_gate_fwd(g, A_log, dt_bias, output_dtype=torch.float32, out=yg))
+    ms_b = timed(lambda: gdn.kda_gate_bwd(g, A_log, dyg, dt_bias, workspace=ws))
+    n = T * H * D
+    part = 128 * 2 * H * D * 4 * 2  # row-block partials, written then read
+    bytes_f, bytes_b = n * (2 + 4), n * (2 + 4 + 2) + part
+    roof = lambda nb, ms: {"bound": "hbm", "achieved": round(nb / (ms / 1e3) / 1e9, 1), "peak": pk_hbm,
+                           "unit": "GB/s", "frac": round(nb / (ms / 1e3) / 1e9 / pk_hbm, 4),
+                           "bytes_per_call": int(nb)}
+    return {"workload": f"kda_gate_T{T}_H{H}_D{D}_bf16in", "fwd_ms": round(ms_f, 4),
+            "bwd_ms": round(ms_b, 4), "fwd_roofline": roof(bytes_f, ms_f),
+            "bwd_roofline": roof(bytes_b, ms_b)}
 
 
 # ----------------------------------------------------------------- reference arm (oracle)

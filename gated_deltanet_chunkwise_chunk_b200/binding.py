@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(6)
-GDN_DTYPE_FP32, GDN_DTYPE_BF16 = 0, 1
+GDN_DTYPE_FP32, GDN_DTYPE_BF16, GDN_DTYPE_FP16 = 0, 1, 2
 GDN_FLAG_BWD_REUSE_FWD = 1
 
 # Every symbol include/gdn.h declares (checked by the tests).
@@ -25,7 +25,8 @@ EXPORTED = ("gdn_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_max_ch
             "gdn_build_chunk_indices", "gdn_chunk_table_device", "gdn_device_status",
             "gdn_status_string", "gdn_version", "gdn_launch_count", "gdn_profile",
             "gdn_profile_read", "gdn_chunk_fwd_noalloc", "gdn_noalloc_scratch_bytes",
-            "gdn_recurrent_fwd", "gdn_recurrent_workspace_bytes")
+            "gdn_recurrent_fwd", "gdn_recurrent_workspace_bytes", "gdn_kda_gate_fwd",
+            "gdn_kda_gate_bwd", "gdn_kda_gate_workspace_bytes")
 
 
 class gdn_dims(ctypes.Structure):
@@ -58,6 +59,12 @@ def _load() -> ctypes.CDLL:
     lib.gdn_recurrent_fwd.restype = I32
     lib.gdn_recurrent_workspace_bytes.argtypes = []
     lib.gdn_recurrent_workspace_bytes.restype = SZ
+    lib.gdn_kda_gate_fwd.argtypes = [I64, I64, I64, I32, P, P, P, I32, P, P]
+    lib.gdn_kda_gate_fwd.restype = I32
+    lib.gdn_kda_gate_bwd.argtypes = [I64, I64, I64, I32, P, P, P, I32, P, P, P, P, P, SZ, P]
+    lib.gdn_kda_gate_bwd.restype = I32
+    lib.gdn_kda_gate_workspace_bytes.argtypes = [I64, I64, I64]
+    lib.gdn_kda_gate_workspace_bytes.restype = SZ
     lib.gdn_max_chunks.argtypes = [D, I32]
     lib.gdn_max_chunks.restype = I64
     lib.gdn_build_chunk_indices.argtypes = [D, P, P, I64]
@@ -211,6 +218,57 @@ def gdn_recurrent_fwd(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None, ini
     if rc != GDN_OK:
         raise GDNError("gdn_recurrent_fwd", rc)
     return o, ht
+
+
+_TORCH_DT = {torch.float32: GDN_DTYPE_FP32, torch.bfloat16: GDN_DTYPE_BF16,
+             torch.float16: GDN_DTYPE_FP16}
+
+
+def _kda_shape(g, A_log, dt_bias):
+    if g.dim() < 2:
+        raise ValueError("g needs at least [H, D] trailing dims")
+    H, D = g.shape[-2], g.shape[-1]
+    T = g.numel() // (H * D) if H * D else 0
+    _check("g", g, g.dtype, tuple(g.shape), g.device)
+    _check("A_log", A_log, torch.float32, (H,), g.device)
+    if dt_bias is not None:
+        _check("dt_bias", dt_bias, torch.float32, (H * D,), g.device)
+    if g.dtype not in _TORCH_DT:
+        raise ValueError(f"g dtype {g.dtype} is not fp32, bf16 or fp16")
+    return T, H, D
+
+
+def kda_gate_fwd(g, A_log, dt_bias=None, output_dtype=torch.float32, out=None):
+    """KDA gate: yg = -exp(A_log[h]) * softplus(g + dt_bias[h*D+d]) for g [..., H, D]."""
+    T, H, D = _kda_shape(g, A_log, dt_bias)
+    yg = out if out is not None else torch.empty(g.shape, dtype=output_dtype, device=g.device)
+    _check("out", yg, output_dtype, tuple(g.shape), g.device)
+    rc = lib.gdn_kda_gate_fwd(T, H, D, _TORCH_DT[g.dtype], _ptr(g), _ptr(A_log), _ptr(dt_bias),
+                              _TORCH_DT[output_dtype], _ptr(yg), _stream())
+    if rc != GDN_OK:
+        raise GDNError("gdn_kda_gate_fwd", rc)
+    return yg
+
+
+def kda_gate_bwd(g, A_log, dyg, dt_bias=None, workspace=None):
+    """Backward of kda_gate_fwd: returns (dg, dA_log, ddt_bias or None)."""
+    T, H, D = _kda_shape(g, A_log, dt_bias)
+    _check("dyg", dyg, dyg.dtype, tuple(g.shape), g.device)
+    need = int(lib.gdn_kda_gate_workspace_bytes(T, H, D))
+    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=g.device)
+    dg = torch.empty_like(g)
+    dA = torch.empty(H, dtype=torch.float32, device=g.device)
+    ddt = torch.empty(H * D, dtype=torch.float32, device=g.device) if dt_bias is not None else None
+    rc = lib.gdn_kda_gate_bwd(T, H, D, _TORCH_DT[g.dtype], _ptr(g), _ptr(A_log), _ptr(dt_bias),
+                              _TORCH_DT[dyg.dtype], _ptr(dyg), _ptr(dg), _ptr(dA), _ptr(ddt),
+                              _ptr(ws), ws.numel(), _stream())
+    if rc != GDN_OK:
+        raise GDNError("gdn_kda_gate_bwd", rc)
+    return dg, dA, ddt
+
+
+def kda_gate_workspace_bytes(T: int, H: int, D: int) -> int:
+    return int(lib.gdn_kda_gate_workspace_bytes(T, H, D))
 
 
 def recurrent_workspace_bytes() -> int:

@@ -355,6 +355,52 @@ int gdn_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const voi
   return cuda_status(e);
 }
 
+static int kda_check(int64_t T, int64_t H, int64_t D, int32_t dt1, int32_t dt2) {
+  if (T < 0 || H <= 0 || D <= 0 || H > 65535) return GDN_ERR_INVALID_ARG;
+  if (H * D > ((int64_t)1 << 24) || T > ((int64_t)1 << 62) / (H * D)) return GDN_ERR_INVALID_ARG;
+  auto ok_dt = [](int32_t t) {
+    return t == GDN_DTYPE_FP32 || t == GDN_DTYPE_BF16 || t == GDN_DTYPE_FP16;
+  };
+  return ok_dt(dt1) && ok_dt(dt2) ? GDN_OK : GDN_ERR_UNSUPPORTED;
+}
+
+size_t gdn_kda_gate_workspace_bytes(int64_t T, int64_t H, int64_t D) {
+  if (kda_check(T, H, D, GDN_DTYPE_FP32, GDN_DTYPE_FP32) != GDN_OK) return 0;
+  return kda_gate_workspace_bytes(H, D);
+}
+
+int gdn_kda_gate_fwd(int64_t T, int64_t H, int64_t D, int32_t in_dtype, const void* g,
+                     const float* A_log, const float* dt_bias, int32_t out_dtype, void* yg,
+                     void* stream) {
+  int rc = kda_check(T, H, D, in_dtype, out_dtype);
+  if (rc) return rc;
+  const bool empty = T == 0;
+  if ((!g && !empty) || (!yg && !empty) || !A_log) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(g) || !aligned16(yg) || !aligned16(A_log) || !aligned16(dt_bias))
+    return GDN_ERR_INVALID_ARG;
+  return cuda_status(kda_gate_forward(T, (int)H, (int)D, in_dtype, g, A_log, dt_bias, out_dtype, yg,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+int gdn_kda_gate_bwd(int64_t T, int64_t H, int64_t D, int32_t in_dtype, const void* g,
+                     const float* A_log, const float* dt_bias, int32_t dy_dtype, const void* dyg,
+                     void* dg, float* dA_log, float* ddt_bias, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  int rc = kda_check(T, H, D, in_dtype, dy_dtype);
+  if (rc) return rc;
+  const bool empty = T == 0;
+  if ((!g && !empty) || (!dyg && !empty) || (!dg && !empty) || !A_log) return GDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {g, A_log, dt_bias, dyg, dg, dA_log, ddt_bias};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return GDN_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) ||
+      workspace_bytes < kda_gate_workspace_bytes(H, D))
+    return GDN_ERR_WORKSPACE;
+  return cuda_status(kda_gate_backward(T, (int)H, (int)D, in_dtype, g, A_log, dt_bias, dy_dtype, dyg, dg,
+                                       dA_log, ddt_bias, static_cast<float*>(workspace),
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 int gdn_device_status(const void* workspace, void* stream) {
   if (!workspace) return GDN_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

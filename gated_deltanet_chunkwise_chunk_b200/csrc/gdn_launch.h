@@ -30,6 +30,13 @@ cudaError_t launch_bwd_tokens(const Problem& p, const Args& a, const Work& w, bo
                               cudaStream_t s);
 
 // fp32 CUDA-core path (FFMA tiles): used for fp32 tensors.
+// KDA gate (per-channel gate) forward and backward; dtypes are gdn_dtype codes.
+size_t kda_gate_workspace_bytes(int64_t H, int64_t D);
+cudaError_t kda_gate_forward(int64_t T, int H, int D, int in_dtype, const void* g, const float* A_log,
+                             const float* dt_bias, int out_dtype, void* yg, cudaStream_t s);
+cudaError_t kda_gate_backward(int64_t T, int H, int D, int in_dtype, const void* g, const float* A_log,
+                              const float* dt_bias, int dy_dtype, const void* dyg, void* dg,
+                              float* dA_log, float* ddt_bias, float* part, cudaStream_t s);
 // Token-by-token forward (decoding, short prefills); status: device status word.
 cudaError_t recurrent_forward(const Problem& p, const Args& a, int* status, bool bf16, cudaStream_t s);
 cudaError_t ffma_forward(const Problem& p, const Args& a, const Work& w, bool bf16, bool bwd_prep,

@@ -63,7 +63,11 @@ typedef enum gdn_status {
   GDN_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up (reported by gdn_device_status) */
 } gdn_status;
 
-typedef enum gdn_dtype { GDN_DTYPE_FP32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype;
+typedef enum gdn_dtype {
+  GDN_DTYPE_FP32 = 0,
+  GDN_DTYPE_BF16 = 1,
+  GDN_DTYPE_FP16 = 2  /* the KDA gate entry points only */
+} gdn_dtype;
 
 typedef struct gdn_dims {
   int64_t B, T, H, HV, K, V;
@@ -154,6 +158,33 @@ int gdn_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const voi
 
 /* GDN_RECURRENT_WORKSPACE_BYTES. */
 size_t gdn_recurrent_workspace_bytes(void);
+
+/* KDA gate: the per-channel gate of Kimi-style delta attention ("KDA gate" task of the
+ * MindSpeed-Ops issue tracker, sections on the formula, the computation flow and the API):
+ *   yg[t,h,d] = -exp(A_log[h]) * softplus(g[t,h,d] + dt_bias[h*D + d]),
+ *   softplus(x) = x if x > 20 else log(1 + e^x), computed in fp32.
+ * g, yg: [T, H, D] row-major (any leading dims flattened into T) in in_dtype / out_dtype
+ * (gdn_dtype: fp32, bf16 or fp16); A_log [H] fp32; dt_bias [H*D] fp32 or NULL (no bias).
+ * All buffers on the device, 16-byte aligned; launches on `stream`; allocates nothing.
+ * Returns GDN_ERR_INVALID_ARG for null or misaligned pointers or bad sizes (H <= 65535,
+ * H*D <= 2^24), GDN_ERR_UNSUPPORTED for an unknown dtype.  The chunkwise KDA attention itself
+ * is not provided. */
+int gdn_kda_gate_fwd(int64_t T, int64_t H, int64_t D, int32_t in_dtype, const void* g,
+                     const float* A_log, const float* dt_bias, int32_t out_dtype, void* yg,
+                     void* stream);
+
+/* Backward of the KDA gate for dyg = dL/dyg ([T,H,D] in dy_dtype):
+ *   dg = dyg * (-exp(A_log[h])) * (x > 20 ? 1 : sigmoid(x))    ([T,H,D] in in_dtype),
+ *   dA_log[h] = sum_{t,d} dyg * yg,   ddt_bias[h*D+d] = sum_t dg   (fp32; either may be NULL).
+ * The two sums are deterministic (fixed-order two-pass reduction).  workspace: at least
+ * gdn_kda_gate_workspace_bytes(T, H, D) bytes, 256-byte aligned. */
+int gdn_kda_gate_bwd(int64_t T, int64_t H, int64_t D, int32_t in_dtype, const void* g,
+                     const float* A_log, const float* dt_bias, int32_t dy_dtype, const void* dyg,
+                     void* dg, float* dA_log, float* ddt_bias, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of gdn_kda_gate_bwd (0 for invalid sizes). */
+size_t gdn_kda_gate_workspace_bytes(int64_t T, int64_t H, int64_t D);
 
 /* Upper bound on the number of 64-token chunks (the grid size used for chunk kernels). */
 int64_t gdn_max_chunks(const gdn_dims* d, int varlen);
