@@ -106,4 +106,13 @@ __device__ __forceinline__ bool call_failed(const Work& w) {
   return *((volatile int*)w.status) != 0;
 }
 
+// Streaming multiprocessors of the current device (grid sizes of persistent and streaming kernels).
+inline int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
 }  // namespace gdn

@@ -317,15 +317,6 @@ __device__ __forceinline__ float quad_sum(float x) {
 __device__ __forceinline__ bool failed(const Work& w) { return *((volatile int*)w.status) != 0; }
 
 
-// Streaming multiprocessors of the current device (grid size of the persistent kernels).
-inline int num_sms() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-    return 148;
-  return n;
-}
-
 // Launch helper: raises the dynamic shared-memory limit, counts/brackets the launch.
 template <typename Kern, typename... A>
 cudaError_t tgo(const char* name, Kern kern, dim3 grid, int threads, size_t smem, cudaStream_t s,

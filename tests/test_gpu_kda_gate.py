@@ -1,14 +1,18 @@
 """GPU parity of the KDA gate (gdn_kda_gate_fwd / gdn_kda_gate_bwd) against the fp64 oracle,
-on the shapes and dtypes of the pages' own test list (T, H, D) x {fp32, fp16, bf16} x {bias,
-no bias}, plus the x > 20 branch.  The kernel computes in fp32 and rounds once to the output
-dtype.  Error bound per element, derived from that arithmetic: x = g + dt_bias is rounded
-once in fp32 (|dx| <= 2^-24 |x|), and softplus and sigmoid both have a relative sensitivity
-|d log f / dx| <= 1, so x's rounding costs at most 2^-24 |x| relative; expf, log1pf, the
-reciprocal and the products add a few fp32 ulps (8 allowed); the output rounding adds 2^-p
-(p = 24, 11, 8 for fp32, fp16, bf16; half an ulp is at most 2^-p relative), plus half the
-subnormal spacing for fp16.  The two parameter-gradient sums are fp32 accumulations along
-fixed chains of length L (rows per block, then blocks, then the tree), so their bound is
-(L + per-term bound) * 2^-24 times the sum of the absolute terms."""
+on the shapes of the pages' test list (T, H, D), their block-edge sequence lengths, fp32 / fp16
+/ bf16 in and out, with and without dt_bias, the x > 20 branch, and a D that is not a multiple
+of 8 (the scalar path).
+
+The pages accept |out - ref| <= 1e-3 + 1e-3 |ref| against an fp32 reference; the bounds here
+are far tighter, derived from the kernel's fp32 arithmetic, in units u = 2^-24 relative:
+x = g + dt_bias rounds once (|x| u; softplus and sigmoid have |d log f / dx| <= 1); the fast
+exponential e = exp(-|x|) has the documented error 2 + 1.173|x| ulp (<= (4 + 2.35|x|) u); the two
+approximate divisions 2 ulp each; the artanh series for log1p, expf(A_log) and the products a
+few u more.  Hence (4|x| + 24) u on top of the output rounding 2^-p (p = 24, 11, 8 for fp32,
+fp16, bf16), plus half the subnormal spacing of fp16 and a 1e-35 floor for the flushed range.
+The two parameter-gradient sums are fp32 accumulations along fixed chains of length L (rows
+per block lane, up to 256 lanes, 8 strands of blocks, 8 in a strand's tail, the tree), so their bound is
+(L + per-term bound) u times the sum of the absolute terms."""
 from __future__ import annotations
 
 import numpy as np
@@ -31,7 +35,7 @@ def _inputs(T, H, D, dtype, with_bias, seed):
     return g, A_log, dt_bias
 
 
-SUBNORMAL_HALF = {torch.float32: 2.0 ** -150, torch.float16: 2.0 ** -25, torch.bfloat16: 2.0 ** -134}
+FLOOR = {torch.float32: 1e-35, torch.float16: 2.0 ** -25, torch.bfloat16: 1e-35}
 
 
 def _x(g, dt_bias):
@@ -43,7 +47,7 @@ def _x(g, dt_bias):
 def _close(got, ref, x, dtype):
     got = got.double().cpu().numpy()
     err = np.abs(got - ref)
-    bound = (ULP[dtype] + (np.abs(x) + 8.0) * 2.0 ** -24) * np.abs(ref) + SUBNORMAL_HALF[dtype]
+    bound = (ULP[dtype] + (4.0 * np.abs(x) + 24.0) * 2.0 ** -24) * np.abs(ref) + FLOOR[dtype]
     assert (err <= bound).all(), f"max excess {float((err - bound).max()):.3e}"
 
 
@@ -77,9 +81,9 @@ def test_backward(T, H, D, dtype, with_bias):
     rdg, rdA, rddt = okda.bwd(g, A_log, dyg, dt_bias)
     x = _x(g, dt_bias)
     _close(dg, rdg, x, dtype)
-    # the sums: chains of T/128 rows, 128 blocks, then D/256 + 8 tree levels
-    L = -(-T // 128) + 128 + -(-D // 256) + 8
-    per = L + float(np.abs(x).max()) + 8.0
+    # the sums: a block lane's rows, the lanes, 8 strands of blocks, the strand sum, the tree
+    L = T + 256 + 296 + 8 + -(-D // 256) + 8
+    per = L + 4.0 * float(np.abs(x).max()) + 24.0
     yg = okda.fwd(g, A_log, dt_bias)
     scaleA = np.abs(dyg.double().numpy() * yg).sum(axis=(0, 2))
     assert (np.abs(dA.double().cpu().numpy() - rdA) <= per * 2.0 ** -24 * scaleA).all()
@@ -88,6 +92,56 @@ def test_backward(T, H, D, dtype, with_bias):
         assert (np.abs(ddt.double().cpu().numpy() - rddt) <= per * 2.0 ** -24 * scaleB).all()
     else:
         assert ddt is None
+
+
+EDGE_T = [1, 16, 31, 32, 33, 63, 64, 65, 127, 128, 129, 512, 1024, 2048, 4096]
+EDGE_HD = [(4, 64), (8, 96), (12, 128), (16, 256), (32, 64)]
+
+
+@pytest.mark.parametrize("T", EDGE_T)
+def test_block_edges_forward_and_backward(T):
+    """The pages' sequence lengths around block boundaries, each with one (H, D) of theirs."""
+    import gated_deltanet_chunkwise_chunk_b200 as gdn
+    H, D = EDGE_HD[EDGE_T.index(T) % len(EDGE_HD)]
+    for dtype in (torch.float32, torch.float16, torch.bfloat16):
+        for with_bias in (True, False):
+            g, A_log, dt_bias = _inputs(T, H, D, dtype, with_bias, seed=T + 1000 * D)
+            dev = lambda x: None if x is None else x.cuda()
+            x = _x(g, dt_bias)
+            yg = gdn.kda_gate_fwd(dev(g), dev(A_log), dev(dt_bias), output_dtype=dtype)
+            torch.cuda.synchronize()
+            _close(yg, okda.fwd(g, A_log, dt_bias), x, dtype)
+    g, A_log, dt_bias = _inputs(T, H, D, torch.bfloat16, True, seed=T + 7)
+    dyg = torch.randn(T, H, D, generator=torch.Generator().manual_seed(T)).to(torch.bfloat16)
+    dg, dA, ddt = gdn.kda_gate_bwd(g.cuda(), A_log.cuda(), dyg.cuda(), dt_bias.cuda())
+    torch.cuda.synchronize()
+    rdg, rdA, rddt = okda.bwd(g, A_log, dyg, dt_bias)
+    x = _x(g, dt_bias)
+    _close(dg, rdg, x, torch.bfloat16)
+    per = (T + 256 + 296 + 8 + 1 + 8) + 4.0 * float(np.abs(x).max()) + 24.0
+    scaleA = np.abs(dyg.double().numpy() * okda.fwd(g, A_log, dt_bias)).sum(axis=(0, 2))
+    assert (np.abs(dA.double().cpu().numpy() - rdA) <= per * 2.0 ** -24 * scaleA).all()
+    scaleB = np.abs(rdg).sum(axis=0).reshape(-1)
+    assert (np.abs(ddt.double().cpu().numpy() - rddt) <= per * 2.0 ** -24 * scaleB).all()
+
+
+@pytest.mark.parametrize("T,H,D", [(33, 3, 20), (129, 5, 3), (1, 1, 1), (300, 2, 12)])
+def test_head_dim_not_a_multiple_of_8(T, H, D):
+    import gated_deltanet_chunkwise_chunk_b200 as gdn
+    g, A_log, dt_bias = _inputs(T, H, D, torch.float16, True, seed=D)
+    dyg = torch.randn(T, H, D, generator=torch.Generator().manual_seed(1))
+    yg = gdn.kda_gate_fwd(g.cuda(), A_log.cuda(), dt_bias.cuda(), output_dtype=torch.float32)
+    dg, dA, ddt = gdn.kda_gate_bwd(g.cuda(), A_log.cuda(), dyg.cuda(), dt_bias.cuda())
+    torch.cuda.synchronize()
+    x = _x(g, dt_bias)
+    _close(yg, okda.fwd(g, A_log, dt_bias), x, torch.float32)
+    rdg, rdA, rddt = okda.bwd(g, A_log, dyg, dt_bias)
+    _close(dg, rdg, x, torch.float16)
+    per = (T + 256 + 296 + 8 + 1 + 8) + 4.0 * float(np.abs(x).max()) + 24.0
+    scaleA = np.abs(dyg.double().numpy() * okda.fwd(g, A_log, dt_bias)).sum(axis=(0, 2))
+    assert (np.abs(dA.double().cpu().numpy() - rdA) <= per * 2.0 ** -24 * scaleA).all()
+    scaleB = np.abs(rdg).sum(axis=0).reshape(-1)
+    assert (np.abs(ddt.double().cpu().numpy() - rddt) <= per * 2.0 ** -24 * scaleB).all()
 
 
 def test_backward_is_deterministic_and_empty_input_is_a_no_op():
