@@ -1,0 +1,110 @@
+"""CPU pins of the KDA recurrent oracle (oracle/kda.py), each against something other than the
+oracle's own loop: the Gated DeltaNet C++ oracle when every channel shares one gate (an
+independent implementation of that special case), the closed form of a pure per-channel
+decay (beta = 0), the exact-write invariant of the delta rule with per-channel gates, a
+brute-force product of the dense transition matrices, and varlen packing."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+from oracle import kda, oracle
+
+
+def _case(rng, B=1, T=23, H=2, HV=4, K=8, V=6, h0=True, gate_scale=2.0):
+    q = rng.standard_normal((B, T, H, K))
+    k = rng.standard_normal((B, T, H, K))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    q /= np.linalg.norm(q, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, T, HV, V))
+    g = rng.standard_normal((B, T, HV, K)) * gate_scale
+    A_log = np.log(rng.uniform(0.05, 1.0, HV))
+    dt_bias = rng.standard_normal(HV * K) * 0.5
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((B, T, HV))))
+    S0 = rng.standard_normal((B, HV, K, V)) * 0.3 if h0 else None
+    return q, k, v, g, A_log, dt_bias, beta, S0
+
+
+def test_channel_constant_gate_is_gated_deltanet():
+    rng = np.random.default_rng(11)
+    q, k, v, g, A_log, dt_bias, beta, S0 = _case(rng, B=2, T=37)
+    a = rng.standard_normal(g.shape[:3]) * 3.0           # one raw gate per (b, t, hv)
+    g = np.repeat(a[..., None], g.shape[-1], axis=-1)
+    dtb = rng.standard_normal(g.shape[2])
+    dt_bias = np.repeat(dtb, g.shape[-1])
+    o, ht = kda.recurrent_fwd(q, k, v, g, A_log, dt_bias, beta, h0=S0)
+    ro, rht, _ = oracle.fwd(q, k, v, a, A_log, dtb, beta, h0=S0)
+    np.testing.assert_allclose(o, ro, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(ht, rht, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("K,V", [(8, 5), (6, 6)])
+def test_beta_zero_is_a_per_channel_decay(K, V):
+    """beta = 0: S_t = S_0 Diag(exp(cumsum yg)), so o_t = scale * S_0 (e^{Gamma_t} * q_t).
+    The square case catches a decay applied along the value axis instead of the key axis."""
+    rng = np.random.default_rng(12)
+    q, k, v, g, A_log, dt_bias, beta, S0 = _case(rng, K=K, V=V)
+    beta[:] = 0.0
+    o, ht = kda.recurrent_fwd(q, k, v, g, A_log, dt_bias, beta, scale=0.7, h0=S0)
+    x = g + dt_bias.reshape(g.shape[2], g.shape[3])
+    yg = -np.exp(A_log)[:, None] * np.where(x > 20, x, np.log1p(np.exp(np.minimum(x, 20))))
+    Gam = np.cumsum(yg, axis=1)                           # [B,T,HV,K]
+    H, HV = q.shape[2], v.shape[2]
+    for hv in range(HV):
+        qq = q[0, :, hv // (HV // H)]                      # [T,K]
+        ref = 0.7 * np.einsum("kv,tk->tv", S0[0, hv], np.exp(Gam[0, :, hv]) * qq)
+        np.testing.assert_allclose(o[0, :, hv], ref, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(ht[0, hv], S0[0, hv] * np.exp(Gam[0, -1, hv])[:, None],
+                                   rtol=1e-12, atol=1e-14)
+
+
+def test_exact_write_with_per_channel_gates():
+    """beta = 1 and unit keys: after the step, S_t k_t = v_t whatever the decay was."""
+    rng = np.random.default_rng(13)
+    q, k, v, g, A_log, dt_bias, beta, S0 = _case(rng, T=19)
+    beta[:] = 1.0
+    H, HV = q.shape[2], v.shape[2]
+    o, _ = kda.recurrent_fwd(k, k, v, g, A_log, dt_bias, beta, scale=1.0, h0=S0)
+    np.testing.assert_allclose(o, v, rtol=1e-10, atol=1e-11)
+
+
+def test_dense_transition_products():
+    """Brute force: the state after T tokens as S_0 P_1 ... P_T + sum_t beta_t v_t k_t^T P_{t+1}..P_T
+    with P_t = Diag(alpha_t)(I - beta_t k_t k_t^T) formed as dense K x K matrices."""
+    rng = np.random.default_rng(14)
+    q, k, v, g, A_log, dt_bias, beta, S0 = _case(rng, T=9, H=1, HV=1, K=5, V=3)
+    o, ht = kda.recurrent_fwd(q, k, v, g, A_log, dt_bias, beta, h0=S0)
+    x = g[0, :, 0] + dt_bias.reshape(1, -1)
+    alpha = np.exp(-np.exp(A_log[0]) * np.log1p(np.exp(x)))  # |x| < 20 here
+    K = 5
+    P = [np.diag(alpha[t]) @ (np.eye(K) - beta[0, t, 0] * np.outer(k[0, t, 0], k[0, t, 0]))
+         for t in range(9)]
+    S = S0[0, 0].T.copy()
+    for t in range(9):
+        S = S @ P[t] + beta[0, t, 0] * np.outer(v[0, t, 0], k[0, t, 0])
+        np.testing.assert_allclose(o[0, t, 0], K ** -0.5 * S @ q[0, t, 0], rtol=1e-12, atol=1e-13)
+    # and the closed sum for the final state
+    Ssum = S0[0, 0].T.copy()
+    for t in range(9):
+        Ssum = Ssum @ P[t]
+    for t in range(9):
+        M = np.outer(v[0, t, 0], k[0, t, 0]) * beta[0, t, 0]
+        for s in range(t + 1, 9):
+            M = M @ P[s]
+        Ssum += M
+    np.testing.assert_allclose(ht[0, 0].T, Ssum, rtol=1e-12, atol=1e-13)
+
+
+def test_varlen_equals_independent_sequences():
+    rng = np.random.default_rng(15)
+    lens = [5, 0, 11, 1]
+    T = sum(lens)
+    q, k, v, g, A_log, dt_bias, beta, _ = _case(rng, T=T)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    S0 = rng.standard_normal((len(lens), v.shape[2], q.shape[3], v.shape[3]))
+    o, ht = kda.recurrent_fwd(q, k, v, g, A_log, dt_bias, beta, cu_seqlens=cu, h0=S0)
+    for n, (a, b) in enumerate(zip(cu[:-1], cu[1:])):
+        sl = slice(a, b)
+        on, hn = kda.recurrent_fwd(q[:, sl], k[:, sl], v[:, sl], g[:, sl], A_log, dt_bias,
+                                   beta[:, sl], h0=S0[n:n + 1])
+        assert np.array_equal(o[:, sl], on) and np.array_equal(ht[n], hn[0])
