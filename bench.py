@@ -340,6 +340,7 @@ def main():
     full = args.config == 2 and args.T is None
     decode = decode_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"]) if full else None
     kda = kda_gate_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"]) if full else None
+    kda_decode = decode_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"], kda=True) if full else None
 
     tokens = case.tokens
     value = aggregate_mtok_s(world, tokens, ms)
@@ -375,6 +376,7 @@ def main():
         "e2e": e2e,
         "decode": decode,
         "kda_gate": kda,
+        "kda_decode": kda_decode,
         "clocks": clocks,
         "peaks_source": pk["source"],
     }
@@ -547,22 +549,27 @@ def e2e_measure(gdn, case, dev, ws, nsteps: int, dist) -> dict:
 DECODE = dict(B=256, H=16, HV=32, K=128, V=128)
 
 
-def decode_measure(gdn, dev, pk_hbm: float, steps: int = 20) -> dict:
+def decode_measure(gdn, dev, pk_hbm: float, steps: int = 20, kda: bool = False) -> dict:
     """One decode step (T = 1) of 256 sequences with the layer's heads, through
-    gdn_recurrent_fwd with the state updated in place: HBM-bound on the fp32 state, read and
-    written once per (sequence, value head).  A secondary measurement beside the training step."""
+    gdn_recurrent_fwd (or, with kda, gdn_kda_recurrent_fwd: a gate per key channel) with the
+    state updated in place: HBM-bound on the fp32 state, read and written once per (sequence,
+    value head).  A secondary measurement beside the training step."""
     c = DECODE
     case = synth.make_case(B=c["B"], T=1, H=c["H"], HV=c["HV"], K=c["K"], V=c["V"], dtype="bf16",
                            seed=4242, h0=True, name="decode")
     t = lambda x: None if x is None else x.to(dev).contiguous()
     d = dict(q=t(case.q), k=t(case.k), v=t(case.v), g_raw=t(case.a), A_log=t(case.A_log),
              dt_bias=t(case.dt_bias), beta=t(case.beta))
+    if kda:
+        g_raw, A_log, dt_bias = synth.kda_gate_inputs(case, 4243)
+        d.update(g_raw=t(g_raw), A_log=t(A_log), dt_bias=t(dt_bias))
     st = t(case.h0)
     o = torch.empty_like(d["v"])
     ws = torch.empty(gdn.recurrent_workspace_bytes(), dtype=torch.uint8, device=dev)
+    fn = gdn.gdn_kda_recurrent_fwd if kda else gdn.gdn_recurrent_fwd
 
     def step():
-        gdn.gdn_recurrent_fwd(**d, initial_state=st, final_state=st, out=o, workspace=ws)
+        fn(**d, initial_state=st, final_state=st, out=o, workspace=ws)
 
     for _ in range(3):
         step()
@@ -576,9 +583,11 @@ def decode_measure(gdn, dev, pk_hbm: float, steps: int = 20) -> dict:
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
     B, H, HV, K, V = c["B"], c["H"], c["HV"], c["K"], c["V"]
-    nbytes = B * HV * K * V * 4 * 2 + B * (2 * H * K + 2 * HV * V) * 2 + B * HV * 8 + HV * 8
+    gate = B * HV * K * 4 + HV * K * 4 + HV * 4 if kda else B * HV * 4 + HV * 8
+    nbytes = B * HV * K * V * 4 * 2 + B * (2 * H * K + 2 * HV * V) * 2 + B * HV * 4 + gate
     gbs = nbytes / (ms / 1e3) / 1e9
-    return {"workload": f"decode_B{B}_H{H}_HV{HV}_D{K}_bf16", "tokens_per_step": B,
+    name = "kda_decode" if kda else "decode"
+    return {"workload": f"{name}_B{B}_H{H}_HV{HV}_D{K}_bf16", "tokens_per_step": B,
             "ms_per_step": round(ms, 4), "mtok_s": round(B / (ms / 1e3) / 1e6, 3),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk_hbm, "unit": "GB/s",
                          "frac": round(gbs / pk_hbm, 4), "bytes_per_step": int(nbytes),

@@ -26,7 +26,7 @@ EXPORTED = ("gdn_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_max_ch
             "gdn_status_string", "gdn_version", "gdn_launch_count", "gdn_profile",
             "gdn_profile_read", "gdn_chunk_fwd_noalloc", "gdn_noalloc_scratch_bytes",
             "gdn_recurrent_fwd", "gdn_recurrent_workspace_bytes", "gdn_kda_gate_fwd",
-            "gdn_kda_gate_bwd", "gdn_kda_gate_workspace_bytes")
+            "gdn_kda_gate_bwd", "gdn_kda_gate_workspace_bytes", "gdn_kda_recurrent_fwd")
 
 
 class gdn_dims(ctypes.Structure):
@@ -57,6 +57,8 @@ def _load() -> ctypes.CDLL:
     lib.gdn_chunk_bwd.restype = I32
     lib.gdn_recurrent_fwd.argtypes = [D] + [P] * 12 + [SZ, P]
     lib.gdn_recurrent_fwd.restype = I32
+    lib.gdn_kda_recurrent_fwd.argtypes = [D] + [P] * 12 + [SZ, P]
+    lib.gdn_kda_recurrent_fwd.restype = I32
     lib.gdn_recurrent_workspace_bytes.argtypes = []
     lib.gdn_recurrent_workspace_bytes.restype = SZ
     lib.gdn_kda_gate_fwd.argtypes = [I64, I64, I64, I32, P, P, P, I32, P, P]
@@ -217,6 +219,33 @@ def gdn_recurrent_fwd(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None, ini
                                workspace.numel(), _stream())
     if rc != GDN_OK:
         raise GDNError("gdn_recurrent_fwd", rc)
+    return o, ht
+
+
+def gdn_kda_recurrent_fwd(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None,
+                          initial_state=None, scale=0.0, out=None, final_state=None, workspace=None):
+    """KDA (per-key-channel gate) token-by-token forward: returns (o, final_state).  As
+    gdn_recurrent_fwd with g_raw [B,T,HV,K] and dt_bias [HV*K] (or None)."""
+    B, T, H, K = q.shape
+    HV = v.shape[2]
+    Nst = _check_inputs(q, k, v, None, A_log, None, beta, cu_seqlens, initial_state)
+    _check("g_raw", g_raw, torch.float32, (B, T, HV, K), q.device)
+    _check("dt_bias", dt_bias, torch.float32, (HV * K,), q.device)
+    dims = make_dims(q, v, cu_seqlens, scale)
+    need = int(lib.gdn_recurrent_workspace_bytes())
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    elif workspace.numel() < need:
+        raise ValueError(f"workspace holds {workspace.numel()} bytes, the call needs {need}")
+    o = out if out is not None else torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    ht = final_state if final_state is not None else torch.empty(
+        (Nst, HV, K, v.shape[3]), dtype=torch.float32, device=q.device)
+    rc = lib.gdn_kda_recurrent_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g_raw),
+                                   _ptr(A_log), _ptr(dt_bias), _ptr(beta), _ptr(cu_seqlens),
+                                   _ptr(initial_state), _ptr(o), _ptr(ht), _ptr(workspace),
+                                   workspace.numel(), _stream())
+    if rc != GDN_OK:
+        raise GDNError("gdn_kda_recurrent_fwd", rc)
     return o, ht
 
 

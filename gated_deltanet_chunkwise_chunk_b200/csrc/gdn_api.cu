@@ -319,10 +319,11 @@ int gdn_chunk_table_device(const gdn_dims* d, const int64_t* cu_seqlens, int32_t
 
 size_t gdn_recurrent_workspace_bytes(void) { return GDN_RECURRENT_WORKSPACE_BYTES; }
 
-int gdn_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
-                      const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,
-                      const int64_t* cu_seqlens, const float* initial_state, void* o,
-                      float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
+static int recurrent_common(const gdn_dims* d, const void* q, const void* k, const void* v,
+                            const float* g_raw, const float* A_log, const float* dt_bias,
+                            const float* beta, const int64_t* cu_seqlens, const float* initial_state,
+                            void* o, float* final_state, void* workspace, size_t workspace_bytes,
+                            void* stream, bool kda) {
   const bool varlen = cu_seqlens != nullptr;
   int rc = check_dims(d, varlen);
   if (rc) return rc;
@@ -330,7 +331,7 @@ int gdn_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const voi
   const void* tok[] = {q, k, v, g_raw, beta, o};
   for (const void* x : tok)
     if ((!x && !empty) || !aligned16(x)) return GDN_ERR_INVALID_ARG;
-  if (!A_log || !dt_bias || !aligned16(A_log) || !aligned16(dt_bias)) return GDN_ERR_INVALID_ARG;
+  if (!A_log || (!dt_bias && !kda) || !aligned16(A_log) || !aligned16(dt_bias)) return GDN_ERR_INVALID_ARG;
   if (!aligned16(cu_seqlens) || !aligned16(initial_state) || !aligned16(final_state))
     return GDN_ERR_INVALID_ARG;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) ||
@@ -351,8 +352,26 @@ int gdn_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const voi
   a.ht = final_state;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, 64, s);  // the device status word
-  if (e == cudaSuccess) e = recurrent_forward(p, a, static_cast<int*>(workspace), d->dtype == GDN_DTYPE_BF16, s);
+  if (e == cudaSuccess)
+    e = recurrent_forward(p, a, static_cast<int*>(workspace), d->dtype == GDN_DTYPE_BF16, s, kda);
   return cuda_status(e);
+}
+
+int gdn_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                      const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,
+                      const int64_t* cu_seqlens, const float* initial_state, void* o,
+                      float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
+  return recurrent_common(d, q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens, initial_state, o,
+                          final_state, workspace, workspace_bytes, stream, false);
+}
+
+int gdn_kda_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                          const float* g_raw, const float* A_log, const float* dt_bias,
+                          const float* beta, const int64_t* cu_seqlens, const float* initial_state,
+                          void* o, float* final_state, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  return recurrent_common(d, q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens, initial_state, o,
+                          final_state, workspace, workspace_bytes, stream, true);
 }
 
 static int kda_check(int64_t T, int64_t H, int64_t D, int32_t dt1, int32_t dt2) {

@@ -6,6 +6,10 @@
 // (the decay applies before the erase, as in the chunkwise algebra).  HBM-bound at T = 1:
 // 2 x 4KV bytes of state per (sequence, value head) plus the token vectors.
 //
+// KDA variant (template flag KDA): the decay is per key channel c, S <- S Diag(e^{yg_t}) with
+// yg_t[c] = -exp(A_log) softplus(g_raw[t, hv, c] + dt_bias[hv*K + c]) (the KDA gate of the
+// MindSpeed-Ops "KDA gate" task, fused here); everything else is unchanged.
+//
 // CTA (sequence, value head, z) holds rows v0 = 32z .. v0+31 of S.  Thread (kg, vg) keeps
 // S[v0+4vg .. +3][kg*K/16 .. (kg+1)*K/16) in fp32 registers, so the state moves as 16-byte
 // rows of h[k][v]; the 16 k-groups of a column block sit in one warp (lane = kg + 16 (vg%2)),
@@ -18,12 +22,12 @@ namespace {
 
 constexpr int RV = 32;  // state rows per CTA
 
-template <typename T, int K>
+template <typename T, int K, bool KDA>
 __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* status) {
   constexpr int KQ = K / 16;  // state columns per thread
   const int n = blockIdx.x, hv = blockIdx.y, hk = hv / p.G, v0 = RV * blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, kg = lane & 15, vg = 2 * (tid >> 5) + (lane >> 4);
-  __shared__ float sk[K], sq[K], sv[RV], sdec, sbeta;
+  __shared__ float sk[K], sq[K], sv[RV], sdec, sbeta, sdk[KDA ? K : 1];
   int bos, eos;
   if (p.varlen) {
     bos = (int)a.cu[n];
@@ -49,7 +53,7 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
   const T* k = static_cast<const T*>(a.k);
   const T* v = static_cast<const T*>(a.v);
   T* o = static_cast<T*>(a.o);
-  const float nexp = -expf(a.A_log[hv]), dtb = a.dt_bias[hv];
+  const float nexp = -expf(a.A_log[hv]), dtb = KDA ? 0.f : a.dt_bias[hv];
   auto rowsum = [](float x) {  // over the 16 k-groups of this lane half
     x += __shfl_xor_sync(0xffffffffu, x, 1);
     x += __shfl_xor_sync(0xffffffffu, x, 2);
@@ -65,18 +69,28 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
       sq[i] = to_f<T>(q[qk0 + i]);
     }
     if (tid < RV) sv[tid] = to_f<T>(v[v_0 + tid]);
+    if constexpr (KDA) {  // per-channel decay of this token
+      const size_t g0 = ((size_t)t * p.HV + hv) * K;
+      for (int i = tid; i < K; i += 128) {
+        const float x = a.g_raw[g0 + i] + (a.dt_bias ? a.dt_bias[(size_t)hv * K + i] : 0.f);
+        sdk[i] = expf(nexp * (x > 20.f ? x : log1pf(expf(x))));
+      }
+    }
     if (tid == 0) {
       const size_t gi = (size_t)t * p.HV + hv;
-      const float x = a.g_raw[gi] + dtb;
-      sdec = expf(nexp * (x > 20.f ? x : log1pf(expf(x))));
+      if constexpr (!KDA) {
+        const float x = a.g_raw[gi] + dtb;
+        sdec = expf(nexp * (x > 20.f ? x : log1pf(expf(x))));
+      }
       sbeta = a.beta[gi];
     }
     __syncthreads();
-    const float dec = sdec, b = sbeta;
+    const float b = sbeta;
     float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < KQ; ++i) {
       const float kv = sk[kg * KQ + i];
+      const float dec = KDA ? sdk[kg * KQ + i] : sdec;
       S4[i].x *= dec; S4[i].y *= dec; S4[i].z *= dec; S4[i].w *= dec;
       e.x += S4[i].x * kv; e.y += S4[i].y * kv; e.z += S4[i].z * kv; e.w += S4[i].w * kv;
     }
@@ -107,22 +121,25 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
   }
 }
 
-template <typename T>
+template <typename T, bool KDA>
 cudaError_t launch_t(const Problem& p, const Args& a, int* status, cudaStream_t s) {
   const dim3 grid(p.Nst, p.HV, p.V / RV);
   if (p.K == 128)
-    k_recurrent_fwd<T, 128><<<grid, 128, 0, s>>>(p, a, status);
+    k_recurrent_fwd<T, 128, KDA><<<grid, 128, 0, s>>>(p, a, status);
   else
-    k_recurrent_fwd<T, 64><<<grid, 128, 0, s>>>(p, a, status);
+    k_recurrent_fwd<T, 64, KDA><<<grid, 128, 0, s>>>(p, a, status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t recurrent_forward(const Problem& p, const Args& a, int* status, bool bf16, cudaStream_t s) {
+cudaError_t recurrent_forward(const Problem& p, const Args& a, int* status, bool bf16, cudaStream_t s,
+                              bool kda) {
   if (p.Nst == 0) return cudaSuccess;
-  ProfScope ps("recurrent_fwd", s);
-  return bf16 ? launch_t<__nv_bfloat16>(p, a, status, s) : launch_t<float>(p, a, status, s);
+  ProfScope ps(kda ? "kda_recurrent_fwd" : "recurrent_fwd", s);
+  if (kda)
+    return bf16 ? launch_t<__nv_bfloat16, true>(p, a, status, s) : launch_t<float, true>(p, a, status, s);
+  return bf16 ? launch_t<__nv_bfloat16, false>(p, a, status, s) : launch_t<float, false>(p, a, status, s);
 }
 
 }  // namespace gdn

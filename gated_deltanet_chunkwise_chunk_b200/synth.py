@@ -140,6 +140,23 @@ def make_case(B=1, T=64, H=1, HV=1, K=64, V=64, dtype="fp32", seed=0, lengths=No
                 cu_seqlens=cu, h0=h0_t, dht=dht_t, seed=seed, name=name)
 
 
+def kda_gate_inputs(case: Case, seed: int, with_bias: bool = True, long_memory: bool = False):
+    """Per-key-channel gate inputs for the KDA form of a case: g_raw [B,T,HV,K] ~ N(0,1) and
+    dt_bias [HV*K] ~ N(0, 0.5) (or None), with the case's A_log; ``long_memory`` gives
+    A_log = log U(0.01, 0.1) and dt_bias = -4 as for the scalar gate.  Returns
+    (g_raw, A_log, dt_bias) as fp32 CPU tensors."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    g = _normal(rng, (case.B, case.T, case.HV, case.K))
+    if long_memory:
+        A_log = np.log(rng.uniform(0.01, 0.1, size=case.HV)).astype(np.float32)
+        dtb = np.full(case.HV * case.K, -4.0, dtype=np.float32)
+    else:
+        A_log = case.A_log.numpy()
+        dtb = _normal(rng, (case.HV * case.K,), 0.5)
+    return (torch.from_numpy(g), torch.from_numpy(np.ascontiguousarray(A_log)),
+            torch.from_numpy(dtb) if with_bias else None)
+
+
 def config_case(idx: int, seed: int | None = None, T: int | None = None) -> Case:
     """The seeded case of workload ``idx`` (seed defaults to 1000 + idx).  ``T`` overrides
     the sequence length of a dense workload (a smaller case of the same shape)."""

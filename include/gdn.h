@@ -183,6 +183,21 @@ int gdn_kda_gate_bwd(int64_t T, int64_t H, int64_t D, int32_t in_dtype, const vo
                      void* dg, float* dA_log, float* ddt_bias, void* workspace,
                      size_t workspace_bytes, void* stream);
 
+/* KDA (per-channel gated) delta rule, token by token, for decoding and short prefills:
+ *   S_t = S_{t-1} Diag(exp(yg_t)) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = scale S_t q_t,
+ *   yg_t[c] = -exp(A_log[hv]) * softplus(g_raw[t,hv,c] + dt_bias[hv*K + c])   (the KDA gate),
+ * i.e. gdn_recurrent_fwd with the scalar decay of each value head replaced by a decay per key
+ * channel (the pages give the KDA gate and name the KDA chunk kernels; the recurrence is the
+ * Gated DeltaNet one with that gate).  Arguments as gdn_recurrent_fwd except
+ *   g_raw    [B,T,HV,K] fp32 (raw per-channel gate input),
+ *   dt_bias  [HV*K] fp32, or NULL for none.
+ * Same workspace, status word, in-place state and error behaviour as gdn_recurrent_fwd. */
+int gdn_kda_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                          const float* g_raw, const float* A_log, const float* dt_bias,
+                          const float* beta, const int64_t* cu_seqlens, const float* initial_state,
+                          void* o, float* final_state, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
 /* Workspace bytes of gdn_kda_gate_bwd (0 for invalid sizes). */
 size_t gdn_kda_gate_workspace_bytes(int64_t T, int64_t H, int64_t D);
 
