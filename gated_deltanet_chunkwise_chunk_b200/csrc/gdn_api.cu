@@ -328,6 +328,7 @@ static int recurrent_common(const gdn_dims* d, const void* q, const void* k, con
   int rc = check_dims(d, varlen);
   if (rc) return rc;
   const bool empty = d->B * d->T == 0;
+  if ((varlen ? d->N : d->B) * (d->V / 32) > (int64_t)INT32_MAX) return GDN_ERR_INVALID_ARG;  // grid.x
   const void* tok[] = {q, k, v, g_raw, beta, o};
   for (const void* x : tok)
     if ((!x && !empty) || !aligned16(x)) return GDN_ERR_INVALID_ARG;

@@ -25,7 +25,10 @@ constexpr int RV = 32;  // state rows per CTA
 template <typename T, int K, bool KDA>
 __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* status) {
   constexpr int KQ = K / 16;  // state columns per thread
-  const int n = blockIdx.x, hv = blockIdx.y, hk = hv / p.G, v0 = RV * blockIdx.z;
+  // blockIdx.x = n * (V / RV) + slice: the slices of one state are neighbours in launch order,
+  // so the four 128-byte pieces of each 512-byte state row are fetched together
+  const int nz = p.V / RV;
+  const int n = blockIdx.x / nz, hv = blockIdx.y, hk = hv / p.G, v0 = RV * (blockIdx.x % nz);
   const int tid = threadIdx.x, lane = tid & 31, kg = lane & 15, vg = 2 * (tid >> 5) + (lane >> 4);
   __shared__ float sk[K], sq[K], sv[RV], sdec, sbeta, sdk[KDA ? K : 1];
   int bos, eos;
@@ -61,29 +64,30 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
     x += __shfl_xor_sync(0xffffffffu, x, 8);
     return x;
   };
+  const size_t dtb_k = (size_t)hv * K;
   for (int t = bos; t < eos; ++t) {
-    __syncthreads();  // the previous token's vectors are no longer read
+    // every load of this token first (one latency), spread over the threads; then one round
+    // of shared-memory stores between two barriers (K <= 128: one channel per thread)
     const size_t qk0 = ((size_t)t * p.H + hk) * K, v_0 = ((size_t)t * p.HV + hv) * p.V + v0;
-    for (int i = tid; i < K; i += 128) {
-      sk[i] = to_f<T>(k[qk0 + i]);
-      sq[i] = to_f<T>(q[qk0 + i]);
+    const size_t gi = (size_t)t * p.HV + hv;
+    float kf = 0.f, qf = 0.f, vf = 0.f, gf = 0.f, bf = 0.f;
+    if (tid < K) {
+      kf = to_f<T>(k[qk0 + tid]);
+      qf = to_f<T>(q[qk0 + tid]);
+      if constexpr (KDA) gf = a.g_raw[gi * K + tid] + (a.dt_bias ? a.dt_bias[dtb_k + tid] : 0.f);
     }
-    if (tid < RV) sv[tid] = to_f<T>(v[v_0 + tid]);
-    if constexpr (KDA) {  // per-channel decay of this token
-      const size_t g0 = ((size_t)t * p.HV + hv) * K;
-      for (int i = tid; i < K; i += 128) {
-        const float x = a.g_raw[g0 + i] + (a.dt_bias ? a.dt_bias[(size_t)hv * K + i] : 0.f);
-        sdk[i] = expf(nexp * (x > 20.f ? x : log1pf(expf(x))));
-      }
+    if (tid < RV) vf = to_f<T>(v[v_0 + tid]);
+    if (!KDA && tid == 64) gf = a.g_raw[gi] + dtb;
+    if (tid == 96) bf = a.beta[gi];
+    __syncthreads();  // the previous token's vectors are no longer read
+    if (tid < K) {
+      sk[tid] = kf;
+      sq[tid] = qf;
+      if constexpr (KDA) sdk[tid] = expf(nexp * (gf > 20.f ? gf : log1pf(expf(gf))));
     }
-    if (tid == 0) {
-      const size_t gi = (size_t)t * p.HV + hv;
-      if constexpr (!KDA) {
-        const float x = a.g_raw[gi] + dtb;
-        sdec = expf(nexp * (x > 20.f ? x : log1pf(expf(x))));
-      }
-      sbeta = a.beta[gi];
-    }
+    if (tid < RV) sv[tid] = vf;
+    if (!KDA && tid == 64) sdec = expf(nexp * (gf > 20.f ? gf : log1pf(expf(gf))));
+    if (tid == 96) sbeta = bf;
     __syncthreads();
     const float b = sbeta;
     float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -123,7 +127,7 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
 
 template <typename T, bool KDA>
 cudaError_t launch_t(const Problem& p, const Args& a, int* status, cudaStream_t s) {
-  const dim3 grid(p.Nst, p.HV, p.V / RV);
+  const dim3 grid((unsigned)p.Nst * (unsigned)(p.V / RV), p.HV);
   if (p.K == 128)
     k_recurrent_fwd<T, 128, KDA><<<grid, 128, 0, s>>>(p, a, status);
   else

@@ -148,7 +148,8 @@ size_t gdn_noalloc_scratch_bytes(void);
  * T = 1 decode steps and prefills of a few tokens, gdn_chunk_fwd for long sequences.
  * final_state may be the same buffer as initial_state (the state is updated in place).
  * workspace: at least GDN_RECURRENT_WORKSPACE_BYTES, 256-byte aligned; it holds the device
- * status word (gdn_device_status reports invalid cu_seqlens as GDN_ERR_INVALID_ARG). */
+ * status word (gdn_device_status reports invalid cu_seqlens as GDN_ERR_INVALID_ARG).
+ * Besides the size limits above, (number of sequences) * V / 32 < 2^31 (GDN_ERR_INVALID_ARG). */
 #define GDN_RECURRENT_WORKSPACE_BYTES ((size_t)256)
 int gdn_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
                       const float* g_raw, const float* A_log, const float* dt_bias,
