@@ -26,7 +26,8 @@ EXPORTED = ("gdn_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_max_ch
             "gdn_status_string", "gdn_version", "gdn_launch_count", "gdn_profile",
             "gdn_profile_read", "gdn_chunk_fwd_noalloc", "gdn_noalloc_scratch_bytes",
             "gdn_recurrent_fwd", "gdn_recurrent_workspace_bytes", "gdn_kda_gate_fwd",
-            "gdn_kda_gate_bwd", "gdn_kda_gate_workspace_bytes", "gdn_kda_recurrent_fwd")
+            "gdn_kda_gate_bwd", "gdn_kda_gate_workspace_bytes", "gdn_kda_recurrent_fwd",
+            "gdn_kda_chunk_fwd", "gdn_kda_chunk_workspace_bytes")
 
 
 class gdn_dims(ctypes.Structure):
@@ -57,6 +58,10 @@ def _load() -> ctypes.CDLL:
     lib.gdn_chunk_bwd.restype = I32
     lib.gdn_recurrent_fwd.argtypes = [D] + [P] * 12 + [SZ, P]
     lib.gdn_recurrent_fwd.restype = I32
+    lib.gdn_kda_chunk_fwd.argtypes = [D] + [P] * 12 + [SZ, P]
+    lib.gdn_kda_chunk_fwd.restype = I32
+    lib.gdn_kda_chunk_workspace_bytes.argtypes = [D, I32]
+    lib.gdn_kda_chunk_workspace_bytes.restype = SZ
     lib.gdn_kda_recurrent_fwd.argtypes = [D] + [P] * 12 + [SZ, P]
     lib.gdn_kda_recurrent_fwd.restype = I32
     lib.gdn_recurrent_workspace_bytes.argtypes = []
@@ -246,6 +251,39 @@ def gdn_kda_recurrent_fwd(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None,
                                    workspace.numel(), _stream())
     if rc != GDN_OK:
         raise GDNError("gdn_kda_recurrent_fwd", rc)
+    return o, ht
+
+
+def kda_chunk_workspace_bytes(dims: gdn_dims, varlen: bool) -> int:
+    return int(lib.gdn_kda_chunk_workspace_bytes(ctypes.byref(dims), int(varlen)))
+
+
+def gdn_kda_chunk_fwd(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None, initial_state=None,
+                      scale=0.0, output_final_state=True, out=None, final_state=None, workspace=None):
+    """Chunkwise KDA forward (per-key-channel gate, long sequences): returns (o, final_state or
+    None).  Arguments as gdn_kda_recurrent_fwd."""
+    B, T, H, K = q.shape
+    HV = v.shape[2]
+    Nst = _check_inputs(q, k, v, None, A_log, None, beta, cu_seqlens, initial_state)
+    _check("g_raw", g_raw, torch.float32, (B, T, HV, K), q.device)
+    _check("dt_bias", dt_bias, torch.float32, (HV * K,), q.device)
+    dims = make_dims(q, v, cu_seqlens, scale)
+    need = kda_chunk_workspace_bytes(dims, cu_seqlens is not None)
+    if need == 0:
+        raise GDNError("gdn_kda_chunk_workspace_bytes", GDN_ERR_INVALID_ARG)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    o = out if out is not None else torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    ht = None
+    if output_final_state:
+        ht = final_state if final_state is not None else torch.empty(
+            (Nst, HV, K, v.shape[3]), dtype=torch.float32, device=q.device)
+    rc = lib.gdn_kda_chunk_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g_raw),
+                               _ptr(A_log), _ptr(dt_bias), _ptr(beta), _ptr(cu_seqlens),
+                               _ptr(initial_state), _ptr(o), _ptr(ht), _ptr(workspace),
+                               workspace.numel(), _stream())
+    if rc != GDN_OK:
+        raise GDNError("gdn_kda_chunk_fwd", rc)
     return o, ht
 
 

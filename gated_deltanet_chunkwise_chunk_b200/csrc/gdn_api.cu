@@ -146,6 +146,36 @@ Problem make_problem(const gdn_dims& d, bool varlen) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
 
+// Workspace of the chunkwise KDA forward.
+struct KdaPlan {
+  size_t status, seq_tab, chunk_tab, W, Ut, Kh, Qt, P, eGC, h, U, total;
+};
+
+KdaPlan make_kda_plan(const gdn_dims& d, bool varlen) {
+  KdaPlan pl{};
+  const size_t NC = (size_t)max_chunks(d, varlen), Nst = varlen ? (size_t)d.N : (size_t)d.B;
+  const size_t HV = d.HV, K = d.K, V = d.V, f = sizeof(float);
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o += up(bytes);
+    return at;
+  };
+  pl.status = take(64);
+  pl.seq_tab = take(Nst * sizeof(int4));
+  pl.chunk_tab = take(NC * sizeof(int4));
+  pl.W = take(NC * HV * CH * K * f);
+  pl.Ut = take(NC * HV * CH * V * f);
+  pl.Kh = take(NC * HV * CH * K * f);
+  pl.Qt = take(NC * HV * CH * K * f);
+  pl.P = take(NC * HV * CH * CH * f);
+  pl.eGC = take(NC * HV * K * f);
+  pl.h = take(NC * HV * V * K * f);
+  pl.U = take(NC * HV * CH * V * f);
+  pl.total = o;
+  return pl;
+}
+
 // Steps shared by the forward and the backward: chunk table, gate + in-chunk cumsum.
 cudaError_t prologue(const Problem& p, const Args& a, const Work& w, cudaStream_t s) {
   cudaError_t e = launch_chunk_table(p, a.cu, w, s);
@@ -373,6 +403,65 @@ int gdn_kda_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const
                           void* stream) {
   return recurrent_common(d, q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens, initial_state, o,
                           final_state, workspace, workspace_bytes, stream, true);
+}
+
+size_t gdn_kda_chunk_workspace_bytes(const gdn_dims* d, int varlen) {
+  if (check_dims(d, varlen != 0) != GDN_OK) return 0;
+  return make_kda_plan(*d, varlen != 0).total;
+}
+
+int gdn_kda_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                      const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,
+                      const int64_t* cu_seqlens, const float* initial_state, void* o,
+                      float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
+  const bool varlen = cu_seqlens != nullptr;
+  int rc = check_dims(d, varlen);
+  if (rc) return rc;
+  const bool empty = d->B * d->T == 0;
+  const void* tok[] = {q, k, v, g_raw, beta, o};
+  for (const void* x : tok)
+    if ((!x && !empty) || !aligned16(x)) return GDN_ERR_INVALID_ARG;
+  if (!A_log || !aligned16(A_log) || !aligned16(dt_bias)) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(cu_seqlens) || !aligned16(initial_state) || !aligned16(final_state))
+    return GDN_ERR_INVALID_ARG;
+  const KdaPlan pl = make_kda_plan(*d, varlen);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) || workspace_bytes < pl.total)
+    return GDN_ERR_WORKSPACE;
+  const Problem p = make_problem(*d, varlen);
+  Args a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.g_raw = g_raw;
+  a.A_log = A_log;
+  a.dt_bias = dt_bias;
+  a.beta = beta;
+  a.cu = cu_seqlens;
+  a.h0 = initial_state;
+  a.o = o;
+  a.ht = final_state;
+  char* b = static_cast<char*>(workspace);
+  KdaWork w{};
+  w.status = reinterpret_cast<int*>(b + pl.status);
+  w.seq_tab = reinterpret_cast<int4*>(b + pl.seq_tab);
+  w.chunk_tab = reinterpret_cast<int4*>(b + pl.chunk_tab);
+  auto fp = [&](size_t off) { return reinterpret_cast<float*>(b + off); };
+  w.W = fp(pl.W);
+  w.Ut = fp(pl.Ut);
+  w.Kh = fp(pl.Kh);
+  w.Qt = fp(pl.Qt);
+  w.P = fp(pl.P);
+  w.eGC = fp(pl.eGC);
+  w.h = fp(pl.h);
+  w.U = fp(pl.U);
+  Work cw{};  // the chunk table kernel's view of the same status word and tables
+  cw.status = w.status;
+  cw.seq_tab = w.seq_tab;
+  cw.chunk_tab = w.chunk_tab;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_chunk_table(p, cu_seqlens, cw, s);
+  if (e == cudaSuccess) e = kda_chunk_forward(p, a, w, d->dtype == GDN_DTYPE_BF16, s);
+  return cuda_status(e);
 }
 
 static int kda_check(int64_t T, int64_t H, int64_t D, int32_t dt1, int32_t dt2) {

@@ -50,6 +50,21 @@ struct Work {
   float* pgp;         // [PG_BLOCKS][HV][2]    partial sums of the gate-parameter gradients
 };
 
+// Workspace of the chunkwise KDA forward (fp32, per chunk gc and value head hv).
+struct KdaWork {
+  int* status;     // [0] device status word, [1] chunk count
+  int4* seq_tab;   // [Nst]
+  int4* chunk_tab; // [NCmax]
+  float* W;        // [NCmax][HV][64][K]   T diag(beta) (k e^{Gam})
+  float* Ut;       // [NCmax][HV][64][V]   T diag(beta) V
+  float* Kh;       // [NCmax][HV][64][K]   k e^{Gam_C - Gam}
+  float* Qt;       // [NCmax][HV][64][K]   q e^{Gam}
+  float* P;        // [NCmax][HV][64][64]  sum_c q_i k_j e^{Gam_i - Gam_j}, lower incl. diagonal
+  float* eGC;      // [NCmax][HV][K]       e^{Gam_C}
+  float* h;        // [NCmax][HV][V][K]    state entering the chunk (S orientation)
+  float* U;        // [NCmax][HV][64][V]   U~ - W S^T
+};
+
 // Pointers of one call (inputs and outputs as given by the caller).
 struct Args {
   const void* q;

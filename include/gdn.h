@@ -199,6 +199,23 @@ int gdn_kda_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const
                           void* o, float* final_state, void* workspace, size_t workspace_bytes,
                           void* stream);
 
+/* Chunkwise forward of the same KDA recurrence as gdn_kda_recurrent_fwd, for long sequences:
+ * 64-token chunks, the per-channel decay carried through 16-token sub-chunks (every factor an
+ * exponential of a non-positive number), a sequential state pass over the chunks, fp32
+ * arithmetic on CUDA cores.  Arguments, layouts and results as gdn_kda_recurrent_fwd
+ * (g_raw [B,T,HV,K] fp32, dt_bias [HV*K] or NULL; o for every token, final_state after each
+ * sequence's last token; final_state may be NULL).  workspace: at least
+ * gdn_kda_chunk_workspace_bytes(d, varlen) bytes, 256-byte aligned; it also holds the device
+ * status word (gdn_device_status: GDN_ERR_INVALID_ARG for invalid cu_seqlens).  Same size
+ * limits and error returns as gdn_chunk_fwd. */
+int gdn_kda_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                      const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,
+                      const int64_t* cu_seqlens, const float* initial_state, void* o,
+                      float* final_state, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of gdn_kda_chunk_fwd (0 for invalid dimensions). */
+size_t gdn_kda_chunk_workspace_bytes(const gdn_dims* d, int varlen);
+
 /* Workspace bytes of gdn_kda_gate_bwd (0 for invalid sizes). */
 size_t gdn_kda_gate_workspace_bytes(int64_t T, int64_t H, int64_t D);
 
