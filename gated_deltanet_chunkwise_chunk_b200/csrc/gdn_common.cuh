@@ -61,7 +61,7 @@ struct KdaWork {
   float* Qt;       // [NCmax][HV][64][K]   q e^{Gam}
   float* P;        // [NCmax][HV][64][64]  sum_c q_i k_j e^{Gam_i - Gam_j}, lower incl. diagonal
   float* eGC;      // [NCmax][HV][K]       e^{Gam_C}
-  float* h;        // [NCmax][HV][V][K]    state entering the chunk (S orientation)
+  float* h;        // [NCmax][HV][K][V]    state entering the chunk (h[k][v] = S[v][k])
   float* U;        // [NCmax][HV][64][V]   U~ - W S^T
 };
 

@@ -25,12 +25,15 @@
 #include "ffma_tiles.cuh"
 #include "gdn_common.cuh"
 #include "gdn_launch.h"
+#include "gdn_tc_common.cuh"  // unit_lower_inverse64, LDA
 
 namespace gdn {
 namespace {
 
 constexpr int SUB = 16;  // sub-chunk length
+constexpr int RS = 52;   // row stride of the transposed key tile R^T (16-byte rows for float4 reads)
 constexpr float LOG2E = 1.4426950408889634f;
+using tcx::LDA;          // row stride of A, T and the inverse's scratch
 
 __device__ __forceinline__ bool kda_failed(const KdaWork& w) { return *((volatile int*)w.status) != 0; }
 
@@ -39,9 +42,58 @@ __device__ __forceinline__ float warp_total(float x) {
   return x;
 }
 
-size_t wy_smem(int K, int V) { return (size_t)(3 * CH * K + CH * V + 2 * CH * CH + 80 * K + CH) * sizeof(float); }
-size_t scan_smem(int K) { return (size_t)(32 * K + 2 * CH * K + CH * 32 + K) * sizeof(float); }
-size_t out_smem(int K, int V) { return (size_t)(CH * K + CH * CH + CH * V) * sizeof(float); }
+// 16-byte global -> shared copies (cp.async), all in flight until cp_async_wait_all.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
+// n floats (n % 4 == 0, both ends 16-byte aligned), issued by every thread, not waited for
+__device__ __forceinline__ void copy_async(float* dst, const float* src, int n) {
+  for (int i = threadIdx.x; i < n / 4; i += blockDim.x) cp_async16(dst + 4 * i, src + 4 * i);
+}
+
+// Rows [0, L) of a 64 x D token tile (row stride rs elements, D % 8 == 0) into fp32 shared
+// memory, rows past L zero: 16-byte loads, all of a thread's loads issued before any is used.
+template <typename T>
+__device__ __forceinline__ void load_tile(float* dst, const T* src, size_t rs, int L, int D) {
+  constexpr int E = 16 / sizeof(T);       // elements per 16-byte vector
+  constexpr int NV = CH * 128 / E / 256;  // vectors per thread at D = 128
+  const int nvec = CH * D / E;
+  uint4 r[NV];
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int vi = threadIdx.x + 256 * k, t = vi * E / D, c = vi * E % D;
+    r[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (vi < nvec && t < L) r[k] = __ldg(reinterpret_cast<const uint4*>(src + (size_t)t * rs + c));
+  }
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int vi = threadIdx.x + 256 * k;
+    if (vi >= nvec) continue;
+    float* d = dst + vi * E;
+    if constexpr (E == 4) {
+      *reinterpret_cast<uint4*>(d) = r[k];
+    } else {
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&r[k]);
+      const float2 f0 = __bfloat1622float2(h2[0]), f1 = __bfloat1622float2(h2[1]);
+      const float2 f2 = __bfloat1622float2(h2[2]), f3 = __bfloat1622float2(h2[3]);
+      *reinterpret_cast<float4*>(d) = make_float4(f0.x, f0.y, f1.x, f1.y);
+      *reinterpret_cast<float4*>(d + 4) = make_float4(f2.x, f2.y, f3.x, f3.y);
+    }
+  }
+}
+
+__host__ __device__ constexpr int wy_scratch(int K) {
+  return 2 * SUB * (K + 1) + RS * K > 2 * CH * LDA ? 2 * SUB * (K + 1) + RS * K : 2 * CH * LDA;
+}
+size_t wy_smem(int K, int V) {
+  return (size_t)(3 * CH * K + CH * V + CH * LDA + CH * CH + wy_scratch(K) + CH) * sizeof(float);
+}
+size_t scan_smem(int K) { return (size_t)(32 * (K + 1) + CH * (K + 1) + CH * K + CH * 32 + K) * sizeof(float); }
+size_t out_smem(int K, int V) { return (size_t)(CH * K + CH * CH + K * V + 2 * CH * V) * sizeof(float); }
 
 template <typename T>
 __global__ void __launch_bounds__(256) k_kda_wy(Problem p, Args a, KdaWork w) {
@@ -56,31 +108,39 @@ __global__ void __launch_bounds__(256) k_kda_wy(Problem p, Args a, KdaWork w) {
   float* sQ = sK + CH * K;    // [64][K] queries
   float* sG = sQ + CH * K;    // [64][K] Gam * log2(e)
   float* sV = sG + CH * K;    // [64][V]
-  float* sA = sV + CH * V;    // [64][64]
-  float* sP = sA + CH * CH;   // [64][64]
-  float* sX = sP + CH * CH;   // scratch: Lk [16][K], Lq [16][K], R [48][K]; later T [64][64]
-  float* sb = sX + 80 * K;    // [64] beta, 0 past L
+  float* sA = sV + CH * V;    // [64][LDA]
+  float* sP = sA + CH * LDA;  // [64][64]
+  float* sX = sP + CH * CH;   // scratch: Lk [16][K+1], Lq [16][K+1], R^T [K][RS]; later T, X [64][LDA]
+  float* sb = sX + wy_scratch(K);  // [64] beta, 0 past L
   const size_t rs = (size_t)p.H * K;
-  load_rows<T>(sK, static_cast<const T*>(a.k) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
-  load_rows<T>(sQ, static_cast<const T*>(a.q) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
-  load_rows<T>(sV, static_cast<const T*>(a.v) + ((size_t)tok0 * p.HV + hv) * V, (size_t)p.HV * V, L, V);
+  load_tile<T>(sK, static_cast<const T*>(a.k) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
+  load_tile<T>(sQ, static_cast<const T*>(a.q) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
+  load_tile<T>(sV, static_cast<const T*>(a.v) + ((size_t)tok0 * p.HV + hv) * V, (size_t)p.HV * V, L, V);
+  load_tile<float>(sG, a.g_raw + ((size_t)tok0 * p.HV + hv) * K, (size_t)p.HV * K, L, K);
   if (tid < CH) sb[tid] = tid < L ? a.beta[(size_t)(tok0 + tid) * p.HV + hv] : 0.f;
-  {  // gate and its inclusive cumsum per channel; rows past L keep the last value
+  __syncthreads();
+  {  // the gate of every (token, channel), rows past L zero; then the cumsum per channel
     const float nexp = -expf(a.A_log[hv]);
-    const float* gr = a.g_raw + ((size_t)tok0 * p.HV + hv) * K;
+    for (int x = tid; x < CH * K; x += blockDim.x) {
+      const int i = x / K, c = x % K;
+      float yg = 0.f;
+      if (i < L) {
+        const float z = sG[x] + (a.dt_bias ? a.dt_bias[(size_t)hv * K + c] : 0.f);
+        yg = nexp * (z > 20.f ? z : log1pf(expf(z)));
+      }
+      sG[x] = yg;
+    }
+    __syncthreads();
     for (int c = tid; c < K; c += blockDim.x) {
-      const float bias = a.dt_bias ? a.dt_bias[(size_t)hv * K + c] : 0.f;
       float acc = 0.f;
       for (int i = 0; i < CH; ++i) {
-        if (i < L) {
-          const float x = gr[(size_t)i * p.HV * K + c] + bias;
-          acc += nexp * (x > 20.f ? x : log1pf(expf(x)));
-        }
+        acc += sG[i * K + c];
         sG[i * K + c] = acc * LOG2E;
       }
     }
   }
-  for (int x = tid; x < 2 * CH * CH; x += blockDim.x) sA[x] = 0.f;  // sA and sP
+  for (int x = tid; x < CH * LDA; x += blockDim.x) sA[x] = 0.f;
+  for (int x = tid; x < CH * CH; x += blockDim.x) sP[x] = 0.f;
   __syncthreads();
   // diagonal sub-blocks, one warp per pair (i, j), j <= i in one sub-chunk, lanes over channels
   constexpr int PAIRS = SUB * (SUB + 1) / 2;
@@ -98,51 +158,57 @@ __global__ void __launch_bounds__(256) k_kda_wy(Problem p, Args a, KdaWork w) {
     sa = warp_total(sa);
     sp = warp_total(sp);
     if (lane == 0) {
-      if (j < i) sA[i * CH + j] = sb[i] * sa;
+      if (j < i) sA[i * LDA + j] = sb[i] * sa;
       sP[i * CH + j] = sp;
     }
   }
   // blocks below the diagonal, through the reference token r = last token before sub-chunk blk
-  float* Lk = sX;
-  float* Lq = sX + SUB * K;
-  float* R = sX + 2 * SUB * K;
+  float* Lk = sX;                    // [16][K+1]
+  float* Lq = sX + SUB * (K + 1);    // [16][K+1]
+  float* RT = sX + 2 * SUB * (K + 1);  // [K][RS]: RT[c][j] = k_j[c] e^{Gam_r[c] - Gam_j[c]}
   for (int blk = 1; blk < CH / SUB; ++blk) {
     const int r = blk * SUB - 1, nj = blk * SUB;
     __syncthreads();  // the previous block's products are done with the scratch
     for (int x = tid; x < SUB * K; x += blockDim.x) {
-      const int i = blk * SUB + x / K, c = x % K;
+      const int ii = x / K, c = x % K, i = blk * SUB + ii;
       const float ex = exp2f(sG[i * K + c] - sG[r * K + c]);
-      Lk[x] = sK[i * K + c] * ex;
-      Lq[x] = sQ[i * K + c] * ex;
+      Lk[ii * (K + 1) + c] = sK[i * K + c] * ex;
+      Lq[ii * (K + 1) + c] = sQ[i * K + c] * ex;
     }
     for (int x = tid; x < nj * K; x += blockDim.x) {
       const int j = x / K, c = x % K;
-      R[x] = sK[x] * exp2f(sG[r * K + c] - sG[j * K + c]);
+      RT[c * RS + j] = sK[x] * exp2f(sG[r * K + c] - sG[x]);
     }
     __syncthreads();
-    mm(SUB, nj, K, sA + blk * SUB * CH, CH, 1.f, false, Lk, K, 1, R, 1, K);
-    mm(SUB, nj, K, sP + blk * SUB * CH, CH, 1.f, false, Lq, K, 1, R, 1, K);
-  }
-  __syncthreads();
-  for (int x = tid; x < CH * CH; x += blockDim.x) {  // beta_i on the blocks below the diagonal
-    const int i = x / CH, j = x % CH;
-    if (j < (i / SUB) * SUB) sA[x] *= sb[i];
+    // one 1 x 4 strip of A (times beta_i) or P per task: all threads busy for every block
+    const int ns = nj / 4, per = SUB * ns;
+    for (int tk = tid; tk < 2 * per; tk += blockDim.x) {
+      const int mat = tk / per, ii = (tk % per) / ns, j4 = 4 * (tk % ns), i = blk * SUB + ii;
+      const float* lrow = (mat ? Lq : Lk) + ii * (K + 1);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int c = 0; c < K; ++c) {
+        const float l = lrow[c];
+        const float4 rt = *reinterpret_cast<const float4*>(RT + c * RS + j4);
+        acc.x = fmaf(l, rt.x, acc.x);
+        acc.y = fmaf(l, rt.y, acc.y);
+        acc.z = fmaf(l, rt.z, acc.z);
+        acc.w = fmaf(l, rt.w, acc.w);
+      }
+      if (mat) {
+        *reinterpret_cast<float4*>(sP + i * CH + j4) = acc;
+      } else {
+        const float b = sb[i];
+        *reinterpret_cast<float4*>(sA + i * LDA + j4) = make_float4(b * acc.x, b * acc.y, b * acc.z, b * acc.w);
+      }
+    }
   }
   __syncthreads();
   const size_t u = (size_t)gc * p.HV + hv;
   float* gP = w.P + u * CH * CH;
   for (int x = tid; x < CH * CH; x += blockDim.x) gP[x] = sP[x];
-  // T = (I + A)^-1 by forward substitution, one column per thread
   float* sT = sX;
-  if (tid < CH) {
-    const int n = tid;
-    for (int r = 0; r < CH; ++r) {
-      float s = r == n ? 1.f : 0.f;
-      if (r > n)
-        for (int j = n; j < r; ++j) s -= sA[r * CH + j] * sT[j * CH + n];
-      sT[r * CH + n] = s;
-    }
-  }
+  tcx::unit_lower_inverse64(sA, sT, sX + CH * LDA, tid);  // T = (I + A)^-1 (ends with a barrier)
   // K^ = k e^{Gam_C - Gam}, Q~ = q e^{Gam}, e^{Gam_C}; then beta e^{Gam} k in place for W
   const size_t uk = u * CH * K;
   for (int x = tid; x < CH * K; x += blockDim.x) {
@@ -155,49 +221,89 @@ __global__ void __launch_bounds__(256) k_kda_wy(Problem p, Args a, KdaWork w) {
   for (int c = tid; c < K; c += blockDim.x) w.eGC[u * K + c] = exp2f(sG[(CH - 1) * K + c]);
   for (int x = tid; x < CH * V; x += blockDim.x) sV[x] *= sb[x / V];
   __syncthreads();
-  mm(CH, K, CH, w.W + uk, K, 1.f, false, sT, CH, 1, sK, K, 1);
-  mm(CH, V, CH, w.Ut + u * CH * V, V, 1.f, false, sT, CH, 1, sV, V, 1);
+  mm(CH, K, CH, w.W + uk, K, 1.f, false, sT, LDA, 1, sK, K, 1);
+  mm(CH, V, CH, w.Ut + u * CH * V, V, 1.f, false, sT, LDA, 1, sV, V, 1);
 }
 
-// Sequential scan of one (sequence, value head, rows v0..v0+31 of S): stores S entering each
-// chunk and U = U~ - W S^T for those rows, returns the final state.
+// Sequential scan of one (sequence, value head, rows v0..v0+31 of S): stores the state entering
+// each chunk (h[k][v] orientation) and U = U~ - W S^T for those rows, returns the final state.
+// The next chunk's W, K^, U~ slice and e^{Gam_C} are loaded into registers while the current
+// chunk's products run.
 __global__ void __launch_bounds__(256) k_kda_scan(Problem p, Args a, KdaWork w) {
   if (kda_failed(w)) return;
   const int n = blockIdx.x, hv = blockIdx.y, v0 = 32 * blockIdx.z, K = p.K, V = p.V, tid = threadIdx.x;
   const int4 sq = w.seq_tab[n];
   extern __shared__ float sm[];
-  float* sS = sm;            // [32][K]
-  float* sW = sS + 32 * K;   // [64][K]
-  float* sKh = sW + CH * K;  // [64][K]
-  float* sU = sKh + CH * K;  // [64][32]
-  float* sE = sU + CH * 32;  // [K] e^{Gam_C}
-  for (int x = tid; x < 32 * K; x += blockDim.x) {
-    const int vv = x / K, c = x % K;
-    sS[x] = a.h0 ? a.h0[(((size_t)n * p.HV + hv) * K + c) * V + v0 + vv] : 0.f;
+  float* sS = sm;                  // [32][K+1]
+  float* sW = sS + 32 * (K + 1);   // [64][K+1]
+  float* sKh = sW + CH * (K + 1);  // [64][K]
+  float* sU = sKh + CH * K;        // [64][32]
+  float* sE = sU + CH * 32;        // [K] e^{Gam_C}
+  for (int x = tid; x < 32 * K; x += blockDim.x) {  // lanes along v: coalesced h0 reads
+    const int vv = x % 32, c = x / 32;
+    sS[vv * (K + 1) + c] = a.h0 ? a.h0[(((size_t)n * p.HV + hv) * K + c) * V + v0 + vv] : 0.f;
   }
+  constexpr int NW = CH * 128 / 4 / 256;  // float4 of a [64][128] tile per thread
+  const int nw = CH * K / 4 / 256;        // 8 (K = 128) or 4 (K = 64)
+  float4 rW[NW], rK[NW];
+  float rU[CH * 32 / 256], rE = 0.f;
+  auto fetch = [&](size_t u) {
+    const float4* gw = reinterpret_cast<const float4*>(w.W + u * CH * K);
+    const float4* gk = reinterpret_cast<const float4*>(w.Kh + u * CH * K);
+#pragma unroll
+    for (int r = 0; r < NW; ++r)
+      if (r < nw) {
+        rW[r] = gw[tid + 256 * r];
+        rK[r] = gk[tid + 256 * r];
+      }
+#pragma unroll
+    for (int r = 0; r < CH * 32 / 256; ++r) {
+      const int x = tid + 256 * r;
+      rU[r] = w.Ut[u * CH * V + (x / 32) * V + v0 + x % 32];
+    }
+    if (tid < K) rE = w.eGC[u * K + tid];
+  };
+  auto stash = [&]() {
+#pragma unroll
+    for (int r = 0; r < NW; ++r)
+      if (r < nw) {
+        const int x = 4 * (tid + 256 * r), i = x / K, c = x % K;
+        float* d = sW + i * (K + 1) + c;
+        d[0] = rW[r].x; d[1] = rW[r].y; d[2] = rW[r].z; d[3] = rW[r].w;
+        *reinterpret_cast<float4*>(sKh + x) = rK[r];
+      }
+#pragma unroll
+    for (int r = 0; r < CH * 32 / 256; ++r) sU[tid + 256 * r] = rU[r];
+    if (tid < K) sE[tid] = rE;
+  };
+  if (sq.y > 0) fetch((size_t)sq.x * p.HV + hv);
   for (int ci = 0; ci < sq.y; ++ci) {
     const size_t u = (size_t)(sq.x + ci) * p.HV + hv;
     __syncthreads();  // the previous chunk is done with every buffer
-    copy_f(sW, w.W + u * CH * K, CH * K);
-    copy_f(sKh, w.Kh + u * CH * K, CH * K);
-    for (int x = tid; x < CH * 32; x += blockDim.x) sU[x] = w.Ut[u * CH * V + (x / 32) * V + v0 + x % 32];
-    for (int c = tid; c < K; c += blockDim.x) sE[c] = w.eGC[u * K + c];
-    float* h = w.h + u * V * K + (size_t)v0 * K;
-    for (int x = tid; x < 32 * K; x += blockDim.x) h[x] = sS[x];
+    stash();
+    float* h = w.h + u * K * V;  // h[k][v] of the state entering the chunk
+    for (int x = tid; x < 32 * K; x += blockDim.x) {
+      const int vv = x % 32, c = x / 32;
+      h[(size_t)c * V + v0 + vv] = sS[vv * (K + 1) + c];
+    }
     __syncthreads();
-    mm(CH, 32, K, sU, 32, -1.f, true, sW, K, 1, sS, 1, K);  // U = U~ - W S^T
+    if (ci + 1 < sq.y) fetch(u + p.HV);
+    mm(CH, 32, K, sU, 32, -1.f, true, sW, K + 1, 1, sS, 1, K + 1);  // U = U~ - W S^T
     __syncthreads();
     float* U = w.U + u * CH * V;
     for (int x = tid; x < CH * 32; x += blockDim.x) U[(x / 32) * V + v0 + x % 32] = sU[x];
-    for (int x = tid; x < 32 * K; x += blockDim.x) sS[x] *= sE[x % K];
+    for (int x = tid; x < 32 * K; x += blockDim.x) {
+      const int vv = x / K, c = x % K;
+      sS[vv * (K + 1) + c] *= sE[c];
+    }
     __syncthreads();
-    mm(32, K, CH, sS, K, 1.f, true, sU, 1, 32, sKh, K, 1);  // S' = S Diag(e^{Gam_C}) + U^T K^
+    mm(32, K, CH, sS, K + 1, 1.f, true, sU, 1, 32, sKh, K, 1);  // S' = S Diag(e^{Gam_C}) + U^T K^
   }
   __syncthreads();
   if (a.ht)
     for (int x = tid; x < 32 * K; x += blockDim.x) {
-      const int vv = x / K, c = x % K;
-      a.ht[(((size_t)n * p.HV + hv) * K + c) * V + v0 + vv] = sS[x];
+      const int vv = x % 32, c = x / 32;
+      a.ht[(((size_t)n * p.HV + hv) * K + c) * V + v0 + vv] = sS[vv * (K + 1) + c];
     }
 }
 
@@ -212,13 +318,18 @@ __global__ void __launch_bounds__(256) k_kda_out(Problem p, Args a, KdaWork w) {
   extern __shared__ float sm[];
   float* sQt = sm;           // [64][K]
   float* sP = sQt + CH * K;  // [64][64]
-  float* sO = sP + CH * CH;  // [64][V]
+  float* sH = sP + CH * CH;  // [K][V]  state entering the chunk, h[k][v]
+  float* sU = sH + K * V;    // [64][V]
+  float* sO = sU + CH * V;   // [64][V]
   const size_t u = (size_t)gc * p.HV + hv;
-  copy_f(sQt, w.Qt + u * CH * K, CH * K);
-  copy_f(sP, w.P + u * CH * CH, CH * CH);
+  copy_async(sQt, w.Qt + u * CH * K, CH * K);
+  copy_async(sP, w.P + u * CH * CH, CH * CH);
+  copy_async(sH, w.h + u * K * V, K * V);
+  copy_async(sU, w.U + u * CH * V, CH * V);
+  cp_async_wait_all();
   __syncthreads();
-  mm(CH, V, CH, sO, V, 1.f, false, sP, CH, 1, w.U + u * CH * V, V, 1);
-  mm(CH, V, K, sO, V, 1.f, true, sQt, K, 1, w.h + u * V * K, 1, K);
+  mm(CH, V, CH, sO, V, 1.f, false, sP, CH, 1, sU, V, 1);
+  mm(CH, V, K, sO, V, 1.f, true, sQt, K, 1, sH, V, 1);
   __syncthreads();
   T* o = static_cast<T*>(a.o) + ((size_t)tok0 * p.HV + hv) * V;
   for (int x = threadIdx.x; x < L * V; x += blockDim.x)
