@@ -125,3 +125,58 @@ def test_chunk_algebra_equals_the_recurrence(T, strong):
     o2, ht2 = kca.forward(q, k, v, g, A_log, dt_bias, beta, h0=S0)
     np.testing.assert_allclose(o2, o, rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(ht2, ht, rtol=1e-9, atol=1e-11)
+
+
+def _loss(q, k, v, g, A_log, dt_bias, beta, S0, dO, dht, cu=None):
+    o, ht = kda.recurrent_fwd(q, k, v, g, A_log, dt_bias, beta, cu_seqlens=cu, h0=S0)
+    return float(np.sum(dO * o) + np.sum(dht * ht))
+
+
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_backward_matches_central_differences(with_bias):
+    rng = np.random.default_rng(31)
+    q, k, v, g, A_log, dt_bias, beta, S0 = _case(rng, B=1, T=6, H=1, HV=2, K=4, V=3)
+    g[0, 0, 0, :2] = [20.5, 30.0]  # the softplus pass-through
+    if not with_bias:
+        dt_bias = None
+    dO = rng.standard_normal(v.shape)
+    dht = rng.standard_normal(S0.shape)
+    gr = kda.recurrent_bwd(q, k, v, g, A_log, dt_bias, beta, dO, h0=S0, dht=dht)
+    eps = 1e-6
+    args = dict(q=q, k=k, v=v, g=g, A_log=A_log, dt_bias=dt_bias, beta=beta, S0=S0)
+    checks = [("q", "dq", (0, 2, 0, 1)), ("k", "dk", (0, 3, 0, 2)), ("k", "dk", (0, 0, 0, 0)),
+              ("v", "dv", (0, 4, 1, 2)), ("beta", "dbeta", (0, 1, 1)), ("g", "dg_raw", (0, 0, 0, 1)),
+              ("g", "dg_raw", (0, 5, 1, 3)), ("g", "dg_raw", (0, 2, 0, 2)), ("S0", "dh0", (0, 1, 2, 0)),
+              ("A_log", "dA_log", (1,))]
+    if with_bias:
+        checks.append(("dt_bias", "ddt_bias", (5,)))
+    for name, gname, idx in checks:
+        p_, m_ = dict(args), dict(args)
+        p_[name] = args[name].copy()
+        m_[name] = args[name].copy()
+        p_[name][idx] += eps
+        m_[name][idx] -= eps
+        fd = (_loss(**p_, dO=dO, dht=dht) - _loss(**m_, dO=dO, dht=dht)) / (2 * eps)
+        assert abs(fd - gr[gname][idx]) <= 1e-6 * max(1.0, abs(fd)), (gname, idx, fd, gr[gname][idx])
+    if not with_bias:
+        assert gr["ddt_bias"] is None
+
+
+def test_backward_channel_constant_gate_is_gated_deltanet():
+    """A gate shared by every channel: the KDA gradients equal the C++ Gated DeltaNet oracle's,
+    with the per-channel gate gradients summed over channels."""
+    rng = np.random.default_rng(32)
+    q, k, v, g, A_log, dt_bias, beta, S0 = _case(rng, B=2, T=21, H=2, HV=4, K=8, V=6)
+    a = rng.standard_normal(g.shape[:3]) * 3.0
+    K = g.shape[-1]
+    g = np.repeat(a[..., None], K, axis=-1)
+    dtb = rng.standard_normal(g.shape[2])
+    dO = rng.standard_normal(v.shape)
+    dht = rng.standard_normal(S0.shape)
+    gr = kda.recurrent_bwd(q, k, v, g, A_log, np.repeat(dtb, K), beta, dO, h0=S0, dht=dht)
+    ref = oracle.bwd(q, k, v, a, A_log, dtb, beta, dO, h0=S0, dht=dht)
+    for key in ("dq", "dk", "dv", "dbeta", "dh0", "dA_log"):
+        np.testing.assert_allclose(gr[key], ref[key], rtol=1e-9, atol=1e-11, err_msg=key)
+    np.testing.assert_allclose(gr["dg"].sum(-1), ref["dg"], rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(gr["dg_raw"].sum(-1), ref["da"], rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(gr["ddt_bias"].reshape(-1, K).sum(-1), ref["ddt_bias"], rtol=1e-9, atol=1e-11)
