@@ -92,3 +92,120 @@ def forward(q, k, v, g_raw, A_log, dt_bias, beta, scale=None, h0=None):
                 o[bb, c0:c0 + n, hv] = O[:n]
             ht[bb, hv] = S.T
     return o, ht
+
+
+def gated_rows(Wt, R, Gam):
+    """F_i = sum_{j <= i} Wt_ij R_j e^{Gam_i - Gam_j}  (per channel), sub-chunk form."""
+    F = np.zeros_like(R)
+    for a in range(C // SUB):
+        ia = slice(a * SUB, (a + 1) * SUB)
+        if a > 0:
+            r = a * SUB - 1
+            RT = R[:a * SUB] * np.exp(Gam[r] - Gam[:a * SUB])
+            F[ia] += np.exp(Gam[ia] - Gam[r]) * (Wt[ia, :a * SUB] @ RT)
+        for i in range(a * SUB, (a + 1) * SUB):
+            for j in range(a * SUB, i + 1):
+                F[i] += Wt[i, j] * R[j] * np.exp(Gam[i] - Gam[j])
+    return F
+
+
+def gated_cols(Wt, L, Gam):
+    """G_j = sum_{i >= j} Wt_ij L_i e^{Gam_i - Gam_j}  (per channel), sub-chunk form."""
+    Gm = np.zeros_like(L)
+    for a in range(C // SUB):
+        ia = slice(a * SUB, (a + 1) * SUB)
+        if a > 0:
+            r = a * SUB - 1
+            Ls = L[ia] * np.exp(Gam[ia] - Gam[r])
+            Gm[:a * SUB] += np.exp(Gam[r] - Gam[:a * SUB]) * (Wt[ia, :a * SUB].T @ Ls)
+        for i in range(a * SUB, (a + 1) * SUB):
+            for j in range(a * SUB, i + 1):
+                Gm[j] += Wt[i, j] * L[i] * np.exp(Gam[i] - Gam[j])
+    return Gm
+
+
+def bwd_unit(Qc, Kc, Vc, ygc, b, S, dO, dSn, scale):
+    """One chunk backward: returns (dQ, dK, dV, db, dyg, dS_entering) for loss
+    sum(dO * O) + sum(dSn * S_next), S (V x K) the state entering the chunk."""
+    Gam = np.cumsum(ygc, axis=0)
+    A, P = intra(Qc, Kc, Gam, b)
+    T = np.linalg.inv(np.eye(C) + A)
+    eG, eC = np.exp(Gam), np.exp(Gam[-1])
+    Kt, Qt, Kh = Kc * eG, Qc * eG, Kc * np.exp(Gam[-1] - Gam)
+    X, Y = b[:, None] * Kt, b[:, None] * Vc
+    W, Ut = T @ X, T @ Y
+    U = Ut - W @ S.T
+    # scan part
+    dU = scale * P.T @ dO + Kh @ dSn.T
+    dS = dSn * eC[None, :] + scale * dO.T @ Qt - dU.T @ W
+    # output and state products
+    dQt = scale * dO @ S
+    dP = np.tril(scale * dO @ U.T)
+    dKh = U @ dSn
+    dW = -dU @ S
+    dGam = dQt * Qt - dKh * Kh
+    dGamC = np.sum(dKh * Kh, axis=0) + np.sum(dSn * S, axis=0) * eC
+    dQ = dQt * eG
+    dK = dKh * np.exp(Gam[-1] - Gam)
+    # P_ij = sum_c q_i k_j e^{Gam_i - Gam_j}
+    F2 = gated_rows(dP, Kc, Gam)
+    G2 = gated_cols(dP, Qc, Gam)
+    dQ += F2
+    dK += G2
+    dGam += Qc * F2 - Kc * G2
+    # WY part
+    dT = dW @ X.T + dU @ Y.T
+    dX, dY = T.T @ dW, T.T @ dU
+    dV = b[:, None] * dY
+    db = np.sum(dY * Vc, axis=1) + np.sum(dX * Kt, axis=1)
+    dKt = b[:, None] * dX
+    dK += dKt * eG
+    dGam += dKt * Kt
+    dA = np.tril(-T.T @ dT @ T.T, -1)
+    # A_ij = b_i sum_c k_i k_j e^{Gam_i - Gam_j}
+    F1 = gated_rows(dA, Kc, Gam)              # without b
+    G1 = gated_cols(b[:, None] * dA, Kc, Gam)
+    db += np.sum(Kc * F1, axis=1)
+    dK += b[:, None] * F1 + G1
+    dGam += b[:, None] * Kc * F1 - Kc * G1
+    dGam[-1] += dGamC
+    dyg = np.cumsum(dGam[::-1], axis=0)[::-1]
+    return dQ, dK, dV, db, dyg, dS
+
+
+def backward(q, k, v, g_raw, A_log, dt_bias, beta, dO, scale=None, h0=None, dht=None):
+    """Dense batch: dq, dk, dv, dbeta, dyg (dL/dlog-decay, [B,T,HV,K]), dh0."""
+    q, k, v, g_raw, beta, dO = (np.asarray(x, dtype=np.float64) for x in (q, k, v, g_raw, beta, dO))
+    A_log = np.asarray(A_log, dtype=np.float64)
+    B, T, H, K = q.shape
+    HV, V = v.shape[2], v.shape[3]
+    G = HV // H
+    if scale is None:
+        scale = K ** -0.5
+    dtb = None if dt_bias is None else np.asarray(dt_bias, dtype=np.float64).reshape(HV, K)
+    out = dict(dq=np.zeros((B, T, H, K)), dk=np.zeros((B, T, H, K)), dv=np.zeros((B, T, HV, V)),
+               dbeta=np.zeros((B, T, HV)), dg=np.zeros((B, T, HV, K)), dh0=np.zeros((B, HV, K, V)))
+    for bb in range(B):
+        for hv in range(HV):
+            yg = _gate(g_raw[bb, :, hv], A_log[hv], None if dtb is None else dtb[hv])
+            S = np.zeros((V, K)) if h0 is None else np.asarray(h0[bb, hv], dtype=np.float64).T.copy()
+            chunks, states = [], []
+            for c0 in range(0, T, C):
+                n = min(C, T - c0)
+                pad = lambda x, n=n: np.concatenate([x, np.zeros((C - n,) + x.shape[1:])]) if n < C else x
+                ch = (pad(q[bb, c0:c0 + n, hv // G]), pad(k[bb, c0:c0 + n, hv // G]),
+                      pad(v[bb, c0:c0 + n, hv]), pad(yg[c0:c0 + n]), pad(beta[bb, c0:c0 + n, hv]),
+                      pad(dO[bb, c0:c0 + n, hv]), c0, n)
+                chunks.append(ch)
+                states.append(S)
+                _, S, _ = fwd_unit(ch[0], ch[1], ch[2], ch[3], ch[4], S, scale)
+            dS = np.zeros((V, K)) if dht is None else np.asarray(dht[bb, hv], dtype=np.float64).T.copy()
+            for (Qc, Kc, Vc, ygc, bc, dOc, c0, n), S0 in zip(chunks[::-1], states[::-1]):
+                dQ, dK, dV, db, dyg, dS = bwd_unit(Qc, Kc, Vc, ygc, bc, S0, dOc, dS, scale)
+                out["dq"][bb, c0:c0 + n, hv // G] += dQ[:n]
+                out["dk"][bb, c0:c0 + n, hv // G] += dK[:n]
+                out["dv"][bb, c0:c0 + n, hv] = dV[:n]
+                out["dbeta"][bb, c0:c0 + n, hv] = db[:n]
+                out["dg"][bb, c0:c0 + n, hv] = dyg[:n]
+            out["dh0"][bb, hv] = dS.T
+    return out

@@ -180,3 +180,21 @@ def test_backward_channel_constant_gate_is_gated_deltanet():
     np.testing.assert_allclose(gr["dg"].sum(-1), ref["dg"], rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(gr["dg_raw"].sum(-1), ref["da"], rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(gr["ddt_bias"].reshape(-1, K).sum(-1), ref["ddt_bias"], rtol=1e-9, atol=1e-11)
+
+
+@pytest.mark.parametrize("T,strong", [(1, False), (40, False), (64, True), (65, False), (150, True)])
+def test_chunk_backward_algebra_equals_the_oracle(T, strong):
+    """The chunk-form backward the CUDA kernels implement (tests/kda_chunk_algebra.py: scan,
+    output/state products, gated per-channel products of dP and dA in sub-chunk form, WY
+    backward, reverse cumsum of dGam) equals the token-by-token oracle backward."""
+    from . import kda_chunk_algebra as kca
+    rng = np.random.default_rng(40 + T)
+    q, k, v, g, A_log, dt_bias, beta, S0 = _case(rng, B=1, T=T, H=2, HV=4, K=16, V=8)
+    if strong:
+        A_log = np.log(rng.uniform(1.0, 16.0, 4))
+    dO = rng.standard_normal(v.shape)
+    dht = rng.standard_normal(S0.shape)
+    ref = kda.recurrent_bwd(q, k, v, g, A_log, dt_bias, beta, dO, h0=S0, dht=dht)
+    got = kca.backward(q, k, v, g, A_log, dt_bias, beta, dO, h0=S0, dht=dht)
+    for key in ("dq", "dk", "dv", "dbeta", "dg", "dh0"):
+        np.testing.assert_allclose(got[key], ref[key], rtol=1e-8, atol=1e-10, err_msg=key)
