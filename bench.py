@@ -600,55 +600,67 @@ FFMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # fp32 lanes x 2 FLOP x max SM clo
 
 
 def kda_chunk_measure(gdn, dev, pk_hbm: float, steps: int = 5) -> dict:
-    """Chunkwise KDA forward (per-key-channel gate) at the layer's shape: B = 1, T = 32768,
-    H = 16, HV = 32, K = V = 128, bf16 tokens.  fp32 on CUDA cores, so the bound is the FFMA
-    rate (FLOPs per (chunk, value head): A and P 0.53 M FMA, W and U~ 1.05 M, scan 2.10 M,
-    output 1.57 M)."""
+    """Chunkwise KDA (per-key-channel gate) at the layer's shape: B = 1, T = 32768, H = 16,
+    HV = 32, K = V = 128, bf16 tokens: the forward alone and a training step (forward +
+    backward reading the forward's intermediates).  fp32 on CUDA cores, so the bound is the
+    FFMA rate (FLOPs per (chunk, value head): forward A and P 0.53 M FMA, W and U~ 1.05 M, scan
+    2.10 M, output 1.57 M)."""
     case = synth.make_case(B=1, T=32768, H=16, HV=32, K=128, V=128, dtype="bf16", seed=4244,
                            h0=True, name="kda_chunk")
     g_raw, A_log, dt_bias = synth.kda_gate_inputs(case, 4245)
     t = lambda x: None if x is None else x.to(dev).contiguous()
     d = dict(q=t(case.q), k=t(case.k), v=t(case.v), g_raw=t(g_raw), A_log=t(A_log),
-             dt_bias=t(dt_bias), beta=t(case.beta), initial_state=t(case.h0))
+             dt_bias=t(dt_bias), beta=t(case.beta))
+    h0, dO = t(case.h0), t(case.dO)
     dims = gdn.make_dims(d["q"], d["v"])
-    ws = torch.empty(gdn.kda_chunk_workspace_bytes(dims, False), dtype=torch.uint8, device=dev)
+    ws = torch.empty(gdn.kda_chunk_workspace_bytes(dims, False, True), dtype=torch.uint8, device=dev)
     o = torch.empty_like(d["v"])
-    ht = torch.empty_like(d["initial_state"])
+    ht = torch.empty_like(h0)
+    outs = dict(dq=torch.empty_like(d["q"]), dk=torch.empty_like(d["k"]), dv=torch.empty_like(d["v"]),
+                dbeta=torch.empty_like(d["beta"]), dg=torch.empty_like(d["g_raw"]), dh0=torch.empty_like(h0),
+                dg_raw=torch.empty_like(d["g_raw"]), dA_log=torch.empty_like(d["A_log"]),
+                ddt_bias=torch.empty_like(d["dt_bias"]))
 
     def fwd():
-        gdn.gdn_kda_chunk_fwd(**d, out=o, final_state=ht, workspace=ws)
+        gdn.gdn_kda_chunk_fwd(**d, initial_state=h0, out=o, final_state=ht, workspace=ws)
 
-    for _ in range(3):
+    def step():
         fwd()
-    torch.cuda.synchronize()
+        gdn.gdn_kda_chunk_bwd(**d, d_o=dO, workspace=ws, outs=outs)
+
     stream = torch.cuda.current_stream()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        fwd()
-    b.record(stream)
-    torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    ms_f, ms = timed(fwd), timed(step)
     gdn.profile(True)
-    fwd()
+    step()
     prof = gdn.profile_read()
     gdn.profile(False)
     units = (32768 // 64) * 32
     K = V = 128
     fma = {"kda_wy": 2 * 1536 * K + 2 * 544 * K + 64 * 64 * K + 64 * 64 * V,
            "kda_scan": 64 * V * K + V * K * 64, "kda_out": 64 * V * 64 + 64 * V * K}
-    flops = 2 * units * sum(fma.values())
-    tflops = flops / (ms / 1e3) / 1e12
     kern = {k: round(v[1], 4) for k, v in prof.items()}
     top = max(fma, key=lambda k: kern.get(k, 0.0))
     top_tf = 2 * units * fma[top] / (kern[top] / 1e3) / 1e12
-    return {"workload": "kda_chunk_fwd_B1_T32768_H16_HV32_D128_bf16", "ms": round(ms, 4),
-            "mtok_s": round(32768 / (ms / 1e3) / 1e6, 3), "kernels_ms": kern,
+    return {"workload": "kda_chunk_B1_T32768_H16_HV32_D128_bf16", "fwd_ms": round(ms_f, 4),
+            "fwd_mtok_s": round(32768 / (ms_f / 1e3) / 1e6, 3), "step_ms": round(ms, 4),
+            "step_mtok_s": round(32768 / (ms / 1e3) / 1e6, 3), "kernels_ms": kern,
             "roofline": {"kernel": top, "bound": "alu", "achieved": round(top_tf, 2),
                          "peak": round(FFMA_TFLOPS, 1), "unit": "TFLOP/s",
                          "frac": round(top_tf / FFMA_TFLOPS, 4),
-                         "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz (FFMA)"},
-            "forward_tflops": round(tflops, 2)}
+                         "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz (FFMA)"}}
 
 
 def kda_gate_measure(gdn, dev, pk_hbm: float, steps: int = 20) -> dict:

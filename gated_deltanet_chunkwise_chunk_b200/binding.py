@@ -27,7 +27,7 @@ EXPORTED = ("gdn_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_max_ch
             "gdn_profile_read", "gdn_chunk_fwd_noalloc", "gdn_noalloc_scratch_bytes",
             "gdn_recurrent_fwd", "gdn_recurrent_workspace_bytes", "gdn_kda_gate_fwd",
             "gdn_kda_gate_bwd", "gdn_kda_gate_workspace_bytes", "gdn_kda_recurrent_fwd",
-            "gdn_kda_chunk_fwd", "gdn_kda_chunk_workspace_bytes")
+            "gdn_kda_chunk_fwd", "gdn_kda_chunk_bwd", "gdn_kda_chunk_workspace_bytes")
 
 
 class gdn_dims(ctypes.Structure):
@@ -60,7 +60,9 @@ def _load() -> ctypes.CDLL:
     lib.gdn_recurrent_fwd.restype = I32
     lib.gdn_kda_chunk_fwd.argtypes = [D] + [P] * 12 + [SZ, P]
     lib.gdn_kda_chunk_fwd.restype = I32
-    lib.gdn_kda_chunk_workspace_bytes.argtypes = [D, I32]
+    lib.gdn_kda_chunk_bwd.argtypes = [D] + [P] * 20 + [SZ, P]
+    lib.gdn_kda_chunk_bwd.restype = I32
+    lib.gdn_kda_chunk_workspace_bytes.argtypes = [D, I32, I32]
     lib.gdn_kda_chunk_workspace_bytes.restype = SZ
     lib.gdn_kda_recurrent_fwd.argtypes = [D] + [P] * 12 + [SZ, P]
     lib.gdn_kda_recurrent_fwd.restype = I32
@@ -254,8 +256,8 @@ def gdn_kda_recurrent_fwd(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None,
     return o, ht
 
 
-def kda_chunk_workspace_bytes(dims: gdn_dims, varlen: bool) -> int:
-    return int(lib.gdn_kda_chunk_workspace_bytes(ctypes.byref(dims), int(varlen)))
+def kda_chunk_workspace_bytes(dims: gdn_dims, varlen: bool, backward: bool = False) -> int:
+    return int(lib.gdn_kda_chunk_workspace_bytes(ctypes.byref(dims), int(varlen), int(backward)))
 
 
 def gdn_kda_chunk_fwd(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None, initial_state=None,
@@ -285,6 +287,45 @@ def gdn_kda_chunk_fwd(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None, ini
     if rc != GDN_OK:
         raise GDNError("gdn_kda_chunk_fwd", rc)
     return o, ht
+
+
+def gdn_kda_chunk_bwd(q, k, v, g_raw, A_log, dt_bias, beta, d_o, workspace, cu_seqlens=None,
+                      dht=None, scale=0.0, want_dh0=True, want_param_grads=True, outs=None):
+    """Backward of gdn_kda_chunk_fwd.  `workspace` must be the one a gdn_kda_chunk_fwd call with
+    the same inputs used, sized with kda_chunk_workspace_bytes(dims, varlen, backward=True).
+    Returns a dict with dq, dk, dv, dbeta, dg (dL/dyg, [B,T,HV,K]) and, when asked, dh0,
+    dg_raw, dA_log, ddt_bias (None without dt_bias)."""
+    B, T, H, K = q.shape
+    HV, V = v.shape[2], v.shape[3]
+    Nst = _check_inputs(q, k, v, None, A_log, None, beta, cu_seqlens, None)
+    _check("g_raw", g_raw, torch.float32, (B, T, HV, K), q.device)
+    _check("dt_bias", dt_bias, torch.float32, (HV * K,), q.device)
+    _check("d_o", d_o, q.dtype, (B, T, HV, V), q.device)
+    _check("dht", dht, torch.float32, (Nst, HV, K, V), q.device)
+    dims = make_dims(q, v, cu_seqlens, scale)
+    need = kda_chunk_workspace_bytes(dims, cu_seqlens is not None, True)
+    if workspace.numel() < need:
+        raise ValueError(f"workspace holds {workspace.numel()} bytes, the backward needs {need}")
+    dev = q.device
+    if outs is None:
+        outs = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                    dbeta=torch.empty((B, T, HV), dtype=torch.float32, device=dev),
+                    dg=torch.empty((B, T, HV, K), dtype=torch.float32, device=dev))
+        if want_dh0:
+            outs["dh0"] = torch.empty((Nst, HV, K, V), dtype=torch.float32, device=dev)
+        if want_param_grads:
+            outs["dg_raw"] = torch.empty((B, T, HV, K), dtype=torch.float32, device=dev)
+            outs["dA_log"] = torch.empty(HV, dtype=torch.float32, device=dev)
+            outs["ddt_bias"] = (torch.empty(HV * K, dtype=torch.float32, device=dev)
+                                if dt_bias is not None else None)
+    g = lambda name: _ptr(outs.get(name))
+    rc = lib.gdn_kda_chunk_bwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g_raw), _ptr(A_log),
+                               _ptr(dt_bias), _ptr(beta), _ptr(cu_seqlens), _ptr(d_o), _ptr(dht),
+                               g("dq"), g("dk"), g("dv"), g("dg"), g("dbeta"), g("dh0"), g("dg_raw"),
+                               g("dA_log"), g("ddt_bias"), _ptr(workspace), workspace.numel(), _stream())
+    if rc != GDN_OK:
+        raise GDNError("gdn_kda_chunk_bwd", rc)
+    return outs
 
 
 _TORCH_DT = {torch.float32: GDN_DTYPE_FP32, torch.bfloat16: GDN_DTYPE_BF16,

@@ -148,10 +148,12 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA
 
 // Workspace of the chunkwise KDA forward.
 struct KdaPlan {
-  size_t status, seq_tab, chunk_tab, W, Ut, Kh, Qt, P, eGC, h, U, total;
+  size_t status, seq_tab, chunk_tab, W, Ut, Kh, Qt, P, eGC, h, U;
+  size_t Gam, Tm, dU, dh, dW, dGam, dqp, dkp, pgp;  // pass 1 only
+  size_t total;
 };
 
-KdaPlan make_kda_plan(const gdn_dims& d, bool varlen) {
+KdaPlan make_kda_plan(const gdn_dims& d, bool varlen, int pass) {
   KdaPlan pl{};
   const size_t NC = (size_t)max_chunks(d, varlen), Nst = varlen ? (size_t)d.N : (size_t)d.B;
   const size_t HV = d.HV, K = d.K, V = d.V, f = sizeof(float);
@@ -172,8 +174,46 @@ KdaPlan make_kda_plan(const gdn_dims& d, bool varlen) {
   pl.eGC = take(NC * HV * K * f);
   pl.h = take(NC * HV * V * K * f);
   pl.U = take(NC * HV * CH * V * f);
+  if (pass == 1) {
+    pl.Gam = take(NC * HV * CH * K * f);
+    pl.Tm = take(NC * HV * CH * CH * f);
+    pl.dU = take(NC * HV * CH * V * f);
+    pl.dh = take(NC * HV * V * K * f);
+    pl.dW = take(NC * HV * CH * K * f);
+    pl.dGam = take(NC * HV * CH * K * f);
+    pl.dqp = take(NC * HV * CH * K * f);
+    pl.dkp = take(NC * HV * CH * K * f);
+    pl.pgp = take(NC * HV * (K + 1) * f);
+  }
   pl.total = o;
   return pl;
+}
+
+KdaWork carve_kda(const KdaPlan& pl, void* ws) {
+  char* b = static_cast<char*>(ws);
+  KdaWork w{};
+  w.status = reinterpret_cast<int*>(b + pl.status);
+  w.seq_tab = reinterpret_cast<int4*>(b + pl.seq_tab);
+  w.chunk_tab = reinterpret_cast<int4*>(b + pl.chunk_tab);
+  auto fp = [&](size_t off) { return off ? reinterpret_cast<float*>(b + off) : nullptr; };
+  w.W = fp(pl.W);
+  w.Ut = fp(pl.Ut);
+  w.Kh = fp(pl.Kh);
+  w.Qt = fp(pl.Qt);
+  w.P = fp(pl.P);
+  w.eGC = fp(pl.eGC);
+  w.h = fp(pl.h);
+  w.U = fp(pl.U);
+  w.Gam = fp(pl.Gam);
+  w.Tm = fp(pl.Tm);
+  w.dU = fp(pl.dU);
+  w.dh = fp(pl.dh);
+  w.dW = fp(pl.dW);
+  w.dGam = fp(pl.dGam);
+  w.dqp = fp(pl.dqp);
+  w.dkp = fp(pl.dkp);
+  w.pgp = fp(pl.pgp);
+  return w;
 }
 
 // Steps shared by the forward and the backward: chunk table, gate + in-chunk cumsum.
@@ -405,9 +445,9 @@ int gdn_kda_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const
                           final_state, workspace, workspace_bytes, stream, true);
 }
 
-size_t gdn_kda_chunk_workspace_bytes(const gdn_dims* d, int varlen) {
-  if (check_dims(d, varlen != 0) != GDN_OK) return 0;
-  return make_kda_plan(*d, varlen != 0).total;
+size_t gdn_kda_chunk_workspace_bytes(const gdn_dims* d, int varlen, int pass) {
+  if (check_dims(d, varlen != 0) != GDN_OK || (pass != 0 && pass != 1)) return 0;
+  return make_kda_plan(*d, varlen != 0, pass).total;
 }
 
 int gdn_kda_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
@@ -424,9 +464,11 @@ int gdn_kda_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const voi
   if (!A_log || !aligned16(A_log) || !aligned16(dt_bias)) return GDN_ERR_INVALID_ARG;
   if (!aligned16(cu_seqlens) || !aligned16(initial_state) || !aligned16(final_state))
     return GDN_ERR_INVALID_ARG;
-  const KdaPlan pl = make_kda_plan(*d, varlen);
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) || workspace_bytes < pl.total)
+  const KdaPlan pl0 = make_kda_plan(*d, varlen, 0), pl1 = make_kda_plan(*d, varlen, 1);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) || workspace_bytes < pl0.total)
     return GDN_ERR_WORKSPACE;
+  // a workspace sized for the backward also keeps what the backward reads
+  const KdaPlan& pl = workspace_bytes >= pl1.total ? pl1 : pl0;
   const Problem p = make_problem(*d, varlen);
   Args a{};
   a.q = q;
@@ -440,20 +482,7 @@ int gdn_kda_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const voi
   a.h0 = initial_state;
   a.o = o;
   a.ht = final_state;
-  char* b = static_cast<char*>(workspace);
-  KdaWork w{};
-  w.status = reinterpret_cast<int*>(b + pl.status);
-  w.seq_tab = reinterpret_cast<int4*>(b + pl.seq_tab);
-  w.chunk_tab = reinterpret_cast<int4*>(b + pl.chunk_tab);
-  auto fp = [&](size_t off) { return reinterpret_cast<float*>(b + off); };
-  w.W = fp(pl.W);
-  w.Ut = fp(pl.Ut);
-  w.Kh = fp(pl.Kh);
-  w.Qt = fp(pl.Qt);
-  w.P = fp(pl.P);
-  w.eGC = fp(pl.eGC);
-  w.h = fp(pl.h);
-  w.U = fp(pl.U);
+  const KdaWork w = carve_kda(pl, workspace);
   Work cw{};  // the chunk table kernel's view of the same status word and tables
   cw.status = w.status;
   cw.seq_tab = w.seq_tab;
@@ -462,6 +491,51 @@ int gdn_kda_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const voi
   cudaError_t e = launch_chunk_table(p, cu_seqlens, cw, s);
   if (e == cudaSuccess) e = kda_chunk_forward(p, a, w, d->dtype == GDN_DTYPE_BF16, s);
   return cuda_status(e);
+}
+
+int gdn_kda_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                      const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,
+                      const int64_t* cu_seqlens, const void* d_o, const float* dht, void* dq, void* dk,
+                      void* dv, float* dg, float* dbeta, float* dh0, float* dg_raw, float* dA_log,
+                      float* ddt_bias, void* workspace, size_t workspace_bytes, void* stream) {
+  const bool varlen = cu_seqlens != nullptr;
+  int rc = check_dims(d, varlen);
+  if (rc) return rc;
+  const bool empty = d->B * d->T == 0;
+  const void* tok[] = {q, k, v, g_raw, beta, d_o, dq, dk, dv, dg, dbeta};
+  for (const void* x : tok)
+    if ((!x && !empty) || !aligned16(x)) return GDN_ERR_INVALID_ARG;
+  if (!A_log || !aligned16(A_log) || !aligned16(dt_bias)) return GDN_ERR_INVALID_ARG;
+  if (ddt_bias && !dt_bias) return GDN_ERR_INVALID_ARG;
+  const void* opt[] = {cu_seqlens, dht, dh0, dg_raw, dA_log, ddt_bias};
+  for (const void* x : opt)
+    if (!aligned16(x)) return GDN_ERR_INVALID_ARG;
+  const KdaPlan pl = make_kda_plan(*d, varlen, 1);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) || workspace_bytes < pl.total)
+    return GDN_ERR_WORKSPACE;
+  const Problem p = make_problem(*d, varlen);
+  Args a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.g_raw = g_raw;
+  a.A_log = A_log;
+  a.dt_bias = dt_bias;
+  a.beta = beta;
+  a.cu = cu_seqlens;
+  a.dO = d_o;
+  a.dht = dht;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dg = dg;
+  a.dbeta = dbeta;
+  a.dh0 = dh0;
+  a.dg_raw = dg_raw;
+  a.dA_log = dA_log;
+  a.ddt_bias = ddt_bias;
+  return cuda_status(kda_chunk_backward(p, a, carve_kda(pl, workspace), d->dtype == GDN_DTYPE_BF16,
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 static int kda_check(int64_t T, int64_t H, int64_t D, int32_t dt1, int32_t dt2) {

@@ -61,8 +61,18 @@ struct KdaWork {
   float* Qt;       // [NCmax][HV][64][K]   q e^{Gam}
   float* P;        // [NCmax][HV][64][64]  sum_c q_i k_j e^{Gam_i - Gam_j}, lower incl. diagonal
   float* eGC;      // [NCmax][HV][K]       e^{Gam_C}
-  float* h;        // [NCmax][HV][K][V]    state entering the chunk (h[k][v] = S[v][k])
+  float* h;        // [NCmax][HV][V][K]    state entering the chunk (S orientation)
   float* U;        // [NCmax][HV][64][V]   U~ - W S^T
+  // kept by a forward whose workspace is sized for the backward, and the backward's own
+  float* Gam;      // [NCmax][HV][64][K]   in-chunk cumsum of the log-decay, times log2(e)
+  float* Tm;       // [NCmax][HV][64][64]  (I + A)^-1
+  float* dU;       // [NCmax][HV][64][V]   dL/dU, then dY = T^T dU
+  float* dh;       // [NCmax][HV][V][K]    dL/dS leaving the chunk
+  float* dW;       // [NCmax][HV][64][K]   dL/dW, then dX = T^T dW
+  float* dGam;     // [NCmax][HV][64][K]   dL/dGam, then dL/dyg
+  float* dqp;      // [NCmax][HV][64][K]   per-value-head dq share
+  float* dkp;      // [NCmax][HV][64][K]   per-value-head dk share
+  float* pgp;      // [NCmax][HV][K+1]     per-chunk sums of dL/d dt_bias (K) and dL/dA_log (1)
 };
 
 // Pointers of one call (inputs and outputs as given by the caller).

@@ -93,7 +93,7 @@ size_t wy_smem(int K, int V) {
   return (size_t)(3 * CH * K + CH * V + CH * LDA + CH * CH + wy_scratch(K) + CH) * sizeof(float);
 }
 size_t scan_smem(int K) { return (size_t)(32 * (K + 1) + CH * (K + 1) + CH * K + CH * 32 + K) * sizeof(float); }
-size_t out_smem(int K, int V) { return (size_t)(CH * K + CH * CH + K * V + 2 * CH * V) * sizeof(float); }
+size_t out_smem(int K, int V) { return (size_t)(CH * K + CH * CH + K * (V + 1) + 2 * CH * V) * sizeof(float); }
 
 template <typename T>
 __global__ void __launch_bounds__(256) k_kda_wy(Problem p, Args a, KdaWork w) {
@@ -207,8 +207,12 @@ __global__ void __launch_bounds__(256) k_kda_wy(Problem p, Args a, KdaWork w) {
   const size_t u = (size_t)gc * p.HV + hv;
   float* gP = w.P + u * CH * CH;
   for (int x = tid; x < CH * CH; x += blockDim.x) gP[x] = sP[x];
+  if (w.Gam)
+    for (int x = tid; x < CH * K; x += blockDim.x) w.Gam[u * CH * K + x] = sG[x];
   float* sT = sX;
   tcx::unit_lower_inverse64(sA, sT, sX + CH * LDA, tid);  // T = (I + A)^-1 (ends with a barrier)
+  if (w.Tm)
+    for (int x = tid; x < CH * CH; x += blockDim.x) w.Tm[u * CH * CH + x] = sT[(x / CH) * LDA + x % CH];
   // K^ = k e^{Gam_C - Gam}, Q~ = q e^{Gam}, e^{Gam_C}; then beta e^{Gam} k in place for W
   const size_t uk = u * CH * K;
   for (int x = tid; x < CH * K; x += blockDim.x) {
@@ -226,7 +230,7 @@ __global__ void __launch_bounds__(256) k_kda_wy(Problem p, Args a, KdaWork w) {
 }
 
 // Sequential scan of one (sequence, value head, rows v0..v0+31 of S): stores the state entering
-// each chunk (h[k][v] orientation) and U = U~ - W S^T for those rows, returns the final state.
+// each chunk (rows v of S, [V][K]) and U = U~ - W S^T for those rows, returns the final state.
 // The next chunk's W, K^, U~ slice and e^{Gam_C} are loaded into registers while the current
 // chunk's products run.
 __global__ void __launch_bounds__(256) k_kda_scan(Problem p, Args a, KdaWork w) {
@@ -281,11 +285,8 @@ __global__ void __launch_bounds__(256) k_kda_scan(Problem p, Args a, KdaWork w) 
     const size_t u = (size_t)(sq.x + ci) * p.HV + hv;
     __syncthreads();  // the previous chunk is done with every buffer
     stash();
-    float* h = w.h + u * K * V;  // h[k][v] of the state entering the chunk
-    for (int x = tid; x < 32 * K; x += blockDim.x) {
-      const int vv = x % 32, c = x / 32;
-      h[(size_t)c * V + v0 + vv] = sS[vv * (K + 1) + c];
-    }
+    float* h = w.h + u * V * K + (size_t)v0 * K;  // rows v0.. of the state entering the chunk
+    for (int x = tid; x < 32 * K; x += blockDim.x) h[x] = sS[(x / K) * (K + 1) + x % K];
     __syncthreads();
     if (ci + 1 < sq.y) fetch(u + p.HV);
     mm(CH, 32, K, sU, 32, -1.f, true, sW, K + 1, 1, sS, 1, K + 1);  // U = U~ - W S^T
@@ -316,20 +317,30 @@ __global__ void __launch_bounds__(256) k_kda_out(Problem p, Args a, KdaWork w) {
   if (e.x < 0) return;
   const int K = p.K, V = p.V, L = e.z, tok0 = e.w;
   extern __shared__ float sm[];
-  float* sQt = sm;           // [64][K]
-  float* sP = sQt + CH * K;  // [64][64]
-  float* sH = sP + CH * CH;  // [K][V]  state entering the chunk, h[k][v]
-  float* sU = sH + K * V;    // [64][V]
-  float* sO = sU + CH * V;   // [64][V]
+  float* sQt = sm;                 // [64][K]
+  float* sP = sQt + CH * K;        // [64][64]
+  float* sH = sP + CH * CH;        // [K][V+1]  h[k][v] = S[v][k] of the state entering the chunk
+  float* sU = sH + K * (V + 1);    // [64][V]
+  float* sO = sU + CH * V;         // [64][V]
   const size_t u = (size_t)gc * p.HV + hv;
   copy_async(sQt, w.Qt + u * CH * K, CH * K);
   copy_async(sP, w.P + u * CH * CH, CH * CH);
-  copy_async(sH, w.h + u * K * V, K * V);
   copy_async(sU, w.U + u * CH * V, CH * V);
+  {  // S ([V][K] in memory) transposed into h[k][v]
+    const float4* S4 = reinterpret_cast<const float4*>(w.h + u * V * K);
+    for (int x = threadIdx.x; x < V * K / 4; x += blockDim.x) {
+      const float4 f = S4[x];
+      const int v = x / (K / 4), c = 4 * (x % (K / 4));
+      sH[c * (V + 1) + v] = f.x;
+      sH[(c + 1) * (V + 1) + v] = f.y;
+      sH[(c + 2) * (V + 1) + v] = f.z;
+      sH[(c + 3) * (V + 1) + v] = f.w;
+    }
+  }
   cp_async_wait_all();
   __syncthreads();
   mm(CH, V, CH, sO, V, 1.f, false, sP, CH, 1, sU, V, 1);
-  mm(CH, V, K, sO, V, 1.f, true, sQt, K, 1, sH, V, 1);
+  mm(CH, V, K, sO, V, 1.f, true, sQt, K, 1, sH, V + 1, 1);
   __syncthreads();
   T* o = static_cast<T*>(a.o) + ((size_t)tok0 * p.HV + hv) * V;
   for (int x = threadIdx.x; x < L * V; x += blockDim.x)

@@ -1,0 +1,447 @@
+// Chunkwise backward of the KDA delta rule (a decay per key channel), fp32 on CUDA cores, for
+// L = sum(dO * o) + sum(dht * h_final).  It reads the intermediates a forward kept in the same
+// workspace (W, K^, Q~, P, e^{Gam_C}, the entering states S, U, Gam, T).  Per 64-token chunk,
+// with dS' = dL/dS leaving the chunk, X = diag(beta) (k e^{Gam}), Y = diag(beta) V:
+//   dU = scale P^T dO + K^ dS'^T,            dS = dS' Diag(e^{Gam_C}) + scale dO^T Q~ - dU^T W
+//   dQ~ = scale dO S,  dP = scale dO U^T (lower incl. diagonal),  dK^ = U dS',  dW = -dU S
+//   dT = dW X^T + dU Y^T,  dX = T^T dW,  dY = T^T dU,  dA = -T^T dT T^T (strictly lower)
+//   dv = beta dY,  dbeta = rowsum(dY * V) + rowsum(dX * k e^{Gam}) + rowsum(k * F1)
+//   dq = dQ~ e^{Gam} + F2,   dk = dK^ e^{Gam_C - Gam} + beta dX e^{Gam} + G2 + beta F1 + G1
+//   dGam = dQ~ Q~ - dK^ K^ + beta dX (k e^{Gam}) + q F2 - k G2 + beta k F1 - k G1,
+//   dGam_C += colsum(dK^ K^) + e^{Gam_C} colsum(dS' * S)
+// where F_i = sum_{j<=i} Wt_ij R_j e^{Gam_i - Gam_j} and G_j = sum_{i>=j} Wt_ij L_i e^{Gam_i - Gam_j}
+// are per-channel gated products (F2, G2: Wt = dP, R = k, L = q; F1: Wt = dA, R = k; G1: Wt =
+// diag(beta) dA, L = k), taken in 16-token sub-chunks as in the forward.  dyg is the reverse
+// in-chunk cumsum of dGam; the KDA gate's chain gives dg_raw, dA_log and ddt_bias.
+//
+// Kernels: k_kda_bwd_scan (sequence, value head, 32-row slice of S; reverse over the chunks),
+// k_kda_bwd_dqk and k_kda_bwd_wy per (chunk, value head), then the group sum of the dq/dk
+// shares and a fixed-order sum of the gate-parameter gradients.
+#include <type_traits>
+
+#include "ffma_tiles.cuh"
+#include "gdn_common.cuh"
+#include "gdn_launch.h"
+#include "gdn_tc_common.cuh"  // LDA
+
+namespace gdn {
+namespace {
+
+constexpr int SUB = 16;
+constexpr int LDP = CH + 1;  // row stride of the 64 x 64 gradient matrices
+using tcx::LDA;
+
+__device__ __forceinline__ bool kda_failed(const KdaWork& w) { return *((volatile int*)w.status) != 0; }
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
+__device__ __forceinline__ void copy_async(float* dst, const float* src, int n) {
+  for (int i = threadIdx.x; i < n / 4; i += blockDim.x) cp_async16(dst + 4 * i, src + 4 * i);
+}
+
+// Rows [0, L) of a 64 x D token tile (row stride rs) into fp32 shared memory with row stride
+// ldd, rows past L zero.
+template <typename T>
+__device__ __forceinline__ void load_tok(float* dst, int ldd, const T* src, size_t rs, int L, int D) {
+  for (int x = threadIdx.x; x < CH * D; x += blockDim.x) {
+    const int t = x / D, c = x % D;
+    dst[t * ldd + c] = t < L ? to_f<T>(src[(size_t)t * rs + c]) : 0.f;
+  }
+}
+
+// Per-channel gated products of a 64 x 64 weight Wt (lower triangle used, ldw) with row
+// operand R and column operand Lm ([64][K], row stride K), Gam2 = Gam * log2(e) ([64][K]):
+//   F_i = sum_{j<=i} Wt_ij R_j e^{Gam_i - Gam_j},   G_j = sum_{i>=j} colw_i Wt_ij Lm_i e^{Gam_i - Gam_j}
+// (colw = per-row weights of the column product, or null).  Each result element is handed to
+// sink(i, c, F) / sinkG(j, c, G) once per phase; phases are separated by barriers.
+// scratch: [64][K] floats.  Ends with a barrier.
+template <typename SinkF, typename SinkG>
+__device__ void gated_products(const float* Wt, int ldw, const float* R, const float* Lm,
+                               const float* colw, const float* G2, int K, float* scratch,
+                               SinkF sinkF, SinkG sinkG) {
+  const int tid = threadIdx.x;
+  // diagonal sub-blocks, one (row, channel) per thread
+  for (int x = tid; x < CH * K; x += blockDim.x) {
+    const int i = x / K, c = x % K, b0 = (i / SUB) * SUB;
+    const float gi = G2[x];
+    float f = 0.f, g = 0.f;
+    for (int j = b0; j <= i; ++j) f += Wt[i * ldw + j] * R[j * K + c] * exp2f(gi - G2[j * K + c]);
+    for (int r = i; r < b0 + SUB; ++r) {  // this row as the column index j = i
+      const float wr = Wt[r * ldw + i] * (colw ? colw[r] : 1.f);
+      g += wr * Lm[r * K + c] * exp2f(G2[r * K + c] - gi);
+    }
+    sinkF(i, c, f);
+    sinkG(i, c, g);
+  }
+  __syncthreads();
+  float* RT = scratch;                 // [48][K]: R_j e^{Gam_r - Gam_j}, j < 16 a
+  float* Ls = scratch + 3 * SUB * K;   // [16][K]: colw_i Lm_i e^{Gam_i - Gam_r}, i in sub-chunk a
+  for (int a = 1; a < CH / SUB; ++a) {
+    const int r = a * SUB - 1, nj = a * SUB;
+    for (int x = tid; x < nj * K; x += blockDim.x) {
+      const int c = x % K;
+      RT[x] = R[x] * exp2f(G2[r * K + c] - G2[x]);
+    }
+    for (int x = tid; x < SUB * K; x += blockDim.x) {
+      const int i = a * SUB + x / K, c = x % K;
+      Ls[x] = (colw ? colw[i] : 1.f) * Lm[i * K + c] * exp2f(G2[i * K + c] - G2[r * K + c]);
+    }
+    __syncthreads();
+    for (int x = tid; x < SUB * K; x += blockDim.x) {  // rows i of sub-chunk a
+      const int i = a * SUB + x / K, c = x % K;
+      float acc = 0.f;
+      for (int j = 0; j < nj; ++j) acc += Wt[i * ldw + j] * RT[j * K + c];
+      sinkF(i, c, acc * exp2f(G2[i * K + c] - G2[r * K + c]));
+    }
+    for (int x = tid; x < nj * K; x += blockDim.x) {  // columns j before sub-chunk a
+      const int j = x / K, c = x % K;
+      float acc = 0.f;
+      for (int ii = 0; ii < SUB; ++ii) acc += Wt[(a * SUB + ii) * ldw + j] * Ls[ii * K + c];
+      sinkG(j, c, acc * exp2f(G2[r * K + c] - G2[j * K + c]));
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------- reverse state scan
+template <typename T>
+__global__ void __launch_bounds__(256) k_kda_bwd_scan(Problem p, Args a, KdaWork w) {
+  if (kda_failed(w)) return;
+  const int n = blockIdx.x, hv = blockIdx.y, v0 = 32 * blockIdx.z, K = p.K, V = p.V, tid = threadIdx.x;
+  const int4 sq = w.seq_tab[n];
+  extern __shared__ float sm[];
+  float* sdS = sm;                 // [32][K+1]  rows v0.. of dS
+  float* sP = sdS + 32 * (K + 1);  // [64][64]
+  float* sKh = sP + CH * CH;       // [64][K]
+  float* sQt = sKh + CH * K;       // [64][K]
+  float* sW = sQt + CH * K;        // [64][K]
+  float* sdO = sW + CH * K;        // [64][32]
+  float* sdU = sdO + CH * 32;      // [64][32]
+  float* sE = sdU + CH * 32;       // [K]
+  for (int x = tid; x < 32 * K; x += blockDim.x) {
+    const int vv = x % 32, c = x / 32;
+    sdS[vv * (K + 1) + c] = a.dht ? a.dht[(((size_t)n * p.HV + hv) * K + c) * V + v0 + vv] : 0.f;
+  }
+  const T* dO = static_cast<const T*>(a.dO);
+  for (int ci = sq.y - 1; ci >= 0; --ci) {
+    const int gc = sq.x + ci;
+    const int4 e = w.chunk_tab[gc];
+    const size_t u = (size_t)gc * p.HV + hv;
+    __syncthreads();  // the previous chunk is done with every buffer
+    copy_async(sP, w.P + u * CH * CH, CH * CH);
+    copy_async(sKh, w.Kh + u * CH * K, CH * K);
+    copy_async(sQt, w.Qt + u * CH * K, CH * K);
+    copy_async(sW, w.W + u * CH * K, CH * K);
+    copy_async(sE, w.eGC + u * K, K);
+    for (int x = tid; x < CH * 32; x += blockDim.x) {
+      const int i = x / 32, vv = x % 32;
+      sdO[x] = i < e.z ? to_f<T>(dO[((size_t)(e.w + i) * p.HV + hv) * V + v0 + vv]) : 0.f;
+    }
+    float* dh = w.dh + u * V * K + (size_t)v0 * K;  // dS' (leaving the chunk), rows v0..
+    for (int x = tid; x < 32 * K; x += blockDim.x) dh[x] = sdS[(x / K) * (K + 1) + x % K];
+    cp_async_wait_all();
+    __syncthreads();
+    mm(CH, 32, CH, sdU, 32, p.scale, false, sP, 1, CH, sdO, 32, 1);   // scale P^T dO
+    mm(CH, 32, K, sdU, 32, 1.f, true, sKh, K, 1, sdS, 1, K + 1);      // + K^ dS'^T
+    __syncthreads();
+    float* dU = w.dU + u * CH * V;
+    for (int x = tid; x < CH * 32; x += blockDim.x) dU[(x / 32) * V + v0 + x % 32] = sdU[x];
+    for (int x = tid; x < 32 * K; x += blockDim.x) sdS[(x / K) * (K + 1) + x % K] *= sE[x % K];
+    __syncthreads();
+    mm(32, K, CH, sdS, K + 1, p.scale, true, sdO, 1, 32, sQt, K, 1);  // + scale dO^T Q~
+    mm(32, K, CH, sdS, K + 1, -1.f, true, sdU, 1, 32, sW, K, 1);      // - dU^T W
+  }
+  __syncthreads();
+  if (a.dh0)
+    for (int x = tid; x < 32 * K; x += blockDim.x) {
+      const int vv = x % 32, c = x / 32;
+      a.dh0[(((size_t)n * p.HV + hv) * K + c) * V + v0 + vv] = sdS[vv * (K + 1) + c];
+    }
+}
+
+// ---------------------------------------------------------------- output-side terms
+// dP, dK^ (with the Gam_C column terms), dQ~, dW = -dU S, and the dP gated products.
+// Writes the unit's dq and dk shares, dGam and dW.
+template <typename T>
+__global__ void __launch_bounds__(256) k_kda_bwd_dqk(Problem p, Args a, KdaWork w) {
+  if (kda_failed(w)) return;
+  const int gc = blockIdx.x, hv = blockIdx.y;
+  const int4 e = w.chunk_tab[gc];
+  if (e.x < 0) return;
+  const int K = p.K, V = p.V, L = e.z, tok0 = e.w, hk = hv / p.G, tid = threadIdx.x;
+  extern __shared__ float sm[];
+  float* sQ = sm;                  // [64][K]
+  float* sK = sQ + CH * K;         // [64][K]
+  float* sG = sK + CH * K;         // [64][K]  Gam * log2(e)
+  float* sR1 = sG + CH * K;        // [64][max(V, K)]  dO, then scratch of the gated products
+  float* sR2 = sR1 + CH * (V > K ? V : K);  // [64][V+1]  U, then dU
+  float* sdP = sR2 + CH * (V + 1); // [64][65]
+  float* sGC = sdP + CH * LDP;     // [K]  dL/dGam_C
+  const size_t u = (size_t)gc * p.HV + hv, uk = u * CH * K;
+  const size_t rs = (size_t)p.H * K;
+  load_tok<T>(sQ, K, static_cast<const T*>(a.q) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
+  load_tok<T>(sK, K, static_cast<const T*>(a.k) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
+  load_tok<T>(sR1, V, static_cast<const T*>(a.dO) + ((size_t)tok0 * p.HV + hv) * V, (size_t)p.HV * V, L, V);
+  copy_async(sG, w.Gam + uk, CH * K);
+  for (int x = tid; x < CH * V; x += blockDim.x) sR2[(x / V) * (V + 1) + x % V] = w.U[u * CH * V + x];
+  cp_async_wait_all();
+  __syncthreads();
+  const float* S = w.h + u * V * K;    // [V][K]
+  const float* dSn = w.dh + u * V * K; // [V][K]
+  float* dqp = w.dqp + uk;
+  float* dkp = w.dkp + uk;
+  float* dG = w.dGam + uk;
+  // dP = scale dO U^T, lower triangle incl. diagonal
+  mm(CH, CH, V, sdP, LDP, p.scale, false, sR1, V, 1, sR2, 1, V + 1);
+  // dK^ = U dS' (raw, into the dk share)
+  mm(CH, K, V, dkp, K, 1.f, false, sR2, V + 1, 1, dSn, K, 1);
+  // dQ~ = scale dO S (raw, into the dq share)
+  mm(CH, K, V, dqp, K, p.scale, false, sR1, V, 1, S, K, 1);
+  __syncthreads();
+  for (int x = tid; x < CH * CH; x += blockDim.x)
+    if (x % CH > x / CH) sdP[(x / CH) * LDP + x % CH] = 0.f;
+  for (int c = tid; c < K; c += blockDim.x) {  // dL/dGam_C
+    const float gC = sG[(CH - 1) * K + c];
+    float s = 0.f;
+    for (int i = 0; i < CH; ++i) s += dkp[i * K + c] * sK[i * K + c] * exp2f(gC - sG[i * K + c]);
+    float t = 0.f;
+    for (int v = 0; v < V; ++v) t += dSn[(size_t)v * K + c] * S[(size_t)v * K + c];
+    sGC[c] = s + exp2f(gC) * t;
+  }
+  __syncthreads();
+  for (int x = tid; x < CH * K; x += blockDim.x) {
+    const int i = x / K, c = x % K;
+    const float g = sG[x], eg = exp2f(g), kh = exp2f(sG[(CH - 1) * K + c] - g);
+    const float dkh = dkp[x], dqt = dqp[x];
+    dkp[x] = dkh * kh;
+    dqp[x] = dqt * eg;
+    dG[x] = dqt * sQ[x] * eg - dkh * sK[x] * kh + (i == CH - 1 ? sGC[c] : 0.f);
+  }
+  // dW = -dU S
+  for (int x = tid; x < CH * V; x += blockDim.x) sR2[(x / V) * (V + 1) + x % V] = w.dU[u * CH * V + x];
+  __syncthreads();
+  mm(CH, K, V, w.dW + uk, K, -1.f, false, sR2, V + 1, 1, S, K, 1);
+  // P_ij = sum_c q_i k_j e^{Gam_i - Gam_j}: dq += F2, dk += G2, dGam += q F2 - k G2
+  gated_products(sdP, LDP, sK, sQ, nullptr, sG, K, sR1,
+                 [&](int i, int c, float f) {
+                   dqp[i * K + c] += f;
+                   dG[i * K + c] += sQ[i * K + c] * f;
+                 },
+                 [&](int j, int c, float g) {
+                   dkp[j * K + c] += g;
+                   dG[j * K + c] -= sK[j * K + c] * g;
+                 });
+}
+
+// ---------------------------------------------------------------- WY backward, gate chain
+template <typename T>
+__global__ void __launch_bounds__(256) k_kda_bwd_wy(Problem p, Args a, KdaWork w) {
+  if (kda_failed(w)) return;
+  const int gc = blockIdx.x, hv = blockIdx.y;
+  const int4 e = w.chunk_tab[gc];
+  if (e.x < 0) return;
+  const int K = p.K, V = p.V, L = e.z, tok0 = e.w, hk = hv / p.G, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
+  const int big = (V > K ? V : K) * CH > CH * LDP ? (V > K ? V : K) * CH : CH * LDP;
+  extern __shared__ float sm[];
+  float* sK = sm;                  // [64][K]
+  float* sG = sK + CH * K;         // [64][K]
+  float* sX = sG + CH * K;         // [64][K+1]  beta k e^{Gam}, then F1
+  float* sY = sX + CH * (K + 1);   // [64][V+1]  beta V
+  float* sdW = sY + CH * (V + 1);  // [big]  dW [64][K], then Z [64][65]
+  float* sdU = sdW + big;          // [big]  dU [64][V], then scratch, then g_raw [64][K]
+  float* sT = sdU + big;           // [64][LDA]
+  float* sdT = sT + CH * LDA;      // [64][65]  dT, then dA
+  float* sb = sdT + CH * LDP;      // [64]
+  float* sdb = sb + CH;            // [64]
+  const size_t u = (size_t)gc * p.HV + hv, uk = u * CH * K;
+  const size_t rs = (size_t)p.H * K;
+  load_tok<T>(sK, K, static_cast<const T*>(a.k) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
+  load_tok<T>(sY, V + 1, static_cast<const T*>(a.v) + ((size_t)tok0 * p.HV + hv) * V, (size_t)p.HV * V, L, V);
+  copy_async(sG, w.Gam + uk, CH * K);
+  copy_async(sdW, w.dW + uk, CH * K);
+  copy_async(sdU, w.dU + u * CH * V, CH * V);
+  if (tid < CH) sb[tid] = tid < L ? a.beta[(size_t)(tok0 + tid) * p.HV + hv] : 0.f;
+  for (int x = tid; x < CH * CH; x += blockDim.x)
+    sT[(x / CH) * LDA + x % CH] = w.Tm[u * CH * CH + x];
+  cp_async_wait_all();
+  __syncthreads();
+  for (int x = tid; x < CH * K; x += blockDim.x) {
+    const int i = x / K, c = x % K;
+    sX[i * (K + 1) + c] = sb[i] * sK[x] * exp2f(sG[x]);
+  }
+  for (int x = tid; x < CH * V; x += blockDim.x) sY[(x / V) * (V + 1) + x % V] *= sb[x / V];
+  __syncthreads();
+  // dT = dW X^T + dU Y^T
+  mm(CH, CH, K, sdT, LDP, 1.f, false, sdW, K, 1, sX, 1, K + 1);
+  mm(CH, CH, V, sdT, LDP, 1.f, true, sdU, V, 1, sY, 1, V + 1);
+  // dX = T^T dW, dY = T^T dU (into the global dW and dU of this unit)
+  float* dX = w.dW + uk;
+  float* dY = w.dU + u * CH * V;
+  mm(CH, K, CH, dX, K, 1.f, false, sT, 1, LDA, sdW, K, 1);
+  mm(CH, V, CH, dY, V, 1.f, false, sT, 1, LDA, sdU, V, 1);
+  __syncthreads();
+  float* dkp = w.dkp + uk;
+  float* dG = w.dGam + uk;
+  // dv = beta dY; dbeta = rowsum(dY V) + rowsum(dX k e^{Gam}); dk += beta dX e^{Gam}
+  T* dv = static_cast<T*>(a.dv);
+  const T* vin = static_cast<const T*>(a.v);
+  for (int i = warp; i < CH; i += nwarp) {
+    float s = 0.f;
+    for (int v = lane; v < V; v += 32) {
+      const float y = dY[i * V + v];
+      if (i < L) {
+        const size_t o = ((size_t)(tok0 + i) * p.HV + hv) * V + v;
+        s += y * to_f<T>(vin[o]);
+        dv[o] = from_f<T>(sb[i] * y);
+      }
+    }
+    for (int c = lane; c < K; c += 32) {
+      const float eg = exp2f(sG[i * K + c]), dx = dX[i * K + c], kt = sK[i * K + c] * eg;
+      s += dx * kt;
+      dkp[i * K + c] += sb[i] * dx * eg;
+      dG[i * K + c] += sb[i] * dx * kt;
+    }
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) sdb[i] = s;
+  }
+  // dA = -T^T (dT T^T), strictly lower
+  float* sZ = sdW;
+  mm(CH, CH, CH, sZ, LDP, 1.f, false, sdT, LDP, 1, sT, 1, LDA);
+  __syncthreads();
+  mm(CH, CH, CH, sdT, LDP, -1.f, false, sT, 1, LDA, sZ, LDP, 1);
+  __syncthreads();
+  for (int x = tid; x < CH * CH; x += blockDim.x)
+    if (x % CH >= x / CH) sdT[(x / CH) * LDP + x % CH] = 0.f;
+  for (int x = tid; x < CH * (K + 1); x += blockDim.x) sX[x] = 0.f;  // F1 accumulator
+  __syncthreads();
+  // A_ij = beta_i sum_c k_i k_j e^{Gam_i - Gam_j}: F1 (rows, weights dA), G1 (columns, beta_i dA)
+  gated_products(sdT, LDP, sK, sK, sb, sG, K, sdU,
+                 [&](int i, int c, float f) { sX[i * (K + 1) + c] += f; },
+                 [&](int j, int c, float g) {
+                   dkp[j * K + c] += g;
+                   dG[j * K + c] -= sK[j * K + c] * g;
+                 });
+  // F1 terms: dk += beta F1, dGam += beta k F1, dbeta += rowsum(k F1)
+  for (int i = warp; i < CH; i += nwarp) {
+    float s = 0.f;
+    for (int c = lane; c < K; c += 32) {
+      const float f = sX[i * (K + 1) + c], kk = sK[i * K + c];
+      s += kk * f;
+      dkp[i * K + c] += sb[i] * f;
+      dG[i * K + c] += sb[i] * kk * f;
+    }
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0 && i < L) a.dbeta[(size_t)(tok0 + i) * p.HV + hv] = sdb[i] + s;
+  }
+  // the raw gate inputs of this unit, for the gate chain
+  float* sg = sdU;
+  for (int x = tid; x < CH * K; x += blockDim.x) {
+    const int i = x / K;
+    sg[x] = i < L ? a.g_raw[((size_t)(tok0 + i) * p.HV + hv) * K + x % K] : 0.f;
+  }
+  __syncthreads();
+  // dyg = reverse in-chunk cumsum of dGam; gate chain; per-chunk parameter sums
+  const float nexp = -expf(a.A_log[hv]);
+  float* pg = w.pgp + u * (K + 1);
+  float pA = 0.f;
+  for (int c = tid; c < K; c += blockDim.x) {
+    const float bias = a.dt_bias ? a.dt_bias[(size_t)hv * K + c] : 0.f;
+    float acc = 0.f, pB = 0.f;
+    for (int i = CH - 1; i >= 0; --i) {
+      acc += dG[i * K + c];
+      if (i < L) {
+        const size_t o = ((size_t)(tok0 + i) * p.HV + hv) * K + c;
+        const float x = sg[i * K + c] + bias;
+        const float sp = x > 20.f ? x : log1pf(expf(x));
+        const float sig = x > 20.f ? 1.f : 1.f / (1.f + expf(-x));
+        const float dgr = acc * nexp * sig;
+        a.dg[o] = acc;
+        if (a.dg_raw) a.dg_raw[o] = dgr;
+        pA += acc * nexp * sp;
+        pB += dgr;
+      }
+    }
+    pg[c] = pB;
+  }
+  for (int off = 16; off > 0; off >>= 1) pA += __shfl_xor_sync(0xffffffffu, pA, off);
+  __syncthreads();
+  if (lane == 0) sdb[warp] = pA;
+  __syncthreads();
+  if (tid == 0) {
+    float s = 0.f;
+    for (int q = 0; q < nwarp; ++q) s += sdb[q];
+    pg[K] = s;
+  }
+}
+
+// dA_log[hv] and ddt_bias[hv*K + c]: the per-chunk sums added in chunk order.
+__global__ void __launch_bounds__(256) k_kda_param_grads(Problem p, Args a, KdaWork w) {
+  if (kda_failed(w)) return;
+  const int hv = blockIdx.x, K = p.K;
+  for (int c = threadIdx.x; c <= K; c += blockDim.x) {
+    float s = 0.f;
+    for (int gc = 0; gc < p.NCmax; ++gc) {
+      if (w.chunk_tab[gc].x < 0) break;
+      s += w.pgp[((size_t)gc * p.HV + hv) * (K + 1) + c];
+    }
+    if (c < K && a.ddt_bias) a.ddt_bias[(size_t)hv * K + c] = s;
+    if (c == K && a.dA_log) a.dA_log[hv] = s;
+  }
+}
+
+size_t scan_smem(int K) { return (size_t)(32 * (K + 1) + CH * CH + 3 * CH * K + 2 * CH * 32 + K) * sizeof(float); }
+size_t dqk_smem(int K, int V) {
+  return (size_t)(3 * CH * K + CH * (V > K ? V : K) + CH * (V + 1) + CH * LDP + K) * sizeof(float);
+}
+size_t wy_smem(int K, int V) {
+  const int big = (V > K ? V : K) * CH > CH * LDP ? (V > K ? V : K) * CH : CH * LDP;
+  return (size_t)(2 * CH * K + CH * (K + 1) + CH * (V + 1) + 2 * big + CH * LDA + CH * LDP + 2 * CH) *
+         sizeof(float);
+}
+
+template <typename Kern>
+cudaError_t go(const char* name, Kern kern, dim3 grid, size_t smem, cudaStream_t s, const Problem& p,
+               const Args& a, const KdaWork& w) {
+  if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  ProfScope ps(name, s);
+  kern<<<grid, 256, smem, s>>>(p, a, w);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t backward_t(const Problem& p, const Args& a, const KdaWork& w, cudaStream_t s) {
+  cudaError_t e = go("kda_bwd_scan", k_kda_bwd_scan<T>, dim3(p.Nst, p.HV, p.V / 32), scan_smem(p.K), s, p, a, w);
+  if (e == cudaSuccess)
+    e = go("kda_bwd_dqk", k_kda_bwd_dqk<T>, dim3(p.NCmax, p.HV), dqk_smem(p.K, p.V), s, p, a, w);
+  if (e == cudaSuccess)
+    e = go("kda_bwd_wy", k_kda_bwd_wy<T>, dim3(p.NCmax, p.HV), wy_smem(p.K, p.V), s, p, a, w);
+  if (e != cudaSuccess) return e;
+  Work gw{};  // the group sum's view of the shares
+  gw.status = w.status;
+  gw.chunk_tab = w.chunk_tab;
+  gw.dqp = w.dqp;
+  gw.dkp = w.dkp;
+  e = launch_dqdk_group_sum(p, a, gw, std::is_same<T, __nv_bfloat16>::value, s);
+  if (e == cudaSuccess && (a.dA_log || a.ddt_bias)) {  // zeros when there are no chunks
+    ProfScope ps("kda_param_grads", s);
+    k_kda_param_grads<<<p.HV, 256, 0, s>>>(p, a, w);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace
+
+cudaError_t kda_chunk_backward(const Problem& p, const Args& a, const KdaWork& w, bool bf16, cudaStream_t s) {
+  return bf16 ? backward_t<__nv_bfloat16>(p, a, w, s) : backward_t<float>(p, a, w, s);
+}
+
+}  // namespace gdn

@@ -333,17 +333,20 @@ cudaError_t launch_bwd_tokens(const Problem& p, const Args& a, const Work& w, bo
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  {
-    ProfScope ps("dqdk_group_sum", s);
-    const dim3 g(p.NCmax, p.H);
-    if (bf16)
-      k_dqdk_group_sum<__nv_bfloat16><<<g, 256, 0, s>>>(p, a, w);
-    else
-      k_dqdk_group_sum<float><<<g, 256, 0, s>>>(p, a, w);
-  }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_dqdk_group_sum(p, a, w, bf16, s)) != cudaSuccess) return e;
   if (a.dA_log || a.ddt_bias) e = launch_param_grads(p, a, w, s);
   return e;
+}
+
+cudaError_t launch_dqdk_group_sum(const Problem& p, const Args& a, const Work& w, bool bf16, cudaStream_t s) {
+  if (p.NCmax == 0) return cudaSuccess;
+  ProfScope ps("dqdk_group_sum", s);
+  const dim3 g(p.NCmax, p.H);
+  if (bf16)
+    k_dqdk_group_sum<__nv_bfloat16><<<g, 256, 0, s>>>(p, a, w);
+  else
+    k_dqdk_group_sum<float><<<g, 256, 0, s>>>(p, a, w);
+  return cudaGetLastError();
 }
 
 }  // namespace gdn

@@ -205,16 +205,33 @@ int gdn_kda_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const
  * arithmetic on CUDA cores.  Arguments, layouts and results as gdn_kda_recurrent_fwd
  * (g_raw [B,T,HV,K] fp32, dt_bias [HV*K] or NULL; o for every token, final_state after each
  * sequence's last token; final_state may be NULL).  workspace: at least
- * gdn_kda_chunk_workspace_bytes(d, varlen) bytes, 256-byte aligned; it also holds the device
- * status word (gdn_device_status: GDN_ERR_INVALID_ARG for invalid cu_seqlens).  Same size
- * limits and error returns as gdn_chunk_fwd. */
+ * gdn_kda_chunk_workspace_bytes(d, varlen, 0) bytes, 256-byte aligned; it also holds the device
+ * status word (gdn_device_status: GDN_ERR_INVALID_ARG for invalid cu_seqlens).  Given at least
+ * gdn_kda_chunk_workspace_bytes(d, varlen, 1) bytes, the forward also keeps in it what
+ * gdn_kda_chunk_bwd reads.  Same size limits and error returns as gdn_chunk_fwd. */
 int gdn_kda_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const void* v,
                       const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,
                       const int64_t* cu_seqlens, const float* initial_state, void* o,
                       float* final_state, void* workspace, size_t workspace_bytes, void* stream);
 
-/* Workspace bytes of gdn_kda_chunk_fwd (0 for invalid dimensions). */
-size_t gdn_kda_chunk_workspace_bytes(const gdn_dims* d, int varlen);
+/* Backward of gdn_kda_chunk_fwd for L = sum(d_o * o) + sum(dht * final_state): reads the
+ * intermediates a gdn_kda_chunk_fwd call with the same inputs left in `workspace` (which must
+ * then be at least gdn_kda_chunk_workspace_bytes(d, varlen, 1) bytes; the forward's status
+ * word is honoured), and writes
+ *   dq, dk [B,T,H,K] and dv [B,T,HV,V] (input dtype), dbeta [B,T,HV] fp32,
+ *   dg [B,T,HV,K] fp32 = dL/dyg (the per-channel log-decay),
+ *   dg_raw [B,T,HV,K] fp32 (may be NULL), dh0 [Nst,HV,K,V] fp32 (may be NULL),
+ *   dA_log [HV] fp32 (may be NULL), ddt_bias [HV*K] fp32 (may be NULL; needs dt_bias).
+ * dht may be NULL (zero).  The parameter sums are deterministic (fixed chunk order). */
+int gdn_kda_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v,
+                      const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,
+                      const int64_t* cu_seqlens, const void* d_o, const float* dht, void* dq, void* dk,
+                      void* dv, float* dg, float* dbeta, float* dh0, float* dg_raw, float* dA_log,
+                      float* ddt_bias, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of gdn_kda_chunk_fwd (pass 0) or of a forward + backward pair (pass 1); 0 for
+ * invalid dimensions. */
+size_t gdn_kda_chunk_workspace_bytes(const gdn_dims* d, int varlen, int pass);
 
 /* Workspace bytes of gdn_kda_gate_bwd (0 for invalid sizes). */
 size_t gdn_kda_gate_workspace_bytes(int64_t T, int64_t H, int64_t D);
