@@ -42,50 +42,6 @@ __device__ __forceinline__ float warp_total(float x) {
   return x;
 }
 
-// 16-byte global -> shared copies (cp.async), all in flight until cp_async_wait_all.
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
-}
-// n floats (n % 4 == 0, both ends 16-byte aligned), issued by every thread, not waited for
-__device__ __forceinline__ void copy_async(float* dst, const float* src, int n) {
-  for (int i = threadIdx.x; i < n / 4; i += blockDim.x) cp_async16(dst + 4 * i, src + 4 * i);
-}
-
-// Rows [0, L) of a 64 x D token tile (row stride rs elements, D % 8 == 0) into fp32 shared
-// memory, rows past L zero: 16-byte loads, all of a thread's loads issued before any is used.
-template <typename T>
-__device__ __forceinline__ void load_tile(float* dst, const T* src, size_t rs, int L, int D) {
-  constexpr int E = 16 / sizeof(T);       // elements per 16-byte vector
-  constexpr int NV = CH * 128 / E / 256;  // vectors per thread at D = 128
-  const int nvec = CH * D / E;
-  uint4 r[NV];
-#pragma unroll
-  for (int k = 0; k < NV; ++k) {
-    const int vi = threadIdx.x + 256 * k, t = vi * E / D, c = vi * E % D;
-    r[k] = make_uint4(0u, 0u, 0u, 0u);
-    if (vi < nvec && t < L) r[k] = __ldg(reinterpret_cast<const uint4*>(src + (size_t)t * rs + c));
-  }
-#pragma unroll
-  for (int k = 0; k < NV; ++k) {
-    const int vi = threadIdx.x + 256 * k;
-    if (vi >= nvec) continue;
-    float* d = dst + vi * E;
-    if constexpr (E == 4) {
-      *reinterpret_cast<uint4*>(d) = r[k];
-    } else {
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&r[k]);
-      const float2 f0 = __bfloat1622float2(h2[0]), f1 = __bfloat1622float2(h2[1]);
-      const float2 f2 = __bfloat1622float2(h2[2]), f3 = __bfloat1622float2(h2[3]);
-      *reinterpret_cast<float4*>(d) = make_float4(f0.x, f0.y, f1.x, f1.y);
-      *reinterpret_cast<float4*>(d + 4) = make_float4(f2.x, f2.y, f3.x, f3.y);
-    }
-  }
-}
-
 __host__ __device__ constexpr int wy_scratch(int K) {
   return 2 * SUB * (K + 1) + RS * K > 2 * CH * LDA ? 2 * SUB * (K + 1) + RS * K : 2 * CH * LDA;
 }
@@ -113,10 +69,10 @@ __global__ void __launch_bounds__(256) k_kda_wy(Problem p, Args a, KdaWork w) {
   float* sX = sP + CH * CH;   // scratch: Lk [16][K+1], Lq [16][K+1], R^T [K][RS]; later T, X [64][LDA]
   float* sb = sX + wy_scratch(K);  // [64] beta, 0 past L
   const size_t rs = (size_t)p.H * K;
-  load_tile<T>(sK, static_cast<const T*>(a.k) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
-  load_tile<T>(sQ, static_cast<const T*>(a.q) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
-  load_tile<T>(sV, static_cast<const T*>(a.v) + ((size_t)tok0 * p.HV + hv) * V, (size_t)p.HV * V, L, V);
-  load_tile<float>(sG, a.g_raw + ((size_t)tok0 * p.HV + hv) * K, (size_t)p.HV * K, L, K);
+  load_tile<T>(sK, K, static_cast<const T*>(a.k) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
+  load_tile<T>(sQ, K, static_cast<const T*>(a.q) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
+  load_tile<T>(sV, V, static_cast<const T*>(a.v) + ((size_t)tok0 * p.HV + hv) * V, (size_t)p.HV * V, L, V);
+  load_tile<float>(sG, K, a.g_raw + ((size_t)tok0 * p.HV + hv) * K, (size_t)p.HV * K, L, K);
   if (tid < CH) sb[tid] = tid < L ? a.beta[(size_t)(tok0 + tid) * p.HV + hv] : 0.f;
   __syncthreads();
   {  // the gate of every (token, channel), rows past L zero; then the cumsum per channel

@@ -33,27 +33,6 @@ using tcx::LDA;
 
 __device__ __forceinline__ bool kda_failed(const KdaWork& w) { return *((volatile int*)w.status) != 0; }
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
-}
-__device__ __forceinline__ void copy_async(float* dst, const float* src, int n) {
-  for (int i = threadIdx.x; i < n / 4; i += blockDim.x) cp_async16(dst + 4 * i, src + 4 * i);
-}
-
-// Rows [0, L) of a 64 x D token tile (row stride rs) into fp32 shared memory with row stride
-// ldd, rows past L zero.
-template <typename T>
-__device__ __forceinline__ void load_tok(float* dst, int ldd, const T* src, size_t rs, int L, int D) {
-  for (int x = threadIdx.x; x < CH * D; x += blockDim.x) {
-    const int t = x / D, c = x % D;
-    dst[t * ldd + c] = t < L ? to_f<T>(src[(size_t)t * rs + c]) : 0.f;
-  }
-}
-
 // Per-channel gated products of a 64 x 64 weight Wt (lower triangle used, ldw) with row
 // operand R and column operand Lm ([64][K], row stride K), Gam2 = Gam * log2(e) ([64][K]):
 //   F_i = sum_{j<=i} Wt_ij R_j e^{Gam_i - Gam_j},   G_j = sum_{i>=j} colw_i Wt_ij Lm_i e^{Gam_i - Gam_j}
@@ -165,8 +144,11 @@ __global__ void __launch_bounds__(256) k_kda_bwd_scan(Problem p, Args a, KdaWork
 }
 
 // ---------------------------------------------------------------- output-side terms
-// dP, dK^ (with the Gam_C column terms), dQ~, dW = -dU S, and the dP gated products.
-// Writes the unit's dq and dk shares, dGam and dW.
+// dP, dQ~, dW = -dU S, dK^ (with the Gam_C column terms) and the dP gated products.  Writes the
+// unit's dq and dk shares, dGam and dW.  Every product reads both operands from shared memory:
+// a 64 KB region holds S, then dS', then q and k.
+__host__ __device__ constexpr int dqk_x1(int K, int V) { return V * K > 2 * CH * K ? V * K : 2 * CH * K; }
+
 template <typename T>
 __global__ void __launch_bounds__(256) k_kda_bwd_dqk(Problem p, Args a, KdaWork w) {
   if (kda_failed(w)) return;
@@ -174,44 +156,68 @@ __global__ void __launch_bounds__(256) k_kda_bwd_dqk(Problem p, Args a, KdaWork 
   const int4 e = w.chunk_tab[gc];
   if (e.x < 0) return;
   const int K = p.K, V = p.V, L = e.z, tok0 = e.w, hk = hv / p.G, tid = threadIdx.x;
+  const int NP = blockDim.x / K, part = tid / K, cc = tid % K;  // column-sum parts (2 or 4)
   extern __shared__ float sm[];
-  float* sQ = sm;                  // [64][K]
-  float* sK = sQ + CH * K;         // [64][K]
-  float* sG = sK + CH * K;         // [64][K]  Gam * log2(e)
-  float* sR1 = sG + CH * K;        // [64][max(V, K)]  dO, then scratch of the gated products
-  float* sR2 = sR1 + CH * (V > K ? V : K);  // [64][V+1]  U, then dU
-  float* sdP = sR2 + CH * (V + 1); // [64][65]
-  float* sGC = sdP + CH * LDP;     // [K]  dL/dGam_C
+  float* sX1 = sm;                  // S [V][K], then dS' [V][K], then q [64][K] | k [64][K]
+  float* sG = sX1 + dqk_x1(K, V);   // [64][K]  Gam * log2(e)
+  float* sR1 = sG + CH * K;         // [64][max(V, K)]  dO, then dU, then scratch
+  float* sR2 = sR1 + CH * (V > K ? V : K);  // [64][V+1]  U
+  float* sdP = sR2 + CH * (V + 1);  // [64][65]
+  float* sred = sdP + CH * LDP;     // [NP][K] partial column sums
+  float* sGC = sred + 4 * K;        // [K]  dL/dGam_C
   const size_t u = (size_t)gc * p.HV + hv, uk = u * CH * K;
-  const size_t rs = (size_t)p.H * K;
-  load_tok<T>(sQ, K, static_cast<const T*>(a.q) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
-  load_tok<T>(sK, K, static_cast<const T*>(a.k) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
-  load_tok<T>(sR1, V, static_cast<const T*>(a.dO) + ((size_t)tok0 * p.HV + hv) * V, (size_t)p.HV * V, L, V);
-  copy_async(sG, w.Gam + uk, CH * K);
-  for (int x = tid; x < CH * V; x += blockDim.x) sR2[(x / V) * (V + 1) + x % V] = w.U[u * CH * V + x];
-  cp_async_wait_all();
-  __syncthreads();
-  const float* S = w.h + u * V * K;    // [V][K]
-  const float* dSn = w.dh + u * V * K; // [V][K]
   float* dqp = w.dqp + uk;
   float* dkp = w.dkp + uk;
   float* dG = w.dGam + uk;
-  // dP = scale dO U^T, lower triangle incl. diagonal
-  mm(CH, CH, V, sdP, LDP, p.scale, false, sR1, V, 1, sR2, 1, V + 1);
-  // dK^ = U dS' (raw, into the dk share)
-  mm(CH, K, V, dkp, K, 1.f, false, sR2, V + 1, 1, dSn, K, 1);
-  // dQ~ = scale dO S (raw, into the dq share)
-  mm(CH, K, V, dqp, K, p.scale, false, sR1, V, 1, S, K, 1);
+  copy_async(sX1, w.h + u * V * K, V * K);
+  copy_async(sG, w.Gam + uk, CH * K);
+  load_tile<T>(sR1, V, static_cast<const T*>(a.dO) + ((size_t)tok0 * p.HV + hv) * V, (size_t)p.HV * V, L, V);
+  for (int x = tid; x < CH * V; x += blockDim.x) sR2[(x / V) * (V + 1) + x % V] = w.U[u * CH * V + x];
+  cp_async_wait_all();
   __syncthreads();
+  mm(CH, CH, V, sdP, LDP, p.scale, false, sR1, V, 1, sR2, 1, V + 1);  // dP = scale dO U^T
+  mm(CH, K, V, dqp, K, p.scale, false, sR1, V, 1, sX1, K, 1);         // dQ~ = scale dO S (raw)
+  {  // e^{Gam_C} colsum(dS' * S), part of dL/dGam_C
+    const float* dSn = w.dh + u * V * K;
+    float t = 0.f;
+    for (int v = part; v < V; v += NP) t += dSn[(size_t)v * K + cc] * sX1[v * K + cc];
+    sred[part * K + cc] = t;
+  }
+  __syncthreads();
+  if (tid < K) {
+    float t = 0.f;
+    for (int q = 0; q < NP; ++q) t += sred[q * K + tid];
+    sGC[tid] = exp2f(sG[(CH - 1) * K + tid]) * t;
+  }
   for (int x = tid; x < CH * CH; x += blockDim.x)
     if (x % CH > x / CH) sdP[(x / CH) * LDP + x % CH] = 0.f;
-  for (int c = tid; c < K; c += blockDim.x) {  // dL/dGam_C
-    const float gC = sG[(CH - 1) * K + c];
-    float s = 0.f;
-    for (int i = 0; i < CH; ++i) s += dkp[i * K + c] * sK[i * K + c] * exp2f(gC - sG[i * K + c]);
+  copy_async(sR1, w.dU + u * CH * V, CH * V);  // dO is done
+  cp_async_wait_all();
+  __syncthreads();
+  mm(CH, K, V, w.dW + uk, K, -1.f, false, sR1, V, 1, sX1, K, 1);  // dW = -dU S
+  __syncthreads();
+  copy_async(sX1, w.dh + u * V * K, V * K);  // S is done
+  cp_async_wait_all();
+  __syncthreads();
+  mm(CH, K, V, dkp, K, 1.f, false, sR2, V + 1, 1, sX1, K, 1);  // dK^ = U dS' (raw)
+  __syncthreads();
+  float* sQ = sX1;
+  float* sK = sX1 + CH * K;
+  const size_t rs = (size_t)p.H * K;
+  load_tile<T>(sQ, K, static_cast<const T*>(a.q) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
+  load_tile<T>(sK, K, static_cast<const T*>(a.k) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
+  __syncthreads();
+  {  // colsum(dK^ * K^), the rest of dL/dGam_C
+    const float gC = sG[(CH - 1) * K + cc];
     float t = 0.f;
-    for (int v = 0; v < V; ++v) t += dSn[(size_t)v * K + c] * S[(size_t)v * K + c];
-    sGC[c] = s + exp2f(gC) * t;
+    for (int i = part; i < CH; i += NP) t += dkp[i * K + cc] * sK[i * K + cc] * exp2f(gC - sG[i * K + cc]);
+    sred[part * K + cc] = t;
+  }
+  __syncthreads();
+  if (tid < K) {
+    float t = 0.f;
+    for (int q = 0; q < NP; ++q) t += sred[q * K + tid];
+    sGC[tid] += t;
   }
   __syncthreads();
   for (int x = tid; x < CH * K; x += blockDim.x) {
@@ -222,10 +228,7 @@ __global__ void __launch_bounds__(256) k_kda_bwd_dqk(Problem p, Args a, KdaWork 
     dqp[x] = dqt * eg;
     dG[x] = dqt * sQ[x] * eg - dkh * sK[x] * kh + (i == CH - 1 ? sGC[c] : 0.f);
   }
-  // dW = -dU S
-  for (int x = tid; x < CH * V; x += blockDim.x) sR2[(x / V) * (V + 1) + x % V] = w.dU[u * CH * V + x];
   __syncthreads();
-  mm(CH, K, V, w.dW + uk, K, -1.f, false, sR2, V + 1, 1, S, K, 1);
   // P_ij = sum_c q_i k_j e^{Gam_i - Gam_j}: dq += F2, dk += G2, dGam += q F2 - k G2
   gated_products(sdP, LDP, sK, sQ, nullptr, sG, K, sR1,
                  [&](int i, int c, float f) {
@@ -261,8 +264,8 @@ __global__ void __launch_bounds__(256) k_kda_bwd_wy(Problem p, Args a, KdaWork w
   float* sdb = sb + CH;            // [64]
   const size_t u = (size_t)gc * p.HV + hv, uk = u * CH * K;
   const size_t rs = (size_t)p.H * K;
-  load_tok<T>(sK, K, static_cast<const T*>(a.k) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
-  load_tok<T>(sY, V + 1, static_cast<const T*>(a.v) + ((size_t)tok0 * p.HV + hv) * V, (size_t)p.HV * V, L, V);
+  load_tile<T>(sK, K, static_cast<const T*>(a.k) + ((size_t)tok0 * p.H + hk) * K, rs, L, K);
+  load_tile<T>(sY, V + 1, static_cast<const T*>(a.v) + ((size_t)tok0 * p.HV + hv) * V, (size_t)p.HV * V, L, V);
   copy_async(sG, w.Gam + uk, CH * K);
   copy_async(sdW, w.dW + uk, CH * K);
   copy_async(sdU, w.dU + u * CH * V, CH * V);
@@ -339,44 +342,56 @@ __global__ void __launch_bounds__(256) k_kda_bwd_wy(Problem p, Args a, KdaWork w
     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
     if (lane == 0 && i < L) a.dbeta[(size_t)(tok0 + i) * p.HV + hv] = sdb[i] + s;
   }
-  // the raw gate inputs of this unit, for the gate chain
-  float* sg = sdU;
-  for (int x = tid; x < CH * K; x += blockDim.x) {
-    const int i = x / K;
-    sg[x] = i < L ? a.g_raw[((size_t)(tok0 + i) * p.HV + hv) * K + x % K] : 0.f;
+  __syncthreads();
+  // the unit's dGam and raw gate inputs in shared memory (the F1 terms above are in dGam)
+  float* sdG = sdW;  // Z is done
+  float* sg = sdU;   // the scratch is done
+  copy_async(sdG, dG, CH * K);
+  load_tile<float>(sg, K, a.g_raw + ((size_t)tok0 * p.HV + hv) * K, (size_t)p.HV * K, L, K);
+  cp_async_wait_all();
+  __syncthreads();
+  // dyg = reverse in-chunk cumsum of dGam: NP row parts, each offset by the parts below it
+  const int NP = blockDim.x / K, part = tid / K, cc = tid % K, rows = CH / NP;
+  float* sred = sT;  // [NP][K]; T is done
+  {
+    float t = 0.f;
+    for (int i = part * rows; i < (part + 1) * rows; ++i) t += sdG[i * K + cc];
+    sred[part * K + cc] = t;
   }
   __syncthreads();
-  // dyg = reverse in-chunk cumsum of dGam; gate chain; per-chunk parameter sums
   const float nexp = -expf(a.A_log[hv]);
-  float* pg = w.pgp + u * (K + 1);
-  float pA = 0.f;
-  for (int c = tid; c < K; c += blockDim.x) {
-    const float bias = a.dt_bias ? a.dt_bias[(size_t)hv * K + c] : 0.f;
-    float acc = 0.f, pB = 0.f;
-    for (int i = CH - 1; i >= 0; --i) {
-      acc += dG[i * K + c];
-      if (i < L) {
-        const size_t o = ((size_t)(tok0 + i) * p.HV + hv) * K + c;
-        const float x = sg[i * K + c] + bias;
-        const float sp = x > 20.f ? x : log1pf(expf(x));
-        const float sig = x > 20.f ? 1.f : 1.f / (1.f + expf(-x));
-        const float dgr = acc * nexp * sig;
-        a.dg[o] = acc;
-        if (a.dg_raw) a.dg_raw[o] = dgr;
-        pA += acc * nexp * sp;
-        pB += dgr;
-      }
+  const float bias = a.dt_bias ? a.dt_bias[(size_t)hv * K + cc] : 0.f;
+  float acc = 0.f, pA = 0.f, pB = 0.f;
+  for (int q = part + 1; q < NP; ++q) acc += sred[q * K + cc];
+  for (int i = (part + 1) * rows - 1; i >= part * rows; --i) {
+    acc += sdG[i * K + cc];
+    if (i < L) {
+      const size_t o = ((size_t)(tok0 + i) * p.HV + hv) * K + cc;
+      const float x = sg[i * K + cc] + bias;
+      const float sp = x > 20.f ? x : log1pf(expf(x));
+      const float sig = x > 20.f ? 1.f : 1.f / (1.f + expf(-x));
+      const float dgr = acc * nexp * sig;
+      a.dg[o] = acc;
+      if (a.dg_raw) a.dg_raw[o] = dgr;
+      pA += acc * nexp * sp;
+      pB += dgr;
     }
-    pg[c] = pB;
   }
-  for (int off = 16; off > 0; off >>= 1) pA += __shfl_xor_sync(0xffffffffu, pA, off);
   __syncthreads();
+  sred[part * K + cc] = pB;
+  for (int off = 16; off > 0; off >>= 1) pA += __shfl_xor_sync(0xffffffffu, pA, off);
   if (lane == 0) sdb[warp] = pA;
   __syncthreads();
+  float* pg = w.pgp + u * (K + 1);
+  if (tid < K) {
+    float t = 0.f;
+    for (int q = 0; q < NP; ++q) t += sred[q * K + tid];
+    pg[tid] = t;
+  }
   if (tid == 0) {
-    float s = 0.f;
-    for (int q = 0; q < nwarp; ++q) s += sdb[q];
-    pg[K] = s;
+    float t = 0.f;
+    for (int q = 0; q < nwarp; ++q) t += sdb[q];
+    pg[K] = t;
   }
 }
 
@@ -397,7 +412,8 @@ __global__ void __launch_bounds__(256) k_kda_param_grads(Problem p, Args a, KdaW
 
 size_t scan_smem(int K) { return (size_t)(32 * (K + 1) + CH * CH + 3 * CH * K + 2 * CH * 32 + K) * sizeof(float); }
 size_t dqk_smem(int K, int V) {
-  return (size_t)(3 * CH * K + CH * (V > K ? V : K) + CH * (V + 1) + CH * LDP + K) * sizeof(float);
+  return (size_t)(dqk_x1(K, V) + CH * K + CH * (V > K ? V : K) + CH * (V + 1) + CH * LDP + 5 * K) *
+         sizeof(float);
 }
 size_t wy_smem(int K, int V) {
   const int big = (V > K ? V : K) * CH > CH * LDP ? (V > K ? V : K) * CH : CH * LDP;
