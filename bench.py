@@ -649,14 +649,19 @@ def kda_chunk_measure(gdn, dev, pk_hbm: float, steps: int = 5) -> dict:
     gdn.profile(False)
     units = (32768 // 64) * 32
     K = V = 128
+    # FMA per (chunk, value head) of each kernel's products
     fma = {"kda_wy": 2 * 1536 * K + 2 * 544 * K + 64 * 64 * K + 64 * 64 * V,
-           "kda_scan": 64 * V * K + V * K * 64, "kda_out": 64 * V * 64 + 64 * V * K}
+           "kda_scan": 64 * V * K + V * K * 64, "kda_out": 64 * V * 64 + 64 * V * K,
+           "kda_bwd_scan": 64 * 64 * V + 3 * 64 * V * K,
+           "kda_bwd_dqk": 64 * 64 * V + 3 * 64 * V * K + 2 * (1536 + 544) * K,
+           "kda_bwd_wy": 2 * 64 * 64 * (K + V) + 2 * 64 * 64 * 64 + 2 * (1536 + 544) * K}
     kern = {k: round(v[1], 4) for k, v in prof.items()}
     top = max(fma, key=lambda k: kern.get(k, 0.0))
     top_tf = 2 * units * fma[top] / (kern[top] / 1e3) / 1e12
     return {"workload": "kda_chunk_B1_T32768_H16_HV32_D128_bf16", "fwd_ms": round(ms_f, 4),
             "fwd_mtok_s": round(32768 / (ms_f / 1e3) / 1e6, 3), "step_ms": round(ms, 4),
             "step_mtok_s": round(32768 / (ms / 1e3) / 1e6, 3), "kernels_ms": kern,
+            "step_tflops": round(2 * units * sum(fma.values()) / (ms / 1e3) / 1e12, 2),
             "roofline": {"kernel": top, "bound": "alu", "achieved": round(top_tf, 2),
                          "peak": round(FFMA_TFLOPS, 1), "unit": "TFLOP/s",
                          "frac": round(top_tf / FFMA_TFLOPS, 4),
