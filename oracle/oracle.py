@@ -56,8 +56,8 @@ def _load():
 def _f64(x):
     if x is None:
         return None
-    if hasattr(x, "detach"):  # torch tensor
-        x = x.detach().float().cpu().numpy()
+    if hasattr(x, "detach"):  # torch tensor: every float dtype widened exactly to float64
+        x = x.detach().cpu().double().numpy()
     return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
 
 
