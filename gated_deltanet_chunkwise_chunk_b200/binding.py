@@ -27,7 +27,8 @@ EXPORTED = ("gdn_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_max_ch
             "gdn_profile_read", "gdn_chunk_fwd_noalloc", "gdn_noalloc_scratch_bytes",
             "gdn_recurrent_fwd", "gdn_recurrent_workspace_bytes", "gdn_kda_gate_fwd",
             "gdn_kda_gate_bwd", "gdn_kda_gate_workspace_bytes", "gdn_kda_recurrent_fwd",
-            "gdn_kda_chunk_fwd", "gdn_kda_chunk_bwd", "gdn_kda_chunk_workspace_bytes")
+            "gdn_kda_chunk_fwd", "gdn_kda_chunk_bwd", "gdn_kda_chunk_workspace_bytes",
+            "gdn_state_affine")
 
 
 class gdn_dims(ctypes.Structure):
@@ -60,6 +61,8 @@ def _load() -> ctypes.CDLL:
     lib.gdn_recurrent_fwd.restype = I32
     lib.gdn_kda_chunk_fwd.argtypes = [D] + [P] * 12 + [SZ, P]
     lib.gdn_kda_chunk_fwd.restype = I32
+    lib.gdn_state_affine.argtypes = [I64, I64, I64, P, I32, P, P, P, P]
+    lib.gdn_state_affine.restype = I32
     lib.gdn_kda_chunk_bwd.argtypes = [D] + [P] * 20 + [SZ, P]
     lib.gdn_kda_chunk_bwd.restype = I32
     lib.gdn_kda_chunk_workspace_bytes.argtypes = [D, I32, I32]
@@ -326,6 +329,24 @@ def gdn_kda_chunk_bwd(q, k, v, g_raw, A_log, dt_bias, beta, d_o, workspace, cu_s
     if rc != GDN_OK:
         raise GDNError("gdn_kda_chunk_bwd", rc)
     return outs
+
+
+def state_affine(A, X, B=None, transpose=False, out=None):
+    """out[n] = op(A[n]) X[n] + B[n] over the leading dims: A [..., K, K], X and B [..., K, V]
+    fp32 (op = transpose when asked).  `out` may be X."""
+    K, V = X.shape[-2], X.shape[-1]
+    count = X.numel() // (K * V) if X.numel() else 0
+    _check("A", A, torch.float32, tuple(X.shape[:-2]) + (K, K), X.device)
+    _check("B", B, torch.float32, tuple(X.shape), X.device)
+    if not X.is_contiguous() or X.dtype != torch.float32:
+        raise ValueError("X: expected contiguous float32")
+    out = out if out is not None else torch.empty_like(X)
+    _check("out", out, torch.float32, tuple(X.shape), X.device)
+    rc = lib.gdn_state_affine(count, K, V, _ptr(A), int(bool(transpose)), _ptr(X), _ptr(B), _ptr(out),
+                              _stream())
+    if rc != GDN_OK:
+        raise GDNError("gdn_state_affine", rc)
+    return out
 
 
 _TORCH_DT = {torch.float32: GDN_DTYPE_FP32, torch.bfloat16: GDN_DTYPE_BF16,

@@ -538,6 +538,16 @@ int gdn_kda_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const voi
                                         static_cast<cudaStream_t>(stream)));
 }
 
+int gdn_state_affine(int64_t count, int64_t K, int64_t V, const float* A, int transpose_a, const float* X,
+                     const float* B, float* out, void* stream) {
+  if (count < 0 || count > INT32_MAX || K < 1 || K > 128 || V < 32 || V % 32 || V / 32 > 65535)
+    return GDN_ERR_INVALID_ARG;
+  if (count > 0 && (!A || !X || !out)) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(X) || !aligned16(B) || !aligned16(out)) return GDN_ERR_INVALID_ARG;
+  return cuda_status(state_affine(count, (int)K, (int)V, A, transpose_a != 0, X, B, out,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
 static int kda_check(int64_t T, int64_t H, int64_t D, int32_t dt1, int32_t dt2) {
   if (T < 0 || H <= 0 || D <= 0 || H > 65535) return GDN_ERR_INVALID_ARG;
   if (H * D > ((int64_t)1 << 24) || T > ((int64_t)1 << 62) / (H * D)) return GDN_ERR_INVALID_ARG;

@@ -38,6 +38,8 @@ cudaError_t kda_gate_backward(int64_t T, int H, int D, int in_dtype, const void*
                               const float* dt_bias, int dy_dtype, const void* dyg, void* dg,
                               float* dA_log, float* ddt_bias, float* part, cudaStream_t s);
 // Token-by-token forward (decoding, short prefills); status: device status word.
+cudaError_t state_affine(int64_t count, int K, int V, const float* A, bool transA, const float* X,
+                         const float* Bm, float* out, cudaStream_t s);
 cudaError_t launch_dqdk_group_sum(const Problem& p, const Args& a, const Work& w, bool bf16, cudaStream_t s);
 cudaError_t kda_chunk_backward(const Problem& p, const Args& a, const KdaWork& w, bool bf16, cudaStream_t s);
 cudaError_t kda_chunk_forward(const Problem& p, const Args& a, const KdaWork& w, bool bf16, cudaStream_t s);

@@ -236,6 +236,19 @@ size_t gdn_kda_chunk_workspace_bytes(const gdn_dims* d, int varlen, int pass);
 /* Workspace bytes of gdn_kda_gate_bwd (0 for invalid sizes). */
 size_t gdn_kda_gate_workspace_bytes(int64_t T, int64_t H, int64_t D);
 
+/* Affine maps of states, for context parallelism over T (a sequence split into segments, one
+ * per rank).  A segment maps the state entering it to the state leaving it affinely; in the
+ * [K][V] layout of the state arguments above, h_end = Mt h_start + Bh, where Mt (K x K) is the
+ * final_state gdn_chunk_fwd returns for the segment from initial_state = I with v = 0 (K = V),
+ * and Bh the one it returns from initial_state = 0 (the state after a segment is linear in the
+ * state before it, as every step of the recurrence is).  The gradient entering the segment is
+ * Mt^T dh_end + D, D the dh0 of gdn_chunk_bwd for the segment with dht = 0.
+ *   out[n] = op(A[n]) X[n] + B[n],  n < count,  op(A) = A or A^T (transpose_a != 0),
+ * A [count][K][K], X, B, out [count][K][V] fp32 device pointers (B may be NULL; out may be X).
+ * 1 <= K <= 128, V a multiple of 32; GDN_ERR_INVALID_ARG otherwise. */
+int gdn_state_affine(int64_t count, int64_t K, int64_t V, const float* A, int transpose_a, const float* X,
+                     const float* B, float* out, void* stream);
+
 /* Upper bound on the number of 64-token chunks (the grid size used for chunk kernels). */
 int64_t gdn_max_chunks(const gdn_dims* d, int varlen);
 
