@@ -100,6 +100,46 @@ def test_entry_points_reject_bad_arguments_before_launch():
     assert lib.gdn_recurrent_workspace_bytes() == 256
 
 
+def test_kda_and_state_entry_points_reject_bad_arguments_before_launch():
+    d = _dims()
+    lib = binding.lib
+    P = ctypes.c_void_p
+    al, mis, null = P(4096), P(4097), None
+    # KDA gate: bad sizes, unknown dtype, null input, misaligned pointer, small workspace
+    assert lib.gdn_kda_gate_fwd(8, 0, 64, 1, al, al, null, 0, al, null) == binding.GDN_ERR_INVALID_ARG
+    assert lib.gdn_kda_gate_fwd(8, 4, 64, 9, al, al, null, 0, al, null) == binding.GDN_ERR_UNSUPPORTED
+    assert lib.gdn_kda_gate_fwd(8, 4, 64, 1, null, al, null, 0, al, null) == binding.GDN_ERR_INVALID_ARG
+    assert lib.gdn_kda_gate_fwd(8, 4, 64, 1, mis, al, null, 0, al, null) == binding.GDN_ERR_INVALID_ARG
+    assert lib.gdn_kda_gate_bwd(8, 4, 64, 1, al, al, null, 0, al, al, al, null, al, 16, null) == \
+        binding.GDN_ERR_WORKSPACE
+    assert lib.gdn_kda_gate_workspace_bytes(8, 4, 64) > 0
+    assert lib.gdn_kda_gate_workspace_bytes(8, 1 << 13, 1 << 12) == 0  # H*D > 2^24
+    # KDA recurrence: dt_bias may be NULL, A_log may not
+    rc = lib.gdn_kda_recurrent_fwd(ctypes.byref(d), al, al, al, al, null, null, al, null, null, al,
+                                   null, al, 1 << 20, null)
+    assert rc == binding.GDN_ERR_INVALID_ARG
+    # chunkwise KDA: workspace sizes by pass, too small a workspace, backward needs pass-1 size
+    w0 = lib.gdn_kda_chunk_workspace_bytes(ctypes.byref(d), 0, 0)
+    w1 = lib.gdn_kda_chunk_workspace_bytes(ctypes.byref(d), 0, 1)
+    assert 0 < w0 < w1
+    assert lib.gdn_kda_chunk_workspace_bytes(ctypes.byref(d), 0, 2) == 0
+    assert lib.gdn_kda_chunk_workspace_bytes(ctypes.byref(_dims(K=96)), 0, 0) == 0
+    rc = lib.gdn_kda_chunk_fwd(ctypes.byref(d), al, al, al, al, al, null, al, null, null, al, null,
+                               al, w0 - 256, null)
+    assert rc == binding.GDN_ERR_WORKSPACE
+    rc = lib.gdn_kda_chunk_bwd(ctypes.byref(d), al, al, al, al, al, null, al, null, al, null, al, al,
+                               al, al, al, null, null, null, null, al, w0, null)
+    assert rc == binding.GDN_ERR_WORKSPACE
+    rc = lib.gdn_kda_chunk_bwd(ctypes.byref(d), al, al, al, al, al, null, al, null, al, null, al, al,
+                               al, al, al, null, null, null, al, al, w1, null)  # ddt_bias without dt_bias
+    assert rc == binding.GDN_ERR_INVALID_ARG
+    # state affine maps: K, V limits, null operands
+    assert lib.gdn_state_affine(4, 129, 128, al, 0, al, null, al, null) == binding.GDN_ERR_INVALID_ARG
+    assert lib.gdn_state_affine(4, 128, 48, al, 0, al, null, al, null) == binding.GDN_ERR_INVALID_ARG
+    assert lib.gdn_state_affine(4, 128, 128, null, 0, al, null, al, null) == binding.GDN_ERR_INVALID_ARG
+    assert lib.gdn_state_affine(4, 128, 128, al, 0, mis, null, al, null) == binding.GDN_ERR_INVALID_ARG
+
+
 def _enumerate(cu, B, T):
     """Plain enumeration of 64-token chunks: (sequence, chunk, tokens, first flat token)."""
     out = []
