@@ -257,8 +257,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--T", type=int, default=None,
                     help="override the sequence length of a dense workload (smaller profiling cases)")
-    ap.add_argument("--workload", default="gdn", choices=["gdn", "kda_chunk"],
-                    help="kda_chunk: only the chunkwise KDA measurement (its T from --T, default 32768)")
+    ap.add_argument("--workload", default="gdn", choices=["gdn", "kda_chunk", "decode"],
+                    help="kda_chunk: only the chunkwise KDA measurement (its T from --T, default 32768); "
+                         "decode: only the decode-step measurement")
     ap.add_argument("--ref-budget", type=float, default=90.0,
                     help="seconds of oracle work over the whole --impl reference run")
     args = ap.parse_args()
@@ -274,6 +275,13 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.workload == "decode":
+        line = decode_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"], steps=max(1, args.steps))
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if dist:
+            dist.destroy_process_group()
+        return
     if args.workload == "kda_chunk":
         line = kda_chunk_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"], steps=max(1, args.steps),
                                  T=args.T or 32768)

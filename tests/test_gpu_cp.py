@@ -65,7 +65,7 @@ def _emulate(case, bounds, dO):
 
 
 @pytest.mark.parametrize("bounds,long_memory", [([0, 200, 512], False), ([0, 64, 130, 300, 512], False),
-                                                ([0, 150, 333, 700], True)])
+                                                ([0, 150, 333, 700], True), ([0, 0, 200, 512], True)])
 def test_segments_equal_the_whole_sequence(bounds, long_memory):
     T = bounds[-1]
     case = synth.make_case(B=1, T=T, H=2, HV=4, K=128, V=128, dtype="bf16", seed=700 + T, h0=True,

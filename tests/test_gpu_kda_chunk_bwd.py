@@ -104,3 +104,21 @@ def test_layer_heads_1024_tokens():
     case = synth.make_case(B=1, T=1024, H=16, HV=32, K=128, V=128, dtype="bf16", seed=650, h0=True,
                            name="kda_bwd_layer")
     _run(case, seed=651)
+
+
+def test_empty_input_passes_the_gradient_through():
+    import gated_deltanet_chunkwise_chunk_b200 as gdn
+    case = synth.make_case(B=2, T=0, H=1, HV=2, K=64, V=64, dtype="bf16", seed=660, h0=True, dht=True,
+                           name="kda_bwd_T0")
+    g_raw, A_log, dt_bias = synth.kda_gate_inputs(case, 661)
+    d = to_dev(case)
+    d["g_raw"], d["A_log"], d["dt_bias"] = g_raw.cuda(), A_log.cuda(), dt_bias.cuda()
+    dims = gdn.make_dims(d["q"], d["v"])
+    ws = torch.empty(gdn.kda_chunk_workspace_bytes(dims, False, True), dtype=torch.uint8, device="cuda")
+    o, ht = gdn.gdn_kda_chunk_fwd(**d, workspace=ws)
+    d.pop("initial_state")
+    d_o = torch.empty(2, 0, 2, 64, dtype=torch.bfloat16, device="cuda")
+    out = gdn.gdn_kda_chunk_bwd(**d, d_o=d_o, dht=case.dht.cuda(), workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(ht.cpu(), case.h0) and torch.equal(out["dh0"].cpu(), case.dht)
+    assert torch.all(out["dA_log"] == 0) and torch.all(out["ddt_bias"] == 0)
