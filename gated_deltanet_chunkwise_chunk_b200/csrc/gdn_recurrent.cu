@@ -30,7 +30,10 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
   const int nz = p.V / RV;
   const int n = blockIdx.x / nz, hv = blockIdx.y, hk = hv / p.G, v0 = RV * (blockIdx.x % nz);
   const int tid = threadIdx.x, lane = tid & 31, kg = lane & 15, vg = 2 * (tid >> 5) + (lane >> 4);
-  __shared__ float sk[K], sq[K], sv[RV], sdec, sbeta, sdk[KDA ? K : 1];
+  __shared__ __align__(16) float sk[K];
+  __shared__ __align__(16) float sq[K];
+  __shared__ __align__(16) float sdk[KDA ? K : 4];
+  __shared__ float sv[RV], sdec, sbeta;
   int bos, eos;
   if (p.varlen) {
     bos = (int)a.cu[n];
@@ -57,12 +60,24 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
   const T* v = static_cast<const T*>(a.v);
   T* o = static_cast<T*>(a.o);
   const float nexp = -expf(a.A_log[hv]), dtb = KDA ? 0.f : a.dt_bias[hv];
-  auto rowsum = [](float x) {  // over the 16 k-groups of this lane half
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    x += __shfl_xor_sync(0xffffffffu, x, 2);
-    x += __shfl_xor_sync(0xffffffffu, x, 4);
-    x += __shfl_xor_sync(0xffffffffu, x, 8);
-    return x;
+  // Sums over the 16 k-groups of this lane half of four values at once: each butterfly step
+  // halves the values a lane carries (2 + 1 shuffles), two more steps finish the sum; lane
+  // kg = 4j then holds the total of value j (x, y, z, w for j = 0..3).  5 shuffles, not 16.
+  const bool b3 = kg & 8, b2 = kg & 4;
+  auto rowsum4 = [&](const float4& e) {
+    float s0 = b3 ? e.z : e.x, s1 = b3 ? e.w : e.y;
+    s0 += __shfl_xor_sync(0xffffffffu, b3 ? e.x : e.z, 8);
+    s1 += __shfl_xor_sync(0xffffffffu, b3 ? e.y : e.w, 8);
+    float t = b2 ? s1 : s0;
+    t += __shfl_xor_sync(0xffffffffu, b2 ? s0 : s1, 4);
+    t += __shfl_xor_sync(0xffffffffu, t, 2);
+    t += __shfl_xor_sync(0xffffffffu, t, 1);
+    return t;
+  };
+  const int half = lane & 16;
+  auto gather4 = [&](float t) {  // the four totals to every lane of the half
+    return make_float4(__shfl_sync(0xffffffffu, t, half), __shfl_sync(0xffffffffu, t, half + 4),
+                       __shfl_sync(0xffffffffu, t, half + 8), __shfl_sync(0xffffffffu, t, half + 12));
   };
   const size_t dtb_k = (size_t)hv * K;
   for (int t = bos; t < eos; ++t) {
@@ -90,33 +105,39 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
     if (tid == 96) sbeta = bf;
     __syncthreads();
     const float b = sbeta;
+    float kv[KQ], qv[KQ], dv[KQ];  // this thread's channels, read as 16-byte vectors
+#pragma unroll
+    for (int i = 0; i < KQ; i += 4) {
+      const float4 k4 = *reinterpret_cast<const float4*>(sk + kg * KQ + i);
+      const float4 q4 = *reinterpret_cast<const float4*>(sq + kg * KQ + i);
+      kv[i] = k4.x; kv[i + 1] = k4.y; kv[i + 2] = k4.z; kv[i + 3] = k4.w;
+      qv[i] = q4.x; qv[i + 1] = q4.y; qv[i + 2] = q4.z; qv[i + 3] = q4.w;
+      if constexpr (KDA) {
+        const float4 d4 = *reinterpret_cast<const float4*>(sdk + kg * KQ + i);
+        dv[i] = d4.x; dv[i + 1] = d4.y; dv[i + 2] = d4.z; dv[i + 3] = d4.w;
+      } else {
+        dv[i] = dv[i + 1] = dv[i + 2] = dv[i + 3] = sdec;
+      }
+    }
     float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < KQ; ++i) {
-      const float kv = sk[kg * KQ + i];
-      const float dec = KDA ? sdk[kg * KQ + i] : sdec;
+      const float dec = dv[i];
       S4[i].x *= dec; S4[i].y *= dec; S4[i].z *= dec; S4[i].w *= dec;
-      e.x += S4[i].x * kv; e.y += S4[i].y * kv; e.z += S4[i].z * kv; e.w += S4[i].w * kv;
+      e.x += S4[i].x * kv[i]; e.y += S4[i].y * kv[i]; e.z += S4[i].z * kv[i]; e.w += S4[i].w * kv[i];
     }
-    e.x = rowsum(e.x); e.y = rowsum(e.y); e.z = rowsum(e.z); e.w = rowsum(e.w);
+    e = gather4(rowsum4(e));
     const float* vv = sv + 4 * vg;
     const float dx = b * (vv[0] - e.x), dy = b * (vv[1] - e.y), dz = b * (vv[2] - e.z),
                 dw = b * (vv[3] - e.w);
     float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < KQ; ++i) {
-      const float kv = sk[kg * KQ + i], qv = sq[kg * KQ + i];
-      S4[i].x += dx * kv; S4[i].y += dy * kv; S4[i].z += dz * kv; S4[i].w += dw * kv;
-      y.x += S4[i].x * qv; y.y += S4[i].y * qv; y.z += S4[i].z * qv; y.w += S4[i].w * qv;
+      S4[i].x += dx * kv[i]; S4[i].y += dy * kv[i]; S4[i].z += dz * kv[i]; S4[i].w += dw * kv[i];
+      y.x += S4[i].x * qv[i]; y.y += S4[i].y * qv[i]; y.z += S4[i].z * qv[i]; y.w += S4[i].w * qv[i];
     }
-    y.x = rowsum(y.x); y.y = rowsum(y.y); y.z = rowsum(y.z); y.w = rowsum(y.w);
-    if (kg == 0) {
-      T* oo = o + v_0 + 4 * vg;
-      oo[0] = from_f<T>(p.scale * y.x);
-      oo[1] = from_f<T>(p.scale * y.y);
-      oo[2] = from_f<T>(p.scale * y.z);
-      oo[3] = from_f<T>(p.scale * y.w);
-    }
+    const float yt = rowsum4(y);  // lane kg = 4j holds output column j
+    if ((kg & 3) == 0) o[v_0 + 4 * vg + (kg >> 2)] = from_f<T>(p.scale * yt);
   }
   if (a.ht) {
 #pragma unroll
