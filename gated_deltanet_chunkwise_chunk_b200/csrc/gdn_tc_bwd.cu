@@ -476,7 +476,6 @@ struct DqkSmem {
   static constexpr int ROW = G + 256;                        // [3][2][64] per-row partials
   static constexpr int RED = ROW + 3 * 2 * 64 * 4;           // [8]
   static constexpr int TOTAL = RED + 64;
-  static constexpr int LOAD_BYTES = 6 * TILE64 + 7 * TILE128;
 };
 
 __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
