@@ -662,6 +662,11 @@ def kda_chunk_measure(gdn, dev, pk_hbm: float, steps: int = 5, T: int = 32768) -
 
     ms = timed(step)  # the step first: a capture of the first six KDA launches sees every kernel
     ms_f = timed(fwd)
+    # the same forward token by token (the recurrent kernel), for comparison
+    o2, ht2 = torch.empty_like(o), torch.empty_like(ht)
+    wsr = torch.empty(gdn.recurrent_workspace_bytes(), dtype=torch.uint8, device=dev)
+    ms_r = timed(lambda: gdn.gdn_kda_recurrent_fwd(**d, initial_state=h0, out=o2, final_state=ht2,
+                                                   workspace=wsr))
     gdn.profile(True)
     step()
     prof = gdn.profile_read()
@@ -679,7 +684,8 @@ def kda_chunk_measure(gdn, dev, pk_hbm: float, steps: int = 5, T: int = 32768) -
     top_tf = 2 * units * fma[top] / (kern[top] / 1e3) / 1e12
     return {"workload": f"kda_chunk_B1_T{T}_H16_HV32_D128_bf16", "fwd_ms": round(ms_f, 4),
             "fwd_mtok_s": round(T / (ms_f / 1e3) / 1e6, 3), "step_ms": round(ms, 4),
-            "step_mtok_s": round(T / (ms / 1e3) / 1e6, 3), "kernels_ms": kern,
+            "step_mtok_s": round(T / (ms / 1e3) / 1e6, 3), "recurrent_fwd_ms": round(ms_r, 4),
+            "kernels_ms": kern,
             "step_tflops": round(2 * units * sum(fma.values()) / (ms / 1e3) / 1e12, 2),
             "roofline": {"kernel": top, "bound": "alu", "achieved": round(top_tf, 2),
                          "peak": round(FFMA_TFLOPS, 1), "unit": "TFLOP/s",
