@@ -9,13 +9,16 @@ namespace gdn {
 // A(m,kk) = A[m*am + kk*ak], B(kk,n) = B[kk*bk + n*bn], C(m,n) = C[m*ldc + n].
 // M and N multiples of 4.  Each thread owns 4x4 outputs: rows 4*tm.., columns tn + j*N/4.
 // Ownership depends only on (M, N, blockDim), so back-to-back calls with the same shape
-// may accumulate into the same C without a barrier.
+// may accumulate into the same C without a barrier.  tri = 1: A is lower triangular (A(m,kk) = 0
+// for kk > m), tri = 2: upper (A(m,kk) = 0 for kk < m); the loop skips those exact zeros.
 __device__ __forceinline__ void mm(int M, int N, int Kd, float* C, int ldc, float alpha, bool acc,
-                                   const float* A, int am, int ak, const float* B, int bk, int bn) {
+                                   const float* A, int am, int ak, const float* B, int bk, int bn,
+                                   int tri = 0) {
   const int nct = N / 4;
   const int ntile = (M / 4) * nct;
   for (int ti = threadIdx.x; ti < ntile; ti += blockDim.x) {
     const int tm = ti / nct, tn = ti % nct;
+    const int k0 = tri == 2 ? min(Kd, 4 * tm) : 0, k1 = tri == 1 ? min(Kd, 4 * tm + 4) : Kd;
     float r[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -24,7 +27,7 @@ __device__ __forceinline__ void mm(int M, int N, int Kd, float* C, int ldc, floa
     const float* a0 = A + (size_t)(tm * 4) * am;
     const float* b0 = B + (size_t)tn * bn;
 #pragma unroll 4
-    for (int kk = 0; kk < Kd; ++kk) {
+    for (int kk = k0; kk < k1; ++kk) {
       float av[4], bv[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) av[i] = a0[(size_t)i * am + (size_t)kk * ak];

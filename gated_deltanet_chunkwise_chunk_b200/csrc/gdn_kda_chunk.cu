@@ -181,8 +181,8 @@ __global__ void __launch_bounds__(256) k_kda_wy(Problem p, Args a, KdaWork w) {
   for (int c = tid; c < K; c += blockDim.x) w.eGC[u * K + c] = exp2f(sG[(CH - 1) * K + c]);
   for (int x = tid; x < CH * V; x += blockDim.x) sV[x] *= sb[x / V];
   __syncthreads();
-  mm(CH, K, CH, w.W + uk, K, 1.f, false, sT, LDA, 1, sK, K, 1);
-  mm(CH, V, CH, w.Ut + u * CH * V, V, 1.f, false, sT, LDA, 1, sV, V, 1);
+  mm(CH, K, CH, w.W + uk, K, 1.f, false, sT, LDA, 1, sK, K, 1, 1);  // T lower triangular
+  mm(CH, V, CH, w.Ut + u * CH * V, V, 1.f, false, sT, LDA, 1, sV, V, 1, 1);
 }
 
 // Sequential scan of one (sequence, value head, rows v0..v0+31 of S): stores the state entering
@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(256) k_kda_out(Problem p, Args a, KdaWork w) {
   }
   cp_async_wait_all();
   __syncthreads();
-  mm(CH, V, CH, sO, V, 1.f, false, sP, CH, 1, sU, V, 1);
+  mm(CH, V, CH, sO, V, 1.f, false, sP, CH, 1, sU, V, 1, 1);  // P lower triangular
   mm(CH, V, K, sO, V, 1.f, true, sQt, K, 1, sH, V + 1, 1);
   __syncthreads();
   T* o = static_cast<T*>(a.o) + ((size_t)tok0 * p.HV + hv) * V;

@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(256) k_kda_bwd_scan(Problem p, Args a, KdaWork
     for (int x = tid; x < 32 * K; x += blockDim.x) dh[x] = sdS[(x / K) * (K + 1) + x % K];
     cp_async_wait_all();
     __syncthreads();
-    mm(CH, 32, CH, sdU, 32, p.scale, false, sP, 1, CH, sdO, 32, 1);   // scale P^T dO
+    mm(CH, 32, CH, sdU, 32, p.scale, false, sP, 1, CH, sdO, 32, 1, 2);  // scale P^T dO (P^T upper)
     mm(CH, 32, K, sdU, 32, 1.f, true, sKh, K, 1, sdS, 1, K + 1);      // + K^ dS'^T
     __syncthreads();
     float* dU = w.dU + u * CH * V;
@@ -286,8 +286,8 @@ __global__ void __launch_bounds__(256) k_kda_bwd_wy(Problem p, Args a, KdaWork w
   // dX = T^T dW, dY = T^T dU (into the global dW and dU of this unit)
   float* dX = w.dW + uk;
   float* dY = w.dU + u * CH * V;
-  mm(CH, K, CH, dX, K, 1.f, false, sT, 1, LDA, sdW, K, 1);
-  mm(CH, V, CH, dY, V, 1.f, false, sT, 1, LDA, sdU, V, 1);
+  mm(CH, K, CH, dX, K, 1.f, false, sT, 1, LDA, sdW, K, 1, 2);  // T^T upper triangular
+  mm(CH, V, CH, dY, V, 1.f, false, sT, 1, LDA, sdU, V, 1, 2);
   __syncthreads();
   float* dkp = w.dkp + uk;
   float* dG = w.dGam + uk;
@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(256) k_kda_bwd_wy(Problem p, Args a, KdaWork w
   float* sZ = sdW;
   mm(CH, CH, CH, sZ, LDP, 1.f, false, sdT, LDP, 1, sT, 1, LDA);
   __syncthreads();
-  mm(CH, CH, CH, sdT, LDP, -1.f, false, sT, 1, LDA, sZ, LDP, 1);
+  mm(CH, CH, CH, sdT, LDP, -1.f, false, sT, 1, LDA, sZ, LDP, 1, 2);
   __syncthreads();
   for (int x = tid; x < CH * CH; x += blockDim.x)
     if (x % CH >= x / CH) sdT[(x / CH) * LDP + x % CH] = 0.f;
