@@ -27,9 +27,12 @@ def _seg(c, a, b):
     return (c.q[:, a:b], c.k[:, a:b], c.v[:, a:b], c.a[:, a:b], c.A_log, c.dt_bias, c.beta[:, a:b])
 
 
-@pytest.mark.parametrize("bounds", [[0, 37], [0, 20, 37], [0, 1, 15, 36, 37], [0, 0, 30, 37]])
-def test_fold_algebra_matches_the_whole_sequence(bounds):
+@pytest.mark.parametrize("bounds,with_dht", [([0, 37], True), ([0, 20, 37], True), ([0, 1, 15, 36, 37], True),
+                                             ([0, 0, 30, 37], True), ([0, 11, 25, 37], False)])
+def test_fold_algebra_matches_the_whole_sequence(bounds, with_dht):
     c, dO = _case(37, 71)
+    if not with_dht:
+        c.dht = None
     ops = OracleOps()
     segs = [_seg(c, a, b) for a, b in zip(bounds[:-1], bounds[1:])]
     sums = [cp.segment_summary(ops, *s) for s in segs]
@@ -111,3 +114,9 @@ def test_two_gloo_ranks_exchange():
     for key in ("dA_log", "ddt_bias"):  # all-reduced: every rank holds the total
         for r in (0, 1):
             np.testing.assert_allclose(res[r][2][key], g_ref[key], rtol=1e-8, atol=1e-9)
+
+
+def test_segment_summary_needs_square_states():
+    c = synth.make_case(B=1, T=5, H=1, HV=1, K=16, V=8, dtype="fp32", seed=1, h0=True)
+    with pytest.raises(ValueError):
+        cp.segment_summary(OracleOps(), *_seg(c, 0, 5))
