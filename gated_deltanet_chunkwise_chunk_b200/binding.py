@@ -266,7 +266,9 @@ def kda_chunk_workspace_bytes(dims: gdn_dims, varlen: bool, backward: bool = Fal
 def gdn_kda_chunk_fwd(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None, initial_state=None,
                       scale=0.0, output_final_state=True, out=None, final_state=None, workspace=None):
     """Chunkwise KDA forward (per-key-channel gate, long sequences): returns (o, final_state or
-    None).  Arguments as gdn_kda_recurrent_fwd."""
+    None).  Arguments as gdn_kda_recurrent_fwd.  For a gdn_kda_chunk_bwd afterwards, pass a
+    workspace of kda_chunk_workspace_bytes(dims, varlen, backward=True) bytes: the forward then
+    keeps in it what the backward reads."""
     B, T, H, K = q.shape
     HV = v.shape[2]
     Nst = _check_inputs(q, k, v, None, A_log, None, beta, cu_seqlens, initial_state)
