@@ -198,3 +198,25 @@ def test_chunk_backward_algebra_equals_the_oracle(T, strong):
     got = kca.backward(q, k, v, g, A_log, dt_bias, beta, dO, h0=S0, dht=dht)
     for key in ("dq", "dk", "dv", "dbeta", "dg", "dh0"):
         np.testing.assert_allclose(got[key], ref[key], rtol=1e-8, atol=1e-10, err_msg=key)
+
+
+def test_outputs_are_jointly_linear_in_values_and_initial_state():
+    """For fixed keys, queries, gates and beta both recurrences are linear in (v, h0): the
+    oracles' outputs and final states must combine linearly (a nonlinear term in v or S fails)."""
+    rng = np.random.default_rng(51)
+    q, k, v1, g, A_log, dt_bias, beta, S1 = _case(rng, B=1, T=29, H=2, HV=4, K=8, V=6)
+    v2 = rng.standard_normal(v1.shape)
+    S2 = rng.standard_normal(S1.shape)
+    al, be = 0.7, -1.3
+    o1, h1 = kda.recurrent_fwd(q, k, v1, g, A_log, dt_bias, beta, h0=S1)
+    o2, h2 = kda.recurrent_fwd(q, k, v2, g, A_log, dt_bias, beta, h0=S2)
+    o3, h3 = kda.recurrent_fwd(q, k, al * v1 + be * v2, g, A_log, dt_bias, beta, h0=al * S1 + be * S2)
+    np.testing.assert_allclose(o3, al * o1 + be * o2, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(h3, al * h1 + be * h2, rtol=1e-10, atol=1e-12)
+    a = rng.standard_normal(g.shape[:3])
+    dtb = rng.standard_normal(g.shape[2])
+    p1 = oracle.fwd(q, k, v1, a, A_log, dtb, beta, h0=S1)
+    p2 = oracle.fwd(q, k, v2, a, A_log, dtb, beta, h0=S2)
+    p3 = oracle.fwd(q, k, al * v1 + be * v2, a, A_log, dtb, beta, h0=al * S1 + be * S2)
+    np.testing.assert_allclose(p3[0], al * p1[0] + be * p2[0], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(p3[1], al * p1[1] + be * p2[1], rtol=1e-10, atol=1e-12)
