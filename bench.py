@@ -108,7 +108,7 @@ def step_bytes(case, e: int) -> tuple[float, float]:
 
 
 def peaks() -> dict:
-    p = dict(FALLBACK)
+    p = dict(FALLBACK)  # every key present even if the measured file lacks one
     src = "fallback"
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -181,11 +181,13 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- oracle baseline
 def oracle_sample(case, budget_s: float = 12.0) -> dict:
-    """fp64 oracle (fwd + bwd) on the first Ts tokens of every batch row and every head of
-    the workload, Ts doubled from 64 until one run costs about a third of the budget."""
+    """fp64 oracle (fwd + bwd) on a bounded sample of the workload, every head: the first Ts
+    tokens of every batch row (Ts doubled from 64), or for a packed varlen batch its first m
+    sequences (m doubled from 1), grown until one run costs about a third of the budget.
+    Returns the sample's throughput and the measured time of that one sample run."""
     from oracle import oracle
 
-    def run(Ts):
+    def run_dense(Ts):
         sub = dict(q=case.q[:, :Ts], k=case.k[:, :Ts], v=case.v[:, :Ts], a=case.a[:, :Ts],
                    A_log=case.A_log, dt_bias=case.dt_bias, beta=case.beta[:, :Ts])
         t0 = time.perf_counter()
@@ -193,20 +195,41 @@ def oracle_sample(case, budget_s: float = 12.0) -> dict:
         oracle.bwd(**sub, dO=case.dO[:, :Ts], h0=case.h0, dht=case.dht)
         return time.perf_counter() - t0
 
+    def run_varlen(m):
+        cu = case.cu_seqlens[: m + 1]
+        Ts = int(cu[-1])
+        sub = dict(q=case.q[:, :Ts], k=case.k[:, :Ts], v=case.v[:, :Ts], a=case.a[:, :Ts],
+                   A_log=case.A_log, dt_bias=case.dt_bias, beta=case.beta[:, :Ts])
+        h0 = None if case.h0 is None else case.h0[:m]
+        dht = None if case.dht is None else case.dht[:m]
+        t0 = time.perf_counter()
+        oracle.fwd(**sub, cu_seqlens=cu.numpy(), h0=h0)
+        oracle.bwd(**sub, dO=case.dO[:, :Ts], cu_seqlens=cu.numpy(), h0=h0, dht=dht)
+        return time.perf_counter() - t0
+
     if case.cu_seqlens is not None:
-        raise ValueError("the oracle sample uses dense batches")
-    Ts = 64
-    dt = run(Ts)
-    while dt < budget_s / 3 and Ts * 2 <= case.T:
-        Ts *= 2
-        dt = run(Ts)
-    units = case.B * case.HV
+        m, nseq = 1, case.N
+        dt = run_varlen(m)
+        while dt < budget_s / 3 and m * 2 <= nseq:
+            m *= 2
+            dt = run_varlen(m)
+        tok = int(case.cu_seqlens[m])
+        units = m * case.HV
+        what = f"first {m} of {nseq} packed sequences ({tok} of {case.tokens} tokens)"
+    else:
+        Ts = 64
+        dt = run_dense(Ts)
+        while dt < budget_s / 3 and Ts * 2 <= case.T:
+            Ts *= 2
+            dt = run_dense(Ts)
+        tok = case.B * Ts
+        units = case.B * case.HV
+        what = f"{case.B} batch rows, first {Ts} of {case.T} tokens ({tok} tokens)"
     cores = min(os.cpu_count() or 1, units)
-    tok = case.B * Ts
     return {"value": tok / dt / 1e6, "unit": "M tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"fp64 token-by-token oracle fwd+bwd, all {case.HV} value heads x {case.B} "
-                      f"batch rows, first {Ts} of {case.T} tokens ({tok} tokens, {dt:.1f} s)",
-            "seconds": dt}
+            "sample": f"fp64 token-by-token oracle fwd+bwd, all {case.HV} value heads, {what}, "
+                      f"{dt:.2f} s",
+            "seconds": dt, "tokens": tok}
 
 
 # ----------------------------------------------------------------- ranks
@@ -260,6 +283,8 @@ def main():
     ap.add_argument("--workload", default="gdn", choices=["gdn", "kda_chunk", "decode"],
                     help="kda_chunk: only the chunkwise KDA measurement (its T from --T, default 32768); "
                          "decode: only the decode-step measurement")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the lines of the other workloads in the default run")
     ap.add_argument("--ref-budget", type=float, default=90.0,
                     help="seconds of oracle work over the whole --impl reference run")
     args = ap.parse_args()
@@ -291,6 +316,64 @@ def main():
             dist.destroy_process_group()
         return
     case = synth.config_case(args.config, seed=1000 + args.config + 7919 * rank, T=args.T)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+    sampler = ClockSampler(vis[local].strip() if len(vis) > local and vis[local].strip() else local)
+    m = measure_case(gdn, case, dev, args.steps, args.warmup, dist, world, sampler=sampler,
+                     e2e_steps=args.e2e_steps)
+    full = args.config == 2 and args.T is None
+    decode = decode_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"]) if full else None
+    kda = kda_gate_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"]) if full else None
+    kda_decode = decode_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"], kda=True) if full else None
+    kda_chunk = kda_chunk_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"]) if full else None
+
+    line = {
+        "metric": METRIC, "value": m["value"], "unit": "M tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": m["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": case.dtype, "data": "synthetic (seeded N(0,1)/sigmoid/log-uniform inputs; no dataset)",
+        "config": {"workload": case.name, "B": case.B, "T": case.T, "H": case.H, "HV": case.HV,
+                   "K": case.K, "V": case.V, "chunk": C, "global_batch": case.B * world,
+                   "seq_len": case.T, "parallelism": f"dp{world} (independent batches)",
+                   "l2": "no flush: each step streams ~1 GB (inputs alone > 126 MB L2)"},
+    }
+    line.update({k: v for k, v in m.items() if k not in ("value", "ms_per_step")})
+    line.update({"decode": decode, "kda_gate": kda, "kda_decode": kda_decode, "kda_chunk": kda_chunk,
+                 "peaks_source": peaks()["source"]})
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        try:
+            line["cpu_baseline"] = oracle_sample(case)
+            for k in ("seconds", "tokens"):
+                line["cpu_baseline"].pop(k, None)
+        except Exception as ex:  # noqa: BLE001
+            line["cpu_baseline"] = {"error": str(ex)}
+    if full and not args.no_other_configs:
+        # the other workloads of the pages' shapes: same step, same measurements
+        others = {}
+        for idx in (0, 1, 3, 4):
+            oc = synth.config_case(idx, seed=1000 + idx + 7919 * rank)
+            sub = measure_case(gdn, oc, dev, args.steps, args.warmup, dist, world, sampler=None,
+                               e2e_steps=3)
+            sub["config"] = {"workload": oc.name, "B": oc.B, "T": oc.T, "tokens": oc.tokens,
+                             "H": oc.H, "HV": oc.HV, "K": oc.K, "V": oc.V, "dtype": oc.dtype}
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                cb = oracle_sample(oc, budget_s=6.0)
+                sub["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+            others[f"config{idx}"] = sub
+            del oc
+        line["other_workloads"] = others
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def measure_case(gdn, case, dev, steps: int, warmup: int, dist, world: int, sampler=None,
+                 e2e_steps: int = 3) -> dict:
+    """One workload: W warm-up steps, then K timed training steps (forward + backward reading
+    the forward's saved intermediates) and K timed forwards, CUDA events on the launching
+    stream, max over ranks; then a profiled pass (events around every launch) for the
+    per-kernel times and the dominant kernel's roofline, and the end-to-end number."""
     e = 2 if case.dtype == "bf16" else 4
     t = lambda x: None if x is None else x.to(dev).contiguous()
     inp = dict(q=t(case.q), k=t(case.k), v=t(case.v), g_raw=t(case.a), A_log=t(case.A_log),
@@ -332,18 +415,17 @@ def main():
             dist.barrier()
         return a.elapsed_time(b) / n
 
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
-    sampler = ClockSampler(vis[local].strip() if len(vis) > local and vis[local].strip() else local)
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-    sampler.start()
-    time.sleep(0.3)
+    if sampler is not None:
+        sampler.start()
+        time.sleep(0.3)
     n0 = gdn.launch_count()
-    ms = timed(step, args.steps)
-    launches = gdn.launch_count() - n0
-    clocks = sampler.stop()
-    ms_fwd = timed(fwd, max(1, args.steps))
+    ms = timed(step, steps)
+    launches = (gdn.launch_count() - n0) // max(1, steps) * steps
+    clocks = sampler.stop() if sampler is not None else None
+    ms_fwd = timed(fwd, max(1, steps))
     ms, ms_fwd = max_over_ranks([ms, ms_fwd], dist, dev)
 
     # per-kernel device time (separate pass: events around every launch on its stream)
@@ -353,16 +435,8 @@ def main():
     prof = gdn.profile_read()
     gdn.profile(False)
 
-    # end to end through the public API with host buffers
-    e2e = e2e_measure(gdn, case, dev, ws, args.e2e_steps, dist)
-    full = args.config == 2 and args.T is None
-    decode = decode_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"]) if full else None
-    kda = kda_gate_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"]) if full else None
-    kda_decode = decode_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"], kda=True) if full else None
-    kda_chunk = kda_chunk_measure(gdn, dev, pk_hbm=peaks()["hbm_gbs"]) if full else None
-
+    e2e = e2e_measure(gdn, case, dev, ws, e2e_steps, dist)
     tokens = case.tokens
-    value = aggregate_mtok_s(world, tokens, ms)
     pk = peaks()
     fflop, bflop = step_flops_per_token_head(case.K, case.V)
     th = tokens * case.HV
@@ -370,53 +444,40 @@ def main():
     flops = th * (fflop + bflop)
     nbytes = fbytes + bbytes
     t_roof_ds = max(flops / (DATASHEET["tensor_tflops"] * 1e12), nbytes / (DATASHEET["hbm_gbs"] * 1e9))
+    t_roof_b = max(flops / (pk["bf16_tflops"] * 1e12), nbytes / (pk["hbm_gbs"] * 1e9))
     t_roof_m = max(flops / (pk["bf16_tflops_sustained"] * 1e12), nbytes / (pk["hbm_gbs"] * 1e9))
-    roof = kernel_roofline(prof, case, pk)
-
-    line = {
-        "metric": METRIC, "value": round(value, 3), "unit": "M tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": case.dtype, "data": "synthetic (seeded N(0,1)/sigmoid/log-uniform inputs; no dataset)",
-        "config": {"workload": case.name, "B": case.B, "T": case.T, "H": case.H, "HV": case.HV,
-                   "K": case.K, "V": case.V, "chunk": C, "global_batch": case.B * world,
-                   "seq_len": case.T, "parallelism": f"dp{world} (independent batches)",
-                   "l2": "no flush: each step streams ~1 GB (inputs alone > 126 MB L2)"},
+    t_froof = max(th * fflop / (pk["bf16_tflops"] * 1e12), fbytes / (pk["hbm_gbs"] * 1e9))
+    del ws
+    return {
+        "value": round(aggregate_mtok_s(world, tokens, ms), 3), "ms_per_step": round(ms, 4),
         "fwd_mtok_s": round(aggregate_mtok_s(world, tokens, ms_fwd), 3),
         "ms_fwd": round(ms_fwd, 4),
         "step_roofline": {"flops": flops, "bytes": nbytes,
+                          "bound": "tensor" if flops / 2.25e15 >= nbytes / 8e12 else "hbm",
                           "frac_datasheet": round(t_roof_ds / (ms / 1e3), 4),
+                          "frac_measured_burst": round(t_roof_b / (ms / 1e3), 4),
                           "frac_measured": round(t_roof_m / (ms / 1e3), 4),
+                          "fwd_frac_measured_burst": round(t_froof / (ms_fwd / 1e3), 4),
                           "roofline_mtok_s_datasheet": round(tokens / t_roof_ds / 1e6, 2),
-                          "note": "max(FLOP/bf16 peak, bytes/HBM) over the whole fwd+bwd step"},
-        "roofline": roof,
+                          "note": "max(FLOP/bf16 peak, bytes/HBM) over the whole fwd+bwd step; "
+                                  "frac_measured uses the sustained bf16 peak, _burst the burst one"},
+        "roofline": kernel_roofline(prof, case, pk),
         "kernels": {k: {"launches": v[0], "ms_per_step": round(v[1] / 2, 4)} for k, v in prof.items()},
         "gpu_launches": int(launches),
         "e2e": e2e,
-        "decode": decode,
-        "kda_gate": kda,
-        "kda_decode": kda_decode,
-        "kda_chunk": kda_chunk,
         "clocks": clocks,
-        "peaks_source": pk["source"],
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        try:
-            line["cpu_baseline"] = oracle_sample(case)
-            line["cpu_baseline"].pop("seconds", None)
-        except Exception as ex:  # noqa: BLE001
-            line["cpu_baseline"] = {"error": str(ex)}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if dist:
-        dist.barrier()
-        dist.destroy_process_group()
 
 
 def kernel_roofline(prof: dict, case, pk: dict) -> dict | None:
-    """Roofline of the kernel with the largest share of device time: its algorithmic FLOPs
-    and HBM bytes per launch (per-unit figures x units), the bound being whichever of
-    FLOPs / bf16 peak and bytes / HBM bandwidth takes longer."""
+    """Roofline of the kernel with the largest share of device time.  `achieved` is the
+    kernel's algorithmic work per launch over its measured launch time: the FLOPs of its
+    products per token and value head (the method's steps, full 64-row tiles) times the
+    launch's token-heads, against the bf16 tensor peak.  The method's algorithmic bytes do not
+    count the chunk intermediates that pass between kernels, and the chunk kernels' inputs
+    are mostly such intermediates, so their binding bound is the tensor peak.  The bytes the
+    kernel moves under the current kernel split (intermediates included) are reported
+    beside it as `hbm_with_intermediates`."""
     if not prof:
         return None
     name, (launches, total_ms) = max(prof.items(), key=lambda kv: kv[1][1])
@@ -437,19 +498,22 @@ def kernel_roofline(prof: dict, case, pk: dict) -> dict | None:
                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                     "peak_source": "fp32 FFMA: 148 SM x 128 lanes x 2 FLOP x 1.965 GHz"})
         return out
-    t_tc = fl * th / (pk["bf16_tflops"] * 1e12) if fl is not None else 0.0
-    t_hbm = by * units / (pk["hbm_gbs"] * 1e9) if by is not None else 0.0
-    if by is not None and t_hbm >= t_tc:
-        achieved = by * units / per_launch_s / 1e9
-        out.update({"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
-                    "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
-                    "algorithmic_bytes": int(by * units), "bytes_per_unit": int(by),
-                    "peak_source": f"HBM copy, {pk['source']}"})
-    elif fl is not None:
+    if fl is not None:
         achieved = fl * th / per_launch_s / 1e12
         out.update({"bound": "tensor", "achieved": round(achieved, 3), "peak": pk["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": traffic,
-                    "peak_source": f"bf16 burst, {pk['source']}"})
+                    "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4),
+                    "frac_sustained_peak": round(achieved / pk.get("bf16_tflops_sustained",
+                                                                    pk["bf16_tflops"]), 4),
+                    "flops_per_token_head": fl, "flops_per_launch": int(fl * th),
+                    "traffic": traffic,
+                    "peak_source": f"bf16 dense burst, {pk['source']}"})
+    if by is not None:
+        gbs = by * units / per_launch_s / 1e9
+        out["hbm_with_intermediates"] = {
+            "bytes_per_unit": int(by), "bytes_per_launch": int(by * units), "achieved": round(gbs, 1),
+            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+            "note": "tiles this kernel reads and writes once under the current kernel split, "
+                    "inter-kernel intermediates included (not the method's algorithmic bytes)"}
     return out
 
 
@@ -741,29 +805,33 @@ def reference_arm(args, rank, world, dist):
     case = synth.config_case(args.config, seed=1000 + args.config)
     from oracle import oracle
     oracle.build()
-    samples = []
     budget = max(0.5, args.ref_budget / max(1, args.steps + args.warmup))
     info = None
+    secs, toks = [], []
     for i in range(args.warmup + args.steps):
         info = oracle_sample(case, budget_s=budget)
         if i >= args.warmup:
-            samples.append(info["value"])
-    value = statistics.mean(samples)
-    tokens_per_step = case.tokens
-    ms = tokens_per_step / (value * 1e6) * 1e3
+            secs.append(info["seconds"])
+            toks.append(info["tokens"])
+    # one step = one bounded sample of the workload; the time is the measured time of it
+    ms = 1e3 * statistics.mean(secs)
+    tokens_per_step = int(statistics.mean(toks))
+    value = tokens_per_step / (ms / 1e3) / 1e6
     cpu = {k: info[k] for k in ("unit", "cores", "kind", "sample")}
     cpu["value"] = round(value, 6)
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "M tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": round(ms, 3), "tokens_per_step": tokens_per_step,
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": case.name, "B": case.B, "T": case.T, "H": case.H, "HV": case.HV,
                        "K": case.K, "V": case.V, "chunk": C},
             "cpu_baseline": cpu,
             "e2e": {"value": round(value, 6), "unit": "M tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
-            "note": "the reference arm is the fp64 token-by-token oracle on the host cores, "
-                    "each step a bounded sample of the workload (tokens/s of that sample)"}
+            "note": "the reference arm is the fp64 token-by-token oracle on the host cores; each "
+                    "step is a bounded sample of the workload (tokens_per_step tokens, all heads) "
+                    "and ms_per_step its measured time"}
     print(json.dumps(line), flush=True)
     if dist:
         dist.destroy_process_group()

@@ -3,8 +3,9 @@
 Argument marshalling only: it checks torch tensors (device, dtype, contiguity, shape),
 allocates outputs and the workspace with torch, and passes raw pointers plus the current
 CUDA stream to the C entry points of the same names.  Every step of the computation runs
-in the library's CUDA kernels.  There is no fallback: if the shared library is missing,
-importing this module raises.
+in the library's CUDA kernels.  There is no fallback: the shared library is loaded on the
+first call into it (so that processes which only use the seeded input generators never map
+it), and that call raises if the library is missing.
 """
 from __future__ import annotations
 
@@ -24,7 +25,7 @@ GDN_FLAG_BWD_REUSE_FWD = 1
 EXPORTED = ("gdn_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_max_chunks",
             "gdn_build_chunk_indices", "gdn_chunk_table_device", "gdn_device_status",
             "gdn_status_string", "gdn_version", "gdn_launch_count", "gdn_profile",
-            "gdn_profile_read", "gdn_chunk_fwd_noalloc", "gdn_noalloc_scratch_bytes",
+            "gdn_profile_read", "gdn_chunk_fwd_noalloc", "gdn_noalloc_scratch_bytes", "gdn_noalloc_device_status",
             "gdn_recurrent_fwd", "gdn_recurrent_workspace_bytes", "gdn_kda_gate_fwd",
             "gdn_kda_gate_bwd", "gdn_kda_gate_workspace_bytes", "gdn_kda_recurrent_fwd",
             "gdn_kda_chunk_fwd", "gdn_kda_chunk_bwd", "gdn_kda_chunk_workspace_bytes",
@@ -93,6 +94,8 @@ def _load() -> ctypes.CDLL:
     lib.gdn_chunk_fwd_noalloc.restype = I32
     lib.gdn_noalloc_scratch_bytes.argtypes = []
     lib.gdn_noalloc_scratch_bytes.restype = SZ
+    lib.gdn_noalloc_device_status.argtypes = [P]
+    lib.gdn_noalloc_device_status.restype = I32
     lib.gdn_launch_count.argtypes = []
     lib.gdn_launch_count.restype = I64
     lib.gdn_profile.argtypes = [I32]
@@ -102,7 +105,18 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-lib = _load()
+class _Lazy:
+    """The loaded library, opened on first attribute access (raises ImportError if missing)."""
+
+    _lib = None
+
+    def __getattr__(self, name):
+        if _Lazy._lib is None:
+            _Lazy._lib = _load()
+        return getattr(_Lazy._lib, name)
+
+
+lib = _Lazy()
 
 
 def status_string(status: int) -> str:
@@ -408,6 +422,11 @@ def recurrent_workspace_bytes() -> int:
 
 def noalloc_scratch_bytes() -> int:
     return int(lib.gdn_noalloc_scratch_bytes())
+
+
+def noalloc_device_status() -> int:
+    """Status word of the last gdn_chunk_fwd_noalloc call on this device (synchronises)."""
+    return int(lib.gdn_noalloc_device_status(_stream()))
 
 
 def gdn_chunk_bwd(q, k, v, g_raw, A_log, dt_bias, beta, d_o, cu_seqlens=None, initial_state=None,

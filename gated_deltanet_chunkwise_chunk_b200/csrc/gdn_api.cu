@@ -258,6 +258,8 @@ int gdn_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const void* v
   const Plan pl = make_plan(*d, varlen, 0);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) || workspace_bytes < pl.total)
     return GDN_ERR_WORKSPACE;
+  // shapes the tcgen05 path covers never run on the CUDA-core kernels instead
+  if (tc_supported(*d) && !tc_ready()) return GDN_ERR_UNSUPPORTED;
   const Problem p = make_problem(*d, varlen);
   Args a{};
   a.q = q;
@@ -303,6 +305,8 @@ int gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v
   const Plan pl = make_plan(*d, varlen, 1);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) || workspace_bytes < pl.total)
     return GDN_ERR_WORKSPACE;
+  // shapes the tcgen05 path covers never run on the CUDA-core kernels instead
+  if (tc_bwd_supported(*d) && !tc_ready()) return GDN_ERR_UNSUPPORTED;
   const Problem p = make_problem(*d, varlen);
   Args a{};
   a.q = q;

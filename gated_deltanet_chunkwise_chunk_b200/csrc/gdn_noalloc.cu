@@ -6,35 +6,24 @@
 // gdn_chunk_fwd_noalloc runs the same forward as gdn_chunk_fwd with its scratch taken
 // from one file-scope device array of fixed size, reserved when the library is loaded on a
 // device and held until the process exits.
-#include <mutex>
-
 #include "gdn.h"
 
 namespace {
 
 constexpr size_t kScratchBytes = GDN_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 
 // The scratch the forward runs in.  Every call on a device shares it.
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_scratch on the current device, looked up once per device.  The
-// array's name is only a host-side stand-in in host code; its device address must come
-// from cudaGetSymbolAddress with the device current.
+// Device address of g_scratch in the current device's context.  The array's name is only a
+// host-side stand-in in host code; its device address comes from cudaGetSymbolAddress with
+// the device current.  It is looked up on every call (a host-side query, no stream work), so
+// a context that was reset and recreated, where the module and its array may sit elsewhere,
+// is never handed a stale address.
 int scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) return GDN_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) return GDN_ERR_CUDA;
+  *out = p;
   return GDN_OK;
 }
 
@@ -58,6 +47,13 @@ int gdn_chunk_fwd_noalloc(const gdn_dims* d, const void* q, const void* k, const
   // status word and the chunk tables, and every later region is written before it is read.
   return gdn_chunk_fwd(d, q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens, initial_state, o,
                        final_state, scratch, kScratchBytes, stream);
+}
+
+int gdn_noalloc_device_status(void* stream) {
+  void* scratch = nullptr;
+  const int rc = scratch_address(&scratch);
+  if (rc != GDN_OK) return rc;
+  return gdn_device_status(scratch, stream);
 }
 
 }  // extern "C"

@@ -639,15 +639,12 @@ cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const L
 }  // namespace
 
 bool tc_supported(const gdn_dims& d) {
-  static const bool disabled = getenv("GDN_DISABLE_TC") != nullptr;
-  return !disabled && d.dtype == GDN_DTYPE_BF16 && d.K == 128 && d.V == 128 && d.B * d.T > 0 &&
-         encoder() != nullptr;
+  return d.dtype == GDN_DTYPE_BF16 && d.K == 128 && d.V == 128 && d.B * d.T > 0;
 }
 
-bool tc_bwd_supported(const gdn_dims& d) {
-  static const bool disabled = getenv("GDN_DISABLE_TC_BWD") != nullptr;
-  return !disabled && tc_supported(d);
-}
+bool tc_bwd_supported(const gdn_dims& d) { return tc_supported(d); }
+
+bool tc_ready() { return encoder() != nullptr; }
 
 size_t tc_workspace_bytes(const gdn_dims& d, size_t NC, int pass) {
   return tc_bytes(NC, (size_t)d.HV, pass);

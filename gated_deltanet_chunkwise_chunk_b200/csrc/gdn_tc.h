@@ -12,6 +12,10 @@ namespace gdn {
 bool tc_supported(const gdn_dims& d);
 // True when the tcgen05 backward kernels cover them as well.
 bool tc_bwd_supported(const gdn_dims& d);
+// True when the driver's tensor-map encoder is available.  Shapes the tcgen05 path covers
+// never fall back to the CUDA-core kernels: without the encoder their calls fail with
+// GDN_ERR_UNSUPPORTED.
+bool tc_ready();
 // Bytes of the tcgen05 path's own workspace region for NC chunks.
 size_t tc_workspace_bytes(const gdn_dims& d, size_t NC, int pass);
 cudaError_t tc_forward(const Problem& p, const Args& a, const Work& w, void* tc_ws, cudaStream_t s);

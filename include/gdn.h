@@ -57,7 +57,9 @@ extern "C" {
 typedef enum gdn_status {
   GDN_OK = 0,
   GDN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad cu_seqlens */
-  GDN_ERR_UNSUPPORTED = 2,   /* K or V not in {64,128}, unknown dtype */
+  GDN_ERR_UNSUPPORTED = 2,   /* K or V not in {64,128}, unknown dtype; or a bf16 K = V = 128
+                                problem (always run on the tcgen05 kernels) while the driver's
+                                tensor-map encoder cannot be obtained */
   GDN_ERR_WORKSPACE = 3,     /* workspace null/misaligned or smaller than gdn_workspace_bytes */
   GDN_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
   GDN_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up (reported by gdn_device_status) */
@@ -125,10 +127,13 @@ int gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v
  * GPU which loads the library holds until the process exits.  Calls whose
  * gdn_workspace_bytes(d, varlen, 0) exceeds that size return GDN_ERR_WORKSPACE before any
  * launch.  The entry point allocates nothing (no cudaMalloc/cudaFree, no library
- * allocator).  Its first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call before any stream
- * capture.  All calls share the one array and it keeps the last call's contents, so calls
- * that overlap on the GPU (different streams, or host threads) race: serialise them. */
+ * allocator).  Every call looks up the array's device address in the current device's
+ * context (cudaGetSymbolAddress, a host-side query); the first call on a device also loads
+ * the module there, so make that first call before any stream capture.  All calls share the
+ * one array and it keeps the last call's contents, so calls that overlap on the GPU
+ * (different streams, or host threads) race, on the scratch and on the status word it holds:
+ * serialise them.  Problems only the device sees (invalid cu_seqlens, a bounded wait that ran
+ * out) are read back with gdn_noalloc_device_status. */
 #define GDN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 int gdn_chunk_fwd_noalloc(const gdn_dims* d, const void* q, const void* k, const void* v,
                           const float* g_raw, const float* A_log, const float* dt_bias,
@@ -137,6 +142,12 @@ int gdn_chunk_fwd_noalloc(const gdn_dims* d, const void* q, const void* k, const
 
 /* Size in bytes of the array gdn_chunk_fwd_noalloc uses (GDN_NOALLOC_SCRATCH_BYTES). */
 size_t gdn_noalloc_scratch_bytes(void);
+
+/* gdn_device_status for gdn_chunk_fwd_noalloc: synchronises `stream` and returns the status
+ * word the last allocation-free call on the current device left in the shared array
+ * (GDN_OK, GDN_ERR_INVALID_ARG for invalid cu_seqlens, GDN_ERR_TIMEOUT), or GDN_ERR_CUDA if
+ * the array's address cannot be looked up.  No counterpart on the pages (packaging). */
+int gdn_noalloc_device_status(void* stream);
 
 /* Token-by-token (recurrent) forward for decoding and short prefills: the same operation and
  * the same arguments as gdn_chunk_fwd (o for every token, final_state after each sequence's
@@ -168,8 +179,8 @@ size_t gdn_recurrent_workspace_bytes(void);
  * (gdn_dtype: fp32, bf16 or fp16); A_log [H] fp32; dt_bias [H*D] fp32 or NULL (no bias).
  * All buffers on the device, 16-byte aligned; launches on `stream`; allocates nothing.
  * Returns GDN_ERR_INVALID_ARG for null or misaligned pointers or bad sizes (H <= 65535,
- * H*D <= 2^24), GDN_ERR_UNSUPPORTED for an unknown dtype.  The chunkwise KDA attention itself
- * is not provided. */
+ * H*D <= 2^24), GDN_ERR_UNSUPPORTED for an unknown dtype.  The KDA recurrence and its chunkwise
+ * forward and backward are the gdn_kda_* entry points below. */
 int gdn_kda_gate_fwd(int64_t T, int64_t H, int64_t D, int32_t in_dtype, const void* g,
                      const float* A_log, const float* dt_bias, int32_t out_dtype, void* yg,
                      void* stream);

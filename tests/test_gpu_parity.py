@@ -207,3 +207,26 @@ def test_long_sequence_four_times_the_layer_length():
     case = synth.make_case(B=1, T=131072, H=1, HV=2, K=128, V=128, dtype="bf16", seed=77,
                            h0=True, dht=True, name="long_T131072")
     _assert_parity(case)
+
+
+@pytest.mark.parametrize("lengths", [None, [300, 0, 77]])
+def test_bf16_d128_runs_on_the_tensor_core_kernels(lengths):
+    """bf16 with K = V = 128 always takes the tcgen05 kernels (no silent CUDA-core fallback):
+    the per-launch profile of one forward + backward names only tcgen05 and prologue kernels,
+    and every step of the chunk path is among them."""
+    import gated_deltanet_chunkwise_chunk_b200 as gdn
+    case = synth.make_case(B=1 if lengths else 2, T=200, H=2, HV=4, K=128, V=128, dtype="bf16",
+                           seed=61, lengths=lengths, h0=True, dht=True, name="tc_path")
+    gdn.profile(True)
+    try:
+        run_gpu(case)
+        torch.cuda.synchronize()
+        names = set(gdn.profile_read())
+    finally:
+        gdn.profile(False)
+    assert not any(n.startswith("ffma_") for n in names), names
+    tc = {n for n in names if n.startswith("tc_")}
+    assert len(tc) >= 6, names
+    for step in ("wy", "out", "dvlocal", "dqkwg", "wy_bwd"):
+        assert f"tc_{step}" in tc, (step, names)
+    assert any("scan_fwd" in n for n in tc) and any("scan_bwd" in n for n in tc), names
