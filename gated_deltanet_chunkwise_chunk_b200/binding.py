@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libgdn_b200.so")
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(6)
 GDN_DTYPE_FP32, GDN_DTYPE_BF16, GDN_DTYPE_FP16 = 0, 1, 2
 GDN_FLAG_BWD_REUSE_FWD = 1
+GDN_FLAG_TEST_WAIT_TIMEOUT = 1 << 30  # tests of the failure path only
 
 # Every symbol include/gdn.h declares (checked by the tests).
 EXPORTED = ("gdn_workspace_bytes", "gdn_chunk_fwd", "gdn_chunk_bwd", "gdn_max_chunks",
@@ -186,10 +187,13 @@ def _check_inputs(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens, initial_stat
 
 
 def gdn_chunk_fwd(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens=None, initial_state=None,
-                  scale=0.0, output_final_state=True, workspace=None, out=None, final_state=None):
-    """Forward: returns (o, final_state or None).  See include/gdn.h for layouts."""
+                  scale=0.0, output_final_state=True, workspace=None, out=None, final_state=None,
+                  flags=0):
+    """Forward: returns (o, final_state or None).  See include/gdn.h for layouts; `flags` is
+    passed through in gdn_dims.flags."""
     Nst = _check_inputs(q, k, v, g_raw, A_log, dt_bias, beta, cu_seqlens, initial_state)
     dims = make_dims(q, v, cu_seqlens, scale)
+    dims.flags = int(flags)
     ws = _workspace(dims, cu_seqlens is not None, False, workspace, q.device)
     o = out if out is not None else torch.empty(v.shape, dtype=q.dtype, device=q.device)
     ht = None

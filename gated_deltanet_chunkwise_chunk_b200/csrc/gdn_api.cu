@@ -141,6 +141,7 @@ Problem make_problem(const gdn_dims& d, bool varlen) {
   p.varlen = varlen ? 1 : 0;
   p.NCmax = (int)max_chunks(d, varlen);
   p.scale = d.scale > 0.f ? d.scale : 1.f / std::sqrt((float)d.K);
+  p.test_timeout = (d.flags & GDN_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
   return p;
 }
 

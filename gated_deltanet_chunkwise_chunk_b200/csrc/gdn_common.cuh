@@ -20,6 +20,7 @@ struct Problem {
   int varlen;   // 1 when cu_seqlens is used
   int NCmax;    // grid bound on the number of chunks
   float scale;
+  int test_timeout;  // GDN_FLAG_TEST_WAIT_TIMEOUT: the forward pass withholds one arrive (tests only)
 };
 
 // Workspace carve-up (device pointers into the caller's workspace).  Intermediates are

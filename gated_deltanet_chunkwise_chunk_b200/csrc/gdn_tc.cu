@@ -9,6 +9,7 @@
 // Intermediates between kernels are bf16 tiles in HBM, laid out so that one TMA box loads
 // each as a tensor-core operand:  W^T, U~^T, U^T: [unit][128][64];  S (h): [unit][128][128].
 #include <cstdio>
+#include <vector>
 
 #include "gdn_tc_common.cuh"
 
@@ -39,9 +40,10 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
                                                const __grid_constant__ CUtensorMap mk,
                                                const __grid_constant__ CUtensorMap mv,
                                                const __grid_constant__ CUtensorMap mWT,
-                                               const __grid_constant__ CUtensorMap mUtT, int store_T) {
+                                               const __grid_constant__ CUtensorMap mUtT, int store_T,
+                                               int gc0) {
   if (failed(w)) return;
-  const int gc = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
+  const int gc = gc0 + blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
   const int4 e = w.chunk_tab[gc];
   if (e.x < 0) return;
   const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -210,248 +212,6 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
 }
 
 // ======================================================================================
-// Sequential state scan.  The rows of S (value index v) evolve independently: row v of
-//   U = U~ - W S^T   and   S' = e^{G_C} S + U^T diag(e^{G_C-G}) K
-// only involves row v of S and column v of U~.  So the scan is split over value slices:
-// CTA (sequence, value head, z) carries rows v0 = 32z .. v0+31 (4 CTAs per head), which
-// quarters the work on each chunk step of the sequential chain and fills 4x more SMs.
-// The products are taken transposed, so that the 32-row slice is the N side:
-//   MMA1: D1 = W S_z^T           (M=64 i, N=32 v, K=128 k)     W^T tile as MN-major A
-//   U = U~ - D1;  Ud = diag(e^{G_C-G}) U      (bf16 [32 v][64 i] tiles, K-major B)
-//   MMA2: D2 = K^T Ud            (M=128 k, N=32 v, K=64 i)     K tile as MN-major A
-//   S_z^T = e^{G_C} S_z^T + D2   (thread k keeps S[v0..v0+31][k] in fp32 registers)
-// 128 threads: thread 0 issues the MMAs, thread 32 the TMA stores (and waits on them; bulk
-// groups are per thread), thread 64 the TMA loads; two CTA-wide barriers per chunk step.
-// The slice of S entering each chunk and the slice of U^T are written out by TMA stores;
-// the chunk's W^T, U~^T slice and K tiles are prefetched one chunk ahead (double buffer).
-// ======================================================================================
-struct ScanSmem {
-  static constexpr int BUF = 0;                               // 2 x {W^T, K, U~^T slice}
-  static constexpr int BUF_BYTES = 2 * TILE128 + TILE_VS;
-  static constexpr int S = 2 * BUF_BYTES;                     // 2 x [32][128] bf16 state slice
-  static constexpr int UD = S + 4 * TILE_VS;                  // [32][64] Ud^T slice
-  static constexpr int UO = UD + TILE_VS;                     // 2 x [32][64] U^T staging
-  static constexpr int DEC = UO + 2 * TILE_VS;                // 2 x 64 floats e^{G_C - G_i}
-  static constexpr int EGC = DEC + 2 * 256;                   // 2 floats e^{G_C}
-  static constexpr int TOTAL = EGC + 64;
-};
-
-__global__ void __launch_bounds__(128) k_tc_scan_fwd(Problem p, Args a, Work w, TcWork t,
-                                                     const __grid_constant__ CUtensorMap mk,
-                                                     const __grid_constant__ CUtensorMap mWT,
-                                                     const __grid_constant__ CUtensorMap mUtT32,
-                                                     const __grid_constant__ CUtensorMap mUT32,
-                                                     const __grid_constant__ CUtensorMap mh32,
-                                                     int write_final) {
-  if (failed(w)) return;
-  const int n = blockIdx.x, hv = blockIdx.y, hk = hv / p.G, v0 = VS * blockIdx.z;
-  const int4 sq = w.seq_tab[n];
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  extern __shared__ unsigned char smraw[];
-  unsigned char* sm = align1k(smraw);
-  unsigned char* sUd = sm + ScanSmem::UD;
-  float* sDecb = reinterpret_cast<float*>(sm + ScanSmem::DEC);
-  float* sEGC = reinterpret_cast<float*>(sm + ScanSmem::EGC);
-  __shared__ uint64_t barT[2], barM1, barM2;
-  __shared__ uint32_t tslot;
-  int* err = w.status;
-  if (tid == 0) {
-    mbar_init(&barT[0], 1);
-    mbar_init(&barT[1], 1);
-    mbar_init(&barM1, 1);
-    mbar_init(&barM2, 1);
-    mbar_fence_init();
-  }
-  __syncthreads();
-  if (warp == 0) {
-    tmem_alloc(&tslot, 64);
-    tmem_relinquish();
-  }
-  // thread k = tid holds S[v0 + i][k], i < 32 (initial state h0[k][v] = S[v][k], fp32)
-  float S[VS];
-  const size_t st = ((size_t)n * p.HV + hv) * D * D + (size_t)tid * D + v0;
-#pragma unroll
-  for (int i = 0; i < VS; i += 4) {
-    const float4 x = a.h0 ? *reinterpret_cast<const float4*>(a.h0 + st + i) : make_float4(0, 0, 0, 0);
-    S[i] = x.x; S[i + 1] = x.y; S[i + 2] = x.z; S[i + 3] = x.w;
-  }
-  // element (v, k) of a [32][128] slice tile: the thread's column k, rows i < 32
-  const uint32_t scol = (uint32_t)((tid >> 6) * TILE_VS + ((tid & 7) << 1));
-  const int sj = (tid & 63) >> 3;
-#define S_OFF(i) (scol + (uint32_t)((i) * 128 + (((sj) ^ ((i) & 7)) << 4)))
-#pragma unroll
-  for (int i = 0; i < VS; ++i) st_bf16(sm + ScanSmem::S, S_OFF(i), S[i]);
-  auto issue = [&](int c) {
-    const int gc = sq.x + c, buf = c & 1;
-    const int tok = sq.z + 64 * c;  // chunks of a sequence are consecutive, 64 tokens apart
-    unsigned char* b = sm + ScanSmem::BUF + buf * ScanSmem::BUF_BYTES;
-    const int row = (gc * p.HV + hv) * D;
-    mbar_expect_tx(&barT[buf], 2 * TILE128 + TILE_VS);
-    tma_load_3d(b, &mWT, 0, row, 0, &barT[buf]);
-    tma_load_3d(b + TILE128, &mk, 0, hk, tok, &barT[buf]);
-    tma_load_3d(b + TILE128 + TILE64, &mk, 64, hk, tok, &barT[buf]);
-    tma_load_3d(b + 2 * TILE128, &mUtT32, 0, row + v0, 0, &barT[buf]);
-  };
-  const size_t vec0 = ((size_t)hv * p.NCmax + sq.x) * 64;  // chunk vectors of this sequence
-  if (tid == 64 && sq.y > 0) issue(0);
-  if (tid >= 64 && sq.y > 0) {
-    sDecb[tid - 64] = w.Dec[vec0 + tid - 64];
-    if (tid == 127) sEGC[0] = w.EG[vec0 + 63];
-  }
-  fence_proxy_async();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tb = tslot;
-  const uint32_t tD1 = taddr(tb, 0, 0), tD2 = taddr(tb, 0, 32);
-  // U-phase element mapping (16-lane TMEM loads of the M=64 accumulator): rows
-  // i = 16 warp + lane/4 (+8), columns v = 8j + 2(lane%4) + {0,1}
-  const int ui = 16 * warp + (lane >> 2), uv = 2 * (lane & 3);
-  // per-thread byte offsets of the U-phase elements in a [32][64] slice tile:
-  // element (v = 8j + uv + e, i = ui + 8r) sits at uoff[r][e] + 1024 j
-  uint32_t uoff[2][2];
-#pragma unroll
-  for (int r = 0; r < 2; ++r)
-#pragma unroll
-    for (int e = 0; e < 2; ++e)
-      uoff[r][e] = (uint32_t)((uv + e) * 128 + (((2 * warp + r) ^ (uv + e)) << 4) + ((lane >> 2) << 1));
-  uint32_t phT[2] = {0, 0}, phM = 0;
-  bool ok = true;
-  for (int c = 0; c < sq.y; ++c) {
-    const int gc = sq.x + c, buf = c & 1;
-    const bool more = c + 1 < sq.y;
-    unsigned char* b = sm + ScanSmem::BUF + buf * ScanSmem::BUF_BYTES;
-    unsigned char* sS = sm + ScanSmem::S + buf * 2 * TILE_VS;       // S slice entering chunk c
-    unsigned char* sSn = sm + ScanSmem::S + (buf ^ 1) * 2 * TILE_VS;
-    const float* sDec = sDecb + buf * 64;
-    const int srow = (gc * p.HV + hv) * D + v0;
-    bool okt = true;
-    if (tid == 0) {  // MMA1: D1 = W S_z^T
-      okt = mbar_wait(&barT[buf], phT[buf], err);
-      if (okt) {
-        const uint64_t da = desc_mnmajor(smem_u32(b), 0, TILE128);
-        const uint64_t db = desc_kmajor(smem_u32(sS), 0, TILE_VS);
-        constexpr uint32_t id = idesc_bf16(64, VS, true, false);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-          mma_bf16(tD1, da + mnstep_off(s), db + kstep_off(s, TILE_VS), id, s > 0);
-        mma_commit(&barM1);
-      }
-    } else if (tid == 32) {  // S slice entering this chunk -> h;  U^T slice of chunk c-1
-      tma_store_3d(&mh32, sS, 0, srow, 0);
-      tma_store_3d(&mh32, sS + TILE_VS, 64, srow, 0);
-      if (c > 0) tma_store_3d(&mUT32, sm + ScanSmem::UO + (buf ^ 1) * TILE_VS, 0, srow - p.HV * D, 0);
-      tma_store_commit();
-    } else if (tid == 64 && more) {
-      issue(c + 1);
-    }
-    float dn = 0.f, en = 0.f;  // next chunk's decay vectors, stored at the end of this step
-    if (tid >= 64 && more) {
-      dn = w.Dec[vec0 + (size_t)(c + 1) * 64 + tid - 64];
-      if (tid == 127) en = w.EG[vec0 + (size_t)(c + 1) * 64 + 63];
-    }
-    // while MMA1 runs: this thread's U~ elements and decay factors
-    okt = okt && mbar_wait(&barT[buf], phT[buf], err);
-    phT[buf] ^= 1;
-    float u[16];
-    {
-      const unsigned char* ut = b + 2 * TILE128;
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) u[4 * j + 2 * r + e] = ld_bf16(ut, uoff[r][e] + 1024 * j);
-    }
-    const float dec0 = sDec[ui], dec1 = sDec[ui + 8];
-    okt = okt && mbar_wait(&barM1, phM, err);
-    tc_fence_after();
-    {  // U = U~ - D1 (kept for the U^T staging); Ud = e^{G_C-G_i} U -> MMA2 operand
-      float d[16];
-      tmem_ld16dp_x4(taddr(tb, 32 * warp, 0), d);
-      tmem_wait_ld();
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int q = 4 * j + 2 * r + e;
-            u[q] -= d[q];
-            st_bf16(sUd, uoff[r][e] + 1024 * j, u[q] * (r ? dec1 : dec0));
-          }
-    }
-    // the stores of chunk c-1 (h, and U^T of c-2) must be done reading before the barrier
-    // below releases writes into their buffers (the next-state tile, this U^T staging)
-    if (tid == 32) tma_store_wait_read<1>();
-    fence_proxy_async();
-    tc_fence_before();
-    ok = __syncthreads_and(ok && okt);
-    tc_fence_after();
-    if (!ok) break;
-    if (tid == 0) {  // MMA2: D2 = K^T Ud
-      const uint64_t da = desc_mnmajor(smem_u32(b + TILE128), 0, TILE64);
-      const uint64_t db = desc_kmajor(smem_u32(sUd), 0, TILE_VS);
-      constexpr uint32_t id = idesc_bf16(128, VS, true, false);
-#pragma unroll
-      for (int s = 0; s < 4; ++s)
-        mma_bf16(tD2, da + mnstep_off(s), db + kstep_off(s, TILE_VS), id, s > 0);
-      mma_commit(&barM2);
-    }
-    {  // while MMA2 runs: U^T staging (stored by TMA at the start of the next step)
-      unsigned char* sUo = sm + ScanSmem::UO + buf * TILE_VS;
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) st_bf16(sUo, uoff[r][e] + 1024 * j, u[4 * j + 2 * r + e]);
-    }
-    okt = mbar_wait(&barM2, phM, err);
-    phM ^= 1;
-    tc_fence_after();
-    {
-      const float eg = sEGC[buf];
-      float d[VS];
-      tmem_ld16(taddr(tb, 32 * warp, 32), d);
-      tmem_ld16(taddr(tb, 32 * warp, 48), d + 16);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < VS; ++i) {
-        S[i] = eg * S[i] + d[i];
-        st_bf16(sSn, S_OFF(i), S[i]);  // its last reader, the h store of chunk c-1, is done
-      }
-    }
-    if (tid >= 64 && more) {
-      sDecb[(buf ^ 1) * 64 + tid - 64] = dn;
-      if (tid == 127) sEGC[buf ^ 1] = en;
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    ok = __syncthreads_and(ok && okt);
-    tc_fence_after();
-    if (!ok) break;
-  }
-#undef S_OFF
-  if (tid == 32) {
-    if (ok && sq.y > 0) {  // U^T slice of the last chunk
-      const int c = sq.y - 1;
-      tma_store_3d(&mUT32, sm + ScanSmem::UO + (c & 1) * TILE_VS, 0, ((sq.x + c) * p.HV + hv) * D + v0, 0);
-      tma_store_commit();
-    }
-    tma_store_wait0();
-  }
-  if (ok && write_final && a.ht) {
-#pragma unroll
-    for (int i = 0; i < VS; i += 4)
-      *reinterpret_cast<float4*>(a.ht + st + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tslot, 64);
-}
-
-// ======================================================================================
 // chunk_fwd_o.  One CTA (256 threads) per (chunk, value head):
 //   X = Q S^T (M=64, N=128), QK = Q K^T (M=64, N=64) -> P = QK * Gam (bf16 tile)
 //   Y = P U (M=64, N=128, B = U^T K-major);  O = scale (e^{G_i} X + Y)
@@ -460,9 +220,9 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
                                                 const __grid_constant__ CUtensorMap mq,
                                                 const __grid_constant__ CUtensorMap mk,
                                                 const __grid_constant__ CUtensorMap mUT,
-                                                const __grid_constant__ CUtensorMap mh) {
+                                                const __grid_constant__ CUtensorMap mh, int gc0) {
   if (failed(w)) return;
-  const int gc = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
+  const int gc = gc0 + blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
   const int4 e = w.chunk_tab[gc];
   if (e.x < 0) return;
   const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -508,8 +268,9 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
   if (ok && tid == 0) {
     const uint32_t q = smem_u32(sQ), k = smem_u32(sK), h = smem_u32(sH);
     for (int s = 0; s < 8; ++s) {
-      mma_bf16(taddr(tb, 0, 0), desc_kmajor(q, s, TILE64), desc_kmajor(h, s, TILE128),
-               idesc_bf16(64, 128, false, false), s > 0);
+      // S is stored transposed ([k][v]): an MN-major B operand
+      mma_bf16(taddr(tb, 0, 0), desc_kmajor(q, s, TILE64), desc_mnmajor(h, s, TILE128),
+               idesc_bf16(64, 128, false, true), s > 0);
       mma_bf16(taddr(tb, 0, 128), desc_kmajor(q, s, TILE64), desc_kmajor(k, s, TILE64),
                idesc_bf16(64, 64, false, false), s > 0);
     }
@@ -597,9 +358,6 @@ Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
   L.ok &= map_rows(&L.m.UtT, L.t.UtT, urows, 64, 128);
   L.ok &= map_rows(&L.m.UT, L.t.UT, urows, 64, 128);
   L.ok &= map_rows(&L.m.h, L.t.h, urows, 128, 128);
-  L.ok &= map_rows(&L.m.UtT32, L.t.UtT, urows, 64, VS);
-  L.ok &= map_rows(&L.m.UT32, L.t.UT, urows, 64, VS);
-  L.ok &= map_rows(&L.m.h32, L.t.h, urows, 128, VS);
   if (pass == 1) {
     const uint64_t trows = (uint64_t)p.NCmax * p.HV * 64;
     L.ok &= map_rows(&L.m.dUlT, L.t.dUlT, urows, 64, 128);
@@ -608,10 +366,6 @@ Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
     L.ok &= map_rows(&L.m.dh, L.t.dh, urows, 128, 128);
     L.ok &= map_rows(&L.m.dW, L.t.dW, trows, 128, 64);
     L.ok &= map_rows(&L.m.Tm, L.t.Tm, 2 * trows, 64, 64);
-    L.ok &= map_rows(&L.m.dUlT32, L.t.dUlT, urows, 64, VS);
-    L.ok &= map_rows(&L.m.dUT32, L.t.dUT, urows, 64, VS);
-    L.ok &= map_rows(&L.m.dUTl32, L.t.dUTl, urows, 64, VS);
-    L.ok &= map_rows(&L.m.dh32, L.t.dh, urows, 128, VS);
   }
   return L;
 }
@@ -619,19 +373,45 @@ Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
 cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const Launch& L,
                          bool bwd_prep, cudaStream_t s) {
   if (!L.ok) return cudaErrorInvalidValue;
+  const size_t out_smem = 1024 + 6 * TILE64 + 3 * TILE128 + 256;
+  auto wy = [&](int c0, int c1, cudaStream_t st) {
+    return tgo("tc_wy", k_tc_wy, dim3(c1 - c0, p.HV), 256, (size_t)1024 + WySmem::TOTAL, st, p, w,
+               L.t, L.m.k, L.m.v, L.m.WT, L.m.UtT, 1, c0);
+  };
+  auto out = [&](int c0, int c1, cudaStream_t st) {
+    return tgo("tc_out", k_tc_out, dim3(c1 - c0, p.HV), 256, out_smem, st, p, a, w, L.t, L.m.q,
+               L.m.k, L.m.UT, L.m.h, c0);
+  };
+  float* ht = bwd_prep ? nullptr : a.ht;
+  const Segments sg = segments(p);
   cudaError_t e;
-  const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV, NVS);
-  if ((e = tgo("tc_wy", k_tc_wy, gu, 256, (size_t)1024 + WySmem::TOTAL, s, p, w, L.t, L.m.k, L.m.v,
-               L.m.WT, L.m.UtT, 1)))
-    return e;
-  Args a2 = a;
-  if ((e = tgo("tc_scan_fwd", k_tc_scan_fwd, gs, 128, (size_t)1024 + ScanSmem::TOTAL, s, p, a2, w,
-              L.t, L.m.k, L.m.WT, L.m.UtT32, L.m.UT32, L.m.h32, bwd_prep ? 0 : 1)))
-    return e;
-  if (!bwd_prep) {
-    const size_t out_smem = 1024 + 6 * TILE64 + 3 * TILE128 + 256;
-    if ((e = tgo("tc_out", k_tc_out, gu, 256, out_smem, s, p, a, w, L.t, L.m.q, L.m.k, L.m.UT, L.m.h)))
-      return e;
+  if (sg.n == 1) {
+    if ((e = wy(0, p.NCmax, s))) return e;
+    if ((e = tc_scan_fwd(p, a, w, L.t, L.m, ScanRange{0, p.NCmax, a.h0, ht}, s))) return e;
+    if (!bwd_prep && (e = out(0, p.NCmax, s))) return e;
+    return cudaSuccess;
+  }
+  // Segments of the sequence's chunks: the pass over segment i (on the side stream) runs
+  // while the WY kernels of later segments and the outputs of earlier ones run on `s`.
+  SideLock side;
+  if (!side.ok()) return cudaErrorInvalidResourceHandle;
+  cudaStream_t hs = side.stream();
+  if ((e = side.fork(s))) return e;
+  std::vector<cudaEvent_t> wy_done(sg.n), scan_done(sg.n);
+  for (int i = 0; i < sg.n; ++i) {
+    if ((e = wy(sg.c[i], sg.c[i + 1], s))) return e;
+    if ((e = side.record(s, &wy_done[i]))) return e;
+  }
+  for (int i = 0; i < sg.n; ++i) {
+    if ((e = cudaStreamWaitEvent(hs, wy_done[i], 0))) return e;
+    const ScanRange r{sg.c[i], sg.c[i + 1], i == 0 ? a.h0 : L.t.hand,
+                      i + 1 == sg.n ? ht : L.t.hand};
+    if ((e = tc_scan_fwd(p, a, w, L.t, L.m, r, hs))) return e;
+    if ((e = side.record(hs, &scan_done[i]))) return e;
+  }
+  for (int i = 0; i < sg.n; ++i) {
+    if ((e = cudaStreamWaitEvent(s, scan_done[i], 0))) return e;
+    if (!bwd_prep && (e = out(sg.c[i], sg.c[i + 1], s))) return e;
   }
   return cudaSuccess;
 }

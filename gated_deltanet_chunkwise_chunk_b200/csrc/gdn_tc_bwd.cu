@@ -1,4 +1,4 @@
-// tcgen05 backward kernels (bf16, K = V = 128).  Per chunk (64 tokens) and value head, with
+// tcgen05 backward kernels (bf16, K = V = 128; the reverse state pass is in gdn_tc_scan.cu).  Per chunk (64 tokens) and value head, with
 // S the state entering the chunk, dS' = dL/dS leaving it, P = (Q K^T) * Gam (lower incl.
 // diagonal), D_j = e^{G_C - G_j}:
 //   dv_local  dU_loc = scale P^T dO
@@ -9,6 +9,8 @@
 //             dv = beta dY;  dbeta;  dk += diag(beta e^G) dX + dAs K + dAs^T K;  dG terms
 // (X = diag(beta e^G) K, Y = diag(beta) V, dAs = dA * Gam * beta_i).  Column sums go through
 // shared memory in a fixed order, so results are bitwise reproducible.
+#include <vector>
+
 #include "gdn_tc_common.cuh"
 
 namespace gdn {
@@ -27,9 +29,9 @@ __device__ __forceinline__ float warp_sum(float x) {
 __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
                                                     const __grid_constant__ CUtensorMap mq,
                                                     const __grid_constant__ CUtensorMap mk,
-                                                    const __grid_constant__ CUtensorMap mdO) {
+                                                    const __grid_constant__ CUtensorMap mdO, int gc0) {
   if (failed(w)) return;
-  const int gc = blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
+  const int gc = gc0 + blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
   const int4 e = w.chunk_tab[gc];
   if (e.x < 0) return;
   const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -138,329 +140,6 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
 }
 
 // ======================================================================================
-// Reverse state scan.  As in the forward, the rows v of dS evolve independently, so CTA
-// (sequence, value head, z) carries the slice dS[v0 .. v0+31][:] (v0 = 32z), with the
-// products taken transposed (the slice is the N side).  Thread k keeps dS[v0+i][k] (i < 32)
-// in fp32 registers.  The operands that carry the chain (dS and dU) are compensated bf16
-// pairs (hi + lo), and dU^T is written out as such a pair.  Tiles are single-buffered: each
-// group is reloaded for the next chunk as soon as its last reader is done.
-//   MMA1:  E = K dS_z^T                                (M=64 j, N=32 v, K=128 k)
-//   dU = dU_loc + diag(e^{G_C-G}) E                    (bf16 hi/lo [32 v][64 j] tiles)
-//   MMA2:  F' = Q^T (-scale diag(e^G) dO_z) + W^T dU   (M=128 k, N=32 v, K=64 i)
-//   dS_z^T = e^{G_C} dS_z^T - F'
-// A tensor-core instruction costs about the same at N=32 and N=64 here, so each hi/lo pair
-// is one N=64 operand (hi rows, then lo rows) and the two halves of the result are summed in
-// the epilogue: 8 + 4 + 4 instructions per chunk instead of 16 + 4 + 8.
-// ======================================================================================
-struct BwdScanSmem {
-  static constexpr int K = 0, Q = 2 * TILE64, O = 4 * TILE64;  // [64][128], [64][128], [64][64]
-  static constexpr int W = 5 * TILE64;                          // W^T [128][64]
-  static constexpr int UL = W + TILE128;                        // dU_loc^T slice [32][64]
-  // dS slice as a compensated pair stacked along N: k-block j (64 k) at SHL + 8K j holds the
-  // hi rows [32][64] then the lo rows, so one N=64 operand carries both parts
-  static constexpr int SHL = UL + TILE_VS;
-  // -scale e^G dO^T slice [32][64] followed by 32 zero rows (an N=64 operand whose second
-  // half initialises the lo columns of the accumulator)
-  static constexpr int OSZ = SHL + 4 * TILE_VS;
-  static constexpr int UHL = OSZ + 2 * TILE_VS;                 // 2 x {dU^T hi, lo} [32][64] each
-  static constexpr int DEC = UHL + 4 * TILE_VS;                 // 2 x 64: e^{G_C - G_j}
-  static constexpr int EG = DEC + 512;                          // 2 x 64: scale e^{G_i} (0 past L)
-  static constexpr int EGC = EG + 512;                          // 2 floats e^{G_C}
-  static constexpr int TOTAL = EGC + 64;
-};
-
-// Roles as in the forward scan: thread 0 MMAs, thread 32 TMA stores, thread 64 TMA loads;
-// two CTA-wide barriers per chunk step.
-__global__ void __launch_bounds__(256) k_tc_scan_bwd(Problem p, Args a, Work w, TcWork t,
-                                                     const __grid_constant__ CUtensorMap mq,
-                                                     const __grid_constant__ CUtensorMap mk,
-                                                     const __grid_constant__ CUtensorMap mdO,
-                                                     const __grid_constant__ CUtensorMap mWT,
-                                                     const __grid_constant__ CUtensorMap mdUlT32,
-                                                     const __grid_constant__ CUtensorMap mdUT32,
-                                                     const __grid_constant__ CUtensorMap mdUTl32,
-                                                     const __grid_constant__ CUtensorMap mdh32) {
-  if (failed(w)) return;
-  const int n = blockIdx.x, hv = blockIdx.y, hk = hv / p.G, v0 = VS * blockIdx.z;
-  const int4 sq = w.seq_tab[n];
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int wq = warp & 3, wg = warp >> 2;   // TMEM lane quarter, column half of the slice
-  const int kk = tid & 127, vc = 16 * wg;    // this thread: column kk of dS, slice rows vc..vc+15
-  extern __shared__ unsigned char smraw[];
-  unsigned char* sm = align1k(smraw);
-  unsigned char* sK = sm + BwdScanSmem::K;
-  unsigned char* sQ = sm + BwdScanSmem::Q;
-  unsigned char* sO = sm + BwdScanSmem::O;
-  unsigned char* sW = sm + BwdScanSmem::W;
-  unsigned char* sUL = sm + BwdScanSmem::UL;
-  unsigned char* sSHL = sm + BwdScanSmem::SHL;
-  unsigned char* sOS = sm + BwdScanSmem::OSZ;
-  float* sDecb = reinterpret_cast<float*>(sm + BwdScanSmem::DEC);
-  float* sEGb = reinterpret_cast<float*>(sm + BwdScanSmem::EG);
-  float* sEGC = reinterpret_cast<float*>(sm + BwdScanSmem::EGC);
-  __shared__ uint64_t barK, barQO, barW, barU, barM1, barM2;
-  __shared__ uint32_t tslot;
-  int* err = w.status;
-  if (tid == 0) {
-    mbar_init(&barK, 1);
-    mbar_init(&barQO, 1);
-    mbar_init(&barW, 1);
-    mbar_init(&barU, 1);
-    mbar_init(&barM1, 1);
-    mbar_init(&barM2, 1);
-    mbar_fence_init();
-  }
-  __syncthreads();
-  if (warp == 0) {
-    tmem_alloc(&tslot, 128);
-    tmem_relinquish();
-  }
-  float S[16];
-  const size_t st = ((size_t)n * p.HV + hv) * D * D + (size_t)kk * D + v0 + vc;
-#pragma unroll
-  for (int i = 0; i < 16; i += 4) {
-    const float4 x = a.dht ? *reinterpret_cast<const float4*>(a.dht + st + i) : make_float4(0, 0, 0, 0);
-    S[i] = x.x; S[i + 1] = x.y; S[i + 2] = x.z; S[i + 3] = x.w;
-  }
-  const uint32_t scol = (uint32_t)((kk >> 6) * 2 * TILE_VS + ((kk & 7) << 1) + vc * 128);
-  const int sj = (kk & 63) >> 3;
-#define S_OFF(i) (scol + (uint32_t)((i) * 128 + (((sj) ^ ((i) & 7)) << 4)))
-  auto store_dS = [&]() {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const bf16 h = __float2bfloat16_rn(S[i]);
-      st_bf16_raw(sSHL, S_OFF(i), h);
-      st_bf16_raw(sSHL + TILE_VS, S_OFF(i), __float2bfloat16_rn(S[i] - __bfloat162float(h)));
-    }
-  };
-  store_dS();
-  for (int i = tid; i < TILE_VS / 16; i += 256)  // the zero half of the scaled-dO operand
-    reinterpret_cast<uint4*>(sOS + TILE_VS)[i] = make_uint4(0, 0, 0, 0);
-  auto row_of = [&](int c) { return ((sq.x + c) * p.HV + hv) * D; };
-  auto tok_of = [&](int c) { return sq.z + 64 * c; };
-  const int ocol = v0 & ~63, vo = v0 & 63;  // dO column block holding the slice, offset in it
-  auto issue_K = [&](int c) {
-    mbar_expect_tx(&barK, 2 * TILE64);
-    tma_load_3d(sK, &mk, 0, hk, tok_of(c), &barK);
-    tma_load_3d(sK + TILE64, &mk, 64, hk, tok_of(c), &barK);
-  };
-  auto issue_QO = [&](int c) {
-    mbar_expect_tx(&barQO, 3 * TILE64);
-    tma_load_3d(sQ, &mq, 0, hk, tok_of(c), &barQO);
-    tma_load_3d(sQ + TILE64, &mq, 64, hk, tok_of(c), &barQO);
-    tma_load_3d(sO, &mdO, ocol, hv, tok_of(c), &barQO);
-  };
-  auto issue_W = [&](int c) {
-    mbar_expect_tx(&barW, TILE128);
-    tma_load_3d(sW, &mWT, 0, row_of(c), 0, &barW);
-  };
-  auto issue_U = [&](int c) {
-    mbar_expect_tx(&barU, TILE_VS);
-    tma_load_3d(sUL, &mdUlT32, 0, row_of(c) + v0, 0, &barU);
-  };
-  const size_t vec0 = ((size_t)hv * p.NCmax + sq.x) * 64;  // chunk vectors of this sequence
-  auto len_of = [&](int c) { return min(64, sq.w - 64 * c); };
-  if (tid == 64 && sq.y > 0) {
-    issue_K(sq.y - 1);
-    issue_QO(sq.y - 1);
-    issue_W(sq.y - 1);
-    issue_U(sq.y - 1);
-  }
-  const bool vec_thread = tid >= 128 && tid < 192;  // loads the per-chunk vectors
-  if (vec_thread && sq.y > 0) {
-    const int c = sq.y - 1, j = tid - 128;
-    const size_t o = vec0 + (size_t)c * 64 + j;
-    sDecb[j] = w.Dec[o];
-    const float eg = w.EG[o];
-    sEGb[j] = j < len_of(c) ? p.scale * eg : 0.f;
-    if (j == 63) sEGC[0] = eg;
-  }
-  fence_proxy_async();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tb = tslot;
-  // TMEM: E (M=64) hi/lo parts in columns [0,32) / [32,64); F' (M=128) in [64,96) / [96,128)
-  const uint32_t tE = taddr(tb, 0, 0), tF = taddr(tb, 0, 64);
-  // U-phase elements (this warpgroup's 16 of the 32 columns): rows j' = 16 wq + lane/4 (+8 r),
-  // columns v = vc + 8j + 2(lane%4) + e (j < 2), at byte offset uoff[r][e] + 1024 (2 wg + j)
-  const int ui = 16 * wq + (lane >> 2), uv = 2 * (lane & 3);
-  uint32_t uoff[2][2];
-#pragma unroll
-  for (int r = 0; r < 2; ++r)
-#pragma unroll
-    for (int e = 0; e < 2; ++e)
-      uoff[r][e] = (uint32_t)(2048 * wg + (uv + e) * 128 + (((2 * wq + r) ^ (uv + e)) << 4) +
-                              ((lane >> 2) << 1));
-  uint32_t ph = 0, phM = 0;  // the tile barriers complete once per chunk, barM1/barM2 once each
-  bool ok = true;
-  for (int idx = 0; idx < sq.y; ++idx) {
-    const int c = sq.y - 1 - idx, buf = idx & 1;
-    const bool more = idx + 1 < sq.y;
-    const int L = len_of(c);
-    const int srow = row_of(c) + v0;
-    const float* sDec = sDecb + buf * 64;
-    const float* sEG = sEGb + buf * 64;
-    unsigned char* sUH = sm + BwdScanSmem::UHL + buf * 2 * TILE_VS;   // hi rows, then lo rows
-    unsigned char* sULo = sUH + TILE_VS;
-    bool okt = true;
-    if (L < 64) {  // ragged chunk: K rows past its end are zeroed before the chain MMA
-      okt = mbar_wait(&barK, ph, err);
-      zero_tail_rows(sK, L, tid, 256);
-      fence_proxy_async();
-      __syncthreads();
-    }
-    if (tid == 0) {  // MMA1 (the chain): E = K dS_z^T with the compensated dS pair
-      okt = okt && mbar_wait(&barK, ph, err);
-      if (okt) {
-        const uint64_t dk = desc_kmajor(smem_u32(sK), 0, TILE64);
-        const uint64_t dhl = desc_kmajor(smem_u32(sSHL), 0, 2 * TILE_VS);
-        constexpr uint32_t id = idesc_bf16(64, 2 * VS, false, false);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)  // [E_hi | E_lo] = K [dS_hi; dS_lo]^T
-          mma_bf16(tE, dk + kstep_off(s, TILE64), dhl + kstep_off(s, 2 * TILE_VS), id, s > 0);
-        mma_commit(&barM1);
-      }
-    } else if (tid == 32) {  // dS slice leaving this chunk -> dh
-      tma_store_3d(&mdh32, sSHL, 0, srow, 0);
-      tma_store_3d(&mdh32, sSHL + 2 * TILE_VS, 64, srow, 0);
-      tma_store_commit();
-    }
-    float dn = 0.f, en = 0.f, egc = 0.f;  // next chunk's vectors, stored at the end of the step
-    if (vec_thread && more) {
-      const int j = tid - 128;
-      const size_t o = vec0 + (size_t)(c - 1) * 64 + j;
-      dn = w.Dec[o];
-      const float eg = w.EG[o];
-      en = j < len_of(c - 1) ? p.scale * eg : 0.f;
-      egc = eg;
-    }
-    // off the chain while MMA1 runs: -scale e^{G_i} dO[i][v0+v] -> [32 v][64 i] (0 past L),
-    // then this thread's dU_loc elements and decay factors
-    okt = okt && mbar_wait(&barQO, ph, err);
-    {
-      const int i = tid & 63, cq = tid >> 6;
-      float f[8];
-      ld_chunk_f(sO, i, (vo >> 3) + cq, TILE64, f);
-      const float sc = -sEG[i];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) st_bf16(sOS, sw128(8 * cq + e, i, TILE_VS), f[e] * sc);
-    }
-    okt = okt && mbar_wait(&barU, ph, err);
-    float u[8];
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-#pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) u[4 * j + 2 * r + e] = ld_bf16(sUL, uoff[r][e] + 1024 * j);
-    const float dec0 = sDec[ui], dec1 = sDec[ui + 8];
-    // the scaled dO tile is complete: its product with Q^T (off the chain) queues behind MMA1
-    fence_proxy_async();
-    tc_fence_before();
-    okt = __syncthreads_and(okt);
-    tc_fence_after();
-    if (tid == 0 && okt) {
-      const uint64_t dQ_ = desc_mnmajor(smem_u32(sQ), 0, TILE64);
-      const uint64_t dOS = desc_kmajor(smem_u32(sOS), 0, 2 * TILE_VS);
-      constexpr uint32_t idQ = idesc_bf16(128, 2 * VS, true, false);  // lo columns start at 0
-#pragma unroll
-      for (int s = 0; s < 4; ++s)  // F' = Q^T (-scale diag(e^G) dO_z)
-        mma_bf16(tF, dQ_ + mnstep_off(s), dOS + kstep_off(s, TILE_VS), idQ, s > 0);
-    }
-    okt = okt && mbar_wait(&barM1, phM, err);
-    tc_fence_after();
-    if (tid == 64 && more) issue_K(c - 1);  // K consumed by MMA1
-    {
-      float d[8], dl[8];
-      tmem_ld16dp_x2(taddr(tb, 32 * wq, vc), d);
-      tmem_ld16dp_x2(taddr(tb, 32 * wq, VS + vc), dl);
-      tmem_wait_ld();
-#pragma unroll
-      for (int q = 0; q < 8; ++q) d[q] += dl[q];
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int q = 4 * j + 2 * r + e;
-            const float x = u[q] + (r ? dec1 : dec0) * d[q];
-            const bf16 h = __float2bfloat16_rn(x);
-            const uint32_t off = uoff[r][e] + 1024 * j;
-            st_bf16_raw(sUH, off, h);
-            st_bf16_raw(sULo, off, __float2bfloat16_rn(x - __bfloat162float(h)));
-          }
-    }
-    // the dh store of this chunk must be done reading dS before the barrier releases the
-    // dS update below, and the dU^T store of chunk c+1 before its staging is rewritten
-    if (tid == 32) tma_store_wait_read0();
-    fence_proxy_async();
-    tc_fence_before();
-    ok = __syncthreads_and(ok && okt);
-    tc_fence_after();
-    if (!ok) break;
-    if (tid == 0) {
-      okt = mbar_wait(&barW, ph, err);
-      if (okt) {
-        const uint64_t dW_ = desc_kmajor(smem_u32(sW), 0, TILE128);
-        const uint64_t dHL = desc_kmajor(smem_u32(sUH), 0, 2 * TILE_VS);
-        constexpr uint32_t idW = idesc_bf16(128, 2 * VS, false, false);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)  // [F'_hi | F'_lo] += W^T [dU_hi | dU_lo]
-          mma_bf16(tF, dW_ + kstep_off(s, TILE128), dHL + kstep_off(s, 2 * TILE_VS), idW, 1);
-        mma_commit(&barM2);
-      }
-    } else if (tid == 32) {  // dU^T of this chunk (hi, lo) -> global
-      tma_store_3d(&mdUT32, sUH, 0, srow, 0);
-      tma_store_3d(&mdUTl32, sULo, 0, srow, 0);
-      tma_store_commit();
-    } else if (tid == 64 && more) {
-      issue_U(c - 1);  // dU_loc^T consumed
-    }
-    okt = okt && mbar_wait(&barM2, phM, err);
-    phM ^= 1;
-    ph ^= 1;
-    tc_fence_after();
-    if (tid == 64 && more) {  // W^T, Q, dO consumed
-      issue_W(c - 1);
-      issue_QO(c - 1);
-    }
-    {
-      const float eg = sEGC[buf];
-      float d[16], dl[16];
-      tmem_ld16(taddr(tb, 32 * wq, 64 + vc), d);
-      tmem_ld16(taddr(tb, 32 * wq, 64 + VS + vc), dl);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) S[i] = eg * S[i] - (d[i] + dl[i]);
-    }
-    store_dS();
-    if (vec_thread && more) {
-      const int j = tid - 128;
-      sDecb[(buf ^ 1) * 64 + j] = dn;
-      sEGb[(buf ^ 1) * 64 + j] = en;
-      if (j == 63) sEGC[buf ^ 1] = egc;
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    ok = __syncthreads_and(ok && okt);
-    tc_fence_after();
-    if (!ok) break;
-  }
-#undef S_OFF
-  if (tid == 32) tma_store_wait0();
-  if (ok && a.dh0) {
-#pragma unroll
-    for (int i = 0; i < 16; i += 4)
-      *reinterpret_cast<float4*>(a.dh0 + st + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tslot, 128);
-}
-
-// ======================================================================================
 // dqkwg.  One CTA (256 threads) per (chunk, value head).  TMEM columns:
 //   [0,64) Q K^T   [64,128) dO U^T   [128,256) dO S -> dQ   [256,384) U dS' -> dK   [384,512) dU S
 // M=64 accumulators are read with 16-lane loads: warp w covers rows 16(w%4) .. +15, thread t
@@ -487,7 +166,8 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
                                                   const __grid_constant__ CUtensorMap mdUTl,
                                                   const __grid_constant__ CUtensorMap mh,
                                                   const __grid_constant__ CUtensorMap mdh,
-                                                  const __grid_constant__ CUtensorMap mdW) {
+                                                  const __grid_constant__ CUtensorMap mdW,
+                                                  UnitRange ur) {
   if (failed(w)) return;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int half = warp >> 2, sub = 32 * (warp & 3);
@@ -512,7 +192,6 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
   __shared__ uint64_t barA, barB, barM;
   __shared__ uint32_t tslot;
   int* err = w.status;
-  const int nunits = p.NCmax * p.HV;
   if (tid == 0) {
     mbar_init(&barA, 1);
     mbar_init(&barB, 1);
@@ -524,8 +203,8 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
     tmem_alloc(&tslot, 512);
     tmem_relinquish();
   }
-  // units u = gc * HV + hv in order; chunk-table entries past the chunk count are invalid
-  auto valid = [&](int u) { return u < nunits && w.chunk_tab[u / p.HV].x >= 0; };
+  // units u = gc * HV + hv in [u0, u1); chunk-table entries past the chunk count are invalid
+  auto valid = [&](int u) { return u >= ur.u0 && u < ur.u1 && w.chunk_tab[u / p.HV].x >= 0; };
   auto load_A = [&](int u) {
     const int gc = u / p.HV, hk = (u % p.HV) / p.G, tok0 = w.chunk_tab[gc].w;
     mbar_expect_tx(&barA, 4 * TILE64 + TILE128);
@@ -547,7 +226,14 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
     tma_load_3d(sdH, &mdh, 0, u * D, 0, &barB);
     tma_load_3d(sdH + TILE128, &mdh, 64, u * D, 0, &barB);
   };
-  int u = blockIdx.x;
+  // units are handed out in order by an atomic counter (a CTA that starts late, behind other
+  // work on its SM, simply takes fewer); thread 0 takes the next one a unit ahead
+  __shared__ int s_unit[2];
+  int u = -1;
+  if (tid == 0) {
+    u = ur.u0 + atomicAdd(ur.ctr, 1);
+    s_unit[0] = u;
+  }
   // parity of a load group issued and not yet waited on, or -1 (thread 0 issues all loads)
   int pendA = -1, pendB = -1;
   if (tid == 0 && valid(u)) {
@@ -558,21 +244,24 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  u = s_unit[0];
   const uint32_t tb = tslot;
   bool ok = true;
-  for (uint32_t it = 0; valid(u); ++it, u += gridDim.x) {
+  int nu = -1;
+  for (uint32_t it = 0; valid(u); ++it, u = nu) {
     const int gc = u / p.HV, hv = u % p.HV;
     const int4 e = w.chunk_tab[gc];
     const int L = e.z;
     const size_t unit = (size_t)u;
-    const int nu = u + gridDim.x;
-    const bool nvalid = valid(nu);
+    if (tid == 0) s_unit[(it + 1) & 1] = ur.u0 + atomicAdd(ur.ctr, 1);
     const uint32_t ph = it & 1;
     if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
     const bool got = mbar_wait(&barA, ph, err) && mbar_wait(&barB, ph, err);
     if (tid == 0) pendA = pendB = got ? -1 : (int)ph;
     ok = __syncthreads_and(ok && got);
     if (!ok) break;
+    nu = s_unit[(it + 1) & 1];
+    const bool nvalid = valid(nu);
     if (L < 64) {
       zero_tail_rows(sQ, L, tid, 256);
       zero_tail_rows(sK, L, tid, 256);
@@ -589,16 +278,17 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
                  idesc_bf16(64, 64, false, false), acc);
         mma_bf16(taddr(tb, 0, 64), desc_kmajor(o, s, TILE64), desc_mnmajor(ut, s, TILE128),
                  idesc_bf16(64, 64, false, true), acc);
-        mma_bf16(taddr(tb, 0, 128), desc_kmajor(o, s, TILE64), desc_mnmajor(h, s, TILE128),
-                 idesc_bf16(64, 128, false, true), acc);
-        mma_bf16(taddr(tb, 0, 256), desc_mnmajor(ut, s, TILE128), desc_mnmajor(dh, s, TILE128),
-                 idesc_bf16(64, 128, true, true), acc);
-        mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dut, s, TILE128), desc_mnmajor(h, s, TILE128),
-                 idesc_bf16(64, 128, true, true), acc);
+        // S and dS' tiles are stored transposed ([k][v]): K-major B operands here
+        mma_bf16(taddr(tb, 0, 128), desc_kmajor(o, s, TILE64), desc_kmajor(h, s, TILE128),
+                 idesc_bf16(64, 128, false, false), acc);
+        mma_bf16(taddr(tb, 0, 256), desc_mnmajor(ut, s, TILE128), desc_kmajor(dh, s, TILE128),
+                 idesc_bf16(64, 128, true, false), acc);
+        mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dut, s, TILE128), desc_kmajor(h, s, TILE128),
+                 idesc_bf16(64, 128, true, false), acc);
       }
       for (int s = 0; s < 8; ++s)
-        mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dutl, s, TILE128), desc_mnmajor(h, s, TILE128),
-                 idesc_bf16(64, 128, true, true), 1);
+        mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dutl, s, TILE128), desc_kmajor(h, s, TILE128),
+                 idesc_bf16(64, 128, true, false), 1);
       mma_commit(&barM);
     }
     // <dS', S> over the two bf16 state tiles (while the MMAs run)
@@ -798,7 +488,8 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
                                                    const __grid_constant__ CUtensorMap mTm,
                                                    const __grid_constant__ CUtensorMap mdW,
                                                    const __grid_constant__ CUtensorMap mdUT,
-                                                   const __grid_constant__ CUtensorMap mdUTl) {
+                                                   const __grid_constant__ CUtensorMap mdUTl,
+                                                   UnitRange ur) {
   if (failed(w)) return;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int half = warp >> 2, sub = 32 * (warp & 3);
@@ -829,7 +520,6 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   __shared__ uint64_t barA, barB, barC, barM;
   __shared__ uint32_t tslot;
   int* err = w.status;
-  const int nunits = p.NCmax * p.HV;
   if (tid == 0) {
     mbar_init(&barA, 1);
     mbar_init(&barB, 1);
@@ -842,7 +532,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     tmem_alloc(&tslot, 512);
     tmem_relinquish();
   }
-  auto valid = [&](int u) { return u < nunits && w.chunk_tab[u / p.HV].x >= 0; };
+  auto valid = [&](int u) { return u >= ur.u0 && u < ur.u1 && w.chunk_tab[u / p.HV].x >= 0; };
   auto load_A = [&](int u, int buf) {
     const int hk = (u % p.HV) / p.G, tok0 = w.chunk_tab[u / p.HV].w;
     unsigned char* dst = sKb + buf * 2 * TILE64;
@@ -865,7 +555,13 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     tma_load_3d(sT, &mTm, 0, u * 128, 0, &barC);
     tma_load_3d(sTl, &mTm, 0, u * 128 + 64, 0, &barC);
   };
-  int u = blockIdx.x;
+  // units handed out in order by an atomic counter, the next one taken a unit ahead
+  __shared__ int s_unit[2];
+  int u = -1;
+  if (tid == 0) {
+    u = ur.u0 + atomicAdd(ur.ctr, 1);
+    s_unit[0] = u;
+  }
   int pendA = -1, pendB = -1, pendC = -1;  // parity of a load group in flight (thread 0)
   if (tid == 0 && valid(u)) {
     load_A(u, 0);
@@ -876,15 +572,16 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  u = s_unit[0];
   const uint32_t tb = tslot;
   bool ok = true;
-  for (uint32_t it = 0; valid(u); ++it, u += gridDim.x) {
+  int nu = -1;
+  for (uint32_t it = 0; valid(u); ++it, u = nu) {
     const int gc = u / p.HV, hv = u % p.HV;
     const int4 e = w.chunk_tab[gc];
     const int L = e.z, tok0 = e.w;
     const size_t unit = (size_t)u;
-    const int nu = u + gridDim.x;
-    const bool nvalid = valid(nu);
+    if (tid == 0) s_unit[(it + 1) & 1] = ur.u0 + atomicAdd(ur.ctr, 1);
     const uint32_t ph = it & 1;
     if (tid < 64) {
       const size_t o = ((size_t)hv * p.NCmax + gc) * 64 + tid;
@@ -897,6 +594,8 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     if (tid == 0) pendA = pendB = pendC = got ? -1 : (int)ph;
     ok = __syncthreads_and(ok && got);
     if (!ok) break;
+    nu = s_unit[(it + 1) & 1];
+    const bool nvalid = valid(nu);
     unsigned char* sK = sKb + (it & 1) * 2 * TILE64;
     if (tid == 0 && nvalid) {  // the other K buffer was last read by the previous unit
       load_A(nu, (int)(ph ^ 1));
@@ -1156,21 +855,49 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
 
 cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, const TcWork& t,
                                 const TcMaps& m, cudaStream_t s) {
+  const Segments sg = segments(p);
   cudaError_t e;
-  const dim3 gu(p.NCmax, p.HV), gs(p.Nst, p.HV, NVS);
-  if ((e = tgo("tc_dvlocal", k_tc_dvlocal, gu, 128, 1024 + 8 * TILE64 + 256, s, p, w, t, m.q, m.k,
-               m.dO)))
-    return e;
-  if ((e = tgo("tc_scan_bwd", k_tc_scan_bwd, gs, 256, 1024 + BwdScanSmem::TOTAL, s, p, a, w, t, m.q,
-               m.k, m.dO, m.WT, m.dUlT32, m.dUT32, m.dUTl32, m.dh32)))
-    return e;
-  const dim3 gp((unsigned)std::min<long long>((long long)p.NCmax * p.HV, num_sms()));
-  if ((e = tgo("tc_dqkwg", k_tc_dqkwg, gp, 256, 1024 + DqkSmem::TOTAL, s, p, w, t, m.q, m.k, m.dO,
-               m.UT, m.dUT, m.dUTl, m.h, m.dh, m.dW)))
-    return e;
-  if ((e = tgo("tc_wy_bwd", k_tc_wy_bwd, gp, 256, 1024 + WyBwdSmem::TOTAL, s, p, a, w, t, m.k, m.v,
-               m.Tm, m.dW, m.dUT, m.dUTl)))
-    return e;
+  // one work counter per persistent launch, zero before any of them starts
+  if ((e = cudaMemsetAsync(t.ctr, 0, kCounters * sizeof(int), s))) return e;
+  auto dvlocal = [&](int c0, int c1, cudaStream_t st) {
+    return tgo("tc_dvlocal", k_tc_dvlocal, dim3(c1 - c0, p.HV), 128, 1024 + 8 * TILE64 + 256, st, p, w,
+               t, m.q, m.k, m.dO, c0);
+  };
+  auto chunk_kernels = [&](int i, int c0, int c1, cudaStream_t st) {
+    const int units = (c1 - c0) * p.HV;
+    const dim3 gp((unsigned)std::min(units, num_sms()));
+    if ((e = tgo("tc_dqkwg", k_tc_dqkwg, gp, 256, 1024 + DqkSmem::TOTAL, st, p, w, t, m.q, m.k, m.dO,
+                 m.UT, m.dUT, m.dUTl, m.h, m.dh, m.dW, UnitRange{c0 * p.HV, c1 * p.HV, t.ctr + 2 * i})))
+      return e;
+    return tgo("tc_wy_bwd", k_tc_wy_bwd, gp, 256, 1024 + WyBwdSmem::TOTAL, st, p, a, w, t, m.k, m.v,
+               m.Tm, m.dW, m.dUT, m.dUTl, UnitRange{c0 * p.HV, c1 * p.HV, t.ctr + 2 * i + 1});
+  };
+  if (sg.n == 1) {
+    if ((e = dvlocal(0, p.NCmax, s))) return e;
+    if ((e = tc_scan_bwd(p, a, w, t, m, ScanRange{0, p.NCmax, a.dht, a.dh0}, s))) return e;
+    return chunk_kernels(0, 0, p.NCmax, s);
+  }
+  // Segments in reverse: the reverse pass over segment i (side stream) runs while dv_local of
+  // earlier segments and dqkwg / wy_bwd of later (already passed) segments run on `s`.
+  SideLock side;
+  if (!side.ok()) return cudaErrorInvalidResourceHandle;
+  cudaStream_t hs = side.stream();
+  if ((e = side.fork(s))) return e;
+  std::vector<cudaEvent_t> dv_done(sg.n), scan_done(sg.n);
+  for (int i = sg.n - 1; i >= 0; --i) {
+    if ((e = dvlocal(sg.c[i], sg.c[i + 1], s))) return e;
+    if ((e = side.record(s, &dv_done[i]))) return e;
+  }
+  for (int i = sg.n - 1; i >= 0; --i) {
+    if ((e = cudaStreamWaitEvent(hs, dv_done[i], 0))) return e;
+    const ScanRange r{sg.c[i], sg.c[i + 1], i + 1 == sg.n ? a.dht : t.hand, i == 0 ? a.dh0 : t.hand};
+    if ((e = tc_scan_bwd(p, a, w, t, m, r, hs))) return e;
+    if ((e = side.record(hs, &scan_done[i]))) return e;
+  }
+  for (int i = sg.n - 1; i >= 0; --i) {
+    if ((e = cudaStreamWaitEvent(s, scan_done[i], 0))) return e;
+    if ((e = chunk_kernels(i, sg.c[i], sg.c[i + 1], s))) return e;
+  }
   return cudaSuccess;
 }
 

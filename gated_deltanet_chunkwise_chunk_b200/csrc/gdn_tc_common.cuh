@@ -18,9 +18,6 @@ using namespace tc;
 constexpr int D = 128;                 // head dimension (K = V = 128 on this path)
 constexpr int TILE64 = 64 * 128;       // bytes of a [64 rows x 64 bf16] block
 constexpr int TILE128 = 128 * 128;     // bytes of a [128 rows x 64 bf16] block
-constexpr int VS = 32;                 // value rows of the state carried by one scan CTA
-constexpr int NVS = D / VS;            // scan CTAs per (sequence, value head)
-constexpr int TILE_VS = VS * 128;      // bytes of a [32 rows x 64 bf16] block
 
 // ------------------------------------------------------------------ tensor maps (host)
 typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -73,24 +70,88 @@ struct TcMaps {
   CUtensorMap dh;                     // [unit*128][128]     (backward)
   CUtensorMap dW;                     // [unit*64][128]      (backward)
   CUtensorMap Tm;                     // [unit*64][64]       (backward)
-  // the same [unit*128][..] arrays with 32-row boxes (one value slice of the scans)
-  CUtensorMap UtT32, UT32, h32, dUlT32, dUT32, dUTl32, dh32;
 };
 
 struct TcWork {
   bf16* WT;     // [NC*HV][128][64]
   bf16* UtT;    // [NC*HV][128][64]
   bf16* UT;     // [NC*HV][128][64]
-  bf16* h;      // [NC*HV][128][128]
+  bf16* h;      // [NC*HV][128 k][128 v]  state entering the chunk, transposed (S^T)
   bf16* Tm;     // [NC*HV][2][64][64] (backward only) (I + A)^-1 as hi, lo bf16 parts
   bf16* dUlT;   // [NC*HV][128][64]  dv_local^T = scale (P^T dO)^T
-  bf16* dh;     // [NC*HV][128][128] dL/dS leaving the chunk (S orientation [v][k])
+  bf16* dh;     // [NC*HV][128 k][128 v] dL/dS leaving the chunk, transposed (dS^T)
   bf16* dUT;    // [NC*HV][128][64]  dU^T (full), hi part
   bf16* dUTl;   // [NC*HV][128][64]  dU^T lo part (dU^T - hi)
   bf16* dW;     // [NC*HV][64][128]  dL/dW
+  float* hand;  // [HV][128][128] fp32: the state passed between launches of a segmented pass
+  int* ctr;     // [kCounters] work counters of the persistent backward kernels
+};
+
+// A single sequence's chunks are split into segments so that the sequential pass over one
+// segment (one CTA per value head, few SMs) overlaps the chunk-parallel kernels of others.
+constexpr int kMaxSeg = 8;          // segments of a pass
+constexpr int kSegChunks = 32;      // at least this many chunks per segment
+constexpr int kCounters = 2 * kMaxSeg;
+
+struct Segments {
+  int n;                  // number of segments (1 = one launch per kernel over all chunks)
+  int c[kMaxSeg + 1];     // segment i covers chunks [c[i], c[i+1])
+};
+
+inline Segments segments(const Problem& p) {
+  Segments sg{};
+  sg.n = 1;
+  sg.c[0] = 0;
+  sg.c[1] = p.NCmax;
+  // only one sequence (chunks of one segment are contiguous in the chunk table), and only
+  // when the pass leaves most SMs to the other kernels
+  if (p.Nst != 1 || 2 * p.HV > num_sms()) return sg;
+  const int n = std::min(kMaxSeg, p.NCmax / kSegChunks);
+  if (n < 2) return sg;
+  sg.n = n;
+  for (int i = 0; i <= n; ++i) sg.c[i] = (int)((long long)p.NCmax * i / n);
+  return sg;
+}
+
+// The library's side stream on the current device (highest priority, so the sequential pass's
+// CTAs are placed first when SMs free up) and a pool of events, held under a per-device lock
+// while one call queues its work (concurrent calls from several host threads take turns).
+class SideLock {
+ public:
+  SideLock();
+  ~SideLock();
+  SideLock(const SideLock&) = delete;
+  SideLock& operator=(const SideLock&) = delete;
+  bool ok() const { return ok_; }
+  cudaStream_t stream() const;
+  // the side stream waits for the work queued on s so far
+  cudaError_t fork(cudaStream_t s);
+  // records the next pool event on st
+  cudaError_t record(cudaStream_t st, cudaEvent_t* ev);
+
+ private:
+  void* dev_ = nullptr;
+  int next_ = 0;
+  bool ok_ = false;
 };
 
 inline size_t align_up(size_t x) { return (x + 1023) / 1024 * 1024; }
+
+// Chunks [c0, c1) of every sequence (clamped to its length) for one launch of a sequential
+// pass, with the state it enters with and the state it leaves ([Nst][HV][K][V] fp32 in the
+// [k][v] layout; NULL = zero / not written).
+struct ScanRange {
+  int c0, c1;
+  const float* s_in;
+  float* s_out;
+};
+
+// Units u = chunk * HV + value head in [u0, u1) for one launch of a persistent kernel, handed
+// out in order by the atomic counter *ctr (zero before the launch).
+struct UnitRange {
+  int u0, u1;
+  int* ctr;
+};
 
 inline TcWork carve_tc(void* base, size_t NC, size_t HV, int pass) {
   char* b = static_cast<char*>(base);
@@ -107,6 +168,8 @@ inline TcWork carve_tc(void* base, size_t NC, size_t HV, int pass) {
   t.UT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
   t.h = reinterpret_cast<bf16*>(take(units * D * D * 2));
   t.Tm = reinterpret_cast<bf16*>(take(units * 2 * 64 * 64 * 2));  // written by every forward
+  t.hand = reinterpret_cast<float*>(take(HV * D * D * 4));
+  t.ctr = reinterpret_cast<int*>(take(kCounters * sizeof(int)));
   if (pass == 1) {
     t.dUlT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
     t.dh = reinterpret_cast<bf16*>(take(units * D * D * 2));
@@ -121,6 +184,7 @@ inline size_t tc_bytes(size_t NC, size_t HV, int pass) {
   const size_t units = NC * HV;
   size_t o = 3 * align_up(units * D * 64 * 2) + align_up(units * D * D * 2);
   o += align_up(units * 2 * 64 * 64 * 2);
+  o += align_up(HV * D * D * 4) + align_up(kCounters * sizeof(int));
   if (pass == 1)
     o += 3 * align_up(units * D * 64 * 2) +
          align_up(units * D * D * 2) + align_up(units * 64 * D * 2);
@@ -331,6 +395,11 @@ cudaError_t tgo(const char* name, Kern kern, dim3 grid, int threads, size_t smem
 
 cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, const TcWork& t,
                                 const TcMaps& m, cudaStream_t s);
+// The sequential passes over the chunks (gdn_tc_scan.cu): one CTA per (sequence, value head).
+cudaError_t tc_scan_fwd(const Problem& p, const Args& a, const Work& w, const TcWork& t,
+                        const TcMaps& m, const ScanRange& sr, cudaStream_t s);
+cudaError_t tc_scan_bwd(const Problem& p, const Args& a, const Work& w, const TcWork& t,
+                        const TcMaps& m, const ScanRange& sr, cudaStream_t s);
 
 }  // namespace tcx
 }  // namespace gdn

@@ -42,18 +42,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete; gives up after ~2^31 SM cycles
-// (about a second), sets *err (if non-null) to GDN_ERR_TIMEOUT and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+// Waits for the phase with the given parity to complete; gives up after `limit` SM cycles,
+// sets *err (if non-null) to GDN_ERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, int* err, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > (1ll << 31)) {
+    if (clock64() - t0 > limit) {
       if (err) atomicExch(err, 5 /* GDN_ERR_TIMEOUT */);
       return false;
     }
   }
+}
+
+// The same with the library's limit of ~2^31 SM cycles (about a second).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+  return mbar_wait_for(bar, parity, err, 1ll << 31);
 }
 
 // ------------------------------------------------------------------ fences

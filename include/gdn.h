@@ -88,7 +88,15 @@ typedef enum gdn_flags {
    * workspace must be sized for the backward (gdn_workspace_bytes(.., 1) >= the forward's)
    * and passed to both calls.  Honoured by the bf16 K = V = 128 path; other paths always
    * recompute, with identical results. */
-  GDN_FLAG_BWD_REUSE_FWD = 1
+  GDN_FLAG_BWD_REUSE_FWD = 1,
+  /* Tests of the failure path only (no counterpart on the pages): on the bf16 K = V = 128
+   * path, the forward's sequential pass over the chunks withholds its first chain product, so
+   * the wait for it runs out after ~2^20 cycles (under a millisecond) instead of completing.
+   * The pass then stops cleanly: the copies it issued land, the products it issued finish,
+   * its tensor memory is freed, later kernels of the call skip their work, and
+   * gdn_device_status reports GDN_ERR_TIMEOUT.  Outputs are not written.  Nothing faults
+   * and nothing hangs; the next call without the flag runs normally. */
+  GDN_FLAG_TEST_WAIT_TIMEOUT = 1 << 30
 } gdn_flags;
 
 /* Size limits (GDN_ERR_INVALID_ARG beyond them): B*T < 2^31 tokens, HV <= 65535, and

@@ -12,6 +12,12 @@ Per chunk (tokens i=0..63, zero-padded past the sequence end with g=0, beta=0):
   O = scale (diag(e^G) Q S^T + (Q K^T * Gam) U)
   S' = e^{G_C} S + U^T diag(e^{G_C - G}) K           (G_C = G at the last position)
 The backward mirrors these products term by term.
+
+With affine=True the passes over the chunks take the form the sequential CUDA passes use:
+the chunk step is affine in the state, so with D = diag(e^{G_C - G}) (zero past the chunk's
+last token), N = W^T D K and B = U~^T D K (neither depends on the state):
+  S' = e^{G_C} S + B - S N
+  dS = e^{G_C} dS' - (W^T dU_loc - scale Q^T diag(e^G) dO + N dS'^T)^T,  dU_loc = scale P^T dO
 """
 from __future__ import annotations
 
@@ -42,7 +48,7 @@ def _chunk_terms(Q, K, V, g, b):
     return G, Gam, A, T, X, Y, W, Ut, low_incl, low_strict
 
 
-def fwd_unit(q, k, v, g, beta, S0, scale):
+def fwd_unit(q, k, v, g, beta, S0, scale, affine=False):
     """q,k [L,K]; v [L,V]; g, beta [L]; S0 [V,K] (S orientation).  Returns o [L,V], S_final."""
     L = len(g)
     S = S0.copy()
@@ -57,11 +63,15 @@ def fwd_unit(q, k, v, g, beta, S0, scale):
         O = scale * (np.exp(G)[:, None] * (Q @ S.T) + P @ U)
         o[c0:c0 + n] = O[:n]
         GC = G[-1]
-        S = np.exp(GC) * S + (U * np.exp(GC - G)[:, None]).T @ K
+        if affine:
+            Dk = (np.exp(GC - G) * (np.arange(C) < n))[:, None] * K
+            S = np.exp(GC) * S + Ut.T @ Dk - S @ (W.T @ Dk)
+        else:
+            S = np.exp(GC) * S + (U * np.exp(GC - G)[:, None]).T @ K
     return o, S
 
 
-def bwd_unit(q, k, v, g, beta, S0, dO, dSfin, scale):
+def bwd_unit(q, k, v, g, beta, S0, dO, dSfin, scale, affine=False):
     """Chunkwise backward.  Returns dq, dk, dv, dg, dbeta, dS0 for one (sequence, head)."""
     L = len(g)
     nck = (L + C - 1) // C
@@ -103,7 +113,14 @@ def bwd_unit(q, k, v, g, beta, S0, dO, dSfin, scale):
         dG -= r
         dG[-1] += np.exp(GC) * (dSn * Sc).sum() + r.sum()
         # state chain
-        dS = np.exp(GC) * dSn + scale * (np.exp(G)[:, None] * dOc).T @ Q - dU.T @ W
+        if affine:
+            live = (np.arange(C) < n)
+            Dk = (D * live)[:, None] * K
+            acc = W.T @ (scale * P.T @ dOc) + Q.T @ (-scale * (np.exp(G) * live)[:, None] * dOc) \
+                + (W.T @ Dk) @ dSn.T
+            dS = np.exp(GC) * dSn - acc.T
+        else:
+            dS = np.exp(GC) * dSn + scale * (np.exp(G)[:, None] * dOc).T @ Q - dU.T @ W
         # WY backward
         dT = dU @ Y.T + dW @ X.T
         dX = T.T @ dW

@@ -260,10 +260,13 @@ def test_backward_matches_central_differences(T):
 
 
 # ---------------------------------------------------------------- the chunk algebra
+@pytest.mark.parametrize("affine", [False, True])
 @pytest.mark.parametrize("L", [1, 63, 64, 65, 150])
-def test_chunk_algebra_equals_token_recurrence(L):
+def test_chunk_algebra_equals_token_recurrence(L, affine):
     """The 64-token chunk reassociation the CUDA kernels implement (A, (I+A)^-1, W, U~,
-    state scan, output, and every backward term) equals the token-level oracle."""
+    state scan, output, and every backward term) equals the token-level oracle; with
+    affine=True the passes over the chunks take the affine form S' = e^{G_C} S + B - S N the
+    sequential kernels use (and its adjoint)."""
     K, V = 16, 12
     c = _case(L, K=K, V=V, seed=20 + L)
     r = _rng(200 + L)
@@ -274,16 +277,18 @@ def test_chunk_algebra_equals_token_recurrence(L):
     gr = oracle.bwd(**c, dO=dO, dht=dht, scale=scale)
     args = (c["q"][0, :, 0], c["k"][0, :, 0], c["v"][0, :, 0], g[0, :, 0], c["beta"][0, :, 0],
             c["h0"][0, 0].T)
-    oc, Sc = chunk_algebra.fwd_unit(*args, scale)
+    oc, Sc = chunk_algebra.fwd_unit(*args, scale, affine=affine)
     np.testing.assert_allclose(oc, o[0, :, 0], rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(Sc.T, ht[0, 0], rtol=1e-9, atol=1e-11)
-    dq, dk, dv, dg, db, dS0 = chunk_algebra.bwd_unit(*args, dO[0, :, 0], dht[0, 0].T, scale)
+    dq, dk, dv, dg, db, dS0 = chunk_algebra.bwd_unit(*args, dO[0, :, 0], dht[0, 0].T, scale,
+                                                     affine=affine)
     for got, ref in [(dq, gr["dq"][0, :, 0]), (dk, gr["dk"][0, :, 0]), (dv, gr["dv"][0, :, 0]),
                      (dg, gr["dg"][0, :, 0]), (db, gr["dbeta"][0, :, 0]), (dS0.T, gr["dh0"][0, 0])]:
         np.testing.assert_allclose(got, ref, rtol=1e-8, atol=1e-10)
 
 
-def test_chunk_algebra_long_memory_decay():
+@pytest.mark.parametrize("affine", [False, True])
+def test_chunk_algebra_long_memory_decay(affine):
     """Same equality when the decay is weak, so the state crosses many chunks."""
     L, K, V = 200, 8, 8
     c = _case(L, K=K, V=V, seed=31)
@@ -292,5 +297,5 @@ def test_chunk_algebra_long_memory_decay():
     o, ht, g = oracle.fwd(**c)
     assert np.abs(g).max() < 0.05
     oc, Sc = chunk_algebra.fwd_unit(c["q"][0, :, 0], c["k"][0, :, 0], c["v"][0, :, 0], g[0, :, 0],
-                                    c["beta"][0, :, 0], c["h0"][0, 0].T, K ** -0.5)
+                                    c["beta"][0, :, 0], c["h0"][0, 0].T, K ** -0.5, affine=affine)
     np.testing.assert_allclose(oc, o[0, :, 0], rtol=1e-9, atol=1e-11)
