@@ -87,9 +87,9 @@ Plan make_plan(const gdn_dims& d, bool varlen, int pass) {
     // the tcgen05 region starts at the same offset for both passes, so a backward can read
     // what the forward left in the same workspace
     pl.tc = take(tc_workspace_bytes(d, NC, pass));
-    if (pass == 1) {  // fp32 per-value-head dq/dk shares and dG parts, read by the final assembly
-      pl.dqp = take(NC * HV * CH * K * f);
-      pl.dkp = take(NC * HV * CH * K * f);
+    if (pass == 1) {  // fp32 per-value-head dq/dk shares (128 wide) and dG parts, read by the final assembly
+      pl.dqp = take(NC * HV * CH * 128 * f);
+      pl.dkp = take(NC * HV * CH * 128 * f);
       pl.dG = take(HV * NC * CH * f);
       pl.dG2 = take(HV * NC * CH * f);
     }
@@ -142,6 +142,7 @@ Problem make_problem(const gdn_dims& d, bool varlen) {
   p.NCmax = (int)max_chunks(d, varlen);
   p.scale = d.scale > 0.f ? d.scale : 1.f / std::sqrt((float)d.K);
   p.test_timeout = (d.flags & GDN_FLAG_TEST_WAIT_TIMEOUT) ? 1 : 0;
+  p.share_ld = (int)d.K;
   return p;
 }
 
@@ -308,7 +309,8 @@ int gdn_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v
     return GDN_ERR_WORKSPACE;
   // shapes the tcgen05 path covers never run on the CUDA-core kernels instead
   if (tc_bwd_supported(*d) && !tc_ready()) return GDN_ERR_UNSUPPORTED;
-  const Problem p = make_problem(*d, varlen);
+  Problem p = make_problem(*d, varlen);
+  if (tc_bwd_supported(*d)) p.share_ld = 128;  // the tcgen05 kernels' shares are 128 wide
   Args a{};
   a.q = q;
   a.k = k;

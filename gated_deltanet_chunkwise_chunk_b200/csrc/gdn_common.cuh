@@ -21,6 +21,7 @@ struct Problem {
   int NCmax;    // grid bound on the number of chunks
   float scale;
   int test_timeout;  // GDN_FLAG_TEST_WAIT_TIMEOUT: the forward pass withholds one arrive (tests only)
+  int share_ld;      // row stride of the per-value-head dq/dk shares (K, or 128 on the tcgen05 path)
 };
 
 // Workspace carve-up (device pointers into the caller's workspace).  Intermediates are

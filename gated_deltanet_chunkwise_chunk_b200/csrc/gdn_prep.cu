@@ -173,14 +173,14 @@ __global__ void __launch_bounds__(256) k_dqdk_group_sum(Problem p, Args a, Work 
   const int gc = blockIdx.x, h = blockIdx.y;
   const int4 e = w.chunk_tab[gc];
   if (e.x < 0) return;
-  const int L = e.z, tok0 = e.w, K = p.K;
+  const int L = e.z, tok0 = e.w, K = p.K, ld = p.share_ld;
   T* dq = static_cast<T*>(a.dq);
   T* dk = static_cast<T*>(a.dk);
-  const size_t base = ((size_t)gc * p.HV + (size_t)h * p.G) * CH * K;  // value head h*G, row 0
+  const size_t base = ((size_t)gc * p.HV + (size_t)h * p.G) * CH * ld;  // value head h*G, row 0
   for (int i = 4 * threadIdx.x; i < L * K; i += 4 * blockDim.x) {
     float4 sq = make_float4(0.f, 0.f, 0.f, 0.f), sk = sq;
     for (int j = 0; j < p.G; ++j) {
-      const size_t o = base + (size_t)j * CH * K + i;
+      const size_t o = base + (size_t)j * CH * ld + (size_t)(i / K) * ld + i % K;
       const float4 x = *reinterpret_cast<const float4*>(w.dqp + o);
       const float4 y = *reinterpret_cast<const float4*>(w.dkp + o);
       sq.x += x.x; sq.y += x.y; sq.z += x.z; sq.w += x.w;

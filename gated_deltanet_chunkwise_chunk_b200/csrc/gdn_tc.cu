@@ -32,15 +32,16 @@ struct WySmem {
   static constexpr int TX = R1, TY = R1 + TILE64, TXL = R1 + 2 * TILE64, TYL = R1 + 3 * TILE64;
   static constexpr int A = R1, X = R1 + 64 * LDA * 4;    // fp32 [64][LDA] each
   static constexpr int T = R1 + 34 * 1024;              // fp32 [64][LDA]
-  static constexpr int G = T + 64 * LDA * 4, B = G + 256, EG = B + 256;
-  static constexpr int TOTAL = EG + 256;
+  static constexpr int G = T + 64 * LDA * 4, B = G + 256, EG = B + 256, DEC = EG + 256;
+  static constexpr int TOTAL = DEC + 256;
 };
 
 __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
                                                const __grid_constant__ CUtensorMap mk,
                                                const __grid_constant__ CUtensorMap mv,
                                                const __grid_constant__ CUtensorMap mWT,
-                                               const __grid_constant__ CUtensorMap mUtT, int store_T,
+                                               const __grid_constant__ CUtensorMap mUtT,
+                                               const __grid_constant__ CUtensorMap mDK, int store_T,
                                                int gc0) {
   if (failed(w)) return;
   const int gc = gc0 + blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
@@ -62,6 +63,7 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
   float* sG = reinterpret_cast<float*>(sm + WySmem::G);
   float* sb = reinterpret_cast<float*>(sm + WySmem::B);
   float* sEG = reinterpret_cast<float*>(sm + WySmem::EG);   // beta_j e^{G_j}
+  float* sDec = reinterpret_cast<float*>(sm + WySmem::DEC); // e^{G_C - G_j}, zero past the end
   __shared__ uint64_t bar[2];
   __shared__ uint32_t tslot;
   int* err = w.status;
@@ -88,6 +90,7 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
     sG[tid] = g;
     sb[tid] = bb;
     sEG[tid] = bb * expf(g);
+    sDec[tid] = tid < L ? w.Dec[o] : 0.f;
   }
   tc_fence_before();
   __syncthreads();
@@ -196,6 +199,16 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
       st_chunk_f(sWst, r, 4 * half + j, TILE128, x + 8 * j);
       st_chunk_f(sUst, r, 4 * half + j, TILE128, y + 8 * j);
     }
+    // the products are done with K: it becomes D K (read by both sequential passes)
+    for (int idx = tid; idx < 64 * 16; idx += 256) {
+      const int rr = idx >> 4, jj = idx & 15;
+      float f[8];
+      ld_chunk_f(sK, rr, jj, TILE64, f);
+      const float d = sDec[rr];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) f[q] *= d;
+      st_chunk_f(sK, rr, jj, TILE64, f);
+    }
     fence_proxy_async();
   }
   __syncthreads();
@@ -203,6 +216,8 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
     const int row = (gc * p.HV + hv) * D;
     tma_store_3d(&mWT, sm + WySmem::R1, 0, row, 0);
     tma_store_3d(&mUtT, sm + WySmem::R1 + TILE128, 0, row, 0);
+    tma_store_3d(&mDK, sK, 0, (gc * p.HV + hv) * 64, 0);
+    tma_store_3d(&mDK, sK + TILE64, 64, (gc * p.HV + hv) * 64, 0);
     tma_store_commit();
     tma_store_wait_read0();
   }
@@ -212,13 +227,17 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
 }
 
 // ======================================================================================
-// chunk_fwd_o.  One CTA (256 threads) per (chunk, value head):
-//   X = Q S^T (M=64, N=128), QK = Q K^T (M=64, N=64) -> P = QK * Gam (bf16 tile)
+// chunk_fwd_o.  One CTA (256 threads) per (chunk, value head), S the state entering the chunk:
+//   X = Q S^T (M=64, N=128), QK = Q K^T (M=64, N=64), Uc = S W^T (M=128 v, N=64 i)
+//   U^T = U~^T - Uc (v_new; also stored for the backward), P = QK * Gam (bf16 hi/lo tile)
 //   Y = P U (M=64, N=128, B = U^T K-major);  O = scale (e^{G_i} X + Y)
+// With o = NULL (the backward's recompute) only U^T is produced.
 // ======================================================================================
 __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWork t,
                                                 const __grid_constant__ CUtensorMap mq,
                                                 const __grid_constant__ CUtensorMap mk,
+                                                const __grid_constant__ CUtensorMap mUtT,
+                                                const __grid_constant__ CUtensorMap mWT,
                                                 const __grid_constant__ CUtensorMap mUT,
                                                 const __grid_constant__ CUtensorMap mh, int gc0) {
   if (failed(w)) return;
@@ -230,9 +249,10 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
   unsigned char* sm = align1k(smraw);
   unsigned char* sQ = sm;                    // [64][128]
   unsigned char* sK = sQ + 2 * TILE64;       // [64][128]
-  unsigned char* sH = sK + 2 * TILE64;       // [128][128]
-  unsigned char* sU = sH + 2 * TILE128;      // [128][64]  U^T
-  unsigned char* sP = sU + TILE128;          // [64][64] hi part
+  unsigned char* sH = sK + 2 * TILE64;       // S^T [128 k][128 v]
+  unsigned char* sU = sH + 2 * TILE128;      // U~^T [128][64], then U^T in place
+  unsigned char* sW = sU + TILE128;          // W^T [128][64]
+  unsigned char* sP = sW + TILE128;          // [64][64] hi part
   unsigned char* sPl = sP + TILE64;          // lo part
   float* sG = reinterpret_cast<float*>(sPl + TILE64);
   __shared__ uint64_t bar[2];
@@ -248,16 +268,17 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
     tmem_alloc(&tslot, 256);
     tmem_relinquish();
   }
+  const int row = (gc * p.HV + hv) * D;
   if (tid == 0) {
-    const int row = (gc * p.HV + hv) * D;
-    mbar_expect_tx(&bar[0], 4 * TILE64 + 3 * TILE128);
+    mbar_expect_tx(&bar[0], 4 * TILE64 + 4 * TILE128);
     tma_load_3d(sQ, &mq, 0, hk, tok0, &bar[0]);
     tma_load_3d(sQ + TILE64, &mq, 64, hk, tok0, &bar[0]);
     tma_load_3d(sK, &mk, 0, hk, tok0, &bar[0]);
     tma_load_3d(sK + TILE64, &mk, 64, hk, tok0, &bar[0]);
     tma_load_3d(sH, &mh, 0, row, 0, &bar[0]);
     tma_load_3d(sH + TILE128, &mh, 64, row, 0, &bar[0]);
-    tma_load_3d(sU, &mUT, 0, row, 0, &bar[0]);
+    tma_load_3d(sU, &mUtT, 0, row, 0, &bar[0]);
+    tma_load_3d(sW, &mWT, 0, row, 0, &bar[0]);
   }
   if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
   tc_fence_before();
@@ -266,13 +287,15 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
   const uint32_t tb = tslot;
   bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
   if (ok && tid == 0) {
-    const uint32_t q = smem_u32(sQ), k = smem_u32(sK), h = smem_u32(sH);
+    const uint32_t q = smem_u32(sQ), k = smem_u32(sK), h = smem_u32(sH), wt = smem_u32(sW);
     for (int s = 0; s < 8; ++s) {
-      // S is stored transposed ([k][v]): an MN-major B operand
+      // S is stored transposed ([k][v]): an MN-major B operand here, an MN-major A below
       mma_bf16(taddr(tb, 0, 0), desc_kmajor(q, s, TILE64), desc_mnmajor(h, s, TILE128),
                idesc_bf16(64, 128, false, true), s > 0);
       mma_bf16(taddr(tb, 0, 128), desc_kmajor(q, s, TILE64), desc_kmajor(k, s, TILE64),
                idesc_bf16(64, 64, false, false), s > 0);
+      mma_bf16(taddr(tb, 0, 192), desc_mnmajor(h, s, TILE128), desc_mnmajor(wt, s, TILE128),
+               idesc_bf16(128, 64, true, true), s > 0);
     }
     mma_commit(&bar[1]);
   }
@@ -298,12 +321,28 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
       st_pair_split(sP, sPl, r0, c, TILE64, f[0], f[1]);
       st_pair_split(sP, sPl, r0 + 8, c, TILE64, f[2], f[3]);
     }
+    // U^T = U~^T - S W^T (M=128 accumulator: lane = value row v), columns [32 half, +32), in place
+    float x[32];
+    const int v = 32 * (warp & 3) + lane;
+    tmem_ld16(taddr(tb, 32 * (warp & 3), 192 + 32 * half), x);
+    tmem_ld16(taddr(tb, 32 * (warp & 3), 192 + 32 * half + 16), x + 16);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float f[8];
+      ld_chunk_f(sU, v, 4 * half + j, TILE128, f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) f[q] -= x[8 * j + q];
+      st_chunk_f(sU, v, 4 * half + j, TILE128, f);
+    }
   }
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (ok && tid == 0) {
+    tma_store_3d(&mUT, sU, 0, row, 0);  // v_new for the backward
+    tma_store_commit();
     const uint32_t pp = smem_u32(sP), pl = smem_u32(sPl), u = smem_u32(sU);
     for (int s = 0; s < 4; ++s)
       mma_bf16(taddr(tb, 0, 128), desc_kmajor(pp, s, TILE64), desc_kmajor(u, s, TILE128),
@@ -315,24 +354,26 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
   tc_fence_after();
-  if (ok) {  // O = scale (e^{G_i} X + Y), columns [64 half, +64)
+  if (ok && a.o) {  // O = scale (e^{G_i} X + Y), columns [64 half, +64)
     float x[32], y[32];
     tmem_ld16dp_x8(taddr(tb, 32 * (warp & 3), 64 * half), x);
     tmem_ld16dp_x8(taddr(tb, 32 * (warp & 3), 128 + 64 * half), y);
     tmem_wait_ld();
     const float e0 = __expf(g0) * p.scale, e1 = __expf(g1) * p.scale;
-    bf16* o0 = static_cast<bf16*>(a.o) + ((size_t)(tok0 + r0) * p.HV + hv) * D + 64 * half + cq;
-    bf16* o1 = o0 + (size_t)8 * p.HV * D;
+    bf16* o0 = static_cast<bf16*>(a.o) + ((size_t)(tok0 + r0) * p.HV + hv) * p.V + 64 * half + cq;
+    bf16* o1 = o0 + (size_t)8 * p.HV * p.V;
+    const bool live = 64 * half < p.V;  // columns past a 64-wide value head are padding
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      if (r0 < L)
+      if (live && r0 < L)
         *reinterpret_cast<uint32_t*>(o0 + 8 * j) =
             pack_bf16(e0 * x[4 * j] + p.scale * y[4 * j], e0 * x[4 * j + 1] + p.scale * y[4 * j + 1]);
-      if (r0 + 8 < L)
+      if (live && r0 + 8 < L)
         *reinterpret_cast<uint32_t*>(o1 + 8 * j) =
             pack_bf16(e1 * x[4 * j + 2] + p.scale * y[4 * j + 2], e1 * x[4 * j + 3] + p.scale * y[4 * j + 3]);
     }
   }
+  if (tid == 0) tma_store_wait0();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tb, 256);
@@ -350,14 +391,15 @@ Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
   const int ntok = p.B * p.T;
   L.t = carve_tc(tc_ws, (size_t)p.NCmax, (size_t)p.HV, pass);
   const uint64_t urows = (uint64_t)p.NCmax * p.HV * D;
-  L.ok &= map_tokens(&L.m.q, a.q, ntok, p.H);
-  L.ok &= map_tokens(&L.m.k, a.k, ntok, p.H);
-  L.ok &= map_tokens(&L.m.v, a.v, ntok, p.HV);
-  if (a.dO) L.ok &= map_tokens(&L.m.dO, a.dO, ntok, p.HV);
+  L.ok &= map_tokens(&L.m.q, a.q, ntok, p.H, p.K);
+  L.ok &= map_tokens(&L.m.k, a.k, ntok, p.H, p.K);
+  L.ok &= map_tokens(&L.m.v, a.v, ntok, p.HV, p.V);
+  if (a.dO) L.ok &= map_tokens(&L.m.dO, a.dO, ntok, p.HV, p.V);
   L.ok &= map_rows(&L.m.WT, L.t.WT, urows, 64, 128);
   L.ok &= map_rows(&L.m.UtT, L.t.UtT, urows, 64, 128);
   L.ok &= map_rows(&L.m.UT, L.t.UT, urows, 64, 128);
   L.ok &= map_rows(&L.m.h, L.t.h, urows, 128, 128);
+  L.ok &= map_rows(&L.m.DK, L.t.DK, (uint64_t)p.NCmax * p.HV * 64, 128, 64);
   if (pass == 1) {
     const uint64_t trows = (uint64_t)p.NCmax * p.HV * 64;
     L.ok &= map_rows(&L.m.dUlT, L.t.dUlT, urows, 64, 128);
@@ -365,6 +407,7 @@ Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
     L.ok &= map_rows(&L.m.dUTl, L.t.dUTl, urows, 64, 128);
     L.ok &= map_rows(&L.m.dh, L.t.dh, urows, 128, 128);
     L.ok &= map_rows(&L.m.dW, L.t.dW, trows, 128, 64);
+    L.ok &= map_rows(&L.m.Op, L.t.Op, trows, 128, 64);
     L.ok &= map_rows(&L.m.Tm, L.t.Tm, 2 * trows, 64, 64);
   }
   return L;
@@ -373,14 +416,16 @@ Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
 cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const Launch& L,
                          bool bwd_prep, cudaStream_t s) {
   if (!L.ok) return cudaErrorInvalidValue;
-  const size_t out_smem = 1024 + 6 * TILE64 + 3 * TILE128 + 256;
+  const size_t out_smem = 1024 + 6 * TILE64 + 4 * TILE128 + 256;
+  Args ao = a;
+  if (bwd_prep) ao.o = nullptr;  // the backward's recompute only needs v_new from the output kernel
   auto wy = [&](int c0, int c1, cudaStream_t st) {
     return tgo("tc_wy", k_tc_wy, dim3(c1 - c0, p.HV), 256, (size_t)1024 + WySmem::TOTAL, st, p, w,
-               L.t, L.m.k, L.m.v, L.m.WT, L.m.UtT, 1, c0);
+               L.t, L.m.k, L.m.v, L.m.WT, L.m.UtT, L.m.DK, 1, c0);
   };
   auto out = [&](int c0, int c1, cudaStream_t st) {
-    return tgo("tc_out", k_tc_out, dim3(c1 - c0, p.HV), 256, out_smem, st, p, a, w, L.t, L.m.q,
-               L.m.k, L.m.UT, L.m.h, c0);
+    return tgo("tc_out", k_tc_out, dim3(c1 - c0, p.HV), 256, out_smem, st, p, ao, w, L.t, L.m.q,
+               L.m.k, L.m.UtT, L.m.WT, L.m.UT, L.m.h, c0);
   };
   float* ht = bwd_prep ? nullptr : a.ht;
   const Segments sg = segments(p);
@@ -388,8 +433,7 @@ cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const L
   if (sg.n == 1) {
     if ((e = wy(0, p.NCmax, s))) return e;
     if ((e = tc_scan_fwd(p, a, w, L.t, L.m, ScanRange{0, p.NCmax, a.h0, ht}, s))) return e;
-    if (!bwd_prep && (e = out(0, p.NCmax, s))) return e;
-    return cudaSuccess;
+    return out(0, p.NCmax, s);
   }
   // Segments of the sequence's chunks: the pass over segment i (on the side stream) runs
   // while the WY kernels of later segments and the outputs of earlier ones run on `s`.
@@ -411,7 +455,7 @@ cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const L
   }
   for (int i = 0; i < sg.n; ++i) {
     if ((e = cudaStreamWaitEvent(s, scan_done[i], 0))) return e;
-    if (!bwd_prep && (e = out(sg.c[i], sg.c[i + 1], s))) return e;
+    if ((e = out(sg.c[i], sg.c[i + 1], s))) return e;
   }
   return cudaSuccess;
 }
@@ -419,7 +463,10 @@ cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const L
 }  // namespace
 
 bool tc_supported(const gdn_dims& d) {
-  return d.dtype == GDN_DTYPE_BF16 && d.K == 128 && d.V == 128 && d.B * d.T > 0;
+  // 64-wide heads run on the same 128-wide tiles: their token maps are 64 columns wide, so the
+  // second 64-column box of every token tile reads as zeros and adds nothing to any product
+  return d.dtype == GDN_DTYPE_BF16 && (d.K == 64 || d.K == 128) && (d.V == 64 || d.V == 128) &&
+         d.B * d.T > 0;
 }
 
 bool tc_bwd_supported(const gdn_dims& d) { return tc_supported(d); }

@@ -29,7 +29,8 @@ __device__ __forceinline__ float warp_sum(float x) {
 __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
                                                     const __grid_constant__ CUtensorMap mq,
                                                     const __grid_constant__ CUtensorMap mk,
-                                                    const __grid_constant__ CUtensorMap mdO, int gc0) {
+                                                    const __grid_constant__ CUtensorMap mdO,
+                                                    const __grid_constant__ CUtensorMap mOp, int gc0) {
   if (failed(w)) return;
   const int gc = gc0 + blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
   const int4 e = w.chunk_tab[gc];
@@ -43,6 +44,7 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
   unsigned char* sP = sO + 2 * TILE64;      // P hi
   unsigned char* sPl = sP + TILE64;         // P lo
   float* sG = reinterpret_cast<float*>(sPl + TILE64);
+  float* sEo = sG + 64;                     // -scale e^{G_i}, zero past the chunk end
   __shared__ uint64_t bar[2];
   __shared__ uint32_t tslot;
   int* err = w.status;
@@ -65,7 +67,11 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
     tma_load_3d(sO, &mdO, 0, hv, tok0, &bar[0]);
     tma_load_3d(sO + TILE64, &mdO, 64, hv, tok0, &bar[0]);
   }
-  if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
+  if (tid < 64) {
+    const size_t o = ((size_t)hv * p.NCmax + gc) * 64 + tid;
+    sG[tid] = w.G[o];
+    sEo[tid] = tid < L ? -p.scale * w.EG[o] : 0.f;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -133,6 +139,25 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
       *reinterpret_cast<uint4*>(row + c) = a0;
       *reinterpret_cast<uint4*>(row + c + 8) = a1;
     }
+    // the products are done with dO: it becomes O' = -scale e^G dO for the reverse pass
+    for (int idx = tid; idx < 64 * 16; idx += 128) {
+      const int r = idx >> 4, j = idx & 15;
+      float f[8];
+      ld_chunk_f(sO, r, j, TILE64, f);
+      const float sc = sEo[r];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) f[q] *= sc;
+      st_chunk_f(sO, r, j, TILE64, f);
+    }
+    fence_proxy_async();
+  }
+  __syncthreads();
+  if (ok && tid == 0) {
+    const int orow = (gc * p.HV + hv) * 64;
+    tma_store_3d(&mOp, sO, 0, orow, 0);
+    tma_store_3d(&mOp, sO + TILE64, 64, orow, 0);
+    tma_store_commit();
+    tma_store_wait0();
   }
   tc_fence_before();
   __syncthreads();
@@ -670,8 +695,9 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
       tmem_wait_ld();
       const float s0 = b0 * sEG[r0], s1 = b1 * sEG[r1];
       float px0 = 0.f, px1 = 0.f, py0 = 0.f, py1 = 0.f;
-      bf16* dv0 = static_cast<bf16*>(a.dv) + ((size_t)(tok0 + r0) * p.HV + hv) * D + 64 * half + cq;
-      bf16* dv1 = dv0 + (size_t)8 * p.HV * D;
+      bf16* dv0 = static_cast<bf16*>(a.dv) + ((size_t)(tok0 + r0) * p.HV + hv) * p.V + 64 * half + cq;
+      bf16* dv1 = dv0 + (size_t)8 * p.HV * p.V;
+      const bool live = 64 * half < p.V;  // columns past a 64-wide value head are padding
   #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int c = 64 * half + 8 * j + cq;
@@ -682,9 +708,9 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
         x[4 * j] *= s0; x[4 * j + 1] *= s0; x[4 * j + 2] *= s1; x[4 * j + 3] *= s1;
         py0 += y[4 * j] * v0.x + y[4 * j + 1] * v0.y;
         py1 += y[4 * j + 2] * v1.x + y[4 * j + 3] * v1.y;
-        if (r0 < L)
+        if (live && r0 < L)
           *reinterpret_cast<uint32_t*>(dv0 + 8 * j) = pack_bf16(b0 * y[4 * j], b0 * y[4 * j + 1]);
-        if (r1 < L)
+        if (live && r1 < L)
           *reinterpret_cast<uint32_t*>(dv1 + 8 * j) = pack_bf16(b1 * y[4 * j + 2], b1 * y[4 * j + 3]);
       }
       tmem_st16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
@@ -860,8 +886,8 @@ cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, 
   // one work counter per persistent launch, zero before any of them starts
   if ((e = cudaMemsetAsync(t.ctr, 0, kCounters * sizeof(int), s))) return e;
   auto dvlocal = [&](int c0, int c1, cudaStream_t st) {
-    return tgo("tc_dvlocal", k_tc_dvlocal, dim3(c1 - c0, p.HV), 128, 1024 + 8 * TILE64 + 256, st, p, w,
-               t, m.q, m.k, m.dO, c0);
+    return tgo("tc_dvlocal", k_tc_dvlocal, dim3(c1 - c0, p.HV), 128, 1024 + 8 * TILE64 + 512, st, p, w,
+               t, m.q, m.k, m.dO, m.Op, c0);
   };
   auto chunk_kernels = [&](int i, int c0, int c1, cudaStream_t st) {
     const int units = (c1 - c0) * p.HV;

@@ -53,9 +53,11 @@ inline bool map3(CUtensorMap* m, const void* base, uint64_t cols, uint64_t mid, 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// token tensor [ntok][heads][128] -> 3D map (col, head, token), box = 64 cols x 1 head x 64 tokens
-inline bool map_tokens(CUtensorMap* m, const void* base, int ntok, int heads) {
-  return map3(m, base, D, heads, ntok, D, (uint64_t)heads * D, 1, 64);
+// token tensor [ntok][heads][dim] -> 3D map (col, head, token), box = 64 cols x 1 head x 64
+// tokens.  With dim = 64 the box at column 64 lies past the tensor and reads as zeros, which is
+// how 64-wide heads run on the 128-wide tiles.
+inline bool map_tokens(CUtensorMap* m, const void* base, int ntok, int heads, int dim) {
+  return map3(m, base, (uint64_t)dim, heads, ntok, (uint64_t)dim, (uint64_t)heads * dim, 1, 64);
 }
 // 2D row-major [rows][cols] bf16, box = 64 cols x box_rows rows (as a 3D map with outer = 1)
 inline bool map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
@@ -70,6 +72,8 @@ struct TcMaps {
   CUtensorMap dh;                     // [unit*128][128]     (backward)
   CUtensorMap dW;                     // [unit*64][128]      (backward)
   CUtensorMap Tm;                     // [unit*64][64]       (backward)
+  CUtensorMap DK;                     // [unit*64][128]      keys scaled by e^{G_C - G_i}
+  CUtensorMap Op;                     // [unit*64][128]      -scale e^{G_i} dO   (backward)
 };
 
 struct TcWork {
@@ -83,6 +87,8 @@ struct TcWork {
   bf16* dUT;    // [NC*HV][128][64]  dU^T (full), hi part
   bf16* dUTl;   // [NC*HV][128][64]  dU^T lo part (dU^T - hi)
   bf16* dW;     // [NC*HV][64][128]  dL/dW
+  bf16* DK;     // [NC*HV][64][128]  D K = e^{G_C - G_i} k_i (zero past the chunk end), per value head
+  bf16* Op;     // [NC*HV][64][128]  O' = -scale e^{G_i} dO_i (zero past the chunk end)  (backward)
   float* hand;  // [HV][128][128] fp32: the state passed between launches of a segmented pass
   int* ctr;     // [kCounters] work counters of the persistent backward kernels
 };
@@ -168,6 +174,7 @@ inline TcWork carve_tc(void* base, size_t NC, size_t HV, int pass) {
   t.UT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
   t.h = reinterpret_cast<bf16*>(take(units * D * D * 2));
   t.Tm = reinterpret_cast<bf16*>(take(units * 2 * 64 * 64 * 2));  // written by every forward
+  t.DK = reinterpret_cast<bf16*>(take(units * 64 * D * 2));
   t.hand = reinterpret_cast<float*>(take(HV * D * D * 4));
   t.ctr = reinterpret_cast<int*>(take(kCounters * sizeof(int)));
   if (pass == 1) {
@@ -176,6 +183,7 @@ inline TcWork carve_tc(void* base, size_t NC, size_t HV, int pass) {
     t.dUT = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
     t.dUTl = reinterpret_cast<bf16*>(take(units * D * 64 * 2));
     t.dW = reinterpret_cast<bf16*>(take(units * 64 * D * 2));
+    t.Op = reinterpret_cast<bf16*>(take(units * 64 * D * 2));
   }
   return t;
 }
@@ -184,10 +192,11 @@ inline size_t tc_bytes(size_t NC, size_t HV, int pass) {
   const size_t units = NC * HV;
   size_t o = 3 * align_up(units * D * 64 * 2) + align_up(units * D * D * 2);
   o += align_up(units * 2 * 64 * 64 * 2);
+  o += align_up(units * 64 * D * 2);
   o += align_up(HV * D * D * 4) + align_up(kCounters * sizeof(int));
   if (pass == 1)
     o += 3 * align_up(units * D * 64 * 2) +
-         align_up(units * D * D * 2) + align_up(units * 64 * D * 2);
+         align_up(units * D * D * 2) + 2 * align_up(units * 64 * D * 2);
   return o;
 }
 

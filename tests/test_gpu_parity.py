@@ -209,21 +209,24 @@ def test_long_sequence_four_times_the_layer_length():
     _assert_parity(case)
 
 
-@pytest.mark.parametrize("lengths", [None, [300, 0, 77]])
-def test_bf16_d128_runs_on_the_tensor_core_kernels(lengths):
-    """bf16 with K = V = 128 always takes the tcgen05 kernels (no silent CUDA-core fallback):
-    the per-launch profile of one forward + backward names only tcgen05 and prologue kernels,
-    and every step of the chunk path is among them."""
+@pytest.mark.parametrize("KV,lengths", [((128, 128), None), ((128, 128), [300, 0, 77]),
+                                        ((64, 64), None), ((64, 128), [130, 5]), ((128, 64), None)])
+def test_bf16_runs_on_the_tensor_core_kernels(KV, lengths):
+    """bf16 always takes the tcgen05 kernels (no silent CUDA-core fallback), 64-wide heads
+    included: the per-launch profile of one forward + backward names only tcgen05 and prologue
+    kernels, every step of the chunk path is among them, and the results match the oracle."""
     import gated_deltanet_chunkwise_chunk_b200 as gdn
-    case = synth.make_case(B=1 if lengths else 2, T=200, H=2, HV=4, K=128, V=128, dtype="bf16",
-                           seed=61, lengths=lengths, h0=True, dht=True, name="tc_path")
+    K, V = KV
+    case = synth.make_case(B=1 if lengths else 2, T=200, H=2, HV=4, K=K, V=V, dtype="bf16",
+                           seed=61, lengths=lengths, h0=True, dht=True, name=f"tc_path_K{K}V{V}")
     gdn.profile(True)
     try:
-        run_gpu(case)
+        gpu = run_gpu(case)
         torch.cuda.synchronize()
         names = set(gdn.profile_read())
     finally:
         gdn.profile(False)
+    _assert_parity(case, gpu=gpu)
     assert not any(n.startswith("ffma_") for n in names), names
     tc = {n for n in names if n.startswith("tc_")}
     assert len(tc) >= 6, names
