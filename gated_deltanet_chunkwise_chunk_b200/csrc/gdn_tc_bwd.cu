@@ -273,6 +273,12 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
   const uint32_t tb = tslot;
   bool ok = true;
   int nu = -1;
+  // the unit's in-chunk gate sums, read into a register a unit ahead (their load latency
+  // then overlaps the previous unit instead of stalling this one)
+  auto g_of = [&](int uu) {
+    return (tid < 64 && valid(uu)) ? w.G[((size_t)(uu % p.HV) * p.NCmax + uu / p.HV) * 64 + tid] : 0.f;
+  };
+  float g_next = g_of(u);
   for (uint32_t it = 0; valid(u); ++it, u = nu) {
     const int gc = u / p.HV, hv = u % p.HV;
     const int4 e = w.chunk_tab[gc];
@@ -280,13 +286,14 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
     const size_t unit = (size_t)u;
     if (tid == 0) s_unit[(it + 1) & 1] = ur.u0 + atomicAdd(ur.ctr, 1);
     const uint32_t ph = it & 1;
-    if (tid < 64) sG[tid] = w.G[((size_t)hv * p.NCmax + gc) * 64 + tid];
+    if (tid < 64) sG[tid] = g_next;
     const bool got = mbar_wait(&barA, ph, err) && mbar_wait(&barB, ph, err);
     if (tid == 0) pendA = pendB = got ? -1 : (int)ph;
     ok = __syncthreads_and(ok && got);
     if (!ok) break;
     nu = s_unit[(it + 1) & 1];
     const bool nvalid = valid(nu);
+    g_next = g_of(nu);
     if (L < 64) {
       zero_tail_rows(sQ, L, tid, 256);
       zero_tail_rows(sK, L, tid, 256);
@@ -601,6 +608,16 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   const uint32_t tb = tslot;
   bool ok = true;
   int nu = -1;
+  // the unit's gate sums and beta, read into registers a unit ahead (see dqkwg)
+  float g_next = 0.f, b_next = 0.f;
+  auto vec_of = [&](int uu) {
+    if (tid < 64 && valid(uu)) {
+      const size_t o = ((size_t)(uu % p.HV) * p.NCmax + uu / p.HV) * 64 + tid;
+      g_next = w.G[o];
+      b_next = w.beta_p[o];
+    }
+  };
+  vec_of(u);
   for (uint32_t it = 0; valid(u); ++it, u = nu) {
     const int gc = u / p.HV, hv = u % p.HV;
     const int4 e = w.chunk_tab[gc];
@@ -609,11 +626,9 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     if (tid == 0) s_unit[(it + 1) & 1] = ur.u0 + atomicAdd(ur.ctr, 1);
     const uint32_t ph = it & 1;
     if (tid < 64) {
-      const size_t o = ((size_t)hv * p.NCmax + gc) * 64 + tid;
-      const float g = w.G[o];
-      sG[tid] = g;
-      sb[tid] = w.beta_p[o];
-      sEG[tid] = __expf(g);
+      sG[tid] = g_next;
+      sb[tid] = b_next;
+      sEG[tid] = __expf(g_next);
     }
     const bool got = mbar_wait(&barA, ph, err) && mbar_wait(&barB, ph, err) && mbar_wait(&barC, ph, err);
     if (tid == 0) pendA = pendB = pendC = got ? -1 : (int)ph;
@@ -621,6 +636,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     if (!ok) break;
     nu = s_unit[(it + 1) & 1];
     const bool nvalid = valid(nu);
+    vec_of(nu);
     unsigned char* sK = sKb + (it & 1) * 2 * TILE64;
     if (tid == 0 && nvalid) {  // the other K buffer was last read by the previous unit
       load_A(nu, (int)(ph ^ 1));
