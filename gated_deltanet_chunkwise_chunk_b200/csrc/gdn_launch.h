@@ -26,8 +26,10 @@ cudaError_t launch_chunk_table(const Problem& p, const int64_t* cu, const Work& 
 cudaError_t launch_chunk_table_only(const Problem& p, const int64_t* cu, int4* table, int* count,
                                     cudaStream_t s);
 cudaError_t launch_gate_cumsum(const Problem& p, const Args& a, const Work& w, cudaStream_t s);
+// dg and dbeta per token, the parameter gradients and (group_sum) dq, dk from per-value-head
+// shares; the tensor-core path writes dq and dk itself and passes group_sum = false.
 cudaError_t launch_bwd_tokens(const Problem& p, const Args& a, const Work& w, bool bf16,
-                              cudaStream_t s);
+                              cudaStream_t s, bool group_sum = true);
 
 // fp32 CUDA-core path (FFMA tiles): used for fp32 tensors.
 // KDA gate (per-channel gate) forward and backward; dtypes are gdn_dtype codes.

@@ -324,7 +324,7 @@ cudaError_t launch_param_grads(const Problem& p, const Args& a, const Work& w, c
 }
 
 cudaError_t launch_bwd_tokens(const Problem& p, const Args& a, const Work& w, bool bf16,
-                              cudaStream_t s) {
+                              cudaStream_t s, bool group_sum) {
   if (p.NCmax == 0 && !(a.dA_log || a.ddt_bias)) return cudaSuccess;
   if (p.NCmax == 0) return launch_param_grads(p, a, w, s);
   {
@@ -333,7 +333,7 @@ cudaError_t launch_bwd_tokens(const Problem& p, const Args& a, const Work& w, bo
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if ((e = launch_dqdk_group_sum(p, a, w, bf16, s)) != cudaSuccess) return e;
+  if (group_sum && (e = launch_dqdk_group_sum(p, a, w, bf16, s)) != cudaSuccess) return e;
   if (a.dA_log || a.ddt_bias) e = launch_param_grads(p, a, w, s);
   return e;
 }

@@ -34,6 +34,8 @@ struct WySmem {
   static constexpr int T = R1 + 34 * 1024;              // fp32 [64][LDA]
   static constexpr int G = T + 64 * LDA * 4, B = G + 256, EG = B + 256, DEC = EG + 256;
   static constexpr int TOTAL = DEC + 256;
+  static constexpr int NB1 = R1 + 2 * TILE128;           // second -N^T box (solve scratch)
+  static_assert(NB1 + TILE128 <= G, "-N^T staging overlaps the per-token vectors");
 };
 
 __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
@@ -41,7 +43,8 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
                                                const __grid_constant__ CUtensorMap mv,
                                                const __grid_constant__ CUtensorMap mWT,
                                                const __grid_constant__ CUtensorMap mUtT,
-                                               const __grid_constant__ CUtensorMap mDK, int store_T,
+                                               const __grid_constant__ CUtensorMap mDK,
+                                               const __grid_constant__ CUtensorMap mNT, int store_T,
                                                int gc0) {
   if (failed(w)) return;
   const int gc = gc0 + blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
@@ -211,14 +214,53 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
     }
     fence_proxy_async();
   }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const int row = (gc * p.HV + hv) * D;
   if (ok && tid == 0) {
-    const int row = (gc * p.HV + hv) * D;
     tma_store_3d(&mWT, sm + WySmem::R1, 0, row, 0);
     tma_store_3d(&mUtT, sm + WySmem::R1 + TILE128, 0, row, 0);
     tma_store_3d(&mDK, sK, 0, (gc * p.HV + hv) * 64, 0);
     tma_store_3d(&mDK, sK + TILE64, 64, (gc * p.HV + hv) * 64, 0);
     tma_store_commit();
+    // N^T = (D K)^T W, the state-free factor of the chunk's affine state map (M=128 k',
+    // N=128 k, K=64 i; A = D K MN-major, B = W^T K-major), into TMEM columns [128, 256)
+    const uint64_t dk = desc_mnmajor(smem_u32(sK), 0, TILE64);
+    const uint64_t dw = desc_kmajor(smem_u32(sm + WySmem::R1), 0, TILE128);
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+      mma_bf16(taddr(tb, 0, 128), dk + mnstep_off(s), dw + kstep_off(s, TILE128),
+               idesc_bf16(128, 128, true, false), s > 0);
+    mma_commit(&bar[1]);
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
+  tc_fence_after();
+  if (ok) {
+    // -N^T as a bf16 [128 k'][128 k] K-major tile (two 64-column boxes: V's space and a free
+    // part of the solve's scratch), the A operand of both sequential passes' chain products
+    const int r = sub + lane;
+    unsigned char* sNst = sm + (half ? WySmem::NB1 : WySmem::V);
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      float x[32];
+      tmem_ld16(taddr(tb, sub, 128 + 64 * half + 32 * part), x);
+      tmem_ld16(taddr(tb, sub, 128 + 64 * half + 32 * part + 16), x + 16);
+      tmem_wait_ld();
+#pragma unroll
+      for (int q = 0; q < 32; ++q) x[q] = -x[q];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) st_chunk_f(sNst, r, 4 * part + j, TILE128, x + 8 * j);
+    }
+    fence_proxy_async();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    if (ok) {
+      tma_store_3d(&mNT, sm + WySmem::V, 0, row, 0);
+      tma_store_3d(&mNT, sm + WySmem::NB1, 64, row, 0);
+      tma_store_commit();
+    }
     tma_store_wait_read0();
   }
   tc_fence_before();
@@ -252,9 +294,11 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
   unsigned char* sH = sK + 2 * TILE64;       // S^T [128 k][128 v]
   unsigned char* sU = sH + 2 * TILE128;      // U~^T [128][64], then U^T in place
   unsigned char* sW = sU + TILE128;          // W^T [128][64]
-  unsigned char* sP = sW + TILE128;          // [64][64] hi part
-  unsigned char* sPl = sP + TILE64;          // lo part
-  float* sG = reinterpret_cast<float*>(sPl + TILE64);
+  // P (hi, lo [64][64] each) is written once the first products have read K: it takes K's
+  // place, so that two CTAs fit on an SM
+  unsigned char* sP = sK;
+  unsigned char* sPl = sK + TILE64;
+  float* sG = reinterpret_cast<float*>(sW + TILE128);
   __shared__ uint64_t bar[2];
   __shared__ uint32_t tslot;
   int* err = w.status;
@@ -400,6 +444,7 @@ Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
   L.ok &= map_rows(&L.m.UT, L.t.UT, urows, 64, 128);
   L.ok &= map_rows(&L.m.h, L.t.h, urows, 128, 128);
   L.ok &= map_rows(&L.m.DK, L.t.DK, (uint64_t)p.NCmax * p.HV * 64, 128, 64);
+  L.ok &= map_rows(&L.m.NT, L.t.NT, urows, 128, 128);
   if (pass == 1) {
     const uint64_t trows = (uint64_t)p.NCmax * p.HV * 64;
     L.ok &= map_rows(&L.m.dUlT, L.t.dUlT, urows, 64, 128);
@@ -416,12 +461,12 @@ Launch setup(const Problem& p, const Args& a, void* tc_ws, int pass) {
 cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const Launch& L,
                          bool bwd_prep, cudaStream_t s) {
   if (!L.ok) return cudaErrorInvalidValue;
-  const size_t out_smem = 1024 + 6 * TILE64 + 4 * TILE128 + 256;
+  const size_t out_smem = 1024 + 4 * TILE64 + 4 * TILE128 + 256;
   Args ao = a;
   if (bwd_prep) ao.o = nullptr;  // the backward's recompute only needs v_new from the output kernel
   auto wy = [&](int c0, int c1, cudaStream_t st) {
     return tgo("tc_wy", k_tc_wy, dim3(c1 - c0, p.HV), 256, (size_t)1024 + WySmem::TOTAL, st, p, w,
-               L.t, L.m.k, L.m.v, L.m.WT, L.m.UtT, L.m.DK, 1, c0);
+               L.t, L.m.k, L.m.v, L.m.WT, L.m.UtT, L.m.DK, L.m.NT, 1, c0);
   };
   auto out = [&](int c0, int c1, cudaStream_t st) {
     return tgo("tc_out", k_tc_out, dim3(c1 - c0, p.HV), 256, out_smem, st, p, ao, w, L.t, L.m.q,
@@ -489,7 +534,7 @@ cudaError_t tc_backward(const Problem& p, const Args& a, const Work& w, void* tc
   if (!reuse_fwd && (e = forward_impl(p, a, w, L, true, s)) != cudaSuccess) return e;
   if (!L.ok) return cudaErrorInvalidValue;
   if ((e = tc_backward_kernels(p, a, w, L.t, L.m, s)) != cudaSuccess) return e;
-  return launch_bwd_tokens(p, a, w, true, s);
+  return launch_bwd_tokens(p, a, w, true, s, false);  // dqkwg and wy_bwd write dq, dk
 }
 
 }  // namespace gdn

@@ -182,7 +182,7 @@ struct DqkSmem {
   static constexpr int TOTAL = RED + 64;
 };
 
-__global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
+__global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Args a, Work w, TcWork t,
                                                   const __grid_constant__ CUtensorMap mq,
                                                   const __grid_constant__ CUtensorMap mk,
                                                   const __grid_constant__ CUtensorMap mdO,
@@ -229,7 +229,15 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
     tmem_relinquish();
   }
   // units u = gc * HV + hv in [u0, u1); chunk-table entries past the chunk count are invalid
+  // Units u = chunk * HV + hv in [u0, u1), handed out in k-head groups (chunk, hk) by an atomic
+  // counter: a CTA runs the G value heads of a group back to back and sums their dq and dk
+  // shares itself.  Chunk-table entries past the chunk count are invalid.
   auto valid = [&](int u) { return u >= ur.u0 && u < ur.u1 && w.chunk_tab[u / p.HV].x >= 0; };
+  auto next_of = [&](int u) {  // thread 0: the unit after u (a counter fetch at a group's end)
+    if (u >= 0 && (u % p.HV) % p.G + 1 < p.G) return u + 1;
+    const int kk = ur.u0 / p.G + atomicAdd(ur.ctr, 1);
+    return kk < ur.u1 / p.G ? (kk / p.H) * p.HV + (kk % p.H) * p.G : -1;
+  };
   auto load_A = [&](int u) {
     const int gc = u / p.HV, hk = (u % p.HV) / p.G, tok0 = w.chunk_tab[gc].w;
     mbar_expect_tx(&barA, 4 * TILE64 + TILE128);
@@ -256,7 +264,7 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
   __shared__ int s_unit[2];
   int u = -1;
   if (tid == 0) {
-    u = ur.u0 + atomicAdd(ur.ctr, 1);
+    u = next_of(-1);
     s_unit[0] = u;
   }
   // parity of a load group issued and not yet waited on, or -1 (thread 0 issues all loads)
@@ -282,9 +290,9 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
   for (uint32_t it = 0; valid(u); ++it, u = nu) {
     const int gc = u / p.HV, hv = u % p.HV;
     const int4 e = w.chunk_tab[gc];
-    const int L = e.z;
+    const int L = e.z, tok0 = e.w;
     const size_t unit = (size_t)u;
-    if (tid == 0) s_unit[(it + 1) & 1] = ur.u0 + atomicAdd(ur.ctr, 1);
+    if (tid == 0) s_unit[(it + 1) & 1] = next_of(u);
     const uint32_t ph = it & 1;
     if (tid < 64) sG[tid] = g_next;
     const bool got = mbar_wait(&barA, ph, err) && mbar_wait(&barB, ph, err);
@@ -467,18 +475,48 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Work w, TcWork t,
       pendA = (int)(ph ^ 1);
     }
     {
+      // dq, dk of this value head, summed over the group's value heads in order: the running
+      // sums sit in this CTA's two scratch tiles (fp32, cache-resident); after the last value
+      // head dq is final (bf16 out) and dk goes to the k-head's fp32 tile that wy_bwd completes
       float x[32], y[32];
       tmem_ld16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
       tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), y);
       tmem_wait_ld();
-      float* dq0 = w.dqp + (unit * 64 + r0) * D + 64 * half + cq;
-      float* dk0 = w.dkp + (unit * 64 + r0) * D + 64 * half + cq;
+      const int j = hv % p.G;
+      float* sq0 = w.dqp + ((size_t)blockIdx.x * 64 + r0) * D + 64 * half + cq;
+      float* sk0 = w.dqp + ((size_t)(gridDim.x + blockIdx.x) * 64 + r0) * D + 64 * half + cq;
+      if (j > 0) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        *reinterpret_cast<float2*>(dq0 + 8 * j) = make_float2(x[4 * j], x[4 * j + 1]);
-        *reinterpret_cast<float2*>(dq0 + 8 * D + 8 * j) = make_float2(x[4 * j + 2], x[4 * j + 3]);
-        *reinterpret_cast<float2*>(dk0 + 8 * j) = make_float2(y[4 * j], y[4 * j + 1]);
-        *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j) = make_float2(y[4 * j + 2], y[4 * j + 3]);
+        for (int jj = 0; jj < 8; ++jj) {
+          const float2 a0 = *reinterpret_cast<const float2*>(sq0 + 8 * jj);
+          const float2 a1 = *reinterpret_cast<const float2*>(sq0 + 8 * D + 8 * jj);
+          const float2 b0 = *reinterpret_cast<const float2*>(sk0 + 8 * jj);
+          const float2 b1 = *reinterpret_cast<const float2*>(sk0 + 8 * D + 8 * jj);
+          x[4 * jj] += a0.x; x[4 * jj + 1] += a0.y; x[4 * jj + 2] += a1.x; x[4 * jj + 3] += a1.y;
+          y[4 * jj] += b0.x; y[4 * jj + 1] += b0.y; y[4 * jj + 2] += b1.x; y[4 * jj + 3] += b1.y;
+        }
+      }
+      if (j + 1 < p.G) {
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          *reinterpret_cast<float2*>(sq0 + 8 * jj) = make_float2(x[4 * jj], x[4 * jj + 1]);
+          *reinterpret_cast<float2*>(sq0 + 8 * D + 8 * jj) = make_float2(x[4 * jj + 2], x[4 * jj + 3]);
+          *reinterpret_cast<float2*>(sk0 + 8 * jj) = make_float2(y[4 * jj], y[4 * jj + 1]);
+          *reinterpret_cast<float2*>(sk0 + 8 * D + 8 * jj) = make_float2(y[4 * jj + 2], y[4 * jj + 3]);
+        }
+      } else {
+        const int hk = hv / p.G;
+        float* dk0 = w.dkp + (((size_t)gc * p.H + hk) * 64 + r0) * D + 64 * half + cq;
+        bf16* q0 = static_cast<bf16*>(a.dq) + ((size_t)(tok0 + r0) * p.H + hk) * p.K + 64 * half + cq;
+        bf16* q1 = q0 + (size_t)8 * p.H * p.K;
+        const bool live = 64 * half < p.K;  // columns past a 64-wide key head are padding
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          *reinterpret_cast<float2*>(dk0 + 8 * jj) = make_float2(y[4 * jj], y[4 * jj + 1]);
+          *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * jj) = make_float2(y[4 * jj + 2], y[4 * jj + 3]);
+          if (live && r0 < L) *reinterpret_cast<uint32_t*>(q0 + 8 * jj) = pack_bf16(x[4 * jj], x[4 * jj + 1]);
+          if (live && r1 < L) *reinterpret_cast<uint32_t*>(q1 + 8 * jj) = pack_bf16(x[4 * jj + 2], x[4 * jj + 3]);
+        }
       }
     }
     // the next unit's first MMAs overwrite every TMEM column read above
@@ -564,7 +602,15 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     tmem_alloc(&tslot, 512);
     tmem_relinquish();
   }
+  // Units u = chunk * HV + hv in [u0, u1), handed out in k-head groups (chunk, hk) by an atomic
+  // counter: a CTA runs the G value heads of a group back to back and sums their dq and dk
+  // shares itself.  Chunk-table entries past the chunk count are invalid.
   auto valid = [&](int u) { return u >= ur.u0 && u < ur.u1 && w.chunk_tab[u / p.HV].x >= 0; };
+  auto next_of = [&](int u) {  // thread 0: the unit after u (a counter fetch at a group's end)
+    if (u >= 0 && (u % p.HV) % p.G + 1 < p.G) return u + 1;
+    const int kk = ur.u0 / p.G + atomicAdd(ur.ctr, 1);
+    return kk < ur.u1 / p.G ? (kk / p.H) * p.HV + (kk % p.H) * p.G : -1;
+  };
   auto load_A = [&](int u, int buf) {
     const int hk = (u % p.HV) / p.G, tok0 = w.chunk_tab[u / p.HV].w;
     unsigned char* dst = sKb + buf * 2 * TILE64;
@@ -591,7 +637,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   __shared__ int s_unit[2];
   int u = -1;
   if (tid == 0) {
-    u = ur.u0 + atomicAdd(ur.ctr, 1);
+    u = next_of(-1);
     s_unit[0] = u;
   }
   int pendA = -1, pendB = -1, pendC = -1;  // parity of a load group in flight (thread 0)
@@ -622,8 +668,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     const int gc = u / p.HV, hv = u % p.HV;
     const int4 e = w.chunk_tab[gc];
     const int L = e.z, tok0 = e.w;
-    const size_t unit = (size_t)u;
-    if (tid == 0) s_unit[(it + 1) & 1] = ur.u0 + atomicAdd(ur.ctr, 1);
+    if (tid == 0) s_unit[(it + 1) & 1] = next_of(u);
     const uint32_t ph = it & 1;
     if (tid < 64) {
       sG[tid] = g_next;
@@ -866,16 +911,40 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     ok = __syncthreads_and(ok && mbar_wait(&barM, 1, err));
     tc_fence_after();
     if (!ok) break;
-    {  // this kernel's dk share, added onto dqkwg's in L2 (one reduction per element onto a
-       // value written by the previous kernel: the sum is the same on every run)
+    {  // this kernel's dk share, summed over the group's value heads in order (running sum in
+       // this CTA's scratch tile), then added to dqkwg's k-head tile: dk final, bf16 out
       float x[32];
       tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
       tmem_wait_ld();
-      float* dk0 = w.dkp + (unit * 64 + r0) * D + 64 * half + cq;
+      const int j = hv % p.G;
+      float* s0 = w.dqp + ((size_t)blockIdx.x * 64 + r0) * D + 64 * half + cq;
+      if (j > 0) {
   #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        atomicAdd(reinterpret_cast<float2*>(dk0 + 8 * j), make_float2(x[4 * j], x[4 * j + 1]));
-        atomicAdd(reinterpret_cast<float2*>(dk0 + 8 * D + 8 * j), make_float2(x[4 * j + 2], x[4 * j + 3]));
+        for (int jj = 0; jj < 8; ++jj) {
+          const float2 a0 = *reinterpret_cast<const float2*>(s0 + 8 * jj);
+          const float2 a1 = *reinterpret_cast<const float2*>(s0 + 8 * D + 8 * jj);
+          x[4 * jj] += a0.x; x[4 * jj + 1] += a0.y; x[4 * jj + 2] += a1.x; x[4 * jj + 3] += a1.y;
+        }
+      }
+      if (j + 1 < p.G) {
+  #pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          *reinterpret_cast<float2*>(s0 + 8 * jj) = make_float2(x[4 * jj], x[4 * jj + 1]);
+          *reinterpret_cast<float2*>(s0 + 8 * D + 8 * jj) = make_float2(x[4 * jj + 2], x[4 * jj + 3]);
+        }
+      } else {
+        const int hk = hv / p.G;
+        const float* p0 = w.dkp + (((size_t)gc * p.H + hk) * 64 + r0) * D + 64 * half + cq;
+        bf16* k0 = static_cast<bf16*>(a.dk) + ((size_t)(tok0 + r0) * p.H + hk) * p.K + 64 * half + cq;
+        bf16* k1 = k0 + (size_t)8 * p.H * p.K;
+        const bool live = 64 * half < p.K;
+  #pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const float2 a0 = *reinterpret_cast<const float2*>(p0 + 8 * jj);
+          const float2 a1 = *reinterpret_cast<const float2*>(p0 + 8 * D + 8 * jj);
+          if (live && r0 < L) *reinterpret_cast<uint32_t*>(k0 + 8 * jj) = pack_bf16(x[4 * jj] + a0.x, x[4 * jj + 1] + a0.y);
+          if (live && r1 < L) *reinterpret_cast<uint32_t*>(k1 + 8 * jj) = pack_bf16(x[4 * jj + 2] + a1.x, x[4 * jj + 3] + a1.y);
+        }
       }
     }
     // the next unit's first MMAs overwrite every TMEM column read above
@@ -906,9 +975,11 @@ cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, 
                t, m.q, m.k, m.dO, m.Op, c0);
   };
   auto chunk_kernels = [&](int i, int c0, int c1, cudaStream_t st) {
-    const int units = (c1 - c0) * p.HV;
-    const dim3 gp((unsigned)std::min(units, num_sms()));
-    if ((e = tgo("tc_dqkwg", k_tc_dqkwg, gp, 256, 1024 + DqkSmem::TOTAL, st, p, w, t, m.q, m.k, m.dO,
+    // persistent CTAs over k-head groups; 2 * grid <= units for G >= 2, so every CTA's two
+    // scratch tiles fit in the dq share area
+    const int groups = (c1 - c0) * p.H;
+    const dim3 gp((unsigned)std::min(groups, num_sms()));
+    if ((e = tgo("tc_dqkwg", k_tc_dqkwg, gp, 256, 1024 + DqkSmem::TOTAL, st, p, a, w, t, m.q, m.k, m.dO,
                  m.UT, m.dUT, m.dUTl, m.h, m.dh, m.dW, UnitRange{c0 * p.HV, c1 * p.HV, t.ctr + 2 * i})))
       return e;
     return tgo("tc_wy_bwd", k_tc_wy_bwd, gp, 256, 1024 + WyBwdSmem::TOTAL, st, p, a, w, t, m.k, m.v,

@@ -73,6 +73,7 @@ struct TcMaps {
   CUtensorMap dW;                     // [unit*64][128]      (backward)
   CUtensorMap Tm;                     // [unit*64][64]       (backward)
   CUtensorMap DK;                     // [unit*64][128]      keys scaled by e^{G_C - G_i}
+  CUtensorMap NT;                     // [unit*128][128]     -N^T of the chunk's state map
   CUtensorMap Op;                     // [unit*64][128]      -scale e^{G_i} dO   (backward)
 };
 
@@ -88,6 +89,7 @@ struct TcWork {
   bf16* dUTl;   // [NC*HV][128][64]  dU^T lo part (dU^T - hi)
   bf16* dW;     // [NC*HV][64][128]  dL/dW
   bf16* DK;     // [NC*HV][64][128]  D K = e^{G_C - G_i} k_i (zero past the chunk end), per value head
+  bf16* NT;     // [NC*HV][128 k'][128 k]  -N^T, N = W^T D K (the state map's K x K factor)
   bf16* Op;     // [NC*HV][64][128]  O' = -scale e^{G_i} dO_i (zero past the chunk end)  (backward)
   float* hand;  // [HV][128][128] fp32: the state passed between launches of a segmented pass
   int* ctr;     // [kCounters] work counters of the persistent backward kernels
@@ -175,6 +177,7 @@ inline TcWork carve_tc(void* base, size_t NC, size_t HV, int pass) {
   t.h = reinterpret_cast<bf16*>(take(units * D * D * 2));
   t.Tm = reinterpret_cast<bf16*>(take(units * 2 * 64 * 64 * 2));  // written by every forward
   t.DK = reinterpret_cast<bf16*>(take(units * 64 * D * 2));
+  t.NT = reinterpret_cast<bf16*>(take(units * D * D * 2));
   t.hand = reinterpret_cast<float*>(take(HV * D * D * 4));
   t.ctr = reinterpret_cast<int*>(take(kCounters * sizeof(int)));
   if (pass == 1) {
@@ -190,7 +193,7 @@ inline TcWork carve_tc(void* base, size_t NC, size_t HV, int pass) {
 
 inline size_t tc_bytes(size_t NC, size_t HV, int pass) {
   const size_t units = NC * HV;
-  size_t o = 3 * align_up(units * D * 64 * 2) + align_up(units * D * D * 2);
+  size_t o = 3 * align_up(units * D * 64 * 2) + 2 * align_up(units * D * D * 2);
   o += align_up(units * 2 * 64 * 64 * 2);
   o += align_up(units * 64 * D * 2);
   o += align_up(HV * D * D * 4) + align_up(kCounters * sizeof(int));

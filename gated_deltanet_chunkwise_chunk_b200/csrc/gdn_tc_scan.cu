@@ -30,29 +30,28 @@ __device__ __forceinline__ void st_global_32B(void* p, const uint32_t* v) {
 
 // ======================================================================================
 // Forward.  Thread (warp w, lane l): TMEM lane quarter q = w & 3, row = 32q + l, column group
-// cg = w >> 2 (32 state columns).  Thread 0 issues the MMAs, thread 64 the h stores, thread 96
-// the loads.  Per chunk c, in tensor-pipe order:
+// cg = w >> 2 (32 state columns).  Thread 0 issues the MMAs, thread 96 the loads; every thread
+// writes its part of h (the bf16 state entering each chunk) with plain stores.  -N^T comes ready from the WY kernel, so per chunk c the tensor pipe runs
 //   chain(c)  ACC[c&1] += (-N_c^T) S_c^T       M=128 k', N=128 v, K=128 k   (8 instr)
-//   N(c+1)    NT        = (D K)^T W            M=128 k', N=128 k, K=64 i    (4)
 //   B(c+1)    ACC[~]    = (D K)^T U~           M=128 k', N=128 v, K=64 i    (4)
-// all issued together; the next chain product waits only for the state update and -N^T.
+// and the step's critical path is the chain product, the state update and one barrier.
 // (v_new = U~ - W S^T is left to the output kernel, which reads S anyway: on the sequential
 // pass every tensor-core instruction counts, at roughly 60-130 cycles each.)
-// Shared memory: three input stages {U~^T [128][64], W^T [128][64], D K [64][128]} with e^{G_i},
-// S^T bf16 [128 k][128 v] (MN-major B of the chain), -N^T bf16 [128 k'][128 k].
+// Shared memory: three input stages {U~^T [128][64], -N^T [128][128], D K [64][128]} with
+// e^{G_i}, and S^T bf16 [128 k][128 v] (MN-major B of the chain).
 // ======================================================================================
 struct Fwd2Smem {
-  static constexpr int STAGE = 3 * TILE128;
+  static constexpr int UT = 0, NT = TILE128, DK = 3 * TILE128;   // within a stage
+  static constexpr int STAGE = 4 * TILE128;
   static constexpr int S = 3 * STAGE;
-  static constexpr int N = S + 2 * TILE128;
-  static constexpr int VEC = N + 2 * TILE128;               // 3 x {(unused)[64], e^G[64]}
+  static constexpr int VEC = S + 2 * TILE128;               // 3 x {(unused)[64], e^G[64]}
   static constexpr int TOTAL = VEC + 3 * 512;
 };
+static_assert(1024 + Fwd2Smem::TOTAL + 256 <= 227 * 1024, "forward pass shared memory");
 
 __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
     Problem p, Args a, Work w, TcWork t, const __grid_constant__ CUtensorMap mDK,
-    const __grid_constant__ CUtensorMap mWT, const __grid_constant__ CUtensorMap mUtT,
-    const __grid_constant__ CUtensorMap mh, ScanRange sr) {
+    const __grid_constant__ CUtensorMap mNT, const __grid_constant__ CUtensorMap mUtT, ScanRange sr) {
   // one read of the status word decides for the whole CTA (barriers below need every thread)
   __shared__ int s_fail;
   if (threadIdx.x == 0) s_fail = failed(w);
@@ -69,10 +68,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
   unsigned char* sS = sm + Fwd2Smem::S;
-  unsigned char* sN = sm + Fwd2Smem::N;
   auto stage = [&](int c) { return sm + (c % 3) * Fwd2Smem::STAGE; };
   auto vecp = [&](int c) { return reinterpret_cast<float*>(sm + Fwd2Smem::VEC + (c % 3) * 512); };
-  __shared__ uint64_t barL[3], barC, barN, barE;
+  __shared__ uint64_t barL[3], barC, barE;
   __shared__ uint32_t tslot;
   int* err = w.status;
   // the test flag withholds the first chain product; its wait then runs out quickly
@@ -80,7 +78,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
   if (tid == 0) {
     for (int i = 0; i < 3; ++i) mbar_init(&barL[i], 1);
     mbar_init(&barC, 1);
-    mbar_init(&barN, 1);
     mbar_init(&barE, 1);
     mbar_fence_init();
   }
@@ -90,17 +87,18 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
     tmem_relinquish();
   }
   auto unit_row = [&](int c) { return ((sq.x + c) * p.HV + hv) * D; };
-  // thread 96: chunk c's tiles (U~^T, W^T and D K, written by the WY kernel) and its e^{G_i}
+  // thread 96: chunk c's tiles (U~^T, -N^T and D K, written by the WY kernel) and its e^{G_i}
   auto issue_load = [&](int c) {
     unsigned char* b = stage(c);
     uint64_t* bar = &barL[c % 3];
     const int r = unit_row(c);
     const size_t o = ((size_t)hv * p.NCmax + sq.x + c) * 64;
-    mbar_expect_tx(bar, 2 * TILE128 + 2 * TILE64 + 256);
-    tma_load_3d(b, &mUtT, 0, r, 0, bar);
-    tma_load_3d(b + TILE128, &mWT, 0, r, 0, bar);
-    tma_load_3d(b + 2 * TILE128, &mDK, 0, r / 2, 0, bar);
-    tma_load_3d(b + 2 * TILE128 + TILE64, &mDK, 64, r / 2, 0, bar);
+    mbar_expect_tx(bar, 4 * TILE128 + 256);
+    tma_load_3d(b + Fwd2Smem::UT, &mUtT, 0, r, 0, bar);
+    tma_load_3d(b + Fwd2Smem::NT, &mNT, 0, r, 0, bar);
+    tma_load_3d(b + Fwd2Smem::NT + TILE128, &mNT, 64, r, 0, bar);
+    tma_load_3d(b + Fwd2Smem::DK, &mDK, 0, r / 2, 0, bar);
+    tma_load_3d(b + Fwd2Smem::DK + TILE64, &mDK, 64, r / 2, 0, bar);
     bulk_load(vecp(c) + 64, w.EG + o, 256, bar);
   };
   // chunk c is the (c/3)-th load into stage c%3: its barrier phase has parity (c/3)&1
@@ -120,51 +118,38 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
                                           : make_float4(0, 0, 0, 0);
     S[v] = x.x; S[v + 1] = x.y; S[v + 2] = x.z; S[v + 3] = x.w;
   }
-  auto put_state = [&]() {  // bf16 S^T row part -> the chain operand tile
+  // S^T entering chunk c (this thread's row part) as bf16: the chain operand tile and h[c]
+  auto put_state = [&](int c) {
+    uint32_t pk[16];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) st_chunk_f(sS, row, 4 * cg + j, TILE128, S + 8 * j);
+    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(S[2 * i], S[2 * i + 1]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<uint4*>(sS + sw128_chunk(row, 4 * cg + j, TILE128)) =
+          make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+    bf16* g = t.h + ((size_t)unit_row(c) + row) * D + 32 * cg;
+    st_global_32B(g, pk);
+    st_global_32B(g + 16, pk + 8);
   };
-  auto store_h = [&](int c) {  // thread 64: h[c] <- the S^T tile
-    tma_store_3d(&mh, sS, 0, unit_row(c), 0);
-    tma_store_3d(&mh, sS + TILE128, 64, unit_row(c), 0);
-    tma_store_commit();
-  };
-  if (nc > 0) put_state();
+  if (nc > 0) put_state(0);
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
-  const uint32_t tACC0 = taddr(tb, 0, 0), tNT = taddr(tb, 0, 256);
-  if (tid == 64 && nc > 0) store_h(0);
-  // N(c) into NT and B(c) into ACC[c&1] (K of chunk c already scaled)
-  auto issue_nb = [&](int c) {
+  const uint32_t tACC0 = taddr(tb, 0, 0);
+  // B(c) = (D K)^T U~ into ACC[c&1] (K of chunk c already scaled by D)
+  auto issue_b = [&](int c) {
     unsigned char* b = stage(c);
-    const uint64_t dk = desc_mnmajor(smem_u32(b + 2 * TILE128), 0, TILE64);
-    const uint64_t dw = desc_kmajor(smem_u32(b + TILE128), 0, TILE128);
-    const uint64_t du = desc_kmajor(smem_u32(b), 0, TILE128);
-    constexpr uint32_t id = idesc_bf16(128, 128, true, false);
+    const uint64_t dk = desc_mnmajor(smem_u32(b + Fwd2Smem::DK), 0, TILE64);
+    const uint64_t du = desc_kmajor(smem_u32(b + Fwd2Smem::UT), 0, TILE128);
     const uint32_t tacc = tACC0 + (uint32_t)(128 * (c & 1));
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {  // N and B interleaved (independent accumulators)
-      mma_bf16(tNT, dk + mnstep_off(s), dw + kstep_off(s, TILE128), id, s > 0);
-      mma_bf16(tacc, dk + mnstep_off(s), du + kstep_off(s, TILE128), id, s > 0);
-    }
-    mma_commit(&barN);
-  };
-  // -N^T (TMEM lanes k', columns k) -> bf16 K-major rows of sN; 32 columns per thread
-  auto n_epilogue = [&]() {
-    float x[32];
-    tmem_ld16(taddr(tb, 32 * qd, 256 + 32 * cg), x);
-    tmem_ld16(taddr(tb, 32 * qd, 256 + 32 * cg + 16), x + 16);
-    tmem_wait_ld();
-#pragma unroll
-    for (int q = 0; q < 32; ++q) x[q] = -x[q];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) st_chunk_f(sN, row, 4 * cg + j, TILE128, x + 8 * j);
+    for (int s = 0; s < 4; ++s)
+      mma_bf16(tacc, dk + mnstep_off(s), du + kstep_off(s, TILE128), idesc_bf16(128, 128, true, false), s > 0);
   };
   bool ok = true;
-  // prologue: the first two chunks' tiles, N(0) and B(0), -N_0^T in shared memory
+  // prologue: the first two chunks' tiles, B(0)
   if (nc > 0) {
     bool okp = true;
     for (int c = 0; c < min(2, nc); ++c) okp = okp && mbar_wait(&barL[c], load_par(c), err);
@@ -172,21 +157,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
     ok = __syncthreads_and(okp);
     tc_fence_after();
     if (ok) confirmed = min(2, nc);
-    if (ok && tid == 0) issue_nb(0);
-    okp = ok && mbar_wait(&barN, 0, err);
-    tc_fence_after();
-    if (okp) n_epilogue();
-    fence_proxy_async();
-    tc_fence_before();
-    ok = __syncthreads_and(ok && okp);
-    tc_fence_after();
+    if (ok && tid == 0) issue_b(0);
   }
   for (int c = 0; ok && c < nc; ++c) {
     const bool more = c + 1 < nc;
     const float egc = vecp(c)[64 + 63];
-    // (1) every product of this step at once
+    // (1) the chain product, then the next chunk's state-free product behind it
     if (tid == 0) {
-      const uint64_t da = desc_kmajor(smem_u32(sN), 0, TILE128);
+      const uint64_t da = desc_kmajor(smem_u32(stage(c) + Fwd2Smem::NT), 0, TILE128);
       const uint64_t dsB = desc_mnmajor(smem_u32(sS), 0, TILE128);
       const uint32_t tacc = tACC0 + (uint32_t)(128 * (c & 1));
       if (!(p.test_timeout && c == 0)) {  // the test flag withholds the first chain product
@@ -195,7 +173,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
           mma_bf16(tacc, da + kstep_off(s, TILE128), dsB + mnstep_off(s), idesc_bf16(128, 128, false, true), 1);
         mma_commit(&barC);
       }
-      if (more) issue_nb(c + 1);
+      if (more) issue_b(c + 1);
     }
     // (2) S_{c+1}^T = e^{G_C} S_c^T + ACC
     bool okt = mbar_wait_for(&barC, c & 1, err, wait_limit);
@@ -208,30 +186,19 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
 #pragma unroll
       for (int q = 0; q < 32; ++q) S[q] = egc * S[q] + x[q];
     }
-    // (4) the tiles of the chunk two ahead have landed
+    // (3) the tiles of the chunk two ahead have landed; the next state operand and h[c+1]
     if (c + 2 < nc) okt = okt && mbar_wait(&barL[(c + 2) % 3], load_par(c + 2), err);
-    if (tid == 64) tma_store_wait_read0();  // h[c] has been read out of the S^T tile
+    if (more && okt) put_state(c + 1);
+    fence_proxy_async();
     tc_fence_before();
     ok = __syncthreads_and(ok && okt);
     tc_fence_after();
     if (!ok) break;
     confirmed = min(c + 3, nc);
-    // (5) stage c%3 (its products N(c), B(c) finished before chain(c)) refills with chunk c+3
+    // (4) stage c%3 (chain(c) and B(c) have read it) refills with chunk c+3
     if (loaded < nc) {
       if (tid == 96) issue_load(loaded);
       ++loaded;
-    }
-    // (6) the next step's operands: S_{c+1}^T and -N_{c+1}^T
-    if (more) {
-      put_state();
-      okt = mbar_wait(&barN, (c + 1) & 1, err);
-      tc_fence_after();
-      if (okt) n_epilogue();
-      fence_proxy_async();
-      tc_fence_before();
-      ok = __syncthreads_and(ok && okt);
-      tc_fence_after();
-      if (ok && tid == 64) store_h(c + 1);
     }
   }
   if (ok && sr.s_out && st_live) {  // the final state, or the state handed to the next launch
@@ -243,7 +210,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
   // CTA frees its tensor memory and leaves
   if (!ok && tid == 96)
     for (int c = confirmed; c < loaded; ++c) mbar_wait(&barL[c % 3], load_par(c), nullptr);
-  if (tid == 64) tma_store_wait0();
   if (tid == 0) {
     mma_commit(&barE);
     mbar_wait(&barE, 0, nullptr);
@@ -258,38 +224,38 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
 // everything transposed (TMEM lane = key index k):
 //   dS_c^T = e^{G_C} dS'^T - ACC,   ACC = W^T dU_loc + Q^T O' + N dS'^T,  O' = -scale e^G dO
 //   dU_c^T = dU_loc^T + dS' K^T D                      (written out as a bf16 hi/lo pair)
-// Per chunk, in tensor-pipe order:
-//   N(c)     NT   = W^T (D K)                 M=128 k, N=128 k'', K=64 i   (4 instr)
-//   dU(c)    DU   = dS' (D K)^T, hi + lo      M=128 v, N=64 i,   K=128 k   (16)
-//   ... O' scaled, N copied to shared memory ...
-//   I(c)     DU  += dU_loc^T I                M=128 v, N=64 i,   K=64 i'   (4)
-//   F(c)     ACC  = W^T dU_loc + Q^T O'       M=128 k, N=128 v,  K=64 i    (8)
-//   chain(c) ACC += N (dS'^T hi + lo)         M=128 k, N=128 v,  K=128 k'' (16)
-// dU_loc enters dU through the identity product, so once F(c) has run, the slot of Q, dO and
-// dU_loc is free and the previous chunk's tiles stream in while the chain product runs.
-// Shared memory: two slots of {D K [64][128], W^T [128][64]} with e^{G_i}, one of {Q [64][128],
-// O' [64][128], dU_loc^T [128][64]}, N bf16 [128][128] (K-major A), dS'^T hi and lo
-// [128 k''][128 v], the 64 x 64 identity.  D K comes from the WY kernel and O' from dv_local.
+// -N^T comes ready from the WY kernel (read here as an MN-major A operand with the negate bit
+// set), O' from dv_local.  Per chunk, in tensor-pipe order:
+//   chain(c)  ACC[c&1] += N (dS'^T hi + lo)       M=128 k, N=128 v, K=128 k''  (16 instr)
+//   dU(c)     DU[c&1]  += dS' (D K)^T, hi + lo    M=128 v, N=64 i,  K=128 k    (16)
+//   I(c-1)    DU[~]     = dU_loc^T I              M=128 v, N=64 i,  K=64 i'    (4)
+//   F(c-1)    ACC[~]    = W^T dU_loc + Q^T O'     M=128 k, N=128 v, K=64 i     (8)
+// The state-free products of the next chunk go in behind this chunk's, into the other
+// accumulators, so the pipe keeps working while the state is updated and written back.
+// Shared memory: two slots of -N^T [128][128] with e^{G_i}; one of D K [64][128]; one of
+// {Q [64][128], O' [64][128], W^T [128][64], dU_loc^T [128][64]}; dS'^T hi and lo [128][128];
+// the 64 x 64 identity.
 // ======================================================================================
 struct Bwd2Smem {
-  static constexpr int KW = 0;                              // 2 x {K (2 x TILE64), W^T}
-  static constexpr int KW_BYTES = 2 * TILE128;
-  static constexpr int Q = 2 * KW_BYTES;
+  static constexpr int NS = 0;                              // 2 x -N^T (two 64-column boxes)
+  static constexpr int DK = 4 * TILE128;
+  static constexpr int Q = DK + TILE128;
   static constexpr int O = Q + TILE128;
-  static constexpr int UL = O + TILE128;
-  static constexpr int N = UL + TILE128;
-  static constexpr int DSH = N + 2 * TILE128;
+  static constexpr int W = O + TILE128;
+  static constexpr int UL = W + TILE128;
+  static constexpr int DSH = UL + TILE128;
   static constexpr int DSL = DSH + 2 * TILE128;
   static constexpr int ID = DSL + 2 * TILE128;              // identity [64][64] bf16
-  static constexpr int VEC = ID + TILE64;                   // 2 x {D[64], e^G[64]} (raw)
-  static constexpr int TOTAL = VEC + 2 * 512;
+  static constexpr int VEC = ID + TILE64;                   // 2 x e^G[64]
+  static constexpr int TOTAL = VEC + 2 * 256;
 };
+static_assert(1024 + Bwd2Smem::TOTAL + 256 <= 227 * 1024, "backward pass shared memory");
 
 __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
     Problem p, Args a, Work w, TcWork t, const __grid_constant__ CUtensorMap mq,
     const __grid_constant__ CUtensorMap mDK, const __grid_constant__ CUtensorMap mOp,
     const __grid_constant__ CUtensorMap mWT, const __grid_constant__ CUtensorMap mdUlT,
-    const __grid_constant__ CUtensorMap mdh, ScanRange sr) {
+    const __grid_constant__ CUtensorMap mNT, ScanRange sr) {
   __shared__ int s_fail;
   if (threadIdx.x == 0) s_fail = failed(w);
   __syncthreads();
@@ -302,27 +268,27 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
   const int qd = warp & 3, cg = warp >> 2, row = 32 * qd + lane;
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
+  unsigned char* sDKt = sm + Bwd2Smem::DK;
   unsigned char* sQ = sm + Bwd2Smem::Q;
   unsigned char* sO = sm + Bwd2Smem::O;
+  unsigned char* sW = sm + Bwd2Smem::W;
   unsigned char* sUl = sm + Bwd2Smem::UL;
-  unsigned char* sN = sm + Bwd2Smem::N;
   unsigned char* sDH = sm + Bwd2Smem::DSH;
   unsigned char* sDL = sm + Bwd2Smem::DSL;
   unsigned char* sI = sm + Bwd2Smem::ID;
-  auto sK = [&](int c) { return sm + Bwd2Smem::KW + (c & 1) * Bwd2Smem::KW_BYTES; };
-  auto sW = [&](int c) { return sK(c) + TILE128; };
-  auto vecp = [&](int c) { return reinterpret_cast<float*>(sm + Bwd2Smem::VEC + (c & 1) * 512); };
-  __shared__ uint64_t barKW[2], barQOU, barN, barDU, barF, barC, barE;
+  auto sN = [&](int c) { return sm + Bwd2Smem::NS + (c & 1) * 2 * TILE128; };
+  auto vecp = [&](int c) { return reinterpret_cast<float*>(sm + Bwd2Smem::VEC + (c & 1) * 256); };
+  __shared__ uint64_t barN[2], barDK, barQ, barF, barC, barDU, barE;
   __shared__ uint32_t tslot;
   int* err = w.status;
   if (tid == 0) {
-    mbar_init(&barKW[0], 1);
-    mbar_init(&barKW[1], 1);
-    mbar_init(&barQOU, 1);
-    mbar_init(&barN, 1);
-    mbar_init(&barDU, 1);
+    mbar_init(&barN[0], 1);
+    mbar_init(&barN[1], 1);
+    mbar_init(&barDK, 1);
+    mbar_init(&barQ, 1);
     mbar_init(&barF, 1);
     mbar_init(&barC, 1);
+    mbar_init(&barDU, 1);
     mbar_init(&barE, 1);
     mbar_fence_init();
   }
@@ -333,34 +299,48 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
   }
   auto unit_row = [&](int c) { return ((sq.x + c) * p.HV + hv) * D; };
   auto tok_of = [&](int c) { return sq.z + 64 * c; };
-  // chunks are loaded in iteration order nc-1, nc-2, ...: chunk c's {K, W} is the j-th load
-  // into slot c&1 with j = (nc-1-c)/2, its {Q, dO, dU_loc} the (nc-1-c)-th into their slot
-  auto kw_par = [&](int c) { return (uint32_t)(((nc - 1 - c) >> 1) & 1); };
-  auto qou_par = [&](int c) { return (uint32_t)((nc - 1 - c) & 1); };
-  // thread 32: chunk c's D K (the WY kernel's) and W^T, and its e^{G_i}
-  auto issue_kw = [&](int c) {
-    uint64_t* bar = &barKW[c & 1];
+  // Chunks go in iteration order nc-1, nc-2, ...  A single-slot barrier (D K; Q, O', W, dU_loc;
+  // and the commit barriers) completes its j-th phase for chunk nc-1-j; the -N^T slot c&1
+  // completes its j-th phase for chunk nc-1-2j-((nc-1-c)&1).
+  auto par = [&](int c) { return (uint32_t)((nc - 1 - c) & 1); };
+  auto npar = [&](int c) { return (uint32_t)(((nc - 1 - c) >> 1) & 1); };
+  // loads issued per barrier, counted by the issuing thread: on an error exit it waits for the
+  // last one of each (phases complete in order, so the others have landed too)
+  int n_iss0 = 0, n_iss1 = 0, dk_iss = 0, q_iss = 0;
+  // thread 32: chunk c's -N^T and e^{G_i}; its D K
+  auto issue_n = [&](int c) {
+    uint64_t* bar = &barN[c & 1];
     const size_t o = ((size_t)hv * p.NCmax + sq.x + c) * 64;
     mbar_expect_tx(bar, 2 * TILE128 + 256);
-    tma_load_3d(sK(c), &mDK, 0, unit_row(c) / 2, 0, bar);
-    tma_load_3d(sK(c) + TILE64, &mDK, 64, unit_row(c) / 2, 0, bar);
-    tma_load_3d(sW(c), &mWT, 0, unit_row(c), 0, bar);
-    bulk_load(vecp(c) + 64, w.EG + o, 256, bar);
+    tma_load_3d(sN(c), &mNT, 0, unit_row(c), 0, bar);
+    tma_load_3d(sN(c) + TILE128, &mNT, 64, unit_row(c), 0, bar);
+    bulk_load(vecp(c), w.EG + o, 256, bar);
+    if (c & 1) ++n_iss1; else ++n_iss0;
   };
-  // thread 96: chunk c's Q, O' = -scale e^G dO (the dv_local kernel's) and dU_loc^T
-  auto issue_qou = [&](int c) {
-    mbar_expect_tx(&barQOU, 3 * TILE128);
-    tma_load_3d(sQ, &mq, 0, hk, tok_of(c), &barQOU);
-    tma_load_3d(sQ + TILE64, &mq, 64, hk, tok_of(c), &barQOU);
-    tma_load_3d(sO, &mOp, 0, unit_row(c) / 2, 0, &barQOU);
-    tma_load_3d(sO + TILE64, &mOp, 64, unit_row(c) / 2, 0, &barQOU);
-    tma_load_3d(sUl, &mdUlT, 0, unit_row(c), 0, &barQOU);
+  auto issue_dk = [&](int c) {
+    mbar_expect_tx(&barDK, TILE128);
+    tma_load_3d(sDKt, &mDK, 0, unit_row(c) / 2, 0, &barDK);
+    tma_load_3d(sDKt + TILE64, &mDK, 64, unit_row(c) / 2, 0, &barDK);
+    ++dk_iss;
   };
-  int kw_issued = 0, qou_issued = 0;  // loads issued, in iteration order (same count in every thread)
-  int kw_seen = 0, qou_seen = 0;      // loads every thread saw complete
-  if (tid == 32 && nc > 0) issue_kw(nc - 1);
-  if (tid == 96 && nc > 0) issue_qou(nc - 1);
-  if (nc > 0) kw_issued = qou_issued = 1;
+  // thread 96: chunk c's Q, O' = -scale e^G dO (the dv_local kernel's), W^T and dU_loc^T
+  auto issue_q = [&](int c) {
+    mbar_expect_tx(&barQ, 4 * TILE128);
+    tma_load_3d(sQ, &mq, 0, hk, tok_of(c), &barQ);
+    tma_load_3d(sQ + TILE64, &mq, 64, hk, tok_of(c), &barQ);
+    tma_load_3d(sO, &mOp, 0, unit_row(c) / 2, 0, &barQ);
+    tma_load_3d(sO + TILE64, &mOp, 64, unit_row(c) / 2, 0, &barQ);
+    tma_load_3d(sW, &mWT, 0, unit_row(c), 0, &barQ);
+    tma_load_3d(sUl, &mdUlT, 0, unit_row(c), 0, &barQ);
+    ++q_iss;
+  };
+  if (nc > 0) {
+    if (tid == 32) {
+      issue_n(nc - 1);
+      issue_dk(nc - 1);
+    }
+    if (tid == 96) issue_q(nc - 1);
+  }
   // this thread's part of dS'^T: row `row`, columns 32 cg .. 32 cg + 31
   float S[32];
   // states are [Nst][HV][K][V]; rows k >= K and columns v >= V of a narrower head are padding
@@ -379,114 +359,120 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
     for (int q = 0; q < 8; ++q) f[q] = (8 * j + q == r) ? 1.f : 0.f;
     st_chunk_f(sI, r, j, TILE64, f);
   }
-  auto put_state = [&]() {  // dS'^T row part as a compensated bf16 pair
+  // dS'^T leaving chunk c (this thread's row part) as a compensated bf16 pair for the next
+  // products, and its hi part as dh[c]
+  auto put_state = [&](int c) {
+    uint32_t ph[16], pl[16];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) st_chunk_split(sDH, sDL, row, 4 * cg + j, TILE128, S + 8 * j);
+    for (int i = 0; i < 16; ++i) {
+      const float h0 = __bfloat162float(__float2bfloat16_rn(S[2 * i]));
+      const float h1 = __bfloat162float(__float2bfloat16_rn(S[2 * i + 1]));
+      ph[i] = pack_bf16(h0, h1);
+      pl[i] = pack_bf16(S[2 * i] - h0, S[2 * i + 1] - h1);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t o = sw128_chunk(row, 4 * cg + j, TILE128);
+      *reinterpret_cast<uint4*>(sDH + o) = make_uint4(ph[4 * j], ph[4 * j + 1], ph[4 * j + 2], ph[4 * j + 3]);
+      *reinterpret_cast<uint4*>(sDL + o) = make_uint4(pl[4 * j], pl[4 * j + 1], pl[4 * j + 2], pl[4 * j + 3]);
+    }
+    bf16* g = t.dh + ((size_t)unit_row(c) + row) * D + 32 * cg;
+    st_global_32B(g, ph);
+    st_global_32B(g + 16, ph + 8);
   };
-  auto store_dh = [&](int c) {  // thread 64: dh[c] <- the hi tile
-    tma_store_3d(&mdh, sDH, 0, unit_row(c), 0);
-    tma_store_3d(&mdh, sDH + TILE128, 64, unit_row(c), 0);
-    tma_store_commit();
-  };
-  if (nc > 0) put_state();
+  if (nc > 0) put_state(nc - 1);
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
-  const uint32_t tACC = taddr(tb, 0, 0), tNT = taddr(tb, 0, 128), tDU = taddr(tb, 0, 256);
-  if (tid == 64 && nc > 0) store_dh(nc - 1);
+  auto tACC = [&](int c) { return taddr(tb, 0, 128 * (c & 1)); };
+  auto tDU = [&](int c) { return taddr(tb, 0, 256 + 64 * (c & 1)); };
+  // I(c) and F(c): the state-free products of chunk c (thread 0)
+  auto issue_if = [&](int c) {
+    const uint64_t dul = desc_kmajor(smem_u32(sUl), 0, TILE128);
+    const uint64_t di = desc_kmajor(smem_u32(sI), 0, TILE64);
+    const uint64_t dwA = desc_kmajor(smem_u32(sW), 0, TILE128);
+    const uint64_t dq = desc_mnmajor(smem_u32(sQ), 0, TILE64);
+    const uint64_t dO_ = desc_mnmajor(smem_u32(sO), 0, TILE64);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      mma_bf16(tDU(c), dul + kstep_off(s, TILE128), di + kstep_off(s, TILE64), idesc_bf16(128, 64, false, false), s > 0);
+      mma_bf16(tACC(c), dwA + kstep_off(s, TILE128), dul + kstep_off(s, TILE128),
+               idesc_bf16(128, 128, false, false), s > 0);
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+      mma_bf16(tACC(c), dq + mnstep_off(s), dO_ + mnstep_off(s), idesc_bf16(128, 128, true, true), 1);
+    mma_commit(&barF);
+  };
   bool ok = true;
-  if (nc > 0) {  // the first chunk's D K and W^T
-    bool okp = mbar_wait(&barKW[(nc - 1) & 1], kw_par(nc - 1), err);
+  if (nc > 0) {  // the last chunk's Q, O', W, dU_loc, then its state-free products
+    const bool okp = mbar_wait(&barQ, par(nc - 1), err);
     tc_fence_before();
     ok = __syncthreads_and(okp);
     tc_fence_after();
-    if (ok) kw_seen = 1;
+    if (ok && tid == 0) issue_if(nc - 1);
   }
+  // the chain's A operand: -N^T read MN-major is -N; the negate bit makes it N
+  constexpr uint32_t kNegA = 1u << 13;
   for (int idx = 0; ok && idx < nc; ++idx) {
     const int c = nc - 1 - idx;
     const bool more = c > 0;
-    const float* vc = vecp(c);
-    // (1) N(c), dU(c) (state and K only); the previous chunk's K and W stream into the other slot
-    if (tid == 0) {
-      const uint64_t dw = desc_kmajor(smem_u32(sW(c)), 0, TILE128);
-      const uint64_t dkB = desc_mnmajor(smem_u32(sK(c)), 0, TILE64);
-      constexpr uint32_t idN = idesc_bf16(128, 128, false, true);
-      const uint64_t dkK = desc_kmajor(smem_u32(sK(c)), 0, TILE64);
-      constexpr uint32_t idU = idesc_bf16(128, 64, true, false);
+    // (1) chunk c's -N^T; the chain product, then dU(c) once D K has landed
+    bool okt = mbar_wait(&barN[c & 1], npar(c), err);
+    tc_fence_after();
+    const float egc = vecp(c)[63];
+    if (tid == 0 && okt) {
+      const uint64_t dn = desc_mnmajor(smem_u32(sN(c)), 0, TILE128);
       const uint64_t dah = desc_mnmajor(smem_u32(sDH), 0, TILE128);
       const uint64_t dal = desc_mnmajor(smem_u32(sDL), 0, TILE128);
-      // N = W^T (D K) interleaved with dU^T = dS' (D K)^T (hi, then lo): independent accumulators
+      constexpr uint32_t idC = idesc_bf16(128, 128, true, true) | kNegA;
 #pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        if (s < 4) mma_bf16(tNT, dw + kstep_off(s, TILE128), dkB + mnstep_off(s), idN, s > 0);
-        mma_bf16(tDU, dah + mnstep_off(s), dkK + kstep_off(s, TILE64), idU, s > 0);
+      for (int s = 0; s < 8; ++s) mma_bf16(tACC(c), dn + mnstep_off(s), dah + mnstep_off(s), idC, 1);
+#pragma unroll
+      for (int s = 0; s < 8; ++s) mma_bf16(tACC(c), dn + mnstep_off(s), dal + mnstep_off(s), idC, 1);
+      mma_commit(&barC);
+      okt = mbar_wait(&barDK, par(c), err);
+      tc_fence_after();
+      if (okt) {
+        const uint64_t dkK = desc_kmajor(smem_u32(sDKt), 0, TILE64);
+        constexpr uint32_t idU = idesc_bf16(128, 64, true, false);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) mma_bf16(tDU(c), dah + mnstep_off(s), dkK + kstep_off(s, TILE64), idU, 1);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) mma_bf16(tDU(c), dal + mnstep_off(s), dkK + kstep_off(s, TILE64), idU, 1);
+        mma_commit(&barDU);
       }
-      mma_commit(&barN);
-#pragma unroll
-      for (int s = 0; s < 8; ++s) mma_bf16(tDU, dal + mnstep_off(s), dkK + kstep_off(s, TILE64), idU, 1);
     }
-    if (tid == 32 && more) issue_kw(c - 1);
-    if (more) ++kw_issued;
-    if (tid == 64) tma_store_wait_read0();  // the last dh store has read the hi tile
-    // (2) this chunk's Q, O', dU_loc; N -> shared memory
-    bool okt = mbar_wait(&barQOU, qou_par(c), err);
-    okt = okt && mbar_wait(&barN, idx & 1, err);
+    // the slot of chunk c+1's -N^T (its chain product finished) takes chunk c-1's
+    if (tid == 32 && more) issue_n(c - 1);
+    // chunk c's F and I have run: the next chunk's Q, O', W, dU_loc replace theirs
+    if (tid == 96 && more && mbar_wait(&barF, par(c), err)) issue_q(c - 1);
+    // (2) dS_c^T = e^{G_C} dS'^T - ACC
+    okt = okt && mbar_wait(&barC, par(c), err);
     tc_fence_after();
     if (okt) {
       float x[32];
-      tmem_ld16(taddr(tb, 32 * qd, 128 + 32 * cg), x);
-      tmem_ld16(taddr(tb, 32 * qd, 128 + 32 * cg + 16), x + 16);
+      tmem_ld16(taddr(tb, 32 * qd, 128 * (c & 1) + 32 * cg), x);
+      tmem_ld16(taddr(tb, 32 * qd, 128 * (c & 1) + 32 * cg + 16), x + 16);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 4; ++j) st_chunk_f(sN, row, 4 * cg + j, TILE128, x + 8 * j);
+      for (int q = 0; q < 32; ++q) S[q] = egc * S[q] - x[q];
     }
-    fence_proxy_async();
-    tc_fence_before();
-    ok = __syncthreads_and(ok && okt);
-    tc_fence_after();
-    if (!ok) break;
-    qou_seen = idx + 1;
-    // (3) dU_loc into dU, F, then the chain product
-    if (tid == 0) {
-      const uint64_t dul = desc_kmajor(smem_u32(sUl), 0, TILE128);
-      const uint64_t di = desc_kmajor(smem_u32(sI), 0, TILE64);
-      const uint64_t dwA = desc_kmajor(smem_u32(sW(c)), 0, TILE128);
-      const uint64_t dq = desc_mnmajor(smem_u32(sQ), 0, TILE64);
-      const uint64_t dO_ = desc_mnmajor(smem_u32(sO), 0, TILE64);
-      // dU^T += dU_loc^T I interleaved with F = W^T dU_loc + Q^T O'
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        mma_bf16(tDU, dul + kstep_off(s, TILE128), di + kstep_off(s, TILE64), idesc_bf16(128, 64, false, false), 1);
-        mma_bf16(tACC, dwA + kstep_off(s, TILE128), dul + kstep_off(s, TILE128),
-                 idesc_bf16(128, 128, false, false), s > 0);
-      }
-      mma_commit(&barDU);
-#pragma unroll
-      for (int s = 0; s < 4; ++s)
-        mma_bf16(tACC, dq + mnstep_off(s), dO_ + mnstep_off(s), idesc_bf16(128, 128, true, true), 1);
-      mma_commit(&barF);
-      const uint64_t dn = desc_kmajor(smem_u32(sN), 0, TILE128);
-      for (int part = 0; part < 2; ++part) {
-        const uint64_t db = desc_mnmajor(smem_u32(part ? sDL : sDH), 0, TILE128);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)  // + N dS'^T, hi then lo
-          mma_bf16(tACC, dn + kstep_off(s, TILE128), db + mnstep_off(s), idesc_bf16(128, 128, false, true), 1);
-      }
-      mma_commit(&barC);
+    // the previous chunk's state-free products go in behind this chunk's
+    if (tid == 0 && more && okt) {
+      okt = mbar_wait(&barQ, par(c - 1), err);
+      tc_fence_after();
+      if (okt) issue_if(c - 1);
     }
-    // (4) the previous chunk's Q, dO, dU_loc once F has read this chunk's
-    if (tid == 96 && more) {
-      if (mbar_wait(&barF, idx & 1, err)) issue_qou(c - 1);
-    }
-    if (more) ++qou_issued;
-    // dU^T = DU as a hi/lo pair (rows v, 16 columns per thread), straight to the workspace
-    okt = mbar_wait(&barDU, idx & 1, err);
+    // (3) dU^T = DU as a hi/lo pair (rows v, 16 columns per thread), straight to the workspace
+    okt = okt && mbar_wait(&barDU, par(c), err);
     tc_fence_after();
     if (okt) {
+      if (tid == 32 && more) issue_dk(c - 1);  // dU(c) has read D K
       float x[16];
-      tmem_ld16(taddr(tb, 32 * qd, 256 + 16 * cg), x);
+      tmem_ld16(taddr(tb, 32 * qd, 256 + 64 * (c & 1) + 16 * cg), x);
       tmem_wait_ld();
       bf16* hrow = t.dUT + ((size_t)unit_row(c) + row) * 64 + 16 * cg;
       bf16* lrow = t.dUTl + ((size_t)unit_row(c) + row) * 64 + 16 * cg;
@@ -500,42 +486,27 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
       }
       st_global_32B(hrow, ph);  // 16 columns = one full 32-byte sector per row and part
       st_global_32B(lrow, pl);
-    }
-    // the previous chunk's D K and W^T have landed
-    if (more) okt = okt && mbar_wait(&barKW[(c - 1) & 1], kw_par(c - 1), err);
-    // dS_c^T = e^{G_C} dS'^T - ACC, then its hi/lo copy for the next step
-    okt = okt && mbar_wait(&barC, idx & 1, err);
-    tc_fence_after();
-    if (okt) {
-      const float egc = vc[64 + 63];
-      float x[32];
-      tmem_ld16(taddr(tb, 32 * qd, 32 * cg), x);
-      tmem_ld16(taddr(tb, 32 * qd, 32 * cg + 16), x + 16);
-      tmem_wait_ld();
-#pragma unroll
-      for (int q = 0; q < 32; ++q) S[q] = egc * S[q] - x[q];
-      if (more) put_state();
+      // (4) both products of chunk c have read dS'^T: the next one (and dh[c-1]) replaces it
+      if (more) put_state(c - 1);
     }
     fence_proxy_async();
     tc_fence_before();
     ok = __syncthreads_and(ok && okt);
     tc_fence_after();
-    if (!ok) break;
-    if (more) kw_seen = idx + 2;
-    // (5) dh of chunk c-1: the gradient leaving it (a launch over earlier chunks writes the one
-    // leaving chunk cb-1 itself, from the state this launch hands on)
-    if (tid == 64 && more) store_dh(c - 1);
   }
   if (ok && sr.s_out && st_live) {  // dh0, or the gradient handed to the launch of earlier chunks
 #pragma unroll
     for (int v = 0; v < 32; v += 4)
       *reinterpret_cast<float4*>(sr.s_out + st_off + v) = make_float4(S[v], S[v + 1], S[v + 2], S[v + 3]);
   }
-  if (!ok && tid == 32)  // let issued loads land before the CTA leaves
-    for (int j = kw_seen; j < kw_issued; ++j) mbar_wait(&barKW[(nc - 1 - j) & 1], kw_par(nc - 1 - j), nullptr);
-  if (!ok && tid == 96)
-    for (int j = qou_seen; j < qou_issued; ++j) mbar_wait(&barQOU, qou_par(nc - 1 - j), nullptr);
-  if (tid == 64) tma_store_wait0();
+  // before the CTA leaves (after an error too): the last load on each barrier has landed, so
+  // every earlier one has; every MMA issued has finished
+  if (tid == 32) {
+    if (n_iss0 > 0) mbar_wait(&barN[0], (uint32_t)((n_iss0 - 1) & 1), nullptr);
+    if (n_iss1 > 0) mbar_wait(&barN[1], (uint32_t)((n_iss1 - 1) & 1), nullptr);
+    if (dk_iss > 0) mbar_wait(&barDK, (uint32_t)((dk_iss - 1) & 1), nullptr);
+  }
+  if (tid == 96 && q_iss > 0) mbar_wait(&barQ, (uint32_t)((q_iss - 1) & 1), nullptr);
   if (tid == 0) {
     mma_commit(&barE);
     mbar_wait(&barE, 0, nullptr);
@@ -551,14 +522,14 @@ cudaError_t tc_scan_fwd(const Problem& p, const Args& a, const Work& w, const Tc
                         const TcMaps& m, const ScanRange& sr, cudaStream_t s) {
   const dim3 grid(p.Nst, p.HV);
   return tgo("tc_scan_fwd", k_tc_scan_fwd2, grid, kScanThreads, (size_t)1024 + Fwd2Smem::TOTAL, s, p, a,
-             w, t, m.DK, m.WT, m.UtT, m.h, sr);
+             w, t, m.DK, m.NT, m.UtT, sr);
 }
 
 cudaError_t tc_scan_bwd(const Problem& p, const Args& a, const Work& w, const TcWork& t,
                         const TcMaps& m, const ScanRange& sr, cudaStream_t s) {
   const dim3 grid(p.Nst, p.HV);
   return tgo("tc_scan_bwd", k_tc_scan_bwd2, grid, kScanThreads, (size_t)1024 + Bwd2Smem::TOTAL, s, p, a,
-             w, t, m.q, m.DK, m.Op, m.WT, m.dUlT, m.dh, sr);
+             w, t, m.q, m.DK, m.Op, m.WT, m.dUlT, m.NT, sr);
 }
 
 }  // namespace tcx

@@ -61,6 +61,33 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
   return mbar_wait_for(bar, parity, err, 1ll << 31);
 }
 
+// The same, also giving up as soon as *abort is non-zero: a shared flag that any thread of the
+// CTA sets when one of its waits runs out (a timeout here sets it too), so that a CTA whose
+// roles hand work to each other through barriers winds down together.
+__device__ __forceinline__ bool mbar_wait_abort(uint64_t* bar, uint32_t parity, int* err,
+                                                volatile int* abort, long long limit = 1ll << 31) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > limit) {
+      if (err) atomicExch(err, 5 /* GDN_ERR_TIMEOUT */);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// Named CTA barriers (ids 1..15; 0 is __syncthreads): producers arrive without waiting, the
+// consumer warp waits until `count` threads (a multiple of 32) have arrived or synced.
+__device__ __forceinline__ void nbar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void nbar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ------------------------------------------------------------------ fences
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -67,6 +67,16 @@ def test_head_dims(dtype, KV):
     _assert_parity(case)
 
 
+@pytest.mark.parametrize("H,HV,lengths", [(2, 2, None), (1, 4, None), (2, 8, [70, 0, 129, 5]),
+                                           (1, 8, [300])])
+def test_value_head_groups_bf16(H, HV, lengths):
+    """G = HV/H value heads share a k-head: dq and dk are sums over the group, which the
+    tensor-core backward forms inside its kernels (G = 1, 4, 8)."""
+    case = synth.make_case(B=1 if lengths else 2, T=300, H=H, HV=HV, K=128, V=128, dtype="bf16",
+                           seed=90 + HV, lengths=lengths, h0=True, dht=True, name=f"H{H}HV{HV}")
+    _assert_parity(case)
+
+
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 def test_varlen_ragged(dtype):
     lens = [1, 63, 64, 65, 127, 128, 129, 300, 0, 17]
