@@ -335,9 +335,9 @@ def main():
         "config": {"workload": case.name, "B": case.B, "T": case.T, "H": case.H, "HV": case.HV,
                    "K": case.K, "V": case.V, "chunk": C, "global_batch": case.B * world,
                    "seq_len": case.T, "parallelism": f"dp{world} (independent batches)",
-                   "l2": "no flush: each step streams ~1 GB (inputs alone > 126 MB L2)"},
+                   "l2": m["l2"]},
     }
-    line.update({k: v for k, v in m.items() if k not in ("value", "ms_per_step")})
+    line.update({k: v for k, v in m.items() if k not in ("value", "ms_per_step", "l2")})
     line.update({"decode": decode, "kda_gate": kda, "kda_decode": kda_decode, "kda_chunk": kda_chunk,
                  "peaks_source": peaks()["source"]})
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -361,6 +361,17 @@ def main():
                 sub["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
             others[f"config{idx}"] = sub
             del oc
+        # the one shape the G_T_CONTIG page times itself (section on measured gains):
+        # B=2, T=2048, H=4, HV=8 with 64-wide key and value heads
+        pc = synth.make_case(B=2, T=2048, H=4, HV=8, K=64, V=64, dtype="bf16", seed=1100 + 7919 * rank,
+                             name="bf16_B2_T2048_H4_HV8_D64")
+        sub = measure_case(gdn, pc, dev, args.steps, args.warmup, dist, world, sampler=None, e2e_steps=3)
+        sub["config"] = {"workload": pc.name, "B": pc.B, "T": pc.T, "tokens": pc.tokens, "H": pc.H,
+                         "HV": pc.HV, "K": pc.K, "V": pc.V, "dtype": pc.dtype}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            cb = oracle_sample(pc, budget_s=6.0)
+            sub["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        others["pages_k64"] = sub
         line["other_workloads"] = others
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -401,20 +412,38 @@ def measure_case(gdn, case, dev, steps: int, warmup: int, dist, world: int, samp
         gdn.gdn_chunk_bwd(**inp, d_o=dO, dht=dht, workspace=ws, outs=outs, reuse_forward=True)
 
     stream = torch.cuda.current_stream()
+    # a workload whose tensors fit in L2 (126 MB) is timed one step at a time with L2 flushed
+    # before each (a 256 MB write outside the timed events); a larger one streams its inputs
+    # from HBM anyway and is timed as one run of steps
+    footprint = sum(x.numel() * x.element_size() for x in list(inp.values()) + [dO, dht]
+                    if x is not None)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if footprint < (256 << 20) else None
 
     def timed(fn, n):
         if dist:
             dist.barrier()
         torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(n):
-            fn()
-        b.record(stream)
-        torch.cuda.synchronize()
+        if flush is None:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(n):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            total = a.elapsed_time(b)
+        else:
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(n)]
+            for a, b in ev:
+                flush.zero_()
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+            total = sum(a.elapsed_time(b) for a, b in ev)
         if dist:
             dist.barrier()
-        return a.elapsed_time(b) / n
+        return total / n
 
     for _ in range(warmup):
         step()
@@ -467,10 +496,12 @@ def measure_case(gdn, case, dev, steps: int, warmup: int, dist, world: int, samp
         "gpu_launches": int(launches),
         "e2e": e2e,
         "clocks": clocks,
+        "l2": ("flushed before each timed step (256 MB write outside the events)" if flush is not None
+               else "no flush: the step's tensors exceed 256 MB, twice the 126 MB L2"),
     }
 
 
-def kernel_roofline(prof: dict, case, pk: dict) -> dict | None:
+def kernel_roofline(prof: dict, case, pk: dict, steps: int = 2) -> dict | None:
     """Roofline of the kernel with the largest share of device time.  `achieved` is the
     kernel's algorithmic work per launch over its measured launch time: the FLOPs of its
     products per token and value head (the method's steps, full 64-row tiles) times the
@@ -478,19 +509,22 @@ def kernel_roofline(prof: dict, case, pk: dict) -> dict | None:
     count the chunk intermediates that pass between kernels, and the chunk kernels' inputs
     are mostly such intermediates, so their binding bound is the tensor peak.  The bytes the
     kernel moves under the current kernel split (intermediates included) are reported
-    beside it as `hbm_with_intermediates`."""
+    beside it as `hbm_with_intermediates`.  `prof` covers `steps` steps; a kernel launched
+    several times per step (one launch per segment of the chunks) does its step's work in
+    those launches together, so a launch's work is the step's divided by its launches."""
     if not prof:
         return None
     name, (launches, total_ms) = max(prof.items(), key=lambda kv: kv[1][1])
     per_launch_s = total_ms / launches / 1e3
+    per_step = launches / steps  # launches per step
     fl = kernel_flops_per_token_head(case.K, case.V).get(name)
-    th = case.tokens * case.HV
+    th = case.tokens * case.HV / per_step  # token-heads of one launch
     e = 2 if case.dtype == "bf16" else 4
-    units = chunks_of(case) * case.HV
+    units = chunks_of(case) * case.HV / per_step
     by = kernel_bytes_per_unit(case.K, case.V, case.HV // case.H, e).get(name)
     out = {"kernel": name, "launch_ms": round(per_launch_s * 1e3, 4),
            "share": round(total_ms / sum(v[1] for v in prof.values()), 4),
-           "units_per_launch": units}
+           "units_per_launch": round(units, 1), "launches_per_step": per_step}
     traffic = _traffic(name, case)
     if fl is not None and name.startswith("ffma_"):
         achieved = fl * th / per_launch_s / 1e12

@@ -19,8 +19,6 @@ namespace tcx {
 
 namespace {
 
-constexpr int kScanThreads = 512;
-
 // One 32-byte (256-bit) global store: a whole sector per thread.
 __device__ __forceinline__ void st_global_32B(void* p, const uint32_t* v) {
   asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]),
@@ -29,17 +27,24 @@ __device__ __forceinline__ void st_global_32B(void* p, const uint32_t* v) {
 }
 
 // ======================================================================================
-// Forward.  Thread (warp w, lane l): TMEM lane quarter q = w & 3, row = 32q + l, column group
-// cg = w >> 2 (32 state columns).  Thread 0 issues the MMAs, thread 96 the loads; every thread
-// writes its part of h (the bf16 state entering each chunk) with plain stores.  -N^T comes ready from the WY kernel, so per chunk c the tensor pipe runs
+// Forward.  Warps 0..15 hold the state: warp w, lane l has TMEM lane quarter q = w & 3,
+// row = 32q + l, column group cg = w >> 2 (32 state columns).  Warp 16 is the control warp:
+// its lane 0 issues every MMA and every load, so that a thread blocked in issuing tensor-core
+// instructions (they are accepted at roughly the rate the pipe executes them) never delays the
+// state update.  -N^T comes ready from the WY kernel, so per chunk c the tensor pipe runs
 //   chain(c)  ACC[c&1] += (-N_c^T) S_c^T       M=128 k', N=128 v, K=128 k   (8 instr)
 //   B(c+1)    ACC[~]    = (D K)^T U~           M=128 k', N=128 v, K=64 i    (4)
-// and the step's critical path is the chain product, the state update and one barrier.
-// (v_new = U~ - W S^T is left to the output kernel, which reads S anyway: on the sequential
-// pass every tensor-core instruction counts, at roughly 60-130 cycles each.)
+// State warps: wait for chain(c), update S, write its bf16 copy (the next chain operand, and h)
+// and sync on named barrier 1 with the control warp, which then issues the next chain product.
+// Every thread of the CTA takes part in every round of that barrier (a blocking sync, also on
+// the error path), so no warp can reach a round early.
+// (v_new = U~ - W S^T is left to the output kernel, which reads S anyway.)
 // Shared memory: three input stages {U~^T [128][64], -N^T [128][128], D K [64][128]} with
 // e^{G_i}, and S^T bf16 [128 k][128 v] (MN-major B of the chain).
 // ======================================================================================
+constexpr int kStateThreads = 512;
+constexpr int kScanThreadsWS = kStateThreads + 32;
+
 struct Fwd2Smem {
   static constexpr int UT = 0, NT = TILE128, DK = 3 * TILE128;   // within a stage
   static constexpr int STAGE = 4 * TILE128;
@@ -49,7 +54,7 @@ struct Fwd2Smem {
 };
 static_assert(1024 + Fwd2Smem::TOTAL + 256 <= 227 * 1024, "forward pass shared memory");
 
-__global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
+__global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_fwd2(
     Problem p, Args a, Work w, TcWork t, const __grid_constant__ CUtensorMap mDK,
     const __grid_constant__ CUtensorMap mNT, const __grid_constant__ CUtensorMap mUtT, ScanRange sr) {
   // one read of the status word decides for the whole CTA (barriers below need every thread)
@@ -64,7 +69,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
   const int cb = min(max(sr.c0, 0), sq0.y), nc = max(min(sr.c1, sq0.y) - cb, 0);
   const int4 sq = make_int4(sq0.x + cb, nc, sq0.z + 64 * cb, sq0.w - 64 * cb);
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int qd = warp & 3, cg = warp >> 2, row = 32 * qd + lane;
+  const bool ctl = warp == kStateThreads / 32;
+  const int qd = warp & 3, cg = (warp >> 2) & 3, row = 32 * qd + lane;
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
   unsigned char* sS = sm + Fwd2Smem::S;
@@ -72,6 +78,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
   auto vecp = [&](int c) { return reinterpret_cast<float*>(sm + Fwd2Smem::VEC + (c % 3) * 512); };
   __shared__ uint64_t barL[3], barC, barE;
   __shared__ uint32_t tslot;
+  __shared__ volatile int s_abort;
   int* err = w.status;
   // the test flag withholds the first chain product; its wait then runs out quickly
   const long long wait_limit = p.test_timeout ? (1ll << 20) : (1ll << 31);
@@ -79,6 +86,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
     for (int i = 0; i < 3; ++i) mbar_init(&barL[i], 1);
     mbar_init(&barC, 1);
     mbar_init(&barE, 1);
+    s_abort = 0;
     mbar_fence_init();
   }
   __syncthreads();
@@ -87,7 +95,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
     tmem_relinquish();
   }
   auto unit_row = [&](int c) { return ((sq.x + c) * p.HV + hv) * D; };
-  // thread 96: chunk c's tiles (U~^T, -N^T and D K, written by the WY kernel) and its e^{G_i}
+  // control lane: chunk c's tiles (U~^T, -N^T and D K, written by the WY kernel) and e^{G_i}
+  int loaded = 0;  // chunks whose loads were issued, in order 0, 1, 2, ... (control lane)
   auto issue_load = [&](int c) {
     unsigned char* b = stage(c);
     uint64_t* bar = &barL[c % 3];
@@ -100,17 +109,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
     tma_load_3d(b + Fwd2Smem::DK, &mDK, 0, r / 2, 0, bar);
     tma_load_3d(b + Fwd2Smem::DK + TILE64, &mDK, 64, r / 2, 0, bar);
     bulk_load(vecp(c) + 64, w.EG + o, 256, bar);
+    ++loaded;
   };
   // chunk c is the (c/3)-th load into stage c%3: its barrier phase has parity (c/3)&1
   auto load_par = [](int c) { return (uint32_t)((c / 3) & 1); };
-  int loaded = min(3, nc);  // chunks whose loads were issued (the same count in every thread)
-  int confirmed = 0;        // chunks whose loads every thread saw complete
-  if (tid == 96)
-    for (int c = 0; c < loaded; ++c) issue_load(c);
+  const bool issuer = tid == kStateThreads;
+  if (issuer)
+    for (int c = 0; c < min(3, nc); ++c) issue_load(c);
   // this thread's part of S^T: row `row`, columns 32 cg .. 32 cg + 31
   float S[32];
   // states are [Nst][HV][K][V]; rows k >= K and columns v >= V of a narrower head are padding
-  const bool st_live = row < p.K && 32 * cg < p.V;
+  const bool st_live = !ctl && row < p.K && 32 * cg < p.V;
   const size_t st_off = (((size_t)n * p.HV + hv) * p.K + row) * p.V + 32 * cg;
 #pragma unroll
   for (int v = 0; v < 32; v += 4) {
@@ -131,86 +140,87 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
     st_global_32B(g, pk);
     st_global_32B(g + 16, pk + 8);
   };
-  if (nc > 0) put_state(0);
-  fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
   const uint32_t tACC0 = taddr(tb, 0, 0);
-  // B(c) = (D K)^T U~ into ACC[c&1] (K of chunk c already scaled by D)
-  auto issue_b = [&](int c) {
-    unsigned char* b = stage(c);
-    const uint64_t dk = desc_mnmajor(smem_u32(b + Fwd2Smem::DK), 0, TILE64);
-    const uint64_t du = desc_kmajor(smem_u32(b + Fwd2Smem::UT), 0, TILE128);
-    const uint32_t tacc = tACC0 + (uint32_t)(128 * (c & 1));
-#pragma unroll
-    for (int s = 0; s < 4; ++s)
-      mma_bf16(tacc, dk + mnstep_off(s), du + kstep_off(s, TILE128), idesc_bf16(128, 128, true, false), s > 0);
-  };
-  bool ok = true;
-  // prologue: the first two chunks' tiles, B(0)
-  if (nc > 0) {
-    bool okp = true;
-    for (int c = 0; c < min(2, nc); ++c) okp = okp && mbar_wait(&barL[c], load_par(c), err);
-    tc_fence_before();
-    ok = __syncthreads_and(okp);
-    tc_fence_after();
-    if (ok) confirmed = min(2, nc);
-    if (ok && tid == 0) issue_b(0);
-  }
-  for (int c = 0; ok && c < nc; ++c) {
-    const bool more = c + 1 < nc;
-    const float egc = vecp(c)[64 + 63];
-    // (1) the chain product, then the next chunk's state-free product behind it
-    if (tid == 0) {
-      const uint64_t da = desc_kmajor(smem_u32(stage(c) + Fwd2Smem::NT), 0, TILE128);
-      const uint64_t dsB = desc_mnmajor(smem_u32(sS), 0, TILE128);
+  if (ctl) {
+    // B(c) = (D K)^T U~ into ACC[c&1] (K of chunk c already scaled by D)
+    auto issue_b = [&](int c) {
+      unsigned char* b = stage(c);
+      const uint64_t dk = desc_mnmajor(smem_u32(b + Fwd2Smem::DK), 0, TILE64);
+      const uint64_t du = desc_kmajor(smem_u32(b + Fwd2Smem::UT), 0, TILE128);
       const uint32_t tacc = tACC0 + (uint32_t)(128 * (c & 1));
-      if (!(p.test_timeout && c == 0)) {  // the test flag withholds the first chain product
 #pragma unroll
-        for (int s = 0; s < 8; ++s)  // chain: ACC += (-N^T) S^T
-          mma_bf16(tacc, da + kstep_off(s, TILE128), dsB + mnstep_off(s), idesc_bf16(128, 128, false, true), 1);
-        mma_commit(&barC);
+      for (int s = 0; s < 4; ++s)
+        mma_bf16(tacc, dk + mnstep_off(s), du + kstep_off(s, TILE128), idesc_bf16(128, 128, true, false), s > 0);
+    };
+    if (issuer && nc > 0 && mbar_wait_abort(&barL[0], load_par(0), err, &s_abort)) issue_b(0);
+    for (int c = 0; c < nc; ++c) {
+      nbar_sync(1, kScanThreadsWS);  // S_c^T is in shared memory (the whole warp syncs)
+      if (issuer && !s_abort) {
+        tc_fence_after();
+        if (!(p.test_timeout && c == 0)) {  // the test flag withholds the first chain product
+          const uint64_t da = desc_kmajor(smem_u32(stage(c) + Fwd2Smem::NT), 0, TILE128);
+          const uint64_t dsB = desc_mnmajor(smem_u32(sS), 0, TILE128);
+          const uint32_t tacc = tACC0 + (uint32_t)(128 * (c & 1));
+#pragma unroll
+          for (int s = 0; s < 8; ++s)  // chain: ACC += (-N^T) S^T
+            mma_bf16(tacc, da + kstep_off(s, TILE128), dsB + mnstep_off(s), idesc_bf16(128, 128, false, true), 1);
+          mma_commit(&barC);
+        }
+        if (c + 1 < nc && mbar_wait_abort(&barL[(c + 1) % 3], load_par(c + 1), err, &s_abort)) issue_b(c + 1);
+        // stage c%3 (read by B(c) and chain(c)) refills with chunk c+3
+        if (c + 3 < nc && mbar_wait_abort(&barC, c & 1, err, &s_abort)) issue_load(c + 3);
       }
-      if (more) issue_b(c + 1);
     }
-    // (2) S_{c+1}^T = e^{G_C} S_c^T + ACC
-    bool okt = mbar_wait_for(&barC, c & 1, err, wait_limit);
-    tc_fence_after();
-    if (okt) {
-      float x[32];
-      tmem_ld16(taddr(tb, 32 * qd, 128 * (c & 1) + 32 * cg), x);
-      tmem_ld16(taddr(tb, 32 * qd, 128 * (c & 1) + 32 * cg + 16), x + 16);
-      tmem_wait_ld();
-#pragma unroll
-      for (int q = 0; q < 32; ++q) S[q] = egc * S[q] + x[q];
-    }
-    // (3) the tiles of the chunk two ahead have landed; the next state operand and h[c+1]
-    if (c + 2 < nc) okt = okt && mbar_wait(&barL[(c + 2) % 3], load_par(c + 2), err);
-    if (more && okt) put_state(c + 1);
+  } else if (nc > 0) {
+    // state warps: e^{G_C} of the next chunk is read before the barrier round (its stage is
+    // refilled only after the chain product that round releases)
+    float egc = 0.f;
+    if (mbar_wait_abort(&barL[0], load_par(0), err, &s_abort)) egc = vecp(0)[64 + 63];
+    put_state(0);
     fence_proxy_async();
     tc_fence_before();
-    ok = __syncthreads_and(ok && okt);
-    tc_fence_after();
-    if (!ok) break;
-    confirmed = min(c + 3, nc);
-    // (4) stage c%3 (chain(c) and B(c) have read it) refills with chunk c+3
-    if (loaded < nc) {
-      if (tid == 96) issue_load(loaded);
-      ++loaded;
+    nbar_sync(1, kScanThreadsWS);
+    for (int c = 0; c < nc; ++c) {
+      // S_{c+1}^T = e^{G_C} S_c^T + ACC
+      bool okt = !s_abort && mbar_wait_abort(&barC, c & 1, err, &s_abort, wait_limit);
+      tc_fence_after();
+      if (okt) {
+        float x[32];
+        tmem_ld16(taddr(tb, 32 * qd, 128 * (c & 1) + 32 * cg), x);
+        tmem_ld16(taddr(tb, 32 * qd, 128 * (c & 1) + 32 * cg + 16), x + 16);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 32; ++q) S[q] = egc * S[q] + x[q];
+      }
+      if (c + 1 < nc) {
+        okt = okt && mbar_wait_abort(&barL[(c + 1) % 3], load_par(c + 1), err, &s_abort);
+        if (okt) {
+          egc = vecp(c + 1)[64 + 63];
+          put_state(c + 1);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        nbar_sync(1, kScanThreadsWS);
+      }
     }
   }
+  tc_fence_before();
+  __syncthreads();
+  const bool ok = !s_abort;
   if (ok && sr.s_out && st_live) {  // the final state, or the state handed to the next launch
 #pragma unroll
     for (int v = 0; v < 32; v += 4)
       *reinterpret_cast<float4*>(sr.s_out + st_off + v) = make_float4(S[v], S[v + 1], S[v + 2], S[v + 3]);
   }
-  // on an error exit, let the loads that were issued land and the MMAs finish before the
-  // CTA frees its tensor memory and leaves
-  if (!ok && tid == 96)
-    for (int c = confirmed; c < loaded; ++c) mbar_wait(&barL[c % 3], load_par(c), nullptr);
-  if (tid == 0) {
+  // before the CTA leaves (after an error too): the last load into each stage has landed, so
+  // every earlier one has; every MMA issued has finished
+  if (issuer) {
+    for (int b = 0; b < 3; ++b)  // stage b's last load was its ((loaded - 1 - b) / 3)-th
+      if (loaded > b) mbar_wait(&barL[b], (uint32_t)(((loaded - 1 - b) / 3) & 1), nullptr);
     mma_commit(&barE);
     mbar_wait(&barE, 0, nullptr);
   }
@@ -225,7 +235,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_fwd2(
 //   dS_c^T = e^{G_C} dS'^T - ACC,   ACC = W^T dU_loc + Q^T O' + N dS'^T,  O' = -scale e^G dO
 //   dU_c^T = dU_loc^T + dS' K^T D                      (written out as a bf16 hi/lo pair)
 // -N^T comes ready from the WY kernel (read here as an MN-major A operand with the negate bit
-// set), O' from dv_local.  Per chunk, in tensor-pipe order:
+// set), O' from dv_local.  Roles as in the forward pass: warps 0..15 hold dS', warp 16's lane 0
+// issues every MMA and load.  Per chunk, in tensor-pipe order:
 //   chain(c)  ACC[c&1] += N (dS'^T hi + lo)       M=128 k, N=128 v, K=128 k''  (16 instr)
 //   dU(c)     DU[c&1]  += dS' (D K)^T, hi + lo    M=128 v, N=64 i,  K=128 k    (16)
 //   I(c-1)    DU[~]     = dU_loc^T I              M=128 v, N=64 i,  K=64 i'    (4)
@@ -251,7 +262,7 @@ struct Bwd2Smem {
 };
 static_assert(1024 + Bwd2Smem::TOTAL + 256 <= 227 * 1024, "backward pass shared memory");
 
-__global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
+__global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_bwd2(
     Problem p, Args a, Work w, TcWork t, const __grid_constant__ CUtensorMap mq,
     const __grid_constant__ CUtensorMap mDK, const __grid_constant__ CUtensorMap mOp,
     const __grid_constant__ CUtensorMap mWT, const __grid_constant__ CUtensorMap mdUlT,
@@ -265,7 +276,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
   const int cb = min(max(sr.c0, 0), sq0.y), nc = max(min(sr.c1, sq0.y) - cb, 0);
   const int4 sq = make_int4(sq0.x + cb, nc, sq0.z + 64 * cb, sq0.w - 64 * cb);
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int qd = warp & 3, cg = warp >> 2, row = 32 * qd + lane;
+  const bool ctl = warp == kStateThreads / 32, issuer = tid == kStateThreads;
+  const int qd = warp & 3, cg = (warp >> 2) & 3, row = 32 * qd + lane;
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
   unsigned char* sDKt = sm + Bwd2Smem::DK;
@@ -280,6 +292,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
   auto vecp = [&](int c) { return reinterpret_cast<float*>(sm + Bwd2Smem::VEC + (c & 1) * 256); };
   __shared__ uint64_t barN[2], barDK, barQ, barF, barC, barDU, barE;
   __shared__ uint32_t tslot;
+  __shared__ volatile int s_abort;
   int* err = w.status;
   if (tid == 0) {
     mbar_init(&barN[0], 1);
@@ -290,6 +303,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
     mbar_init(&barC, 1);
     mbar_init(&barDU, 1);
     mbar_init(&barE, 1);
+    s_abort = 0;
     mbar_fence_init();
   }
   __syncthreads();
@@ -304,11 +318,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
   // completes its j-th phase for chunk nc-1-2j-((nc-1-c)&1).
   auto par = [&](int c) { return (uint32_t)((nc - 1 - c) & 1); };
   auto npar = [&](int c) { return (uint32_t)(((nc - 1 - c) >> 1) & 1); };
-  // loads issued per barrier, counted by the issuing thread: on an error exit it waits for the
-  // last one of each (phases complete in order, so the others have landed too)
+  // loads issued per barrier (control lane): on the way out it waits for the last one of each
   int n_iss0 = 0, n_iss1 = 0, dk_iss = 0, q_iss = 0;
-  // thread 32: chunk c's -N^T and e^{G_i}; its D K
-  auto issue_n = [&](int c) {
+  auto issue_n = [&](int c) {  // chunk c's -N^T and e^{G_i}
     uint64_t* bar = &barN[c & 1];
     const size_t o = ((size_t)hv * p.NCmax + sq.x + c) * 64;
     mbar_expect_tx(bar, 2 * TILE128 + 256);
@@ -323,7 +335,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
     tma_load_3d(sDKt + TILE64, &mDK, 64, unit_row(c) / 2, 0, &barDK);
     ++dk_iss;
   };
-  // thread 96: chunk c's Q, O' = -scale e^G dO (the dv_local kernel's), W^T and dU_loc^T
+  // chunk c's Q, O' = -scale e^G dO (the dv_local kernel's), W^T and dU_loc^T
   auto issue_q = [&](int c) {
     mbar_expect_tx(&barQ, 4 * TILE128);
     tma_load_3d(sQ, &mq, 0, hk, tok_of(c), &barQ);
@@ -334,17 +346,15 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
     tma_load_3d(sUl, &mdUlT, 0, unit_row(c), 0, &barQ);
     ++q_iss;
   };
-  if (nc > 0) {
-    if (tid == 32) {
-      issue_n(nc - 1);
-      issue_dk(nc - 1);
-    }
-    if (tid == 96) issue_q(nc - 1);
+  if (issuer && nc > 0) {
+    issue_n(nc - 1);
+    issue_dk(nc - 1);
+    issue_q(nc - 1);
   }
   // this thread's part of dS'^T: row `row`, columns 32 cg .. 32 cg + 31
   float S[32];
   // states are [Nst][HV][K][V]; rows k >= K and columns v >= V of a narrower head are padding
-  const bool st_live = row < p.K && 32 * cg < p.V;
+  const bool st_live = !ctl && row < p.K && 32 * cg < p.V;
   const size_t st_off = (((size_t)n * p.HV + hv) * p.K + row) * p.V + 32 * cg;
 #pragma unroll
   for (int v = 0; v < 32; v += 4) {
@@ -352,7 +362,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
                                           : make_float4(0, 0, 0, 0);
     S[v] = x.x; S[v + 1] = x.y; S[v + 2] = x.z; S[v + 3] = x.w;
   }
-  {  // the 64 x 64 identity (bf16), one 16-byte chunk per thread
+  if (!ctl) {  // the 64 x 64 identity (bf16), one 16-byte chunk per state thread
     const int r = tid >> 3, j = tid & 7;
     float f[8];
 #pragma unroll
@@ -380,62 +390,62 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
     st_global_32B(g, ph);
     st_global_32B(g + 16, ph + 8);
   };
-  if (nc > 0) put_state(nc - 1);
-  fence_proxy_async();
+  fence_proxy_async();  // the identity, before any product reads it
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tslot;
   auto tACC = [&](int c) { return taddr(tb, 0, 128 * (c & 1)); };
   auto tDU = [&](int c) { return taddr(tb, 0, 256 + 64 * (c & 1)); };
-  // I(c) and F(c): the state-free products of chunk c (thread 0)
-  auto issue_if = [&](int c) {
-    const uint64_t dul = desc_kmajor(smem_u32(sUl), 0, TILE128);
-    const uint64_t di = desc_kmajor(smem_u32(sI), 0, TILE64);
-    const uint64_t dwA = desc_kmajor(smem_u32(sW), 0, TILE128);
-    const uint64_t dq = desc_mnmajor(smem_u32(sQ), 0, TILE64);
-    const uint64_t dO_ = desc_mnmajor(smem_u32(sO), 0, TILE64);
+  if (ctl) {
+    // I(c) and F(c): the state-free products of chunk c
+    auto issue_if = [&](int c) {
+      const uint64_t dul = desc_kmajor(smem_u32(sUl), 0, TILE128);
+      const uint64_t di = desc_kmajor(smem_u32(sI), 0, TILE64);
+      const uint64_t dwA = desc_kmajor(smem_u32(sW), 0, TILE128);
+      const uint64_t dq = desc_mnmajor(smem_u32(sQ), 0, TILE64);
+      const uint64_t dO_ = desc_mnmajor(smem_u32(sO), 0, TILE64);
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      mma_bf16(tDU(c), dul + kstep_off(s, TILE128), di + kstep_off(s, TILE64), idesc_bf16(128, 64, false, false), s > 0);
-      mma_bf16(tACC(c), dwA + kstep_off(s, TILE128), dul + kstep_off(s, TILE128),
-               idesc_bf16(128, 128, false, false), s > 0);
-    }
+      for (int s = 0; s < 4; ++s) {
+        mma_bf16(tDU(c), dul + kstep_off(s, TILE128), di + kstep_off(s, TILE64), idesc_bf16(128, 64, false, false), s > 0);
+        mma_bf16(tACC(c), dwA + kstep_off(s, TILE128), dul + kstep_off(s, TILE128),
+                 idesc_bf16(128, 128, false, false), s > 0);
+      }
 #pragma unroll
-    for (int s = 0; s < 4; ++s)
-      mma_bf16(tACC(c), dq + mnstep_off(s), dO_ + mnstep_off(s), idesc_bf16(128, 128, true, true), 1);
-    mma_commit(&barF);
-  };
-  bool ok = true;
-  if (nc > 0) {  // the last chunk's Q, O', W, dU_loc, then its state-free products
-    const bool okp = mbar_wait(&barQ, par(nc - 1), err);
-    tc_fence_before();
-    ok = __syncthreads_and(okp);
-    tc_fence_after();
-    if (ok && tid == 0) issue_if(nc - 1);
-  }
-  // the chain's A operand: -N^T read MN-major is -N; the negate bit makes it N
-  constexpr uint32_t kNegA = 1u << 13;
-  for (int idx = 0; ok && idx < nc; ++idx) {
-    const int c = nc - 1 - idx;
-    const bool more = c > 0;
-    // (1) chunk c's -N^T; the chain product, then dU(c) once D K has landed
-    bool okt = mbar_wait(&barN[c & 1], npar(c), err);
-    tc_fence_after();
-    const float egc = vecp(c)[63];
-    if (tid == 0 && okt) {
-      const uint64_t dn = desc_mnmajor(smem_u32(sN(c)), 0, TILE128);
+      for (int s = 0; s < 4; ++s)
+        mma_bf16(tACC(c), dq + mnstep_off(s), dO_ + mnstep_off(s), idesc_bf16(128, 128, true, true), 1);
+      mma_commit(&barF);
+    };
+    if (issuer && nc > 0 && mbar_wait_abort(&barQ, par(nc - 1), err, &s_abort)) issue_if(nc - 1);
+    // the chain's A operand: -N^T read MN-major is -N; the negate bit makes it N
+    constexpr uint32_t kNegA = 1u << 13;
+    for (int idx = 0; idx < nc; ++idx) {
+      const int c = nc - 1 - idx;
+      nbar_sync(1, kScanThreadsWS);  // dS'_c^T is in shared memory (the whole warp syncs)
+      if (!issuer || s_abort) continue;
+      tc_fence_after();
       const uint64_t dah = desc_mnmajor(smem_u32(sDH), 0, TILE128);
       const uint64_t dal = desc_mnmajor(smem_u32(sDL), 0, TILE128);
-      constexpr uint32_t idC = idesc_bf16(128, 128, true, true) | kNegA;
+      // the -N^T slot of chunk c+1 (its chain product finished before the state warps released
+      // dS'_c) takes chunk c-1's
+      if (c > 0) issue_n(c - 1);
+      if (!mbar_wait_abort(&barN[c & 1], npar(c), err, &s_abort)) continue;
+      {
+        const uint64_t dn = desc_mnmajor(smem_u32(sN(c)), 0, TILE128);
+        constexpr uint32_t idC = idesc_bf16(128, 128, true, true) | kNegA;
 #pragma unroll
-      for (int s = 0; s < 8; ++s) mma_bf16(tACC(c), dn + mnstep_off(s), dah + mnstep_off(s), idC, 1);
+        for (int s = 0; s < 8; ++s) mma_bf16(tACC(c), dn + mnstep_off(s), dah + mnstep_off(s), idC, 1);
 #pragma unroll
-      for (int s = 0; s < 8; ++s) mma_bf16(tACC(c), dn + mnstep_off(s), dal + mnstep_off(s), idC, 1);
-      mma_commit(&barC);
-      okt = mbar_wait(&barDK, par(c), err);
-      tc_fence_after();
-      if (okt) {
+        for (int s = 0; s < 8; ++s) mma_bf16(tACC(c), dn + mnstep_off(s), dal + mnstep_off(s), idC, 1);
+        mma_commit(&barC);
+      }
+      // chunk c's F and I have run: chunk c-1's Q, O', W, dU_loc replace theirs
+      if (c > 0) {
+        if (!mbar_wait_abort(&barF, par(c), err, &s_abort)) continue;
+        issue_q(c - 1);
+      }
+      if (!mbar_wait_abort(&barDK, par(c), err, &s_abort)) continue;
+      {
         const uint64_t dkK = desc_kmajor(smem_u32(sDKt), 0, TILE64);
         constexpr uint32_t idU = idesc_bf16(128, 64, true, false);
 #pragma unroll
@@ -444,70 +454,83 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
         for (int s = 0; s < 8; ++s) mma_bf16(tDU(c), dal + mnstep_off(s), dkK + kstep_off(s, TILE64), idU, 1);
         mma_commit(&barDU);
       }
+      if (c == 0) continue;
+      // the previous chunk's state-free products go in behind this chunk's; D K is replaced
+      // once dU(c) has read it
+      if (!mbar_wait_abort(&barQ, par(c - 1), err, &s_abort)) continue;
+      issue_if(c - 1);
+      if (mbar_wait_abort(&barDU, par(c), err, &s_abort)) issue_dk(c - 1);
     }
-    // the slot of chunk c+1's -N^T (its chain product finished) takes chunk c-1's
-    if (tid == 32 && more) issue_n(c - 1);
-    // chunk c's F and I have run: the next chunk's Q, O', W, dU_loc replace theirs
-    if (tid == 96 && more && mbar_wait(&barF, par(c), err)) issue_q(c - 1);
-    // (2) dS_c^T = e^{G_C} dS'^T - ACC
-    okt = okt && mbar_wait(&barC, par(c), err);
-    tc_fence_after();
-    if (okt) {
-      float x[32];
-      tmem_ld16(taddr(tb, 32 * qd, 128 * (c & 1) + 32 * cg), x);
-      tmem_ld16(taddr(tb, 32 * qd, 128 * (c & 1) + 32 * cg + 16), x + 16);
-      tmem_wait_ld();
-#pragma unroll
-      for (int q = 0; q < 32; ++q) S[q] = egc * S[q] - x[q];
-    }
-    // the previous chunk's state-free products go in behind this chunk's
-    if (tid == 0 && more && okt) {
-      okt = mbar_wait(&barQ, par(c - 1), err);
-      tc_fence_after();
-      if (okt) issue_if(c - 1);
-    }
-    // (3) dU^T = DU as a hi/lo pair (rows v, 16 columns per thread), straight to the workspace
-    okt = okt && mbar_wait(&barDU, par(c), err);
-    tc_fence_after();
-    if (okt) {
-      if (tid == 32 && more) issue_dk(c - 1);  // dU(c) has read D K
-      float x[16];
-      tmem_ld16(taddr(tb, 32 * qd, 256 + 64 * (c & 1) + 16 * cg), x);
-      tmem_wait_ld();
-      bf16* hrow = t.dUT + ((size_t)unit_row(c) + row) * 64 + 16 * cg;
-      bf16* lrow = t.dUTl + ((size_t)unit_row(c) + row) * 64 + 16 * cg;
-      uint32_t ph[8], pl[8];
-#pragma unroll
-      for (int q = 0; q < 16; q += 2) {
-        const float h0 = __bfloat162float(__float2bfloat16_rn(x[q]));
-        const float h1 = __bfloat162float(__float2bfloat16_rn(x[q + 1]));
-        ph[q / 2] = pack_bf16(h0, h1);
-        pl[q / 2] = pack_bf16(x[q] - h0, x[q + 1] - h1);
-      }
-      st_global_32B(hrow, ph);  // 16 columns = one full 32-byte sector per row and part
-      st_global_32B(lrow, pl);
-      // (4) both products of chunk c have read dS'^T: the next one (and dh[c-1]) replaces it
-      if (more) put_state(c - 1);
-    }
+  } else if (nc > 0) {
+    // state warps: e^{G_C} of a chunk is read before the barrier round that releases its chain
+    // product (its -N^T slot is refilled only after that product)
+    float egc = 0.f;
+    if (mbar_wait_abort(&barN[(nc - 1) & 1], npar(nc - 1), err, &s_abort)) egc = vecp(nc - 1)[63];
+    put_state(nc - 1);
     fence_proxy_async();
     tc_fence_before();
-    ok = __syncthreads_and(ok && okt);
-    tc_fence_after();
+    nbar_sync(1, kScanThreadsWS);
+    for (int idx = 0; idx < nc; ++idx) {
+      const int c = nc - 1 - idx;
+      const bool more = c > 0;
+      // (1) dS_c^T = e^{G_C} dS'^T - ACC
+      bool okt = !s_abort && mbar_wait_abort(&barC, par(c), err, &s_abort);
+      tc_fence_after();
+      if (okt) {
+        float x[32];
+        tmem_ld16(taddr(tb, 32 * qd, 128 * (c & 1) + 32 * cg), x);
+        tmem_ld16(taddr(tb, 32 * qd, 128 * (c & 1) + 32 * cg + 16), x + 16);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 32; ++q) S[q] = egc * S[q] - x[q];
+      }
+      // (2) dU^T = DU as a hi/lo pair (rows v, 16 columns per thread), straight to the workspace
+      okt = okt && mbar_wait_abort(&barDU, par(c), err, &s_abort);
+      tc_fence_after();
+      if (okt) {
+        float x[16];
+        tmem_ld16(taddr(tb, 32 * qd, 256 + 64 * (c & 1) + 16 * cg), x);
+        tmem_wait_ld();
+        bf16* hrow = t.dUT + ((size_t)unit_row(c) + row) * 64 + 16 * cg;
+        bf16* lrow = t.dUTl + ((size_t)unit_row(c) + row) * 64 + 16 * cg;
+        uint32_t ph[8], pl[8];
+#pragma unroll
+        for (int q = 0; q < 16; q += 2) {
+          const float h0 = __bfloat162float(__float2bfloat16_rn(x[q]));
+          const float h1 = __bfloat162float(__float2bfloat16_rn(x[q + 1]));
+          ph[q / 2] = pack_bf16(h0, h1);
+          pl[q / 2] = pack_bf16(x[q] - h0, x[q + 1] - h1);
+        }
+        st_global_32B(hrow, ph);  // 16 columns = one full 32-byte sector per row and part
+        st_global_32B(lrow, pl);
+      }
+      if (more) {
+        // (3) both products of chunk c have read dS'^T: the next one (and dh[c-1]) replaces it
+        okt = okt && mbar_wait_abort(&barN[(c - 1) & 1], npar(c - 1), err, &s_abort);
+        if (okt) {
+          egc = vecp(c - 1)[63];
+          put_state(c - 1);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        nbar_sync(1, kScanThreadsWS);
+      }
+    }
   }
-  if (ok && sr.s_out && st_live) {  // dh0, or the gradient handed to the launch of earlier chunks
+  tc_fence_before();
+  __syncthreads();
+  if (!s_abort && sr.s_out && st_live) {  // dh0, or the gradient handed to the launch of earlier chunks
 #pragma unroll
     for (int v = 0; v < 32; v += 4)
       *reinterpret_cast<float4*>(sr.s_out + st_off + v) = make_float4(S[v], S[v + 1], S[v + 2], S[v + 3]);
   }
   // before the CTA leaves (after an error too): the last load on each barrier has landed, so
   // every earlier one has; every MMA issued has finished
-  if (tid == 32) {
+  if (issuer) {
     if (n_iss0 > 0) mbar_wait(&barN[0], (uint32_t)((n_iss0 - 1) & 1), nullptr);
     if (n_iss1 > 0) mbar_wait(&barN[1], (uint32_t)((n_iss1 - 1) & 1), nullptr);
     if (dk_iss > 0) mbar_wait(&barDK, (uint32_t)((dk_iss - 1) & 1), nullptr);
-  }
-  if (tid == 96 && q_iss > 0) mbar_wait(&barQ, (uint32_t)((q_iss - 1) & 1), nullptr);
-  if (tid == 0) {
+    if (q_iss > 0) mbar_wait(&barQ, (uint32_t)((q_iss - 1) & 1), nullptr);
     mma_commit(&barE);
     mbar_wait(&barE, 0, nullptr);
   }
@@ -521,14 +544,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_tc_scan_bwd2(
 cudaError_t tc_scan_fwd(const Problem& p, const Args& a, const Work& w, const TcWork& t,
                         const TcMaps& m, const ScanRange& sr, cudaStream_t s) {
   const dim3 grid(p.Nst, p.HV);
-  return tgo("tc_scan_fwd", k_tc_scan_fwd2, grid, kScanThreads, (size_t)1024 + Fwd2Smem::TOTAL, s, p, a,
+  return tgo("tc_scan_fwd", k_tc_scan_fwd2, grid, kScanThreadsWS, (size_t)1024 + Fwd2Smem::TOTAL, s, p, a,
              w, t, m.DK, m.NT, m.UtT, sr);
 }
 
 cudaError_t tc_scan_bwd(const Problem& p, const Args& a, const Work& w, const TcWork& t,
                         const TcMaps& m, const ScanRange& sr, cudaStream_t s) {
   const dim3 grid(p.Nst, p.HV);
-  return tgo("tc_scan_bwd", k_tc_scan_bwd2, grid, kScanThreads, (size_t)1024 + Bwd2Smem::TOTAL, s, p, a,
+  return tgo("tc_scan_bwd", k_tc_scan_bwd2, grid, kScanThreadsWS, (size_t)1024 + Bwd2Smem::TOTAL, s, p, a,
              w, t, m.q, m.DK, m.Op, m.WT, m.dUlT, m.NT, sr);
 }
 

@@ -79,13 +79,12 @@ __device__ __forceinline__ bool mbar_wait_abort(uint64_t* bar, uint32_t parity, 
   }
 }
 
-// Named CTA barriers (ids 1..15; 0 is __syncthreads): producers arrive without waiting, the
-// consumer warp waits until `count` threads (a multiple of 32) have arrived or synced.
-__device__ __forceinline__ void nbar_arrive(int id, int count) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
+// Named CTA barrier (ids 1..15; 0 is __syncthreads): waits until `count` threads (a multiple
+// of 32) have synced.  The non-aligned form, preceded by a warp reconvergence: every lane of a
+// participating warp takes part, whatever path it took before.
 __device__ __forceinline__ void nbar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+  __syncwarp();
+  asm volatile("barrier.cta.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ------------------------------------------------------------------ fences

@@ -40,13 +40,26 @@ def test_dominant_kernel_tensor_fraction_from_algorithmic_flops():
 
 def test_bytes_with_intermediates_reported_separately():
     case = _case()
-    r = bench.kernel_roofline({"tc_wy": (1, 0.5)}, case, PK)
+    r = bench.kernel_roofline({"tc_wy": (1, 0.5)}, case, PK, steps=1)
     units = (8192 // 64) * 32
     per_unit = bench.kernel_bytes_per_unit(128, 128, 2, 2)["tc_wy"]
     h = r["hbm_with_intermediates"]
     assert h["bytes_per_launch"] == int(per_unit * units)
     assert h["achieved"] == pytest.approx(per_unit * units / 0.5e-3 / 1e9, rel=1e-3)
     assert h["frac"] == pytest.approx(h["achieved"] / 6000.0, rel=1e-3)
+
+
+def test_segmented_launches_share_the_step():
+    """A kernel launched once per segment (8 per step, 2 steps profiled) does a step's work
+    in 8 launches: per launch an eighth of the units, achieved over the step's kernel time."""
+    case = _case()
+    r = bench.kernel_roofline({"tc_scan_bwd": (16, 2.4), "tc_wy": (16, 0.8)}, case, PK, steps=2)
+    units = (8192 // 64) * 32
+    assert r["kernel"] == "tc_scan_bwd" and r["launches_per_step"] == 8
+    assert r["units_per_launch"] == units / 8
+    fl = 6 * 128 * 128
+    assert r["achieved"] == pytest.approx(fl * 8192 * 32 / 1.2e-3 / 1e12, rel=1e-3)
+    assert r["launch_ms"] == pytest.approx(2.4 / 16, rel=1e-3)
 
 
 def test_no_profile_no_roofline():
