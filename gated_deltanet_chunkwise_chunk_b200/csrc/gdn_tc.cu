@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
   // KK^T: M=64, N=64, K=128 (both K-major) -> TMEM cols [0,64)
   if (ok && tid == 0) {
     const uint32_t k = smem_u32(sK);
+#pragma unroll
     for (int s = 0; s < 8; ++s)
       mma_bf16(taddr(tb, 0, 0), desc_kmajor(k, s, TILE64), desc_kmajor(k, s, TILE64),
                idesc_bf16(64, 64, false, false), s > 0);
@@ -169,12 +170,14 @@ __global__ void __launch_bounds__(256) k_tc_wy(Problem p, Work w, TcWork t,
   if (ok && tid == 0) {
     const uint32_t k = smem_u32(sK), vv = smem_u32(sV), tx = smem_u32(sTX), ty = smem_u32(sTY),
                    txl = smem_u32(sTXl), tyl = smem_u32(sTYl);
+#pragma unroll
     for (int s = 0; s < 4; ++s) {
       mma_bf16(taddr(tb, 0, 64), desc_mnmajor(k, s, TILE64), desc_kmajor(tx, s, TILE64),
                idesc_bf16(128, 64, true, false), s > 0);
       mma_bf16(taddr(tb, 0, 128), desc_mnmajor(vv, s, TILE64), desc_kmajor(ty, s, TILE64),
                idesc_bf16(128, 64, true, false), s > 0);
     }
+#pragma unroll
     for (int s = 0; s < 4; ++s) {
       mma_bf16(taddr(tb, 0, 64), desc_mnmajor(k, s, TILE64), desc_kmajor(txl, s, TILE64),
                idesc_bf16(128, 64, true, false), 1);
@@ -332,6 +335,7 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
   bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
   if (ok && tid == 0) {
     const uint32_t q = smem_u32(sQ), k = smem_u32(sK), h = smem_u32(sH), wt = smem_u32(sW);
+#pragma unroll
     for (int s = 0; s < 8; ++s) {
       // S is stored transposed ([k][v]): an MN-major B operand here, an MN-major A below
       mma_bf16(taddr(tb, 0, 0), desc_kmajor(q, s, TILE64), desc_mnmajor(h, s, TILE128),
@@ -388,9 +392,11 @@ __global__ void __launch_bounds__(256) k_tc_out(Problem p, Args a, Work w, TcWor
     tma_store_3d(&mUT, sU, 0, row, 0);  // v_new for the backward
     tma_store_commit();
     const uint32_t pp = smem_u32(sP), pl = smem_u32(sPl), u = smem_u32(sU);
+#pragma unroll
     for (int s = 0; s < 4; ++s)
       mma_bf16(taddr(tb, 0, 128), desc_kmajor(pp, s, TILE64), desc_kmajor(u, s, TILE128),
                idesc_bf16(64, 128, false, false), s > 0);
+#pragma unroll
     for (int s = 0; s < 4; ++s)
       mma_bf16(taddr(tb, 0, 128), desc_kmajor(pl, s, TILE64), desc_kmajor(u, s, TILE128),
                idesc_bf16(64, 128, false, false), 1);

@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
   bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
   if (ok && tid == 0) {
     const uint32_t q = smem_u32(sQ), k = smem_u32(sK);
+#pragma unroll
     for (int s = 0; s < 8; ++s)
       mma_bf16(taddr(tb, 0, 0), desc_kmajor(q, s, TILE64), desc_kmajor(k, s, TILE64),
                idesc_bf16(64, 64, false, false), s > 0);
@@ -113,9 +114,11 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
   tc_fence_after();
   if (ok && tid == 0) {
     const uint32_t o = smem_u32(sO), pp = smem_u32(sP), pl = smem_u32(sPl);
+#pragma unroll
     for (int s = 0; s < 4; ++s)
       mma_bf16(taddr(tb, 0, 64), desc_mnmajor(o, s, TILE64), desc_mnmajor(pp, s, TILE64),
                idesc_bf16(128, 64, true, true), s > 0);
+#pragma unroll
     for (int s = 0; s < 4; ++s)
       mma_bf16(taddr(tb, 0, 64), desc_mnmajor(o, s, TILE64), desc_mnmajor(pl, s, TILE64),
                idesc_bf16(128, 64, true, true), 1);
@@ -312,6 +315,7 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Args a, Work w, TcW
     if (tid == 0) {
       const uint32_t q = smem_u32(sQ), k = smem_u32(sK), o = smem_u32(sO), ut = smem_u32(sUT),
                      dut = smem_u32(sdUT), dutl = smem_u32(sdUTl), h = smem_u32(sH), dh = smem_u32(sdH);
+#pragma unroll
       for (int s = 0; s < 8; ++s) {
         const uint32_t acc = s > 0;
         mma_bf16(taddr(tb, 0, 0), desc_kmajor(q, s, TILE64), desc_kmajor(k, s, TILE64),
@@ -326,6 +330,7 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Args a, Work w, TcW
         mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dut, s, TILE128), desc_kmajor(h, s, TILE128),
                  idesc_bf16(64, 128, true, false), acc);
       }
+#pragma unroll
       for (int s = 0; s < 8; ++s)
         mma_bf16(taddr(tb, 0, 384), desc_mnmajor(dutl, s, TILE128), desc_kmajor(h, s, TILE128),
                  idesc_bf16(64, 128, true, false), 1);
@@ -439,8 +444,10 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Args a, Work w, TcW
       tma_store_3d(&mdW, sUT + TILE64, 64, (int)unit * 64, 0);
       tma_store_commit();
       const uint32_t k = smem_u32(sK), q = smem_u32(sQ);
+#pragma unroll
       for (int part = 0; part < 2; ++part) {
         const uint32_t pg = smem_u32(part ? sPGl : sPG);
+#pragma unroll
         for (int s = 0; s < 4; ++s) {
           mma_bf16(taddr(tb, 0, 128), desc_kmajor(pg, s, TILE64), desc_mnmajor(k, s, TILE64),
                    idesc_bf16(64, 128, false, true), 1);
@@ -696,6 +703,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aT = smem_u32(sT), aTl = smem_u32(sTl),
                    aW = smem_u32(sdW), aU = smem_u32(sdUT), aUl = smem_u32(sdUTl);
     if (tid == 0) {
+#pragma unroll
       for (int s = 0; s < 8; ++s) {
         const uint32_t acc = s > 0;
         mma_bf16(taddr(tb, 0, 0), desc_mnmajor(aU, s, TILE128), desc_kmajor(aV, s, TILE64),
@@ -707,8 +715,10 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
         mma_bf16(taddr(tb, 0, 128), desc_kmajor(aK, s, TILE64), desc_kmajor(aK, s, TILE64),
                  idesc_bf16(64, 64, false, false), acc);
       }
+#pragma unroll
       for (int part = 0; part < 2; ++part) {
         const uint32_t tt = part ? aTl : aT;
+#pragma unroll
         for (int s = 0; s < 4; ++s) {
           const uint32_t acc = part > 0 || s > 0;
           mma_bf16(taddr(tb, 0, 256), desc_mnmajor(tt, s, TILE64), desc_mnmajor(aW, s, TILE64),
@@ -795,7 +805,9 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     if (tid == 0) {
       const uint32_t dt = smem_u32(sdT), dtl = smem_u32(sdTl);
       const uint32_t pa[3] = {aT, aT, aTl}, pb[3] = {dt, dtl, dt};
+#pragma unroll
       for (int part = 0; part < 3; ++part)
+#pragma unroll
         for (int s = 0; s < 4; ++s)
           mma_bf16(taddr(tb, 0, 0), desc_mnmajor(pa[part], s, TILE64), desc_mnmajor(pb[part], s, TILE64),
                    idesc_bf16(64, 64, true, true), part > 0 || s > 0);
@@ -823,7 +835,9 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     if (tid == 0) {
       const uint32_t zz = smem_u32(sZ), zl = smem_u32(sZl);
       const uint32_t pa[3] = {zz, zz, zl}, pb[3] = {aT, aTl, aT};
+#pragma unroll
       for (int part = 0; part < 3; ++part)
+#pragma unroll
         for (int s = 0; s < 4; ++s)
           mma_bf16(taddr(tb, 0, 64), desc_kmajor(pa[part], s, TILE64), desc_kmajor(pb[part], s, TILE64),
                    idesc_bf16(64, 64, false, false), part > 0 || s > 0);
@@ -881,8 +895,10 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     tc_fence_after();
     // dk += dAs K + dAs^T K onto beta e^G dX
     if (tid == 0) {
+#pragma unroll
       for (int part = 0; part < 2; ++part) {
         const uint32_t as = smem_u32(part ? sAsl : sAs);
+#pragma unroll
         for (int s = 0; s < 4; ++s) {
           mma_bf16(taddr(tb, 0, 256), desc_kmajor(as, s, TILE64), desc_mnmajor(aK, s, TILE64),
                    idesc_bf16(64, 128, false, true), 1);

@@ -8,10 +8,11 @@
 //   backward   dS = e^{G_C} dS' + scale (e^G dO)^T Q - dU^T W,  dU = dU_loc + D K dS'^T
 //              = e^{G_C} dS' - (W^T dU_loc - scale Q^T e^G dO + N dS'^T)^T
 // N and B (and the backward's state-free terms) do not depend on the state, so they are built
-// off the chain; the chain itself is one tensor-core product per chunk (S N) instead of two
-// dependent ones (W S^T, then U^T D K).  Everything is kept transposed so that TMEM lane = key
-// index k: the state S^T [k][v] is held in fp32 registers, four threads per row k (512 threads,
-// 32 values each), and its bf16 copy that feeds the next product is written row by row.
+// off the chain (N by the WY kernel); the chain itself is one tensor-core product per chunk
+// (S N) instead of two dependent ones (W S^T, then U^T D K).  Everything is kept transposed so
+// that TMEM lane = key index k: the state S^T [k][v] is held in fp32 registers by 16 state
+// warps, four threads per row k (32 values each), and its bf16 copy that feeds the next product
+// is written row by row; a 17th warp issues the MMAs, the loads and the bulk stores.
 #include "gdn_tc_common.cuh"
 
 namespace gdn {
@@ -19,23 +20,17 @@ namespace tcx {
 
 namespace {
 
-// One 32-byte (256-bit) global store: a whole sector per thread.
-__device__ __forceinline__ void st_global_32B(void* p, const uint32_t* v) {
-  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]),
-               "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-               : "memory");
-}
-
 // ======================================================================================
 // Forward.  Warps 0..15 hold the state: warp w, lane l has TMEM lane quarter q = w & 3,
 // row = 32q + l, column group cg = w >> 2 (32 state columns).  Warp 16 is the control warp:
-// its lane 0 issues every MMA and every load, so that a thread blocked in issuing tensor-core
-// instructions (they are accepted at roughly the rate the pipe executes them) never delays the
-// state update.  -N^T comes ready from the WY kernel, so per chunk c the tensor pipe runs
+// its lane 0 issues every MMA, load and bulk store, so that a thread blocked in issuing
+// tensor-core instructions never delays the state update.  -N^T comes ready from the WY kernel, so per chunk c the tensor pipe runs
 //   chain(c)  ACC[c&1] += (-N_c^T) S_c^T       M=128 k', N=128 v, K=128 k   (8 instr)
 //   B(c+1)    ACC[~]    = (D K)^T U~           M=128 k', N=128 v, K=64 i    (4)
-// State warps: wait for chain(c), update S, write its bf16 copy (the next chain operand, and h)
-// and sync on named barrier 1 with the control warp, which then issues the next chain product.
+// State warps: wait for chain(c), update S, write its bf16 copy (the next chain operand) and sync
+// on named barrier 1 with the control warp, which then issues the next chain product and stores
+// the tile as h with a bulk copy (per-thread stores of rows 256 bytes apart cost more than the
+// whole chain product).
 // Every thread of the CTA takes part in every round of that barrier (a blocking sync, also on
 // the error path), so no warp can reach a round early.
 // (v_new = U~ - W S^T is left to the output kernel, which reads S anyway.)
@@ -56,7 +51,8 @@ static_assert(1024 + Fwd2Smem::TOTAL + 256 <= 227 * 1024, "forward pass shared m
 
 __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_fwd2(
     Problem p, Args a, Work w, TcWork t, const __grid_constant__ CUtensorMap mDK,
-    const __grid_constant__ CUtensorMap mNT, const __grid_constant__ CUtensorMap mUtT, ScanRange sr) {
+    const __grid_constant__ CUtensorMap mNT, const __grid_constant__ CUtensorMap mUtT,
+    const __grid_constant__ CUtensorMap mh, ScanRange sr) {
   // one read of the status word decides for the whole CTA (barriers below need every thread)
   __shared__ int s_fail;
   if (threadIdx.x == 0) s_fail = failed(w);
@@ -76,7 +72,8 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_fwd2(
   unsigned char* sS = sm + Fwd2Smem::S;
   auto stage = [&](int c) { return sm + (c % 3) * Fwd2Smem::STAGE; };
   auto vecp = [&](int c) { return reinterpret_cast<float*>(sm + Fwd2Smem::VEC + (c % 3) * 512); };
-  __shared__ uint64_t barL[3], barC, barE;
+  // barH: the bulk store of h[c] has read the S^T tile (the state warps may rewrite it)
+  __shared__ uint64_t barL[3], barC, barH, barE;
   __shared__ uint32_t tslot;
   __shared__ volatile int s_abort;
   int* err = w.status;
@@ -85,6 +82,7 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_fwd2(
   if (tid == 0) {
     for (int i = 0; i < 3; ++i) mbar_init(&barL[i], 1);
     mbar_init(&barC, 1);
+    mbar_init(&barH, 1);
     mbar_init(&barE, 1);
     s_abort = 0;
     mbar_fence_init();
@@ -127,18 +125,10 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_fwd2(
                                           : make_float4(0, 0, 0, 0);
     S[v] = x.x; S[v + 1] = x.y; S[v + 2] = x.z; S[v + 3] = x.w;
   }
-  // S^T entering chunk c (this thread's row part) as bf16: the chain operand tile and h[c]
-  auto put_state = [&](int c) {
-    uint32_t pk[16];
+  // S^T entering a chunk (this thread's row part) as bf16: the chain operand tile (stored as h)
+  auto put_state = [&]() {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(S[2 * i], S[2 * i + 1]);
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      *reinterpret_cast<uint4*>(sS + sw128_chunk(row, 4 * cg + j, TILE128)) =
-          make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-    bf16* g = t.h + ((size_t)unit_row(c) + row) * D + 32 * cg;
-    st_global_32B(g, pk);
-    st_global_32B(g + 16, pk + 8);
+    for (int j = 0; j < 4; ++j) st_chunk_f(sS, row, 4 * cg + j, TILE128, S + 8 * j);
   };
   tc_fence_before();
   __syncthreads();
@@ -161,6 +151,9 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_fwd2(
       nbar_sync(1, kScanThreadsWS);  // S_c^T is in shared memory (the whole warp syncs)
       if (issuer && !s_abort) {
         tc_fence_after();
+        tma_store_3d(&mh, sS, 0, unit_row(c), 0);  // h[c]
+        tma_store_3d(&mh, sS + TILE128, 64, unit_row(c), 0);
+        tma_store_commit();
         if (!(p.test_timeout && c == 0)) {  // the test flag withholds the first chain product
           const uint64_t da = desc_kmajor(smem_u32(stage(c) + Fwd2Smem::NT), 0, TILE128);
           const uint64_t dsB = desc_mnmajor(smem_u32(sS), 0, TILE128);
@@ -169,6 +162,10 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_fwd2(
           for (int s = 0; s < 8; ++s)  // chain: ACC += (-N^T) S^T
             mma_bf16(tacc, da + kstep_off(s, TILE128), dsB + mnstep_off(s), idesc_bf16(128, 128, false, true), 1);
           mma_commit(&barC);
+        }
+        if (c + 1 < nc) {  // the S^T tile is free once the store has read it
+          tma_store_wait_read0();
+          mbar_arrive(&barH);
         }
         if (c + 1 < nc && mbar_wait_abort(&barL[(c + 1) % 3], load_par(c + 1), err, &s_abort)) issue_b(c + 1);
         // stage c%3 (read by B(c) and chain(c)) refills with chunk c+3
@@ -180,7 +177,7 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_fwd2(
     // refilled only after the chain product that round releases)
     float egc = 0.f;
     if (mbar_wait_abort(&barL[0], load_par(0), err, &s_abort)) egc = vecp(0)[64 + 63];
-    put_state(0);
+    put_state();
     fence_proxy_async();
     tc_fence_before();
     nbar_sync(1, kScanThreadsWS);
@@ -198,10 +195,9 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_fwd2(
       }
       if (c + 1 < nc) {
         okt = okt && mbar_wait_abort(&barL[(c + 1) % 3], load_par(c + 1), err, &s_abort);
-        if (okt) {
-          egc = vecp(c + 1)[64 + 63];
-          put_state(c + 1);
-        }
+        if (okt) egc = vecp(c + 1)[64 + 63];
+        okt = okt && mbar_wait_abort(&barH, c & 1, err, &s_abort);
+        if (okt) put_state();
         fence_proxy_async();
         tc_fence_before();
         nbar_sync(1, kScanThreadsWS);
@@ -221,6 +217,7 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_fwd2(
   if (issuer) {
     for (int b = 0; b < 3; ++b)  // stage b's last load was its ((loaded - 1 - b) / 3)-th
       if (loaded > b) mbar_wait(&barL[b], (uint32_t)(((loaded - 1 - b) / 3) & 1), nullptr);
+    tma_store_wait0();
     mma_commit(&barE);
     mbar_wait(&barE, 0, nullptr);
   }
@@ -242,7 +239,9 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_fwd2(
 //   I(c-1)    DU[~]     = dU_loc^T I              M=128 v, N=64 i,  K=64 i'    (4)
 //   F(c-1)    ACC[~]    = W^T dU_loc + Q^T O'     M=128 k, N=128 v, K=64 i     (8)
 // The state-free products of the next chunk go in behind this chunk's, into the other
-// accumulators, so the pipe keeps working while the state is updated and written back.
+// accumulators, so the pipe keeps working while the state is updated and written back.  dh
+// (the hi tile of dS') and dU^T (staged by the state warps in the -N^T slot its chain product
+// has finished with) leave by bulk copies the control lane issues after the barrier.
 // Shared memory: two slots of -N^T [128][128] with e^{G_i}; one of D K [64][128]; one of
 // {Q [64][128], O' [64][128], W^T [128][64], dU_loc^T [128][64]}; dS'^T hi and lo [128][128];
 // the 64 x 64 identity.
@@ -266,7 +265,8 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_bwd2(
     Problem p, Args a, Work w, TcWork t, const __grid_constant__ CUtensorMap mq,
     const __grid_constant__ CUtensorMap mDK, const __grid_constant__ CUtensorMap mOp,
     const __grid_constant__ CUtensorMap mWT, const __grid_constant__ CUtensorMap mdUlT,
-    const __grid_constant__ CUtensorMap mNT, ScanRange sr) {
+    const __grid_constant__ CUtensorMap mNT, const __grid_constant__ CUtensorMap mdh,
+    const __grid_constant__ CUtensorMap mdUT, const __grid_constant__ CUtensorMap mdUTl, ScanRange sr) {
   __shared__ int s_fail;
   if (threadIdx.x == 0) s_fail = failed(w);
   __syncthreads();
@@ -290,11 +290,13 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_bwd2(
   unsigned char* sI = sm + Bwd2Smem::ID;
   auto sN = [&](int c) { return sm + Bwd2Smem::NS + (c & 1) * 2 * TILE128; };
   auto vecp = [&](int c) { return reinterpret_cast<float*>(sm + Bwd2Smem::VEC + (c & 1) * 256); };
-  __shared__ uint64_t barN[2], barDK, barQ, barF, barC, barDU, barE;
+  // barH: the bulk stores issued after a barrier round have read dS'^T hi and the dU^T staging
+  __shared__ uint64_t barN[2], barDK, barQ, barF, barC, barDU, barH, barE;
   __shared__ uint32_t tslot;
   __shared__ volatile int s_abort;
   int* err = w.status;
   if (tid == 0) {
+    mbar_init(&barH, 1);
     mbar_init(&barN[0], 1);
     mbar_init(&barN[1], 1);
     mbar_init(&barDK, 1);
@@ -369,26 +371,11 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_bwd2(
     for (int q = 0; q < 8; ++q) f[q] = (8 * j + q == r) ? 1.f : 0.f;
     st_chunk_f(sI, r, j, TILE64, f);
   }
-  // dS'^T leaving chunk c (this thread's row part) as a compensated bf16 pair for the next
-  // products, and its hi part as dh[c]
-  auto put_state = [&](int c) {
-    uint32_t ph[16], pl[16];
+  // dS'^T leaving a chunk (this thread's row part) as a compensated bf16 pair for the next
+  // products; the hi tile is also dh
+  auto put_state = [&]() {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float h0 = __bfloat162float(__float2bfloat16_rn(S[2 * i]));
-      const float h1 = __bfloat162float(__float2bfloat16_rn(S[2 * i + 1]));
-      ph[i] = pack_bf16(h0, h1);
-      pl[i] = pack_bf16(S[2 * i] - h0, S[2 * i + 1] - h1);
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t o = sw128_chunk(row, 4 * cg + j, TILE128);
-      *reinterpret_cast<uint4*>(sDH + o) = make_uint4(ph[4 * j], ph[4 * j + 1], ph[4 * j + 2], ph[4 * j + 3]);
-      *reinterpret_cast<uint4*>(sDL + o) = make_uint4(pl[4 * j], pl[4 * j + 1], pl[4 * j + 2], pl[4 * j + 3]);
-    }
-    bf16* g = t.dh + ((size_t)unit_row(c) + row) * D + 32 * cg;
-    st_global_32B(g, ph);
-    st_global_32B(g + 16, ph + 8);
+    for (int j = 0; j < 4; ++j) st_chunk_split(sDH, sDL, row, 4 * cg + j, TILE128, S + 8 * j);
   };
   fence_proxy_async();  // the identity, before any product reads it
   tc_fence_before();
@@ -426,9 +413,14 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_bwd2(
       tc_fence_after();
       const uint64_t dah = desc_mnmajor(smem_u32(sDH), 0, TILE128);
       const uint64_t dal = desc_mnmajor(smem_u32(sDL), 0, TILE128);
-      // the -N^T slot of chunk c+1 (its chain product finished before the state warps released
-      // dS'_c) takes chunk c-1's
-      if (c > 0) issue_n(c - 1);
+      // dh[c] = the hi tile; dU^T of chunk c+1, staged in its -N^T slot
+      tma_store_3d(&mdh, sDH, 0, unit_row(c), 0);
+      tma_store_3d(&mdh, sDH + TILE128, 64, unit_row(c), 0);
+      if (c + 1 < nc) {
+        tma_store_3d(&mdUT, sN(c + 1), 0, unit_row(c + 1), 0);
+        tma_store_3d(&mdUTl, sN(c + 1) + TILE128, 0, unit_row(c + 1), 0);
+      }
+      tma_store_commit();
       if (!mbar_wait_abort(&barN[c & 1], npar(c), err, &s_abort)) continue;
       {
         const uint64_t dn = desc_mnmajor(smem_u32(sN(c)), 0, TILE128);
@@ -439,6 +431,11 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_bwd2(
         for (int s = 0; s < 8; ++s) mma_bf16(tACC(c), dn + mnstep_off(s), dal + mnstep_off(s), idC, 1);
         mma_commit(&barC);
       }
+      // once the stores have read them: dS'^T may be rewritten, and the slot of chunk c+1 (its
+      // chain product finished before the state warps released dS'_c) takes chunk c-1's -N^T
+      tma_store_wait_read0();
+      mbar_arrive(&barH);
+      if (c > 0) issue_n(c - 1);
       // chunk c's F and I have run: chunk c-1's Q, O', W, dU_loc replace theirs
       if (c > 0) {
         if (!mbar_wait_abort(&barF, par(c), err, &s_abort)) continue;
@@ -466,7 +463,7 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_bwd2(
     // product (its -N^T slot is refilled only after that product)
     float egc = 0.f;
     if (mbar_wait_abort(&barN[(nc - 1) & 1], npar(nc - 1), err, &s_abort)) egc = vecp(nc - 1)[63];
-    put_state(nc - 1);
+    put_state();
     fence_proxy_async();
     tc_fence_before();
     nbar_sync(1, kScanThreadsWS);
@@ -487,33 +484,24 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_bwd2(
       // (2) dU^T = DU as a hi/lo pair (rows v, 16 columns per thread), straight to the workspace
       okt = okt && mbar_wait_abort(&barDU, par(c), err, &s_abort);
       tc_fence_after();
-      if (okt) {
+      if (okt) {  // staged as two [128 v][64 i] tiles in chunk c's -N^T slot (chain(c) is done)
         float x[16];
         tmem_ld16(taddr(tb, 32 * qd, 256 + 64 * (c & 1) + 16 * cg), x);
         tmem_wait_ld();
-        bf16* hrow = t.dUT + ((size_t)unit_row(c) + row) * 64 + 16 * cg;
-        bf16* lrow = t.dUTl + ((size_t)unit_row(c) + row) * 64 + 16 * cg;
-        uint32_t ph[8], pl[8];
-#pragma unroll
-        for (int q = 0; q < 16; q += 2) {
-          const float h0 = __bfloat162float(__float2bfloat16_rn(x[q]));
-          const float h1 = __bfloat162float(__float2bfloat16_rn(x[q + 1]));
-          ph[q / 2] = pack_bf16(h0, h1);
-          pl[q / 2] = pack_bf16(x[q] - h0, x[q + 1] - h1);
-        }
-        st_global_32B(hrow, ph);  // 16 columns = one full 32-byte sector per row and part
-        st_global_32B(lrow, pl);
+        st_chunk_split(sN(c), sN(c) + TILE128, row, 2 * cg, TILE128, x);
+        st_chunk_split(sN(c), sN(c) + TILE128, row, 2 * cg + 1, TILE128, x + 8);
       }
       if (more) {
         // (3) both products of chunk c have read dS'^T: the next one (and dh[c-1]) replaces it
         okt = okt && mbar_wait_abort(&barN[(c - 1) & 1], npar(c - 1), err, &s_abort);
-        if (okt) {
-          egc = vecp(c - 1)[63];
-          put_state(c - 1);
-        }
+        if (okt) egc = vecp(c - 1)[63];
+        okt = okt && mbar_wait_abort(&barH, par(c), err, &s_abort);
+        if (okt) put_state();
         fence_proxy_async();
         tc_fence_before();
         nbar_sync(1, kScanThreadsWS);
+      } else {
+        fence_proxy_async();  // the last dU^T staging, stored after the final barrier
       }
     }
   }
@@ -524,9 +512,15 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_bwd2(
     for (int v = 0; v < 32; v += 4)
       *reinterpret_cast<float4*>(sr.s_out + st_off + v) = make_float4(S[v], S[v + 1], S[v + 2], S[v + 3]);
   }
-  // before the CTA leaves (after an error too): the last load on each barrier has landed, so
-  // every earlier one has; every MMA issued has finished
+  // before the CTA leaves (after an error too): the first chunk's dU^T is stored, the last load
+  // on each barrier has landed (so every earlier one has), every MMA issued has finished
   if (issuer) {
+    if (nc > 0 && !s_abort) {
+      tma_store_3d(&mdUT, sN(0), 0, unit_row(0), 0);
+      tma_store_3d(&mdUTl, sN(0) + TILE128, 0, unit_row(0), 0);
+      tma_store_commit();
+    }
+    tma_store_wait0();
     if (n_iss0 > 0) mbar_wait(&barN[0], (uint32_t)((n_iss0 - 1) & 1), nullptr);
     if (n_iss1 > 0) mbar_wait(&barN[1], (uint32_t)((n_iss1 - 1) & 1), nullptr);
     if (dk_iss > 0) mbar_wait(&barDK, (uint32_t)((dk_iss - 1) & 1), nullptr);
@@ -545,14 +539,14 @@ cudaError_t tc_scan_fwd(const Problem& p, const Args& a, const Work& w, const Tc
                         const TcMaps& m, const ScanRange& sr, cudaStream_t s) {
   const dim3 grid(p.Nst, p.HV);
   return tgo("tc_scan_fwd", k_tc_scan_fwd2, grid, kScanThreadsWS, (size_t)1024 + Fwd2Smem::TOTAL, s, p, a,
-             w, t, m.DK, m.NT, m.UtT, sr);
+             w, t, m.DK, m.NT, m.UtT, m.h, sr);
 }
 
 cudaError_t tc_scan_bwd(const Problem& p, const Args& a, const Work& w, const TcWork& t,
                         const TcMaps& m, const ScanRange& sr, cudaStream_t s) {
   const dim3 grid(p.Nst, p.HV);
   return tgo("tc_scan_bwd", k_tc_scan_bwd2, grid, kScanThreadsWS, (size_t)1024 + Bwd2Smem::TOTAL, s, p, a,
-             w, t, m.q, m.DK, m.Op, m.WT, m.dUlT, m.NT, sr);
+             w, t, m.q, m.DK, m.Op, m.WT, m.dUlT, m.NT, m.dh, m.dUT, m.dUTl, sr);
 }
 
 }  // namespace tcx

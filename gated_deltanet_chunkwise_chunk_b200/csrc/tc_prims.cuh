@@ -171,6 +171,15 @@ __device__ __forceinline__ uint32_t sw128_chunk(int r, int j, int block_bytes) {
 }
 
 // ------------------------------------------------------------------ descriptors
+// Descriptor step offsets (added to a descriptor; the start address field holds bytes / 16,
+// and addresses stay below 2^18 bytes, so the additions never carry out of the field).  The
+// builders below are written as a base plus such an offset, so that in an unrolled issue loop
+// the base is computed once and each MMA costs one add: a thread that computes descriptors
+// between MMAs issues them several times slower than the tensor pipe runs them (measured).
+__host__ __device__ constexpr uint64_t kstep_off(int s, int block_bytes) {
+  return (uint64_t)(((s >> 2) * block_bytes + (s & 3) * 32) >> 4);
+}
+__host__ __device__ constexpr uint64_t mnstep_off(int s) { return (uint64_t)((s * 2048) >> 4); }
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   uint64_t d = 0;
@@ -184,19 +193,13 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, ui
 // K-major operand (rows = M or N, columns = K) at K step s (16 columns) of a tile whose
 // column blocks are block_bytes apart.
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int s, int block_bytes) {
-  return sdesc(tile + (uint32_t)((s >> 2) * block_bytes + (s & 3) * 32), 16, 1024);
+  return sdesc(tile, 16, 1024) + kstep_off(s, block_bytes);
 }
 // MN-major operand (rows = K, columns = M or N) at K step s (16 rows); MN blocks of 64
 // columns are block_bytes apart.
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int s, int block_bytes) {
-  return sdesc(tile + (uint32_t)(s * 2048), (uint32_t)block_bytes, 1024);
+  return sdesc(tile, (uint32_t)block_bytes, 1024) + mnstep_off(s);
 }
-// Descriptor step offsets (added to a descriptor; the start address field holds bytes / 16,
-// and addresses stay below 2^18 bytes, so the additions never carry out of the field).
-__host__ __device__ constexpr uint64_t kstep_off(int s, int block_bytes) {
-  return (uint64_t)(((s >> 2) * block_bytes + (s & 3) * 32) >> 4);
-}
-__host__ __device__ constexpr uint64_t mnstep_off(int s) { return (uint64_t)((s * 2048) >> 4); }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
