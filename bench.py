@@ -63,28 +63,30 @@ def kernel_bytes_per_unit(K: int, V: int, G: int, e: int) -> dict:
     """HBM bytes each tcgen05 kernel moves per (chunk, value head) unit under the current kernel
     split: every operand tile it reads and every tile it writes once (a k-head's q/k tile is
     shared by its G value heads and counted once), inter-kernel intermediates included (bf16
-    tiles W^T, U~^T, D K, U^T, S, dS, dU_loc^T, O', dU^T hi/lo, dW, T hi/lo; fp32 dq/dk shares;
-    fp32 per-chunk vectors of 64).  Reported beside the roofline, not as the method's bytes."""
+    tiles W^T, U~^T, D K, -N^T, U^T, S, dS, dU_loc^T, O', dU^T hi/lo, dW, T hi/lo; the k-head's
+    fp32 dq/dk tiles; fp32 per-chunk vectors of 64).  Reported beside the roofline, not as the
+    method's bytes."""
     tq = C * K * e / G            # q or k tile, per value head
     tv = C * V * e                # v, o, dO, dv tile
     dk = C * K * e                # D K (per value head: scaled by its own decay), O'
     wt = K * C * e                # W^T, dW
     ut = V * C * e                # U~^T, U^T, dU_loc^T, dU^T (one part)
     st = V * K * e                # S or dS entering/leaving the chunk
+    nt = K * K * e                # -N^T, the state map's K x K factor
     tm = 2 * C * C * e            # T = (I + A)^-1 as a hi/lo pair
-    f32 = C * K * 4               # fp32 dq or dk share
+    f32 = C * K * 4 / G           # the k-head's fp32 dq or dk tile, per value head
     vec = C * 4                   # one per-chunk fp32 vector
     per = {
-        "wy": tq + tv + 3 * vec + wt + ut + tm + dk,
-        "scan_fwd": wt + ut + dk + vec + st,
+        "wy": tq + tv + 3 * vec + wt + ut + tm + dk + nt,
+        "scan_fwd": ut + nt + dk + vec + st,
         "out": 2 * tq + st + wt + ut + vec + tv + ut,
         "dvlocal": 2 * tq + tv + 2 * vec + ut + dk,
-        "scan_bwd": tq + dk + wt + dk + ut + vec + st + 2 * ut,
-        "dqkwg": 2 * tq + tv + 3 * ut + 2 * st + vec + wt + 2 * f32 + vec,
-        "wy_bwd": tq + tv + tm + wt + 2 * ut + 2 * vec + tv + 2 * f32 + 2 * vec,  # dk share added in L2
-        "dqdk_group_sum": 2 * f32 + 2 * tq,
+        "scan_bwd": nt + dk + tq + dk + wt + ut + vec + st + 2 * ut,
+        "dqkwg": 2 * tq + tv + 3 * ut + 2 * st + vec + wt + vec + 2 * f32,
+        "wy_bwd": tq + tv + tm + wt + 2 * ut + 2 * vec + tv + 2 * vec + 2 * f32,  # dk added in L2
+        "dqdk_out": 2 * f32 + 2 * tq,
     }
-    return {f"tc_{k}" if k != "dqdk_group_sum" else k: v for k, v in per.items()}
+    return {f"tc_{k}": v for k, v in per.items()}
 
 
 def step_flops_per_token_head(K: int, V: int) -> tuple[float, float]:

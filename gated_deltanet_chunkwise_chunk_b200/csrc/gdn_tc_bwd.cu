@@ -231,16 +231,18 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Args a, Work w, TcW
     tmem_alloc(&tslot, 512);
     tmem_relinquish();
   }
-  // units u = gc * HV + hv in [u0, u1); chunk-table entries past the chunk count are invalid
   // Units u = chunk * HV + hv in [u0, u1), handed out in k-head groups (chunk, hk) by an atomic
-  // counter: a CTA runs the G value heads of a group back to back and sums their dq and dk
-  // shares itself.  Chunk-table entries past the chunk count are invalid.
-  auto valid = [&](int u) { return u >= ur.u0 && u < ur.u1 && w.chunk_tab[u / p.HV].x >= 0; };
-  auto next_of = [&](int u) {  // thread 0: the unit after u (a counter fetch at a group's end)
+  // counter: a CTA runs the G value heads of a group back to back (their dq and dk shares go
+  // to the k-head's fp32 tiles in a fixed order).  Thread 0 takes the next unit a unit ahead;
+  // -1 marks the end of the work (past the range, or a chunk-table entry past the chunk count).
+  auto next_of = [&](int u) {
     if (u >= 0 && (u % p.HV) % p.G + 1 < p.G) return u + 1;
     const int kk = ur.u0 / p.G + atomicAdd(ur.ctr, 1);
-    return kk < ur.u1 / p.G ? (kk / p.H) * p.HV + (kk % p.H) * p.G : -1;
+    if (kk >= ur.u1 / p.G) return -1;
+    const int gc = kk / p.H;
+    return w.chunk_tab[gc].x >= 0 ? gc * p.HV + (kk % p.H) * p.G : -1;
   };
+  auto valid = [](int u) { return u >= 0; };
   auto load_A = [&](int u) {
     const int gc = u / p.HV, hk = (u % p.HV) / p.G, tok0 = w.chunk_tab[gc].w;
     mbar_expect_tx(&barA, 4 * TILE64 + TILE128);
@@ -293,7 +295,7 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Args a, Work w, TcW
   for (uint32_t it = 0; valid(u); ++it, u = nu) {
     const int gc = u / p.HV, hv = u % p.HV;
     const int4 e = w.chunk_tab[gc];
-    const int L = e.z, tok0 = e.w;
+    const int L = e.z;
     const size_t unit = (size_t)u;
     if (tid == 0) s_unit[(it + 1) & 1] = next_of(u);
     const uint32_t ph = it & 1;
@@ -304,7 +306,6 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Args a, Work w, TcW
     if (!ok) break;
     nu = s_unit[(it + 1) & 1];
     const bool nvalid = valid(nu);
-    g_next = g_of(nu);
     if (L < 64) {
       zero_tail_rows(sQ, L, tid, 256);
       zero_tail_rows(sK, L, tid, 256);
@@ -312,6 +313,7 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Args a, Work w, TcW
     }
     fence_proxy_async();
     __syncthreads();
+    g_next = g_of(nu);  // after the barrier: its latency hides behind this unit's products
     if (tid == 0) {
       const uint32_t q = smem_u32(sQ), k = smem_u32(sK), o = smem_u32(sO), ut = smem_u32(sUT),
                      dut = smem_u32(sdUT), dutl = smem_u32(sdUTl), h = smem_u32(sH), dh = smem_u32(sdH);
@@ -482,47 +484,31 @@ __global__ void __launch_bounds__(256) k_tc_dqkwg(Problem p, Args a, Work w, TcW
       pendA = (int)(ph ^ 1);
     }
     {
-      // dq, dk of this value head, summed over the group's value heads in order: the running
-      // sums sit in this CTA's two scratch tiles (fp32, cache-resident); after the last value
-      // head dq is final (bf16 out) and dk goes to the k-head's fp32 tile that wy_bwd completes
+      // dq, dk of this value head into the k-head's fp32 tiles: the group's first value head
+      // stores, the others add (L2 reductions; one thread's operations on an address stay in
+      // order, so every sum is taken in the same order on every run)
       float x[32], y[32];
       tmem_ld16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
       tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), y);
       tmem_wait_ld();
-      const int j = hv % p.G;
-      float* sq0 = w.dqp + ((size_t)blockIdx.x * 64 + r0) * D + 64 * half + cq;
-      float* sk0 = w.dqp + ((size_t)(gridDim.x + blockIdx.x) * 64 + r0) * D + 64 * half + cq;
-      if (j > 0) {
+      const size_t kk = (size_t)gc * p.H + hv / p.G;
+      float* dq0 = w.dqp + (kk * 64 + r0) * D + 64 * half + cq;
+      float* dk0 = w.dkp + (kk * 64 + r0) * D + 64 * half + cq;
+      if (hv % p.G == 0) {
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
-          const float2 a0 = *reinterpret_cast<const float2*>(sq0 + 8 * jj);
-          const float2 a1 = *reinterpret_cast<const float2*>(sq0 + 8 * D + 8 * jj);
-          const float2 b0 = *reinterpret_cast<const float2*>(sk0 + 8 * jj);
-          const float2 b1 = *reinterpret_cast<const float2*>(sk0 + 8 * D + 8 * jj);
-          x[4 * jj] += a0.x; x[4 * jj + 1] += a0.y; x[4 * jj + 2] += a1.x; x[4 * jj + 3] += a1.y;
-          y[4 * jj] += b0.x; y[4 * jj + 1] += b0.y; y[4 * jj + 2] += b1.x; y[4 * jj + 3] += b1.y;
-        }
-      }
-      if (j + 1 < p.G) {
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          *reinterpret_cast<float2*>(sq0 + 8 * jj) = make_float2(x[4 * jj], x[4 * jj + 1]);
-          *reinterpret_cast<float2*>(sq0 + 8 * D + 8 * jj) = make_float2(x[4 * jj + 2], x[4 * jj + 3]);
-          *reinterpret_cast<float2*>(sk0 + 8 * jj) = make_float2(y[4 * jj], y[4 * jj + 1]);
-          *reinterpret_cast<float2*>(sk0 + 8 * D + 8 * jj) = make_float2(y[4 * jj + 2], y[4 * jj + 3]);
-        }
-      } else {
-        const int hk = hv / p.G;
-        float* dk0 = w.dkp + (((size_t)gc * p.H + hk) * 64 + r0) * D + 64 * half + cq;
-        bf16* q0 = static_cast<bf16*>(a.dq) + ((size_t)(tok0 + r0) * p.H + hk) * p.K + 64 * half + cq;
-        bf16* q1 = q0 + (size_t)8 * p.H * p.K;
-        const bool live = 64 * half < p.K;  // columns past a 64-wide key head are padding
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
+          *reinterpret_cast<float2*>(dq0 + 8 * jj) = make_float2(x[4 * jj], x[4 * jj + 1]);
+          *reinterpret_cast<float2*>(dq0 + 8 * D + 8 * jj) = make_float2(x[4 * jj + 2], x[4 * jj + 3]);
           *reinterpret_cast<float2*>(dk0 + 8 * jj) = make_float2(y[4 * jj], y[4 * jj + 1]);
           *reinterpret_cast<float2*>(dk0 + 8 * D + 8 * jj) = make_float2(y[4 * jj + 2], y[4 * jj + 3]);
-          if (live && r0 < L) *reinterpret_cast<uint32_t*>(q0 + 8 * jj) = pack_bf16(x[4 * jj], x[4 * jj + 1]);
-          if (live && r1 < L) *reinterpret_cast<uint32_t*>(q1 + 8 * jj) = pack_bf16(x[4 * jj + 2], x[4 * jj + 3]);
+        }
+      } else {
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          atomicAdd(reinterpret_cast<float2*>(dq0 + 8 * jj), make_float2(x[4 * jj], x[4 * jj + 1]));
+          atomicAdd(reinterpret_cast<float2*>(dq0 + 8 * D + 8 * jj), make_float2(x[4 * jj + 2], x[4 * jj + 3]));
+          atomicAdd(reinterpret_cast<float2*>(dk0 + 8 * jj), make_float2(y[4 * jj], y[4 * jj + 1]));
+          atomicAdd(reinterpret_cast<float2*>(dk0 + 8 * D + 8 * jj), make_float2(y[4 * jj + 2], y[4 * jj + 3]));
         }
       }
     }
@@ -610,14 +596,17 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     tmem_relinquish();
   }
   // Units u = chunk * HV + hv in [u0, u1), handed out in k-head groups (chunk, hk) by an atomic
-  // counter: a CTA runs the G value heads of a group back to back and sums their dq and dk
-  // shares itself.  Chunk-table entries past the chunk count are invalid.
-  auto valid = [&](int u) { return u >= ur.u0 && u < ur.u1 && w.chunk_tab[u / p.HV].x >= 0; };
-  auto next_of = [&](int u) {  // thread 0: the unit after u (a counter fetch at a group's end)
+  // counter: a CTA runs the G value heads of a group back to back (their dq and dk shares go
+  // to the k-head's fp32 tiles in a fixed order).  Thread 0 takes the next unit a unit ahead;
+  // -1 marks the end of the work (past the range, or a chunk-table entry past the chunk count).
+  auto next_of = [&](int u) {
     if (u >= 0 && (u % p.HV) % p.G + 1 < p.G) return u + 1;
     const int kk = ur.u0 / p.G + atomicAdd(ur.ctr, 1);
-    return kk < ur.u1 / p.G ? (kk / p.H) * p.HV + (kk % p.H) * p.G : -1;
+    if (kk >= ur.u1 / p.G) return -1;
+    const int gc = kk / p.H;
+    return w.chunk_tab[gc].x >= 0 ? gc * p.HV + (kk % p.H) * p.G : -1;
   };
+  auto valid = [](int u) { return u >= 0; };
   auto load_A = [&](int u, int buf) {
     const int hk = (u % p.HV) / p.G, tok0 = w.chunk_tab[u / p.HV].w;
     unsigned char* dst = sKb + buf * 2 * TILE64;
@@ -688,7 +677,6 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     if (!ok) break;
     nu = s_unit[(it + 1) & 1];
     const bool nvalid = valid(nu);
-    vec_of(nu);
     unsigned char* sK = sKb + (it & 1) * 2 * TILE64;
     if (tid == 0 && nvalid) {  // the other K buffer was last read by the previous unit
       load_A(nu, (int)(ph ^ 1));
@@ -700,6 +688,7 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     }
     fence_proxy_async();
     __syncthreads();
+    vec_of(nu);  // after the barrier: its latency hides behind this unit's products
     const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aT = smem_u32(sT), aTl = smem_u32(sTl),
                    aW = smem_u32(sdW), aU = smem_u32(sdUT), aUl = smem_u32(sdUTl);
     if (tid == 0) {
@@ -927,40 +916,15 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
     ok = __syncthreads_and(ok && mbar_wait(&barM, 1, err));
     tc_fence_after();
     if (!ok) break;
-    {  // this kernel's dk share, summed over the group's value heads in order (running sum in
-       // this CTA's scratch tile), then added to dqkwg's k-head tile: dk final, bf16 out
+    {  // this kernel's dk share, added onto dqkwg's k-head tile (value heads in order)
       float x[32];
       tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
       tmem_wait_ld();
-      const int j = hv % p.G;
-      float* s0 = w.dqp + ((size_t)blockIdx.x * 64 + r0) * D + 64 * half + cq;
-      if (j > 0) {
+      float* dk0 = w.dkp + (((size_t)gc * p.H + hv / p.G) * 64 + r0) * D + 64 * half + cq;
   #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const float2 a0 = *reinterpret_cast<const float2*>(s0 + 8 * jj);
-          const float2 a1 = *reinterpret_cast<const float2*>(s0 + 8 * D + 8 * jj);
-          x[4 * jj] += a0.x; x[4 * jj + 1] += a0.y; x[4 * jj + 2] += a1.x; x[4 * jj + 3] += a1.y;
-        }
-      }
-      if (j + 1 < p.G) {
-  #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          *reinterpret_cast<float2*>(s0 + 8 * jj) = make_float2(x[4 * jj], x[4 * jj + 1]);
-          *reinterpret_cast<float2*>(s0 + 8 * D + 8 * jj) = make_float2(x[4 * jj + 2], x[4 * jj + 3]);
-        }
-      } else {
-        const int hk = hv / p.G;
-        const float* p0 = w.dkp + (((size_t)gc * p.H + hk) * 64 + r0) * D + 64 * half + cq;
-        bf16* k0 = static_cast<bf16*>(a.dk) + ((size_t)(tok0 + r0) * p.H + hk) * p.K + 64 * half + cq;
-        bf16* k1 = k0 + (size_t)8 * p.H * p.K;
-        const bool live = 64 * half < p.K;
-  #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const float2 a0 = *reinterpret_cast<const float2*>(p0 + 8 * jj);
-          const float2 a1 = *reinterpret_cast<const float2*>(p0 + 8 * D + 8 * jj);
-          if (live && r0 < L) *reinterpret_cast<uint32_t*>(k0 + 8 * jj) = pack_bf16(x[4 * jj] + a0.x, x[4 * jj + 1] + a0.y);
-          if (live && r1 < L) *reinterpret_cast<uint32_t*>(k1 + 8 * jj) = pack_bf16(x[4 * jj + 2] + a1.x, x[4 * jj + 3] + a1.y);
-        }
+      for (int jj = 0; jj < 8; ++jj) {
+        atomicAdd(reinterpret_cast<float2*>(dk0 + 8 * jj), make_float2(x[4 * jj], x[4 * jj + 1]));
+        atomicAdd(reinterpret_cast<float2*>(dk0 + 8 * D + 8 * jj), make_float2(x[4 * jj + 2], x[4 * jj + 3]));
       }
     }
     // the next unit's first MMAs overwrite every TMEM column read above
@@ -978,6 +942,26 @@ __global__ void __launch_bounds__(256) k_tc_wy_bwd(Problem p, Args a, Work w, Tc
   if (warp == 0) tmem_dealloc(tb, 512);
 }
 
+// dq, dk of one chunk and k-head from their fp32 tiles (the sums dqkwg and wy_bwd formed) to the
+// caller's bf16 [token][head][K] tensors: rows past the chunk's end and columns past a 64-wide
+// head are skipped.  Four columns per thread and step.
+__global__ void __launch_bounds__(256) k_tc_dqdk_out(Problem p, Args a, Work w, int gc0) {
+  if (failed(w)) return;
+  const int gc = gc0 + blockIdx.x, hk = blockIdx.y;
+  const int4 e = w.chunk_tab[gc];
+  if (e.x < 0) return;
+  const int L = e.z, tok0 = e.w, K = p.K;
+  const size_t base = ((size_t)gc * p.H + hk) * 64 * D;
+  for (int i = 4 * threadIdx.x; i < L * K; i += 4 * blockDim.x) {
+    const int t = i / K, c = i % K;
+    const float4 q = *reinterpret_cast<const float4*>(w.dqp + base + (size_t)t * D + c);
+    const float4 k = *reinterpret_cast<const float4*>(w.dkp + base + (size_t)t * D + c);
+    const size_t o = ((size_t)(tok0 + t) * p.H + hk) * K + c;
+    *reinterpret_cast<uint2*>(static_cast<bf16*>(a.dq) + o) = make_uint2(pack_bf16(q.x, q.y), pack_bf16(q.z, q.w));
+    *reinterpret_cast<uint2*>(static_cast<bf16*>(a.dk) + o) = make_uint2(pack_bf16(k.x, k.y), pack_bf16(k.z, k.w));
+  }
+}
+
 }  // namespace
 
 cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, const TcWork& t,
@@ -991,15 +975,16 @@ cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, 
                t, m.q, m.k, m.dO, m.Op, c0);
   };
   auto chunk_kernels = [&](int i, int c0, int c1, cudaStream_t st) {
-    // persistent CTAs over k-head groups; 2 * grid <= units for G >= 2, so every CTA's two
-    // scratch tiles fit in the dq share area
+    // persistent CTAs over k-head groups
     const int groups = (c1 - c0) * p.H;
     const dim3 gp((unsigned)std::min(groups, num_sms()));
     if ((e = tgo("tc_dqkwg", k_tc_dqkwg, gp, 256, 1024 + DqkSmem::TOTAL, st, p, a, w, t, m.q, m.k, m.dO,
                  m.UT, m.dUT, m.dUTl, m.h, m.dh, m.dW, UnitRange{c0 * p.HV, c1 * p.HV, t.ctr + 2 * i})))
       return e;
-    return tgo("tc_wy_bwd", k_tc_wy_bwd, gp, 256, 1024 + WyBwdSmem::TOTAL, st, p, a, w, t, m.k, m.v,
-               m.Tm, m.dW, m.dUT, m.dUTl, UnitRange{c0 * p.HV, c1 * p.HV, t.ctr + 2 * i + 1});
+    if ((e = tgo("tc_wy_bwd", k_tc_wy_bwd, gp, 256, 1024 + WyBwdSmem::TOTAL, st, p, a, w, t, m.k, m.v,
+                 m.Tm, m.dW, m.dUT, m.dUTl, UnitRange{c0 * p.HV, c1 * p.HV, t.ctr + 2 * i + 1})))
+      return e;
+    return tgo("tc_dqdk_out", k_tc_dqdk_out, dim3(c1 - c0, p.H), 256, 0, st, p, a, w, c0);
   };
   if (sg.n == 1) {
     if ((e = dvlocal(0, p.NCmax, s))) return e;
