@@ -479,7 +479,7 @@ cudaError_t forward_impl(const Problem& p, const Args& a, const Work& w, const L
                L.m.k, L.m.UtT, L.m.WT, L.m.UT, L.m.h, c0);
   };
   float* ht = bwd_prep ? nullptr : a.ht;
-  const Segments sg = segments(p);
+  const Segments sg = segments(p, kFwdSeg);
   cudaError_t e;
   if (sg.n == 1) {
     if ((e = wy(0, p.NCmax, s))) return e;

@@ -966,7 +966,7 @@ __global__ void __launch_bounds__(256) k_tc_dqdk_out(Problem p, Args a, Work w, 
 
 cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, const TcWork& t,
                                 const TcMaps& m, cudaStream_t s) {
-  const Segments sg = segments(p);
+  const Segments sg = segments(p, kBwdSeg);
   cudaError_t e;
   // one work counter per persistent launch, zero before any of them starts
   if ((e = cudaMemsetAsync(t.ctr, 0, kCounters * sizeof(int), s))) return e;

@@ -97,7 +97,9 @@ struct TcWork {
 
 // A single sequence's chunks are split into segments so that the sequential pass over one
 // segment (one CTA per value head, few SMs) overlaps the chunk-parallel kernels of others.
-constexpr int kMaxSeg = 8;          // segments of a pass
+constexpr int kMaxSeg = 8;          // segments of a pass (at most)
+constexpr int kFwdSeg = 3;          // the forward's: its chunk kernels outrun its pass
+constexpr int kBwdSeg = 8;          // the backward's: its pass is the longer one
 constexpr int kSegChunks = 32;      // at least this many chunks per segment
 constexpr int kCounters = 2 * kMaxSeg;
 
@@ -106,7 +108,7 @@ struct Segments {
   int c[kMaxSeg + 1];     // segment i covers chunks [c[i], c[i+1])
 };
 
-inline Segments segments(const Problem& p) {
+inline Segments segments(const Problem& p, int max_seg) {
   Segments sg{};
   sg.n = 1;
   sg.c[0] = 0;
@@ -114,7 +116,7 @@ inline Segments segments(const Problem& p) {
   // only one sequence (chunks of one segment are contiguous in the chunk table), and only
   // when the pass leaves most SMs to the other kernels
   if (p.Nst != 1 || 2 * p.HV > num_sms()) return sg;
-  const int n = std::min(kMaxSeg, p.NCmax / kSegChunks);
+  const int n = std::min(std::min(max_seg, kMaxSeg), p.NCmax / kSegChunks);
   if (n < 2) return sg;
   sg.n = n;
   for (int i = 0; i <= n; ++i) sg.c[i] = (int)((long long)p.NCmax * i / n);
