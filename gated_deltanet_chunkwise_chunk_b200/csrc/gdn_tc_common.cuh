@@ -98,8 +98,11 @@ struct TcWork {
 // A single sequence's chunks are split into segments so that the sequential pass over one
 // segment (one CTA per value head, few SMs) overlaps the chunk-parallel kernels of others.
 constexpr int kMaxSeg = 8;          // segments of a pass (at most)
-constexpr int kFwdSeg = 3;          // the forward's: its chunk kernels outrun its pass
-constexpr int kBwdSeg = 8;          // the backward's: its pass is the longer one
+// Segments of the forward and of the backward (measured at 512 chunks x 32 value heads: the
+// forward's pass is short next to its chunk kernels, so fewer, longer launches pay; the
+// backward's longer pass wants finer overlap)
+constexpr int kFwdSeg = 3;
+constexpr int kBwdSeg = 8;
 constexpr int kSegChunks = 32;      // at least this many chunks per segment
 constexpr int kCounters = 2 * kMaxSeg;
 
