@@ -527,7 +527,7 @@ def kernel_roofline(prof: dict, case, pk: dict, steps: int = 2) -> dict | None:
     out = {"kernel": name, "launch_ms": round(per_launch_s * 1e3, 4),
            "share": round(total_ms / sum(v[1] for v in prof.values()), 4),
            "units_per_launch": round(units, 1), "launches_per_step": per_step}
-    traffic = _traffic(name, case)
+    traffic = _traffic(name, case, units)
     if fl is not None and name.startswith("ffma_"):
         achieved = fl * th / per_launch_s / 1e12
         peak = FP32_ALU_TFLOPS
@@ -562,16 +562,21 @@ def chunks_of(case) -> int:
     return case.B * ((case.T + C - 1) // C)
 
 
-def _traffic(name: str, case):
-    """DRAM bytes per launch from the committed ncu summary, when it covers this kernel."""
+def _traffic(name: str, case, units_per_launch: float):
+    """DRAM bytes per launch (read + write) from the committed one-kernel ncu captures, when they
+    cover this kernel at this head shape: measured bytes per unit x the units of one launch."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
+        shape = d.get("shape", {})
+        if (shape.get("K"), shape.get("V"), shape.get("G"), shape.get("dtype")) != (
+                case.K, case.V, case.HV // case.H, case.dtype):
+            return None
         rec = d.get("kernels", {}).get(name)
-        if rec and d.get("workload") == case.name:
-            return rec["bytes_per_launch"]
-    except (OSError, ValueError):
+        if rec:
+            return int(rec["bytes_per_unit"] * units_per_launch)
+    except (OSError, ValueError, KeyError):
         pass
     return None
 
