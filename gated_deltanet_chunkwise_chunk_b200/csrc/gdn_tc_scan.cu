@@ -431,11 +431,6 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_bwd2(
         for (int s = 0; s < 8; ++s) mma_bf16(tACC(c), dn + mnstep_off(s), dal + mnstep_off(s), idC, 1);
         mma_commit(&barC);
       }
-      // once the stores have read them: dS'^T may be rewritten, and the slot of chunk c+1 (its
-      // chain product finished before the state warps released dS'_c) takes chunk c-1's -N^T
-      tma_store_wait_read0();
-      mbar_arrive(&barH);
-      if (c > 0) issue_n(c - 1);
       // chunk c's F and I have run: chunk c-1's Q, O', W, dU_loc replace theirs
       if (c > 0) {
         if (!mbar_wait_abort(&barF, par(c), err, &s_abort)) continue;
@@ -451,7 +446,12 @@ __global__ void __launch_bounds__(kScanThreadsWS, 1) k_tc_scan_bwd2(
         for (int s = 0; s < 8; ++s) mma_bf16(tDU(c), dal + mnstep_off(s), dkK + kstep_off(s, TILE64), idU, 1);
         mma_commit(&barDU);
       }
+      // once the stores have read them: dS'^T may be rewritten, and the slot of chunk c+1 (its
+      // chain product finished before the state warps released dS'_c) takes chunk c-1's -N^T
+      tma_store_wait_read0();
+      mbar_arrive(&barH);
       if (c == 0) continue;
+      issue_n(c - 1);
       // the previous chunk's state-free products go in behind this chunk's; D K is replaced
       // once dU(c) has read it
       if (!mbar_wait_abort(&barQ, par(c - 1), err, &s_abort)) continue;
