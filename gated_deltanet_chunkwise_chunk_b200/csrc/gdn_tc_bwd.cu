@@ -24,13 +24,16 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 // ======================================================================================
-// dv_local: dU_loc^T = scale dO^T P  (M=128 v, N=64 j, K=64 i), after QK^T (M=64).
+// dv_local: dU_loc^T = scale dO^T P  (M=128 v, N=64 j, K=64 i), after QK^T (M=64).  P takes
+// K's place once QK^T has read it, and dU_loc^T K's place again once P has been read, so that
+// four CTAs fit on an SM; both outputs leave by bulk stores.
 // ======================================================================================
 __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
                                                     const __grid_constant__ CUtensorMap mq,
                                                     const __grid_constant__ CUtensorMap mk,
                                                     const __grid_constant__ CUtensorMap mdO,
-                                                    const __grid_constant__ CUtensorMap mOp, int gc0) {
+                                                    const __grid_constant__ CUtensorMap mOp,
+                                                    const __grid_constant__ CUtensorMap mdUlT, int gc0) {
   if (failed(w)) return;
   const int gc = gc0 + blockIdx.x, hv = blockIdx.y, hk = hv / p.G;
   const int4 e = w.chunk_tab[gc];
@@ -41,9 +44,9 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
   unsigned char* sQ = sm;
   unsigned char* sK = sQ + 2 * TILE64;
   unsigned char* sO = sK + 2 * TILE64;
-  unsigned char* sP = sO + 2 * TILE64;      // P hi
-  unsigned char* sPl = sP + TILE64;         // P lo
-  float* sG = reinterpret_cast<float*>(sPl + TILE64);
+  unsigned char* sP = sK;                   // P hi, then dU_loc^T [128][64] over both halves
+  unsigned char* sPl = sK + TILE64;         // P lo
+  float* sG = reinterpret_cast<float*>(sO + 2 * TILE64);
   float* sEo = sG + 64;                     // -scale e^{G_i}, zero past the chunk end
   __shared__ uint64_t bar[2];
   __shared__ uint32_t tslot;
@@ -126,21 +129,17 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 1, err));
   tc_fence_after();
-  if (ok) {
+  if (ok) {  // dU_loc^T row v (TMEM lane), staged as a [128][64] tile where P was
     const int v = 32 * warp + lane;
-    bf16* row = t.dUlT + (((size_t)gc * p.HV + hv) * D + v) * 64;
+#pragma unroll
     for (int c = 0; c < 64; c += 16) {
       float d[16];
       tmem_ld16(taddr(tb, 32 * warp, 64 + c), d);
       tmem_wait_ld();
-      uint4 a0, a1;
+#pragma unroll
       for (int q = 0; q < 16; ++q) d[q] *= p.scale;
-      a0.x = pack_bf16(d[0], d[1]); a0.y = pack_bf16(d[2], d[3]);
-      a0.z = pack_bf16(d[4], d[5]); a0.w = pack_bf16(d[6], d[7]);
-      a1.x = pack_bf16(d[8], d[9]); a1.y = pack_bf16(d[10], d[11]);
-      a1.z = pack_bf16(d[12], d[13]); a1.w = pack_bf16(d[14], d[15]);
-      *reinterpret_cast<uint4*>(row + c) = a0;
-      *reinterpret_cast<uint4*>(row + c + 8) = a1;
+      st_chunk_f(sP, v, c / 8, TILE128, d);
+      st_chunk_f(sP, v, c / 8 + 1, TILE128, d + 8);
     }
     // the products are done with dO: it becomes O' = -scale e^G dO for the reverse pass
     for (int idx = tid; idx < 64 * 16; idx += 128) {
@@ -159,8 +158,9 @@ __global__ void __launch_bounds__(128) k_tc_dvlocal(Problem p, Work w, TcWork t,
     const int orow = (gc * p.HV + hv) * 64;
     tma_store_3d(&mOp, sO, 0, orow, 0);
     tma_store_3d(&mOp, sO + TILE64, 64, orow, 0);
+    tma_store_3d(&mdUlT, sP, 0, (gc * p.HV + hv) * D, 0);
     tma_store_commit();
-    tma_store_wait0();
+    tma_store_wait_read0();
   }
   tc_fence_before();
   __syncthreads();
@@ -971,8 +971,8 @@ cudaError_t tc_backward_kernels(const Problem& p, const Args& a, const Work& w, 
   // one work counter per persistent launch, zero before any of them starts
   if ((e = cudaMemsetAsync(t.ctr, 0, kCounters * sizeof(int), s))) return e;
   auto dvlocal = [&](int c0, int c1, cudaStream_t st) {
-    return tgo("tc_dvlocal", k_tc_dvlocal, dim3(c1 - c0, p.HV), 128, 1024 + 8 * TILE64 + 512, st, p, w,
-               t, m.q, m.k, m.dO, m.Op, c0);
+    return tgo("tc_dvlocal", k_tc_dvlocal, dim3(c1 - c0, p.HV), 128, 1024 + 6 * TILE64 + 512, st, p, w,
+               t, m.q, m.k, m.dO, m.Op, m.dUlT, c0);
   };
   auto chunk_kernels = [&](int i, int c0, int c1, cudaStream_t st) {
     // persistent CTAs over k-head groups
