@@ -13,7 +13,13 @@
 // CTA (sequence, value head, z) holds rows v0 = 32z .. v0+31 of S.  Thread (kg, vg) keeps
 // S[v0+4vg .. +3][kg*K/16 .. (kg+1)*K/16) in fp32 registers, so the state moves as 16-byte
 // rows of h[k][v]; the 16 k-groups of a column block sit in one warp (lane = kg + 16 (vg%2)),
-// so row sums are four shuffles.
+// so row sums are four shuffles.  With a scalar gate each thread reads its own channels of k
+// and q and its rows of v straight from global memory (one vector load each; the 16 k-groups
+// of a warp read whole 256-byte rows) and computes the gate itself, so a token needs no shared
+// memory and no block barrier; the KDA variant shares its per-channel decays through shared
+// memory.
+#include <type_traits>
+
 #include "gdn_common.cuh"
 #include "gdn_launch.h"
 
@@ -21,6 +27,34 @@ namespace gdn {
 namespace {
 
 constexpr int RV = 32;  // state rows per CTA
+
+// N (4 or 8) consecutive elements at p (16-byte aligned for fp32, 8/16-byte for bf16) as floats
+template <typename T, int N>
+__device__ __forceinline__ void ld_floats(const T* p, float* out) {
+  if constexpr (std::is_same<T, float>::value) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(p + i);
+      out[i] = x.x; out[i + 1] = x.y; out[i + 2] = x.z; out[i + 3] = x.w;
+    }
+  } else if constexpr (N == 8) {
+    const uint4 x = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      out[2 * i] = f.x; out[2 * i + 1] = f.y;
+    }
+  } else {
+    const uint2 x = *reinterpret_cast<const uint2*>(p);
+    const uint32_t w[2] = {x.x, x.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      out[2 * i] = f.x; out[2 * i + 1] = f.y;
+    }
+  }
+}
 
 template <typename T, int K, bool KDA>
 __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* status) {
@@ -30,10 +64,10 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
   const int nz = p.V / RV;
   const int n = blockIdx.x / nz, hv = blockIdx.y, hk = hv / p.G, v0 = RV * (blockIdx.x % nz);
   const int tid = threadIdx.x, lane = tid & 31, kg = lane & 15, vg = 2 * (tid >> 5) + (lane >> 4);
-  __shared__ __align__(16) float sk[K];
-  __shared__ __align__(16) float sq[K];
+  __shared__ __align__(16) float sk[KDA ? K : 4];
+  __shared__ __align__(16) float sq[KDA ? K : 4];
   __shared__ __align__(16) float sdk[KDA ? K : 4];
-  __shared__ float sv[RV], sdec, sbeta;
+  __shared__ float sv[RV], sbeta;
   int bos, eos;
   if (p.varlen) {
     bos = (int)a.cu[n];
@@ -81,43 +115,51 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
   };
   const size_t dtb_k = (size_t)hv * K;
   for (int t = bos; t < eos; ++t) {
-    // every load of this token first (one latency), spread over the threads; then one round
-    // of shared-memory stores between two barriers (K <= 128: one channel per thread)
     const size_t qk0 = ((size_t)t * p.H + hk) * K, v_0 = ((size_t)t * p.HV + hv) * p.V + v0;
     const size_t gi = (size_t)t * p.HV + hv;
-    float kf = 0.f, qf = 0.f, vf = 0.f, gf = 0.f, bf = 0.f;
-    if (tid < K) {
-      kf = to_f<T>(k[qk0 + tid]);
-      qf = to_f<T>(q[qk0 + tid]);
-      if constexpr (KDA) gf = a.g_raw[gi * K + tid] + (a.dt_bias ? a.dt_bias[dtb_k + tid] : 0.f);
-    }
-    if (tid < RV) vf = to_f<T>(v[v_0 + tid]);
-    if (!KDA && tid == 64) gf = a.g_raw[gi] + dtb;
-    if (tid == 96) bf = a.beta[gi];
-    __syncthreads();  // the previous token's vectors are no longer read
-    if (tid < K) {
-      sk[tid] = kf;
-      sq[tid] = qf;
-      if constexpr (KDA) sdk[tid] = expf(nexp * (gf > 20.f ? gf : log1pf(expf(gf))));
-    }
-    if (tid < RV) sv[tid] = vf;
-    if (!KDA && tid == 64) sdec = expf(nexp * (gf > 20.f ? gf : log1pf(expf(gf))));
-    if (tid == 96) sbeta = bf;
-    __syncthreads();
-    const float b = sbeta;
-    float kv[KQ], qv[KQ], dv[KQ];  // this thread's channels, read as 16-byte vectors
+    float kv[KQ], qv[KQ], dv[KQ], vv[4];  // this thread's channels and rows
+    float b;
+    if constexpr (!KDA) {
+      ld_floats<T, KQ>(k + qk0 + kg * KQ, kv);
+      ld_floats<T, KQ>(q + qk0 + kg * KQ, qv);
+      ld_floats<T, 4>(v + v_0 + 4 * vg, vv);
+      const float gf = a.g_raw[gi] + dtb;
+      b = a.beta[gi];
+      const float dec = expf(nexp * (gf > 20.f ? gf : log1pf(expf(gf))));
 #pragma unroll
-    for (int i = 0; i < KQ; i += 4) {
-      const float4 k4 = *reinterpret_cast<const float4*>(sk + kg * KQ + i);
-      const float4 q4 = *reinterpret_cast<const float4*>(sq + kg * KQ + i);
-      kv[i] = k4.x; kv[i + 1] = k4.y; kv[i + 2] = k4.z; kv[i + 3] = k4.w;
-      qv[i] = q4.x; qv[i + 1] = q4.y; qv[i + 2] = q4.z; qv[i + 3] = q4.w;
-      if constexpr (KDA) {
-        const float4 d4 = *reinterpret_cast<const float4*>(sdk + kg * KQ + i);
-        dv[i] = d4.x; dv[i + 1] = d4.y; dv[i + 2] = d4.z; dv[i + 3] = d4.w;
-      } else {
-        dv[i] = dv[i + 1] = dv[i + 2] = dv[i + 3] = sdec;
+      for (int i = 0; i < KQ; ++i) dv[i] = dec;
+    } else {
+      // every load of this token first (one latency), spread over the threads; then one round
+      // of shared-memory stores between two barriers (K <= 128: one channel per thread)
+      float kf = 0.f, qf = 0.f, vf = 0.f, gf = 0.f, bf = 0.f;
+      if (tid < K) {
+        kf = to_f<T>(k[qk0 + tid]);
+        qf = to_f<T>(q[qk0 + tid]);
+        gf = a.g_raw[gi * K + tid] + (a.dt_bias ? a.dt_bias[dtb_k + tid] : 0.f);
       }
+      if (tid < RV) vf = to_f<T>(v[v_0 + tid]);
+      if (tid == 96) bf = a.beta[gi];
+      __syncthreads();  // the previous token's vectors are no longer read
+      if (tid < K) {
+        sk[tid] = kf;
+        sq[tid] = qf;
+        sdk[tid] = expf(nexp * (gf > 20.f ? gf : log1pf(expf(gf))));
+      }
+      if (tid < RV) sv[tid] = vf;
+      if (tid == 96) sbeta = bf;
+      __syncthreads();
+      b = sbeta;
+#pragma unroll
+      for (int i = 0; i < KQ; i += 4) {  // read as 16-byte vectors
+        const float4 k4 = *reinterpret_cast<const float4*>(sk + kg * KQ + i);
+        const float4 q4 = *reinterpret_cast<const float4*>(sq + kg * KQ + i);
+        const float4 d4 = *reinterpret_cast<const float4*>(sdk + kg * KQ + i);
+        kv[i] = k4.x; kv[i + 1] = k4.y; kv[i + 2] = k4.z; kv[i + 3] = k4.w;
+        qv[i] = q4.x; qv[i + 1] = q4.y; qv[i + 2] = q4.z; qv[i + 3] = q4.w;
+        dv[i] = d4.x; dv[i + 1] = d4.y; dv[i + 2] = d4.z; dv[i + 3] = d4.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) vv[i] = sv[4 * vg + i];
     }
     float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -127,7 +169,6 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
       e.x += S4[i].x * kv[i]; e.y += S4[i].y * kv[i]; e.z += S4[i].z * kv[i]; e.w += S4[i].w * kv[i];
     }
     e = gather4(rowsum4(e));
-    const float* vv = sv + 4 * vg;
     const float dx = b * (vv[0] - e.x), dy = b * (vv[1] - e.y), dz = b * (vv[2] - e.z),
                 dw = b * (vv[3] - e.w);
     float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
