@@ -36,11 +36,15 @@ __device__ __forceinline__ bool kda_failed(const KdaWork& w) { return *((volatil
 // Per-channel gated products of a 64 x 64 weight Wt (lower triangle used, ldw) with row
 // operand R and column operand Lm ([64][K], row stride K), Gam2 = Gam * log2(e) ([64][K]):
 //   F_i = sum_{j<=i} Wt_ij R_j e^{Gam_i - Gam_j},   G_j = sum_{i>=j} colw_i Wt_ij Lm_i e^{Gam_i - Gam_j}
-// (colw = per-row weights of the column product, or null).  Each result element is handed to
+// (colw = per-row weights of the column product, or null; R and Lm fp32 or bf16).  Each result
+// element is handed to
 // sink(i, c, F) / sinkG(j, c, G) once per phase; phases are separated by barriers.
 // scratch: [64][K] floats.  Ends with a barrier.
-template <typename SinkF, typename SinkG>
-__device__ void gated_products(const float* Wt, int ldw, const float* R, const float* Lm,
+__device__ __forceinline__ float ldf(const float* p) { return *p; }
+__device__ __forceinline__ float ldf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+template <typename TR, typename SinkF, typename SinkG>
+__device__ void gated_products(const float* Wt, int ldw, const TR* R, const TR* Lm,
                                const float* colw, const float* G2, int K, float* scratch,
                                SinkF sinkF, SinkG sinkG) {
   const int tid = threadIdx.x;
@@ -49,10 +53,10 @@ __device__ void gated_products(const float* Wt, int ldw, const float* R, const f
     const int i = x / K, c = x % K, b0 = (i / SUB) * SUB;
     const float gi = G2[x];
     float f = 0.f, g = 0.f;
-    for (int j = b0; j <= i; ++j) f += Wt[i * ldw + j] * R[j * K + c] * exp2f(gi - G2[j * K + c]);
+    for (int j = b0; j <= i; ++j) f += Wt[i * ldw + j] * ldf(R + j * K + c) * exp2f(gi - G2[j * K + c]);
     for (int r = i; r < b0 + SUB; ++r) {  // this row as the column index j = i
       const float wr = Wt[r * ldw + i] * (colw ? colw[r] : 1.f);
-      g += wr * Lm[r * K + c] * exp2f(G2[r * K + c] - gi);
+      g += wr * ldf(Lm + r * K + c) * exp2f(G2[r * K + c] - gi);
     }
     sinkF(i, c, f);
     sinkG(i, c, g);
@@ -64,11 +68,11 @@ __device__ void gated_products(const float* Wt, int ldw, const float* R, const f
     const int r = a * SUB - 1, nj = a * SUB;
     for (int x = tid; x < nj * K; x += blockDim.x) {
       const int c = x % K;
-      RT[x] = R[x] * exp2f(G2[r * K + c] - G2[x]);
+      RT[x] = ldf(R + x) * exp2f(G2[r * K + c] - G2[x]);
     }
     for (int x = tid; x < SUB * K; x += blockDim.x) {
       const int i = a * SUB + x / K, c = x % K;
-      Ls[x] = (colw ? colw[i] : 1.f) * Lm[i * K + c] * exp2f(G2[i * K + c] - G2[r * K + c]);
+      Ls[x] = (colw ? colw[i] : 1.f) * ldf(Lm + i * K + c) * exp2f(G2[i * K + c] - G2[r * K + c]);
     }
     __syncthreads();
     for (int x = tid; x < SUB * K; x += blockDim.x) {  // rows i of sub-chunk a
@@ -85,6 +89,91 @@ __device__ void gated_products(const float* Wt, int ldw, const float* R, const f
     }
     __syncthreads();
   }
+}
+
+// The same products for K = 128 and 256 threads, by channel: thread t owns channel c = t % 128,
+// with its operands in registers.  The diagonal sub-blocks: thread (c, t / 128) takes sub-chunks
+// 2 (t / 128) and 2 (t / 128) + 1, one exponential per pair (i, j) serving both F and G.  The
+// blocks below the diagonal, for each sub-chunk a through r = 16 a - 1: the threads t < 128 form
+// F of a's rows (16 independent accumulators, one pass over the columns j), the others G of the
+// columns before a; the two write disjoint rows of each channel.  The loops over j stay rolled
+// (a fully unrolled form overflows the instruction cache).  Results go to the sinks as above;
+// ends with a barrier.
+template <typename TR, typename SinkF, typename SinkG>
+__device__ __forceinline__ void gated_below(int A, const float* Wt, int ldw, const TR* R, const TR* Lm,
+                                            const float* colw, const float* G2, int c, bool rows,
+                                            SinkF& sinkF, SinkG& sinkG) {
+  constexpr int K = 128;
+  const int I0 = SUB * A, NJ = SUB * A;
+  const float gr = G2[(I0 - 1) * K + c];
+  if (rows) {  // F_i = e^{Gam_i - Gam_r} sum_{j < 16 A} Wt_ij R_j e^{Gam_r - Gam_j}, i in sub-chunk A
+    float acc[SUB];
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) acc[i] = 0.f;
+#pragma unroll 2
+    for (int j = 0; j < NJ; ++j) {
+      const float rt = ldf(R + j * K + c) * exp2f(gr - G2[j * K + c]);
+#pragma unroll
+      for (int i = 0; i < SUB; ++i) acc[i] = fmaf(Wt[(I0 + i) * ldw + j], rt, acc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) sinkF(I0 + i, c, acc[i] * exp2f(G2[(I0 + i) * K + c] - gr));
+  } else {     // G_j = e^{Gam_r - Gam_j} sum_{i in A} colw_i Wt_ij L_i e^{Gam_i - Gam_r}, j < 16 A
+    float ls[SUB];
+#pragma unroll
+    for (int i = 0; i < SUB; ++i)
+      ls[i] = (colw ? colw[I0 + i] : 1.f) * ldf(Lm + (I0 + i) * K + c) * exp2f(G2[(I0 + i) * K + c] - gr);
+#pragma unroll 2
+    for (int j = 0; j < NJ; ++j) {
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+      for (int i = 0; i < SUB; i += 4) {
+        a0 = fmaf(Wt[(I0 + i) * ldw + j], ls[i], a0);
+        a1 = fmaf(Wt[(I0 + i + 1) * ldw + j], ls[i + 1], a1);
+        a2 = fmaf(Wt[(I0 + i + 2) * ldw + j], ls[i + 2], a2);
+        a3 = fmaf(Wt[(I0 + i + 3) * ldw + j], ls[i + 3], a3);
+      }
+      sinkG(j, c, ((a0 + a1) + (a2 + a3)) * exp2f(gr - G2[j * K + c]));
+    }
+  }
+}
+
+template <typename TR, typename SinkF, typename SinkG>
+__device__ void gated_products_k128(const float* Wt, int ldw, const TR* R, const TR* Lm, const float* colw,
+                                    const float* G2, SinkF sinkF, SinkG sinkG) {
+  constexpr int K = 128;
+  const int c = threadIdx.x & 127, hi = threadIdx.x >> 7;
+#pragma unroll 1
+  for (int bb = 0; bb < 2; ++bb) {
+    const int b0 = SUB * (2 * hi + bb);
+    float g[SUB], r[SUB], l[SUB], F[SUB], G[SUB];
+#pragma unroll
+    for (int j = 0; j < SUB; ++j) {
+      g[j] = G2[(b0 + j) * K + c];
+      r[j] = ldf(R + (b0 + j) * K + c);
+      l[j] = (colw ? colw[b0 + j] : 1.f) * ldf(Lm + (b0 + j) * K + c);
+      F[j] = G[j] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < SUB; ++i)
+#pragma unroll
+      for (int j = 0; j <= i; ++j) {
+        const float wt = Wt[(b0 + i) * ldw + b0 + j] * exp2f(g[i] - g[j]);
+        F[i] = fmaf(wt, r[j], F[i]);
+        G[j] = fmaf(wt, l[i], G[j]);
+      }
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) {
+      sinkF(b0 + i, c, F[i]);
+      sinkG(b0 + i, c, G[i]);
+    }
+  }
+#pragma unroll 1
+  for (int A = 1; A < CH / SUB; ++A) {
+    __syncthreads();
+    gated_below(A, Wt, ldw, R, Lm, colw, G2, c, hi == 0, sinkF, sinkG);
+  }
+  __syncthreads();
 }
 
 // ---------------------------------------------------------------- reverse state scan
@@ -239,6 +328,325 @@ __global__ void __launch_bounds__(256) k_kda_bwd_dqk(Problem p, Args a, KdaWork 
                    dkp[j * K + c] += g;
                    dG[j * K + c] -= sK[j * K + c] * g;
                  });
+}
+
+// ---------------------------------------------------------------- output-side terms, tcgen05
+// The same unit's work with the four state-sized products on the tensor cores (bf16 inputs,
+// K = V = 128).  Operands are staged from the fp32 workspace as compensated bf16 pairs
+// (hi = bf16(x), lo = bf16(x - hi)) in 128-byte-swizzled tiles; dO is bf16 already and goes in
+// as one part.  Accumulators (TMEM, M = 64 tokens):
+//   [0, 64)    dP   = dO U^T         (dO.U_hi + dO.U_lo)
+//   [64, 192)  dQ~' = dO S           (dO.S_hi + dO.S_lo)           (before scale and e^{Gam})
+//   [192, 320) dW'  = dU S           (three of the four hi/lo products)
+//   [320, 448) dK^' = U dS'          (same)
+// dS' takes S's tiles once the first three products are done; the dP gated products and the
+// per-channel terms then run on CUDA cores as in k_kda_bwd_dqk.
+namespace kt {
+using namespace tcx;
+constexpr int TILE_T = 64 * 128;  // a [64 rows][64 bf16] block
+constexpr int TILE_S = 128 * 128; // a [128 rows][64 bf16] block
+constexpr int O_DO = 0, O_UH = 16384, O_UL = 32768, O_DUH = 49152, O_DUL = 65536;
+constexpr int O_SH = 81920, O_SL = 114688;                  // S, then dS' (hi, lo)
+// after the last product, over the tiles: the unit's dq, dk and dGam (fp32 [64][128] each,
+// accumulated in shared memory and written out once), q and k (bf16 [64][128], rows past the
+// chunk zero) and the gated products' scratch (fp32 [64][128])
+constexpr int O_ACQ = 0, O_ACK = 32768, O_ACG = 65536, O_QB = 98304, O_KB = 114688, O_SCR = 131072;
+constexpr int O_DP = 163840;                                // fp32 [64][LDP]
+constexpr int O_G = O_DP + CH * LDP * 4;                    // fp32 [64][128] Gam * log2(e)
+constexpr int O_RED = O_G + CH * 128 * 4;                   // fp32 [16][128]
+constexpr int O_GC = O_RED + 16 * 128 * 4;                  // fp32 [128]
+constexpr int DQK_BYTES = O_GC + 128 * 4;
+static_assert(O_SL + 32768 <= O_DP && O_SCR + 32768 <= O_DP, "tiles overlap the fp32 area");
+static_assert(1024 + DQK_BYTES <= 227 * 1024, "dqk shared memory");
+
+// rows [0, R) of an fp32 [R][128] matrix (row stride ld floats) as a hi/lo pair of sw128 tiles
+template <int R>
+__device__ __forceinline__ void stage_split(unsigned char* hi, unsigned char* lo, const float* src, size_t ld) {
+  constexpr int N = R * 16 / 256;  // 16-byte chunks of 8 floats per thread
+  float4 r[2 * N];
+#pragma unroll
+  for (int m = 0; m < N; ++m) {
+    const int x = threadIdx.x + 256 * m, row = x >> 4, j = x & 15;
+    const float4* p = reinterpret_cast<const float4*>(src + row * ld + 8 * j);
+    r[2 * m] = __ldg(p);
+    r[2 * m + 1] = __ldg(p + 1);
+  }
+#pragma unroll
+  for (int m = 0; m < N; ++m) {
+    const int x = threadIdx.x + 256 * m, row = x >> 4, j = x & 15;
+    const float f[8] = {r[2 * m].x, r[2 * m].y, r[2 * m].z, r[2 * m].w,
+                        r[2 * m + 1].x, r[2 * m + 1].y, r[2 * m + 1].z, r[2 * m + 1].w};
+    st_chunk_split(hi, lo, row, j, R * 128, f);
+  }
+}
+// two such matrices with all loads issued before the first store
+template <int R>
+__device__ __forceinline__ void stage_split2(unsigned char* hi0, unsigned char* lo0, const float* src0,
+                                             unsigned char* hi1, unsigned char* lo1, const float* src1, size_t ld) {
+  constexpr int N = R * 16 / 256;
+  float4 r[4 * N];
+#pragma unroll
+  for (int m = 0; m < N; ++m) {
+    const int x = threadIdx.x + 256 * m, row = x >> 4, j = x & 15;
+    const float4* p0 = reinterpret_cast<const float4*>(src0 + row * ld + 8 * j);
+    const float4* p1 = reinterpret_cast<const float4*>(src1 + row * ld + 8 * j);
+    r[4 * m] = __ldg(p0);
+    r[4 * m + 1] = __ldg(p0 + 1);
+    r[4 * m + 2] = __ldg(p1);
+    r[4 * m + 3] = __ldg(p1 + 1);
+  }
+#pragma unroll
+  for (int m = 0; m < N; ++m) {
+    const int x = threadIdx.x + 256 * m, row = x >> 4, j = x & 15;
+    const float f0[8] = {r[4 * m].x, r[4 * m].y, r[4 * m].z, r[4 * m].w,
+                         r[4 * m + 1].x, r[4 * m + 1].y, r[4 * m + 1].z, r[4 * m + 1].w};
+    const float f1[8] = {r[4 * m + 2].x, r[4 * m + 2].y, r[4 * m + 2].z, r[4 * m + 2].w,
+                         r[4 * m + 3].x, r[4 * m + 3].y, r[4 * m + 3].z, r[4 * m + 3].w};
+    st_chunk_split(hi0, lo0, row, j, R * 128, f0);
+    st_chunk_split(hi1, lo1, row, j, R * 128, f1);
+  }
+}
+}  // namespace kt
+
+__global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, KdaWork w) {
+  using namespace kt;
+  if (kda_failed(w)) return;
+  const int gc = blockIdx.x, hv = blockIdx.y;
+  const int4 e = w.chunk_tab[gc];
+  if (e.x < 0) return;
+  constexpr int K = 128, V = 128;
+  const int L = e.z, tok0 = e.w, hk = hv / p.G, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  extern __shared__ unsigned char smraw[];
+  unsigned char* sm = align1k(smraw);
+  float* sdP = reinterpret_cast<float*>(sm + O_DP);
+  float* sG = reinterpret_cast<float*>(sm + O_G);
+  float* sred = reinterpret_cast<float*>(sm + O_RED);
+  float* sGC = reinterpret_cast<float*>(sm + O_GC);
+  __shared__ uint64_t bar[2];
+  __shared__ uint32_t tslot;
+  int* err = w.status;
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tslot, 512);
+    tmem_relinquish();
+  }
+  const size_t u = (size_t)gc * p.HV + hv, uk = u * CH * K;
+  {  // dO rows [0, L) (bf16, zero past L), U, dU, S; Gam
+    const bf16* dO = static_cast<const bf16*>(a.dO) + ((size_t)tok0 * p.HV + hv) * V;
+    uint4 r[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+      r[m] = row < L ? __ldg(reinterpret_cast<const uint4*>(dO + (size_t)row * p.HV * V + 8 * j))
+                     : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+      *reinterpret_cast<uint4*>(sm + O_DO + sw128_chunk(row, j, TILE_T)) = r[m];
+    }
+  }
+  stage_split2<CH>(sm + O_UH, sm + O_UL, w.U + u * CH * V, sm + O_DUH, sm + O_DUL, w.dU + u * CH * V, V);
+  stage_split<128>(sm + O_SH, sm + O_SL, w.h + u * V * K, K);
+  copy_async(sG, w.Gam + uk, CH * K);
+  cp_async_wait_all();
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tslot;
+  const uint32_t aDO = smem_u32(sm + O_DO), aUH = smem_u32(sm + O_UH), aUL = smem_u32(sm + O_UL);
+  const uint32_t aDUH = smem_u32(sm + O_DUH), aDUL = smem_u32(sm + O_DUL);
+  const uint32_t aSH = smem_u32(sm + O_SH), aSL = smem_u32(sm + O_SL);
+  if (tid == 0) {
+    constexpr uint32_t i64 = idesc_bf16(64, 64, false, false), i128 = idesc_bf16(64, 128, false, true);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint64_t dO_ = desc_kmajor(aDO, s, TILE_T);
+      mma_bf16(taddr(tb, 0, 0), dO_, desc_kmajor(aUH, s, TILE_T), i64, s > 0);
+      mma_bf16(taddr(tb, 0, 0), dO_, desc_kmajor(aUL, s, TILE_T), i64, 1);
+      const uint64_t sh = desc_mnmajor(aSH, s, TILE_S), sl = desc_mnmajor(aSL, s, TILE_S);
+      mma_bf16(taddr(tb, 0, 64), dO_, sh, i128, s > 0);
+      mma_bf16(taddr(tb, 0, 64), dO_, sl, i128, 1);
+      const uint64_t duh = desc_kmajor(aDUH, s, TILE_T);
+      mma_bf16(taddr(tb, 0, 192), duh, sh, i128, s > 0);
+      mma_bf16(taddr(tb, 0, 192), duh, sl, i128, 1);
+      mma_bf16(taddr(tb, 0, 192), desc_kmajor(aDUL, s, TILE_T), sh, i128, 1);
+    }
+    mma_commit(&bar[0]);
+  }
+  // dS' (leaving the chunk) into registers while the products run
+  const float* dSn = w.dh + u * V * K;
+  float4 rd[16];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+    const float4* p4 = reinterpret_cast<const float4*>(dSn + (size_t)row * K + 8 * j);
+    rd[2 * m] = __ldg(p4);
+    rd[2 * m + 1] = __ldg(p4 + 1);
+  }
+  bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
+  tc_fence_after();
+  {  // colsum(dS' * S) (S = hi + lo) over this thread's rows, then dS' over S's tiles
+    float cs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const int j = tid & 15;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int row = (tid >> 4) + 16 * m;
+      float h[8], l[8];
+      ld_chunk_f(sm + O_SH, row, j, TILE_S, h);
+      ld_chunk_f(sm + O_SL, row, j, TILE_S, l);
+      const float f[8] = {rd[2 * m].x, rd[2 * m].y, rd[2 * m].z, rd[2 * m].w,
+                          rd[2 * m + 1].x, rd[2 * m + 1].y, rd[2 * m + 1].z, rd[2 * m + 1].w};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) cs[q] = fmaf(f[q], h[q] + l[q], cs[q]);
+      st_chunk_split(sm + O_SH, sm + O_SL, row, j, TILE_S, f);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) sred[(tid >> 4) * 128 + 8 * j + q] = cs[q];
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (ok && tid == 0) {
+    constexpr uint32_t i128 = idesc_bf16(64, 128, false, true);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint64_t uh = desc_kmajor(aUH, s, TILE_T);
+      const uint64_t sh = desc_mnmajor(aSH, s, TILE_S);
+      mma_bf16(taddr(tb, 0, 320), uh, sh, i128, s > 0);
+      mma_bf16(taddr(tb, 0, 320), uh, desc_mnmajor(aSL, s, TILE_S), i128, 1);
+      mma_bf16(taddr(tb, 0, 320), desc_kmajor(aUL, s, TILE_T), sh, i128, 1);
+    }
+    mma_commit(&bar[1]);
+  }
+  if (tid < K) {  // e^{Gam_C} colsum(dS' * S), part of dL/dGam_C
+    float t = 0.f;
+    for (int q = 0; q < 16; ++q) t += sred[q * 128 + tid];
+    sGC[tid] = exp2f(sG[(CH - 1) * K + tid]) * t;
+  }
+  // M = 64 accumulators, 16-lane loads: rows r0 and r0 + 8, columns 8j + cq + {0, 1} of this
+  // warp half's range
+  const int half = warp >> 2, sub = 32 * (warp & 3), r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
+  if (ok) {
+    float d[16];
+    tmem_ld16dp_x4(taddr(tb, sub, 32 * half), d);  // dP, columns [32 half, +32)
+    float x[32];
+    tmem_ld16dp_x8(taddr(tb, sub, 192 + 64 * half), x);  // dW', columns [64 half, +64)
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = r0 + 8 * (q >> 1), c = 32 * half + 8 * j + cq + (q & 1);
+        sdP[i * LDP + c] = c <= i ? p.scale * d[4 * j + q] : 0.f;
+      }
+    float* dW = w.dW + uk;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = 64 * half + 8 * j + cq;
+      *reinterpret_cast<float2*>(dW + r0 * K + c) = make_float2(-x[4 * j], -x[4 * j + 1]);
+      *reinterpret_cast<float2*>(dW + (r0 + 8) * K + c) = make_float2(-x[4 * j + 2], -x[4 * j + 3]);
+    }
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
+  tc_fence_after();
+  bf16* sQ = reinterpret_cast<bf16*>(sm + O_QB);
+  bf16* sK = reinterpret_cast<bf16*>(sm + O_KB);
+  float* acq = reinterpret_cast<float*>(sm + O_ACQ);
+  float* ack = reinterpret_cast<float*>(sm + O_ACK);
+  float* acg = reinterpret_cast<float*>(sm + O_ACG);
+  {  // q and k rows [0, L) as bf16, zero past L
+    const size_t rs = (size_t)p.H * K;
+    const bf16* gq = static_cast<const bf16*>(a.q) + ((size_t)tok0 * p.H + hk) * K;
+    const bf16* gk = static_cast<const bf16*>(a.k) + ((size_t)tok0 * p.H + hk) * K;
+    uint4 rq[4], rk[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+      rq[m] = rk[m] = make_uint4(0u, 0u, 0u, 0u);
+      if (row < L) {
+        rq[m] = __ldg(reinterpret_cast<const uint4*>(gq + row * rs + 8 * j));
+        rk[m] = __ldg(reinterpret_cast<const uint4*>(gk + row * rs + 8 * j));
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int x = tid + 256 * m;
+      reinterpret_cast<uint4*>(sQ)[x] = rq[m];
+      reinterpret_cast<uint4*>(sK)[x] = rk[m];
+    }
+  }
+  __syncthreads();
+  if (ok) {  // dQ~ e^{Gam}, dK^ e^{Gam_C - Gam}, dGam; colsum(dK^ * K^) per column
+    float x[32], y[32];
+    tmem_ld16dp_x8(taddr(tb, sub, 64 + 64 * half), x);
+    tmem_ld16dp_x8(taddr(tb, sub, 320 + 64 * half), y);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float cs[2];
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const int c = 64 * half + 8 * j + cq + b;
+        const float gC = sG[(CH - 1) * K + c];
+        float t = 0.f;
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int i = r0 + 8 * hr, o = i * K + c;
+          const float g = sG[o], eg = exp2f(g), kh = exp2f(gC - g);
+          const float dqt = p.scale * x[4 * j + 2 * hr + b], dkh = y[4 * j + 2 * hr + b];
+          const float kk = __bfloat162float(sK[o]);
+          acq[o] = dqt * eg;
+          ack[o] = dkh * kh;
+          acg[o] = dqt * __bfloat162float(sQ[o]) * eg - dkh * kk * kh;
+          t = fmaf(dkh * kk, kh, t);
+        }
+        t += __shfl_xor_sync(0xffffffffu, t, 4);
+        t += __shfl_xor_sync(0xffffffffu, t, 8);
+        t += __shfl_xor_sync(0xffffffffu, t, 16);
+        cs[b] = t;
+      }
+      if (lane < 4) {
+        const int c = 64 * half + 8 * j + cq;
+        sred[(warp & 3) * 128 + c] = cs[0];
+        sred[(warp & 3) * 128 + c + 1] = cs[1];
+      }
+    }
+  }
+  __syncthreads();
+  if (ok && tid < K)  // the last row collects dL/dGam_C
+    acg[(CH - 1) * K + tid] += sGC[tid] + sred[tid] + sred[128 + tid] + sred[256 + tid] + sred[384 + tid];
+  __syncthreads();
+  if (ok)  // P_ij = sum_c q_i k_j e^{Gam_i - Gam_j}: dq += F2, dk += G2, dGam += q F2 - k G2
+    gated_products_k128(sdP, LDP, sK, sQ, nullptr, sG,
+                   [&](int i, int c, float f) {
+                     acq[i * K + c] += f;
+                     acg[i * K + c] += __bfloat162float(sQ[i * K + c]) * f;
+                   },
+                   [&](int j, int c, float g) {
+                     ack[j * K + c] += g;
+                     acg[j * K + c] -= __bfloat162float(sK[j * K + c]) * g;
+                   });
+  if (ok) {  // the unit's dq and dk shares and dGam (gated_products ends with a barrier)
+    float4* dq4 = reinterpret_cast<float4*>(w.dqp + uk);
+    float4* dk4 = reinterpret_cast<float4*>(w.dkp + uk);
+    float4* dg4 = reinterpret_cast<float4*>(w.dGam + uk);
+    for (int x = tid; x < CH * K / 4; x += 256) {
+      dq4[x] = reinterpret_cast<const float4*>(acq)[x];
+      dk4[x] = reinterpret_cast<const float4*>(ack)[x];
+      dg4[x] = reinterpret_cast<const float4*>(acg)[x];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 512);
 }
 
 // ---------------------------------------------------------------- WY backward, gate chain
@@ -432,11 +840,18 @@ cudaError_t go(const char* name, Kern kern, dim3 grid, size_t smem, cudaStream_t
   return cudaGetLastError();
 }
 
+// bf16 with 128-wide key and value heads runs the tensor-core kernels
+template <typename T>
+bool kda_tc(const Problem& p) {
+  return std::is_same<T, __nv_bfloat16>::value && p.K == 128 && p.V == 128;
+}
+
 template <typename T>
 cudaError_t backward_t(const Problem& p, const Args& a, const KdaWork& w, cudaStream_t s) {
   cudaError_t e = go("kda_bwd_scan", k_kda_bwd_scan<T>, dim3(p.Nst, p.HV, p.V / 32), scan_smem(p.K), s, p, a, w);
   if (e == cudaSuccess)
-    e = go("kda_bwd_dqk", k_kda_bwd_dqk<T>, dim3(p.NCmax, p.HV), dqk_smem(p.K, p.V), s, p, a, w);
+    e = kda_tc<T>(p) ? go("kda_tc_bwd_dqk", k_kda_tc_bwd_dqk, dim3(p.NCmax, p.HV), 1024 + kt::DQK_BYTES, s, p, a, w)
+                     : go("kda_bwd_dqk", k_kda_bwd_dqk<T>, dim3(p.NCmax, p.HV), dqk_smem(p.K, p.V), s, p, a, w);
   if (e == cudaSuccess)
     e = go("kda_bwd_wy", k_kda_bwd_wy<T>, dim3(p.NCmax, p.HV), wy_smem(p.K, p.V), s, p, a, w);
   if (e != cudaSuccess) return e;

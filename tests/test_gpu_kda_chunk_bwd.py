@@ -122,3 +122,21 @@ def test_empty_input_passes_the_gradient_through():
     torch.cuda.synchronize()
     assert torch.equal(ht.cpu(), case.h0) and torch.equal(out["dh0"].cpu(), case.dht)
     assert torch.all(out["dA_log"] == 0) and torch.all(out["ddt_bias"] == 0)
+
+
+def test_bf16_128_runs_the_tensor_core_kernels():
+    """bf16 with 128-wide heads takes the tcgen05 KDA kernels (the per-launch profile names
+    them) and still matches the oracle; fp32 and 64-wide heads keep the CUDA-core kernels."""
+    import gated_deltanet_chunkwise_chunk_b200 as gdn
+    case = synth.make_case(H=2, HV=4, K=128, V=128, dtype="bf16", seed=670,
+                           lengths=[130, 0, 64, 5], h0=True, name="kda_tc_path")
+    gdn.profile(True)
+    try:
+        _run(case, seed=671)
+        torch.cuda.synchronize()
+        names = set(gdn.profile_read())
+    finally:
+        gdn.profile(False)
+    for k in ("kda_tc_bwd_dqk",):
+        assert k in names, (k, names)
+    assert "kda_bwd_dqk" not in names, names
