@@ -803,6 +803,351 @@ __global__ void __launch_bounds__(256) k_kda_bwd_wy(Problem p, Args a, KdaWork w
   }
 }
 
+// ---------------------------------------------------------------- WY backward, tcgen05
+// k_kda_bwd_wy's work for bf16 with K = V = 128, the five products on the tensor cores from
+// compensated bf16 pairs (V is bf16 already).  With X' = k e^{Gam} (X = diag(beta) X'):
+//   [0, 64)    dT = (dW X'^T + dU V^T) diag(beta)     (beta applied to the columns on the way out)
+//   [64, 192)  dX = T^T dW,   [192, 320) dY = T^T dU
+//   [320, 384) Z = dT T^T,    [384, 448) -dA = T^T Z
+// The dk share and dGam of the unit (from k_kda_tc_bwd_dqk) are read into shared memory,
+// collect this kernel's terms there, and dGam goes through the reverse cumsum and the gate
+// chain from there; the dA gated products run by channel.
+namespace kw {
+using namespace tcx;
+constexpr int TT = 64 * 128;                          // [64 rows][64 bf16] block
+// fixed: Gam (fp32), k (bf16 row-major), V (bf16 tile), small vectors
+constexpr int O_G = 0, O_K = 32768, O_V = 49152, O_VEC = 65536;   // vectors: 2 KB
+// region A: dW, dU, X' (hi, lo); after the first products: dk, dGam, F1 (fp32 [64][128] each),
+// F1 giving way to the raw gate inputs once its terms are in
+constexpr int O_A = 67584;
+constexpr int O_DWH = O_A, O_DWL = O_A + 16384, O_DUH = O_A + 32768, O_DUL = O_A + 49152;
+constexpr int O_XH = O_A + 65536, O_XL = O_A + 81920;
+constexpr int O_ACK = O_A, O_ACG = O_A + 32768, O_F1 = O_A + 65536;
+// region B: T, dT, Z (hi, lo [64][64] each); after the last product: dA (fp32 [64][LDP])
+constexpr int O_B = O_A + 98304;
+constexpr int O_TH = O_B, O_TL = O_B + 8192, O_DTH = O_B + 16384, O_DTL = O_B + 24576;
+constexpr int O_ZH = O_B + 32768, O_ZL = O_B + 40960;
+constexpr int O_DA = O_B;
+constexpr int WY_BYTES = O_B + 49152;
+static_assert(CH * LDP * 4 <= 49152, "dA fits region B");
+static_assert(1024 + WY_BYTES <= 227 * 1024, "wy_bwd shared memory");
+}  // namespace kw
+
+__global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_wy(Problem p, Args a, KdaWork w) {
+  using namespace kw;
+  if (kda_failed(w)) return;
+  const int gc = blockIdx.x, hv = blockIdx.y;
+  const int4 e = w.chunk_tab[gc];
+  if (e.x < 0) return;
+  constexpr int K = 128, V = 128;
+  const int L = e.z, tok0 = e.w, hk = hv / p.G, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nwarp = 8;
+  extern __shared__ unsigned char smraw[];
+  unsigned char* sm = align1k(smraw);
+  float* sG = reinterpret_cast<float*>(sm + O_G);
+  bf16* sK = reinterpret_cast<bf16*>(sm + O_K);
+  float* sb = reinterpret_cast<float*>(sm + O_VEC);   // [64] beta, 0 past L
+  float* sdb = sb + 64;                                // [64] dbeta
+  float* sdbp = sb + 128;                              // [2][64] dbeta halves
+  float* sred = sb + 256;                              // [2][128]
+  float* ack = reinterpret_cast<float*>(sm + O_ACK);
+  float* acg = reinterpret_cast<float*>(sm + O_ACG);
+  float* sF1 = reinterpret_cast<float*>(sm + O_F1);
+  float* sdA = reinterpret_cast<float*>(sm + O_DA);
+  __shared__ uint64_t bar[3];
+  __shared__ uint32_t tslot;
+  int* err = w.status;
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_init(&bar[2], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tslot, 512);
+    tmem_relinquish();
+  }
+  const size_t u = (size_t)gc * p.HV + hv, uk = u * CH * K;
+  {  // k (row-major) and V (swizzled tile), rows past L zero; beta
+    const bf16* gk = static_cast<const bf16*>(a.k) + ((size_t)tok0 * p.H + hk) * K;
+    const bf16* gv = static_cast<const bf16*>(a.v) + ((size_t)tok0 * p.HV + hv) * V;
+    uint4 rk[4], rv[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+      rk[m] = rv[m] = make_uint4(0u, 0u, 0u, 0u);
+      if (row < L) {
+        rk[m] = __ldg(reinterpret_cast<const uint4*>(gk + (size_t)row * p.H * K + 8 * j));
+        rv[m] = __ldg(reinterpret_cast<const uint4*>(gv + (size_t)row * p.HV * V + 8 * j));
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+      reinterpret_cast<uint4*>(sK)[x] = rk[m];
+      *reinterpret_cast<uint4*>(sm + O_V + sw128_chunk(row, j, TT)) = rv[m];
+    }
+    if (tid < CH) sb[tid] = tid < L ? a.beta[(size_t)(tok0 + tid) * p.HV + hv] : 0.f;
+  }
+  copy_async(sG, w.Gam + uk, CH * K);
+  kt::stage_split2<CH>(sm + O_DWH, sm + O_DWL, w.dW + uk, sm + O_DUH, sm + O_DUL, w.dU + u * CH * V, K);
+  {  // T (fp32 [64][64]) as a hi/lo pair of one-block tiles
+    float4 r[4];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int x = tid + 256 * m, row = x >> 3, j = x & 7;
+      const float4* p4 = reinterpret_cast<const float4*>(w.Tm + u * CH * CH + row * CH + 8 * j);
+      r[2 * m] = __ldg(p4);
+      r[2 * m + 1] = __ldg(p4 + 1);
+    }
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int x = tid + 256 * m, row = x >> 3, j = x & 7;
+      const float f[8] = {r[2 * m].x, r[2 * m].y, r[2 * m].z, r[2 * m].w,
+                          r[2 * m + 1].x, r[2 * m + 1].y, r[2 * m + 1].z, r[2 * m + 1].w};
+      st_chunk_split(sm + O_TH, sm + O_TL, row, j, TT, f);
+    }
+  }
+  cp_async_wait_all();
+  __syncthreads();
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {  // X' = k e^{Gam}
+    const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+    float f[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int o = row * K + 8 * j + q;
+      f[q] = __bfloat162float(sK[o]) * exp2f(sG[o]);
+    }
+    st_chunk_split(sm + O_XH, sm + O_XL, row, j, TT, f);
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tslot;
+  const uint32_t aDWH = smem_u32(sm + O_DWH), aDWL = smem_u32(sm + O_DWL), aDUH = smem_u32(sm + O_DUH);
+  const uint32_t aDUL = smem_u32(sm + O_DUL), aXH = smem_u32(sm + O_XH), aXL = smem_u32(sm + O_XL);
+  const uint32_t aV = smem_u32(sm + O_V), aTH = smem_u32(sm + O_TH), aTL = smem_u32(sm + O_TL);
+  if (tid == 0) {
+    constexpr uint32_t i64 = idesc_bf16(64, 64, false, false), i128 = idesc_bf16(64, 128, true, true);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {  // dT (before beta)
+      const uint64_t dwh = desc_kmajor(aDWH, s, TT), xh = desc_kmajor(aXH, s, TT);
+      mma_bf16(taddr(tb, 0, 0), dwh, xh, i64, s > 0);
+      mma_bf16(taddr(tb, 0, 0), dwh, desc_kmajor(aXL, s, TT), i64, 1);
+      mma_bf16(taddr(tb, 0, 0), desc_kmajor(aDWL, s, TT), xh, i64, 1);
+      const uint64_t vv = desc_kmajor(aV, s, TT);
+      mma_bf16(taddr(tb, 0, 0), desc_kmajor(aDUH, s, TT), vv, i64, 1);
+      mma_bf16(taddr(tb, 0, 0), desc_kmajor(aDUL, s, TT), vv, i64, 1);
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {  // dX = T^T dW, dY = T^T dU
+      const uint64_t th = desc_mnmajor(aTH, s, TT), tl = desc_mnmajor(aTL, s, TT);
+      const uint64_t dwh = desc_mnmajor(aDWH, s, TT), duh = desc_mnmajor(aDUH, s, TT);
+      mma_bf16(taddr(tb, 0, 64), th, dwh, i128, s > 0);
+      mma_bf16(taddr(tb, 0, 64), th, desc_mnmajor(aDWL, s, TT), i128, 1);
+      mma_bf16(taddr(tb, 0, 64), tl, dwh, i128, 1);
+      mma_bf16(taddr(tb, 0, 192), th, duh, i128, s > 0);
+      mma_bf16(taddr(tb, 0, 192), th, desc_mnmajor(aDUL, s, TT), i128, 1);
+      mma_bf16(taddr(tb, 0, 192), tl, duh, i128, 1);
+    }
+    mma_commit(&bar[0]);
+  }
+  const int half = warp >> 2, sub = 32 * (warp & 3), r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
+  bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
+  tc_fence_after();
+  if (ok) {  // dT diag(beta) as a hi/lo tile
+    float d[16];
+    tmem_ld16dp_x4(taddr(tb, sub, 32 * half), d);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = 32 * half + 8 * j + cq;
+      const float b0 = sb[c], b1 = sb[c + 1];
+      st_pair_split(sm + O_DTH, sm + O_DTL, r0, c, TT, d[4 * j] * b0, d[4 * j + 1] * b1);
+      st_pair_split(sm + O_DTH, sm + O_DTL, r0 + 8, c, TT, d[4 * j + 2] * b0, d[4 * j + 3] * b1);
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t aDTH = smem_u32(sm + O_DTH), aDTL = smem_u32(sm + O_DTL);
+  if (ok && tid == 0) {  // Z = dT T^T
+    constexpr uint32_t i64 = idesc_bf16(64, 64, false, false);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const uint64_t dth = desc_kmajor(aDTH, s, TT), th = desc_kmajor(aTH, s, TT);
+      mma_bf16(taddr(tb, 0, 320), dth, th, i64, s > 0);
+      mma_bf16(taddr(tb, 0, 320), dth, desc_kmajor(aTL, s, TT), i64, 1);
+      mma_bf16(taddr(tb, 0, 320), desc_kmajor(aDTL, s, TT), th, i64, 1);
+    }
+    mma_commit(&bar[1]);
+  }
+  // region A is free: the unit's dk share and dGam from the output-side kernel
+  {
+    const float4* k4 = reinterpret_cast<const float4*>(w.dkp + uk);
+    const float4* g4 = reinterpret_cast<const float4*>(w.dGam + uk);
+    for (int x = tid; x < CH * K / 4; x += 256) {
+      reinterpret_cast<float4*>(ack)[x] = __ldg(k4 + x);
+      reinterpret_cast<float4*>(acg)[x] = __ldg(g4 + x);
+      reinterpret_cast<float4*>(sF1)[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  __syncthreads();
+  if (ok) {  // dv = beta dY; dbeta = rowsum(dY V) + rowsum(dX k e^{Gam}); dk, dGam += beta dX e^{Gam} (1, k)
+    float x[32], y[32];
+    tmem_ld16dp_x8(taddr(tb, sub, 64 + 64 * half), x);
+    tmem_ld16dp_x8(taddr(tb, sub, 192 + 64 * half), y);
+    tmem_wait_ld();
+    bf16* dv = static_cast<bf16*>(a.dv) + ((size_t)tok0 * p.HV + hv) * V;
+    float rs[2] = {0.f, 0.f};
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int i = r0 + 8 * hr;
+      const float bi = sb[i];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = 64 * half + 8 * j + cq;
+        const float y0 = y[4 * j + 2 * hr], y1 = y[4 * j + 2 * hr + 1];
+        const float2 vv = ld_pair(sm + O_V, i, c, TT);
+        rs[hr] += y0 * vv.x + y1 * vv.y;
+        if (i < L) *reinterpret_cast<uint32_t*>(dv + (size_t)i * p.HV * V + c) = pack_bf16(bi * y0, bi * y1);
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          const int o = i * K + c + b;
+          const float eg = exp2f(sG[o]), dx = x[4 * j + 2 * hr + b], kt = __bfloat162float(sK[o]) * eg;
+          rs[hr] = fmaf(dx, kt, rs[hr]);
+          ack[o] = fmaf(bi * dx, eg, ack[o]);
+          acg[o] = fmaf(bi * dx, kt, acg[o]);
+        }
+      }
+    }
+    rs[0] = quad_sum(rs[0]);
+    rs[1] = quad_sum(rs[1]);
+    if ((lane & 3) == 0) {
+      sdbp[half * 64 + r0] = rs[0];
+      sdbp[half * 64 + r0 + 8] = rs[1];
+    }
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
+  tc_fence_after();
+  if (tid < CH) sdb[tid] = sdbp[tid] + sdbp[64 + tid];
+  if (ok) {  // Z as a hi/lo tile
+    float d[16];
+    tmem_ld16dp_x4(taddr(tb, sub, 320 + 32 * half), d);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = 32 * half + 8 * j + cq;
+      st_pair_split(sm + O_ZH, sm + O_ZL, r0, c, TT, d[4 * j], d[4 * j + 1]);
+      st_pair_split(sm + O_ZH, sm + O_ZL, r0 + 8, c, TT, d[4 * j + 2], d[4 * j + 3]);
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (ok && tid == 0) {  // T^T Z
+    constexpr uint32_t i64 = idesc_bf16(64, 64, true, true);
+    const uint32_t aZH = smem_u32(sm + O_ZH), aZL = smem_u32(sm + O_ZL);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const uint64_t th = desc_mnmajor(aTH, s, TT), zh = desc_mnmajor(aZH, s, TT);
+      mma_bf16(taddr(tb, 0, 384), th, zh, i64, s > 0);
+      mma_bf16(taddr(tb, 0, 384), th, desc_mnmajor(aZL, s, TT), i64, 1);
+      mma_bf16(taddr(tb, 0, 384), desc_mnmajor(aTL, s, TT), zh, i64, 1);
+    }
+    mma_commit(&bar[2]);
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[2], 0, err));
+  tc_fence_after();
+  if (ok) {  // dA = -T^T Z, strictly lower, over region B
+    float d[16];
+    tmem_ld16dp_x4(taddr(tb, sub, 384 + 32 * half), d);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = r0 + 8 * (q >> 1), c = 32 * half + 8 * j + cq + (q & 1);
+        sdA[i * LDP + c] = c < i ? -d[4 * j + q] : 0.f;
+      }
+  }
+  __syncthreads();
+  // A_ij = beta_i sum_c k_i k_j e^{Gam_i - Gam_j}: F1 (rows, weights dA), G1 (columns, beta_i dA)
+  if (ok)
+    gated_products_k128(sdA, LDP, sK, sK, sb, sG,
+                        [&](int i, int c, float f) { sF1[i * K + c] += f; },
+                        [&](int j, int c, float g) {
+                          ack[j * K + c] += g;
+                          acg[j * K + c] -= __bfloat162float(sK[j * K + c]) * g;
+                        });
+  // F1 terms: dk += beta F1, dGam += beta k F1, dbeta += rowsum(k F1)
+  for (int i = warp; i < CH; i += nwarp) {
+    float sacc = 0.f;
+    for (int c = lane; c < K; c += 32) {
+      const int o = i * K + c;
+      const float f = sF1[o], kk = __bfloat162float(sK[o]);
+      sacc += kk * f;
+      ack[o] += sb[i] * f;
+      acg[o] += sb[i] * kk * f;
+    }
+    for (int off = 16; off > 0; off >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, off);
+    if (ok && lane == 0 && i < L) a.dbeta[(size_t)(tok0 + i) * p.HV + hv] = sdb[i] + sacc;
+  }
+  __syncthreads();
+  float* sg = sF1;  // F1 is done: the raw gate inputs
+  load_tile<float>(sg, K, a.g_raw + ((size_t)tok0 * p.HV + hv) * K, (size_t)p.HV * K, L, K);
+  {
+    float4* dk4 = reinterpret_cast<float4*>(w.dkp + uk);
+    for (int x = tid; x < CH * K / 4; x += 256) dk4[x] = reinterpret_cast<const float4*>(ack)[x];
+  }
+  __syncthreads();
+  // dyg = reverse in-chunk cumsum of dGam: two row halves, the lower offset by the upper's sum
+  const int part = tid / K, cc = tid % K, rows = CH / 2;
+  {
+    float t = 0.f;
+    for (int i = part * rows; i < (part + 1) * rows; ++i) t += acg[i * K + cc];
+    sred[part * K + cc] = t;
+  }
+  __syncthreads();
+  const float nexp = -expf(a.A_log[hv]);
+  const float bias = a.dt_bias ? a.dt_bias[(size_t)hv * K + cc] : 0.f;
+  float acc = part == 0 ? sred[K + cc] : 0.f, pA = 0.f, pB = 0.f;
+  for (int i = (part + 1) * rows - 1; i >= part * rows; --i) {
+    acc += acg[i * K + cc];
+    if (i < L) {
+      const size_t o = ((size_t)(tok0 + i) * p.HV + hv) * K + cc;
+      const float xg = sg[i * K + cc] + bias;
+      const float sp = xg > 20.f ? xg : log1pf(expf(xg));
+      const float sig = xg > 20.f ? 1.f : 1.f / (1.f + expf(-xg));
+      const float dgr = acc * nexp * sig;
+      a.dg[o] = acc;
+      if (a.dg_raw) a.dg_raw[o] = dgr;
+      pA += acc * nexp * sp;
+      pB += dgr;
+    }
+  }
+  __syncthreads();
+  sred[part * K + cc] = pB;
+  for (int off = 16; off > 0; off >>= 1) pA += __shfl_xor_sync(0xffffffffu, pA, off);
+  if (lane == 0) sdb[warp] = pA;
+  __syncthreads();
+  float* pg = w.pgp + u * (K + 1);
+  if (tid < K) pg[tid] = sred[tid] + sred[K + tid];
+  if (tid == 0) {
+    float t = 0.f;
+    for (int q = 0; q < nwarp; ++q) t += sdb[q];
+    pg[K] = t;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 512);
+}
+
 // dA_log[hv] and ddt_bias[hv*K + c]: the per-chunk sums added in chunk order.
 __global__ void __launch_bounds__(256) k_kda_param_grads(Problem p, Args a, KdaWork w) {
   if (kda_failed(w)) return;
@@ -853,7 +1198,8 @@ cudaError_t backward_t(const Problem& p, const Args& a, const KdaWork& w, cudaSt
     e = kda_tc<T>(p) ? go("kda_tc_bwd_dqk", k_kda_tc_bwd_dqk, dim3(p.NCmax, p.HV), 1024 + kt::DQK_BYTES, s, p, a, w)
                      : go("kda_bwd_dqk", k_kda_bwd_dqk<T>, dim3(p.NCmax, p.HV), dqk_smem(p.K, p.V), s, p, a, w);
   if (e == cudaSuccess)
-    e = go("kda_bwd_wy", k_kda_bwd_wy<T>, dim3(p.NCmax, p.HV), wy_smem(p.K, p.V), s, p, a, w);
+    e = kda_tc<T>(p) ? go("kda_tc_bwd_wy", k_kda_tc_bwd_wy, dim3(p.NCmax, p.HV), 1024 + kw::WY_BYTES, s, p, a, w)
+                     : go("kda_bwd_wy", k_kda_bwd_wy<T>, dim3(p.NCmax, p.HV), wy_smem(p.K, p.V), s, p, a, w);
   if (e != cudaSuccess) return e;
   Work gw{};  // the group sum's view of the shares
   gw.status = w.status;
