@@ -22,6 +22,8 @@
 // Three kernels: k_kda_wy per (chunk, value head) builds everything chunk-local; k_kda_scan per
 // (sequence, value head, 32-row slice of S) carries the state through the chunks; k_kda_out per
 // (chunk, value head) forms the output.
+#include <type_traits>
+
 #include "ffma_tiles.cuh"
 #include "gdn_common.cuh"
 #include "gdn_launch.h"
@@ -185,6 +187,310 @@ __global__ void __launch_bounds__(256) k_kda_wy(Problem p, Args a, KdaWork w) {
   mm(CH, V, CH, w.Ut + u * CH * V, V, 1.f, false, sT, LDA, 1, sV, V, 1, 1);
 }
 
+// k_kda_wy for bf16 with K = V = 128, its products on the tensor cores from compensated bf16
+// pairs.  The blocks of A and P below the diagonal, for each sub-chunk a (through r = 16 a - 1):
+// one M = 64 tile L holds, in every row i >= 16, k_i e^{Gam_i - Gam_r(i)} (Lq the same with
+// q_i), and R_a the rows k_j e^{Gam_r - Gam_j}, j < 16 a; the product L R_a^T holds sub-chunk a's
+// block in rows 16a..16a+15 (the other rows are not read).  The diagonal blocks are summed by
+// channel on CUDA cores meanwhile.  After the blocked inverse: W = T' X' and U~ = T' V with
+// T' = T diag(beta), X' = k e^{Gam}.  TMEM columns: A_a at 0, 16, 48; P_a at 96, 112, 144;
+// W at 256, U~ at 384.
+namespace kf {
+using namespace tcx;
+constexpr int TT = 64 * 128;
+constexpr int O_V = 0, O_KB = 16384, O_QB = 32768, O_G = 49152, O_DD = 81920, O_B = 90112;
+constexpr int O_R = 91136;  // region: the A/P operand tiles, then the inverse and the W/U~ operands
+constexpr int O_LKH = O_R, O_LKL = O_R + 16384, O_LQH = O_R + 32768, O_LQL = O_R + 49152;
+constexpr int O_R1 = O_R + 65536, O_R2 = O_R + 73728, O_R3 = O_R + 90112;  // hi then lo, 16a rows each
+constexpr int O_SA = O_R, O_ST = O_R + 17408, O_SX = O_R + 34816, O_SP = O_R + 52224;
+constexpr int O_TPH = O_R + 53248, O_TPL = O_R + 61440, O_XH = O_R + 69632, O_XL = O_R + 86016;
+constexpr int WYF_BYTES = O_R + 114688;
+static_assert(O_SP + CH * CH * 4 <= O_R + 114688 && O_XL + 16384 <= O_R + 114688, "region");
+static_assert(1024 + WYF_BYTES <= 227 * 1024, "kda wy shared memory");
+static_assert(O_R % 1024 == 0 && O_TPH % 1024 == 0 && O_XH % 1024 == 0, "tile alignment");
+}  // namespace kf
+
+__global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork w) {
+  using namespace kf;
+  if (kda_failed(w)) return;
+  const int gc = blockIdx.x, hv = blockIdx.y;
+  const int4 e = w.chunk_tab[gc];
+  if (e.x < 0) return;
+  constexpr int K = 128, V = 128;
+  const int L = e.z, tok0 = e.w, hk = hv / p.G;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  extern __shared__ unsigned char smraw[];
+  unsigned char* sm = align1k(smraw);
+  bf16* sK = reinterpret_cast<bf16*>(sm + O_KB);
+  bf16* sQ = reinterpret_cast<bf16*>(sm + O_QB);
+  float* sG = reinterpret_cast<float*>(sm + O_G);
+  float* sDA = reinterpret_cast<float*>(sm + O_DD);  // [4][16][16] diagonal blocks of A (times beta_i)
+  float* sDP = sDA + 1024;                           // [4][16][16] of P
+  float* sb = reinterpret_cast<float*>(sm + O_B);
+  __shared__ uint64_t bar[2];
+  __shared__ uint32_t tslot;
+  int* err = w.status;
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tslot, 512);
+    tmem_relinquish();
+  }
+  {  // k, q (row-major bf16), V (swizzled tile), rows past L zero; beta
+    const size_t rs = (size_t)p.H * K;
+    const bf16* gk = static_cast<const bf16*>(a.k) + ((size_t)tok0 * p.H + hk) * K;
+    const bf16* gq = static_cast<const bf16*>(a.q) + ((size_t)tok0 * p.H + hk) * K;
+    const bf16* gv = static_cast<const bf16*>(a.v) + ((size_t)tok0 * p.HV + hv) * V;
+    uint4 rk[4], rq[4], rv[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+      rk[m] = rq[m] = rv[m] = make_uint4(0u, 0u, 0u, 0u);
+      if (row < L) {
+        rk[m] = __ldg(reinterpret_cast<const uint4*>(gk + row * rs + 8 * j));
+        rq[m] = __ldg(reinterpret_cast<const uint4*>(gq + row * rs + 8 * j));
+        rv[m] = __ldg(reinterpret_cast<const uint4*>(gv + (size_t)row * p.HV * V + 8 * j));
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+      reinterpret_cast<uint4*>(sK)[x] = rk[m];
+      reinterpret_cast<uint4*>(sQ)[x] = rq[m];
+      *reinterpret_cast<uint4*>(sm + O_V + sw128_chunk(row, j, TT)) = rv[m];
+    }
+    if (tid < CH) sb[tid] = tid < L ? a.beta[(size_t)(tok0 + tid) * p.HV + hv] : 0.f;
+  }
+  load_tile<float>(sG, K, a.g_raw + ((size_t)tok0 * p.HV + hv) * K, (size_t)p.HV * K, L, K);
+  __syncthreads();
+  {  // the gate of every (token, channel), rows past L zero; then the cumsum per channel
+    const float nexp = -expf(a.A_log[hv]);
+    for (int x = tid; x < CH * K; x += 256) {
+      const int i = x / K, c = x % K;
+      float yg = 0.f;
+      if (i < L) {
+        const float z = sG[x] + (a.dt_bias ? a.dt_bias[(size_t)hv * K + c] : 0.f);
+        yg = nexp * (z > 20.f ? z : log1pf(expf(z)));
+      }
+      sG[x] = yg;
+    }
+    __syncthreads();
+    if (tid < K) {
+      float acc = 0.f;
+      for (int i = 0; i < CH; ++i) {
+        acc += sG[i * K + tid];
+        sG[i * K + tid] = acc * LOG2E;
+      }
+    }
+    __syncthreads();
+  }
+  // L tiles (rows >= 16) and R_a (a = 1, 2, 3) as hi/lo pairs
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+    float fk[8], fq[8];
+    const int r = row >= 16 ? 16 * (row >> 4) - 1 : 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int c = 8 * j + q;
+      const float ex = row >= 16 ? exp2f(sG[row * K + c] - sG[r * K + c]) : 0.f;
+      fk[q] = __bfloat162float(sK[row * K + c]) * ex;
+      fq[q] = __bfloat162float(sQ[row * K + c]) * ex;
+    }
+    st_chunk_split(sm + O_LKH, sm + O_LKL, row, j, TT, fk);
+    st_chunk_split(sm + O_LQH, sm + O_LQL, row, j, TT, fq);
+  }
+  for (int x = tid; x < 96 * 16; x += 256) {  // 16 + 32 + 48 rows of 16 chunks
+    const int ra = x >> 4, j = x & 15;
+    const int A = ra < 16 ? 1 : (ra < 48 ? 2 : 3), row = ra - (A == 1 ? 0 : (A == 2 ? 16 : 48));
+    const int r = 16 * A - 1, off = A == 1 ? O_R1 : (A == 2 ? O_R2 : O_R3), bb = 16 * A * 128;
+    float f[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int c = 8 * j + q;
+      f[q] = __bfloat162float(sK[row * K + c]) * exp2f(sG[r * K + c] - sG[row * K + c]);
+    }
+    st_chunk_split(sm + off, sm + off + 2 * bb, row, j, bb, f);
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tslot;
+  if (tid == 0) {
+    const uint32_t lkh = smem_u32(sm + O_LKH), lkl = smem_u32(sm + O_LKL);
+    const uint32_t lqh = smem_u32(sm + O_LQH), lql = smem_u32(sm + O_LQL);
+#pragma unroll
+    for (int A = 1; A <= 3; ++A) {
+      const int bb = 16 * A * 128;
+      const uint32_t rh = smem_u32(sm + (A == 1 ? O_R1 : (A == 2 ? O_R2 : O_R3))), rl = rh + 2 * bb;
+      const uint32_t id = idesc_bf16(64, 16 * A, false, false);
+      const int ca = A == 1 ? 0 : (A == 2 ? 16 : 48);
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const uint64_t bh = desc_kmajor(rh, s, bb), bl = desc_kmajor(rl, s, bb);
+        const uint64_t akh = desc_kmajor(lkh, s, TT), aqh = desc_kmajor(lqh, s, TT);
+        mma_bf16(taddr(tb, 0, ca), akh, bh, id, s > 0);
+        mma_bf16(taddr(tb, 0, ca), akh, bl, id, 1);
+        mma_bf16(taddr(tb, 0, ca), desc_kmajor(lkl, s, TT), bh, id, 1);
+        mma_bf16(taddr(tb, 0, 96 + ca), aqh, bh, id, s > 0);
+        mma_bf16(taddr(tb, 0, 96 + ca), aqh, bl, id, 1);
+        mma_bf16(taddr(tb, 0, 96 + ca), desc_kmajor(lql, s, TT), bh, id, 1);
+      }
+    }
+    mma_commit(&bar[0]);
+  }
+  // diagonal sub-blocks, one warp per pair (i, j), j <= i in one sub-chunk, lanes over channels
+  constexpr int PAIRS = SUB * (SUB + 1) / 2;
+  for (int pr = warp; pr < (CH / SUB) * PAIRS; pr += 8) {
+    const int blk = pr / PAIRS;
+    int q = pr % PAIRS, ii = 0;
+    while (q > ii) q -= ++ii;  // q in [0, ii]
+    const int i = blk * SUB + ii, j = blk * SUB + q;
+    float sa = 0.f, sp = 0.f;
+    for (int c = lane; c < K; c += 32) {
+      const float kj = __bfloat162float(sK[j * K + c]) * exp2f(sG[i * K + c] - sG[j * K + c]);
+      sa = fmaf(__bfloat162float(sK[i * K + c]), kj, sa);
+      sp = fmaf(__bfloat162float(sQ[i * K + c]), kj, sp);
+    }
+    sa = warp_total(sa);
+    sp = warp_total(sp);
+    if (lane == 0) {
+      sDA[(blk * SUB + ii) * SUB + q] = j < i ? sb[i] * sa : 0.f;
+      sDP[(blk * SUB + ii) * SUB + q] = sp;
+    }
+  }
+  bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
+  tc_fence_after();
+  float* sA = reinterpret_cast<float*>(sm + O_SA);
+  float* sT = reinterpret_cast<float*>(sm + O_ST);
+  float* sX = reinterpret_cast<float*>(sm + O_SX);
+  float* sP = reinterpret_cast<float*>(sm + O_SP);
+  // A (times beta_i, strictly lower) and P (lower incl. the diagonal): diagonal blocks and zeros
+  for (int x = tid; x < CH * CH; x += 256) {
+    const int i = x >> 6, j = x & 63;
+    float va = 0.f, vp = 0.f;
+    if ((i >> 4) == (j >> 4) && j <= i) {
+      va = sDA[(i & ~15) * SUB + (i & 15) * SUB + (j & 15)];
+      vp = sDP[(i & ~15) * SUB + (i & 15) * SUB + (j & 15)];
+    }
+    sA[i * LDA + j] = va;
+    sP[x] = vp;
+  }
+  __syncthreads();
+  {  // the blocks below the diagonal from TMEM: warps of sub-partition a = warp % 4 (a >= 1);
+     // warp half 0 reads A, half 1 reads P
+    const int A = warp & 3, half = warp >> 2;
+    if (ok && A > 0) {
+      const int ca = (half ? 96 : 0) + (A == 1 ? 0 : (A == 2 ? 16 : 48));
+      const int ib = 16 * A + (lane >> 2), cq = 2 * (lane & 3);
+      for (int t = 0; t < A; ++t) {
+        float v[8];
+        tmem_ld16dp_x2(taddr(tb, 32 * A, ca + 16 * t), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            const int i = ib + 8 * (qq >> 1), j = 16 * t + 8 * jj + cq + (qq & 1);
+            const float val = v[4 * jj + qq];
+            if (half) sP[i * CH + j] = val;
+            else sA[i * LDA + j] = sb[i] * val;
+          }
+      }
+    }
+  }
+  __syncthreads();
+  const size_t u = (size_t)gc * p.HV + hv, uk = u * CH * K;
+  {
+    float4* gP = reinterpret_cast<float4*>(w.P + u * CH * CH);
+    for (int x = tid; x < CH * CH / 4; x += 256) gP[x] = reinterpret_cast<const float4*>(sP)[x];
+    if (w.Gam) {
+      float4* gG = reinterpret_cast<float4*>(w.Gam + uk);
+      for (int x = tid; x < CH * K / 4; x += 256) gG[x] = reinterpret_cast<const float4*>(sG)[x];
+    }
+  }
+  tcx::unit_lower_inverse64(sA, sT, sX, tid);  // T = (I + A)^-1 (ends with a barrier)
+  if (w.Tm)
+    for (int x = tid; x < CH * CH; x += 256) w.Tm[u * CH * CH + x] = sT[(x / CH) * LDA + x % CH];
+  // K^ = k e^{Gam_C - Gam}, Q~ = q e^{Gam}, e^{Gam_C}; X' = k e^{Gam} and T' = T diag(beta) as tiles
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+    float fx[8], fh[8], fq[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int c = 8 * j + q, o = row * K + c;
+      const float g = sG[o], kk = __bfloat162float(sK[o]);
+      fx[q] = kk * exp2f(g);
+      fh[q] = kk * exp2f(sG[(CH - 1) * K + c] - g);
+      fq[q] = __bfloat162float(sQ[o]) * exp2f(g);
+    }
+    float4* kh = reinterpret_cast<float4*>(w.Kh + uk + row * K + 8 * j);
+    float4* qt = reinterpret_cast<float4*>(w.Qt + uk + row * K + 8 * j);
+    kh[0] = make_float4(fh[0], fh[1], fh[2], fh[3]);
+    kh[1] = make_float4(fh[4], fh[5], fh[6], fh[7]);
+    qt[0] = make_float4(fq[0], fq[1], fq[2], fq[3]);
+    qt[1] = make_float4(fq[4], fq[5], fq[6], fq[7]);
+    st_chunk_split(sm + O_XH, sm + O_XL, row, j, TT, fx);
+  }
+  for (int c = tid; c < K; c += 256) w.eGC[u * K + c] = exp2f(sG[(CH - 1) * K + c]);
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    const int x = tid + 256 * m, row = x >> 3, j = x & 7;
+    float f[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) f[q] = sT[row * LDA + 8 * j + q] * sb[8 * j + q];
+    st_chunk_split(sm + O_TPH, sm + O_TPL, row, j, TT, f);
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (ok && tid == 0) {
+    const uint32_t th = smem_u32(sm + O_TPH), tl = smem_u32(sm + O_TPL);
+    const uint32_t xh = smem_u32(sm + O_XH), xl = smem_u32(sm + O_XL), vv = smem_u32(sm + O_V);
+    constexpr uint32_t id = idesc_bf16(64, 128, false, true);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const uint64_t ah = desc_kmajor(th, s, TT), al = desc_kmajor(tl, s, TT);
+      const uint64_t bx = desc_mnmajor(xh, s, TT), bv = desc_mnmajor(vv, s, TT);
+      mma_bf16(taddr(tb, 0, 256), ah, bx, id, s > 0);
+      mma_bf16(taddr(tb, 0, 256), ah, desc_mnmajor(xl, s, TT), id, 1);
+      mma_bf16(taddr(tb, 0, 256), al, bx, id, 1);
+      mma_bf16(taddr(tb, 0, 384), ah, bv, id, s > 0);
+      mma_bf16(taddr(tb, 0, 384), al, bv, id, 1);
+    }
+    mma_commit(&bar[1]);
+  }
+  ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
+  tc_fence_after();
+  if (ok) {  // W and U~, M = 64 accumulators (rows r0, r0 + 8)
+    const int half = warp >> 2, sub = 32 * (warp & 3), r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
+    float x[32], y[32];
+    tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
+    tmem_ld16dp_x8(taddr(tb, sub, 384 + 64 * half), y);
+    tmem_wait_ld();
+    float* gW = w.W + uk;
+    float* gU = w.Ut + u * CH * V;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = 64 * half + 8 * j + cq;
+      *reinterpret_cast<float2*>(gW + r0 * K + c) = make_float2(x[4 * j], x[4 * j + 1]);
+      *reinterpret_cast<float2*>(gW + (r0 + 8) * K + c) = make_float2(x[4 * j + 2], x[4 * j + 3]);
+      *reinterpret_cast<float2*>(gU + r0 * V + c) = make_float2(y[4 * j], y[4 * j + 1]);
+      *reinterpret_cast<float2*>(gU + (r0 + 8) * V + c) = make_float2(y[4 * j + 2], y[4 * j + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 512);
+}
+
 // Sequential scan of one (sequence, value head, rows v0..v0+31 of S): stores the state entering
 // each chunk (rows v of S, [V][K]) and U = U~ - W S^T for those rows, returns the final state.
 // The next chunk's W, K^, U~ slice and e^{Gam_C} are loaded into registers while the current
@@ -316,7 +622,9 @@ cudaError_t go(const char* name, Kern kern, dim3 grid, size_t smem, cudaStream_t
 
 template <typename T>
 cudaError_t forward_t(const Problem& p, const Args& a, const KdaWork& w, cudaStream_t s) {
-  cudaError_t e = go("kda_wy", k_kda_wy<T>, dim3(p.NCmax, p.HV), wy_smem(p.K, p.V), s, p, a, w);
+  const bool tc = std::is_same<T, __nv_bfloat16>::value && p.K == 128 && p.V == 128;
+  cudaError_t e = tc ? go("kda_tc_wy", k_kda_tc_wy, dim3(p.NCmax, p.HV), 1024 + kf::WYF_BYTES, s, p, a, w)
+                     : go("kda_wy", k_kda_wy<T>, dim3(p.NCmax, p.HV), wy_smem(p.K, p.V), s, p, a, w);
   if (e == cudaSuccess)
     e = go("kda_scan", k_kda_scan, dim3(p.Nst, p.HV, p.V / 32), scan_smem(p.K), s, p, a, w);
   if (e == cudaSuccess) e = go("kda_out", k_kda_out<T>, dim3(p.NCmax, p.HV), out_smem(p.K, p.V), s, p, a, w);
