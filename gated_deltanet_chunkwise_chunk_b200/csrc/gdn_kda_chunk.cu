@@ -570,6 +570,180 @@ __global__ void __launch_bounds__(256) k_kda_scan(Problem p, Args a, KdaWork w) 
     }
 }
 
+// k_kda_scan for bf16 with K = V = 128: one CTA per (sequence, value head) holds the whole
+// state S [V][K] in fp32 registers (thread: row v = 32 (warp % 4) + lane, columns 64 (warp / 4)..)
+// and takes both products of a chunk on the tensor cores, from compensated bf16 pairs:
+//   U = U~ - W S^T        (M = 64 tokens, N = V;  A = W, B = S, K-major)       TMEM [0, 128)
+//   S' = S Diag(e^{Gam_C}) + U^T K^   (M = V, N = K;  A = U^T, B = K^, MN-major)  TMEM [128, 256)
+// It stores the state entering every chunk and U, as k_kda_scan does.
+namespace ks {
+using namespace tcx;
+constexpr int TT = 64 * 128, TS = 128 * 128;
+constexpr int O_WH = 0, O_WL = 16384, O_KH = 32768, O_KL = 49152, O_UH = 65536, O_UL = 81920;
+constexpr int O_SH = 98304, O_SL = 131072, O_E = 163840;
+constexpr int SCAN_BYTES = O_E + 512;
+static_assert(1024 + SCAN_BYTES <= 227 * 1024, "kda scan shared memory");
+}  // namespace ks
+
+__global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWork w) {
+  using namespace ks;
+  if (kda_failed(w)) return;
+  const int n = blockIdx.x, hv = blockIdx.y;
+  const int4 sq = w.seq_tab[n];
+  constexpr int K = 128, V = 128;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int half = warp >> 2, v = 32 * (warp & 3) + lane, c0 = 64 * half;
+  const int r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);  // 16-lane (M = 64) view
+  extern __shared__ unsigned char smraw[];
+  unsigned char* sm = align1k(smraw);
+  float* sE = reinterpret_cast<float*>(sm + O_E);
+  __shared__ uint64_t bar[2];
+  __shared__ uint32_t tslot;
+  int* err = w.status;
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tslot, 256);
+    tmem_relinquish();
+  }
+  float S[64];
+  {
+    const float* h0 = a.h0 ? a.h0 + ((size_t)n * p.HV + hv) * K * V : nullptr;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) S[c] = h0 ? h0[(size_t)(c0 + c) * V + v] : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tslot;
+  const uint32_t aWH = smem_u32(sm + O_WH), aWL = smem_u32(sm + O_WL), aKH = smem_u32(sm + O_KH);
+  const uint32_t aKL = smem_u32(sm + O_KL), aUH = smem_u32(sm + O_UH), aUL = smem_u32(sm + O_UL);
+  const uint32_t aSH = smem_u32(sm + O_SH), aSL = smem_u32(sm + O_SL);
+  bool ok = true;
+  for (int ci = 0; ci < sq.y && ok; ++ci) {
+    const size_t u = (size_t)(sq.x + ci) * p.HV + hv;
+    {  // the state entering the chunk: stored, and as a hi/lo tile
+      float4* h = reinterpret_cast<float4*>(w.h + u * V * K + (size_t)v * K + c0);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) h[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) st_chunk_split(sm + O_SH, sm + O_SL, v, 8 * half + j, TS, S + 8 * j);
+    }
+    {  // W and K^ as hi/lo tiles, e^{Gam_C}
+      const float* gW = w.W + u * CH * K;
+      const float* gK = w.Kh + u * CH * K;
+      float4 rw[8], rk[8];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+        const float4* pw = reinterpret_cast<const float4*>(gW + row * K + 8 * j);
+        const float4* pk = reinterpret_cast<const float4*>(gK + row * K + 8 * j);
+        rw[2 * m] = __ldg(pw);
+        rw[2 * m + 1] = __ldg(pw + 1);
+        rk[2 * m] = __ldg(pk);
+        rk[2 * m + 1] = __ldg(pk + 1);
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+        const float fw[8] = {rw[2 * m].x, rw[2 * m].y, rw[2 * m].z, rw[2 * m].w,
+                             rw[2 * m + 1].x, rw[2 * m + 1].y, rw[2 * m + 1].z, rw[2 * m + 1].w};
+        const float fk[8] = {rk[2 * m].x, rk[2 * m].y, rk[2 * m].z, rk[2 * m].w,
+                             rk[2 * m + 1].x, rk[2 * m + 1].y, rk[2 * m + 1].z, rk[2 * m + 1].w};
+        st_chunk_split(sm + O_WH, sm + O_WL, row, j, TT, fw);
+        st_chunk_split(sm + O_KH, sm + O_KL, row, j, TT, fk);
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {  // W S^T
+      constexpr uint32_t id = idesc_bf16(64, 128, false, false);
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const uint64_t wh = desc_kmajor(aWH, s, TT), sh = desc_kmajor(aSH, s, TS);
+        mma_bf16(taddr(tb, 0, 0), wh, sh, id, s > 0);
+        mma_bf16(taddr(tb, 0, 0), wh, desc_kmajor(aSL, s, TS), id, 1);
+        mma_bf16(taddr(tb, 0, 0), desc_kmajor(aWL, s, TT), sh, id, 1);
+      }
+      mma_commit(&bar[0]);
+    }
+    // e^{Gam_C} for the state update (into shared memory once every thread is past the last
+    // chunk's update)
+    const float egc = tid < K ? w.eGC[u * K + tid] : 0.f;
+    float ut[32];  // U~ at this thread's (row, column) pairs of the 16-lane view
+    {
+      const float* gU = w.Ut + u * CH * V;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = c0 + 8 * j + cq;
+        const float2 a0 = *reinterpret_cast<const float2*>(gU + r0 * V + c);
+        const float2 a1 = *reinterpret_cast<const float2*>(gU + (r0 + 8) * V + c);
+        ut[4 * j] = a0.x;
+        ut[4 * j + 1] = a0.y;
+        ut[4 * j + 2] = a1.x;
+        ut[4 * j + 3] = a1.y;
+      }
+    }
+    ok = __syncthreads_and(mbar_wait(&bar[0], ci & 1, err));
+    tc_fence_after();
+    if (tid < K) sE[tid] = egc;
+    if (ok) {  // U = U~ - W S^T: stored, and as a hi/lo tile
+      float x[32];
+      tmem_ld16dp_x8(taddr(tb, 32 * (warp & 3), c0), x);
+      tmem_wait_ld();
+      float* gU = w.U + u * CH * V;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = c0 + 8 * j + cq;
+        const float u0 = ut[4 * j] - x[4 * j], u1 = ut[4 * j + 1] - x[4 * j + 1];
+        const float u2 = ut[4 * j + 2] - x[4 * j + 2], u3 = ut[4 * j + 3] - x[4 * j + 3];
+        *reinterpret_cast<float2*>(gU + r0 * V + c) = make_float2(u0, u1);
+        *reinterpret_cast<float2*>(gU + (r0 + 8) * V + c) = make_float2(u2, u3);
+        st_pair_split(sm + O_UH, sm + O_UL, r0, c, TT, u0, u1);
+        st_pair_split(sm + O_UH, sm + O_UL, r0 + 8, c, TT, u2, u3);
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (ok && tid == 0) {  // U^T K^
+      constexpr uint32_t id = idesc_bf16(128, 128, true, true);
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const uint64_t uh = desc_mnmajor(aUH, s, TT), kh = desc_mnmajor(aKH, s, TT);
+        mma_bf16(taddr(tb, 0, 128), uh, kh, id, s > 0);
+        mma_bf16(taddr(tb, 0, 128), uh, desc_mnmajor(aKL, s, TT), id, 1);
+        mma_bf16(taddr(tb, 0, 128), desc_mnmajor(aUL, s, TT), kh, id, 1);
+      }
+      mma_commit(&bar[1]);
+    }
+    ok = __syncthreads_and(ok && mbar_wait(&bar[1], ci & 1, err));
+    tc_fence_after();
+    if (ok) {  // S = S Diag(e^{Gam_C}) + U^T K^  (lane = row v, this half's 64 columns)
+      float x[64];
+      tmem_ld64(taddr(tb, 32 * (warp & 3), 128 + c0), x);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 64; ++c) S[c] = fmaf(S[c], sE[c0 + c], x[c]);
+    }
+  }
+  if (ok && a.ht) {
+    float* ht = a.ht + ((size_t)n * p.HV + hv) * K * V;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) ht[(size_t)(c0 + c) * V + v] = S[c];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 256);
+}
+
 // O = scale (Q~ S^T + P U) for one (chunk, value head)
 template <typename T>
 __global__ void __launch_bounds__(256) k_kda_out(Problem p, Args a, KdaWork w) {
@@ -626,7 +800,8 @@ cudaError_t forward_t(const Problem& p, const Args& a, const KdaWork& w, cudaStr
   cudaError_t e = tc ? go("kda_tc_wy", k_kda_tc_wy, dim3(p.NCmax, p.HV), 1024 + kf::WYF_BYTES, s, p, a, w)
                      : go("kda_wy", k_kda_wy<T>, dim3(p.NCmax, p.HV), wy_smem(p.K, p.V), s, p, a, w);
   if (e == cudaSuccess)
-    e = go("kda_scan", k_kda_scan, dim3(p.Nst, p.HV, p.V / 32), scan_smem(p.K), s, p, a, w);
+    e = tc ? go("kda_tc_scan", k_kda_tc_scan, dim3(p.Nst, p.HV), 1024 + ks::SCAN_BYTES, s, p, a, w)
+           : go("kda_scan", k_kda_scan, dim3(p.Nst, p.HV, p.V / 32), scan_smem(p.K), s, p, a, w);
   if (e == cudaSuccess) e = go("kda_out", k_kda_out<T>, dim3(p.NCmax, p.HV), out_smem(p.K, p.V), s, p, a, w);
   return e;
 }

@@ -232,6 +232,188 @@ __global__ void __launch_bounds__(256) k_kda_bwd_scan(Problem p, Args a, KdaWork
     }
 }
 
+// ---------------------------------------------------------------- reverse state scan, tcgen05
+// k_kda_bwd_scan for bf16 with K = V = 128: one CTA per (sequence, value head) holds dS [V][K] in
+// fp32 registers (thread: row v = 32 (warp % 4) + lane, columns 64 (warp / 4)..) and takes both
+// products of a chunk on the tensor cores (compensated bf16 pairs; dO is bf16 already):
+//   dU = (scale P)^T dO + K^ dS'^T                 (M = 64 tokens, N = V)   TMEM [0, 128)
+//   dS = dS' Diag(e^{Gam_C}) + dO^T (scale Q~) + dU^T (-W)   (M = V, N = K)  TMEM [128, 256)
+namespace kb {
+using namespace tcx;
+constexpr int TT = 64 * 128, TS = 128 * 128;
+constexpr int O_PH = 0, O_PL = 8192, O_DO = 16384, O_KH = 32768, O_KL = 49152, O_QH = 65536;
+constexpr int O_QL = 81920, O_WH = 98304, O_WL = 114688, O_UH = 131072, O_UL = 147456;
+constexpr int O_SH = 163840, O_SL = 196608, O_E = 229376;
+constexpr int BSCAN_BYTES = O_E + 512;
+static_assert(1024 + BSCAN_BYTES <= 227 * 1024, "kda backward scan shared memory");
+}  // namespace kb
+
+__global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, KdaWork w) {
+  using namespace kb;
+  if (kda_failed(w)) return;
+  const int n = blockIdx.x, hv = blockIdx.y;
+  const int4 sq = w.seq_tab[n];
+  constexpr int K = 128, V = 128;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int half = warp >> 2, v = 32 * (warp & 3) + lane, c0 = 64 * half;
+  const int r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
+  extern __shared__ unsigned char smraw[];
+  unsigned char* sm = align1k(smraw);
+  float* sE = reinterpret_cast<float*>(sm + O_E);
+  __shared__ uint64_t bar[2];
+  __shared__ uint32_t tslot;
+  int* err = w.status;
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tslot, 256);
+    tmem_relinquish();
+  }
+  float S[64];  // dS, rows v, columns c0..c0+63
+  {
+    const float* dht = a.dht ? a.dht + ((size_t)n * p.HV + hv) * K * V : nullptr;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) S[c] = dht ? dht[(size_t)(c0 + c) * V + v] : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tslot;
+  const bf16* dO = static_cast<const bf16*>(a.dO);
+  bool ok = true;
+  for (int k = 0; k < sq.y && ok; ++k) {
+    const int ci = sq.y - 1 - k, gc = sq.x + ci;
+    const int4 e = w.chunk_tab[gc];
+    const size_t u = (size_t)gc * p.HV + hv;
+    {  // dS' (leaving the chunk): stored, and as a hi/lo tile
+      float4* dh = reinterpret_cast<float4*>(w.dh + u * V * K + (size_t)v * K + c0);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) dh[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) st_chunk_split(sm + O_SH, sm + O_SL, v, 8 * half + j, TS, S + 8 * j);
+    }
+    {  // scale P, K^, scale Q~, -W as hi/lo tiles; dO (bf16, rows past L zero)
+      const float* gK = w.Kh + u * CH * K;
+      const float* gQ = w.Qt + u * CH * K;
+      const float* gW = w.W + u * CH * K;
+      const float* gP = w.P + u * CH * CH;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+        const float4* pk = reinterpret_cast<const float4*>(gK + row * K + 8 * j);
+        const float4* pq = reinterpret_cast<const float4*>(gQ + row * K + 8 * j);
+        const float4* pw = reinterpret_cast<const float4*>(gW + row * K + 8 * j);
+        const float4 k0 = __ldg(pk), k1 = __ldg(pk + 1), q0 = __ldg(pq), q1 = __ldg(pq + 1);
+        const float4 w0 = __ldg(pw), w1 = __ldg(pw + 1);
+        const uint4 dd = row < e.z ? __ldg(reinterpret_cast<const uint4*>(
+                                         dO + ((size_t)(e.w + row) * p.HV + hv) * V + 8 * j))
+                                   : make_uint4(0u, 0u, 0u, 0u);
+        const float fk[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+        const float sc = p.scale;
+        const float fq[8] = {sc * q0.x, sc * q0.y, sc * q0.z, sc * q0.w, sc * q1.x, sc * q1.y, sc * q1.z, sc * q1.w};
+        const float fw[8] = {-w0.x, -w0.y, -w0.z, -w0.w, -w1.x, -w1.y, -w1.z, -w1.w};
+        st_chunk_split(sm + O_KH, sm + O_KL, row, j, TT, fk);
+        st_chunk_split(sm + O_QH, sm + O_QL, row, j, TT, fq);
+        st_chunk_split(sm + O_WH, sm + O_WL, row, j, TT, fw);
+        *reinterpret_cast<uint4*>(sm + O_DO + sw128_chunk(row, j, TT)) = dd;
+      }
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int x = tid + 256 * m, row = x >> 3, j = x & 7;
+        const float4* pp = reinterpret_cast<const float4*>(gP + row * CH + 8 * j);
+        const float4 p0 = __ldg(pp), p1 = __ldg(pp + 1);
+        const float sc = p.scale;
+        const float f[8] = {sc * p0.x, sc * p0.y, sc * p0.z, sc * p0.w, sc * p1.x, sc * p1.y, sc * p1.z, sc * p1.w};
+        st_chunk_split(sm + O_PH, sm + O_PL, row, j, TT, f);
+      }
+    }
+    const float egc = tid < K ? w.eGC[u * K + tid] : 0.f;
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {  // dU = (scale P)^T dO + K^ dS'^T
+      const uint32_t ph = smem_u32(sm + O_PH), pl = smem_u32(sm + O_PL), d = smem_u32(sm + O_DO);
+      const uint32_t kh = smem_u32(sm + O_KH), kl = smem_u32(sm + O_KL);
+      const uint32_t sh = smem_u32(sm + O_SH), sl = smem_u32(sm + O_SL);
+      constexpr uint32_t i_pd = idesc_bf16(64, 128, true, true), i_ks = idesc_bf16(64, 128, false, false);
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const uint64_t bd = desc_mnmajor(d, s, TT);
+        mma_bf16(taddr(tb, 0, 0), desc_mnmajor(ph, s, TT), bd, i_pd, s > 0);
+        mma_bf16(taddr(tb, 0, 0), desc_mnmajor(pl, s, TT), bd, i_pd, 1);
+      }
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const uint64_t ak = desc_kmajor(kh, s, TT), bs = desc_kmajor(sh, s, TS);
+        mma_bf16(taddr(tb, 0, 0), ak, bs, i_ks, 1);
+        mma_bf16(taddr(tb, 0, 0), ak, desc_kmajor(sl, s, TS), i_ks, 1);
+        mma_bf16(taddr(tb, 0, 0), desc_kmajor(kl, s, TT), bs, i_ks, 1);
+      }
+      mma_commit(&bar[0]);
+    }
+    ok = __syncthreads_and(mbar_wait(&bar[0], k & 1, err));
+    tc_fence_after();
+    if (tid < K) sE[tid] = egc;
+    if (ok) {  // dU: stored, and as a hi/lo tile
+      float x[32];
+      tmem_ld16dp_x8(taddr(tb, 32 * (warp & 3), c0), x);
+      tmem_wait_ld();
+      float* gU = w.dU + u * CH * V;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = c0 + 8 * j + cq;
+        *reinterpret_cast<float2*>(gU + r0 * V + c) = make_float2(x[4 * j], x[4 * j + 1]);
+        *reinterpret_cast<float2*>(gU + (r0 + 8) * V + c) = make_float2(x[4 * j + 2], x[4 * j + 3]);
+        st_pair_split(sm + O_UH, sm + O_UL, r0, c, TT, x[4 * j], x[4 * j + 1]);
+        st_pair_split(sm + O_UH, sm + O_UL, r0 + 8, c, TT, x[4 * j + 2], x[4 * j + 3]);
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (ok && tid == 0) {  // dO^T (scale Q~) + dU^T (-W)
+      const uint32_t d = smem_u32(sm + O_DO), qh = smem_u32(sm + O_QH), ql = smem_u32(sm + O_QL);
+      const uint32_t uh = smem_u32(sm + O_UH), ul = smem_u32(sm + O_UL);
+      const uint32_t wh = smem_u32(sm + O_WH), wl = smem_u32(sm + O_WL);
+      constexpr uint32_t id = idesc_bf16(128, 128, true, true);
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const uint64_t ad = desc_mnmajor(d, s, TT);
+        mma_bf16(taddr(tb, 0, 128), ad, desc_mnmajor(qh, s, TT), id, s > 0);
+        mma_bf16(taddr(tb, 0, 128), ad, desc_mnmajor(ql, s, TT), id, 1);
+        const uint64_t au = desc_mnmajor(uh, s, TT), bw = desc_mnmajor(wh, s, TT);
+        mma_bf16(taddr(tb, 0, 128), au, bw, id, 1);
+        mma_bf16(taddr(tb, 0, 128), au, desc_mnmajor(wl, s, TT), id, 1);
+        mma_bf16(taddr(tb, 0, 128), desc_mnmajor(ul, s, TT), bw, id, 1);
+      }
+      mma_commit(&bar[1]);
+    }
+    ok = __syncthreads_and(ok && mbar_wait(&bar[1], k & 1, err));
+    tc_fence_after();
+    if (ok) {  // dS = dS' Diag(e^{Gam_C}) + the products (lane = row v, this half's columns)
+      float x[64];
+      tmem_ld64(taddr(tb, 32 * (warp & 3), 128 + c0), x);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 64; ++c) S[c] = fmaf(S[c], sE[c0 + c], x[c]);
+    }
+  }
+  if (ok && a.dh0) {
+    float* dh0 = a.dh0 + ((size_t)n * p.HV + hv) * K * V;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) dh0[(size_t)(c0 + c) * V + v] = S[c];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 256);
+}
+
 // ---------------------------------------------------------------- output-side terms
 // dP, dQ~, dW = -dU S, dK^ (with the Gam_C column terms) and the dP gated products.  Writes the
 // unit's dq and dk shares, dGam and dW.  Every product reads both operands from shared memory:
@@ -1193,7 +1375,9 @@ bool kda_tc(const Problem& p) {
 
 template <typename T>
 cudaError_t backward_t(const Problem& p, const Args& a, const KdaWork& w, cudaStream_t s) {
-  cudaError_t e = go("kda_bwd_scan", k_kda_bwd_scan<T>, dim3(p.Nst, p.HV, p.V / 32), scan_smem(p.K), s, p, a, w);
+  cudaError_t e = kda_tc<T>(p)
+      ? go("kda_tc_bwd_scan", k_kda_tc_bwd_scan, dim3(p.Nst, p.HV), 1024 + kb::BSCAN_BYTES, s, p, a, w)
+      : go("kda_bwd_scan", k_kda_bwd_scan<T>, dim3(p.Nst, p.HV, p.V / 32), scan_smem(p.K), s, p, a, w);
   if (e == cudaSuccess)
     e = kda_tc<T>(p) ? go("kda_tc_bwd_dqk", k_kda_tc_bwd_dqk, dim3(p.NCmax, p.HV), 1024 + kt::DQK_BYTES, s, p, a, w)
                      : go("kda_bwd_dqk", k_kda_bwd_dqk<T>, dim3(p.NCmax, p.HV), dqk_smem(p.K, p.V), s, p, a, w);

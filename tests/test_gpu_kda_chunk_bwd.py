@@ -137,7 +137,7 @@ def test_bf16_128_runs_the_tensor_core_kernels():
         names = set(gdn.profile_read())
     finally:
         gdn.profile(False)
-    for k in ("kda_tc_wy", "kda_tc_bwd_dqk", "kda_tc_bwd_wy"):
+    for k in ("kda_tc_wy", "kda_tc_scan", "kda_tc_bwd_scan", "kda_tc_bwd_dqk", "kda_tc_bwd_wy"):
         assert k in names, (k, names)
-    for k in ("kda_wy", "kda_bwd_dqk", "kda_bwd_wy"):
+    for k in ("kda_wy", "kda_scan", "kda_bwd_scan", "kda_bwd_dqk", "kda_bwd_wy"):
         assert k not in names, (k, names)
