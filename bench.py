@@ -786,17 +786,23 @@ def kda_chunk_measure(gdn, dev, pk_hbm: float, steps: int = 5, T: int = 32768) -
            "kda_bwd_dqk": 64 * 64 * V + 3 * 64 * V * K + 2 * (1536 + 544) * K,
            "kda_bwd_wy": 2 * 64 * 64 * (K + V) + 2 * 64 * 64 * 64 + 2 * (1536 + 544) * K}
     kern = {k: round(v[1], 4) for k, v in prof.items()}
-    top = max(fma, key=lambda k: kern.get(k, 0.0))
-    top_tf = 2 * units * fma[top] / (kern[top] / 1e3) / 1e12
+    # bf16 with 128-wide heads runs the tcgen05 kernels (kda_tc_*): same products, tensor peak
+    step_of = {k: k.replace("kda_tc_", "kda_") for k in kern if k.replace("kda_tc_", "kda_") in fma}
+    top = max(step_of, key=lambda k: kern[k])
+    top_tf = 2 * units * fma[step_of[top]] / (kern[top] / 1e3) / 1e12
+    tensor = top.startswith("kda_tc_")
+    pk = peaks()
+    peak = pk["bf16_tflops"] if tensor else FFMA_TFLOPS
+    src = (f"bf16 dense burst, {pk['source']}" if tensor
+           else "148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz (FFMA)")
     return {"workload": f"kda_chunk_B1_T{T}_H16_HV32_D128_bf16", "fwd_ms": round(ms_f, 4),
             "fwd_mtok_s": round(T / (ms_f / 1e3) / 1e6, 3), "step_ms": round(ms, 4),
             "step_mtok_s": round(T / (ms / 1e3) / 1e6, 3), "recurrent_fwd_ms": round(ms_r, 4),
             "kernels_ms": kern,
             "step_tflops": round(2 * units * sum(fma.values()) / (ms / 1e3) / 1e12, 2),
-            "roofline": {"kernel": top, "bound": "alu", "achieved": round(top_tf, 2),
-                         "peak": round(FFMA_TFLOPS, 1), "unit": "TFLOP/s",
-                         "frac": round(top_tf / FFMA_TFLOPS, 4),
-                         "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz (FFMA)"}}
+            "roofline": {"kernel": top, "bound": "tensor" if tensor else "alu",
+                         "achieved": round(top_tf, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+                         "frac": round(top_tf / peak, 4), "peak_source": src}}
 
 
 def kda_gate_measure(gdn, dev, pk_hbm: float, steps: int = 20) -> dict:

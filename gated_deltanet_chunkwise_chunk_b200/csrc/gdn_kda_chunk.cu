@@ -210,6 +210,39 @@ static_assert(1024 + WYF_BYTES <= 227 * 1024, "kda wy shared memory");
 static_assert(O_R % 1024 == 0 && O_TPH % 1024 == 0 && O_XH % 1024 == 0, "tile alignment");
 }  // namespace kf
 
+// Rows [0, R) of one or two fp32 [R][128] matrices (contiguous rows) as hi/lo pairs of sw128
+// tiles, all of a thread's loads issued before its first store (256 threads).
+template <int R>
+__device__ __forceinline__ void kt_split_rows(unsigned char* hi0, unsigned char* lo0, const float* src0,
+                                              unsigned char* hi1, unsigned char* lo1, const float* src1) {
+  constexpr int N = R * 16 / 256;
+  float4 r[4 * N];
+#pragma unroll
+  for (int m = 0; m < N; ++m) {
+    const int x = threadIdx.x + 256 * m, row = x >> 4, j = x & 15;
+    const float4* p0 = reinterpret_cast<const float4*>(src0 + row * 128 + 8 * j);
+    r[4 * m] = __ldg(p0);
+    r[4 * m + 1] = __ldg(p0 + 1);
+    if (src1) {
+      const float4* p1 = reinterpret_cast<const float4*>(src1 + row * 128 + 8 * j);
+      r[4 * m + 2] = __ldg(p1);
+      r[4 * m + 3] = __ldg(p1 + 1);
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < N; ++m) {
+    const int x = threadIdx.x + 256 * m, row = x >> 4, j = x & 15;
+    const float f0[8] = {r[4 * m].x, r[4 * m].y, r[4 * m].z, r[4 * m].w,
+                         r[4 * m + 1].x, r[4 * m + 1].y, r[4 * m + 1].z, r[4 * m + 1].w};
+    tcx::st_chunk_split(hi0, lo0, row, j, R * 128, f0);
+    if (src1) {
+      const float f1[8] = {r[4 * m + 2].x, r[4 * m + 2].y, r[4 * m + 2].z, r[4 * m + 2].w,
+                           r[4 * m + 3].x, r[4 * m + 3].y, r[4 * m + 3].z, r[4 * m + 3].w};
+      tcx::st_chunk_split(hi1, lo1, row, j, R * 128, f1);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork w) {
   using namespace kf;
   if (kda_failed(w)) return;
@@ -783,6 +816,108 @@ __global__ void __launch_bounds__(256) k_kda_out(Problem p, Args a, KdaWork w) {
     o[(size_t)(x / V) * p.HV * V + x % V] = from_f<T>(p.scale * sO[x]);
 }
 
+// k_kda_out for bf16 with K = V = 128: O = scale (Q~ S^T + P U) on the tensor cores from
+// compensated bf16 pairs, one CTA per (chunk, value head); M = 64 tokens, N = V, TMEM [0, 128).
+namespace ko {
+using namespace tcx;
+constexpr int TT = 64 * 128, TS = 128 * 128;
+constexpr int O_QH = 0, O_QL = 16384, O_SH = 32768, O_SL = 65536, O_PH = 98304, O_PL = 106496;
+constexpr int O_UH = 114688, O_UL = 131072;
+constexpr int OUT_BYTES = O_UL + 16384;
+static_assert(1024 + OUT_BYTES <= 227 * 1024, "kda output shared memory");
+}  // namespace ko
+
+__global__ void __launch_bounds__(256, 1) k_kda_tc_out(Problem p, Args a, KdaWork w) {
+  using namespace ko;
+  if (kda_failed(w)) return;
+  const int gc = blockIdx.x, hv = blockIdx.y;
+  const int4 e = w.chunk_tab[gc];
+  if (e.x < 0) return;
+  constexpr int K = 128, V = 128;
+  const int L = e.z, tok0 = e.w, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  extern __shared__ unsigned char smraw[];
+  unsigned char* sm = align1k(smraw);
+  __shared__ uint64_t bar[1];
+  __shared__ uint32_t tslot;
+  int* err = w.status;
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tslot, 128);
+    tmem_relinquish();
+  }
+  const size_t u = (size_t)gc * p.HV + hv;
+  kt_split_rows<CH>(sm + O_QH, sm + O_QL, w.Qt + u * CH * K, sm + O_UH, sm + O_UL, w.U + u * CH * V);
+  kt_split_rows<128>(sm + O_SH, sm + O_SL, w.h + u * V * K, nullptr, nullptr, nullptr);
+  {  // P [64][64]
+    float4 r[4];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int x = tid + 256 * m, row = x >> 3, j = x & 7;
+      const float4* pp = reinterpret_cast<const float4*>(w.P + u * CH * CH + row * CH + 8 * j);
+      r[2 * m] = __ldg(pp);
+      r[2 * m + 1] = __ldg(pp + 1);
+    }
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int x = tid + 256 * m, row = x >> 3, j = x & 7;
+      const float f[8] = {r[2 * m].x, r[2 * m].y, r[2 * m].z, r[2 * m].w,
+                          r[2 * m + 1].x, r[2 * m + 1].y, r[2 * m + 1].z, r[2 * m + 1].w};
+      st_chunk_split(sm + O_PH, sm + O_PL, row, j, TT, f);
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tslot;
+  if (tid == 0) {
+    const uint32_t qh = smem_u32(sm + O_QH), ql = smem_u32(sm + O_QL), sh = smem_u32(sm + O_SH);
+    const uint32_t sl = smem_u32(sm + O_SL), ph = smem_u32(sm + O_PH), pl = smem_u32(sm + O_PL);
+    const uint32_t uh = smem_u32(sm + O_UH), ul = smem_u32(sm + O_UL);
+    constexpr uint32_t i_qs = idesc_bf16(64, 128, false, false), i_pu = idesc_bf16(64, 128, false, true);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {  // Q~ S^T
+      const uint64_t aq = desc_kmajor(qh, s, TT), bs = desc_kmajor(sh, s, TS);
+      mma_bf16(taddr(tb, 0, 0), aq, bs, i_qs, s > 0);
+      mma_bf16(taddr(tb, 0, 0), aq, desc_kmajor(sl, s, TS), i_qs, 1);
+      mma_bf16(taddr(tb, 0, 0), desc_kmajor(ql, s, TT), bs, i_qs, 1);
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {  // + P U
+      const uint64_t ap = desc_kmajor(ph, s, TT), bu = desc_mnmajor(uh, s, TT);
+      mma_bf16(taddr(tb, 0, 0), ap, bu, i_pu, 1);
+      mma_bf16(taddr(tb, 0, 0), ap, desc_mnmajor(ul, s, TT), i_pu, 1);
+      mma_bf16(taddr(tb, 0, 0), desc_kmajor(pl, s, TT), bu, i_pu, 1);
+    }
+    mma_commit(&bar[0]);
+  }
+  const bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
+  tc_fence_after();
+  if (ok) {
+    const int half = warp >> 2, r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
+    float x[32];
+    tmem_ld16dp_x8(taddr(tb, 32 * (warp & 3), 64 * half), x);
+    tmem_wait_ld();
+    bf16* o = static_cast<bf16*>(a.o) + ((size_t)tok0 * p.HV + hv) * V;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = 64 * half + 8 * j + cq;
+      if (r0 < L)
+        *reinterpret_cast<uint32_t*>(o + (size_t)r0 * p.HV * V + c) = pack_bf16(p.scale * x[4 * j], p.scale * x[4 * j + 1]);
+      if (r0 + 8 < L)
+        *reinterpret_cast<uint32_t*>(o + (size_t)(r0 + 8) * p.HV * V + c) =
+            pack_bf16(p.scale * x[4 * j + 2], p.scale * x[4 * j + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 128);
+}
+
 template <typename Kern>
 cudaError_t go(const char* name, Kern kern, dim3 grid, size_t smem, cudaStream_t s, const Problem& p,
                const Args& a, const KdaWork& w) {
@@ -802,7 +937,9 @@ cudaError_t forward_t(const Problem& p, const Args& a, const KdaWork& w, cudaStr
   if (e == cudaSuccess)
     e = tc ? go("kda_tc_scan", k_kda_tc_scan, dim3(p.Nst, p.HV), 1024 + ks::SCAN_BYTES, s, p, a, w)
            : go("kda_scan", k_kda_scan, dim3(p.Nst, p.HV, p.V / 32), scan_smem(p.K), s, p, a, w);
-  if (e == cudaSuccess) e = go("kda_out", k_kda_out<T>, dim3(p.NCmax, p.HV), out_smem(p.K, p.V), s, p, a, w);
+  if (e == cudaSuccess)
+    e = tc ? go("kda_tc_out", k_kda_tc_out, dim3(p.NCmax, p.HV), 1024 + ko::OUT_BYTES, s, p, a, w)
+           : go("kda_out", k_kda_out<T>, dim3(p.NCmax, p.HV), out_smem(p.K, p.V), s, p, a, w);
   return e;
 }
 

@@ -125,8 +125,9 @@ def test_empty_input_passes_the_gradient_through():
 
 
 def test_bf16_128_runs_the_tensor_core_kernels():
-    """bf16 with 128-wide heads takes the tcgen05 KDA kernels (the per-launch profile names
-    them) and still matches the oracle; fp32 and 64-wide heads keep the CUDA-core kernels."""
+    """bf16 with 128-wide heads takes the tcgen05 KDA kernels for every chunk step of the
+    forward and the backward (the per-launch profile names them, and none of the CUDA-core
+    ones) and still matches the oracle; fp32 and 64-wide heads keep the CUDA-core kernels."""
     import gated_deltanet_chunkwise_chunk_b200 as gdn
     case = synth.make_case(H=2, HV=4, K=128, V=128, dtype="bf16", seed=670,
                            lengths=[130, 0, 64, 5], h0=True, name="kda_tc_path")
@@ -137,7 +138,7 @@ def test_bf16_128_runs_the_tensor_core_kernels():
         names = set(gdn.profile_read())
     finally:
         gdn.profile(False)
-    for k in ("kda_tc_wy", "kda_tc_scan", "kda_tc_bwd_scan", "kda_tc_bwd_dqk", "kda_tc_bwd_wy"):
-        assert k in names, (k, names)
-    for k in ("kda_wy", "kda_scan", "kda_bwd_scan", "kda_bwd_dqk", "kda_bwd_wy"):
-        assert k not in names, (k, names)
+    steps = ("wy", "scan", "out", "bwd_scan", "bwd_dqk", "bwd_wy")
+    for k in steps:
+        assert f"kda_tc_{k}" in names, (k, names)
+        assert f"kda_{k}" not in names, (k, names)
