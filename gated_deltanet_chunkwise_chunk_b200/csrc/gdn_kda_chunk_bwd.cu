@@ -296,38 +296,41 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
 #pragma unroll
       for (int j = 0; j < 8; ++j) st_chunk_split(sm + O_SH, sm + O_SL, v, 8 * half + j, TS, S + 8 * j);
     }
-    {  // scale P, K^, scale Q~, -W as hi/lo tiles; dO (bf16, rows past L zero)
+    {  // scale P, K^ as hi/lo tiles; dO (bf16, rows past L zero)
       const float* gK = w.Kh + u * CH * K;
-      const float* gQ = w.Qt + u * CH * K;
-      const float* gW = w.W + u * CH * K;
       const float* gP = w.P + u * CH * CH;
+      float4 rk[8], rp[4];
+      uint4 rd[4];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int x = tid + 256 * m, row = x >> 4, j = x & 15;
         const float4* pk = reinterpret_cast<const float4*>(gK + row * K + 8 * j);
-        const float4* pq = reinterpret_cast<const float4*>(gQ + row * K + 8 * j);
-        const float4* pw = reinterpret_cast<const float4*>(gW + row * K + 8 * j);
-        const float4 k0 = __ldg(pk), k1 = __ldg(pk + 1), q0 = __ldg(pq), q1 = __ldg(pq + 1);
-        const float4 w0 = __ldg(pw), w1 = __ldg(pw + 1);
-        const uint4 dd = row < e.z ? __ldg(reinterpret_cast<const uint4*>(
-                                         dO + ((size_t)(e.w + row) * p.HV + hv) * V + 8 * j))
-                                   : make_uint4(0u, 0u, 0u, 0u);
-        const float fk[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-        const float sc = p.scale;
-        const float fq[8] = {sc * q0.x, sc * q0.y, sc * q0.z, sc * q0.w, sc * q1.x, sc * q1.y, sc * q1.z, sc * q1.w};
-        const float fw[8] = {-w0.x, -w0.y, -w0.z, -w0.w, -w1.x, -w1.y, -w1.z, -w1.w};
-        st_chunk_split(sm + O_KH, sm + O_KL, row, j, TT, fk);
-        st_chunk_split(sm + O_QH, sm + O_QL, row, j, TT, fq);
-        st_chunk_split(sm + O_WH, sm + O_WL, row, j, TT, fw);
-        *reinterpret_cast<uint4*>(sm + O_DO + sw128_chunk(row, j, TT)) = dd;
+        rk[2 * m] = __ldg(pk);
+        rk[2 * m + 1] = __ldg(pk + 1);
+        rd[m] = row < e.z ? __ldg(reinterpret_cast<const uint4*>(dO + ((size_t)(e.w + row) * p.HV + hv) * V + 8 * j))
+                          : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int m = 0; m < 2; ++m) {
         const int x = tid + 256 * m, row = x >> 3, j = x & 7;
         const float4* pp = reinterpret_cast<const float4*>(gP + row * CH + 8 * j);
-        const float4 p0 = __ldg(pp), p1 = __ldg(pp + 1);
-        const float sc = p.scale;
-        const float f[8] = {sc * p0.x, sc * p0.y, sc * p0.z, sc * p0.w, sc * p1.x, sc * p1.y, sc * p1.z, sc * p1.w};
+        rp[2 * m] = __ldg(pp);
+        rp[2 * m + 1] = __ldg(pp + 1);
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+        const float fk[8] = {rk[2 * m].x, rk[2 * m].y, rk[2 * m].z, rk[2 * m].w,
+                             rk[2 * m + 1].x, rk[2 * m + 1].y, rk[2 * m + 1].z, rk[2 * m + 1].w};
+        st_chunk_split(sm + O_KH, sm + O_KL, row, j, TT, fk);
+        *reinterpret_cast<uint4*>(sm + O_DO + sw128_chunk(row, j, TT)) = rd[m];
+      }
+      const float sc = p.scale;
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int x = tid + 256 * m, row = x >> 3, j = x & 7;
+        const float f[8] = {sc * rp[2 * m].x, sc * rp[2 * m].y, sc * rp[2 * m].z, sc * rp[2 * m].w,
+                            sc * rp[2 * m + 1].x, sc * rp[2 * m + 1].y, sc * rp[2 * m + 1].z, sc * rp[2 * m + 1].w};
         st_chunk_split(sm + O_PH, sm + O_PL, row, j, TT, f);
       }
     }
@@ -355,6 +358,32 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
         mma_bf16(taddr(tb, 0, 0), desc_kmajor(kl, s, TT), bs, i_ks, 1);
       }
       mma_commit(&bar[0]);
+    }
+    {  // while they run: scale Q~ and -W as hi/lo tiles (read by the second products only)
+      const float* gQ = w.Qt + u * CH * K;
+      const float* gW = w.W + u * CH * K;
+      float4 rq[8], rw[8];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+        const float4* pq = reinterpret_cast<const float4*>(gQ + row * K + 8 * j);
+        const float4* pw = reinterpret_cast<const float4*>(gW + row * K + 8 * j);
+        rq[2 * m] = __ldg(pq);
+        rq[2 * m + 1] = __ldg(pq + 1);
+        rw[2 * m] = __ldg(pw);
+        rw[2 * m + 1] = __ldg(pw + 1);
+      }
+      const float sc = p.scale;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+        const float fq[8] = {sc * rq[2 * m].x, sc * rq[2 * m].y, sc * rq[2 * m].z, sc * rq[2 * m].w,
+                             sc * rq[2 * m + 1].x, sc * rq[2 * m + 1].y, sc * rq[2 * m + 1].z, sc * rq[2 * m + 1].w};
+        const float fw[8] = {-rw[2 * m].x, -rw[2 * m].y, -rw[2 * m].z, -rw[2 * m].w,
+                             -rw[2 * m + 1].x, -rw[2 * m + 1].y, -rw[2 * m + 1].z, -rw[2 * m + 1].w};
+        st_chunk_split(sm + O_QH, sm + O_QL, row, j, TT, fq);
+        st_chunk_split(sm + O_WH, sm + O_WL, row, j, TT, fw);
+      }
     }
     ok = __syncthreads_and(mbar_wait(&bar[0], k & 1, err));
     tc_fence_after();
