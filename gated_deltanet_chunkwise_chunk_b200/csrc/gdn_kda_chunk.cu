@@ -377,24 +377,60 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork
     }
     mma_commit(&bar[0]);
   }
-  // diagonal sub-blocks, one warp per pair (i, j), j <= i in one sub-chunk, lanes over channels
-  constexpr int PAIRS = SUB * (SUB + 1) / 2;
-  for (int pr = warp; pr < (CH / SUB) * PAIRS; pr += 8) {
-    const int blk = pr / PAIRS;
-    int q = pr % PAIRS, ii = 0;
-    while (q > ii) q -= ++ii;  // q in [0, ii]
-    const int i = blk * SUB + ii, j = blk * SUB + q;
-    float sa = 0.f, sp = 0.f;
-    for (int c = lane; c < K; c += 32) {
-      const float kj = __bfloat162float(sK[j * K + c]) * exp2f(sG[i * K + c] - sG[j * K + c]);
-      sa = fmaf(__bfloat162float(sK[i * K + c]), kj, sa);
-      sp = fmaf(__bfloat162float(sQ[i * K + c]), kj, sp);
+  // diagonal sub-blocks by row: warp w takes rows w, w + 8, ..; lane l the channels 4l..4l+3.  A
+  // row's 16 A and 16 P partial sums (columns j of its sub-chunk, zero for j > i) are summed over
+  // the lanes by one butterfly reduce-scatter (31 shuffles), after which lane l holds column l
+  // of A (l < 16) or l - 16 of P.
+  for (int i = warp; i < CH; i += 8) {
+    const int b0 = i & ~(SUB - 1), c = 4 * lane;
+    float ki[4], qi[4], gi[4];
+    {
+      const float4 g4 = *reinterpret_cast<const float4*>(sG + i * K + c);
+      const uint2 k2 = *reinterpret_cast<const uint2*>(sK + i * K + c);
+      const uint2 q2 = *reinterpret_cast<const uint2*>(sQ + i * K + c);
+      const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&k2.x));
+      const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&k2.y));
+      const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q2.x));
+      const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q2.y));
+      ki[0] = k01.x; ki[1] = k01.y; ki[2] = k23.x; ki[3] = k23.y;
+      qi[0] = q01.x; qi[1] = q01.y; qi[2] = q23.x; qi[3] = q23.y;
+      gi[0] = g4.x; gi[1] = g4.y; gi[2] = g4.z; gi[3] = g4.w;
     }
-    sa = warp_total(sa);
-    sp = warp_total(sp);
-    if (lane == 0) {
-      sDA[(blk * SUB + ii) * SUB + q] = j < i ? sb[i] * sa : 0.f;
-      sDP[(blk * SUB + ii) * SUB + q] = sp;
+    float v[2 * SUB];
+#pragma unroll
+    for (int jj = 0; jj < SUB; ++jj) {
+      const int j = b0 + jj;
+      float sa = 0.f, sp = 0.f;
+      if (j <= i) {
+        const float4 g4 = *reinterpret_cast<const float4*>(sG + j * K + c);
+        const uint2 k2 = *reinterpret_cast<const uint2*>(sK + j * K + c);
+        const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&k2.x));
+        const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&k2.y));
+        const float kj[4] = {k01.x, k01.y, k23.x, k23.y}, gj[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float kk = kj[q] * exp2f(gi[q] - gj[q]);
+          sa = fmaf(ki[q], kk, sa);
+          sp = fmaf(qi[q], kk, sp);
+        }
+      }
+      v[jj] = sa;
+      v[SUB + jj] = sp;
+    }
+#pragma unroll
+    for (int off = 16, n = 2 * SUB; off > 0; off >>= 1, n >>= 1) {
+      const bool up = (lane & off) != 0;
+#pragma unroll
+      for (int x = 0; x < n / 2; ++x) {
+        const float keep = up ? v[x + n / 2] : v[x], give = up ? v[x] : v[x + n / 2];
+        v[x] = keep + __shfl_xor_sync(0xffffffffu, give, off);
+      }
+    }
+    const int jj = lane & (SUB - 1), j = b0 + jj;
+    if (lane < SUB) {
+      if (j <= i) sDA[i * SUB + jj] = j < i ? sb[i] * v[0] : 0.f;
+    } else if (j <= i) {
+      sDP[i * SUB + jj] = v[0];
     }
   }
   bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
