@@ -91,16 +91,30 @@ __device__ void gated_products(const float* Wt, int ldw, const TR* R, const TR* 
   }
 }
 
-// The same products for K = 128 and 256 threads, by channel: thread t owns channel c = t % 128,
-// with its operands in registers.  The diagonal sub-blocks: thread (c, t / 128) takes sub-chunks
-// 2 (t / 128) and 2 (t / 128) + 1, one exponential per pair (i, j) serving both F and G.  The
-// blocks below the diagonal, for each sub-chunk a through r = 16 a - 1: the threads t < 128 form
-// F of a's rows (16 independent accumulators, one pass over the columns j), the others G of the
-// columns before a; the two write disjoint rows of each channel.  The loops over j stay rolled
-// (a fully unrolled form overflows the instruction cache).  Results go to the sinks as above;
-// ends with a barrier.
+// The same products for K = 128 and 256 threads, by channel, with the weights stored transposed
+// (WtT[j * LDT + i] = Wt_ij, rows 16-byte aligned, so that the 16 weights of a column j within a
+// sub-chunk are four 128-bit loads): thread t owns channel c = t % 128, its operands in
+// registers.  The diagonal sub-blocks: thread (c, t / 128) takes sub-chunks 2 (t / 128) and
+// 2 (t / 128) + 1, one exponential per pair (i, j) serving both F and G.  The blocks below the
+// diagonal, for each sub-chunk a through r = 16 a - 1: the threads t < 128 form F of a's rows
+// (16 independent accumulators, one pass over the columns j), the others G of the columns before
+// a; the two write disjoint rows of each channel.  The loops over j stay rolled (a fully unrolled
+// form overflows the instruction cache).  Results go to the sinks as above; ends with a barrier.
+constexpr int LDT = CH + 4;
+
+__device__ __forceinline__ void ld16(const float* p, float* w) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 x = reinterpret_cast<const float4*>(p)[q];
+    w[4 * q] = x.x;
+    w[4 * q + 1] = x.y;
+    w[4 * q + 2] = x.z;
+    w[4 * q + 3] = x.w;
+  }
+}
+
 template <typename TR, typename SinkF, typename SinkG>
-__device__ __forceinline__ void gated_below(int A, const float* Wt, int ldw, const TR* R, const TR* Lm,
+__device__ __forceinline__ void gated_below(int A, const float* WtT, const TR* R, const TR* Lm,
                                             const float* colw, const float* G2, int c, bool rows,
                                             SinkF& sinkF, SinkG& sinkG) {
   constexpr int K = 128;
@@ -113,8 +127,10 @@ __device__ __forceinline__ void gated_below(int A, const float* Wt, int ldw, con
 #pragma unroll 2
     for (int j = 0; j < NJ; ++j) {
       const float rt = ldf(R + j * K + c) * exp2f(gr - G2[j * K + c]);
+      float wv[SUB];
+      ld16(WtT + j * LDT + I0, wv);
 #pragma unroll
-      for (int i = 0; i < SUB; ++i) acc[i] = fmaf(Wt[(I0 + i) * ldw + j], rt, acc[i]);
+      for (int i = 0; i < SUB; ++i) acc[i] = fmaf(wv[i], rt, acc[i]);
     }
 #pragma unroll
     for (int i = 0; i < SUB; ++i) sinkF(I0 + i, c, acc[i] * exp2f(G2[(I0 + i) * K + c] - gr));
@@ -125,13 +141,15 @@ __device__ __forceinline__ void gated_below(int A, const float* Wt, int ldw, con
       ls[i] = (colw ? colw[I0 + i] : 1.f) * ldf(Lm + (I0 + i) * K + c) * exp2f(G2[(I0 + i) * K + c] - gr);
 #pragma unroll 2
     for (int j = 0; j < NJ; ++j) {
+      float wv[SUB];
+      ld16(WtT + j * LDT + I0, wv);
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
       for (int i = 0; i < SUB; i += 4) {
-        a0 = fmaf(Wt[(I0 + i) * ldw + j], ls[i], a0);
-        a1 = fmaf(Wt[(I0 + i + 1) * ldw + j], ls[i + 1], a1);
-        a2 = fmaf(Wt[(I0 + i + 2) * ldw + j], ls[i + 2], a2);
-        a3 = fmaf(Wt[(I0 + i + 3) * ldw + j], ls[i + 3], a3);
+        a0 = fmaf(wv[i], ls[i], a0);
+        a1 = fmaf(wv[i + 1], ls[i + 1], a1);
+        a2 = fmaf(wv[i + 2], ls[i + 2], a2);
+        a3 = fmaf(wv[i + 3], ls[i + 3], a3);
       }
       sinkG(j, c, ((a0 + a1) + (a2 + a3)) * exp2f(gr - G2[j * K + c]));
     }
@@ -139,7 +157,7 @@ __device__ __forceinline__ void gated_below(int A, const float* Wt, int ldw, con
 }
 
 template <typename TR, typename SinkF, typename SinkG>
-__device__ void gated_products_k128(const float* Wt, int ldw, const TR* R, const TR* Lm, const float* colw,
+__device__ void gated_products_k128(const float* WtT, const TR* R, const TR* Lm, const float* colw,
                                     const float* G2, SinkF sinkF, SinkG sinkG) {
   constexpr int K = 128;
   const int c = threadIdx.x & 127, hi = threadIdx.x >> 7;
@@ -155,13 +173,16 @@ __device__ void gated_products_k128(const float* Wt, int ldw, const TR* R, const
       F[j] = G[j] = 0.f;
     }
 #pragma unroll
-    for (int i = 0; i < SUB; ++i)
+    for (int j = 0; j < SUB; ++j) {
+      float wv[SUB];
+      ld16(WtT + (b0 + j) * LDT + b0, wv);
 #pragma unroll
-      for (int j = 0; j <= i; ++j) {
-        const float wt = Wt[(b0 + i) * ldw + b0 + j] * exp2f(g[i] - g[j]);
+      for (int i = j; i < SUB; ++i) {
+        const float wt = wv[i] * exp2f(g[i] - g[j]);
         F[i] = fmaf(wt, r[j], F[i]);
         G[j] = fmaf(wt, l[i], G[j]);
       }
+    }
 #pragma unroll
     for (int i = 0; i < SUB; ++i) {
       sinkF(b0 + i, c, F[i]);
@@ -171,7 +192,7 @@ __device__ void gated_products_k128(const float* Wt, int ldw, const TR* R, const
 #pragma unroll 1
   for (int A = 1; A < CH / SUB; ++A) {
     __syncthreads();
-    gated_below(A, Wt, ldw, R, Lm, colw, G2, c, hi == 0, sinkF, sinkG);
+    gated_below(A, WtT, R, Lm, colw, G2, c, hi == 0, sinkF, sinkG);
   }
   __syncthreads();
 }
@@ -562,8 +583,8 @@ constexpr int O_SH = 81920, O_SL = 114688;                  // S, then dS' (hi, 
 // accumulated in shared memory and written out once), q and k (bf16 [64][128], rows past the
 // chunk zero) and the gated products' scratch (fp32 [64][128])
 constexpr int O_ACQ = 0, O_ACK = 32768, O_ACG = 65536, O_QB = 98304, O_KB = 114688, O_SCR = 131072;
-constexpr int O_DP = 163840;                                // fp32 [64][LDP]
-constexpr int O_G = O_DP + CH * LDP * 4;                    // fp32 [64][128] Gam * log2(e)
+constexpr int O_DP = 163840;                                // fp32 dP^T [64][LDT]
+constexpr int O_G = O_DP + CH * LDT * 4;                    // fp32 [64][128] Gam * log2(e)
 constexpr int O_RED = O_G + CH * 128 * 4;                   // fp32 [16][128]
 constexpr int O_GC = O_RED + 16 * 128 * 4;                  // fp32 [128]
 constexpr int DQK_BYTES = O_GC + 128 * 4;
@@ -756,7 +777,7 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, Kd
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int i = r0 + 8 * (q >> 1), c = 32 * half + 8 * j + cq + (q & 1);
-        sdP[i * LDP + c] = c <= i ? p.scale * d[4 * j + q] : 0.f;
+        sdP[c * LDT + i] = c <= i ? p.scale * d[4 * j + q] : 0.f;
       }
     float* dW = w.dW + uk;
 #pragma unroll
@@ -836,7 +857,7 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, Kd
     acg[(CH - 1) * K + tid] += sGC[tid] + sred[tid] + sred[128 + tid] + sred[256 + tid] + sred[384 + tid];
   __syncthreads();
   if (ok)  // P_ij = sum_c q_i k_j e^{Gam_i - Gam_j}: dq += F2, dk += G2, dGam += q F2 - k G2
-    gated_products_k128(sdP, LDP, sK, sQ, nullptr, sG,
+    gated_products_k128(sdP, sK, sQ, nullptr, sG,
                    [&](int i, int c, float f) {
                      acq[i * K + c] += f;
                      acg[i * K + c] += __bfloat162float(sQ[i * K + c]) * f;
@@ -1040,7 +1061,7 @@ constexpr int O_TH = O_B, O_TL = O_B + 8192, O_DTH = O_B + 16384, O_DTL = O_B + 
 constexpr int O_ZH = O_B + 32768, O_ZL = O_B + 40960;
 constexpr int O_DA = O_B;
 constexpr int WY_BYTES = O_B + 49152;
-static_assert(CH * LDP * 4 <= 49152, "dA fits region B");
+static_assert(CH * LDT * 4 <= 49152, "dA fits region B");
 static_assert(1024 + WY_BYTES <= 227 * 1024, "wy_bwd shared memory");
 }  // namespace kw
 
@@ -1284,13 +1305,13 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_wy(Problem p, Args a, Kda
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int i = r0 + 8 * (q >> 1), c = 32 * half + 8 * j + cq + (q & 1);
-        sdA[i * LDP + c] = c < i ? -d[4 * j + q] : 0.f;
+        sdA[c * LDT + i] = c < i ? -d[4 * j + q] : 0.f;
       }
   }
   __syncthreads();
   // A_ij = beta_i sum_c k_i k_j e^{Gam_i - Gam_j}: F1 (rows, weights dA), G1 (columns, beta_i dA)
   if (ok)
-    gated_products_k128(sdA, LDP, sK, sK, sb, sG,
+    gated_products_k128(sdA, sK, sK, sb, sG,
                         [&](int i, int c, float f) { sF1[i * K + c] += f; },
                         [&](int j, int c, float g) {
                           ack[j * K + c] += g;
