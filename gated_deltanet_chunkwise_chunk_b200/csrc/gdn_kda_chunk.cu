@@ -639,17 +639,18 @@ __global__ void __launch_bounds__(256) k_kda_scan(Problem p, Args a, KdaWork w) 
     }
 }
 
-// k_kda_scan for bf16 with K = V = 128: one CTA per (sequence, value head) holds the whole
-// state S [V][K] in fp32 registers (thread: row v = 32 (warp % 4) + lane, columns 64 (warp / 4)..)
-// and takes both products of a chunk on the tensor cores, from compensated bf16 pairs:
-//   U = U~ - W S^T        (M = 64 tokens, N = V;  A = W, B = S, K-major)       TMEM [0, 128)
-//   S' = S Diag(e^{Gam_C}) + U^T K^   (M = V, N = K;  A = U^T, B = K^, MN-major)  TMEM [128, 256)
+// k_kda_scan for bf16 with K = V = 128: two CTAs per (sequence, value head), each holding half of
+// the state's rows (v in [64 z, 64 z + 64), z = blockIdx.z) in fp32 registers in the layout of an
+// M = 64 accumulator (thread: rows r0 and r0 + 8 of its sub-partition, columns 8j + cq + {0, 1}
+// of its warp half), both products of a chunk on the tensor cores from compensated bf16 pairs:
+//   U[:, z] = U~[:, z] - W S_z^T        (M = 64 tokens, N = 64;  A = W, B = S_z, K-major)   TMEM [0, 64)
+//   S_z' = S_z Diag(e^{Gam_C}) + U[:, z]^T K^   (M = 64, N = K;  A = U^T, B = K^, MN-major) TMEM [128, 256)
 // It stores the state entering every chunk and U, as k_kda_scan does.
 namespace ks {
 using namespace tcx;
-constexpr int TT = 64 * 128, TS = 128 * 128;
-constexpr int O_WH = 0, O_WL = 16384, O_KH = 32768, O_KL = 49152, O_UH = 65536, O_UL = 81920;
-constexpr int O_SH = 98304, O_SL = 131072, O_E = 163840;
+constexpr int TT = 64 * 128;
+constexpr int O_WH = 0, O_WL = 16384, O_KH = 32768, O_KL = 49152, O_UH = 65536, O_UL = 73728;
+constexpr int O_SH = 81920, O_SL = 98304, O_E = 114688;
 constexpr int SCAN_BYTES = O_E + 512;
 static_assert(1024 + SCAN_BYTES <= 227 * 1024, "kda scan shared memory");
 }  // namespace ks
@@ -657,12 +658,13 @@ static_assert(1024 + SCAN_BYTES <= 227 * 1024, "kda scan shared memory");
 __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWork w) {
   using namespace ks;
   if (kda_failed(w)) return;
-  const int n = blockIdx.x, hv = blockIdx.y;
+  const int n = blockIdx.x, hv = blockIdx.y, z = blockIdx.z;
   const int4 sq = w.seq_tab[n];
   constexpr int K = 128, V = 128;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int half = warp >> 2, v = 32 * (warp & 3) + lane, c0 = 64 * half;
-  const int r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);  // 16-lane (M = 64) view
+  const int half = warp >> 2, sub = 32 * (warp & 3);
+  const int r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
+  const int v0 = 64 * z;
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
   float* sE = reinterpret_cast<float*>(sm + O_E);
@@ -679,11 +681,17 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
     tmem_alloc(&tslot, 256);
     tmem_relinquish();
   }
-  float S[64];
+  // S[4j + q]: row v0 + r0 + 8 (q >> 1), column 64 half + 8j + cq + (q & 1)
+  float S[32];
   {
     const float* h0 = a.h0 ? a.h0 + ((size_t)n * p.HV + hv) * K * V : nullptr;
 #pragma unroll
-    for (int c = 0; c < 64; ++c) S[c] = h0 ? h0[(size_t)(c0 + c) * V + v] : 0.f;
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int r = v0 + r0 + 8 * (q >> 1), c = 64 * half + 8 * j + cq + (q & 1);
+        S[4 * j + q] = h0 ? h0[(size_t)c * V + r] : 0.f;
+      }
   }
   tc_fence_before();
   __syncthreads();
@@ -695,14 +703,18 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
   bool ok = true;
   for (int ci = 0; ci < sq.y && ok; ++ci) {
     const size_t u = (size_t)(sq.x + ci) * p.HV + hv;
-    {  // the state entering the chunk: stored, and as a hi/lo tile
-      float4* h = reinterpret_cast<float4*>(w.h + u * V * K + (size_t)v * K + c0);
+    {  // this half of the state entering the chunk: stored, and as a hi/lo tile [64 v][128 k]
+      float* h = w.h + u * V * K + (size_t)v0 * K;
 #pragma unroll
-      for (int q = 0; q < 16; ++q) h[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) st_chunk_split(sm + O_SH, sm + O_SL, v, 8 * half + j, TS, S + 8 * j);
+      for (int j = 0; j < 8; ++j) {
+        const int c = 64 * half + 8 * j + cq;
+        *reinterpret_cast<float2*>(h + r0 * K + c) = make_float2(S[4 * j], S[4 * j + 1]);
+        *reinterpret_cast<float2*>(h + (r0 + 8) * K + c) = make_float2(S[4 * j + 2], S[4 * j + 3]);
+        st_pair_split(sm + O_SH, sm + O_SL, r0, c, TT, S[4 * j], S[4 * j + 1]);
+        st_pair_split(sm + O_SH, sm + O_SL, r0 + 8, c, TT, S[4 * j + 2], S[4 * j + 3]);
+      }
     }
-    {  // W and K^ as hi/lo tiles, e^{Gam_C}
+    {  // W and K^ as hi/lo tiles
       const float* gW = w.W + u * CH * K;
       const float* gK = w.Kh + u * CH * K;
       float4 rw[8], rk[8];
@@ -731,13 +743,13 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid == 0) {  // W S^T
-      constexpr uint32_t id = idesc_bf16(64, 128, false, false);
+    if (tid == 0) {  // W S_z^T
+      constexpr uint32_t id = idesc_bf16(64, 64, false, false);
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        const uint64_t wh = desc_kmajor(aWH, s, TT), sh = desc_kmajor(aSH, s, TS);
+        const uint64_t wh = desc_kmajor(aWH, s, TT), sh = desc_kmajor(aSH, s, TT);
         mma_bf16(taddr(tb, 0, 0), wh, sh, id, s > 0);
-        mma_bf16(taddr(tb, 0, 0), wh, desc_kmajor(aSL, s, TS), id, 1);
+        mma_bf16(taddr(tb, 0, 0), wh, desc_kmajor(aSL, s, TT), id, 1);
         mma_bf16(taddr(tb, 0, 0), desc_kmajor(aWL, s, TT), sh, id, 1);
       }
       mma_commit(&bar[0]);
@@ -745,12 +757,12 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
     // e^{Gam_C} for the state update (into shared memory once every thread is past the last
     // chunk's update)
     const float egc = tid < K ? w.eGC[u * K + tid] : 0.f;
-    float ut[32];  // U~ at this thread's (row, column) pairs of the 16-lane view
+    float ut[16];  // U~ at this thread's (token, value) pairs of the M = 64, N = 64 accumulator
     {
-      const float* gU = w.Ut + u * CH * V;
+      const float* gU = w.Ut + u * CH * V + v0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = c0 + 8 * j + cq;
+      for (int j = 0; j < 4; ++j) {
+        const int c = 32 * half + 8 * j + cq;
         const float2 a0 = *reinterpret_cast<const float2*>(gU + r0 * V + c);
         const float2 a1 = *reinterpret_cast<const float2*>(gU + (r0 + 8) * V + c);
         ut[4 * j] = a0.x;
@@ -762,14 +774,14 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
     ok = __syncthreads_and(mbar_wait(&bar[0], ci & 1, err));
     tc_fence_after();
     if (tid < K) sE[tid] = egc;
-    if (ok) {  // U = U~ - W S^T: stored, and as a hi/lo tile
-      float x[32];
-      tmem_ld16dp_x8(taddr(tb, 32 * (warp & 3), c0), x);
+    if (ok) {  // U = U~ - W S^T for this half's values: stored, and as a hi/lo tile [64 tok][64 v]
+      float x[16];
+      tmem_ld16dp_x4(taddr(tb, sub, 32 * half), x);
       tmem_wait_ld();
-      float* gU = w.U + u * CH * V;
+      float* gU = w.U + u * CH * V + v0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = c0 + 8 * j + cq;
+      for (int j = 0; j < 4; ++j) {
+        const int c = 32 * half + 8 * j + cq;
         const float u0 = ut[4 * j] - x[4 * j], u1 = ut[4 * j + 1] - x[4 * j + 1];
         const float u2 = ut[4 * j + 2] - x[4 * j + 2], u3 = ut[4 * j + 3] - x[4 * j + 3];
         *reinterpret_cast<float2*>(gU + r0 * V + c) = make_float2(u0, u1);
@@ -782,8 +794,8 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (ok && tid == 0) {  // U^T K^
-      constexpr uint32_t id = idesc_bf16(128, 128, true, true);
+    if (ok && tid == 0) {  // U[:, z]^T K^
+      constexpr uint32_t id = idesc_bf16(64, 128, true, true);
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
         const uint64_t uh = desc_mnmajor(aUH, s, TT), kh = desc_mnmajor(aKH, s, TT);
@@ -795,18 +807,26 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
     }
     ok = __syncthreads_and(ok && mbar_wait(&bar[1], ci & 1, err));
     tc_fence_after();
-    if (ok) {  // S = S Diag(e^{Gam_C}) + U^T K^  (lane = row v, this half's 64 columns)
-      float x[64];
-      tmem_ld64(taddr(tb, 32 * (warp & 3), 128 + c0), x);
+    if (ok) {  // S = S Diag(e^{Gam_C}) + U^T K^
+      float x[32];
+      tmem_ld16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 64; ++c) S[c] = fmaf(S[c], sE[c0 + c], x[c]);
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          S[4 * j + q] = fmaf(S[4 * j + q], sE[64 * half + 8 * j + cq + (q & 1)], x[4 * j + q]);
     }
   }
   if (ok && a.ht) {
     float* ht = a.ht + ((size_t)n * p.HV + hv) * K * V;
 #pragma unroll
-    for (int c = 0; c < 64; ++c) ht[(size_t)(c0 + c) * V + v] = S[c];
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int r = v0 + r0 + 8 * (q >> 1), c = 64 * half + 8 * j + cq + (q & 1);
+        ht[(size_t)c * V + r] = S[4 * j + q];
+      }
   }
   tc_fence_before();
   __syncthreads();
@@ -971,7 +991,7 @@ cudaError_t forward_t(const Problem& p, const Args& a, const KdaWork& w, cudaStr
   cudaError_t e = tc ? go("kda_tc_wy", k_kda_tc_wy, dim3(p.NCmax, p.HV), 1024 + kf::WYF_BYTES, s, p, a, w)
                      : go("kda_wy", k_kda_wy<T>, dim3(p.NCmax, p.HV), wy_smem(p.K, p.V), s, p, a, w);
   if (e == cudaSuccess)
-    e = tc ? go("kda_tc_scan", k_kda_tc_scan, dim3(p.Nst, p.HV), 1024 + ks::SCAN_BYTES, s, p, a, w)
+    e = tc ? go("kda_tc_scan", k_kda_tc_scan, dim3(p.Nst, p.HV, 2), 1024 + ks::SCAN_BYTES, s, p, a, w)
            : go("kda_scan", k_kda_scan, dim3(p.Nst, p.HV, p.V / 32), scan_smem(p.K), s, p, a, w);
   if (e == cudaSuccess)
     e = tc ? go("kda_tc_out", k_kda_tc_out, dim3(p.NCmax, p.HV), 1024 + ko::OUT_BYTES, s, p, a, w)

@@ -254,17 +254,17 @@ __global__ void __launch_bounds__(256) k_kda_bwd_scan(Problem p, Args a, KdaWork
 }
 
 // ---------------------------------------------------------------- reverse state scan, tcgen05
-// k_kda_bwd_scan for bf16 with K = V = 128: one CTA per (sequence, value head) holds dS [V][K] in
-// fp32 registers (thread: row v = 32 (warp % 4) + lane, columns 64 (warp / 4)..) and takes both
-// products of a chunk on the tensor cores (compensated bf16 pairs; dO is bf16 already):
-//   dU = (scale P)^T dO + K^ dS'^T                 (M = 64 tokens, N = V)   TMEM [0, 128)
-//   dS = dS' Diag(e^{Gam_C}) + dO^T (scale Q~) + dU^T (-W)   (M = V, N = K)  TMEM [128, 256)
+// k_kda_bwd_scan for bf16 with K = V = 128: two CTAs per (sequence, value head), each holding half
+// of dS's rows (v in [64 z, 64 z + 64)) in fp32 registers in the layout of an M = 64 accumulator,
+// both products of a chunk on the tensor cores (compensated bf16 pairs; dO is bf16 already):
+//   dU[:, z] = (scale P)^T dO[:, z] + K^ dS'_z^T                  (M = 64 tokens, N = 64)  TMEM [0, 64)
+//   dS_z = dS'_z Diag(e^{Gam_C}) + dO[:, z]^T (scale Q~) + dU[:, z]^T (-W)   (M = 64, N = K)  TMEM [128, 256)
 namespace kb {
 using namespace tcx;
-constexpr int TT = 64 * 128, TS = 128 * 128;
-constexpr int O_PH = 0, O_PL = 8192, O_DO = 16384, O_KH = 32768, O_KL = 49152, O_QH = 65536;
-constexpr int O_QL = 81920, O_WH = 98304, O_WL = 114688, O_UH = 131072, O_UL = 147456;
-constexpr int O_SH = 163840, O_SL = 196608, O_E = 229376;
+constexpr int TT = 64 * 128;
+constexpr int O_PH = 0, O_PL = 8192, O_DO = 16384, O_KH = 24576, O_KL = 40960, O_QH = 57344;
+constexpr int O_QL = 73728, O_WH = 90112, O_WL = 106496, O_UH = 122880, O_UL = 131072;
+constexpr int O_SH = 139264, O_SL = 155648, O_E = 172032;
 constexpr int BSCAN_BYTES = O_E + 512;
 static_assert(1024 + BSCAN_BYTES <= 227 * 1024, "kda backward scan shared memory");
 }  // namespace kb
@@ -272,12 +272,13 @@ static_assert(1024 + BSCAN_BYTES <= 227 * 1024, "kda backward scan shared memory
 __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, KdaWork w) {
   using namespace kb;
   if (kda_failed(w)) return;
-  const int n = blockIdx.x, hv = blockIdx.y;
+  const int n = blockIdx.x, hv = blockIdx.y, z = blockIdx.z;
   const int4 sq = w.seq_tab[n];
   constexpr int K = 128, V = 128;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int half = warp >> 2, v = 32 * (warp & 3) + lane, c0 = 64 * half;
+  const int half = warp >> 2, sub = 32 * (warp & 3);
   const int r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
+  const int v0 = 64 * z;
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
   float* sE = reinterpret_cast<float*>(sm + O_E);
@@ -294,11 +295,17 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
     tmem_alloc(&tslot, 256);
     tmem_relinquish();
   }
-  float S[64];  // dS, rows v, columns c0..c0+63
+  // S[4j + q]: dS at row v0 + r0 + 8 (q >> 1), column 64 half + 8j + cq + (q & 1)
+  float S[32];
   {
     const float* dht = a.dht ? a.dht + ((size_t)n * p.HV + hv) * K * V : nullptr;
 #pragma unroll
-    for (int c = 0; c < 64; ++c) S[c] = dht ? dht[(size_t)(c0 + c) * V + v] : 0.f;
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int r = v0 + r0 + 8 * (q >> 1), c = 64 * half + 8 * j + cq + (q & 1);
+        S[4 * j + q] = dht ? dht[(size_t)c * V + r] : 0.f;
+      }
   }
   tc_fence_before();
   __syncthreads();
@@ -310,30 +317,34 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
     const int ci = sq.y - 1 - k, gc = sq.x + ci;
     const int4 e = w.chunk_tab[gc];
     const size_t u = (size_t)gc * p.HV + hv;
-    {  // dS' (leaving the chunk): stored, and as a hi/lo tile
-      float4* dh = reinterpret_cast<float4*>(w.dh + u * V * K + (size_t)v * K + c0);
+    {  // this half of dS' (leaving the chunk): stored, and as a hi/lo tile [64 v][128 k]
+      float* dh = w.dh + u * V * K + (size_t)v0 * K;
 #pragma unroll
-      for (int q = 0; q < 16; ++q) dh[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) st_chunk_split(sm + O_SH, sm + O_SL, v, 8 * half + j, TS, S + 8 * j);
+      for (int j = 0; j < 8; ++j) {
+        const int c = 64 * half + 8 * j + cq;
+        *reinterpret_cast<float2*>(dh + r0 * K + c) = make_float2(S[4 * j], S[4 * j + 1]);
+        *reinterpret_cast<float2*>(dh + (r0 + 8) * K + c) = make_float2(S[4 * j + 2], S[4 * j + 3]);
+        st_pair_split(sm + O_SH, sm + O_SL, r0, c, TT, S[4 * j], S[4 * j + 1]);
+        st_pair_split(sm + O_SH, sm + O_SL, r0 + 8, c, TT, S[4 * j + 2], S[4 * j + 3]);
+      }
     }
-    {  // scale P, K^ as hi/lo tiles; dO (bf16, rows past L zero)
+    {  // scale P, K^ as hi/lo tiles; this half's dO columns (bf16, rows past L zero)
       const float* gK = w.Kh + u * CH * K;
       const float* gP = w.P + u * CH * CH;
       float4 rk[8], rp[4];
-      uint4 rd[4];
+      uint4 rd[2];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int x = tid + 256 * m, row = x >> 4, j = x & 15;
         const float4* pk = reinterpret_cast<const float4*>(gK + row * K + 8 * j);
         rk[2 * m] = __ldg(pk);
         rk[2 * m + 1] = __ldg(pk + 1);
-        rd[m] = row < e.z ? __ldg(reinterpret_cast<const uint4*>(dO + ((size_t)(e.w + row) * p.HV + hv) * V + 8 * j))
-                          : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int m = 0; m < 2; ++m) {
         const int x = tid + 256 * m, row = x >> 3, j = x & 7;
+        rd[m] = row < e.z ? __ldg(reinterpret_cast<const uint4*>(dO + ((size_t)(e.w + row) * p.HV + hv) * V + v0 + 8 * j))
+                          : make_uint4(0u, 0u, 0u, 0u);
         const float4* pp = reinterpret_cast<const float4*>(gP + row * CH + 8 * j);
         rp[2 * m] = __ldg(pp);
         rp[2 * m + 1] = __ldg(pp + 1);
@@ -344,12 +355,12 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
         const float fk[8] = {rk[2 * m].x, rk[2 * m].y, rk[2 * m].z, rk[2 * m].w,
                              rk[2 * m + 1].x, rk[2 * m + 1].y, rk[2 * m + 1].z, rk[2 * m + 1].w};
         st_chunk_split(sm + O_KH, sm + O_KL, row, j, TT, fk);
-        *reinterpret_cast<uint4*>(sm + O_DO + sw128_chunk(row, j, TT)) = rd[m];
       }
       const float sc = p.scale;
 #pragma unroll
       for (int m = 0; m < 2; ++m) {
         const int x = tid + 256 * m, row = x >> 3, j = x & 7;
+        *reinterpret_cast<uint4*>(sm + O_DO + sw128_chunk(row, j, TT)) = rd[m];
         const float f[8] = {sc * rp[2 * m].x, sc * rp[2 * m].y, sc * rp[2 * m].z, sc * rp[2 * m].w,
                             sc * rp[2 * m + 1].x, sc * rp[2 * m + 1].y, sc * rp[2 * m + 1].z, sc * rp[2 * m + 1].w};
         st_chunk_split(sm + O_PH, sm + O_PL, row, j, TT, f);
@@ -360,11 +371,11 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid == 0) {  // dU = (scale P)^T dO + K^ dS'^T
+    if (tid == 0) {  // dU[:, z] = (scale P)^T dO[:, z] + K^ dS'_z^T
       const uint32_t ph = smem_u32(sm + O_PH), pl = smem_u32(sm + O_PL), d = smem_u32(sm + O_DO);
       const uint32_t kh = smem_u32(sm + O_KH), kl = smem_u32(sm + O_KL);
       const uint32_t sh = smem_u32(sm + O_SH), sl = smem_u32(sm + O_SL);
-      constexpr uint32_t i_pd = idesc_bf16(64, 128, true, true), i_ks = idesc_bf16(64, 128, false, false);
+      constexpr uint32_t i_pd = idesc_bf16(64, 64, true, true), i_ks = idesc_bf16(64, 64, false, false);
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
         const uint64_t bd = desc_mnmajor(d, s, TT);
@@ -373,9 +384,9 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
       }
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        const uint64_t ak = desc_kmajor(kh, s, TT), bs = desc_kmajor(sh, s, TS);
+        const uint64_t ak = desc_kmajor(kh, s, TT), bs = desc_kmajor(sh, s, TT);
         mma_bf16(taddr(tb, 0, 0), ak, bs, i_ks, 1);
-        mma_bf16(taddr(tb, 0, 0), ak, desc_kmajor(sl, s, TS), i_ks, 1);
+        mma_bf16(taddr(tb, 0, 0), ak, desc_kmajor(sl, s, TT), i_ks, 1);
         mma_bf16(taddr(tb, 0, 0), desc_kmajor(kl, s, TT), bs, i_ks, 1);
       }
       mma_commit(&bar[0]);
@@ -409,14 +420,14 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
     ok = __syncthreads_and(mbar_wait(&bar[0], k & 1, err));
     tc_fence_after();
     if (tid < K) sE[tid] = egc;
-    if (ok) {  // dU: stored, and as a hi/lo tile
-      float x[32];
-      tmem_ld16dp_x8(taddr(tb, 32 * (warp & 3), c0), x);
+    if (ok) {  // dU for this half's values: stored, and as a hi/lo tile [64 tok][64 v]
+      float x[16];
+      tmem_ld16dp_x4(taddr(tb, sub, 32 * half), x);
       tmem_wait_ld();
-      float* gU = w.dU + u * CH * V;
+      float* gU = w.dU + u * CH * V + v0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = c0 + 8 * j + cq;
+      for (int j = 0; j < 4; ++j) {
+        const int c = 32 * half + 8 * j + cq;
         *reinterpret_cast<float2*>(gU + r0 * V + c) = make_float2(x[4 * j], x[4 * j + 1]);
         *reinterpret_cast<float2*>(gU + (r0 + 8) * V + c) = make_float2(x[4 * j + 2], x[4 * j + 3]);
         st_pair_split(sm + O_UH, sm + O_UL, r0, c, TT, x[4 * j], x[4 * j + 1]);
@@ -427,11 +438,11 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (ok && tid == 0) {  // dO^T (scale Q~) + dU^T (-W)
+    if (ok && tid == 0) {  // dO[:, z]^T (scale Q~) + dU[:, z]^T (-W)
       const uint32_t d = smem_u32(sm + O_DO), qh = smem_u32(sm + O_QH), ql = smem_u32(sm + O_QL);
       const uint32_t uh = smem_u32(sm + O_UH), ul = smem_u32(sm + O_UL);
       const uint32_t wh = smem_u32(sm + O_WH), wl = smem_u32(sm + O_WL);
-      constexpr uint32_t id = idesc_bf16(128, 128, true, true);
+      constexpr uint32_t id = idesc_bf16(64, 128, true, true);
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
         const uint64_t ad = desc_mnmajor(d, s, TT);
@@ -446,18 +457,26 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
     }
     ok = __syncthreads_and(ok && mbar_wait(&bar[1], k & 1, err));
     tc_fence_after();
-    if (ok) {  // dS = dS' Diag(e^{Gam_C}) + the products (lane = row v, this half's columns)
-      float x[64];
-      tmem_ld64(taddr(tb, 32 * (warp & 3), 128 + c0), x);
+    if (ok) {  // dS = dS' Diag(e^{Gam_C}) + the products
+      float x[32];
+      tmem_ld16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 64; ++c) S[c] = fmaf(S[c], sE[c0 + c], x[c]);
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          S[4 * j + q] = fmaf(S[4 * j + q], sE[64 * half + 8 * j + cq + (q & 1)], x[4 * j + q]);
     }
   }
   if (ok && a.dh0) {
     float* dh0 = a.dh0 + ((size_t)n * p.HV + hv) * K * V;
 #pragma unroll
-    for (int c = 0; c < 64; ++c) dh0[(size_t)(c0 + c) * V + v] = S[c];
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int r = v0 + r0 + 8 * (q >> 1), c = 64 * half + 8 * j + cq + (q & 1);
+        dh0[(size_t)c * V + r] = S[4 * j + q];
+      }
   }
   tc_fence_before();
   __syncthreads();
@@ -1426,7 +1445,7 @@ bool kda_tc(const Problem& p) {
 template <typename T>
 cudaError_t backward_t(const Problem& p, const Args& a, const KdaWork& w, cudaStream_t s) {
   cudaError_t e = kda_tc<T>(p)
-      ? go("kda_tc_bwd_scan", k_kda_tc_bwd_scan, dim3(p.Nst, p.HV), 1024 + kb::BSCAN_BYTES, s, p, a, w)
+      ? go("kda_tc_bwd_scan", k_kda_tc_bwd_scan, dim3(p.Nst, p.HV, 2), 1024 + kb::BSCAN_BYTES, s, p, a, w)
       : go("kda_bwd_scan", k_kda_bwd_scan<T>, dim3(p.Nst, p.HV, p.V / 32), scan_smem(p.K), s, p, a, w);
   if (e == cudaSuccess)
     e = kda_tc<T>(p) ? go("kda_tc_bwd_dqk", k_kda_tc_bwd_dqk, dim3(p.NCmax, p.HV), 1024 + kt::DQK_BYTES, s, p, a, w)
