@@ -117,9 +117,10 @@ __global__ void __launch_bounds__(256) k_ffma_scan_fwd(Problem p, Args a, Work w
   const int4 sq = w.seq_tab[n];
   extern __shared__ float sm[];
   float* sS = sm;             // [V][K]
-  float* sU = sS + V * K;     // [64][V]
+  float* sU = sS + V * K;     // [64][V]  U~, then U, then diag(e^{G_C - G}) U
   float* sK = sU + CH * V;    // [64][K]
-  float* sG = sK + CH * K;    // [64]
+  float* sW = sK + CH * K;    // [64][K]
+  float* sG = sW + CH * K;    // [64]
   for (int i = threadIdx.x; i < V * K; i += blockDim.x) {
     const int vv = i / K, kk = i % K;
     sS[i] = a.h0 ? a.h0[(((size_t)n * p.HV + hv) * K + kk) * V + vv] : 0.f;
@@ -129,17 +130,22 @@ __global__ void __launch_bounds__(256) k_ffma_scan_fwd(Problem p, Args a, Work w
     const int gc = sq.x + c;
     const int4 e = w.chunk_tab[gc];
     const size_t uo = (size_t)gc * p.HV + hv;
+    copy_async(sW, w.W + uo * CH * K, CH * K);
+    copy_async(sU, w.Ut + uo * CH * V, CH * V);
     load_rows<T>(sK, static_cast<const T*>(a.k) + ((size_t)e.w * p.H + hk) * K, (size_t)p.H * K,
                  e.z, K);
     load_gb(p, w, gc, hv, sG, nullptr);
     float* U = w.U + uo * CH * V;
     copy_f(w.h + uo * V * K, sS, V * K);
-    copy_f(U, w.Ut + uo * CH * V, CH * V);
+    cp_async_wait_all();
     __syncthreads();
-    mm(CH, V, K, U, V, -1.f, true, w.W + uo * CH * K, K, 1, sS, 1, K);
+    mm(CH, V, K, sU, V, -1.f, true, sW, K, 1, sS, 1, K);  // U = U~ - W S^T
     __syncthreads();
     const float GC = sG[CH - 1];
-    for (int i = threadIdx.x; i < CH * V; i += blockDim.x) sU[i] = U[i] * expf(GC - sG[i / V]);
+    for (int i = threadIdx.x; i < CH * V; i += blockDim.x) {
+      U[i] = sU[i];
+      sU[i] *= expf(GC - sG[i / V]);
+    }
     const float eg = expf(GC);
     for (int i = threadIdx.x; i < V * K; i += blockDim.x) sS[i] *= eg;
     __syncthreads();
@@ -227,7 +233,9 @@ __global__ void __launch_bounds__(256) k_ffma_scan_bwd(Problem p, Args a, Work w
   float* sdS = sm;             // [V][K]
   float* sX = sdS + V * K;     // [64][K]: K * D, then Q
   float* sdO = sX + CH * K;    // [64][V]
-  float* sG = sdO + CH * V;
+  float* sdU = sdO + CH * V;   // [64][V]  dU_loc, then dU
+  float* sW = sdU + CH * V;    // [64][K]
+  float* sG = sW + CH * K;
   float* sD = sG + CH;
   for (int i = threadIdx.x; i < V * K; i += blockDim.x) {
     const int vv = i / K, kk = i % K;
@@ -243,14 +251,18 @@ __global__ void __launch_bounds__(256) k_ffma_scan_bwd(Problem p, Args a, Work w
     const float GC = sG[CH - 1];
     if (threadIdx.x < CH) sD[threadIdx.x] = expf(GC - sG[threadIdx.x]);
     __syncthreads();
+    float* dU = w.dU + uo * CH * V;
+    copy_async(sdU, dU, CH * V);
+    copy_async(sW, w.W + uo * CH * K, CH * K);
     load_rows<T>(sX, static_cast<const T*>(a.k) + ((size_t)e.w * p.H + hk) * K, (size_t)p.H * K,
                  e.z, K, sD);
     copy_f(w.dh + uo * V * K, sdS, V * K);
+    cp_async_wait_all();
     __syncthreads();
-    float* dU = w.dU + uo * CH * V;
-    mm(CH, V, K, dU, V, 1.f, true, sX, K, 1, sdS, 1, K);
+    mm(CH, V, K, sdU, V, 1.f, true, sX, K, 1, sdS, 1, K);  // dU = dU_loc + (D K) dS'^T
     __syncthreads();
     const float eg = expf(GC);
+    for (int i = threadIdx.x; i < CH * V; i += blockDim.x) dU[i] = sdU[i];
     for (int i = threadIdx.x; i < V * K; i += blockDim.x) sdS[i] *= eg;
     if (threadIdx.x < CH) sD[threadIdx.x] = p.scale * expf(sG[threadIdx.x]);
     __syncthreads();
@@ -260,7 +272,7 @@ __global__ void __launch_bounds__(256) k_ffma_scan_bwd(Problem p, Args a, Work w
                  (size_t)p.HV * V, e.z, V, sD);
     __syncthreads();
     mm(V, K, CH, sdS, K, 1.f, true, sdO, 1, V, sX, K, 1);
-    mm(V, K, CH, sdS, K, -1.f, true, dU, 1, V, w.W + uo * CH * K, K, 1);
+    mm(V, K, CH, sdS, K, -1.f, true, sdU, 1, V, sW, K, 1);
     __syncthreads();
   }
   if (a.dh0)
@@ -508,7 +520,7 @@ cudaError_t forward_t(const Problem& p, const Args& a, const Work& w, bool bwd_p
   }
   Args a2 = a;
   if (bwd_prep) a2.ht = nullptr;
-  smem = sizeof(float) * (V * K + CH * V + CH * K + CH);
+  smem = sizeof(float) * (V * K + CH * V + 2 * CH * K + CH);
   if ((e = launch("ffma_scan_fwd", k_ffma_scan_fwd<T>, gs, smem, s, p, a2, w)) != cudaSuccess) return e;
   if (!bwd_prep) {
     smem = sizeof(float) * (2 * CH * K + CH * CH + CH * V + CH);
@@ -524,7 +536,7 @@ cudaError_t backward_t(const Problem& p, const Args& a, const Work& w, cudaStrea
   cudaError_t e;
   size_t smem = sizeof(float) * (2 * CH * K + CH * CH + CH * V + CH);
   if ((e = launch("ffma_dvlocal", k_ffma_dvlocal<T>, gu, smem, s, p, a, w)) != cudaSuccess) return e;
-  smem = sizeof(float) * (V * K + CH * K + CH * V + 2 * CH);
+  smem = sizeof(float) * (V * K + 2 * CH * K + 2 * CH * V + 2 * CH);
   if ((e = launch("ffma_scan_bwd", k_ffma_scan_bwd<T>, gs, smem, s, p, a, w)) != cudaSuccess) return e;
   smem = sizeof(float) * (2 * CH * K + CH * V + 2 * CH * CH + 2 * CH + 8);
   if ((e = launch("ffma_dqkwg", k_ffma_dqkwg<T>, gu, smem, s, p, a, w)) != cudaSuccess) return e;
