@@ -1054,9 +1054,92 @@ __global__ void __launch_bounds__(256) k_kda_bwd_wy(Problem p, Args a, KdaWork w
   }
 }
 
+// The gated products with 512 threads (K = 128): thread t owns channel c = t % 128 and role
+// t / 128.  The diagonal sub-blocks: role = the sub-chunk.  Below the diagonal, for each sub-chunk
+// a: roles 0 and 1 form F of a's rows 16a + 8 role .. + 7, roles 2 and 3 G of the columns
+// j = role - 2, role, .. before a.  Same sums and sinks as gated_products_k128; ends with a barrier.
+template <typename TR, typename SinkF, typename SinkG>
+__device__ void gated_products_k128x4(const float* WtT, const TR* R, const TR* Lm, const float* colw,
+                                      const float* G2, SinkF sinkF, SinkG sinkG) {
+  constexpr int K = 128;
+  const int c = threadIdx.x & 127, role = threadIdx.x >> 7;
+  {
+    const int b0 = SUB * role;
+    float g[SUB], r[SUB], l[SUB], F[SUB], G[SUB];
+#pragma unroll
+    for (int j = 0; j < SUB; ++j) {
+      g[j] = G2[(b0 + j) * K + c];
+      r[j] = ldf(R + (b0 + j) * K + c);
+      l[j] = (colw ? colw[b0 + j] : 1.f) * ldf(Lm + (b0 + j) * K + c);
+      F[j] = G[j] = 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < SUB; ++j) {
+      float wv[SUB];
+      ld16(WtT + (b0 + j) * LDT + b0, wv);
+#pragma unroll
+      for (int i = j; i < SUB; ++i) {
+        const float wt = wv[i] * exp2f(g[i] - g[j]);
+        F[i] = fmaf(wt, r[j], F[i]);
+        G[j] = fmaf(wt, l[i], G[j]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) {
+      sinkF(b0 + i, c, F[i]);
+      sinkG(b0 + i, c, G[i]);
+    }
+  }
+#pragma unroll 1
+  for (int A = 1; A < CH / SUB; ++A) {
+    __syncthreads();
+    const int I0 = SUB * A, NJ = SUB * A;
+    const float gr = G2[(I0 - 1) * K + c];
+    if (role < 2) {  // F_i, i = I0 + 8 role .. + 7
+      const int i0 = I0 + 8 * role;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 2
+      for (int j = 0; j < NJ; ++j) {
+        const float rt = ldf(R + j * K + c) * exp2f(gr - G2[j * K + c]);
+        const float4 w0 = reinterpret_cast<const float4*>(WtT + j * LDT + i0)[0];
+        const float4 w1 = reinterpret_cast<const float4*>(WtT + j * LDT + i0)[1];
+        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wv[i], rt, acc[i]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sinkF(i0 + i, c, acc[i] * exp2f(G2[(i0 + i) * K + c] - gr));
+    } else {         // G_j, j = role - 2, role, .. < 16 A
+      float ls[SUB];
+#pragma unroll
+      for (int i = 0; i < SUB; ++i)
+        ls[i] = (colw ? colw[I0 + i] : 1.f) * ldf(Lm + (I0 + i) * K + c) * exp2f(G2[(I0 + i) * K + c] - gr);
+#pragma unroll 2
+      for (int j = role - 2; j < NJ; j += 2) {
+        float wv[SUB];
+        ld16(WtT + j * LDT + I0, wv);
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int i = 0; i < SUB; i += 4) {
+          a0 = fmaf(wv[i], ls[i], a0);
+          a1 = fmaf(wv[i + 1], ls[i + 1], a1);
+          a2 = fmaf(wv[i + 2], ls[i + 2], a2);
+          a3 = fmaf(wv[i + 3], ls[i + 3], a3);
+        }
+        sinkG(j, c, ((a0 + a1) + (a2 + a3)) * exp2f(gr - G2[j * K + c]));
+      }
+    }
+  }
+  __syncthreads();
+}
+
 // ---------------------------------------------------------------- WY backward, tcgen05
 // k_kda_bwd_wy's work for bf16 with K = V = 128, the five products on the tensor cores from
-// compensated bf16 pairs (V is bf16 already).  With X' = k e^{Gam} (X = diag(beta) X'):
+// compensated bf16 pairs (V is bf16 already), 512 threads (16 warps: four per TMEM
+// sub-partition, each taking a quarter of an accumulator's columns).  With X' = k e^{Gam}
+// (X = diag(beta) X'):
 //   [0, 64)    dT = (dW X'^T + dU V^T) diag(beta)     (beta applied to the columns on the way out)
 //   [64, 192)  dX = T^T dW,   [192, 320) dY = T^T dU
 //   [320, 384) Z = dT T^T,    [384, 448) -dA = T^T Z
@@ -1065,16 +1148,17 @@ __global__ void __launch_bounds__(256) k_kda_bwd_wy(Problem p, Args a, KdaWork w
 // chain from there; the dA gated products run by channel.
 namespace kw {
 using namespace tcx;
+constexpr int NT = 512;
 constexpr int TT = 64 * 128;                          // [64 rows][64 bf16] block
-// fixed: Gam (fp32), k (bf16 row-major), V (bf16 tile), small vectors
-constexpr int O_G = 0, O_K = 32768, O_V = 49152, O_VEC = 65536;   // vectors: 2 KB
+// fixed: Gam (fp32), k (bf16 row-major), V (bf16 tile), small vectors (4 KB)
+constexpr int O_G = 0, O_K = 32768, O_V = 49152, O_VEC = 65536;
 // region A: dW, dU, X' (hi, lo); after the first products: dk, dGam, F1 (fp32 [64][128] each),
 // F1 giving way to the raw gate inputs once its terms are in
-constexpr int O_A = 67584;
+constexpr int O_A = 69632;
 constexpr int O_DWH = O_A, O_DWL = O_A + 16384, O_DUH = O_A + 32768, O_DUL = O_A + 49152;
 constexpr int O_XH = O_A + 65536, O_XL = O_A + 81920;
 constexpr int O_ACK = O_A, O_ACG = O_A + 32768, O_F1 = O_A + 65536;
-// region B: T, dT, Z (hi, lo [64][64] each); after the last product: dA (fp32 [64][LDP])
+// region B: T, dT, Z (hi, lo [64][64] each); after the last product: dA^T (fp32 [64][LDT])
 constexpr int O_B = O_A + 98304;
 constexpr int O_TH = O_B, O_TL = O_B + 8192, O_DTH = O_B + 16384, O_DTL = O_B + 24576;
 constexpr int O_ZH = O_B + 32768, O_ZL = O_B + 40960;
@@ -1082,25 +1166,25 @@ constexpr int O_DA = O_B;
 constexpr int WY_BYTES = O_B + 49152;
 static_assert(CH * LDT * 4 <= 49152, "dA fits region B");
 static_assert(1024 + WY_BYTES <= 227 * 1024, "wy_bwd shared memory");
+static_assert(O_A % 1024 == 0 && O_B % 1024 == 0, "tile alignment");
 }  // namespace kw
 
-__global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_wy(Problem p, Args a, KdaWork w) {
+__global__ void __launch_bounds__(kw::NT, 1) k_kda_tc_bwd_wy(Problem p, Args a, KdaWork w) {
   using namespace kw;
   if (kda_failed(w)) return;
   const int gc = blockIdx.x, hv = blockIdx.y;
   const int4 e = w.chunk_tab[gc];
   if (e.x < 0) return;
-  constexpr int K = 128, V = 128;
+  constexpr int K = 128, V = 128, NW = NT / 32;
   const int L = e.z, tok0 = e.w, hk = hv / p.G, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nwarp = 8;
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
   float* sG = reinterpret_cast<float*>(sm + O_G);
   bf16* sK = reinterpret_cast<bf16*>(sm + O_K);
   float* sb = reinterpret_cast<float*>(sm + O_VEC);   // [64] beta, 0 past L
-  float* sdb = sb + 64;                                // [64] dbeta
-  float* sdbp = sb + 128;                              // [2][64] dbeta halves
-  float* sred = sb + 256;                              // [2][128]
+  float* sdb = sb + 64;                                // [64] dbeta; later [16] warp sums
+  float* sdbp = sb + 128;                              // [4][64] dbeta by column quarter
+  float* sred = sb + 384;                              // [4][128]
   float* ack = reinterpret_cast<float*>(sm + O_ACK);
   float* acg = reinterpret_cast<float*>(sm + O_ACG);
   float* sF1 = reinterpret_cast<float*>(sm + O_F1);
@@ -1120,51 +1204,57 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_wy(Problem p, Args a, Kda
     tmem_relinquish();
   }
   const size_t u = (size_t)gc * p.HV + hv, uk = u * CH * K;
-  {  // k (row-major) and V (swizzled tile), rows past L zero; beta
+  {  // k (row-major) and V (swizzled tile), rows past L zero; beta; dW, dU, T (fp32) loads
     const bf16* gk = static_cast<const bf16*>(a.k) + ((size_t)tok0 * p.H + hk) * K;
     const bf16* gv = static_cast<const bf16*>(a.v) + ((size_t)tok0 * p.HV + hv) * V;
-    uint4 rk[4], rv[4];
+    uint4 rk[2], rv[2];
+    float4 rw[4], ru[4], rt[2];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+    for (int m = 0; m < 2; ++m) {
+      const int x = tid + NT * m, row = x >> 4, j = x & 15;
       rk[m] = rv[m] = make_uint4(0u, 0u, 0u, 0u);
       if (row < L) {
         rk[m] = __ldg(reinterpret_cast<const uint4*>(gk + (size_t)row * p.H * K + 8 * j));
         rv[m] = __ldg(reinterpret_cast<const uint4*>(gv + (size_t)row * p.HV * V + 8 * j));
       }
+      const float4* pw = reinterpret_cast<const float4*>(w.dW + uk + row * K + 8 * j);
+      const float4* pu = reinterpret_cast<const float4*>(w.dU + u * CH * V + row * V + 8 * j);
+      rw[2 * m] = __ldg(pw);
+      rw[2 * m + 1] = __ldg(pw + 1);
+      ru[2 * m] = __ldg(pu);
+      ru[2 * m + 1] = __ldg(pu + 1);
     }
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
-      reinterpret_cast<uint4*>(sK)[x] = rk[m];
-      *reinterpret_cast<uint4*>(sm + O_V + sw128_chunk(row, j, TT)) = rv[m];
+    {
+      const int row = tid >> 3, j = tid & 7;
+      const float4* pt = reinterpret_cast<const float4*>(w.Tm + u * CH * CH + row * CH + 8 * j);
+      rt[0] = __ldg(pt);
+      rt[1] = __ldg(pt + 1);
     }
     if (tid < CH) sb[tid] = tid < L ? a.beta[(size_t)(tok0 + tid) * p.HV + hv] : 0.f;
-  }
-  copy_async(sG, w.Gam + uk, CH * K);
-  kt::stage_split2<CH>(sm + O_DWH, sm + O_DWL, w.dW + uk, sm + O_DUH, sm + O_DUL, w.dU + u * CH * V, K);
-  {  // T (fp32 [64][64]) as a hi/lo pair of one-block tiles
-    float4 r[4];
+    copy_async(sG, w.Gam + uk, CH * K);
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
-      const int x = tid + 256 * m, row = x >> 3, j = x & 7;
-      const float4* p4 = reinterpret_cast<const float4*>(w.Tm + u * CH * CH + row * CH + 8 * j);
-      r[2 * m] = __ldg(p4);
-      r[2 * m + 1] = __ldg(p4 + 1);
+      const int x = tid + NT * m, row = x >> 4, j = x & 15;
+      reinterpret_cast<uint4*>(sK)[x] = rk[m];
+      *reinterpret_cast<uint4*>(sm + O_V + sw128_chunk(row, j, TT)) = rv[m];
+      const float fw[8] = {rw[2 * m].x, rw[2 * m].y, rw[2 * m].z, rw[2 * m].w,
+                           rw[2 * m + 1].x, rw[2 * m + 1].y, rw[2 * m + 1].z, rw[2 * m + 1].w};
+      const float fu[8] = {ru[2 * m].x, ru[2 * m].y, ru[2 * m].z, ru[2 * m].w,
+                           ru[2 * m + 1].x, ru[2 * m + 1].y, ru[2 * m + 1].z, ru[2 * m + 1].w};
+      st_chunk_split(sm + O_DWH, sm + O_DWL, row, j, TT, fw);
+      st_chunk_split(sm + O_DUH, sm + O_DUL, row, j, TT, fu);
     }
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const int x = tid + 256 * m, row = x >> 3, j = x & 7;
-      const float f[8] = {r[2 * m].x, r[2 * m].y, r[2 * m].z, r[2 * m].w,
-                          r[2 * m + 1].x, r[2 * m + 1].y, r[2 * m + 1].z, r[2 * m + 1].w};
+    {
+      const int row = tid >> 3, j = tid & 7;
+      const float f[8] = {rt[0].x, rt[0].y, rt[0].z, rt[0].w, rt[1].x, rt[1].y, rt[1].z, rt[1].w};
       st_chunk_split(sm + O_TH, sm + O_TL, row, j, TT, f);
     }
   }
   cp_async_wait_all();
   __syncthreads();
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {  // X' = k e^{Gam}
-    const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+  for (int m = 0; m < 2; ++m) {  // X' = k e^{Gam}
+    const int x = tid + NT * m, row = x >> 4, j = x & 15;
     float f[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -1206,16 +1296,18 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_wy(Problem p, Args a, Kda
     }
     mma_commit(&bar[0]);
   }
-  const int half = warp >> 2, sub = 32 * (warp & 3), r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
+  // M = 64 accumulators, 16-lane loads: warp (sub-partition warp % 4, quarter warp / 4), rows r0
+  // and r0 + 8, columns (quarter of the accumulator) 8j + cq + {0, 1}
+  const int qt = warp >> 2, sub = 32 * (warp & 3), r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
   bool ok = __syncthreads_and(mbar_wait(&bar[0], 0, err));
   tc_fence_after();
-  if (ok) {  // dT diag(beta) as a hi/lo tile
-    float d[16];
-    tmem_ld16dp_x4(taddr(tb, sub, 32 * half), d);
+  if (ok) {  // dT diag(beta) as a hi/lo tile (columns [16 qt, +16))
+    float d[8];
+    tmem_ld16dp_x2(taddr(tb, sub, 16 * qt), d);
     tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = 32 * half + 8 * j + cq;
+    for (int j = 0; j < 2; ++j) {
+      const int c = 16 * qt + 8 * j + cq;
       const float b0 = sb[c], b1 = sb[c + 1];
       st_pair_split(sm + O_DTH, sm + O_DTL, r0, c, TT, d[4 * j] * b0, d[4 * j + 1] * b1);
       st_pair_split(sm + O_DTH, sm + O_DTL, r0 + 8, c, TT, d[4 * j + 2] * b0, d[4 * j + 3] * b1);
@@ -1241,7 +1333,7 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_wy(Problem p, Args a, Kda
   {
     const float4* k4 = reinterpret_cast<const float4*>(w.dkp + uk);
     const float4* g4 = reinterpret_cast<const float4*>(w.dGam + uk);
-    for (int x = tid; x < CH * K / 4; x += 256) {
+    for (int x = tid; x < CH * K / 4; x += NT) {
       reinterpret_cast<float4*>(ack)[x] = __ldg(k4 + x);
       reinterpret_cast<float4*>(acg)[x] = __ldg(g4 + x);
       reinterpret_cast<float4*>(sF1)[x] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1249,9 +1341,9 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_wy(Problem p, Args a, Kda
   }
   __syncthreads();
   if (ok) {  // dv = beta dY; dbeta = rowsum(dY V) + rowsum(dX k e^{Gam}); dk, dGam += beta dX e^{Gam} (1, k)
-    float x[32], y[32];
-    tmem_ld16dp_x8(taddr(tb, sub, 64 + 64 * half), x);
-    tmem_ld16dp_x8(taddr(tb, sub, 192 + 64 * half), y);
+    float x[16], y[16];
+    tmem_ld16dp_x4(taddr(tb, sub, 64 + 32 * qt), x);
+    tmem_ld16dp_x4(taddr(tb, sub, 192 + 32 * qt), y);
     tmem_wait_ld();
     bf16* dv = static_cast<bf16*>(a.dv) + ((size_t)tok0 * p.HV + hv) * V;
     float rs[2] = {0.f, 0.f};
@@ -1260,8 +1352,8 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_wy(Problem p, Args a, Kda
       const int i = r0 + 8 * hr;
       const float bi = sb[i];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = 64 * half + 8 * j + cq;
+      for (int j = 0; j < 4; ++j) {
+        const int c = 32 * qt + 8 * j + cq;
         const float y0 = y[4 * j + 2 * hr], y1 = y[4 * j + 2 * hr + 1];
         const float2 vv = ld_pair(sm + O_V, i, c, TT);
         rs[hr] += y0 * vv.x + y1 * vv.y;
@@ -1279,20 +1371,20 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_wy(Problem p, Args a, Kda
     rs[0] = quad_sum(rs[0]);
     rs[1] = quad_sum(rs[1]);
     if ((lane & 3) == 0) {
-      sdbp[half * 64 + r0] = rs[0];
-      sdbp[half * 64 + r0 + 8] = rs[1];
+      sdbp[qt * 64 + r0] = rs[0];
+      sdbp[qt * 64 + r0 + 8] = rs[1];
     }
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
   tc_fence_after();
-  if (tid < CH) sdb[tid] = sdbp[tid] + sdbp[64 + tid];
+  if (tid < CH) sdb[tid] = (sdbp[tid] + sdbp[64 + tid]) + (sdbp[128 + tid] + sdbp[192 + tid]);
   if (ok) {  // Z as a hi/lo tile
-    float d[16];
-    tmem_ld16dp_x4(taddr(tb, sub, 320 + 32 * half), d);
+    float d[8];
+    tmem_ld16dp_x2(taddr(tb, sub, 320 + 16 * qt), d);
     tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = 32 * half + 8 * j + cq;
+    for (int j = 0; j < 2; ++j) {
+      const int c = 16 * qt + 8 * j + cq;
       st_pair_split(sm + O_ZH, sm + O_ZL, r0, c, TT, d[4 * j], d[4 * j + 1]);
       st_pair_split(sm + O_ZH, sm + O_ZL, r0 + 8, c, TT, d[4 * j + 2], d[4 * j + 3]);
     }
@@ -1315,29 +1407,29 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_wy(Problem p, Args a, Kda
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[2], 0, err));
   tc_fence_after();
-  if (ok) {  // dA = -T^T Z, strictly lower, over region B
-    float d[16];
-    tmem_ld16dp_x4(taddr(tb, sub, 384 + 32 * half), d);
+  if (ok) {  // dA = -T^T Z, strictly lower, transposed over region B
+    float d[8];
+    tmem_ld16dp_x2(taddr(tb, sub, 384 + 16 * qt), d);
     tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < 2; ++j)
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int i = r0 + 8 * (q >> 1), c = 32 * half + 8 * j + cq + (q & 1);
+        const int i = r0 + 8 * (q >> 1), c = 16 * qt + 8 * j + cq + (q & 1);
         sdA[c * LDT + i] = c < i ? -d[4 * j + q] : 0.f;
       }
   }
   __syncthreads();
   // A_ij = beta_i sum_c k_i k_j e^{Gam_i - Gam_j}: F1 (rows, weights dA), G1 (columns, beta_i dA)
   if (ok)
-    gated_products_k128(sdA, sK, sK, sb, sG,
-                        [&](int i, int c, float f) { sF1[i * K + c] += f; },
-                        [&](int j, int c, float g) {
-                          ack[j * K + c] += g;
-                          acg[j * K + c] -= __bfloat162float(sK[j * K + c]) * g;
-                        });
+    gated_products_k128x4(sdA, sK, sK, sb, sG,
+                          [&](int i, int c, float f) { sF1[i * K + c] += f; },
+                          [&](int j, int c, float g) {
+                            ack[j * K + c] += g;
+                            acg[j * K + c] -= __bfloat162float(sK[j * K + c]) * g;
+                          });
   // F1 terms: dk += beta F1, dGam += beta k F1, dbeta += rowsum(k F1)
-  for (int i = warp; i < CH; i += nwarp) {
+  for (int i = warp; i < CH; i += NW) {
     float sacc = 0.f;
     for (int c = lane; c < K; c += 32) {
       const int o = i * K + c;
@@ -1350,15 +1442,21 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_wy(Problem p, Args a, Kda
     if (ok && lane == 0 && i < L) a.dbeta[(size_t)(tok0 + i) * p.HV + hv] = sdb[i] + sacc;
   }
   __syncthreads();
-  float* sg = sF1;  // F1 is done: the raw gate inputs
-  load_tile<float>(sg, K, a.g_raw + ((size_t)tok0 * p.HV + hv) * K, (size_t)p.HV * K, L, K);
+  float* sg = sF1;  // F1 is done: the raw gate inputs (rows past L zero)
   {
+    const float* gsrc = a.g_raw + ((size_t)tok0 * p.HV + hv) * K;
+    for (int x = tid; x < CH * K / 4; x += NT) {
+      const int row = x >> 5, c4 = x & 31;
+      reinterpret_cast<float4*>(sg)[x] = row < L ? __ldg(reinterpret_cast<const float4*>(gsrc + (size_t)row * p.HV * K) + c4)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float4* dk4 = reinterpret_cast<float4*>(w.dkp + uk);
-    for (int x = tid; x < CH * K / 4; x += 256) dk4[x] = reinterpret_cast<const float4*>(ack)[x];
+    for (int x = tid; x < CH * K / 4; x += NT) dk4[x] = reinterpret_cast<const float4*>(ack)[x];
   }
   __syncthreads();
-  // dyg = reverse in-chunk cumsum of dGam: two row halves, the lower offset by the upper's sum
-  const int part = tid / K, cc = tid % K, rows = CH / 2;
+  // dyg = reverse in-chunk cumsum of dGam: four row parts, each offset by the parts below it
+  constexpr int NP = NT / K, rows = CH / NP;
+  const int part = tid / K, cc = tid % K;
   {
     float t = 0.f;
     for (int i = part * rows; i < (part + 1) * rows; ++i) t += acg[i * K + cc];
@@ -1367,7 +1465,8 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_wy(Problem p, Args a, Kda
   __syncthreads();
   const float nexp = -expf(a.A_log[hv]);
   const float bias = a.dt_bias ? a.dt_bias[(size_t)hv * K + cc] : 0.f;
-  float acc = part == 0 ? sred[K + cc] : 0.f, pA = 0.f, pB = 0.f;
+  float acc = 0.f, pA = 0.f, pB = 0.f;
+  for (int q = part + 1; q < NP; ++q) acc += sred[q * K + cc];
   for (int i = (part + 1) * rows - 1; i >= part * rows; --i) {
     acc += acg[i * K + cc];
     if (i < L) {
@@ -1388,10 +1487,14 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_wy(Problem p, Args a, Kda
   if (lane == 0) sdb[warp] = pA;
   __syncthreads();
   float* pg = w.pgp + u * (K + 1);
-  if (tid < K) pg[tid] = sred[tid] + sred[K + tid];
+  if (tid < K) {
+    float t = 0.f;
+    for (int q = 0; q < NP; ++q) t += sred[q * K + tid];
+    pg[tid] = t;
+  }
   if (tid == 0) {
     float t = 0.f;
-    for (int q = 0; q < nwarp; ++q) t += sdb[q];
+    for (int q = 0; q < NW; ++q) t += sdb[q];
     pg[K] = t;
   }
   tc_fence_before();
@@ -1427,12 +1530,12 @@ size_t wy_smem(int K, int V) {
 
 template <typename Kern>
 cudaError_t go(const char* name, Kern kern, dim3 grid, size_t smem, cudaStream_t s, const Problem& p,
-               const Args& a, const KdaWork& w) {
+               const Args& a, const KdaWork& w, int threads = 256) {
   if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps(name, s);
-  kern<<<grid, 256, smem, s>>>(p, a, w);
+  kern<<<grid, threads, smem, s>>>(p, a, w);
   return cudaGetLastError();
 }
 
@@ -1451,7 +1554,7 @@ cudaError_t backward_t(const Problem& p, const Args& a, const KdaWork& w, cudaSt
     e = kda_tc<T>(p) ? go("kda_tc_bwd_dqk", k_kda_tc_bwd_dqk, dim3(p.NCmax, p.HV), 1024 + kt::DQK_BYTES, s, p, a, w)
                      : go("kda_bwd_dqk", k_kda_bwd_dqk<T>, dim3(p.NCmax, p.HV), dqk_smem(p.K, p.V), s, p, a, w);
   if (e == cudaSuccess)
-    e = kda_tc<T>(p) ? go("kda_tc_bwd_wy", k_kda_tc_bwd_wy, dim3(p.NCmax, p.HV), 1024 + kw::WY_BYTES, s, p, a, w)
+    e = kda_tc<T>(p) ? go("kda_tc_bwd_wy", k_kda_tc_bwd_wy, dim3(p.NCmax, p.HV), 1024 + kw::WY_BYTES, s, p, a, w, kw::NT)
                      : go("kda_bwd_wy", k_kda_bwd_wy<T>, dim3(p.NCmax, p.HV), wy_smem(p.K, p.V), s, p, a, w);
   if (e != cudaSuccess) return e;
   Work gw{};  // the group sum's view of the shares
