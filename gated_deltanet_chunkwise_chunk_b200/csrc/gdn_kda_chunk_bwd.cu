@@ -197,6 +197,87 @@ __device__ void gated_products_k128(const float* WtT, const TR* R, const TR* Lm,
   __syncthreads();
 }
 
+// The gated products with 512 threads (K = 128): thread t owns channel c = t % 128 and role
+// t / 128.  The diagonal sub-blocks: role = the sub-chunk.  Below the diagonal, for each sub-chunk
+// a: roles 0 and 1 form F of a's rows 16a + 8 role .. + 7, roles 2 and 3 G of the columns
+// j = role - 2, role, .. before a.  Same sums and sinks as gated_products_k128; ends with a barrier.
+template <typename TR, typename SinkF, typename SinkG>
+__device__ void gated_products_k128x4(const float* WtT, const TR* R, const TR* Lm, const float* colw,
+                                      const float* G2, SinkF sinkF, SinkG sinkG) {
+  constexpr int K = 128;
+  const int c = threadIdx.x & 127, role = threadIdx.x >> 7;
+  {
+    const int b0 = SUB * role;
+    float g[SUB], r[SUB], l[SUB], F[SUB], G[SUB];
+#pragma unroll
+    for (int j = 0; j < SUB; ++j) {
+      g[j] = G2[(b0 + j) * K + c];
+      r[j] = ldf(R + (b0 + j) * K + c);
+      l[j] = (colw ? colw[b0 + j] : 1.f) * ldf(Lm + (b0 + j) * K + c);
+      F[j] = G[j] = 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < SUB; ++j) {
+      float wv[SUB];
+      ld16(WtT + (b0 + j) * LDT + b0, wv);
+#pragma unroll
+      for (int i = j; i < SUB; ++i) {
+        const float wt = wv[i] * exp2f(g[i] - g[j]);
+        F[i] = fmaf(wt, r[j], F[i]);
+        G[j] = fmaf(wt, l[i], G[j]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) {
+      sinkF(b0 + i, c, F[i]);
+      sinkG(b0 + i, c, G[i]);
+    }
+  }
+#pragma unroll 1
+  for (int A = 1; A < CH / SUB; ++A) {
+    __syncthreads();
+    const int I0 = SUB * A, NJ = SUB * A;
+    const float gr = G2[(I0 - 1) * K + c];
+    if (role < 2) {  // F_i, i = I0 + 8 role .. + 7
+      const int i0 = I0 + 8 * role;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 2
+      for (int j = 0; j < NJ; ++j) {
+        const float rt = ldf(R + j * K + c) * exp2f(gr - G2[j * K + c]);
+        const float4 w0 = reinterpret_cast<const float4*>(WtT + j * LDT + i0)[0];
+        const float4 w1 = reinterpret_cast<const float4*>(WtT + j * LDT + i0)[1];
+        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wv[i], rt, acc[i]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sinkF(i0 + i, c, acc[i] * exp2f(G2[(i0 + i) * K + c] - gr));
+    } else {         // G_j, j = role - 2, role, .. < 16 A
+      float ls[SUB];
+#pragma unroll
+      for (int i = 0; i < SUB; ++i)
+        ls[i] = (colw ? colw[I0 + i] : 1.f) * ldf(Lm + (I0 + i) * K + c) * exp2f(G2[(I0 + i) * K + c] - gr);
+#pragma unroll 2
+      for (int j = role - 2; j < NJ; j += 2) {
+        float wv[SUB];
+        ld16(WtT + j * LDT + I0, wv);
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int i = 0; i < SUB; i += 4) {
+          a0 = fmaf(wv[i], ls[i], a0);
+          a1 = fmaf(wv[i + 1], ls[i + 1], a1);
+          a2 = fmaf(wv[i + 2], ls[i + 2], a2);
+          a3 = fmaf(wv[i + 3], ls[i + 3], a3);
+        }
+        sinkG(j, c, ((a0 + a1) + (a2 + a3)) * exp2f(gr - G2[j * K + c]));
+      }
+    }
+  }
+  __syncthreads();
+}
+
 // ---------------------------------------------------------------- reverse state scan
 template <typename T>
 __global__ void __launch_bounds__(256) k_kda_bwd_scan(Problem p, Args a, KdaWork w) {
@@ -594,6 +675,7 @@ __global__ void __launch_bounds__(256) k_kda_bwd_dqk(Problem p, Args a, KdaWork 
 // per-channel terms then run on CUDA cores as in k_kda_bwd_dqk.
 namespace kt {
 using namespace tcx;
+constexpr int NT = 512;           // threads of the output-side kernel
 constexpr int TILE_T = 64 * 128;  // a [64 rows][64 bf16] block
 constexpr int TILE_S = 128 * 128; // a [128 rows][64 bf16] block
 constexpr int O_DO = 0, O_UH = 16384, O_UL = 32768, O_DUH = 49152, O_DUL = 65536;
@@ -611,34 +693,35 @@ static_assert(O_SL + 32768 <= O_DP && O_SCR + 32768 <= O_DP, "tiles overlap the 
 static_assert(1024 + DQK_BYTES <= 227 * 1024, "dqk shared memory");
 
 // rows [0, R) of an fp32 [R][128] matrix (row stride ld floats) as a hi/lo pair of sw128 tiles
-template <int R>
+// (NT threads)
+template <int R, int NT = 256>
 __device__ __forceinline__ void stage_split(unsigned char* hi, unsigned char* lo, const float* src, size_t ld) {
-  constexpr int N = R * 16 / 256;  // 16-byte chunks of 8 floats per thread
+  constexpr int N = R * 16 / NT;  // 16-byte chunks of 8 floats per thread
   float4 r[2 * N];
 #pragma unroll
   for (int m = 0; m < N; ++m) {
-    const int x = threadIdx.x + 256 * m, row = x >> 4, j = x & 15;
+    const int x = threadIdx.x + NT * m, row = x >> 4, j = x & 15;
     const float4* p = reinterpret_cast<const float4*>(src + row * ld + 8 * j);
     r[2 * m] = __ldg(p);
     r[2 * m + 1] = __ldg(p + 1);
   }
 #pragma unroll
   for (int m = 0; m < N; ++m) {
-    const int x = threadIdx.x + 256 * m, row = x >> 4, j = x & 15;
+    const int x = threadIdx.x + NT * m, row = x >> 4, j = x & 15;
     const float f[8] = {r[2 * m].x, r[2 * m].y, r[2 * m].z, r[2 * m].w,
                         r[2 * m + 1].x, r[2 * m + 1].y, r[2 * m + 1].z, r[2 * m + 1].w};
     st_chunk_split(hi, lo, row, j, R * 128, f);
   }
 }
 // two such matrices with all loads issued before the first store
-template <int R>
+template <int R, int NT = 256>
 __device__ __forceinline__ void stage_split2(unsigned char* hi0, unsigned char* lo0, const float* src0,
                                              unsigned char* hi1, unsigned char* lo1, const float* src1, size_t ld) {
-  constexpr int N = R * 16 / 256;
+  constexpr int N = R * 16 / NT;
   float4 r[4 * N];
 #pragma unroll
   for (int m = 0; m < N; ++m) {
-    const int x = threadIdx.x + 256 * m, row = x >> 4, j = x & 15;
+    const int x = threadIdx.x + NT * m, row = x >> 4, j = x & 15;
     const float4* p0 = reinterpret_cast<const float4*>(src0 + row * ld + 8 * j);
     const float4* p1 = reinterpret_cast<const float4*>(src1 + row * ld + 8 * j);
     r[4 * m] = __ldg(p0);
@@ -648,7 +731,7 @@ __device__ __forceinline__ void stage_split2(unsigned char* hi0, unsigned char* 
   }
 #pragma unroll
   for (int m = 0; m < N; ++m) {
-    const int x = threadIdx.x + 256 * m, row = x >> 4, j = x & 15;
+    const int x = threadIdx.x + NT * m, row = x >> 4, j = x & 15;
     const float f0[8] = {r[4 * m].x, r[4 * m].y, r[4 * m].z, r[4 * m].w,
                          r[4 * m + 1].x, r[4 * m + 1].y, r[4 * m + 1].z, r[4 * m + 1].w};
     const float f1[8] = {r[4 * m + 2].x, r[4 * m + 2].y, r[4 * m + 2].z, r[4 * m + 2].w,
@@ -659,7 +742,7 @@ __device__ __forceinline__ void stage_split2(unsigned char* hi0, unsigned char* 
 }
 }  // namespace kt
 
-__global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, KdaWork w) {
+__global__ void __launch_bounds__(kt::NT, 1) k_kda_tc_bwd_dqk(Problem p, Args a, KdaWork w) {
   using namespace kt;
   if (kda_failed(w)) return;
   const int gc = blockIdx.x, hv = blockIdx.y;
@@ -689,21 +772,21 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, Kd
   const size_t u = (size_t)gc * p.HV + hv, uk = u * CH * K;
   {  // dO rows [0, L) (bf16, zero past L), U, dU, S; Gam
     const bf16* dO = static_cast<const bf16*>(a.dO) + ((size_t)tok0 * p.HV + hv) * V;
-    uint4 r[4];
+    uint4 r[2];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+    for (int m = 0; m < 2; ++m) {
+      const int x = tid + NT * m, row = x >> 4, j = x & 15;
       r[m] = row < L ? __ldg(reinterpret_cast<const uint4*>(dO + (size_t)row * p.HV * V + 8 * j))
                      : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+    for (int m = 0; m < 2; ++m) {
+      const int x = tid + NT * m, row = x >> 4, j = x & 15;
       *reinterpret_cast<uint4*>(sm + O_DO + sw128_chunk(row, j, TILE_T)) = r[m];
     }
   }
-  stage_split2<CH>(sm + O_UH, sm + O_UL, w.U + u * CH * V, sm + O_DUH, sm + O_DUL, w.dU + u * CH * V, V);
-  stage_split<128>(sm + O_SH, sm + O_SL, w.h + u * V * K, K);
+  stage_split2<CH, NT>(sm + O_UH, sm + O_UL, w.U + u * CH * V, sm + O_DUH, sm + O_DUL, w.dU + u * CH * V, V);
+  stage_split<128, NT>(sm + O_SH, sm + O_SL, w.h + u * V * K, K);
   copy_async(sG, w.Gam + uk, CH * K);
   cp_async_wait_all();
   fence_proxy_async();
@@ -733,10 +816,10 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, Kd
   }
   // dS' (leaving the chunk) into registers while the products run
   const float* dSn = w.dh + u * V * K;
-  float4 rd[16];
+  float4 rd[8];
 #pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+  for (int m = 0; m < 4; ++m) {
+    const int x = tid + NT * m, row = x >> 4, j = x & 15;
     const float4* p4 = reinterpret_cast<const float4*>(dSn + (size_t)row * K + 8 * j);
     rd[2 * m] = __ldg(p4);
     rd[2 * m + 1] = __ldg(p4 + 1);
@@ -747,8 +830,8 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, Kd
     float cs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     const int j = tid & 15;
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const int row = (tid >> 4) + 16 * m;
+    for (int m = 0; m < 4; ++m) {
+      const int row = (tid >> 4) + 32 * m;
       float h[8], l[8];
       ld_chunk_f(sm + O_SH, row, j, TILE_S, h);
       ld_chunk_f(sm + O_SL, row, j, TILE_S, l);
@@ -759,7 +842,10 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, Kd
       st_chunk_split(sm + O_SH, sm + O_SL, row, j, TILE_S, f);
     }
 #pragma unroll
-    for (int q = 0; q < 8; ++q) sred[(tid >> 4) * 128 + 8 * j + q] = cs[q];
+    for (int q = 0; q < 8; ++q) cs[q] += __shfl_xor_sync(0xffffffffu, cs[q], 16);  // same j
+    if (lane < 16)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) sred[warp * 128 + 8 * j + q] = cs[q];
   }
   fence_proxy_async();
   tc_fence_before();
@@ -782,26 +868,26 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, Kd
     for (int q = 0; q < 16; ++q) t += sred[q * 128 + tid];
     sGC[tid] = exp2f(sG[(CH - 1) * K + tid]) * t;
   }
-  // M = 64 accumulators, 16-lane loads: rows r0 and r0 + 8, columns 8j + cq + {0, 1} of this
-  // warp half's range
-  const int half = warp >> 2, sub = 32 * (warp & 3), r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
+  // M = 64 accumulators, 16-lane loads: warp (sub-partition warp % 4, quarter warp / 4), rows r0
+  // and r0 + 8, columns 8j + cq + {0, 1} of this warp's quarter of the accumulator
+  const int qt = warp >> 2, sub = 32 * (warp & 3), r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
   if (ok) {
-    float d[16];
-    tmem_ld16dp_x4(taddr(tb, sub, 32 * half), d);  // dP, columns [32 half, +32)
-    float x[32];
-    tmem_ld16dp_x8(taddr(tb, sub, 192 + 64 * half), x);  // dW', columns [64 half, +64)
+    float d[8];
+    tmem_ld16dp_x2(taddr(tb, sub, 16 * qt), d);  // dP, columns [16 qt, +16)
+    float x[16];
+    tmem_ld16dp_x4(taddr(tb, sub, 192 + 32 * qt), x);  // dW', columns [32 qt, +32)
     tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < 2; ++j)
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int i = r0 + 8 * (q >> 1), c = 32 * half + 8 * j + cq + (q & 1);
+        const int i = r0 + 8 * (q >> 1), c = 16 * qt + 8 * j + cq + (q & 1);
         sdP[c * LDT + i] = c <= i ? p.scale * d[4 * j + q] : 0.f;
       }
     float* dW = w.dW + uk;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = 64 * half + 8 * j + cq;
+    for (int j = 0; j < 4; ++j) {
+      const int c = 32 * qt + 8 * j + cq;
       *reinterpret_cast<float2*>(dW + r0 * K + c) = make_float2(-x[4 * j], -x[4 * j + 1]);
       *reinterpret_cast<float2*>(dW + (r0 + 8) * K + c) = make_float2(-x[4 * j + 2], -x[4 * j + 3]);
     }
@@ -817,10 +903,10 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, Kd
     const size_t rs = (size_t)p.H * K;
     const bf16* gq = static_cast<const bf16*>(a.q) + ((size_t)tok0 * p.H + hk) * K;
     const bf16* gk = static_cast<const bf16*>(a.k) + ((size_t)tok0 * p.H + hk) * K;
-    uint4 rq[4], rk[4];
+    uint4 rq[2], rk[2];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+    for (int m = 0; m < 2; ++m) {
+      const int x = tid + NT * m, row = x >> 4, j = x & 15;
       rq[m] = rk[m] = make_uint4(0u, 0u, 0u, 0u);
       if (row < L) {
         rq[m] = __ldg(reinterpret_cast<const uint4*>(gq + row * rs + 8 * j));
@@ -828,24 +914,24 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, Kd
       }
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int x = tid + 256 * m;
+    for (int m = 0; m < 2; ++m) {
+      const int x = tid + NT * m;
       reinterpret_cast<uint4*>(sQ)[x] = rq[m];
       reinterpret_cast<uint4*>(sK)[x] = rk[m];
     }
   }
   __syncthreads();
   if (ok) {  // dQ~ e^{Gam}, dK^ e^{Gam_C - Gam}, dGam; colsum(dK^ * K^) per column
-    float x[32], y[32];
-    tmem_ld16dp_x8(taddr(tb, sub, 64 + 64 * half), x);
-    tmem_ld16dp_x8(taddr(tb, sub, 320 + 64 * half), y);
+    float x[16], y[16];
+    tmem_ld16dp_x4(taddr(tb, sub, 64 + 32 * qt), x);
+    tmem_ld16dp_x4(taddr(tb, sub, 320 + 32 * qt), y);
     tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 4; ++j) {
       float cs[2];
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
-        const int c = 64 * half + 8 * j + cq + b;
+        const int c = 32 * qt + 8 * j + cq + b;
         const float gC = sG[(CH - 1) * K + c];
         float t = 0.f;
 #pragma unroll
@@ -865,7 +951,7 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, Kd
         cs[b] = t;
       }
       if (lane < 4) {
-        const int c = 64 * half + 8 * j + cq;
+        const int c = 32 * qt + 8 * j + cq;
         sred[(warp & 3) * 128 + c] = cs[0];
         sred[(warp & 3) * 128 + c + 1] = cs[1];
       }
@@ -876,7 +962,7 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, Kd
     acg[(CH - 1) * K + tid] += sGC[tid] + sred[tid] + sred[128 + tid] + sred[256 + tid] + sred[384 + tid];
   __syncthreads();
   if (ok)  // P_ij = sum_c q_i k_j e^{Gam_i - Gam_j}: dq += F2, dk += G2, dGam += q F2 - k G2
-    gated_products_k128(sdP, sK, sQ, nullptr, sG,
+    gated_products_k128x4(sdP, sK, sQ, nullptr, sG,
                    [&](int i, int c, float f) {
                      acq[i * K + c] += f;
                      acg[i * K + c] += __bfloat162float(sQ[i * K + c]) * f;
@@ -889,7 +975,7 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_dqk(Problem p, Args a, Kd
     float4* dq4 = reinterpret_cast<float4*>(w.dqp + uk);
     float4* dk4 = reinterpret_cast<float4*>(w.dkp + uk);
     float4* dg4 = reinterpret_cast<float4*>(w.dGam + uk);
-    for (int x = tid; x < CH * K / 4; x += 256) {
+    for (int x = tid; x < CH * K / 4; x += NT) {
       dq4[x] = reinterpret_cast<const float4*>(acq)[x];
       dk4[x] = reinterpret_cast<const float4*>(ack)[x];
       dg4[x] = reinterpret_cast<const float4*>(acg)[x];
@@ -1052,87 +1138,6 @@ __global__ void __launch_bounds__(256) k_kda_bwd_wy(Problem p, Args a, KdaWork w
     for (int q = 0; q < nwarp; ++q) t += sdb[q];
     pg[K] = t;
   }
-}
-
-// The gated products with 512 threads (K = 128): thread t owns channel c = t % 128 and role
-// t / 128.  The diagonal sub-blocks: role = the sub-chunk.  Below the diagonal, for each sub-chunk
-// a: roles 0 and 1 form F of a's rows 16a + 8 role .. + 7, roles 2 and 3 G of the columns
-// j = role - 2, role, .. before a.  Same sums and sinks as gated_products_k128; ends with a barrier.
-template <typename TR, typename SinkF, typename SinkG>
-__device__ void gated_products_k128x4(const float* WtT, const TR* R, const TR* Lm, const float* colw,
-                                      const float* G2, SinkF sinkF, SinkG sinkG) {
-  constexpr int K = 128;
-  const int c = threadIdx.x & 127, role = threadIdx.x >> 7;
-  {
-    const int b0 = SUB * role;
-    float g[SUB], r[SUB], l[SUB], F[SUB], G[SUB];
-#pragma unroll
-    for (int j = 0; j < SUB; ++j) {
-      g[j] = G2[(b0 + j) * K + c];
-      r[j] = ldf(R + (b0 + j) * K + c);
-      l[j] = (colw ? colw[b0 + j] : 1.f) * ldf(Lm + (b0 + j) * K + c);
-      F[j] = G[j] = 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < SUB; ++j) {
-      float wv[SUB];
-      ld16(WtT + (b0 + j) * LDT + b0, wv);
-#pragma unroll
-      for (int i = j; i < SUB; ++i) {
-        const float wt = wv[i] * exp2f(g[i] - g[j]);
-        F[i] = fmaf(wt, r[j], F[i]);
-        G[j] = fmaf(wt, l[i], G[j]);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < SUB; ++i) {
-      sinkF(b0 + i, c, F[i]);
-      sinkG(b0 + i, c, G[i]);
-    }
-  }
-#pragma unroll 1
-  for (int A = 1; A < CH / SUB; ++A) {
-    __syncthreads();
-    const int I0 = SUB * A, NJ = SUB * A;
-    const float gr = G2[(I0 - 1) * K + c];
-    if (role < 2) {  // F_i, i = I0 + 8 role .. + 7
-      const int i0 = I0 + 8 * role;
-      float acc[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll 2
-      for (int j = 0; j < NJ; ++j) {
-        const float rt = ldf(R + j * K + c) * exp2f(gr - G2[j * K + c]);
-        const float4 w0 = reinterpret_cast<const float4*>(WtT + j * LDT + i0)[0];
-        const float4 w1 = reinterpret_cast<const float4*>(WtT + j * LDT + i0)[1];
-        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wv[i], rt, acc[i]);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) sinkF(i0 + i, c, acc[i] * exp2f(G2[(i0 + i) * K + c] - gr));
-    } else {         // G_j, j = role - 2, role, .. < 16 A
-      float ls[SUB];
-#pragma unroll
-      for (int i = 0; i < SUB; ++i)
-        ls[i] = (colw ? colw[I0 + i] : 1.f) * ldf(Lm + (I0 + i) * K + c) * exp2f(G2[(I0 + i) * K + c] - gr);
-#pragma unroll 2
-      for (int j = role - 2; j < NJ; j += 2) {
-        float wv[SUB];
-        ld16(WtT + j * LDT + I0, wv);
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-        for (int i = 0; i < SUB; i += 4) {
-          a0 = fmaf(wv[i], ls[i], a0);
-          a1 = fmaf(wv[i + 1], ls[i + 1], a1);
-          a2 = fmaf(wv[i + 2], ls[i + 2], a2);
-          a3 = fmaf(wv[i + 3], ls[i + 3], a3);
-        }
-        sinkG(j, c, ((a0 + a1) + (a2 + a3)) * exp2f(gr - G2[j * K + c]));
-      }
-    }
-  }
-  __syncthreads();
 }
 
 // ---------------------------------------------------------------- WY backward, tcgen05
@@ -1551,7 +1556,7 @@ cudaError_t backward_t(const Problem& p, const Args& a, const KdaWork& w, cudaSt
       ? go("kda_tc_bwd_scan", k_kda_tc_bwd_scan, dim3(p.Nst, p.HV, 2), 1024 + kb::BSCAN_BYTES, s, p, a, w)
       : go("kda_bwd_scan", k_kda_bwd_scan<T>, dim3(p.Nst, p.HV, p.V / 32), scan_smem(p.K), s, p, a, w);
   if (e == cudaSuccess)
-    e = kda_tc<T>(p) ? go("kda_tc_bwd_dqk", k_kda_tc_bwd_dqk, dim3(p.NCmax, p.HV), 1024 + kt::DQK_BYTES, s, p, a, w)
+    e = kda_tc<T>(p) ? go("kda_tc_bwd_dqk", k_kda_tc_bwd_dqk, dim3(p.NCmax, p.HV), 1024 + kt::DQK_BYTES, s, p, a, w, kt::NT)
                      : go("kda_bwd_dqk", k_kda_bwd_dqk<T>, dim3(p.NCmax, p.HV), dqk_smem(p.K, p.V), s, p, a, w);
   if (e == cudaSuccess)
     e = kda_tc<T>(p) ? go("kda_tc_bwd_wy", k_kda_tc_bwd_wy, dim3(p.NCmax, p.HV), 1024 + kw::WY_BYTES, s, p, a, w, kw::NT)
