@@ -28,6 +28,7 @@
 #include "gdn_common.cuh"
 #include "gdn_launch.h"
 #include "gdn_tc_common.cuh"  // unit_lower_inverse64, LDA
+#include "kda_gate_math.cuh"
 
 namespace gdn {
 namespace {
@@ -307,7 +308,7 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork
       float yg = 0.f;
       if (i < L) {
         const float z = sG[x] + (a.dt_bias ? a.dt_bias[(size_t)hv * K + c] : 0.f);
-        yg = nexp * (z > 20.f ? z : log1pf(expf(z)));
+        yg = nexp * softplus20(z);
       }
       sG[x] = yg;
     }

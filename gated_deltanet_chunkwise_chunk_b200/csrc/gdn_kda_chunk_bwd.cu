@@ -23,6 +23,7 @@
 #include "gdn_common.cuh"
 #include "gdn_launch.h"
 #include "gdn_tc_common.cuh"  // LDA
+#include "kda_gate_math.cuh"
 
 namespace gdn {
 namespace {
@@ -1477,8 +1478,8 @@ __global__ void __launch_bounds__(kw::NT, 1) k_kda_tc_bwd_wy(Problem p, Args a, 
     if (i < L) {
       const size_t o = ((size_t)(tok0 + i) * p.HV + hv) * K + cc;
       const float xg = sg[i * K + cc] + bias;
-      const float sp = xg > 20.f ? xg : log1pf(expf(xg));
-      const float sig = xg > 20.f ? 1.f : 1.f / (1.f + expf(-xg));
+      float sp, sig;
+      softplus_sigmoid(xg, sp, sig);
       const float dgr = acc * nexp * sig;
       a.dg[o] = acc;
       if (a.dg_raw) a.dg_raw[o] = dgr;
