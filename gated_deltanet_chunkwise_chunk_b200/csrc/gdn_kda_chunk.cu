@@ -646,13 +646,16 @@ __global__ void __launch_bounds__(256) k_kda_scan(Problem p, Args a, KdaWork w) 
 // of its warp half), both products of a chunk on the tensor cores from compensated bf16 pairs:
 //   U[:, z] = U~[:, z] - W S_z^T        (M = 64 tokens, N = 64;  A = W, B = S_z, K-major)   TMEM [0, 64)
 //   S_z' = S_z Diag(e^{Gam_C}) + U[:, z]^T K^   (M = 64, N = K;  A = U^T, B = K^, MN-major) TMEM [128, 256)
-// It stores the state entering every chunk and U, as k_kda_scan does.
+// It stores the state entering every chunk and U, as k_kda_scan does.  The next chunk's W and K^
+// are bulk-copied into an fp32 buffer while a chunk's products run, so a chunk's operand tiles
+// are built from shared memory.
 namespace ks {
 using namespace tcx;
 constexpr int TT = 64 * 128;
 constexpr int O_WH = 0, O_WL = 16384, O_KH = 32768, O_KL = 49152, O_UH = 65536, O_UL = 73728;
 constexpr int O_SH = 81920, O_SL = 98304, O_E = 114688;
-constexpr int SCAN_BYTES = O_E + 512;
+constexpr int O_F = 115200;  // fp32 W [64][128] then K^ [64][128] of the next chunk (bulk copies)
+constexpr int SCAN_BYTES = O_F + 2 * 64 * 128 * 4;
 static_assert(1024 + SCAN_BYTES <= 227 * 1024, "kda scan shared memory");
 }  // namespace ks
 
@@ -669,13 +672,21 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
   float* sE = reinterpret_cast<float*>(sm + O_E);
-  __shared__ uint64_t bar[2];
+  __shared__ uint64_t bar[3];
   __shared__ uint32_t tslot;
   int* err = w.status;
+  float* sF = reinterpret_cast<float*>(sm + O_F);
+  auto fetch = [&](size_t uu) {  // thread 0: the chunk's W and K^ into sF
+    mbar_expect_tx(&bar[2], 2 * CH * 128 * 4);
+    bulk_load(sF, w.W + uu * CH * 128, CH * 128 * 4, &bar[2]);
+    bulk_load(sF + CH * 128, w.Kh + uu * CH * 128, CH * 128 * 4, &bar[2]);
+  };
   if (tid == 0) {
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
+    mbar_init(&bar[2], 1);
     mbar_fence_init();
+    if (sq.y > 0) fetch((size_t)sq.x * p.HV + hv);
   }
   __syncthreads();
   if (warp == 0) {
@@ -702,6 +713,7 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
   const uint32_t aKL = smem_u32(sm + O_KL), aUH = smem_u32(sm + O_UH), aUL = smem_u32(sm + O_UL);
   const uint32_t aSH = smem_u32(sm + O_SH), aSL = smem_u32(sm + O_SL);
   bool ok = true;
+  int pend = sq.y > 0 ? 0 : -1;  // parity of the bulk copy in flight (thread 0's view)
   for (int ci = 0; ci < sq.y && ok; ++ci) {
     const size_t u = (size_t)(sq.x + ci) * p.HV + hv;
     {  // this half of the state entering the chunk: stored, and as a hi/lo tile [64 v][128 k]
@@ -715,30 +727,19 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
         st_pair_split(sm + O_SH, sm + O_SL, r0 + 8, c, TT, S[4 * j + 2], S[4 * j + 3]);
       }
     }
-    {  // W and K^ as hi/lo tiles
-      const float* gW = w.W + u * CH * K;
-      const float* gK = w.Kh + u * CH * K;
-      float4 rw[8], rk[8];
+    ok = __syncthreads_and(mbar_wait(&bar[2], ci & 1, err));
+    if (tid == 0 && ok) pend = -1;
+    if (!ok) break;
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int x = tid + 256 * m, row = x >> 4, j = x & 15;
-        const float4* pw = reinterpret_cast<const float4*>(gW + row * K + 8 * j);
-        const float4* pk = reinterpret_cast<const float4*>(gK + row * K + 8 * j);
-        rw[2 * m] = __ldg(pw);
-        rw[2 * m + 1] = __ldg(pw + 1);
-        rk[2 * m] = __ldg(pk);
-        rk[2 * m + 1] = __ldg(pk + 1);
-      }
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int x = tid + 256 * m, row = x >> 4, j = x & 15;
-        const float fw[8] = {rw[2 * m].x, rw[2 * m].y, rw[2 * m].z, rw[2 * m].w,
-                             rw[2 * m + 1].x, rw[2 * m + 1].y, rw[2 * m + 1].z, rw[2 * m + 1].w};
-        const float fk[8] = {rk[2 * m].x, rk[2 * m].y, rk[2 * m].z, rk[2 * m].w,
-                             rk[2 * m + 1].x, rk[2 * m + 1].y, rk[2 * m + 1].z, rk[2 * m + 1].w};
-        st_chunk_split(sm + O_WH, sm + O_WL, row, j, TT, fw);
-        st_chunk_split(sm + O_KH, sm + O_KL, row, j, TT, fk);
-      }
+    for (int m = 0; m < 4; ++m) {  // W and K^ as hi/lo tiles
+      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+      const float4* pw = reinterpret_cast<const float4*>(sF + row * K + 8 * j);
+      const float4* pk = reinterpret_cast<const float4*>(sF + CH * K + row * K + 8 * j);
+      const float4 w0 = pw[0], w1 = pw[1], k0 = pk[0], k1 = pk[1];
+      const float fw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      const float fk[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+      st_chunk_split(sm + O_WH, sm + O_WL, row, j, TT, fw);
+      st_chunk_split(sm + O_KH, sm + O_KL, row, j, TT, fk);
     }
     fence_proxy_async();
     tc_fence_before();
@@ -754,6 +755,10 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
         mma_bf16(taddr(tb, 0, 0), desc_kmajor(aWL, s, TT), sh, id, 1);
       }
       mma_commit(&bar[0]);
+      if (ci + 1 < sq.y) {  // the buffer was read before the barrier above (and fenced)
+        fetch(u + p.HV);
+        pend = (ci + 1) & 1;
+      }
     }
     // e^{Gam_C} for the state update (into shared memory once every thread is past the last
     // chunk's update)
@@ -831,6 +836,7 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
   }
   tc_fence_before();
   __syncthreads();
+  if (tid == 0 && pend >= 0) mbar_wait(&bar[2], (uint32_t)pend, err);  // a copy still in flight lands
   if (warp == 0) tmem_dealloc(tb, 256);
 }
 
