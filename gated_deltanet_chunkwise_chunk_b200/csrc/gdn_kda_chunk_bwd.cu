@@ -92,15 +92,15 @@ __device__ void gated_products(const float* Wt, int ldw, const TR* R, const TR* 
   }
 }
 
-// The same products for K = 128 and 256 threads, by channel, with the weights stored transposed
-// (WtT[j * LDT + i] = Wt_ij, rows 16-byte aligned, so that the 16 weights of a column j within a
-// sub-chunk are four 128-bit loads): thread t owns channel c = t % 128, its operands in
-// registers.  The diagonal sub-blocks: thread (c, t / 128) takes sub-chunks 2 (t / 128) and
-// 2 (t / 128) + 1, one exponential per pair (i, j) serving both F and G.  The blocks below the
-// diagonal, for each sub-chunk a through r = 16 a - 1: the threads t < 128 form F of a's rows
-// (16 independent accumulators, one pass over the columns j), the others G of the columns before
-// a; the two write disjoint rows of each channel.  The loops over j stay rolled (a fully unrolled
-// form overflows the instruction cache).  Results go to the sinks as above; ends with a barrier.
+// The same products for K = 128 and 512 threads, by channel, with the weights stored transposed
+// (WtT[j * LDT + i] = Wt_ij, rows 16-byte aligned, so that the weights of a column j within a
+// sub-chunk are 128-bit loads): thread t owns channel c = t % 128 and role t / 128, its operands
+// in registers.  The diagonal sub-blocks: role = the sub-chunk, one exponential per pair (i, j)
+// serving both F and G.  Below the diagonal, for each sub-chunk a (through r = 16 a - 1): roles 0
+// and 1 form F of a's rows 16a + 8 role .. + 7 (independent accumulators, one pass over the
+// columns j), roles 2 and 3 G of the columns j = role - 2, role, .. before a; F and G write
+// disjoint rows of each channel.  The loops over j stay rolled (a fully unrolled form overflows
+// the instruction cache).  Results go to the sinks as above; ends with a barrier.
 constexpr int LDT = CH + 4;
 
 __device__ __forceinline__ void ld16(const float* p, float* w) {
@@ -114,94 +114,6 @@ __device__ __forceinline__ void ld16(const float* p, float* w) {
   }
 }
 
-template <typename TR, typename SinkF, typename SinkG>
-__device__ __forceinline__ void gated_below(int A, const float* WtT, const TR* R, const TR* Lm,
-                                            const float* colw, const float* G2, int c, bool rows,
-                                            SinkF& sinkF, SinkG& sinkG) {
-  constexpr int K = 128;
-  const int I0 = SUB * A, NJ = SUB * A;
-  const float gr = G2[(I0 - 1) * K + c];
-  if (rows) {  // F_i = e^{Gam_i - Gam_r} sum_{j < 16 A} Wt_ij R_j e^{Gam_r - Gam_j}, i in sub-chunk A
-    float acc[SUB];
-#pragma unroll
-    for (int i = 0; i < SUB; ++i) acc[i] = 0.f;
-#pragma unroll 2
-    for (int j = 0; j < NJ; ++j) {
-      const float rt = ldf(R + j * K + c) * exp2f(gr - G2[j * K + c]);
-      float wv[SUB];
-      ld16(WtT + j * LDT + I0, wv);
-#pragma unroll
-      for (int i = 0; i < SUB; ++i) acc[i] = fmaf(wv[i], rt, acc[i]);
-    }
-#pragma unroll
-    for (int i = 0; i < SUB; ++i) sinkF(I0 + i, c, acc[i] * exp2f(G2[(I0 + i) * K + c] - gr));
-  } else {     // G_j = e^{Gam_r - Gam_j} sum_{i in A} colw_i Wt_ij L_i e^{Gam_i - Gam_r}, j < 16 A
-    float ls[SUB];
-#pragma unroll
-    for (int i = 0; i < SUB; ++i)
-      ls[i] = (colw ? colw[I0 + i] : 1.f) * ldf(Lm + (I0 + i) * K + c) * exp2f(G2[(I0 + i) * K + c] - gr);
-#pragma unroll 2
-    for (int j = 0; j < NJ; ++j) {
-      float wv[SUB];
-      ld16(WtT + j * LDT + I0, wv);
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-      for (int i = 0; i < SUB; i += 4) {
-        a0 = fmaf(wv[i], ls[i], a0);
-        a1 = fmaf(wv[i + 1], ls[i + 1], a1);
-        a2 = fmaf(wv[i + 2], ls[i + 2], a2);
-        a3 = fmaf(wv[i + 3], ls[i + 3], a3);
-      }
-      sinkG(j, c, ((a0 + a1) + (a2 + a3)) * exp2f(gr - G2[j * K + c]));
-    }
-  }
-}
-
-template <typename TR, typename SinkF, typename SinkG>
-__device__ void gated_products_k128(const float* WtT, const TR* R, const TR* Lm, const float* colw,
-                                    const float* G2, SinkF sinkF, SinkG sinkG) {
-  constexpr int K = 128;
-  const int c = threadIdx.x & 127, hi = threadIdx.x >> 7;
-#pragma unroll 1
-  for (int bb = 0; bb < 2; ++bb) {
-    const int b0 = SUB * (2 * hi + bb);
-    float g[SUB], r[SUB], l[SUB], F[SUB], G[SUB];
-#pragma unroll
-    for (int j = 0; j < SUB; ++j) {
-      g[j] = G2[(b0 + j) * K + c];
-      r[j] = ldf(R + (b0 + j) * K + c);
-      l[j] = (colw ? colw[b0 + j] : 1.f) * ldf(Lm + (b0 + j) * K + c);
-      F[j] = G[j] = 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < SUB; ++j) {
-      float wv[SUB];
-      ld16(WtT + (b0 + j) * LDT + b0, wv);
-#pragma unroll
-      for (int i = j; i < SUB; ++i) {
-        const float wt = wv[i] * exp2f(g[i] - g[j]);
-        F[i] = fmaf(wt, r[j], F[i]);
-        G[j] = fmaf(wt, l[i], G[j]);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < SUB; ++i) {
-      sinkF(b0 + i, c, F[i]);
-      sinkG(b0 + i, c, G[i]);
-    }
-  }
-#pragma unroll 1
-  for (int A = 1; A < CH / SUB; ++A) {
-    __syncthreads();
-    gated_below(A, WtT, R, Lm, colw, G2, c, hi == 0, sinkF, sinkG);
-  }
-  __syncthreads();
-}
-
-// The gated products with 512 threads (K = 128): thread t owns channel c = t % 128 and role
-// t / 128.  The diagonal sub-blocks: role = the sub-chunk.  Below the diagonal, for each sub-chunk
-// a: roles 0 and 1 form F of a's rows 16a + 8 role .. + 7, roles 2 and 3 G of the columns
-// j = role - 2, role, .. before a.  Same sums and sinks as gated_products_k128; ends with a barrier.
 template <typename TR, typename SinkF, typename SinkG>
 __device__ void gated_products_k128x4(const float* WtT, const TR* R, const TR* Lm, const float* colw,
                                       const float* G2, SinkF sinkF, SinkG sinkG) {
