@@ -16,9 +16,11 @@ from .gpu_common import compare, to_dev
 pytestmark = pytest.mark.gpu
 
 
-def _parity(case, seed, with_bias=True, long_memory=False):
+def _parity(case, seed, with_bias=True, long_memory=False, strong=False):
     import gated_deltanet_chunkwise_chunk_b200 as gdn
     g_raw, A_log, dt_bias = synth.kda_gate_inputs(case, seed, with_bias, long_memory)
+    if strong:  # most gate inputs past the softplus pass-through (x > 20), decays of -1 .. -100
+        g_raw = 8.0 * g_raw + 14.0
     d = to_dev(case)
     d["g_raw"], d["A_log"] = g_raw.cuda(), A_log.cuda()
     d["dt_bias"] = None if dt_bias is None else dt_bias.cuda()
@@ -81,3 +83,12 @@ def test_empty_input_returns_the_initial_state():
     o, ht = gdn.gdn_kda_chunk_fwd(**d)
     torch.cuda.synchronize()
     assert o.numel() == 0 and torch.equal(ht.cpu(), case.h0)
+
+
+def test_strong_gates_bf16():
+    """Gate inputs mostly past softplus's pass-through (x > 20) and per-token log-decays down to
+    about -100: the in-chunk exponentials underflow to zero inside a 16-token sub-chunk, and the
+    output and final state must still match the oracle (no overflow, no NaN)."""
+    case = synth.make_case(B=2, T=150, H=2, HV=4, K=128, V=128, dtype="bf16", seed=560, h0=True,
+                           name="kda_chunk_strong_gates")
+    _parity(case, seed=561, strong=True)

@@ -18,9 +18,11 @@ from .gpu_common import BF16_GRAD_REL_L2, FP32_MAX_ABS, compare, to_dev
 pytestmark = pytest.mark.gpu
 
 
-def _run(case, seed, with_bias=True, long_memory=False, dht=True):
+def _run(case, seed, with_bias=True, long_memory=False, dht=True, strong=False):
     import gated_deltanet_chunkwise_chunk_b200 as gdn
     g_raw, A_log, dt_bias = synth.kda_gate_inputs(case, seed, with_bias, long_memory)
+    if strong:  # most gate inputs past the softplus pass-through (x > 20), decays of -1 .. -100
+        g_raw = 8.0 * g_raw + 14.0
     rng = np.random.default_rng(seed + 1)
     dO = torch.from_numpy(rng.standard_normal((case.B, case.T, case.HV, case.V)).astype(np.float32))
     dO = dO.to(case.q.dtype)
@@ -142,3 +144,11 @@ def test_bf16_128_runs_the_tensor_core_kernels():
     for k in steps:
         assert f"kda_tc_{k}" in names, (k, names)
         assert f"kda_{k}" not in names, (k, names)
+
+
+def test_strong_gates_bf16():
+    """The backward with gate inputs mostly past softplus's pass-through and per-token
+    log-decays down to about -100 (in-chunk exponentials underflow inside a sub-chunk)."""
+    case = synth.make_case(B=2, T=150, H=2, HV=4, K=128, V=128, dtype="bf16", seed=680, h0=True,
+                           name="kda_bwd_strong_gates")
+    _run(case, seed=681, strong=True)
