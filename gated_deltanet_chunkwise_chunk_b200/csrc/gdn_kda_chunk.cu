@@ -198,6 +198,7 @@ __global__ void __launch_bounds__(256) k_kda_wy(Problem p, Args a, KdaWork w) {
 // W at 256, U~ at 384.
 namespace kf {
 using namespace tcx;
+constexpr int NT = 512;  // threads (16 warps; the blocked inverse runs on the first 256)
 constexpr int TT = 64 * 128;
 constexpr int O_V = 0, O_KB = 16384, O_QB = 32768, O_G = 49152, O_DD = 81920, O_B = 90112;
 constexpr int O_R = 91136;  // region: the A/P operand tiles, then the inverse and the W/U~ operands
@@ -244,7 +245,7 @@ __device__ __forceinline__ void kt_split_rows(unsigned char* hi0, unsigned char*
   }
 }
 
-__global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork w) {
+__global__ void __launch_bounds__(kf::NT, 1) k_kda_tc_wy(Problem p, Args a, KdaWork w) {
   using namespace kf;
   if (kda_failed(w)) return;
   const int gc = blockIdx.x, hv = blockIdx.y;
@@ -253,6 +254,7 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork
   constexpr int K = 128, V = 128;
   const int L = e.z, tok0 = e.w, hk = hv / p.G;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = NT / 32;
   extern __shared__ unsigned char smraw[];
   unsigned char* sm = align1k(smraw);
   bf16* sK = reinterpret_cast<bf16*>(sm + O_KB);
@@ -279,10 +281,10 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork
     const bf16* gk = static_cast<const bf16*>(a.k) + ((size_t)tok0 * p.H + hk) * K;
     const bf16* gq = static_cast<const bf16*>(a.q) + ((size_t)tok0 * p.H + hk) * K;
     const bf16* gv = static_cast<const bf16*>(a.v) + ((size_t)tok0 * p.HV + hv) * V;
-    uint4 rk[4], rq[4], rv[4];
+    uint4 rk[2], rq[2], rv[2];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+    for (int m = 0; m < 2; ++m) {
+      const int x = tid + NT * m, row = x >> 4, j = x & 15;
       rk[m] = rq[m] = rv[m] = make_uint4(0u, 0u, 0u, 0u);
       if (row < L) {
         rk[m] = __ldg(reinterpret_cast<const uint4*>(gk + row * rs + 8 * j));
@@ -291,19 +293,26 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork
       }
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+    for (int m = 0; m < 2; ++m) {
+      const int x = tid + NT * m, row = x >> 4, j = x & 15;
       reinterpret_cast<uint4*>(sK)[x] = rk[m];
       reinterpret_cast<uint4*>(sQ)[x] = rq[m];
       *reinterpret_cast<uint4*>(sm + O_V + sw128_chunk(row, j, TT)) = rv[m];
     }
     if (tid < CH) sb[tid] = tid < L ? a.beta[(size_t)(tok0 + tid) * p.HV + hv] : 0.f;
   }
-  load_tile<float>(sG, K, a.g_raw + ((size_t)tok0 * p.HV + hv) * K, (size_t)p.HV * K, L, K);
+  {  // raw gate inputs, rows past L zero
+    const float* gsrc = a.g_raw + ((size_t)tok0 * p.HV + hv) * K;
+    for (int x = tid; x < CH * K / 4; x += NT) {
+      const int row = x >> 5, c4 = x & 31;
+      reinterpret_cast<float4*>(sG)[x] = row < L ? __ldg(reinterpret_cast<const float4*>(gsrc + (size_t)row * p.HV * K) + c4)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
   __syncthreads();
   {  // the gate of every (token, channel), rows past L zero; then the cumsum per channel
     const float nexp = -expf(a.A_log[hv]);
-    for (int x = tid; x < CH * K; x += 256) {
+    for (int x = tid; x < CH * K; x += NT) {
       const int i = x / K, c = x % K;
       float yg = 0.f;
       if (i < L) {
@@ -324,8 +333,8 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork
   }
   // L tiles (rows >= 16) and R_a (a = 1, 2, 3) as hi/lo pairs
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+  for (int m = 0; m < 2; ++m) {
+    const int x = tid + NT * m, row = x >> 4, j = x & 15;
     float fk[8], fq[8];
     const int r = row >= 16 ? 16 * (row >> 4) - 1 : 0;
 #pragma unroll
@@ -338,7 +347,7 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork
     st_chunk_split(sm + O_LKH, sm + O_LKL, row, j, TT, fk);
     st_chunk_split(sm + O_LQH, sm + O_LQL, row, j, TT, fq);
   }
-  for (int x = tid; x < 96 * 16; x += 256) {  // 16 + 32 + 48 rows of 16 chunks
+  for (int x = tid; x < 96 * 16; x += NT) {  // 16 + 32 + 48 rows of 16 chunks
     const int ra = x >> 4, j = x & 15;
     const int A = ra < 16 ? 1 : (ra < 48 ? 2 : 3), row = ra - (A == 1 ? 0 : (A == 2 ? 16 : 48));
     const int r = 16 * A - 1, off = A == 1 ? O_R1 : (A == 2 ? O_R2 : O_R3), bb = 16 * A * 128;
@@ -382,7 +391,7 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork
   // row's 16 A and 16 P partial sums (columns j of its sub-chunk, zero for j > i) are summed over
   // the lanes by one butterfly reduce-scatter (31 shuffles), after which lane l holds column l
   // of A (l < 16) or l - 16 of P.
-  for (int i = warp; i < CH; i += 8) {
+  for (int i = warp; i < CH; i += NW) {
     const int b0 = i & ~(SUB - 1), c = 4 * lane;
     float ki[4], qi[4], gi[4];
     {
@@ -441,7 +450,7 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork
   float* sX = reinterpret_cast<float*>(sm + O_SX);
   float* sP = reinterpret_cast<float*>(sm + O_SP);
   // A (times beta_i, strictly lower) and P (lower incl. the diagonal): diagonal blocks and zeros
-  for (int x = tid; x < CH * CH; x += 256) {
+  for (int x = tid; x < CH * CH; x += NT) {
     const int i = x >> 6, j = x & 63;
     float va = 0.f, vp = 0.f;
     if ((i >> 4) == (j >> 4) && j <= i) {
@@ -454,11 +463,11 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork
   __syncthreads();
   {  // the blocks below the diagonal from TMEM: warps of sub-partition a = warp % 4 (a >= 1);
      // warp half 0 reads A, half 1 reads P
-    const int A = warp & 3, half = warp >> 2;
+    const int A = warp & 3, half = (warp >> 2) & 1, set = warp >> 3;
     if (ok && A > 0) {
       const int ca = (half ? 96 : 0) + (A == 1 ? 0 : (A == 2 ? 16 : 48));
       const int ib = 16 * A + (lane >> 2), cq = 2 * (lane & 3);
-      for (int t = 0; t < A; ++t) {
+      for (int t = set; t < A; t += 2) {
         float v[8];
         tmem_ld16dp_x2(taddr(tb, 32 * A, ca + 16 * t), v);
         tmem_wait_ld();
@@ -478,19 +487,20 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork
   const size_t u = (size_t)gc * p.HV + hv, uk = u * CH * K;
   {
     float4* gP = reinterpret_cast<float4*>(w.P + u * CH * CH);
-    for (int x = tid; x < CH * CH / 4; x += 256) gP[x] = reinterpret_cast<const float4*>(sP)[x];
+    for (int x = tid; x < CH * CH / 4; x += NT) gP[x] = reinterpret_cast<const float4*>(sP)[x];
     if (w.Gam) {
       float4* gG = reinterpret_cast<float4*>(w.Gam + uk);
-      for (int x = tid; x < CH * K / 4; x += 256) gG[x] = reinterpret_cast<const float4*>(sG)[x];
+      for (int x = tid; x < CH * K / 4; x += NT) gG[x] = reinterpret_cast<const float4*>(sG)[x];
     }
   }
-  tcx::unit_lower_inverse64(sA, sT, sX, tid);  // T = (I + A)^-1 (ends with a barrier)
+  if (tid < 256) tcx::unit_lower_inverse64<2>(sA, sT, sX, tid);  // T = (I + A)^-1 (threads 0..255)
+  __syncthreads();
   if (w.Tm)
-    for (int x = tid; x < CH * CH; x += 256) w.Tm[u * CH * CH + x] = sT[(x / CH) * LDA + x % CH];
+    for (int x = tid; x < CH * CH; x += NT) w.Tm[u * CH * CH + x] = sT[(x / CH) * LDA + x % CH];
   // K^ = k e^{Gam_C - Gam}, Q~ = q e^{Gam}, e^{Gam_C}; X' = k e^{Gam} and T' = T diag(beta) as tiles
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+  for (int m = 0; m < 2; ++m) {
+    const int x = tid + NT * m, row = x >> 4, j = x & 15;
     float fx[8], fh[8], fq[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -508,10 +518,9 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork
     qt[1] = make_float4(fq[4], fq[5], fq[6], fq[7]);
     st_chunk_split(sm + O_XH, sm + O_XL, row, j, TT, fx);
   }
-  for (int c = tid; c < K; c += 256) w.eGC[u * K + c] = exp2f(sG[(CH - 1) * K + c]);
-#pragma unroll
-  for (int m = 0; m < 2; ++m) {
-    const int x = tid + 256 * m, row = x >> 3, j = x & 7;
+  for (int c = tid; c < K; c += NT) w.eGC[u * K + c] = exp2f(sG[(CH - 1) * K + c]);
+  {
+    const int row = tid >> 3, j = tid & 7;
     float f[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) f[q] = sT[row * LDA + 8 * j + q] * sb[8 * j + q];
@@ -539,17 +548,17 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_wy(Problem p, Args a, KdaWork
   }
   ok = __syncthreads_and(ok && mbar_wait(&bar[1], 0, err));
   tc_fence_after();
-  if (ok) {  // W and U~, M = 64 accumulators (rows r0, r0 + 8)
-    const int half = warp >> 2, sub = 32 * (warp & 3), r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
-    float x[32], y[32];
-    tmem_ld16dp_x8(taddr(tb, sub, 256 + 64 * half), x);
-    tmem_ld16dp_x8(taddr(tb, sub, 384 + 64 * half), y);
+  if (ok) {  // W and U~, M = 64 accumulators (rows r0, r0 + 8; this warp's quarter of the columns)
+    const int qt = warp >> 2, sub = 32 * (warp & 3), r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
+    float x[16], y[16];
+    tmem_ld16dp_x4(taddr(tb, sub, 256 + 32 * qt), x);
+    tmem_ld16dp_x4(taddr(tb, sub, 384 + 32 * qt), y);
     tmem_wait_ld();
     float* gW = w.W + uk;
     float* gU = w.Ut + u * CH * V;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = 64 * half + 8 * j + cq;
+    for (int j = 0; j < 4; ++j) {
+      const int c = 32 * qt + 8 * j + cq;
       *reinterpret_cast<float2*>(gW + r0 * K + c) = make_float2(x[4 * j], x[4 * j + 1]);
       *reinterpret_cast<float2*>(gW + (r0 + 8) * K + c) = make_float2(x[4 * j + 2], x[4 * j + 3]);
       *reinterpret_cast<float2*>(gU + r0 * V + c) = make_float2(y[4 * j], y[4 * j + 1]);
@@ -983,19 +992,19 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_out(Problem p, Args a, KdaWor
 
 template <typename Kern>
 cudaError_t go(const char* name, Kern kern, dim3 grid, size_t smem, cudaStream_t s, const Problem& p,
-               const Args& a, const KdaWork& w) {
+               const Args& a, const KdaWork& w, int threads = 256) {
   if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   ProfScope ps(name, s);
-  kern<<<grid, 256, smem, s>>>(p, a, w);
+  kern<<<grid, threads, smem, s>>>(p, a, w);
   return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t forward_t(const Problem& p, const Args& a, const KdaWork& w, cudaStream_t s) {
   const bool tc = std::is_same<T, __nv_bfloat16>::value && p.K == 128 && p.V == 128;
-  cudaError_t e = tc ? go("kda_tc_wy", k_kda_tc_wy, dim3(p.NCmax, p.HV), 1024 + kf::WYF_BYTES, s, p, a, w)
+  cudaError_t e = tc ? go("kda_tc_wy", k_kda_tc_wy, dim3(p.NCmax, p.HV), 1024 + kf::WYF_BYTES, s, p, a, w, kf::NT)
                      : go("kda_wy", k_kda_wy<T>, dim3(p.NCmax, p.HV), wy_smem(p.K, p.V), s, p, a, w);
   if (e == cudaSuccess)
     e = tc ? go("kda_tc_scan", k_kda_tc_scan, dim3(p.Nst, p.HV, 2), 1024 + ks::SCAN_BYTES, s, p, a, w)

@@ -281,6 +281,16 @@ constexpr int LDA = 68;
 //   32-blocks:                     T[32:,:32] = -T[32:,32:] (A[32:,:32] T[:32,:32])
 // Each thread owns 4 consecutive columns of one output row of a product; operands are read
 // as float4 (a row of A four k at a time, a row of T four columns at a time).  sX: [64][LDA].
+// Threads 0..255 take part (kBar: see sync256).
+// The inverse's barrier: the whole CTA (kBar = 0, a 256-thread CTA), or named barrier kBar over
+// threads 0..255 of a larger CTA (the others skip the inverse).
+template <int kBar>
+__device__ __forceinline__ void sync256() {
+  if constexpr (kBar == 0) __syncthreads();
+  else nbar_sync(kBar, 256);
+}
+
+template <int kBar = 0>
 __device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT, float* sX, int tid) {
   const int w = tid >> 5, lane = tid & 31;
   if (w < 4) {
@@ -304,7 +314,7 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT,
       *reinterpret_cast<float4*>(sT + (16 * br + r) * LDA + 16 * bc + 4 * c4) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
-  __syncthreads();
+  sync256<kBar>();
   auto fma4 = [](float4& acc, float a, const float4& b) {
     acc.x += a * b.x; acc.y += a * b.y; acc.z += a * b.z; acc.w += a * b.w;
   };
@@ -324,7 +334,7 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT,
     }
     *reinterpret_cast<float4*>(sX + R1 * LDA + C1) = x;
   }
-  __syncthreads();
+  sync256<kBar>();
   if (tid < 128) {  // T10 = -T11 X
     const int D0 = 16 * (2 * p1 + 1);
     float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -339,7 +349,7 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT,
     }
     *reinterpret_cast<float4*>(sT + R1 * LDA + C1) = make_float4(-y.x, -y.y, -y.z, -y.w);
   }
-  __syncthreads();
+  sync256<kBar>();
   // rows 32 + r2, columns 4c4 .. +3 (all 256 threads)
   const int r2 = tid >> 3, C2 = 4 * (tid & 7), R2 = 32 + r2;
   {  // X = A[32:,:32] T[:32,:32]
@@ -355,7 +365,7 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT,
     }
     *reinterpret_cast<float4*>(sX + R2 * LDA + C2) = x;
   }
-  __syncthreads();
+  sync256<kBar>();
   {  // T[32:,:32] = -T[32:,32:] X
     float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -369,7 +379,7 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* sA, float* sT,
     }
     *reinterpret_cast<float4*>(sT + R2 * LDA + C2) = make_float4(-y.x, -y.y, -y.z, -y.w);
   }
-  __syncthreads();
+  sync256<kBar>();
 }
 
 // Two adjacent bf16 columns (c even) of row r as one 32-bit store, hi and lo parts.
