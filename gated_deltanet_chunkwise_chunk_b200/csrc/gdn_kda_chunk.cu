@@ -660,6 +660,7 @@ __global__ void __launch_bounds__(256) k_kda_scan(Problem p, Args a, KdaWork w) 
 // are built from shared memory.
 namespace ks {
 using namespace tcx;
+constexpr int NT = 512;  // threads: four warps per TMEM sub-partition, a quarter of the columns each
 constexpr int TT = 64 * 128;
 constexpr int O_WH = 0, O_WL = 16384, O_KH = 32768, O_KL = 49152, O_UH = 65536, O_UL = 73728;
 constexpr int O_SH = 81920, O_SL = 98304, O_E = 114688;
@@ -668,14 +669,14 @@ constexpr int SCAN_BYTES = O_F + 2 * 64 * 128 * 4;
 static_assert(1024 + SCAN_BYTES <= 227 * 1024, "kda scan shared memory");
 }  // namespace ks
 
-__global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWork w) {
+__global__ void __launch_bounds__(ks::NT, 1) k_kda_tc_scan(Problem p, Args a, KdaWork w) {
   using namespace ks;
   if (kda_failed(w)) return;
   const int n = blockIdx.x, hv = blockIdx.y, z = blockIdx.z;
   const int4 sq = w.seq_tab[n];
   constexpr int K = 128, V = 128;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int half = warp >> 2, sub = 32 * (warp & 3);
+  const int qt = warp >> 2, sub = 32 * (warp & 3);  // quarter of the columns, sub-partition
   const int r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
   const int v0 = 64 * z;
   extern __shared__ unsigned char smraw[];
@@ -702,15 +703,15 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
     tmem_alloc(&tslot, 256);
     tmem_relinquish();
   }
-  // S[4j + q]: row v0 + r0 + 8 (q >> 1), column 64 half + 8j + cq + (q & 1)
-  float S[32];
+  // S[4j + q]: row v0 + r0 + 8 (q >> 1), column 32 qt + 8j + cq + (q & 1)
+  float S[16];
   {
     const float* h0 = a.h0 ? a.h0 + ((size_t)n * p.HV + hv) * K * V : nullptr;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int r = v0 + r0 + 8 * (q >> 1), c = 64 * half + 8 * j + cq + (q & 1);
+        const int r = v0 + r0 + 8 * (q >> 1), c = 32 * qt + 8 * j + cq + (q & 1);
         S[4 * j + q] = h0 ? h0[(size_t)c * V + r] : 0.f;
       }
   }
@@ -728,8 +729,8 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
     {  // this half of the state entering the chunk: stored, and as a hi/lo tile [64 v][128 k]
       float* h = w.h + u * V * K + (size_t)v0 * K;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = 64 * half + 8 * j + cq;
+      for (int j = 0; j < 4; ++j) {
+        const int c = 32 * qt + 8 * j + cq;
         *reinterpret_cast<float2*>(h + r0 * K + c) = make_float2(S[4 * j], S[4 * j + 1]);
         *reinterpret_cast<float2*>(h + (r0 + 8) * K + c) = make_float2(S[4 * j + 2], S[4 * j + 3]);
         st_pair_split(sm + O_SH, sm + O_SL, r0, c, TT, S[4 * j], S[4 * j + 1]);
@@ -740,8 +741,8 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
     if (tid == 0 && ok) pend = -1;
     if (!ok) break;
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {  // W and K^ as hi/lo tiles
-      const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+    for (int m = 0; m < 2; ++m) {  // W and K^ as hi/lo tiles
+      const int x = tid + NT * m, row = x >> 4, j = x & 15;
       const float4* pw = reinterpret_cast<const float4*>(sF + row * K + 8 * j);
       const float4* pk = reinterpret_cast<const float4*>(sF + CH * K + row * K + 8 * j);
       const float4 w0 = pw[0], w1 = pw[1], k0 = pk[0], k1 = pk[1];
@@ -772,12 +773,12 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
     // e^{Gam_C} for the state update (into shared memory once every thread is past the last
     // chunk's update)
     const float egc = tid < K ? w.eGC[u * K + tid] : 0.f;
-    float ut[16];  // U~ at this thread's (token, value) pairs of the M = 64, N = 64 accumulator
+    float ut[8];  // U~ at this thread's (token, value) pairs of the M = 64, N = 64 accumulator
     {
       const float* gU = w.Ut + u * CH * V + v0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = 32 * half + 8 * j + cq;
+      for (int j = 0; j < 2; ++j) {
+        const int c = 16 * qt + 8 * j + cq;
         const float2 a0 = *reinterpret_cast<const float2*>(gU + r0 * V + c);
         const float2 a1 = *reinterpret_cast<const float2*>(gU + (r0 + 8) * V + c);
         ut[4 * j] = a0.x;
@@ -790,13 +791,13 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
     tc_fence_after();
     if (tid < K) sE[tid] = egc;
     if (ok) {  // U = U~ - W S^T for this half's values: stored, and as a hi/lo tile [64 tok][64 v]
-      float x[16];
-      tmem_ld16dp_x4(taddr(tb, sub, 32 * half), x);
+      float x[8];
+      tmem_ld16dp_x2(taddr(tb, sub, 16 * qt), x);
       tmem_wait_ld();
       float* gU = w.U + u * CH * V + v0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = 32 * half + 8 * j + cq;
+      for (int j = 0; j < 2; ++j) {
+        const int c = 16 * qt + 8 * j + cq;
         const float u0 = ut[4 * j] - x[4 * j], u1 = ut[4 * j + 1] - x[4 * j + 1];
         const float u2 = ut[4 * j + 2] - x[4 * j + 2], u3 = ut[4 * j + 3] - x[4 * j + 3];
         *reinterpret_cast<float2*>(gU + r0 * V + c) = make_float2(u0, u1);
@@ -823,23 +824,23 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_scan(Problem p, Args a, KdaWo
     ok = __syncthreads_and(ok && mbar_wait(&bar[1], ci & 1, err));
     tc_fence_after();
     if (ok) {  // S = S Diag(e^{Gam_C}) + U^T K^
-      float x[32];
-      tmem_ld16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
+      float x[16];
+      tmem_ld16dp_x4(taddr(tb, sub, 128 + 32 * qt), x);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
+      for (int j = 0; j < 4; ++j)
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          S[4 * j + q] = fmaf(S[4 * j + q], sE[64 * half + 8 * j + cq + (q & 1)], x[4 * j + q]);
+          S[4 * j + q] = fmaf(S[4 * j + q], sE[32 * qt + 8 * j + cq + (q & 1)], x[4 * j + q]);
     }
   }
   if (ok && a.ht) {
     float* ht = a.ht + ((size_t)n * p.HV + hv) * K * V;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int r = v0 + r0 + 8 * (q >> 1), c = 64 * half + 8 * j + cq + (q & 1);
+        const int r = v0 + r0 + 8 * (q >> 1), c = 32 * qt + 8 * j + cq + (q & 1);
         ht[(size_t)c * V + r] = S[4 * j + q];
       }
   }
@@ -1007,7 +1008,7 @@ cudaError_t forward_t(const Problem& p, const Args& a, const KdaWork& w, cudaStr
   cudaError_t e = tc ? go("kda_tc_wy", k_kda_tc_wy, dim3(p.NCmax, p.HV), 1024 + kf::WYF_BYTES, s, p, a, w, kf::NT)
                      : go("kda_wy", k_kda_wy<T>, dim3(p.NCmax, p.HV), wy_smem(p.K, p.V), s, p, a, w);
   if (e == cudaSuccess)
-    e = tc ? go("kda_tc_scan", k_kda_tc_scan, dim3(p.Nst, p.HV, 2), 1024 + ks::SCAN_BYTES, s, p, a, w)
+    e = tc ? go("kda_tc_scan", k_kda_tc_scan, dim3(p.Nst, p.HV, 2), 1024 + ks::SCAN_BYTES, s, p, a, w, ks::NT)
            : go("kda_scan", k_kda_scan, dim3(p.Nst, p.HV, p.V / 32), scan_smem(p.K), s, p, a, w);
   if (e == cudaSuccess)
     e = tc ? go("kda_tc_out", k_kda_tc_out, dim3(p.NCmax, p.HV), 1024 + ko::OUT_BYTES, s, p, a, w)

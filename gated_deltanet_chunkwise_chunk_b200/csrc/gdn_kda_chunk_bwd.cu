@@ -255,6 +255,7 @@ __global__ void __launch_bounds__(256) k_kda_bwd_scan(Problem p, Args a, KdaWork
 //   dS_z = dS'_z Diag(e^{Gam_C}) + dO[:, z]^T (scale Q~) + dU[:, z]^T (-W)   (M = 64, N = K)  TMEM [128, 256)
 namespace kb {
 using namespace tcx;
+constexpr int NT = 512;  // threads: four warps per TMEM sub-partition, a quarter of the columns each
 constexpr int TT = 64 * 128;
 constexpr int O_PH = 0, O_PL = 8192, O_DO = 16384, O_KH = 24576, O_KL = 40960, O_QH = 57344;
 constexpr int O_QL = 73728, O_WH = 90112, O_WL = 106496, O_UH = 122880, O_UL = 131072;
@@ -263,14 +264,14 @@ constexpr int BSCAN_BYTES = O_E + 512;
 static_assert(1024 + BSCAN_BYTES <= 227 * 1024, "kda backward scan shared memory");
 }  // namespace kb
 
-__global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, KdaWork w) {
+__global__ void __launch_bounds__(kb::NT, 1) k_kda_tc_bwd_scan(Problem p, Args a, KdaWork w) {
   using namespace kb;
   if (kda_failed(w)) return;
   const int n = blockIdx.x, hv = blockIdx.y, z = blockIdx.z;
   const int4 sq = w.seq_tab[n];
   constexpr int K = 128, V = 128;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int half = warp >> 2, sub = 32 * (warp & 3);
+  const int qt = warp >> 2, sub = 32 * (warp & 3);  // quarter of the columns, sub-partition
   const int r0 = 16 * (warp & 3) + (lane >> 2), cq = 2 * (lane & 3);
   const int v0 = 64 * z;
   extern __shared__ unsigned char smraw[];
@@ -289,15 +290,15 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
     tmem_alloc(&tslot, 256);
     tmem_relinquish();
   }
-  // S[4j + q]: dS at row v0 + r0 + 8 (q >> 1), column 64 half + 8j + cq + (q & 1)
-  float S[32];
+  // S[4j + q]: dS at row v0 + r0 + 8 (q >> 1), column 32 qt + 8j + cq + (q & 1)
+  float S[16];
   {
     const float* dht = a.dht ? a.dht + ((size_t)n * p.HV + hv) * K * V : nullptr;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int r = v0 + r0 + 8 * (q >> 1), c = 64 * half + 8 * j + cq + (q & 1);
+        const int r = v0 + r0 + 8 * (q >> 1), c = 32 * qt + 8 * j + cq + (q & 1);
         S[4 * j + q] = dht ? dht[(size_t)c * V + r] : 0.f;
       }
   }
@@ -314,8 +315,8 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
     {  // this half of dS' (leaving the chunk): stored, and as a hi/lo tile [64 v][128 k]
       float* dh = w.dh + u * V * K + (size_t)v0 * K;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = 64 * half + 8 * j + cq;
+      for (int j = 0; j < 4; ++j) {
+        const int c = 32 * qt + 8 * j + cq;
         *reinterpret_cast<float2*>(dh + r0 * K + c) = make_float2(S[4 * j], S[4 * j + 1]);
         *reinterpret_cast<float2*>(dh + (r0 + 8) * K + c) = make_float2(S[4 * j + 2], S[4 * j + 3]);
         st_pair_split(sm + O_SH, sm + O_SL, r0, c, TT, S[4 * j], S[4 * j + 1]);
@@ -325,18 +326,18 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
     {  // scale P, K^ as hi/lo tiles; this half's dO columns (bf16, rows past L zero)
       const float* gK = w.Kh + u * CH * K;
       const float* gP = w.P + u * CH * CH;
-      float4 rk[8], rp[4];
-      uint4 rd[2];
+      float4 rk[4], rp[2];
+      uint4 rd[1];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+      for (int m = 0; m < 2; ++m) {
+        const int x = tid + NT * m, row = x >> 4, j = x & 15;
         const float4* pk = reinterpret_cast<const float4*>(gK + row * K + 8 * j);
         rk[2 * m] = __ldg(pk);
         rk[2 * m + 1] = __ldg(pk + 1);
       }
 #pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const int x = tid + 256 * m, row = x >> 3, j = x & 7;
+      for (int m = 0; m < 1; ++m) {
+        const int x = tid + NT * m, row = x >> 3, j = x & 7;
         rd[m] = row < e.z ? __ldg(reinterpret_cast<const uint4*>(dO + ((size_t)(e.w + row) * p.HV + hv) * V + v0 + 8 * j))
                           : make_uint4(0u, 0u, 0u, 0u);
         const float4* pp = reinterpret_cast<const float4*>(gP + row * CH + 8 * j);
@@ -344,16 +345,16 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
         rp[2 * m + 1] = __ldg(pp + 1);
       }
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+      for (int m = 0; m < 2; ++m) {
+        const int x = tid + NT * m, row = x >> 4, j = x & 15;
         const float fk[8] = {rk[2 * m].x, rk[2 * m].y, rk[2 * m].z, rk[2 * m].w,
                              rk[2 * m + 1].x, rk[2 * m + 1].y, rk[2 * m + 1].z, rk[2 * m + 1].w};
         st_chunk_split(sm + O_KH, sm + O_KL, row, j, TT, fk);
       }
       const float sc = p.scale;
 #pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const int x = tid + 256 * m, row = x >> 3, j = x & 7;
+      for (int m = 0; m < 1; ++m) {
+        const int x = tid + NT * m, row = x >> 3, j = x & 7;
         *reinterpret_cast<uint4*>(sm + O_DO + sw128_chunk(row, j, TT)) = rd[m];
         const float f[8] = {sc * rp[2 * m].x, sc * rp[2 * m].y, sc * rp[2 * m].z, sc * rp[2 * m].w,
                             sc * rp[2 * m + 1].x, sc * rp[2 * m + 1].y, sc * rp[2 * m + 1].z, sc * rp[2 * m + 1].w};
@@ -388,10 +389,10 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
     {  // while they run: scale Q~ and -W as hi/lo tiles (read by the second products only)
       const float* gQ = w.Qt + u * CH * K;
       const float* gW = w.W + u * CH * K;
-      float4 rq[8], rw[8];
+      float4 rq[4], rw[4];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+      for (int m = 0; m < 2; ++m) {
+        const int x = tid + NT * m, row = x >> 4, j = x & 15;
         const float4* pq = reinterpret_cast<const float4*>(gQ + row * K + 8 * j);
         const float4* pw = reinterpret_cast<const float4*>(gW + row * K + 8 * j);
         rq[2 * m] = __ldg(pq);
@@ -401,8 +402,8 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
       }
       const float sc = p.scale;
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int x = tid + 256 * m, row = x >> 4, j = x & 15;
+      for (int m = 0; m < 2; ++m) {
+        const int x = tid + NT * m, row = x >> 4, j = x & 15;
         const float fq[8] = {sc * rq[2 * m].x, sc * rq[2 * m].y, sc * rq[2 * m].z, sc * rq[2 * m].w,
                              sc * rq[2 * m + 1].x, sc * rq[2 * m + 1].y, sc * rq[2 * m + 1].z, sc * rq[2 * m + 1].w};
         const float fw[8] = {-rw[2 * m].x, -rw[2 * m].y, -rw[2 * m].z, -rw[2 * m].w,
@@ -415,13 +416,13 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
     tc_fence_after();
     if (tid < K) sE[tid] = egc;
     if (ok) {  // dU for this half's values: stored, and as a hi/lo tile [64 tok][64 v]
-      float x[16];
-      tmem_ld16dp_x4(taddr(tb, sub, 32 * half), x);
+      float x[8];
+      tmem_ld16dp_x2(taddr(tb, sub, 16 * qt), x);
       tmem_wait_ld();
       float* gU = w.dU + u * CH * V + v0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = 32 * half + 8 * j + cq;
+      for (int j = 0; j < 2; ++j) {
+        const int c = 16 * qt + 8 * j + cq;
         *reinterpret_cast<float2*>(gU + r0 * V + c) = make_float2(x[4 * j], x[4 * j + 1]);
         *reinterpret_cast<float2*>(gU + (r0 + 8) * V + c) = make_float2(x[4 * j + 2], x[4 * j + 3]);
         st_pair_split(sm + O_UH, sm + O_UL, r0, c, TT, x[4 * j], x[4 * j + 1]);
@@ -452,23 +453,23 @@ __global__ void __launch_bounds__(256, 1) k_kda_tc_bwd_scan(Problem p, Args a, K
     ok = __syncthreads_and(ok && mbar_wait(&bar[1], k & 1, err));
     tc_fence_after();
     if (ok) {  // dS = dS' Diag(e^{Gam_C}) + the products
-      float x[32];
-      tmem_ld16dp_x8(taddr(tb, sub, 128 + 64 * half), x);
+      float x[16];
+      tmem_ld16dp_x4(taddr(tb, sub, 128 + 32 * qt), x);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
+      for (int j = 0; j < 4; ++j)
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          S[4 * j + q] = fmaf(S[4 * j + q], sE[64 * half + 8 * j + cq + (q & 1)], x[4 * j + q]);
+          S[4 * j + q] = fmaf(S[4 * j + q], sE[32 * qt + 8 * j + cq + (q & 1)], x[4 * j + q]);
     }
   }
   if (ok && a.dh0) {
     float* dh0 = a.dh0 + ((size_t)n * p.HV + hv) * K * V;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int r = v0 + r0 + 8 * (q >> 1), c = 64 * half + 8 * j + cq + (q & 1);
+        const int r = v0 + r0 + 8 * (q >> 1), c = 32 * qt + 8 * j + cq + (q & 1);
         dh0[(size_t)c * V + r] = S[4 * j + q];
       }
   }
@@ -1466,7 +1467,7 @@ bool kda_tc(const Problem& p) {
 template <typename T>
 cudaError_t backward_t(const Problem& p, const Args& a, const KdaWork& w, cudaStream_t s) {
   cudaError_t e = kda_tc<T>(p)
-      ? go("kda_tc_bwd_scan", k_kda_tc_bwd_scan, dim3(p.Nst, p.HV, 2), 1024 + kb::BSCAN_BYTES, s, p, a, w)
+      ? go("kda_tc_bwd_scan", k_kda_tc_bwd_scan, dim3(p.Nst, p.HV, 2), 1024 + kb::BSCAN_BYTES, s, p, a, w, kb::NT)
       : go("kda_bwd_scan", k_kda_bwd_scan<T>, dim3(p.Nst, p.HV, p.V / 32), scan_smem(p.K), s, p, a, w);
   if (e == cudaSuccess)
     e = kda_tc<T>(p) ? go("kda_tc_bwd_dqk", k_kda_tc_bwd_dqk, dim3(p.NCmax, p.HV), 1024 + kt::DQK_BYTES, s, p, a, w, kt::NT)
