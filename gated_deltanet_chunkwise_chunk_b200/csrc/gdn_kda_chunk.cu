@@ -655,17 +655,19 @@ __global__ void __launch_bounds__(256) k_kda_scan(Problem p, Args a, KdaWork w) 
 // of its warp half), both products of a chunk on the tensor cores from compensated bf16 pairs:
 //   U[:, z] = U~[:, z] - W S_z^T        (M = 64 tokens, N = 64;  A = W, B = S_z, K-major)   TMEM [0, 64)
 //   S_z' = S_z Diag(e^{Gam_C}) + U[:, z]^T K^   (M = 64, N = K;  A = U^T, B = K^, MN-major) TMEM [128, 256)
-// It stores the state entering every chunk and U, as k_kda_scan does.  The next chunk's W and K^
-// are bulk-copied into an fp32 buffer while a chunk's products run, so a chunk's operand tiles
-// are built from shared memory.
+// It stores the state entering every chunk and U, as k_kda_scan does.  The next chunk's W, K^, U~
+// and e^{Gam_C} are bulk-copied into an fp32 buffer while a chunk's products run, so a chunk reads
+// no global memory on its critical path.
 namespace ks {
 using namespace tcx;
 constexpr int NT = 512;  // threads: four warps per TMEM sub-partition, a quarter of the columns each
 constexpr int TT = 64 * 128;
 constexpr int O_WH = 0, O_WL = 16384, O_KH = 32768, O_KL = 49152, O_UH = 65536, O_UL = 73728;
 constexpr int O_SH = 81920, O_SL = 98304, O_E = 114688;
-constexpr int O_F = 115200;  // fp32 W [64][128] then K^ [64][128] of the next chunk (bulk copies)
-constexpr int SCAN_BYTES = O_F + 2 * 64 * 128 * 4;
+// fp32 W [64][128], K^ [64][128], U~ [64][128] and e^{Gam_C} [128] of the next chunk (bulk copies)
+constexpr int O_F = 115200;
+constexpr int F_BYTES = 3 * 64 * 128 * 4 + 128 * 4;
+constexpr int SCAN_BYTES = O_F + F_BYTES;
 static_assert(1024 + SCAN_BYTES <= 227 * 1024, "kda scan shared memory");
 }  // namespace ks
 
@@ -686,10 +688,12 @@ __global__ void __launch_bounds__(ks::NT, 1) k_kda_tc_scan(Problem p, Args a, Kd
   __shared__ uint32_t tslot;
   int* err = w.status;
   float* sF = reinterpret_cast<float*>(sm + O_F);
-  auto fetch = [&](size_t uu) {  // thread 0: the chunk's W and K^ into sF
-    mbar_expect_tx(&bar[2], 2 * CH * 128 * 4);
+  auto fetch = [&](size_t uu) {  // thread 0: the chunk's W, K^, U~ and e^{Gam_C} into sF
+    mbar_expect_tx(&bar[2], F_BYTES);
     bulk_load(sF, w.W + uu * CH * 128, CH * 128 * 4, &bar[2]);
     bulk_load(sF + CH * 128, w.Kh + uu * CH * 128, CH * 128 * 4, &bar[2]);
+    bulk_load(sF + 2 * CH * 128, w.Ut + uu * CH * 128, CH * 128 * 4, &bar[2]);
+    bulk_load(sF + 3 * CH * 128, w.eGC + uu * 128, 128 * 4, &bar[2]);
   };
   if (tid == 0) {
     mbar_init(&bar[0], 1);
@@ -765,17 +769,14 @@ __global__ void __launch_bounds__(ks::NT, 1) k_kda_tc_scan(Problem p, Args a, Kd
         mma_bf16(taddr(tb, 0, 0), desc_kmajor(aWL, s, TT), sh, id, 1);
       }
       mma_commit(&bar[0]);
-      if (ci + 1 < sq.y) {  // the buffer was read before the barrier above (and fenced)
-        fetch(u + p.HV);
-        pend = (ci + 1) & 1;
-      }
     }
     // e^{Gam_C} for the state update (into shared memory once every thread is past the last
-    // chunk's update)
-    const float egc = tid < K ? w.eGC[u * K + tid] : 0.f;
-    float ut[8];  // U~ at this thread's (token, value) pairs of the M = 64, N = 64 accumulator
+    // chunk's update) and U~ at this thread's (token, value) pairs of the M = 64, N = 64
+    // accumulator, from the staging buffer
+    const float egc = tid < K ? sF[3 * CH * 128 + tid] : 0.f;
+    float ut[8];
     {
-      const float* gU = w.Ut + u * CH * V + v0;
+      const float* gU = sF + 2 * CH * 128 + v0;
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int c = 16 * qt + 8 * j + cq;
@@ -790,6 +791,11 @@ __global__ void __launch_bounds__(ks::NT, 1) k_kda_tc_scan(Problem p, Args a, Kd
     ok = __syncthreads_and(mbar_wait(&bar[0], ci & 1, err));
     tc_fence_after();
     if (tid < K) sE[tid] = egc;
+    if (tid == 0 && ok && ci + 1 < sq.y) {  // every thread has read sF (the barrier above)
+      fence_proxy_async();
+      fetch(u + p.HV);
+      pend = (ci + 1) & 1;
+    }
     if (ok) {  // U = U~ - W S^T for this half's values: stored, and as a hi/lo tile [64 tok][64 v]
       float x[8];
       tmem_ld16dp_x2(taddr(tb, sub, 16 * qt), x);
