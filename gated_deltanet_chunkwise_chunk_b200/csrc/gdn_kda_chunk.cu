@@ -192,8 +192,9 @@ __global__ void __launch_bounds__(256) k_kda_wy(Problem p, Args a, KdaWork w) {
 // pairs.  The blocks of A and P below the diagonal, for each sub-chunk a (through r = 16 a - 1):
 // one M = 64 tile L holds, in every row i >= 16, k_i e^{Gam_i - Gam_r(i)} (Lq the same with
 // q_i), and R_a the rows k_j e^{Gam_r - Gam_j}, j < 16 a; the product L R_a^T holds sub-chunk a's
-// block in rows 16a..16a+15 (the other rows are not read).  The diagonal blocks are summed by
-// channel on CUDA cores meanwhile.  After the blocked inverse: W = T' X' and U~ = T' V with
+// block in rows 16a..16a+15 (the other rows are not read).  The diagonal blocks are summed on
+// CUDA cores meanwhile (a warp per row, lanes over channels, one butterfly reduce-scatter of the
+// row's 32 sums).  After the blocked inverse: W = T' X' and U~ = T' V with
 // T' = T diag(beta), X' = k e^{Gam}.  TMEM columns: A_a at 0, 16, 48; P_a at 96, 112, 144;
 // W at 256, U~ at 384.
 namespace kf {
@@ -462,7 +463,7 @@ __global__ void __launch_bounds__(kf::NT, 1) k_kda_tc_wy(Problem p, Args a, KdaW
   }
   __syncthreads();
   {  // the blocks below the diagonal from TMEM: warps of sub-partition a = warp % 4 (a >= 1);
-     // warp half 0 reads A, half 1 reads P
+     // (warp / 4) % 2 = 0 reads A, 1 reads P; the two warp sets warp / 8 split the 16-column pieces
     const int A = warp & 3, half = (warp >> 2) & 1, set = warp >> 3;
     if (ok && A > 0) {
       const int ca = (half ? 96 : 0) + (A == 1 ? 0 : (A == 2 ? 16 : 48));
@@ -651,8 +652,9 @@ __global__ void __launch_bounds__(256) k_kda_scan(Problem p, Args a, KdaWork w) 
 
 // k_kda_scan for bf16 with K = V = 128: two CTAs per (sequence, value head), each holding half of
 // the state's rows (v in [64 z, 64 z + 64), z = blockIdx.z) in fp32 registers in the layout of an
-// M = 64 accumulator (thread: rows r0 and r0 + 8 of its sub-partition, columns 8j + cq + {0, 1}
-// of its warp half), both products of a chunk on the tensor cores from compensated bf16 pairs:
+// M = 64 accumulator (512 threads; thread: rows r0 and r0 + 8 of its sub-partition, columns
+// 8j + cq + {0, 1} of its warp's quarter), both products of a chunk on the tensor cores from
+// compensated bf16 pairs:
 //   U[:, z] = U~[:, z] - W S_z^T        (M = 64 tokens, N = 64;  A = W, B = S_z, K-major)   TMEM [0, 64)
 //   S_z' = S_z Diag(e^{Gam_C}) + U[:, z]^T K^   (M = 64, N = K;  A = U^T, B = K^, MN-major) TMEM [128, 256)
 // It stores the state entering every chunk and U, as k_kda_scan does.  The next chunk's W, K^, U~
