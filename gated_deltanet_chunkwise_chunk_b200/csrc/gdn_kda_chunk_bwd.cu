@@ -586,7 +586,8 @@ __global__ void __launch_bounds__(256) k_kda_bwd_dqk(Problem p, Args a, KdaWork 
 //   [192, 320) dW'  = dU S           (three of the four hi/lo products)
 //   [320, 448) dK^' = U dS'          (same)
 // dS' takes S's tiles once the first three products are done; the dP gated products and the
-// per-channel terms then run on CUDA cores as in k_kda_bwd_dqk.
+// per-channel terms then run on CUDA cores as in k_kda_bwd_dqk, with dq, dk and dGam accumulated
+// in shared memory.  512 threads: four warps per TMEM sub-partition, a quarter of the columns each.
 namespace kt {
 using namespace tcx;
 constexpr int NT = 512;           // threads of the output-side kernel
