@@ -18,8 +18,10 @@
 // of a warp read whole 256-byte rows) and computes the gate itself, so a token needs no shared
 // memory and no block barrier; the KDA variant shares its per-channel decays through shared
 // memory.
+#include <algorithm>
 #include <type_traits>
 
+#include "ffma_tiles.cuh"  // cp_async16
 #include "gdn_common.cuh"
 #include "gdn_launch.h"
 
@@ -187,8 +189,169 @@ __global__ void __launch_bounds__(128) k_recurrent_fwd(Problem p, Args a, int* s
   }
 }
 
+// Decode steps (one token per sequence, dense, with an entering state): persistent CTAs walk the
+// (sequence, value head, 32-row slice) items in order, the four slices of a state neighbours.  A
+// two-stage cp.async pipeline in shared memory holds the next item's state slice (K x 32 fp32)
+// and token vectors while the current one is updated, so a CTA's loads stay in flight across
+// its items (with one pass per CTA they overlapped only across CTAs).  The update is the
+// recurrent kernel's, thread (kg, vg) holding the same state piece.
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(sa), "l"(gmem));
+}
+
+// A state slice row kk holds its eight 16-byte pieces j at slots j ^ ((kk / 8) % 8), so that the
+// eight rows 8 apart that one load instruction of a warp reads fall on different banks.
+__device__ __forceinline__ int slice_slot(int kk, int j) { return j ^ ((kk >> 3) & 7); }
+
+template <typename T, int K, bool KDA>
+struct DecodeStage {
+  static constexpr int S = K * RV * 4;                       // state slice [K][32] fp32
+  static constexpr int TK = S, TQ = TK + K * (int)sizeof(T);  // k, q vectors
+  static constexpr int TV = TQ + K * (int)sizeof(T);          // v slice [32]
+  static constexpr int TG = TV + RV * (int)sizeof(T);         // gate input(s): K (KDA) or 1
+  static constexpr int TB = TG + (KDA ? K * 4 : 16);          // beta
+  static constexpr int BYTES = (TB + 16 + 15) / 16 * 16;
+};
+
+template <typename T, int K, bool KDA>
+__global__ void __launch_bounds__(128) k_decode_pipe(Problem p, Args a, int nitems) {
+  using St = DecodeStage<T, K, KDA>;
+  constexpr int KQ = K / 16;
+  extern __shared__ __align__(16) unsigned char dsm[];
+  const int nz = p.V / RV, tid = threadIdx.x, lane = tid & 31, kg = lane & 15;
+  const int vg = 2 * (tid >> 5) + (lane >> 4), G = gridDim.x;
+  const T* q = static_cast<const T*>(a.q);
+  const T* k = static_cast<const T*>(a.k);
+  const T* v = static_cast<const T*>(a.v);
+  T* o = static_cast<T*>(a.o);
+  auto issue = [&](int it, int slot) {  // cp.async of item it into stage slot; one group always
+    if (it < nitems) {
+      unsigned char* st = dsm + slot * St::BYTES;
+      const int z = it % nz, nh = it / nz, n = nh / p.HV, hv = nh % p.HV, hk = hv / p.G, v0 = RV * z;
+      const float* h0 = a.h0 + (size_t)nh * K * p.V + v0;
+#pragma unroll
+      for (int m = 0; m < K * RV / 4 / 128; ++m) {  // 16-byte pieces of the slice's rows
+        const int c = tid + 128 * m, kk = c >> 3, j = c & 7;
+        cp_async16(st + (kk * RV + 4 * slice_slot(kk, j)) * 4, h0 + (size_t)kk * p.V + 4 * j);
+      }
+      constexpr int CKQ = K * (int)sizeof(T) / 16, CV = RV * (int)sizeof(T) / 16;
+      const size_t qk0 = ((size_t)n * p.H + hk) * K, gi = (size_t)n * p.HV + hv;
+      if (tid < CKQ) {
+        cp_async16(st + St::TK + 16 * tid, reinterpret_cast<const unsigned char*>(k + qk0) + 16 * tid);
+        cp_async16(st + St::TQ + 16 * tid, reinterpret_cast<const unsigned char*>(q + qk0) + 16 * tid);
+      }
+      if (tid >= 64 && tid < 64 + CV)
+        cp_async16(st + St::TV + 16 * (tid - 64),
+                   reinterpret_cast<const unsigned char*>(v + gi * p.V + v0) + 16 * (tid - 64));
+      if constexpr (KDA) {
+        if (tid >= 96 && tid < 96 + K / 4)
+          cp_async16(st + St::TG + 16 * (tid - 96), a.g_raw + gi * K + 4 * (tid - 96));
+      } else {
+        if (tid == 96) cp_async4(st + St::TG, a.g_raw + gi);
+      }
+      if (tid == 127) cp_async4(st + St::TB, a.beta + gi);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  const int i0 = blockIdx.x;
+  issue(i0, 0);
+  issue(i0 + G, 1);
+  const bool b3 = kg & 8, b2 = kg & 4;
+  auto rowsum4 = [&](const float4& e) {
+    float s0 = b3 ? e.z : e.x, s1 = b3 ? e.w : e.y;
+    s0 += __shfl_xor_sync(0xffffffffu, b3 ? e.x : e.z, 8);
+    s1 += __shfl_xor_sync(0xffffffffu, b3 ? e.y : e.w, 8);
+    float t = b2 ? s1 : s0;
+    t += __shfl_xor_sync(0xffffffffu, b2 ? s0 : s1, 4);
+    t += __shfl_xor_sync(0xffffffffu, t, 2);
+    t += __shfl_xor_sync(0xffffffffu, t, 1);
+    return t;
+  };
+  const int half = lane & 16;
+  auto gather4 = [&](float t) {
+    return make_float4(__shfl_sync(0xffffffffu, t, half), __shfl_sync(0xffffffffu, t, half + 4),
+                       __shfl_sync(0xffffffffu, t, half + 8), __shfl_sync(0xffffffffu, t, half + 12));
+  };
+  int slot = 0;
+  for (int it = i0; it < nitems; it += G, slot ^= 1) {
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+    __syncthreads();  // the item's stage has landed for every thread
+    const unsigned char* st = dsm + slot * St::BYTES;
+    const int z = it % nz, nh = it / nz, n = nh / p.HV, hv = nh % p.HV, v0 = RV * z;
+    float4 S4[KQ];
+    float kv[KQ], qv[KQ], dv[KQ], vv[4];
+#pragma unroll
+    for (int i = 0; i < KQ; ++i)
+      S4[i] = *reinterpret_cast<const float4*>(st + ((kg * KQ + i) * RV + 4 * slice_slot(kg * KQ + i, vg)) * 4);
+    ld_floats<T, KQ>(reinterpret_cast<const T*>(st + St::TK) + kg * KQ, kv);
+    ld_floats<T, KQ>(reinterpret_cast<const T*>(st + St::TQ) + kg * KQ, qv);
+    ld_floats<T, 4>(reinterpret_cast<const T*>(st + St::TV) + 4 * vg, vv);
+    const float b = *reinterpret_cast<const float*>(st + St::TB);
+    const float nexp = -expf(a.A_log[hv]);
+    if constexpr (KDA) {
+      const float* gk = reinterpret_cast<const float*>(st + St::TG);
+#pragma unroll
+      for (int i = 0; i < KQ; ++i) {
+        const int c = kg * KQ + i;
+        const float gf = gk[c] + (a.dt_bias ? a.dt_bias[(size_t)hv * K + c] : 0.f);
+        dv[i] = expf(nexp * (gf > 20.f ? gf : log1pf(expf(gf))));
+      }
+    } else {
+      const float gf = *reinterpret_cast<const float*>(st + St::TG) + a.dt_bias[hv];
+      const float dec = expf(nexp * (gf > 20.f ? gf : log1pf(expf(gf))));
+#pragma unroll
+      for (int i = 0; i < KQ; ++i) dv[i] = dec;
+    }
+    __syncthreads();  // every thread has read the stage: it takes the item two ahead
+    issue(it + 2 * G, slot);
+    float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < KQ; ++i) {
+      const float dec = dv[i];
+      S4[i].x *= dec; S4[i].y *= dec; S4[i].z *= dec; S4[i].w *= dec;
+      e.x += S4[i].x * kv[i]; e.y += S4[i].y * kv[i]; e.z += S4[i].z * kv[i]; e.w += S4[i].w * kv[i];
+    }
+    e = gather4(rowsum4(e));
+    const float dx = b * (vv[0] - e.x), dy = b * (vv[1] - e.y), dz = b * (vv[2] - e.z),
+                dw = b * (vv[3] - e.w);
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < KQ; ++i) {
+      S4[i].x += dx * kv[i]; S4[i].y += dy * kv[i]; S4[i].z += dz * kv[i]; S4[i].w += dw * kv[i];
+      y.x += S4[i].x * qv[i]; y.y += S4[i].y * qv[i]; y.z += S4[i].z * qv[i]; y.w += S4[i].w * qv[i];
+    }
+    const float yt = rowsum4(y);
+    if ((kg & 3) == 0) o[((size_t)n * p.HV + hv) * p.V + v0 + 4 * vg + (kg >> 2)] = from_f<T>(p.scale * yt);
+    if (a.ht) {
+      float* ht = a.ht + (size_t)nh * K * p.V + v0 + 4 * vg;
+#pragma unroll
+      for (int i = 0; i < KQ; ++i) *reinterpret_cast<float4*>(ht + (size_t)(kg * KQ + i) * p.V) = S4[i];
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+template <typename T, int K, bool KDA>
+cudaError_t launch_decode(const Problem& p, const Args& a, cudaStream_t s) {
+  using St = DecodeStage<T, K, KDA>;
+  const int nitems = p.Nst * p.HV * (p.V / RV);
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode_pipe<T, K, KDA>, 128, 2 * St::BYTES);
+  if (e != cudaSuccess) return e;
+  const int grid = std::min(nitems, std::max(1, sms * per_sm));
+  k_decode_pipe<T, K, KDA><<<grid, 128, 2 * St::BYTES, s>>>(p, a, nitems);
+  return cudaGetLastError();
+}
+
 template <typename T, bool KDA>
 cudaError_t launch_t(const Problem& p, const Args& a, int* status, cudaStream_t s) {
+  // a decode step (one token per sequence, an entering state): the pipelined persistent kernel
+  if (!p.varlen && p.T == 1 && a.h0 && p.Nst * p.HV * (p.V / RV) >= 1024)
+    return p.K == 128 ? launch_decode<T, 128, KDA>(p, a, s) : launch_decode<T, 64, KDA>(p, a, s);
   const dim3 grid((unsigned)p.Nst * (unsigned)(p.V / RV), p.HV);
   if (p.K == 128)
     k_recurrent_fwd<T, 128, KDA><<<grid, 128, 0, s>>>(p, a, status);

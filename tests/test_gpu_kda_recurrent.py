@@ -50,6 +50,14 @@ def test_decode_step(dtype, KV, with_bias):
     _parity(case, seed=401, with_bias=with_bias)
 
 
+@pytest.mark.parametrize("dtype,KV", [("bf16", 128), ("fp32", 64), ("bf16", 64)])
+def test_decode_batch_pipelined(dtype, KV):
+    """A KDA decode step over enough items (>= 1024) to take the persistent pipelined kernel."""
+    case = synth.make_case(B=64, T=1, H=4, HV=8, K=KV, V=KV, dtype=dtype, seed=460 + KV, h0=True,
+                           name=f"kda_decode_pipe_{dtype}_{KV}")
+    _parity(case, seed=461)
+
+
 @pytest.mark.parametrize("T", [2, 17, 64, 65, 200])
 def test_short_prefill(T):
     case = synth.make_case(B=2, T=T, H=2, HV=4, K=128, V=128, dtype="bf16", seed=410 + T, h0=True,
@@ -87,6 +95,22 @@ def test_channel_constant_gate_equals_gated_deltanet_bitwise(dtype):
     import gated_deltanet_chunkwise_chunk_b200 as gdn
     case = synth.make_case(B=3, T=40, H=2, HV=4, K=128, V=128, dtype=dtype, seed=450, h0=True,
                            name="kda_vs_gdn")
+    d = to_dev(case)
+    o1, h1 = gdn.gdn_recurrent_fwd(**d)
+    d2 = dict(d)
+    d2["g_raw"] = d["g_raw"][..., None].expand(-1, -1, -1, case.K).contiguous()
+    d2["dt_bias"] = d["dt_bias"][:, None].expand(-1, case.K).contiguous().view(-1)
+    o2, h2 = gdn.gdn_kda_recurrent_fwd(**d2)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_channel_constant_gate_equals_gated_deltanet_bitwise_pipelined(dtype):
+    """The same bitwise equality on a decode batch large enough for the pipelined kernel."""
+    import gated_deltanet_chunkwise_chunk_b200 as gdn
+    case = synth.make_case(B=64, T=1, H=4, HV=8, K=128, V=128, dtype=dtype, seed=470, h0=True,
+                           name="kda_vs_gdn_pipe")
     d = to_dev(case)
     o1, h1 = gdn.gdn_recurrent_fwd(**d)
     d2 = dict(d)

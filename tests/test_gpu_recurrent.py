@@ -45,6 +45,16 @@ def test_decode_step(dtype, KV):
     _assert_parity(case)
 
 
+@pytest.mark.parametrize("in_place", [False, True])
+@pytest.mark.parametrize("dtype,KV", [("bf16", 128), ("fp32", 64), ("fp32", 128), ("bf16", 64)])
+def test_decode_batch_pipelined(dtype, KV, in_place):
+    """A decode step over enough (sequence, value head, 32-row slice) items (>= 1024) to take the
+    persistent pipelined kernel, out of place and with the state updated in place."""
+    case = synth.make_case(B=64, T=1, H=4, HV=8, K=KV, V=KV, dtype=dtype, seed=330 + KV, h0=True,
+                           name=f"decode_pipe_{dtype}_{KV}")
+    _assert_parity(case, in_place=in_place)
+
+
 @pytest.mark.parametrize("T", [2, 5, 37, 64, 65, 200])
 def test_short_prefill(T):
     case = synth.make_case(B=2, T=T, H=2, HV=4, K=128, V=128, dtype="bf16", seed=310 + T, h0=True,
