@@ -24,6 +24,7 @@
 #include "ffma_tiles.cuh"  // cp_async16
 #include "gdn_common.cuh"
 #include "gdn_launch.h"
+#include "kda_gate_math.cuh"
 
 namespace gdn {
 namespace {
@@ -215,7 +216,7 @@ struct DecodeStage {
 };
 
 template <typename T, int K, bool KDA>
-__global__ void __launch_bounds__(128) k_decode_pipe(Problem p, Args a, int nitems) {
+__global__ void __launch_bounds__(128, KDA ? 6 : 4) k_decode_pipe(Problem p, Args a, int nitems) {
   using St = DecodeStage<T, K, KDA>;
   constexpr int KQ = K / 16;
   extern __shared__ __align__(16) unsigned char dsm[];
@@ -295,11 +296,11 @@ __global__ void __launch_bounds__(128) k_decode_pipe(Problem p, Args a, int nite
       for (int i = 0; i < KQ; ++i) {
         const int c = kg * KQ + i;
         const float gf = gk[c] + (a.dt_bias ? a.dt_bias[(size_t)hv * K + c] : 0.f);
-        dv[i] = expf(nexp * (gf > 20.f ? gf : log1pf(expf(gf))));
+        dv[i] = expf(nexp * softplus20(gf));
       }
     } else {
       const float gf = *reinterpret_cast<const float*>(st + St::TG) + a.dt_bias[hv];
-      const float dec = expf(nexp * (gf > 20.f ? gf : log1pf(expf(gf))));
+      const float dec = expf(nexp * softplus20(gf));
 #pragma unroll
       for (int i = 0; i < KQ; ++i) dv[i] = dec;
     }
