@@ -92,3 +92,11 @@ def test_strong_gates_bf16():
     case = synth.make_case(B=2, T=150, H=2, HV=4, K=128, V=128, dtype="bf16", seed=560, h0=True,
                            name="kda_chunk_strong_gates")
     _parity(case, seed=561, strong=True)
+
+
+def test_long_sequence_8192_tokens():
+    """128 chunks per sequence through the tensor-core state pass (compensated bf16 pairs carried
+    along the whole chain), weak decay so the state keeps its history."""
+    case = synth.make_case(B=1, T=8192, H=2, HV=4, K=128, V=128, dtype="bf16", seed=570, h0=True,
+                           name="kda_chunk_T8192")
+    _parity(case, seed=571, long_memory=True)

@@ -152,3 +152,10 @@ def test_strong_gates_bf16():
     case = synth.make_case(B=2, T=150, H=2, HV=4, K=128, V=128, dtype="bf16", seed=680, h0=True,
                            name="kda_bwd_strong_gates")
     _run(case, seed=681, strong=True)
+
+
+def test_long_sequence_8192_tokens():
+    """The backward through 128 chunks per sequence (the reverse tensor-core state pass), weak decay."""
+    case = synth.make_case(B=1, T=8192, H=2, HV=4, K=128, V=128, dtype="bf16", seed=690, h0=True,
+                           name="kda_bwd_T8192")
+    _run(case, seed=691, long_memory=True)
