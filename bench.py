@@ -280,7 +280,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--e2e-steps", type=int, default=24)
     ap.add_argument("--T", type=int, default=None,
                     help="override the sequence length of a dense workload (smaller profiling cases)")
     ap.add_argument("--workload", default="gdn", choices=["gdn", "kda_chunk", "decode"],
@@ -355,7 +355,7 @@ def main():
         for idx in (0, 1, 3, 4):
             oc = synth.config_case(idx, seed=1000 + idx + 7919 * rank)
             sub = measure_case(gdn, oc, dev, args.steps, args.warmup, dist, world, sampler=None,
-                               e2e_steps=3)
+                               e2e_steps=12)
             sub["config"] = {"workload": oc.name, "B": oc.B, "T": oc.T, "tokens": oc.tokens,
                              "H": oc.H, "HV": oc.HV, "K": oc.K, "V": oc.V, "dtype": oc.dtype}
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -367,7 +367,7 @@ def main():
         # B=2, T=2048, H=4, HV=8 with 64-wide key and value heads
         pc = synth.make_case(B=2, T=2048, H=4, HV=8, K=64, V=64, dtype="bf16", seed=1100 + 7919 * rank,
                              name="bf16_B2_T2048_H4_HV8_D64")
-        sub = measure_case(gdn, pc, dev, args.steps, args.warmup, dist, world, sampler=None, e2e_steps=3)
+        sub = measure_case(gdn, pc, dev, args.steps, args.warmup, dist, world, sampler=None, e2e_steps=12)
         sub["config"] = {"workload": pc.name, "B": pc.B, "T": pc.T, "tokens": pc.tokens, "H": pc.H,
                          "HV": pc.HV, "K": pc.K, "V": pc.V, "dtype": pc.dtype}
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -669,7 +669,9 @@ def e2e_measure(gdn, case, dev, ws, nsteps: int, dist) -> dict:
     return {"value": round(aggregate_mtok_s(world, case.tokens, ms), 3), "unit": "M tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(ms, 3), "steps": nsteps,
-            "pipelined": "copies of step i+1 in, step i's kernels, step i-1 out on three streams"}
+            "pipelined": "copies of step i+1 in, step i's kernels, step i-1 out on three streams; "
+                         "the first step's upload and the last step's download are inside the timed "
+                         "region (fill and drain)"}
 
 
 DECODE = dict(B=256, H=16, HV=32, K=128, V=128)
