@@ -220,8 +220,10 @@ int gdn_kda_recurrent_fwd(const gdn_dims* d, const void* q, const void* k, const
 
 /* Chunkwise forward of the same KDA recurrence as gdn_kda_recurrent_fwd, for long sequences:
  * 64-token chunks, the per-channel decay carried through 16-token sub-chunks (every factor an
- * exponential of a non-positive number), a sequential state pass over the chunks, fp32
- * arithmetic on CUDA cores.  Arguments, layouts and results as gdn_kda_recurrent_fwd
+ * exponential of a non-positive number), a sequential state pass over the chunks.  bf16 with
+ * K = V = 128: every product on the tensor cores (operands as compensated bf16 pairs, fp32
+ * accumulation); other dtypes and head sizes: fp32 arithmetic on CUDA cores; the same results
+ * within the tolerances either way.  Arguments, layouts and results as gdn_kda_recurrent_fwd
  * (g_raw [B,T,HV,K] fp32, dt_bias [HV*K] or NULL; o for every token, final_state after each
  * sequence's last token; final_state may be NULL).  workspace: at least
  * gdn_kda_chunk_workspace_bytes(d, varlen, 0) bytes, 256-byte aligned; it also holds the device
@@ -241,7 +243,8 @@ int gdn_kda_chunk_fwd(const gdn_dims* d, const void* q, const void* k, const voi
  *   dg [B,T,HV,K] fp32 = dL/dyg (the per-channel log-decay),
  *   dg_raw [B,T,HV,K] fp32 (may be NULL), dh0 [Nst,HV,K,V] fp32 (may be NULL),
  *   dA_log [HV] fp32 (may be NULL), ddt_bias [HV*K] fp32 (may be NULL; needs dt_bias).
- * dht may be NULL (zero).  The parameter sums are deterministic (fixed chunk order). */
+ * dht may be NULL (zero).  The parameter sums are deterministic (fixed chunk order).  Kernels as
+ * for gdn_kda_chunk_fwd (tensor cores for bf16 with K = V = 128). */
 int gdn_kda_chunk_bwd(const gdn_dims* d, const void* q, const void* k, const void* v,
                       const float* g_raw, const float* A_log, const float* dt_bias, const float* beta,
                       const int64_t* cu_seqlens, const void* d_o, const float* dht, void* dq, void* dk,
