@@ -1422,16 +1422,23 @@ __global__ void __launch_bounds__(kw::NT, 1) k_kda_tc_bwd_wy(Problem p, Args a, 
   if (warp == 0) tmem_dealloc(tb, 512);
 }
 
-// dA_log[hv] and ddt_bias[hv*K + c]: the per-chunk sums added in chunk order.
+// dA_log[hv] and ddt_bias[hv*K + c]: the per-chunk sums of the head's chunks (their count from
+// the chunk table), eight interleaved partial sums added in a fixed order, so the result is the
+// same on every run and the loads of eight chunks are in flight at once.
 __global__ void __launch_bounds__(256) k_kda_param_grads(Problem p, Args a, KdaWork w) {
   if (kda_failed(w)) return;
   const int hv = blockIdx.x, K = p.K;
+  const int nc = max(0, min(w.status[1], p.NCmax));
+  const size_t stride = (size_t)p.HV * (K + 1);
   for (int c = threadIdx.x; c <= K; c += blockDim.x) {
-    float s = 0.f;
-    for (int gc = 0; gc < p.NCmax; ++gc) {
-      if (w.chunk_tab[gc].x < 0) break;
-      s += w.pgp[((size_t)gc * p.HV + hv) * (K + 1) + c];
-    }
+    const float* src = w.pgp + (size_t)hv * (K + 1) + c;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int gc = 0;
+    for (; gc + 8 <= nc; gc += 8)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] += src[(size_t)(gc + q) * stride];
+    for (int q = 0; gc < nc; ++gc, ++q) acc[q] += src[(size_t)gc * stride];
+    const float s = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
     if (c < K && a.ddt_bias) a.ddt_bias[(size_t)hv * K + c] = s;
     if (c == K && a.dA_log) a.dA_log[hv] = s;
   }
